@@ -1,0 +1,213 @@
+"""Float64 CPU oracle for the MTLA hot path -- TEST INFRASTRUCTURE.
+
+This package is the yardstick the CUDA library is checked against. Only the
+tests, the entry module's ``smoke()`` and the benchmark's CPU-baseline leg may
+import it. The product path (``kv_cache_mtla_b200``) never imports, links or
+calls anything here, and nothing here calls the product.
+
+The arithmetic lives in ``mtla_oracle.c`` (plain C, float64, optional OpenMP
+over independent rows); this module only compiles it with gcc and marshals
+numpy arrays through ctypes. See the header of ``mtla_oracle.c`` for the
+passages each function follows and the readings taken where the pages are
+silent.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "mtla_oracle.c")
+_LIB = os.path.join(_HERE, "libmtla_oracle.so")
+
+GATE_COMPUTED, GATE_SUPPLIED, GATE_UNIT = 0, 1, 2
+
+FAULT_NONE = 0
+FAULT_DROP_OWN_PARTIAL = 1
+FAULT_MASK_OFF_BY_ONE = 2
+FAULT_TRANSPOSE_WUK = 3
+FAULT_ROPE_SIGN = 4
+FAULT_SCAN_NO_RESET = 5
+FAULT_DROP_ROPE_KEY = 6
+FAULT_GATE_WRONG_ROW = 7
+FAULT_SCALE = 8
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle into ``libmtla_oracle.so`` beside its source."""
+    if not force and os.path.exists(_LIB) and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC):
+        return _LIB
+    tmp = _LIB + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-std=c99", "-fopenmp", "-fPIC", "-shared", _SRC, "-o", tmp, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB)
+    return _LIB
+
+
+class _Cfg(ctypes.Structure):
+    _fields_ = [
+        ("B", ctypes.c_int32), ("H", ctypes.c_int32), ("d_h", ctypes.c_int32),
+        ("d_c", ctypes.c_int32), ("d_r", ctypes.c_int32), ("s", ctypes.c_int32),
+        ("gate_mode", ctypes.c_int32), ("scale", ctypes.c_double),
+        ("rope_base", ctypes.c_double), ("pe_base", ctypes.c_double),
+    ]
+
+
+@dataclass
+class Cfg:
+    B: int
+    H: int
+    d_h: int
+    d_c: int
+    d_r: int
+    s: int
+    gate_mode: int = GATE_COMPUTED
+    scale: float = 0.0
+    rope_base: float = 10000.0
+    pe_base: float = 10000.0
+
+    @property
+    def D(self) -> int:
+        return self.d_c + self.d_r
+
+    def c(self) -> _Cfg:
+        return _Cfg(self.B, self.H, self.d_h, self.d_c, self.d_r, self.s, self.gate_mode,
+                    self.scale, self.rope_base, self.pe_base)
+
+
+_lib = None
+_P = ctypes.POINTER(ctypes.c_double)
+_PI = ctypes.POINTER(ctypes.c_int64)
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = ctypes.CDLL(build())
+        _lib.orc_pe.argtypes = [ctypes.c_int64, ctypes.c_int32, ctypes.c_double, _P]
+        _lib.orc_rope.argtypes = [ctypes.c_int64, ctypes.c_int32, ctypes.c_double, _P, _P]
+        _lib.orc_gate.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int64, _P, _P, _P, _P]
+        _lib.orc_gate.restype = ctypes.c_double
+        _lib.orc_partials.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int32] + [_P] * 7
+        _lib.orc_attend_rows.argtypes = ([ctypes.POINTER(_Cfg), ctypes.c_int32] + [_P] * 5
+                                         + [ctypes.c_int64, _PI, _P, _P])
+        _lib.orc_prefill.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int32] + [_P] * 13
+        _lib.orc_decode_step.argtypes = ([ctypes.POINTER(_Cfg), ctypes.c_int32] + [_P] * 9
+                                         + [_PI] + [_P] * 5)
+        _lib.orc_prefill_explicit.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int32] + [_P] * 10
+        _lib.orc_set_fault.argtypes = [ctypes.c_int]
+    return _lib
+
+
+def _d(a):
+    """float64 C-contiguous copy (or view) of an array-like; None stays None."""
+    if a is None:
+        return None
+    if hasattr(a, "detach"):
+        a = a.detach().cpu().double().numpy()
+    return np.ascontiguousarray(a, dtype=np.float64)
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(_P)
+
+
+def set_fault(f: int) -> None:
+    """Plant one of the FAULT_* mistakes (tests of the pins only)."""
+    _load().orc_set_fault(int(f))
+
+
+def pe(t: int, d: int, base: float = 10000.0) -> np.ndarray:
+    out = np.zeros(d)
+    _load().orc_pe(t, d, base, _p(out))
+    return out
+
+
+def rope(t: int, x, base: float = 10000.0) -> np.ndarray:
+    x = _d(x)
+    y = np.zeros_like(x)
+    _load().orc_rope(t, x.shape[-1], base, _p(x), _p(y))
+    return y
+
+
+def gate(cfg: Cfg, t: int, c_t, G=None, g=None, w_given=None) -> float:
+    c_t = _d(c_t)
+    wg = None if w_given is None else np.array([w_given], dtype=np.float64)
+    return _load().orc_gate(ctypes.byref(cfg.c()), t, _p(c_t), _p(_d(G)), _p(_d(g)), _p(wg))
+
+
+def partials(cfg: Cfg, c, kr, G=None, g=None, gate_in=None):
+    """(w [B,T], P [B,T,D]) -- the block-prefix partial slots."""
+    c, kr = _d(c), _d(kr)
+    T = c.shape[1]
+    w = np.zeros((cfg.B, T))
+    P = np.zeros((cfg.B, T, cfg.D))
+    G, g, gate_in = _d(G), _d(g), _d(gate_in)
+    _load().orc_partials(ctypes.byref(cfg.c()), T, _p(c), _p(kr), _p(G), _p(g), _p(gate_in),
+                         _p(w), _p(P))
+    return w, P
+
+
+def attend_rows(cfg: Cfg, qc, qr, w_uk, w_uv, P, rows, want_olat: bool = False):
+    """Parallel-form outputs for selected (b, t) rows: out [n,H,d_h] (, olat [n,H,d_c])."""
+    qc, qr, w_uk, w_uv, P = _d(qc), _d(qr), _d(w_uk), _d(w_uv), _d(P)
+    rows = np.ascontiguousarray(rows, dtype=np.int64).reshape(-1, 2)
+    T = qc.shape[1]
+    n = rows.shape[0]
+    out = np.zeros((n, cfg.H, cfg.d_h))
+    olat = np.zeros((n, cfg.H, cfg.d_c)) if want_olat else None
+    _load().orc_attend_rows(ctypes.byref(cfg.c()), T, _p(qc), _p(qr), _p(w_uk), _p(w_uv), _p(P),
+                            n, rows.ctypes.data_as(_PI), _p(out), _p(olat))
+    return (out, olat) if want_olat else out
+
+
+def prefill(cfg: Cfg, c, kr, qc, qr, w_uk, w_uv, G=None, g=None, gate_in=None):
+    """Parallel forward from position 0: dict(out, w, cache, acc)."""
+    c, kr, qc, qr, w_uk, w_uv = map(_d, (c, kr, qc, qr, w_uk, w_uv))
+    G, g, gate_in = _d(G), _d(g), _d(gate_in)
+    T = c.shape[1]
+    n_slots = (T + cfg.s - 1) // cfg.s
+    out = np.zeros((cfg.B, T, cfg.H, cfg.d_h))
+    w = np.zeros((cfg.B, T))
+    cache = np.zeros((cfg.B, n_slots, cfg.D))
+    acc = np.zeros((cfg.B, cfg.D))
+    _load().orc_prefill(ctypes.byref(cfg.c()), T, _p(c), _p(kr), _p(qc), _p(qr), _p(w_uk),
+                        _p(w_uv), _p(G), _p(g), _p(gate_in), _p(out), _p(w), _p(cache), _p(acc))
+    return dict(out=out, w=w, cache=cache, acc=acc)
+
+
+def decode_step(cfg: Cfg, c_new, kr_new, qc, qr, w_uk, w_uv, pos, cache, acc,
+                G=None, g=None, gate_in=None, want_olat: bool = False):
+    """One incremental step. ``cache`` [B,max_slots,D] and ``acc`` [B,D] are
+    float64 numpy arrays updated in place. Returns dict(out, w[, olat])."""
+    assert cache.dtype == np.float64 and cache.flags.c_contiguous
+    assert acc.dtype == np.float64 and acc.flags.c_contiguous
+    c_new, kr_new, qc, qr, w_uk, w_uv = map(_d, (c_new, kr_new, qc, qr, w_uk, w_uv))
+    G, g, gate_in = _d(G), _d(g), _d(gate_in)
+    pos = np.ascontiguousarray(pos, dtype=np.int64)
+    out = np.zeros((cfg.B, cfg.H, cfg.d_h))
+    w = np.zeros(cfg.B)
+    olat = np.zeros((cfg.B, cfg.H, cfg.d_c)) if want_olat else None
+    _load().orc_decode_step(ctypes.byref(cfg.c()), cache.shape[1], _p(c_new), _p(kr_new),
+                            _p(qc), _p(qr), _p(w_uk), _p(w_uv), _p(G), _p(g), _p(gate_in),
+                            pos.ctypes.data_as(_PI), _p(cache), _p(acc), _p(out), _p(w),
+                            _p(olat))
+    res = dict(out=out, w=w)
+    if want_olat:
+        res["olat"] = olat
+    return res
+
+
+def prefill_explicit(cfg: Cfg, c, kr, qc, qr, w_uk, w_uv, G=None, g=None, gate_in=None):
+    """Non-absorbed parallel forward (explicit per-head k, v): out [B,T,H,d_h]."""
+    c, kr, qc, qr, w_uk, w_uv = map(_d, (c, kr, qc, qr, w_uk, w_uv))
+    G, g, gate_in = _d(G), _d(g), _d(gate_in)
+    T = c.shape[1]
+    out = np.zeros((cfg.B, T, cfg.H, cfg.d_h))
+    _load().orc_prefill_explicit(ctypes.byref(cfg.c()), T, _p(c), _p(kr), _p(qc), _p(qr),
+                                 _p(w_uk), _p(w_uv), _p(G), _p(g), _p(gate_in), _p(out))
+    return out

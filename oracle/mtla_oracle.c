@@ -1,0 +1,410 @@
+/*
+ * mtla_oracle.c -- plain float64 CPU oracle for the MTLA attention hot path.
+ *
+ * TEST INFRASTRUCTURE. This file is the yardstick the CUDA path is checked
+ * against; it is not part of the product. Only the tests, the smoke check in
+ * the repository's entry module and the benchmark's CPU-baseline leg load it.
+ * It shares no code, header, table or helper with the CUDA library, and it
+ * never calls it.
+ *
+ * What it follows (page titles and the sections they name):
+ *   [MTLA]  "Multi-head Temporal Latent Attention" (paper summary page):
+ *           Method -- (1) hyper-network merging weights W_t from the latent
+ *           times a positional embedding (Sec. 4.1, Eq. 13); in-place update of
+ *           the slot still being filled during inference; (2) the stride-aware
+ *           causal mask (Sec. 4.2, Fig. 2(c)); (3) decoupled-RoPE keys merged
+ *           along the same axis with the same mask (Sec. 4.3, Eq. 17); matrix
+ *           absorption of W^UK and W^UV kept from MLA.
+ *           Key claims -- the cache holds 9/(4s) elements per token at
+ *           d_c = 4 d_h, d_R = d_h/2 (Sec. 4.3).
+ *   [MLA]   "Multi-Head Latent Attention and Sparse Indexers", section
+ *           "Latent attention changes the representation": the absorption
+ *           identities q.(U_K c) = (U_K^T q).c and sum a U_V c = U_V sum a c.
+ *
+ * Readings taken where the pages are silent or garbled (each is a named
+ * choice, not something the pages fix):
+ *   - slots are 0-based: token t lives in slot floor(t/s); a sequence of n
+ *     tokens owns ceil(n/s) slots;
+ *   - query i attends every finished slot j < floor(i/s) plus its own partial
+ *     slot P_i = sum_{u = s*floor(i/s)}^{i} w_u x_u (the garbled mask sentence
+ *     of Sec. 4.2 read as "finished slots, plus the slot being filled");
+ *   - W_t is a linear layer d_c -> s (+ bias) on c_t * PE_t followed by a
+ *     sigmoid; token t uses output t mod s as one scalar that scales the whole
+ *     vector x_t = [c_t ; RoPE_t(k_t)];
+ *   - PE_t is the interleaved sinusoid PE[2k] = sin(t b^(-2k/d_c)),
+ *     PE[2k+1] = cos(...), b = 10000, over the latent width d_c;
+ *   - RoPE rotates interleaved pairs (x_2k, x_2k+1) by t * base^(-2k/d_R);
+ *     keys are rotated at their own position before merging, queries at
+ *     theirs;
+ *   - scores use scale 1/sqrt(d_h + d_R) unless a scale is given;
+ *   - the merged sum is not normalised.
+ * Parity unpinned: the PE, RoPE-frequency and gate conventions above are
+ * readings only; the pins check their invariants, not the conventions.
+ *
+ * Everything is float64, written as the definitions read, with no blocking,
+ * fusion or reordering. Layouts are row-major:
+ *   c [B,T,d_c]  kr [B,T,d_r]  qc [B,T,H,d_h]  qr [B,T,H,d_r]
+ *   w_uk, w_uv [H,d_h,d_c]   G [s,d_c]   g [s]   gate_in [B,T]
+ *   slot vectors have width D = d_c + d_r: [latent ; rotated key].
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_GATE_COMPUTED 0
+#define ORC_GATE_SUPPLIED 1
+#define ORC_GATE_UNIT 2
+
+typedef struct {
+    int32_t B, H, d_h, d_c, d_r, s;
+    int32_t gate_mode;
+    double scale;     /* 0 => 1/sqrt(d_h + d_r) */
+    double rope_base; /* base of the decoupled-RoPE frequencies */
+    double pe_base;   /* base of the sinusoidal positional embedding */
+} orc_cfg;
+
+/* Planted mistakes, used only by the tests that show the pins catch them.
+ * 0 means the oracle as written. */
+enum {
+    ORC_FAULT_NONE = 0,
+    ORC_FAULT_DROP_OWN_PARTIAL = 1,  /* forget the slot being filled        */
+    ORC_FAULT_MASK_OFF_BY_ONE = 2,   /* let query see finished slot floor(i/s) too */
+    ORC_FAULT_TRANSPOSE_WUK = 3,     /* index W^UK as [d_c,d_h]             */
+    ORC_FAULT_ROPE_SIGN = 4,         /* rotate the wrong way                */
+    ORC_FAULT_SCAN_NO_RESET = 5,     /* never start a fresh slot            */
+    ORC_FAULT_DROP_ROPE_KEY = 6,     /* score only the latent part          */
+    ORC_FAULT_GATE_WRONG_ROW = 7,    /* use gate row (t+1) mod s            */
+    ORC_FAULT_SCALE = 8,             /* scale by 1/sqrt(d_h)                */
+};
+static int orc_fault = ORC_FAULT_NONE;
+void orc_set_fault(int f) { orc_fault = f; }
+
+static double orc_scale(const orc_cfg* cfg) {
+    if (orc_fault == ORC_FAULT_SCALE) return 1.0 / sqrt((double)cfg->d_h);
+    return cfg->scale != 0.0 ? cfg->scale : 1.0 / sqrt((double)(cfg->d_h + cfg->d_r));
+}
+
+/* Sinusoidal positional embedding of width d at position t. */
+void orc_pe(int64_t t, int32_t d, double base, double* pe) {
+    for (int32_t k = 0; 2 * k < d; ++k) {
+        double ang = (double)t * pow(base, -2.0 * k / (double)d);
+        pe[2 * k] = sin(ang);
+        if (2 * k + 1 < d) pe[2 * k + 1] = cos(ang);
+    }
+}
+
+/* Rotary embedding of a d-vector at position t (interleaved pairs). */
+void orc_rope(int64_t t, int32_t d, double base, const double* x, double* y) {
+    for (int32_t k = 0; k < d / 2; ++k) {
+        double ang = (double)t * pow(base, -2.0 * k / (double)d);
+        if (orc_fault == ORC_FAULT_ROPE_SIGN) ang = -ang;
+        double cs = cos(ang), sn = sin(ang);
+        double x0 = x[2 * k], x1 = x[2 * k + 1];
+        y[2 * k] = x0 * cs - x1 * sn;
+        y[2 * k + 1] = x0 * sn + x1 * cs;
+    }
+}
+
+/* Merging weight of token t (MTLA Sec. 4.1, Eq. 13, under the reading above).
+ * w_given points at the supplied weight in SUPPLIED mode. */
+double orc_gate(const orc_cfg* cfg, int64_t t, const double* c_t, const double* G,
+                const double* g, const double* w_given) {
+    if (cfg->gate_mode == ORC_GATE_UNIT) return 1.0;
+    if (cfg->gate_mode == ORC_GATE_SUPPLIED) return *w_given;
+    int32_t d_c = cfg->d_c;
+    int64_t r = t % cfg->s;
+    if (orc_fault == ORC_FAULT_GATE_WRONG_ROW) r = (t + 1) % cfg->s;
+    double* pe = (double*)malloc(sizeof(double) * d_c);
+    orc_pe(t, d_c, cfg->pe_base, pe);
+    double z = g[r];
+    for (int32_t i = 0; i < d_c; ++i) z += G[r * d_c + i] * (c_t[i] * pe[i]);
+    free(pe);
+    return 1.0 / (1.0 + exp(-z));
+}
+
+/* x_t = [c_t ; RoPE_t(k_t)], the vector a token contributes to its slot. */
+static void orc_token_vector(const orc_cfg* cfg, int64_t t, const double* c_t,
+                             const double* k_t, double* x) {
+    memcpy(x, c_t, sizeof(double) * cfg->d_c);
+    orc_rope(t, cfg->d_r, cfg->rope_base, k_t, x + cfg->d_c);
+}
+
+/* Block-prefix partial slots (MTLA Sec. 4.2-4.3):
+ *   P_t = sum_{u = s*floor(t/s)}^{t} w_u x_u,
+ * written out as that sum for every t. Also returns w [B,T]. */
+void orc_partials(const orc_cfg* cfg, int32_t T, const double* c, const double* kr,
+                  const double* G, const double* g, const double* gate_in,
+                  double* w, double* P) {
+    const int32_t B = cfg->B, d_c = cfg->d_c, d_r = cfg->d_r, s = cfg->s;
+    const int32_t D = d_c + d_r;
+    for (int32_t b = 0; b < B; ++b)
+        for (int32_t t = 0; t < T; ++t) {
+            const double* wg = gate_in ? &gate_in[(int64_t)b * T + t] : NULL;
+            w[(int64_t)b * T + t] = orc_gate(cfg, t, &c[((int64_t)b * T + t) * d_c], G, g, wg);
+        }
+#pragma omp parallel for schedule(static)
+    for (int64_t bt = 0; bt < (int64_t)B * T; ++bt) {
+        int32_t b = (int32_t)(bt / T), t = (int32_t)(bt % T);
+        double* x = (double*)malloc(sizeof(double) * D);
+        double* out = &P[bt * D];
+        for (int32_t k = 0; k < D; ++k) out[k] = 0.0;
+        int32_t u0 = s * (t / s);
+        if (orc_fault == ORC_FAULT_SCAN_NO_RESET) u0 = 0;
+        for (int32_t u = u0; u <= t; ++u) {
+            int64_t bu = (int64_t)b * T + u;
+            orc_token_vector(cfg, u, &c[bu * d_c], &kr[bu * d_r], x);
+            for (int32_t k = 0; k < D; ++k) out[k] += w[bu] * x[k];
+        }
+        free(x);
+    }
+}
+
+/* Absorbed query (MLA absorption, W^UK folded into the query):
+ *   qt = [ W_UK[h]^T qC ; RoPE_t(qR) ]   (width D). */
+static void orc_absorb_query(const orc_cfg* cfg, int64_t t, int32_t h, const double* qc_h,
+                             const double* qr_h, const double* w_uk, double* qt) {
+    const int32_t d_h = cfg->d_h, d_c = cfg->d_c;
+    const double* W = &w_uk[(int64_t)h * d_h * d_c];
+    for (int32_t j = 0; j < d_c; ++j) {
+        double acc = 0.0;
+        for (int32_t i = 0; i < d_h; ++i) {
+            double wij = W[(int64_t)i * d_c + j];
+            if (orc_fault == ORC_FAULT_TRANSPOSE_WUK) {
+                int64_t flat = (int64_t)i * d_c + j; /* read as if stored [d_c, d_h] */
+                wij = W[(flat % d_h) * d_c + flat / d_h];
+            }
+            acc += wij * qc_h[i];
+        }
+        qt[j] = acc;
+    }
+    orc_rope(t, cfg->d_r, cfg->rope_base, qr_h, qt + d_c);
+}
+
+/* Softmax attention of one absorbed query over n key vectors (width D);
+ * returns o_lat = sum_k a_k key_k[0:d_c]. */
+static void orc_attend_keys(const orc_cfg* cfg, const double* qt, int64_t n,
+                            const double* const* keys, double* olat) {
+    const int32_t d_c = cfg->d_c, D = cfg->d_c + cfg->d_r;
+    const double scale = orc_scale(cfg);
+    double* e = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+    double m = -INFINITY;
+    int32_t score_width = (orc_fault == ORC_FAULT_DROP_ROPE_KEY) ? d_c : D;
+    for (int64_t k = 0; k < n; ++k) {
+        double acc = 0.0;
+        for (int32_t j = 0; j < score_width; ++j) acc += qt[j] * keys[k][j];
+        e[k] = scale * acc;
+        if (e[k] > m) m = e[k];
+    }
+    double l = 0.0;
+    for (int64_t k = 0; k < n; ++k) {
+        e[k] = exp(e[k] - m);
+        l += e[k];
+    }
+    for (int32_t j = 0; j < d_c; ++j) olat[j] = 0.0;
+    for (int64_t k = 0; k < n; ++k)
+        for (int32_t j = 0; j < d_c; ++j) olat[j] += (e[k] / l) * keys[k][j];
+    free(e);
+}
+
+/* Output absorption: o = W_UV[h] o_lat (width d_h). */
+static void orc_output(const orc_cfg* cfg, int32_t h, const double* olat, const double* w_uv,
+                       double* o) {
+    const int32_t d_h = cfg->d_h, d_c = cfg->d_c;
+    const double* W = &w_uv[(int64_t)h * d_h * d_c];
+    for (int32_t i = 0; i < d_h; ++i) {
+        double acc = 0.0;
+        for (int32_t j = 0; j < d_c; ++j) acc += W[(int64_t)i * d_c + j] * olat[j];
+        o[i] = acc;
+    }
+}
+
+/* The allowed key set of query i (stride-aware causal mask, MTLA Sec. 4.2):
+ * finished slots F_j = P_{js+s-1} for j < floor(i/s), then the own partial
+ * P_i. Fills `keys` (room for floor(i/s)+2 pointers); returns the count. */
+static int64_t orc_allowed_keys(const orc_cfg* cfg, int32_t T, const double* P_b, int32_t i,
+                                const double** keys) {
+    const int32_t s = cfg->s, D = cfg->d_c + cfg->d_r;
+    int64_t n = 0;
+    int32_t nf = i / s;
+    if (orc_fault == ORC_FAULT_MASK_OFF_BY_ONE) nf = i / s + 1;
+    for (int32_t j = 0; j < nf; ++j) {
+        int32_t u = j * s + s - 1;
+        if (u >= T) u = T - 1;
+        keys[n++] = &P_b[(int64_t)u * D];
+    }
+    if (orc_fault != ORC_FAULT_DROP_OWN_PARTIAL) keys[n++] = &P_b[(int64_t)i * D];
+    return n;
+}
+
+/* Parallel (training-form) attention for selected rows (b, t), all heads.
+ * P is the output of orc_partials. rows holds n_rows pairs (b, t).
+ * out [n_rows,H,d_h]; olat [n_rows,H,d_c] may be NULL. */
+void orc_attend_rows(const orc_cfg* cfg, int32_t T, const double* qc, const double* qr,
+                     const double* w_uk, const double* w_uv, const double* P, int64_t n_rows,
+                     const int64_t* rows, double* out, double* olat_out) {
+    const int32_t H = cfg->H, d_h = cfg->d_h, d_c = cfg->d_c, d_r = cfg->d_r;
+    const int32_t D = d_c + d_r;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t rh = 0; rh < n_rows * H; ++rh) {
+        int64_t r = rh / H;
+        int32_t h = (int32_t)(rh % H);
+        int32_t b = (int32_t)rows[2 * r], t = (int32_t)rows[2 * r + 1];
+        int64_t bth = ((int64_t)b * T + t) * H + h;
+        double* qt = (double*)malloc(sizeof(double) * D);
+        double* olat = (double*)malloc(sizeof(double) * d_c);
+        const double** keys = (const double**)malloc(sizeof(double*) * (size_t)(t / cfg->s + 2));
+        orc_absorb_query(cfg, t, h, &qc[bth * d_h], &qr[bth * d_r], w_uk, qt);
+        int64_t n = orc_allowed_keys(cfg, T, &P[(int64_t)b * T * D], t, keys);
+        orc_attend_keys(cfg, qt, n, keys, olat);
+        orc_output(cfg, h, olat, w_uv, &out[(r * H + h) * d_h]);
+        if (olat_out) memcpy(&olat_out[(r * H + h) * d_c], olat, sizeof(double) * d_c);
+        free(keys);
+        free(olat);
+        free(qt);
+    }
+}
+
+/* Full parallel forward over T tokens from position 0.
+ * out [B,T,H,d_h]; w [B,T]; cache [B,ceil(T/s),D] = the cache after T tokens
+ * (finished slots, then the last, possibly partial, slot); acc [B,D] = P_{T-1}. */
+void orc_prefill(const orc_cfg* cfg, int32_t T, const double* c, const double* kr,
+                 const double* qc, const double* qr, const double* w_uk, const double* w_uv,
+                 const double* G, const double* g, const double* gate_in, double* out,
+                 double* w, double* cache, double* acc) {
+    const int32_t B = cfg->B, s = cfg->s, D = cfg->d_c + cfg->d_r;
+    const int32_t n_slots = (T + s - 1) / s;
+    double* P = (double*)malloc(sizeof(double) * (size_t)B * T * D);
+    orc_partials(cfg, T, c, kr, G, g, gate_in, w, P);
+    int64_t* rows = (int64_t*)malloc(sizeof(int64_t) * 2 * (size_t)B * T);
+    for (int32_t b = 0; b < B; ++b)
+        for (int32_t t = 0; t < T; ++t) {
+            rows[2 * ((int64_t)b * T + t)] = b;
+            rows[2 * ((int64_t)b * T + t) + 1] = t;
+        }
+    orc_attend_rows(cfg, T, qc, qr, w_uk, w_uv, P, (int64_t)B * T, rows, out, NULL);
+    for (int32_t b = 0; b < B; ++b) {
+        for (int32_t j = 0; j < n_slots; ++j) {
+            int32_t u = j * s + s - 1;
+            if (u > T - 1) u = T - 1;
+            memcpy(&cache[((int64_t)b * n_slots + j) * D], &P[((int64_t)b * T + u) * D],
+                   sizeof(double) * D);
+        }
+        if (T > 0)
+            memcpy(&acc[(int64_t)b * D], &P[((int64_t)b * T + T - 1) * D], sizeof(double) * D);
+    }
+    free(rows);
+    free(P);
+}
+
+/* One incremental decode step (MTLA Sec. 4.1 inference): token t = pos[b]
+ * of every sequence. Opens a fresh slot when t mod s == 0, otherwise adds
+ * into the slot being filled in place; then the query attends slots
+ * 0..floor(t/s) of the cache.
+ *   c_new [B,d_c]  kr_new [B,d_r]  qc [B,H,d_h]  qr [B,H,d_r]  gate_in [B]
+ *   cache [B,max_slots,D] in/out   acc [B,D] in/out   out [B,H,d_h]
+ *   w_out [B] and olat_out [B,H,d_c] may be NULL. */
+void orc_decode_step(const orc_cfg* cfg, int32_t max_slots, const double* c_new,
+                     const double* kr_new, const double* qc, const double* qr,
+                     const double* w_uk, const double* w_uv, const double* G, const double* g,
+                     const double* gate_in, const int64_t* pos, double* cache, double* acc,
+                     double* out, double* w_out, double* olat_out) {
+    const int32_t B = cfg->B, H = cfg->H, d_h = cfg->d_h, d_c = cfg->d_c, d_r = cfg->d_r;
+    const int32_t s = cfg->s, D = d_c + d_r;
+    for (int32_t b = 0; b < B; ++b) {
+        int64_t t = pos[b];
+        int64_t j = t / s;
+        const double* wg = gate_in ? &gate_in[b] : NULL;
+        double w = orc_gate(cfg, t, &c_new[(int64_t)b * d_c], G, g, wg);
+        if (w_out) w_out[b] = w;
+        double* x = (double*)malloc(sizeof(double) * D);
+        orc_token_vector(cfg, t, &c_new[(int64_t)b * d_c], &kr_new[(int64_t)b * d_r], x);
+        double* a = &acc[(int64_t)b * D];
+        int fresh = (t % s == 0);
+        if (orc_fault == ORC_FAULT_SCAN_NO_RESET) fresh = (t == 0);
+        for (int32_t k = 0; k < D; ++k) a[k] = (fresh ? 0.0 : a[k]) + w * x[k];
+        memcpy(&cache[((int64_t)b * max_slots + j) * D], a, sizeof(double) * D);
+        free(x);
+    }
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t bh = 0; bh < (int64_t)B * H; ++bh) {
+        int32_t b = (int32_t)(bh / H), h = (int32_t)(bh % H);
+        int64_t t = pos[b];
+        int64_t n = t / s + 1;
+        if (orc_fault == ORC_FAULT_DROP_OWN_PARTIAL) n = t / s;
+        double* qt = (double*)malloc(sizeof(double) * D);
+        double* olat = (double*)malloc(sizeof(double) * d_c);
+        const double** keys = (const double**)malloc(sizeof(double*) * (size_t)(n > 0 ? n : 1));
+        for (int64_t k = 0; k < n; ++k) keys[k] = &cache[((int64_t)b * max_slots + k) * D];
+        orc_absorb_query(cfg, t, h, &qc[bh * d_h], &qr[bh * d_r], w_uk, qt);
+        orc_attend_keys(cfg, qt, n, keys, olat);
+        orc_output(cfg, h, olat, w_uv, &out[bh * d_h]);
+        if (olat_out) memcpy(&olat_out[bh * d_c], olat, sizeof(double) * d_c);
+        free(keys);
+        free(olat);
+        free(qt);
+    }
+}
+
+/* The same parallel forward written without absorption: every allowed slot
+ * is expanded to an explicit per-head key k = [W_UK[h] F[0:d_c] ; F[d_c:]]
+ * and value v = W_UV[h] F[0:d_c]; the query is [qC ; RoPE_t(qR)]. Used to
+ * check the absorbed form (MLA absorption identities). out [B,T,H,d_h]. */
+void orc_prefill_explicit(const orc_cfg* cfg, int32_t T, const double* c, const double* kr,
+                          const double* qc, const double* qr, const double* w_uk,
+                          const double* w_uv, const double* G, const double* g,
+                          const double* gate_in, double* out) {
+    const int32_t B = cfg->B, H = cfg->H, d_h = cfg->d_h, d_c = cfg->d_c, d_r = cfg->d_r;
+    const int32_t D = d_c + d_r;
+    const double scale = orc_scale(cfg);
+    double* P = (double*)malloc(sizeof(double) * (size_t)B * T * D);
+    double* w = (double*)malloc(sizeof(double) * (size_t)B * T);
+    orc_partials(cfg, T, c, kr, G, g, gate_in, w, P);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t bth = 0; bth < (int64_t)B * T * H; ++bth) {
+        int32_t h = (int32_t)(bth % H);
+        int32_t t = (int32_t)((bth / H) % T);
+        int32_t b = (int32_t)(bth / ((int64_t)H * T));
+        const double* Wk = &w_uk[(int64_t)h * d_h * d_c];
+        const double* Wv = &w_uv[(int64_t)h * d_h * d_c];
+        double* q = (double*)malloc(sizeof(double) * (d_h + d_r));
+        memcpy(q, &qc[bth * d_h], sizeof(double) * d_h);
+        orc_rope(t, d_r, cfg->rope_base, &qr[bth * d_r], q + d_h);
+        const double** keys = (const double**)malloc(sizeof(double*) * (size_t)(t / cfg->s + 2));
+        int64_t n = orc_allowed_keys(cfg, T, &P[(int64_t)b * T * D], t, keys);
+        double* e = (double*)malloc(sizeof(double) * (size_t)n);
+        double* kfull = (double*)malloc(sizeof(double) * (d_h + d_r));
+        double m = -INFINITY;
+        for (int64_t k = 0; k < n; ++k) {
+            for (int32_t i = 0; i < d_h; ++i) {
+                double acc = 0.0;
+                for (int32_t j = 0; j < d_c; ++j) acc += Wk[(int64_t)i * d_c + j] * keys[k][j];
+                kfull[i] = acc;
+            }
+            for (int32_t r = 0; r < d_r; ++r) kfull[d_h + r] = keys[k][d_c + r];
+            double dot = 0.0;
+            for (int32_t i = 0; i < d_h + d_r; ++i) dot += q[i] * kfull[i];
+            e[k] = scale * dot;
+            if (e[k] > m) m = e[k];
+        }
+        double l = 0.0;
+        for (int64_t k = 0; k < n; ++k) {
+            e[k] = exp(e[k] - m);
+            l += e[k];
+        }
+        double* o = &out[bth * d_h];
+        for (int32_t i = 0; i < d_h; ++i) o[i] = 0.0;
+        for (int64_t k = 0; k < n; ++k)
+            for (int32_t i = 0; i < d_h; ++i) {
+                double v = 0.0;
+                for (int32_t j = 0; j < d_c; ++j) v += Wv[(int64_t)i * d_c + j] * keys[k][j];
+                o[i] += (e[k] / l) * v;
+            }
+        free(kfull);
+        free(e);
+        free(keys);
+        free(q);
+    }
+    free(w);
+    free(P);
+}

@@ -1,0 +1,325 @@
+"""CPU pins for the float64 oracle: checks against what the pages and the
+mathematics fix, none of which retypes the oracle's own formulas.
+
+- printed values: the 9/(4s) cache footprint ("Multi-head Temporal Latent
+  Attention", Key claims, Sec. 4.3) and the 1,152 B latent slot ("Multi-Head
+  Latent Attention and Sparse Indexers", "Work the bytes with units and scope"),
+  as fixtures in tests/golden/cache_footprint.txt;
+- special case reducing to a library routine: s = 1 with unit gates is MLA,
+  i.e. causal softmax attention on explicit keys/values (torch SDPA, float64);
+- algebraic identity: absorbed form == explicit (non-absorbed) form (MLA
+  absorption identities);
+- invariant: incremental decoding == parallel masked forward (Sec. 4.2);
+- brute force: dense enumerated mask over per-token partial slots (tests/brute_force.py);
+- closed forms of the scan, the gate modes, PE and RoPE.
+Finally, each planted mistake in the oracle must trip at least one pin.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import brute_force as bf
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "cache_footprint.txt")
+
+
+def _golden():
+    vals = {}
+    with open(GOLDEN) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            k, v = line.split()
+            vals[k] = float(v)
+    return vals
+
+
+def _rand_problem(B, H, d_h, d_c, d_r, s, T, seed, gate_mode=oracle.GATE_COMPUTED):
+    rng = np.random.default_rng(seed)
+    cfg = oracle.Cfg(B, H, d_h, d_c, d_r, s, gate_mode=gate_mode)
+    p = dict(
+        c=rng.standard_normal((B, T, d_c)),
+        kr=rng.standard_normal((B, T, d_r)),
+        qc=rng.standard_normal((B, T, H, d_h)),
+        qr=rng.standard_normal((B, T, H, d_r)),
+        w_uk=rng.standard_normal((H, d_h, d_c)) / math.sqrt(d_c),
+        w_uv=rng.standard_normal((H, d_h, d_c)) / math.sqrt(d_c),
+        G=rng.standard_normal((s, d_c)) / math.sqrt(d_c),
+        g=rng.standard_normal(s) * 0.5,
+        gate_in=1.0 / (1.0 + np.exp(-rng.standard_normal((B, T)))),
+    )
+    return cfg, p
+
+
+# --------------------------------------------------------------------------- pins
+
+
+def pin_cache_footprint():
+    """Slot count * width per token equals the printed 9/(4s) (MQA units of 2 d_h),
+    and the GLM latent slot equals the printed byte counts."""
+    gold = _golden()
+    d_h = 64
+    for s in (1, 2, 3, 4):
+        cfg = oracle.Cfg(1, 1, d_h, 4 * d_h, d_h // 2, s, gate_mode=oracle.GATE_UNIT)
+        T = 12 * s
+        rng = np.random.default_rng(s)
+        res = oracle.prefill(cfg, rng.standard_normal((1, T, cfg.d_c)),
+                             rng.standard_normal((1, T, cfg.d_r)),
+                             rng.standard_normal((1, T, 1, d_h)),
+                             rng.standard_normal((1, T, 1, cfg.d_r)),
+                             rng.standard_normal((1, d_h, cfg.d_c)),
+                             rng.standard_normal((1, d_h, cfg.d_c)))
+        n_slots, width = res["cache"].shape[1:]
+        per_token = n_slots * width / T / (2 * d_h)
+        if abs(per_token - gold[f"mtla_elements_per_token_s{s}"]) > 1e-12:
+            return False
+    cfg = oracle.Cfg(1, 1, 128, 512, 64, 1, gate_mode=oracle.GATE_UNIT)
+    rng = np.random.default_rng(0)
+    T = 3
+    res = oracle.prefill(cfg, rng.standard_normal((1, T, 512)), rng.standard_normal((1, T, 64)),
+                         rng.standard_normal((1, T, 1, 128)), rng.standard_normal((1, T, 1, 64)),
+                         rng.standard_normal((1, 128, 512)), rng.standard_normal((1, 128, 512)))
+    bytes_per_pos = res["cache"].shape[2] * 2 * res["cache"].shape[1] // T   # bf16
+    return (bytes_per_pos == gold["glm_bytes_per_layer_position"]
+            and bytes_per_pos * 78 == gold["glm_bytes_per_position_78_layers"]
+            and bytes_per_pos * 78 * 1048576 == gold["glm_bytes_1048576_positions_78_layers"])
+
+
+def pin_s1_is_mla_sdpa():
+    """s = 1, unit gates: MTLA == MLA == causal attention on explicit k, v."""
+    B, H, d_h, d_c, d_r, T = 2, 3, 8, 16, 4, 9
+    cfg, p = _rand_problem(B, H, d_h, d_c, d_r, 1, T, seed=11, gate_mode=oracle.GATE_UNIT)
+    got = oracle.prefill(cfg, p["c"], p["kr"], p["qc"], p["qr"], p["w_uk"], p["w_uv"])["out"]
+    # explicit keys/values, RoPE applied through the oracle's rotation
+    kr_rot = np.stack([np.stack([oracle.rope(t, p["kr"][b, t]) for t in range(T)])
+                       for b in range(B)])
+    qr_rot = np.stack([np.stack([np.stack([oracle.rope(t, p["qr"][b, t, h]) for h in range(H)])
+                                 for t in range(T)]) for b in range(B)])
+    c = torch.tensor(p["c"])
+    w_uk = torch.tensor(p["w_uk"])
+    w_uv = torch.tensor(p["w_uv"])
+    k = torch.cat([torch.einsum("btc,hdc->bhtd", c, w_uk),
+                   torch.tensor(kr_rot)[:, None].expand(B, H, T, d_r)], dim=-1)
+    v = torch.einsum("btc,hdc->bhtd", c, w_uv)
+    q = torch.cat([torch.tensor(p["qc"]).permute(0, 2, 1, 3),
+                   torch.tensor(qr_rot).permute(0, 2, 1, 3)], dim=-1)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        q, k, v, is_causal=True, scale=1.0 / math.sqrt(d_h + d_r))
+    ref = ref.permute(0, 2, 1, 3).numpy()
+    return np.max(np.abs(got - ref)) < 1e-12
+
+
+def pin_absorbed_equals_explicit():
+    for s in (1, 2, 3, 4):
+        cfg, p = _rand_problem(2, 2, 8, 24, 4, s, 11, seed=20 + s)
+        a = oracle.prefill(cfg, p["c"], p["kr"], p["qc"], p["qr"], p["w_uk"], p["w_uv"],
+                           p["G"], p["g"])["out"]
+        e = oracle.prefill_explicit(cfg, p["c"], p["kr"], p["qc"], p["qr"], p["w_uk"],
+                                    p["w_uv"], p["G"], p["g"])
+        if not np.max(np.abs(a - e)) < 1e-12:
+            return False
+    return True
+
+
+def pin_incremental_equals_parallel():
+    for s in (1, 2, 3, 4):
+        B, T = 2, 13
+        cfg, p = _rand_problem(B, 2, 8, 16, 4, s, T, seed=40 + s)
+        par = oracle.prefill(cfg, p["c"], p["kr"], p["qc"], p["qr"], p["w_uk"], p["w_uv"],
+                             p["G"], p["g"])
+        max_slots = (T + s - 1) // s + 1
+        cache = np.zeros((B, max_slots, cfg.D))
+        acc = np.zeros((B, cfg.D))
+        outs = []
+        for t in range(T):
+            r = oracle.decode_step(cfg, p["c"][:, t], p["kr"][:, t], p["qc"][:, t], p["qr"][:, t],
+                                   p["w_uk"], p["w_uv"], np.full(B, t), cache, acc,
+                                   p["G"], p["g"])
+            outs.append(r["out"])
+        inc = np.stack(outs, axis=1)
+        n = (T + s - 1) // s
+        if not (np.max(np.abs(inc - par["out"])) < 1e-12
+                and np.max(np.abs(cache[:, :n] - par["cache"])) < 1e-12
+                and np.max(np.abs(acc - par["acc"])) < 1e-12):
+            return False
+    return True
+
+
+def pin_brute_force():
+    for s in (1, 2, 3, 4):
+        for T in (1, s, 7, 16):
+            B, H, d_h, d_c, d_r = 1, 2, 4, 8, 4
+            cfg, p = _rand_problem(B, H, d_h, d_c, d_r, s, T, seed=60 + s * 17 + T,
+                                   gate_mode=oracle.GATE_SUPPLIED)
+            got = oracle.prefill(cfg, p["c"], p["kr"], p["qc"], p["qr"], p["w_uk"], p["w_uv"],
+                                 gate_in=p["gate_in"])
+            x = np.concatenate([p["c"][0], np.stack([oracle.rope(t, p["kr"][0, t])
+                                                     for t in range(T)])], axis=1)
+            P = bf.running_slots(x, p["gate_in"][0], s)
+            q_full = np.concatenate(
+                [p["qc"][0], np.stack([np.stack([oracle.rope(t, p["qr"][0, t, h])
+                                                 for h in range(H)]) for t in range(T)])], axis=2)
+            ref = bf.attention(q_full, P, p["w_uk"], p["w_uv"], s, d_c,
+                               bf.softmax_scale(d_h, d_r))
+            if not np.max(np.abs(got["out"][0] - ref)) < 1e-12:
+                return False
+            mask = bf.dense_mask(T, s)
+            if any(mask[i].sum() != i // s + 1 for i in range(T)):
+                return False
+    return True
+
+
+def pin_scan_closed_form():
+    """Unit gates and all-ones latents: P_t = (t mod s + 1) * 1 on the latent
+    part; finished slots hold s; the cache has ceil(T/s) slots."""
+    for s in (1, 2, 3, 4):
+        T, d_c, d_r = 10, 8, 4
+        cfg = oracle.Cfg(1, 1, 4, d_c, d_r, s, gate_mode=oracle.GATE_UNIT)
+        w, P = oracle.partials(cfg, np.ones((1, T, d_c)), np.zeros((1, T, d_r)))
+        expect = np.array([(t % s) + 1 for t in range(T)], dtype=float)
+        if not (np.all(w == 1.0) and np.allclose(P[0, :, :d_c], expect[:, None], atol=0)
+                and np.all(P[0, :, d_c:] == 0.0)):
+            return False
+        res = oracle.prefill(cfg, np.ones((1, T, d_c)), np.zeros((1, T, d_r)),
+                             np.zeros((1, T, 1, 4)), np.zeros((1, T, 1, d_r)),
+                             np.zeros((1, 4, d_c)), np.zeros((1, 4, d_c)))
+        n = math.ceil(T / s)
+        if res["cache"].shape[1] != n:
+            return False
+        for j in range(n):
+            full = min(s, T - j * s)
+            if not np.all(res["cache"][0, j, :d_c] == full):
+                return False
+    return True
+
+
+def pin_gate_modes():
+    """UNIT -> 1; SUPPLIED passes through; COMPUTED with a zero row r gives
+    sigmoid(g[r]) for tokens t = r mod s; at t = 0 the PE is (0,1,0,1,...) so
+    only the odd latent entries reach the gate."""
+    d_c, s = 8, 3
+    rng = np.random.default_rng(5)
+    c = rng.standard_normal(d_c)
+    G = rng.standard_normal((s, d_c))
+    g = np.array([0.3, -1.2, 2.0])
+    sig = lambda z: 1.0 / (1.0 + math.exp(-z))
+    if oracle.gate(oracle.Cfg(1, 1, 4, d_c, 4, s, gate_mode=oracle.GATE_UNIT), 5, c, G, g) != 1.0:
+        return False
+    if oracle.gate(oracle.Cfg(1, 1, 4, d_c, 4, s, gate_mode=oracle.GATE_SUPPLIED), 5, c, G, g,
+                   w_given=0.37) != 0.37:
+        return False
+    cfg = oracle.Cfg(1, 1, 4, d_c, 4, s)
+    for r in range(s):
+        Gz = G.copy()
+        Gz[r] = 0.0
+        for t in (r, r + s, r + 5 * s):
+            if abs(oracle.gate(cfg, t, c, Gz, g) - sig(g[r])) > 1e-15:
+                return False
+    z0 = g[0] + sum(G[0, i] * c[i] for i in range(1, d_c, 2))
+    return abs(oracle.gate(cfg, 0, c, G, g) - sig(z0)) < 1e-14
+
+
+def pin_rope():
+    """Rotation of pairs: t = 0 is the identity, every pair keeps its norm,
+    scores depend only on the position difference, and the rotation is
+    counter-clockwise (RoFormer's matrix) -- the last is a convention."""
+    rng = np.random.default_rng(9)
+    d = 16
+    q, k = rng.standard_normal(d), rng.standard_normal(d)
+    if not np.array_equal(oracle.rope(0, q), q):
+        return False
+    y = oracle.rope(37, q)
+    if not np.allclose((y[0::2] ** 2 + y[1::2] ** 2), (q[0::2] ** 2 + q[1::2] ** 2), atol=1e-13):
+        return False
+    for m, n, dlt in ((3, 11, 5), (100, 7, 1000), (0, 64, 4095)):
+        a = oracle.rope(m, q) @ oracle.rope(n, k)
+        b = oracle.rope(m + dlt, q) @ oracle.rope(n + dlt, k)
+        if abs(a - b) > 1e-9:
+            return False
+    e0 = np.zeros(d)
+    e0[0] = 1.0
+    y = oracle.rope(1, e0)
+    return abs(y[0] - math.cos(1.0)) < 1e-15 and abs(y[1] - math.sin(1.0)) < 1e-15
+
+
+def pin_pe():
+    d = 32
+    pe0 = oracle.pe(0, d)
+    if not (np.all(pe0[0::2] == 0.0) and np.all(pe0[1::2] == 1.0)):
+        return False
+    for t in (1, 17, 5000):
+        p = oracle.pe(t, d)
+        if not np.allclose(p[0::2] ** 2 + p[1::2] ** 2, 1.0, atol=1e-14):
+            return False
+        if abs(p[0] - math.sin(t)) > 1e-12:      # the first pair turns at unit frequency
+            return False
+    return True
+
+
+PINS = {
+    "cache_footprint": pin_cache_footprint,
+    "s1_is_mla_sdpa": pin_s1_is_mla_sdpa,
+    "absorbed_equals_explicit": pin_absorbed_equals_explicit,
+    "incremental_equals_parallel": pin_incremental_equals_parallel,
+    "brute_force": pin_brute_force,
+    "scan_closed_form": pin_scan_closed_form,
+    "gate_modes": pin_gate_modes,
+    "rope": pin_rope,
+    "pe": pin_pe,
+}
+
+
+@pytest.fixture(autouse=True)
+def _no_fault():
+    oracle.set_fault(oracle.FAULT_NONE)
+    yield
+    oracle.set_fault(oracle.FAULT_NONE)
+
+
+@pytest.mark.parametrize("name", sorted(PINS))
+def test_pin(name):
+    assert PINS[name](), f"oracle pin {name} failed"
+
+
+FAULTS = {
+    "drop_own_partial": oracle.FAULT_DROP_OWN_PARTIAL,
+    "mask_off_by_one": oracle.FAULT_MASK_OFF_BY_ONE,
+    "transpose_wuk": oracle.FAULT_TRANSPOSE_WUK,
+    "rope_sign": oracle.FAULT_ROPE_SIGN,
+    "scan_no_reset": oracle.FAULT_SCAN_NO_RESET,
+    "drop_rope_key": oracle.FAULT_DROP_ROPE_KEY,
+    "gate_wrong_row": oracle.FAULT_GATE_WRONG_ROW,
+    "scale": oracle.FAULT_SCALE,
+}
+
+
+@pytest.mark.parametrize("fault", sorted(FAULTS))
+def test_planted_mistake_is_caught(fault):
+    oracle.set_fault(FAULTS[fault])
+    failed = [name for name, pin in PINS.items() if not pin()]
+    assert failed, f"planted mistake {fault} passed every pin"
+
+
+def test_mask_probe_support():
+    """The one-hot probe used for the GPU mask test: zero queries and unit gates
+    give o_lat = mean of e_j over the slots query i attends, i.e. support
+    {0..floor(i/s)} (oracle side of the bit-exact mask test)."""
+    from kv_cache_mtla_b200 import inputs
+    for s in (1, 2, 3, 4):
+        wl = inputs.TINY_FP32.with_(s=s, gate_mode=inputs.GATE_UNIT)
+        T = 23
+        p = inputs.one_hot_mask_probe(wl, T)
+        cfg = oracle.Cfg(wl.B, wl.H, wl.d_h, wl.d_c, wl.d_r, s, gate_mode=oracle.GATE_UNIT)
+        _, P = oracle.partials(cfg, p["c"], p["kr"])
+        rows = np.array([[0, t] for t in range(T)])
+        w = np.zeros((wl.H, wl.d_h, wl.d_c))
+        _, olat = oracle.attend_rows(cfg, p["qc"], p["qr"], w, w, P, rows, want_olat=True)
+        for t in range(T):
+            support = np.nonzero(olat[t, 0])[0]
+            assert list(support) == list(range(t // s + 1))
+            assert np.allclose(olat[t, 0, support], 1.0 / (t // s + 1), atol=1e-15)
