@@ -1,0 +1,371 @@
+#!/usr/bin/env python
+"""Throughput of the MTLA hot path on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mtla|reference]
+
+Workload (per rank; weak scaling, every rank runs an independent replica):
+the speech-model-scale decode -- B=16 sequences, H=8, d_h=64, d_c=256,
+d_R=32, s=2 -- one step = the parallel prefill of a 1024-token prefix
+(512 slots) followed by 256 incremental decode steps (513..640 slots), i.e.
+every stage of the path: gate, RoPE, block-prefix scan / in-place slot update,
+query absorption, stride-aware masked attention, split merge, output
+absorption. Inputs are seeded synthetic draws (kv_cache_mtla_b200.inputs).
+
+`value` = tokens processed (prefix + decoded) per second over all ranks, from
+CUDA events around each step on the launching stream, the L2 flushed (a
+256 MiB write) before every step outside the events. `e2e` times the same
+steps through the public API with the step's inputs copied from pinned host
+memory and its outputs copied back inside the timed region. `roofline` reports
+the dominant kernel (decode attention) timed by event pairs the library
+records around it. `cpu_baseline` / `--impl reference` time the float64 CPU
+oracle on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from kv_cache_mtla_b200 import inputs, mtla  # noqa: E402
+
+METRIC = "decode latent-cache GB/s and tokens/s at N/s slots; prefill TFLOP/s; % roofline"
+WL = inputs.SPEECH_DECODE
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return ws, rank
+
+
+def _max_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def _barrier(ws: int):
+    if ws > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, dev_index: int):
+        self.dev = dev_index
+        self.proc = None
+        self.path = f"/tmp/mtla_clocks_{os.getpid()}.csv"
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sms, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sms.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        return {"sm_mhz": statistics.median(sms) if sms else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sms)}
+
+
+class Replica:
+    """One rank's problem: weights, cache, inputs of a whole step on the device."""
+
+    def __init__(self, rank: int):
+        wl = WL.with_(seed=WL.seed + 1000 * rank)
+        self.wl = wl
+        self.T, self.S = wl.T, wl.steps
+        self.max_slots = (self.T + self.S + wl.s - 1) // wl.s
+        self.cfg = mtla.make_config(wl.B, wl.H, wl.d_h, wl.d_c, wl.d_r, wl.s, self.max_slots,
+                                    dtype=wl.dtype, gate_mode=wl.gate_mode)
+        self.buf = mtla.Buffers.allocate(self.cfg, inputs.weights(wl), max_tokens=self.T)
+        bf = torch.bfloat16
+        pre = inputs.tokens(wl, self.T, stream=0)
+        dec = inputs.tokens(wl, self.S, stream=1)
+        # host copies (pinned) of one step's inputs, and their device twins
+        self.h = {k: pre[k].to(bf).contiguous().pin_memory() for k in ("c", "kr", "qc", "qr")}
+        for k in ("c", "kr", "qc", "qr"):      # decode tokens, step-major [S, B, ...]
+            self.h["d_" + k] = dec[k].transpose(0, 1).to(bf).contiguous().pin_memory()
+        self.d = {k: v.to("cuda") for k, v in self.h.items()}
+        self.pos = (self.T + torch.arange(self.S, dtype=torch.int32)).repeat_interleave(wl.B)
+        self.pos = self.pos.view(self.S, wl.B).contiguous().to("cuda")
+        self.out_p = torch.empty(wl.B, self.T, wl.H, wl.d_h, device="cuda", dtype=bf)
+        self.out_d = torch.empty(self.S, wl.B, wl.H, wl.d_h, device="cuda", dtype=bf)
+        self.h_out_p = torch.empty(self.out_p.shape, dtype=bf).pin_memory()
+        self.h_out_d = torch.empty(self.out_d.shape, dtype=bf).pin_memory()
+        self.h2d_bytes = sum(v.numel() * v.element_size() for v in self.h.values())
+        self.d2h_bytes = (self.out_p.numel() + self.out_d.numel()) * 2
+        self.tokens_per_step = wl.B * (self.T + self.S)
+
+    def prefill(self):
+        b = self.buf
+        mtla.prefill(self.cfg, self.T, self.d["c"], self.d["kr"], self.d["qc"], self.d["qr"],
+                     b.w_uk, b.w_uv, b.gate_w, b.gate_b, None, self.out_p, b.cache, b.open_slot,
+                     b.workspace)
+
+    def decode(self, k: int):
+        b, d = self.buf, self.d
+        mtla.decode_step(self.cfg, d["d_c"][k], d["d_kr"][k], d["d_qc"][k], d["d_qr"][k], b.w_uk,
+                         b.w_uv, b.gate_w, b.gate_b, None, self.pos[k], b.cache, b.open_slot,
+                         self.out_d[k], b.workspace)
+
+    def step(self, ev=None):
+        self.prefill()
+        if ev is not None:
+            ev.record()
+        for k in range(self.S):
+            self.decode(k)
+
+    def slots_read_per_decode(self):
+        """Slots the k-th decode step attends per sequence: floor(t/s) + 1."""
+        return [(self.T + k) // self.wl.s + 1 for k in range(self.S)]
+
+
+def _cpu_sample(n_decode: int = 8):
+    """The oracle on a bounded sample of the workload: one of the B sequences,
+    the parallel prefill of its 1024-token prefix, then n_decode incremental
+    steps from the oracle's own cache. Returns (tokens, seconds, threads)."""
+    import numpy as np
+
+    import oracle
+    wl = WL.with_(B=1)
+    w = inputs.weights(WL)
+    pre = inputs.tokens(WL, WL.T, stream=0)
+    dec = inputs.tokens(WL, n_decode, stream=1)
+    one = lambda d: {k: (None if v is None else v[:1]) for k, v in d.items()}
+    pre, dec = one(pre), one(dec)
+    cfg = oracle.Cfg(1, wl.H, wl.d_h, wl.d_c, wl.d_r, wl.s, gate_mode=wl.gate_mode)
+    oracle.build()
+    t0 = time.perf_counter()
+    r = oracle.prefill(cfg, pre["c"], pre["kr"], pre["qc"], pre["qr"], w["w_uk"], w["w_uv"],
+                       w["gate_w"], w["gate_b"])
+    max_slots = (WL.T + n_decode + wl.s - 1) // wl.s
+    cache = np.zeros((1, max_slots, wl.D))
+    n = r["cache"].shape[1]
+    cache[:, :n] = r["cache"]
+    acc = r["acc"].copy()
+    for k in range(n_decode):
+        oracle.decode_step(cfg, dec["c"][:, k], dec["kr"][:, k], dec["qc"][:, k], dec["qr"][:, k],
+                           w["w_uk"], w["w_uv"], [WL.T + k], cache, acc, w["gate_w"], w["gate_b"])
+    dt = time.perf_counter() - t0
+    threads = int(os.environ.get("OMP_NUM_THREADS", "0")) or len(os.sched_getaffinity(0))
+    return WL.T + n_decode, dt, threads
+
+
+def _config(ws: int):
+    return {"workload": "speech_decode: B=16/rank, H=8, d_h=64, d_c=256, d_R=32, s=2; "
+                        "prefill 1024 tokens then 256 decode steps",
+            "global_batch": WL.B * ws, "prefix_tokens": WL.T, "decode_steps": WL.steps,
+            "seq_len": WL.T + WL.steps, "parallelism": f"replicas x{ws} (independent sequences)",
+            "l2": "flushed (256 MiB write) before every timed step"}
+
+
+def run_reference(args, ws, rank):
+    if rank != 0:
+        return
+    times, toks, threads = [], 0, 1
+    for i in range(args.warmup + args.steps):
+        n, dt, threads = _cpu_sample()
+        if i >= args.warmup:
+            times.append(dt)
+            toks += n
+    total = sum(times)
+    value = toks / total
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": _config(ws),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": "per step: 1 of 16 sequences, parallel prefill of 1024 tokens + "
+                                   "8 incremental decode steps (float64 C oracle, OpenMP)"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="mtla", choices=["mtla", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    ws, rank = _dist()
+    if args.impl == "reference":
+        run_reference(args, ws, rank)
+        if ws > 1:
+            torch.distributed.destroy_process_group()
+        return
+
+    rep = Replica(rank)
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device="cuda")  # 256 MiB > L2
+    st = torch.cuda.current_stream()
+
+    for _ in range(args.warmup):
+        rep.step()
+    torch.cuda.synchronize()
+    assert mtla.get_device_status() == mtla.OK
+
+    # ---- device-timed steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+            torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    prof = mtla.ProfileEvents(args.steps * (1 + rep.S))
+    launches0 = mtla.kernel_launches()
+    _barrier(ws)
+    with ClockSampler(torch.cuda.current_device()) as clk, prof:
+        for i in range(args.steps):
+            flush.zero_()
+            evs[i][0].record(st)
+            rep.step(evs[i][1])
+            evs[i][2].record(st)
+        torch.cuda.synchronize()
+    _barrier(ws)
+    launches = mtla.kernel_launches() - launches0
+    assert mtla.get_device_status() == mtla.OK
+    step_ms = [a.elapsed_time(c) for a, b, c in evs]
+    pre_ms = [a.elapsed_time(b) for a, b, c in evs]
+    dec_ms = [b.elapsed_time(c) for a, b, c in evs]
+    total_ms = _max_over_ranks(sum(step_ms), ws)
+    value = rep.tokens_per_step * ws * args.steps / (total_ms / 1e3)
+
+    # dominant kernel: decode attention (every call's pair after its prefill pair)
+    durs = prof.durations_ms()
+    per_step = 1 + rep.S
+    attn = [durs[i * per_step + 1 + k] for i in range(args.steps) for k in range(rep.S)]
+    pre_attn = [durs[i * per_step] for i in range(args.steps)]
+    slot_bytes = rep.wl.D * 2
+    slots = rep.slots_read_per_decode()
+    bytes_per_launch = rep.wl.B * slot_bytes * sum(slots) / len(slots)
+    attn_ms = statistics.mean(attn)
+    hbm, tflops_peak, peak_kind = _peaks()
+    achieved = bytes_per_launch / (attn_ms / 1e3) / 1e9
+    # prefill attention flops: 2 * allowed pairs * (D + d_c) * B * H
+    wl = rep.wl
+    pairs = sum(t // wl.s + 1 for t in range(rep.T))
+    pre_flops = 2 * pairs * (wl.D + wl.d_c) * wl.B * wl.H
+    dec_tokens = wl.B * rep.S
+    dec_s = _max_over_ranks(sum(dec_ms), ws) / 1e3
+
+    # ---- end to end through the public API with host buffers
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(args.steps)]
+    _barrier(ws)
+    for i in range(args.steps):
+        flush.zero_()
+        e2e_ev[i][0].record(st)
+        for k, v in rep.h.items():
+            rep.d[k].copy_(v, non_blocking=True)
+        rep.step()
+        rep.h_out_p.copy_(rep.out_p, non_blocking=True)
+        rep.h_out_d.copy_(rep.out_d, non_blocking=True)
+        e2e_ev[i][1].record(st)
+    torch.cuda.synchronize()
+    _barrier(ws)
+    e2e_ms = _max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev), ws)
+    e2e_value = rep.tokens_per_step * ws * args.steps / (e2e_ms / 1e3)
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        n, dt, threads = _cpu_sample()
+        cpu = {"value": n / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+               "sample": f"1 of 16 sequences: parallel prefill of {WL.T} tokens + 8 incremental "
+                         f"decode steps ({dt:.1f} s, float64 C oracle, OpenMP)"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) inputs, random-init weights)",
+            "config": _config(ws),
+            "decode": {"tokens_per_s": dec_tokens * ws / dec_s,
+                       "ms_per_token_step": 1e3 * dec_s / (rep.S * args.steps),
+                       "latent_cache_GBps": wl.B * slot_bytes * sum(slots) * args.steps / dec_s / 1e9,
+                       "slots_per_seq": [slots[0], slots[-1]]},
+            "prefill": {"ms": statistics.mean(pre_ms), "attention_kernel_ms": statistics.mean(pre_attn),
+                        "TFLOPs": pre_flops / (statistics.mean(pre_ms) / 1e3) / 1e12},
+            "roofline": {"kernel": "decode attention", "bound": "hbm", "achieved": achieved,
+                         "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "traffic": None,
+                         "peak_source": f"{peak_kind} hbm_gbs",
+                         "bytes_per_launch": bytes_per_launch, "avg_launch_us": attn_ms * 1e3},
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": rep.h2d_bytes,
+                    "d2h_bytes_per_step": rep.d2h_bytes},
+            "gpu_launches": launches,
+            "clocks": clk.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

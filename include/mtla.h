@@ -1,0 +1,185 @@
+/*
+ * mtla.h -- C ABI of the B200 (sm_100a) MTLA attention library, libmtla.so.
+ *
+ * MTLA (Multi-head Temporal Latent Attention) attends over a KV cache that is
+ * compressed twice: every token is reduced to an MLA-style latent c_t (width
+ * d_c) plus one decoupled-RoPE key k_t (width d_r), and every s consecutive
+ * tokens are merged into one cache slot by a learned gate,
+ *   slot_j = sum_{t in block j} w_t [c_t ; RoPE_t(k_t)].
+ * Queries attend the slots in the absorbed form (W_UK folded into the query,
+ * W_UV applied after the weighted sum) under the stride-aware causal mask:
+ * query t sees every finished slot j < floor(t/s) plus its own slot while it
+ * is being filled.
+ *
+ * Sources (page titles and the sections they name):
+ *   "Multi-head Temporal Latent Attention" (paper summary page), Method:
+ *     (1) merging weights from a hyper-network on the latent times a
+ *         positional embedding (Sec. 4.1, Eq. 13), and the in-place update of
+ *         the slot being filled at inference;
+ *     (2) the stride-aware causal mask for parallel training (Sec. 4.2,
+ *         Fig. 2(c));
+ *     (3) decoupled-RoPE keys merged along the same axis with the same mask
+ *         (Sec. 4.3, Eq. 17); absorption of W^UK and W^UV kept from MLA.
+ *   "Multi-Head Latent Attention and Sparse Indexers", "Latent attention
+ *     changes the representation": q.(U_K c) = (U_K^T q).c and
+ *     sum_j a_j U_V c_j = U_V sum_j a_j c_j.
+ *
+ * Readings where the pages are silent (fixed by this ABI):
+ *   - slots are 0-based: token t lives in slot floor(t/s);
+ *   - w_t = sigmoid(G[t mod s] . (c_t * PE_t) + g[t mod s]) with PE_t the
+ *     interleaved sinusoid of width d_c and base 10000 (MTLA_GATE_COMPUTED);
+ *     the gate may instead be supplied per token (MTLA_GATE_SUPPLIED) or fixed
+ *     to 1 (MTLA_GATE_UNIT);
+ *   - RoPE rotates interleaved pairs (x_2k, x_2k+1) by t * base^(-2k/d_r);
+ *   - the absorbed query is q~ = [W_UK[h]^T qC ; RoPE_t(qR)], the score
+ *     scale * <q~, slot>, the output o = W_UV[h] (sum_j a_j slot_j[0:d_c]).
+ *
+ * Conventions common to every call:
+ *   - All tensors are dense, row-major, on the current CUDA device, and the
+ *     caller owns them. Every pointer must be 16-byte aligned.
+ *   - Storage type: MTLA_BF16 stores activations, weights, cache and output in
+ *     bfloat16 (round-to-nearest-even) and computes in fp32; MTLA_FP32 stores
+ *     and computes everything in fp32 (no tensor-float rounding anywhere).
+ *     Gate parameters, supplied gates and the open-slot accumulator are
+ *     always float32.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy
+ *     default stream) and allocate nothing: scratch comes from `workspace`,
+ *     whose size mtla_workspace_size() reports.
+ *   - Argument errors are found on the host before anything is launched and
+ *     returned as a status; nothing is written then. Errors found on the
+ *     device (a position beyond the cache, a bounded wait that ran out) skip
+ *     the affected work and are latched in a device status word that
+ *     mtla_get_device_status() reads.
+ */
+#ifndef MTLA_H_
+#define MTLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MTLA_OK = 0,
+    MTLA_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size or enum      */
+    MTLA_ERR_UNSUPPORTED = 2,   /* valid MTLA shape this build has no kernel for  */
+    MTLA_ERR_CAPACITY = 3,      /* a position does not fit in max_slots slots     */
+    MTLA_ERR_CUDA = 4,          /* a CUDA runtime call failed                     */
+    MTLA_ERR_TIMEOUT = 5,       /* a bounded device wait ran out (device status)  */
+    MTLA_ERR_WORKSPACE = 6      /* workspace smaller than mtla_workspace_size()   */
+} mtla_status;
+
+typedef enum { MTLA_BF16 = 0, MTLA_FP32 = 1 } mtla_dtype;
+
+typedef enum {
+    MTLA_GATE_COMPUTED = 0,     /* w_t from gate_w, gate_b and the PE (Eq. 13)   */
+    MTLA_GATE_SUPPLIED = 1,     /* w_t read from gate_in                         */
+    MTLA_GATE_UNIT = 2          /* w_t = 1                                       */
+} mtla_gate_mode;
+
+/* Problem description shared by every call.
+ * Supported: 1 <= batch; 1 <= heads <= 128; d_h, d_c, d_r multiples of 16;
+ * d_c + d_r <= 576; d_h <= 256; 1 <= stride <= 8; max_slots >= 1.
+ * Anything else: MTLA_ERR_UNSUPPORTED (or INVALID_ARG for non-positive sizes). */
+typedef struct {
+    int32_t batch;          /* B: sequences                                       */
+    int32_t heads;          /* H: query heads (all share the cache, MQA form)     */
+    int32_t d_h;            /* per-head width of qC and of the output             */
+    int32_t d_c;            /* latent width                                       */
+    int32_t d_r;            /* decoupled-RoPE width of keys and query parts       */
+    int32_t stride;         /* s: tokens merged into one slot                     */
+    int32_t dtype;          /* mtla_dtype                                         */
+    int32_t gate_mode;      /* mtla_gate_mode                                     */
+    float softmax_scale;    /* 0 => 1/sqrt(d_h + d_r)                             */
+    float rope_base;        /* 0 => 10000                                         */
+    int32_t max_slots;      /* slots per sequence in the cache buffer             */
+} mtla_config;
+
+/* Bytes of scratch that mtla_decode_step (any positions) and mtla_prefill
+ * (any T <= max_tokens) need with this config. `bytes` receives the size.
+ * Returns INVALID_ARG / UNSUPPORTED for a bad config. Host only. */
+mtla_status mtla_workspace_size(const mtla_config* cfg, int32_t max_tokens, size_t* bytes);
+
+/* One incremental decode step: one new token for every sequence
+ * (MTLA Method (1): only every s-th step opens a new slot, the steps in
+ * between update the slot being filled in place).
+ *
+ * For each sequence b with t = pos[b]:
+ *   w_t per gate_mode; x = [c_new[b] ; RoPE_t(kr_new[b])];
+ *   open_slot[b] = (t mod s == 0 ? 0 : open_slot[b]) + w_t x     (fp32)
+ *   cache[b, floor(t/s)] = round(open_slot[b])
+ *   for every head h: q~ = [W_UK[h]^T q_c[b,h] ; RoPE_t(q_r[b,h])];
+ *     out[b,h] = W_UV[h] softmax_j(scale <q~, cache[b,j]>) cache[b,j][0:d_c]
+ *     over j = 0 .. floor(t/s).
+ *
+ *   c_new   [B, d_c]        dtype        kr_new [B, d_r] dtype (before RoPE)
+ *   q_c     [B, H, d_h]     dtype        q_r    [B, H, d_r] dtype (before RoPE)
+ *   w_uk    [H, d_h, d_c]   dtype        w_uv   [H, d_h, d_c] dtype
+ *   gate_w  [s, d_c] fp32, gate_b [s] fp32   (COMPUTED only; else may be NULL)
+ *   gate_in [B] fp32                          (SUPPLIED only; else may be NULL)
+ *   pos     [B] int32, device: index of this token = tokens already cached.
+ *           pos[b] >= max_slots * s skips sequence b and latches CAPACITY.
+ *   cache   [B, max_slots, d_c + d_r] dtype, in/out (slot floor(t/s) written)
+ *   open_slot [B, d_c + d_r] fp32, in/out (the slot being filled, unrounded)
+ *   out     [B, H, d_h]     dtype, out
+ *   workspace / workspace_bytes: scratch of at least mtla_workspace_size().
+ * Returns OK once the work is enqueued. */
+mtla_status mtla_decode_step(const mtla_config* cfg,
+                             const void* c_new, const void* kr_new,
+                             const void* q_c, const void* q_r,
+                             const void* w_uk, const void* w_uv,
+                             const float* gate_w, const float* gate_b, const float* gate_in,
+                             const int32_t* pos,
+                             void* cache, float* open_slot, void* out,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/* Parallel (training-form) forward over T tokens from position 0
+ * (MTLA Method (2)-(3): the stride-aware causal mask lets every position see
+ * the finished slots plus its own block's partial slot
+ *   P_t = sum_{u = s*floor(t/s)}^{t} w_u [c_u ; RoPE_u(k_u)],
+ * so the result equals T incremental decode steps).
+ *
+ *   c [B,T,d_c], kr [B,T,d_r], q_c [B,T,H,d_h], q_r [B,T,H,d_r]   dtype
+ *   w_uk, w_uv, gate_w, gate_b as for decode; gate_in [B,T] fp32 (SUPPLIED)
+ *   out       [B,T,H,d_h] dtype, out
+ *   cache_out [B, max_slots, d_c+d_r] dtype, out: slots 0..ceil(T/s)-1 (the
+ *             cache a following mtla_decode_step at pos = T continues from);
+ *             requires max_slots >= ceil(T/s); must not be NULL.
+ *   open_slot_out [B, d_c+d_r] fp32, out, may be NULL: P_{T-1}.
+ * T >= 1. Returns OK once the work is enqueued. */
+mtla_status mtla_prefill(const mtla_config* cfg, int32_t T,
+                         const void* c, const void* kr,
+                         const void* q_c, const void* q_r,
+                         const void* w_uk, const void* w_uv,
+                         const float* gate_w, const float* gate_b, const float* gate_in,
+                         void* out, void* cache_out, float* open_slot_out,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream`, then returns and clears the status latched by
+ * device-side checks on the current device since the last call (OK if none). */
+mtla_status mtla_get_device_status(void* stream);
+
+/* Static English text for a status code. */
+const char* mtla_status_string(mtla_status status);
+
+/* Number of kernels this library has launched in this process (all devices). */
+uint64_t mtla_kernel_launches(void);
+
+/* Timing hook for measurement tools (not thread-safe). After this call, the
+ * i-th following mtla_decode_step / mtla_prefill call (i = 0, 1, ...) records
+ * events[2i] on its stream just before its main attention kernel and
+ * events[2i+1] just after it, while i < n_pairs; later calls record nothing.
+ * `events` holds cudaEvent_t handles created and owned by the caller and must
+ * stay valid while the hook is set. mtla_set_profile_events(NULL, 0) turns
+ * the hook off. mtla_profile_events_recorded() returns how many pairs were
+ * recorded since the hook was set. */
+void mtla_set_profile_events(void* const* events, int32_t n_pairs);
+int32_t mtla_profile_events_recorded(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MTLA_H_ */

@@ -1,0 +1,239 @@
+// mtla_api.cu -- the C ABI of libmtla.so: argument checks, scratch layout,
+// device status word and dispatch to the kernels. See include/mtla.h.
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/mtla.h"
+#include "mtla_internal.h"
+
+namespace mtla {
+
+// Device status word, one per device that loads the library: the first error
+// a kernel finds (a position beyond the cache, a bounded wait that ran out).
+__device__ int g_device_status;
+
+static std::atomic<uint64_t> g_launches{0};
+
+static void* const* g_prof_events = nullptr;
+static int32_t g_prof_pairs = 0;
+static int32_t g_prof_next = 0;
+static bool g_prof_open = false;
+
+void profile_begin(cudaStream_t st) {
+    g_prof_open = false;
+    if (g_prof_events && g_prof_next < g_prof_pairs) {
+        cudaEventRecord((cudaEvent_t)g_prof_events[2 * g_prof_next], st);
+        g_prof_open = true;
+    }
+}
+
+void profile_end(cudaStream_t st) {
+    if (g_prof_open) {
+        cudaEventRecord((cudaEvent_t)g_prof_events[2 * g_prof_next + 1], st);
+        ++g_prof_next;
+        g_prof_open = false;
+    }
+}
+
+// Address of g_device_status on the current device (looked up once per device).
+static cudaError_t status_ptr(int** out) {
+    static int* cached[64] = {nullptr};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!cached[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_device_status);
+        if (e != cudaSuccess) return e;
+        cached[dev] = (int*)p;
+    }
+    *out = cached[dev];
+    return cudaSuccess;
+}
+
+static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+// Validate a config; fill the resolved shape.
+static mtla_status check_config(const mtla_config* cfg, Shape* sh) {
+    if (!cfg) return MTLA_ERR_INVALID_ARG;
+    if (cfg->batch <= 0 || cfg->heads <= 0 || cfg->d_h <= 0 || cfg->d_c <= 0 || cfg->d_r <= 0 ||
+        cfg->stride <= 0 || cfg->max_slots <= 0)
+        return MTLA_ERR_INVALID_ARG;
+    if (cfg->dtype != MTLA_BF16 && cfg->dtype != MTLA_FP32) return MTLA_ERR_INVALID_ARG;
+    if (cfg->gate_mode < MTLA_GATE_COMPUTED || cfg->gate_mode > MTLA_GATE_UNIT)
+        return MTLA_ERR_INVALID_ARG;
+    if (!(cfg->softmax_scale >= 0.f) || !std::isfinite(cfg->softmax_scale)) return MTLA_ERR_INVALID_ARG;
+    if (!(cfg->rope_base >= 0.f) || !std::isfinite(cfg->rope_base) ||
+        (cfg->rope_base != 0.f && cfg->rope_base <= 1.f))
+        return MTLA_ERR_INVALID_ARG;
+    if (cfg->d_h % 16 || cfg->d_c % 16 || cfg->d_r % 16) return MTLA_ERR_UNSUPPORTED;
+    if (cfg->d_c + cfg->d_r > 576 || cfg->d_c > 512 || cfg->heads > 128 || cfg->d_h > 256 ||
+        cfg->stride > 8)
+        return MTLA_ERR_UNSUPPORTED;
+    if ((int64_t)cfg->max_slots * cfg->stride > INT32_MAX) return MTLA_ERR_UNSUPPORTED;
+    sh->B = cfg->batch;
+    sh->H = cfg->heads;
+    sh->d_h = cfg->d_h;
+    sh->d_c = cfg->d_c;
+    sh->d_r = cfg->d_r;
+    sh->s = cfg->stride;
+    sh->D = cfg->d_c + cfg->d_r;
+    sh->gate_mode = cfg->gate_mode;
+    sh->max_slots = cfg->max_slots;
+    sh->scale = cfg->softmax_scale != 0.f ? cfg->softmax_scale
+                                          : (float)(1.0 / std::sqrt((double)(cfg->d_h + cfg->d_r)));
+    sh->log2_rope_base = std::log2(cfg->rope_base != 0.f ? (double)cfg->rope_base : 10000.0);
+    sh->log2_pe_base = std::log2(10000.0);
+    return MTLA_OK;
+}
+
+static size_t decode_ws(const Shape& sh) { return simt_decode_workspace(sh); }
+static size_t prefill_ws(const Shape& sh, int T) { return simt_prefill_workspace(sh, T); }
+
+static mtla_status check_gate_ptrs(const mtla_config* cfg, const float* gate_w, const float* gate_b,
+                                   const float* gate_in) {
+    if (cfg->gate_mode == MTLA_GATE_COMPUTED) {
+        if (!gate_w || !gate_b || !aligned16(gate_w) || !aligned16(gate_b)) return MTLA_ERR_INVALID_ARG;
+    }
+    if (cfg->gate_mode == MTLA_GATE_SUPPLIED) {
+        if (!gate_in || !aligned16(gate_in)) return MTLA_ERR_INVALID_ARG;
+    }
+    return MTLA_OK;
+}
+
+}  // namespace mtla
+
+using namespace mtla;
+
+extern "C" {
+
+mtla_status mtla_workspace_size(const mtla_config* cfg, int32_t max_tokens, size_t* bytes) {
+    Shape sh;
+    if (!bytes || max_tokens < 0) return MTLA_ERR_INVALID_ARG;
+    mtla_status st = check_config(cfg, &sh);
+    if (st != MTLA_OK) return st;
+    size_t d = decode_ws(sh);
+    size_t p = max_tokens > 0 ? prefill_ws(sh, max_tokens) : 0;
+    *bytes = d > p ? d : p;
+    return MTLA_OK;
+}
+
+mtla_status mtla_decode_step(const mtla_config* cfg, const void* c_new, const void* kr_new,
+                             const void* q_c, const void* q_r, const void* w_uk, const void* w_uv,
+                             const float* gate_w, const float* gate_b, const float* gate_in,
+                             const int32_t* pos, void* cache, float* open_slot, void* out,
+                             void* workspace, size_t workspace_bytes, void* stream) {
+    Shape sh;
+    mtla_status st = check_config(cfg, &sh);
+    if (st != MTLA_OK) return st;
+    const void* req[] = {c_new, kr_new, q_c, q_r, w_uk, w_uv, pos, cache, open_slot, out, workspace};
+    for (const void* p : req)
+        if (!p || !aligned16(p)) return MTLA_ERR_INVALID_ARG;
+    st = check_gate_ptrs(cfg, gate_w, gate_b, gate_in);
+    if (st != MTLA_OK) return st;
+    if (workspace_bytes < decode_ws(sh)) return MTLA_ERR_WORKSPACE;
+    DecodeArgs a;
+    a.sh = sh;
+    a.c_new = c_new;
+    a.kr_new = kr_new;
+    a.q_c = q_c;
+    a.q_r = q_r;
+    a.w_uk = w_uk;
+    a.w_uv = w_uv;
+    a.gate_w = gate_w;
+    a.gate_b = gate_b;
+    a.gate_in = gate_in;
+    a.pos = pos;
+    a.cache = cache;
+    a.open_slot = open_slot;
+    a.out = out;
+    a.workspace = workspace;
+    a.workspace_bytes = workspace_bytes;
+    if (status_ptr(&a.status) != cudaSuccess) return MTLA_ERR_CUDA;
+    uint64_t n = 0;
+    cudaError_t e = simt_decode(a, cfg->dtype == MTLA_FP32, (cudaStream_t)stream, &n);
+    g_launches += n;
+    return e == cudaSuccess ? MTLA_OK : MTLA_ERR_CUDA;
+}
+
+mtla_status mtla_prefill(const mtla_config* cfg, int32_t T, const void* c, const void* kr,
+                         const void* q_c, const void* q_r, const void* w_uk, const void* w_uv,
+                         const float* gate_w, const float* gate_b, const float* gate_in, void* out,
+                         void* cache_out, float* open_slot_out, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+    Shape sh;
+    mtla_status st = check_config(cfg, &sh);
+    if (st != MTLA_OK) return st;
+    if (T <= 0) return MTLA_ERR_INVALID_ARG;
+    const void* req[] = {c, kr, q_c, q_r, w_uk, w_uv, out, cache_out, workspace};
+    for (const void* p : req)
+        if (!p || !aligned16(p)) return MTLA_ERR_INVALID_ARG;
+    if (open_slot_out && !aligned16(open_slot_out)) return MTLA_ERR_INVALID_ARG;
+    st = check_gate_ptrs(cfg, gate_w, gate_b, gate_in);
+    if (st != MTLA_OK) return st;
+    if ((int64_t)(T + sh.s - 1) / sh.s > sh.max_slots) return MTLA_ERR_CAPACITY;
+    if (workspace_bytes < prefill_ws(sh, T)) return MTLA_ERR_WORKSPACE;
+    PrefillArgs a;
+    a.sh = sh;
+    a.T = T;
+    a.c = c;
+    a.kr = kr;
+    a.q_c = q_c;
+    a.q_r = q_r;
+    a.w_uk = w_uk;
+    a.w_uv = w_uv;
+    a.gate_w = gate_w;
+    a.gate_b = gate_b;
+    a.gate_in = gate_in;
+    a.out = out;
+    a.cache_out = cache_out;
+    a.open_slot_out = open_slot_out;
+    a.workspace = workspace;
+    a.workspace_bytes = workspace_bytes;
+    if (status_ptr(&a.status) != cudaSuccess) return MTLA_ERR_CUDA;
+    uint64_t n = 0;
+    cudaError_t e = simt_prefill(a, cfg->dtype == MTLA_FP32, (cudaStream_t)stream, &n);
+    g_launches += n;
+    return e == cudaSuccess ? MTLA_OK : MTLA_ERR_CUDA;
+}
+
+mtla_status mtla_get_device_status(void* stream) {
+    int* p = nullptr;
+    if (status_ptr(&p) != cudaSuccess) return MTLA_ERR_CUDA;
+    cudaStream_t s = (cudaStream_t)stream;
+    int v = 0;
+    if (cudaMemcpyAsync(&v, p, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return MTLA_ERR_CUDA;
+    if (cudaMemsetAsync(p, 0, sizeof(int), s) != cudaSuccess) return MTLA_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return MTLA_ERR_CUDA;
+    return (mtla_status)v;
+}
+
+const char* mtla_status_string(mtla_status s) {
+    switch (s) {
+        case MTLA_OK: return "ok";
+        case MTLA_ERR_INVALID_ARG: return "invalid argument";
+        case MTLA_ERR_UNSUPPORTED: return "unsupported shape or option";
+        case MTLA_ERR_CAPACITY: return "position beyond the cache capacity";
+        case MTLA_ERR_CUDA: return "CUDA runtime error";
+        case MTLA_ERR_TIMEOUT: return "device wait timed out";
+        case MTLA_ERR_WORKSPACE: return "workspace too small";
+    }
+    return "unknown status";
+}
+
+uint64_t mtla_kernel_launches(void) { return g_launches.load(); }
+
+void mtla_set_profile_events(void* const* events, int32_t n_pairs) {
+    g_prof_events = (events && n_pairs > 0) ? events : nullptr;
+    g_prof_pairs = g_prof_events ? n_pairs : 0;
+    g_prof_next = 0;
+    g_prof_open = false;
+}
+
+int32_t mtla_profile_events_recorded(void) { return g_prof_next; }
+
+}  // extern "C"

@@ -1,0 +1,73 @@
+// mtla_internal.h -- argument blocks passed from the C ABI to the kernels.
+#pragma once
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace mtla {
+
+struct Shape {
+    int B, H, d_h, d_c, d_r, s, D;
+    int gate_mode;          // 0 computed, 1 supplied, 2 unit
+    int max_slots;
+    float scale;            // softmax scale (resolved)
+    double log2_rope_base;  // log2 of the RoPE base
+    double log2_pe_base;    // log2 of the PE base (10000)
+};
+
+struct DecodeArgs {
+    Shape sh;
+    const void* c_new;
+    const void* kr_new;
+    const void* q_c;
+    const void* q_r;
+    const void* w_uk;
+    const void* w_uv;
+    const float* gate_w;
+    const float* gate_b;
+    const float* gate_in;
+    const int32_t* pos;
+    void* cache;
+    float* open_slot;
+    void* out;
+    void* workspace;
+    size_t workspace_bytes;
+    int* status;            // device status word
+};
+
+struct PrefillArgs {
+    Shape sh;
+    int T;
+    const void* c;
+    const void* kr;
+    const void* q_c;
+    const void* q_r;
+    const void* w_uk;
+    const void* w_uv;
+    const float* gate_w;
+    const float* gate_b;
+    const float* gate_in;
+    void* out;
+    void* cache_out;
+    float* open_slot_out;
+    void* workspace;
+    size_t workspace_bytes;
+    int* status;
+};
+
+// Scratch layouts (bytes), each region 256-byte aligned.
+size_t simt_decode_workspace(const Shape& sh);
+size_t simt_prefill_workspace(const Shape& sh, int T);
+
+// Launchers return cudaSuccess or the launch error; they add the number of
+// kernels they launched to *launches.
+cudaError_t simt_decode(const DecodeArgs& a, bool fp32, cudaStream_t st, uint64_t* launches);
+cudaError_t simt_prefill(const PrefillArgs& a, bool fp32, cudaStream_t st, uint64_t* launches);
+
+// Profile hook: record the next event pair around the main attention kernel.
+void profile_begin(cudaStream_t st);
+void profile_end(cudaStream_t st);
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+}  // namespace mtla

@@ -1,0 +1,422 @@
+// simt_kernels.cu -- CUDA-core kernels of the MTLA decode step and prefill.
+//
+// These are the fp32 path (every product and sum in true fp32 FMA; tensor
+// cores would round operands to tf32) and the reference shape of the work the
+// tensor-core kernels do for bf16. Steps, in the order of "Multi-head Temporal
+// Latent Attention", Method:
+//   gate w_t (Sec. 4.1, Eq. 13) -> RoPE of the decoupled key (Sec. 4.3) ->
+//   merge into the slot being filled (in place at decode; block-prefix scan at
+//   prefill, Sec. 4.2) -> absorbed query [W_UK^T qC ; RoPE(qR)] -> softmax over
+//   the finished slots plus the own partial slot -> W_UV on the weighted latent.
+#include "common.cuh"
+#include "mtla_internal.h"
+
+namespace mtla {
+
+namespace {
+
+constexpr int kMaxD = 576;              // d_c + d_r
+constexpr int kMaxPerLane = kMaxD / 32; // 18
+constexpr int kMaxLatPerLane = 512 / 32;
+
+// ----------------------------------------------------------------- gate
+
+// Merging weight of token t of sequence b; every thread of the block returns it.
+template <typename T>
+__device__ float gate_weight(const Shape& sh, int64_t t, const T* c_t, const float* gate_w,
+                             const float* gate_b, const float* w_given, float* red) {
+    if (sh.gate_mode == 2) return 1.f;
+    if (sh.gate_mode == 1) return *w_given;
+    const int r = (int)(t % sh.s);
+    const float* G = gate_w + (size_t)r * sh.d_c;
+    float z = 0.f;
+    for (int k = threadIdx.x; k < sh.d_c / 2; k += blockDim.x) {
+        float sn, cs;
+        pair_sincos(t, k, sh.d_c, sh.log2_pe_base, &sn, &cs);
+        z = fmaf(G[2 * k] * to_f<T>(c_t[2 * k]), sn, z);
+        z = fmaf(G[2 * k + 1] * to_f<T>(c_t[2 * k + 1]), cs, z);
+    }
+    z = block_sum(z, red) + gate_b[r];
+    return sigmoidf_(z);
+}
+
+// ----------------------------------------------------------------- decode
+
+template <typename T>
+__global__ void __launch_bounds__(128) k_decode_update(DecodeArgs a) {
+    const Shape sh = a.sh;
+    const int b = blockIdx.x;
+    const int64_t t = a.pos[b];
+    if (t < 0 || t >= (int64_t)sh.max_slots * sh.s) {
+        if (threadIdx.x == 0) latch_status(a.status, kStatusCapacity);
+        return;
+    }
+    __shared__ float red[32];
+    const T* c = (const T*)a.c_new + (size_t)b * sh.d_c;
+    const T* kr = (const T*)a.kr_new + (size_t)b * sh.d_r;
+    const float w = gate_weight<T>(sh, t, c, a.gate_w, a.gate_b, a.gate_in ? a.gate_in + b : nullptr, red);
+    float* acc = a.open_slot + (size_t)b * sh.D;
+    T* row = (T*)a.cache + ((size_t)b * sh.max_slots + (size_t)(t / sh.s)) * sh.D;
+    const bool fresh = (t % sh.s) == 0;
+    for (int k = threadIdx.x; k < sh.d_c; k += blockDim.x) {
+        const float v = (fresh ? 0.f : acc[k]) + w * to_f<T>(c[k]);
+        acc[k] = v;
+        row[k] = from_f<T>(v);
+    }
+    for (int k = threadIdx.x; k < sh.d_r / 2; k += blockDim.x) {
+        float sn, cs;
+        pair_sincos(t, k, sh.d_r, sh.log2_rope_base, &sn, &cs);
+        const float x0 = to_f<T>(kr[2 * k]), x1 = to_f<T>(kr[2 * k + 1]);
+        const float y0 = x0 * cs - x1 * sn, y1 = x0 * sn + x1 * cs;
+        float* ar = acc + sh.d_c;
+        const float v0 = (fresh ? 0.f : ar[2 * k]) + w * y0;
+        const float v1 = (fresh ? 0.f : ar[2 * k + 1]) + w * y1;
+        ar[2 * k] = v0;
+        ar[2 * k + 1] = v1;
+        row[sh.d_c + 2 * k] = from_f<T>(v0);
+        row[sh.d_c + 2 * k + 1] = from_f<T>(v1);
+    }
+}
+
+// Absorbed query for `rows` rows (decode: one per sequence; prefill: B*T).
+// grid (rows, H). Position of a row: pos[row] (decode) or row % T (prefill).
+template <typename T>
+__global__ void __launch_bounds__(128) k_absorb_query(Shape sh, const T* qc, const T* qr,
+                                                      const T* w_uk, const int32_t* pos, int T_len,
+                                                      float* qt) {
+    const int row = blockIdx.x, h = blockIdx.y;
+    int64_t t;
+    if (pos) {
+        t = pos[row];
+        if (t < 0 || t >= (int64_t)sh.max_slots * sh.s) return;
+    } else {
+        t = row % T_len;
+    }
+    __shared__ float q[256];
+    const size_t rh = (size_t)row * sh.H + h;
+    for (int i = threadIdx.x; i < sh.d_h; i += blockDim.x) q[i] = to_f<T>(qc[rh * sh.d_h + i]);
+    __syncthreads();
+    const T* W = w_uk + (size_t)h * sh.d_h * sh.d_c;
+    float* out = qt + rh * sh.D;
+    for (int j = threadIdx.x; j < sh.d_c; j += blockDim.x) {
+        float acc = 0.f;
+        for (int i = 0; i < sh.d_h; ++i) acc = fmaf(to_f<T>(W[(size_t)i * sh.d_c + j]), q[i], acc);
+        out[j] = acc;
+    }
+    const T* r = qr + rh * sh.d_r;
+    for (int k = threadIdx.x; k < sh.d_r / 2; k += blockDim.x) {
+        float sn, cs;
+        pair_sincos(t, k, sh.d_r, sh.log2_rope_base, &sn, &cs);
+        const float x0 = to_f<T>(r[2 * k]), x1 = to_f<T>(r[2 * k + 1]);
+        out[sh.d_c + 2 * k] = x0 * cs - x1 * sn;
+        out[sh.d_c + 2 * k + 1] = x0 * sn + x1 * cs;
+    }
+}
+
+// Online-softmax state of one (query, head) row held by a warp: lane l owns
+// latent entries l, l+32, ...
+struct RowState {
+    float m, l;
+    float o[kMaxLatPerLane];
+};
+
+template <typename K>
+__device__ __forceinline__ void row_visit(RowState& st, const float* q, const K* key, int D,
+                                          int d_c, float scale) {
+    const int lane = threadIdx.x & 31;
+    float x[kMaxPerLane];
+    float dot = 0.f;
+#pragma unroll
+    for (int i = 0; i < kMaxPerLane; ++i) {
+        const int idx = lane + 32 * i;
+        float v = 0.f;
+        if (idx < D) v = to_f<K>(key[idx]);
+        x[i] = v;
+        dot = fmaf(q[i], v, dot);
+    }
+    dot = warp_sum(dot) * scale;
+    const float m_new = fmaxf(st.m, dot);
+    const float corr = (st.m == -INFINITY) ? 0.f : expf(st.m - m_new);
+    const float p = expf(dot - m_new);
+    st.l = st.l * corr + p;
+#pragma unroll
+    for (int i = 0; i < kMaxLatPerLane; ++i) {
+        const int idx = lane + 32 * i;
+        if (idx < d_c) st.o[i] = st.o[i] * corr + p * x[i];
+    }
+    st.m = m_new;
+}
+
+// Split-K attention: block (split, b) covers slots [split*chunk, ...) of the
+// n = floor(t/s)+1 slots of sequence b for all heads; writes (o, m, l).
+template <typename T>
+__global__ void __launch_bounds__(256) k_decode_attn(DecodeArgs a, int chunk, int splits,
+                                                     const float* qt, float* part) {
+    const Shape sh = a.sh;
+    const int split = blockIdx.x, b = blockIdx.y;
+    const int64_t t = a.pos[b];
+    if (t < 0 || t >= (int64_t)sh.max_slots * sh.s) return;
+    const int64_t n = t / sh.s + 1;
+    const int64_t j0 = (int64_t)split * chunk;
+    const int64_t j1 = min(n, j0 + chunk);
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const T* cache = (const T*)a.cache + (size_t)b * sh.max_slots * sh.D;
+    for (int h = warp; h < sh.H; h += 8) {
+        float q[kMaxPerLane];
+        const float* qrow = qt + ((size_t)b * sh.H + h) * sh.D;
+#pragma unroll
+        for (int i = 0; i < kMaxPerLane; ++i) {
+            const int idx = lane + 32 * i;
+            q[i] = idx < sh.D ? qrow[idx] : 0.f;
+        }
+        RowState st;
+        st.m = -INFINITY;
+        st.l = 0.f;
+#pragma unroll
+        for (int i = 0; i < kMaxLatPerLane; ++i) st.o[i] = 0.f;
+        for (int64_t j = j0; j < j1; ++j)
+            row_visit<T>(st, q, cache + (size_t)j * sh.D, sh.D, sh.d_c, sh.scale);
+        float* dst = part + (((size_t)b * splits + split) * sh.H + h) * (sh.d_c + 2);
+#pragma unroll
+        for (int i = 0; i < kMaxLatPerLane; ++i) {
+            const int idx = lane + 32 * i;
+            if (idx < sh.d_c) dst[idx] = st.o[i];
+        }
+        if (lane == 0) {
+            dst[sh.d_c] = st.m;
+            dst[sh.d_c + 1] = st.l;
+        }
+    }
+}
+
+// Merge the splits of (b, h) and apply W_UV. grid (H, B).
+template <typename T>
+__global__ void __launch_bounds__(256) k_decode_combine(DecodeArgs a, int chunk, int splits,
+                                                        const float* part) {
+    const Shape sh = a.sh;
+    const int h = blockIdx.x, b = blockIdx.y;
+    const int64_t t = a.pos[b];
+    if (t < 0 || t >= (int64_t)sh.max_slots * sh.s) return;
+    const int64_t n = t / sh.s + 1;
+    const int used = (int)((n + chunk - 1) / chunk);
+    __shared__ float wts[64];
+    __shared__ float olat[512];
+    __shared__ float inv_l;
+    const float* base = part + ((size_t)b * splits * sh.H + h) * (sh.d_c + 2);
+    const size_t sstride = (size_t)sh.H * (sh.d_c + 2);
+    if (threadIdx.x == 0) {
+        float M = -INFINITY;
+        for (int k = 0; k < used; ++k) M = fmaxf(M, base[k * sstride + sh.d_c]);
+        float L = 0.f;
+        for (int k = 0; k < used; ++k) {
+            const float mk = base[k * sstride + sh.d_c];
+            const float wk = (mk == -INFINITY) ? 0.f : expf(mk - M);
+            wts[k] = wk;
+            L += wk * base[k * sstride + sh.d_c + 1];
+        }
+        inv_l = 1.f / L;
+    }
+    __syncthreads();
+    for (int j = threadIdx.x; j < sh.d_c; j += blockDim.x) {
+        float acc = 0.f;
+        for (int k = 0; k < used; ++k) acc = fmaf(wts[k], base[k * sstride + j], acc);
+        olat[j] = acc * inv_l;
+    }
+    __syncthreads();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const T* W = (const T*)a.w_uv + (size_t)h * sh.d_h * sh.d_c;
+    T* out = (T*)a.out + ((size_t)b * sh.H + h) * sh.d_h;
+    for (int i = warp; i < sh.d_h; i += 8) {
+        float acc = 0.f;
+        for (int j = lane; j < sh.d_c; j += 32) acc = fmaf(to_f<T>(W[(size_t)i * sh.d_c + j]), olat[j], acc);
+        acc = warp_sum(acc);
+        if (lane == 0) out[i] = from_f<T>(acc);
+    }
+}
+
+// ----------------------------------------------------------------- prefill
+
+// Block-prefix scan: block (j, b) computes the partial slots P_u of the
+// tokens u of slot j, the finished/last slot of the cache, and the open slot.
+template <typename T>
+__global__ void __launch_bounds__(128) k_prefill_scan(PrefillArgs a, float* P) {
+    const Shape sh = a.sh;
+    const int j = blockIdx.x, b = blockIdx.y;
+    const int Tn = a.T;
+    const int u0 = j * sh.s, u1 = min(u0 + sh.s, Tn);
+    __shared__ float red[32];
+    __shared__ float wsm[8];
+    const T* c = (const T*)a.c + (size_t)b * Tn * sh.d_c;
+    const T* kr = (const T*)a.kr + (size_t)b * Tn * sh.d_r;
+    for (int u = u0; u < u1; ++u) {
+        const float w = gate_weight<T>(sh, u, c + (size_t)u * sh.d_c, a.gate_w, a.gate_b,
+                                       a.gate_in ? a.gate_in + (size_t)b * Tn + u : nullptr, red);
+        if (threadIdx.x == 0) wsm[u - u0] = w;
+    }
+    __syncthreads();
+    T* slot = (T*)a.cache_out + ((size_t)b * sh.max_slots + j) * sh.D;
+    float* open = (u1 == Tn && a.open_slot_out) ? a.open_slot_out + (size_t)b * sh.D : nullptr;
+    for (int k = threadIdx.x; k < sh.d_c; k += blockDim.x) {
+        float acc = 0.f;
+        for (int u = u0; u < u1; ++u) {
+            acc += wsm[u - u0] * to_f<T>(c[(size_t)u * sh.d_c + k]);
+            P[((size_t)b * Tn + u) * sh.D + k] = acc;
+        }
+        slot[k] = from_f<T>(acc);
+        if (open) open[k] = acc;
+    }
+    for (int k = threadIdx.x; k < sh.d_r / 2; k += blockDim.x) {
+        float a0 = 0.f, a1 = 0.f;
+        for (int u = u0; u < u1; ++u) {
+            float sn, cs;
+            pair_sincos(u, k, sh.d_r, sh.log2_rope_base, &sn, &cs);
+            const float x0 = to_f<T>(kr[(size_t)u * sh.d_r + 2 * k]);
+            const float x1 = to_f<T>(kr[(size_t)u * sh.d_r + 2 * k + 1]);
+            a0 += wsm[u - u0] * (x0 * cs - x1 * sn);
+            a1 += wsm[u - u0] * (x0 * sn + x1 * cs);
+            float* pr = P + ((size_t)b * Tn + u) * sh.D + sh.d_c;
+            pr[2 * k] = a0;
+            pr[2 * k + 1] = a1;
+        }
+        slot[sh.d_c + 2 * k] = from_f<T>(a0);
+        slot[sh.d_c + 2 * k + 1] = from_f<T>(a1);
+        if (open) {
+            open[sh.d_c + 2 * k] = a0;
+            open[sh.d_c + 2 * k + 1] = a1;
+        }
+    }
+}
+
+// Masked attention: one warp per (t, h) row; keys are the finished slots
+// j < floor(t/s) (rounded cache) plus the own partial slot P_t (rounded).
+template <typename T>
+__global__ void __launch_bounds__(256) k_prefill_attn(PrefillArgs a, const float* P, const float* qt) {
+    const Shape sh = a.sh;
+    const int b = blockIdx.y;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t row = (int64_t)blockIdx.x * 8 + warp;
+    if (row >= (int64_t)a.T * sh.H) return;
+    const int t = (int)(row / sh.H), h = (int)(row % sh.H);
+    const float* qrow = qt + (((size_t)b * a.T + t) * sh.H + h) * sh.D;
+    float q[kMaxPerLane];
+#pragma unroll
+    for (int i = 0; i < kMaxPerLane; ++i) {
+        const int idx = lane + 32 * i;
+        q[i] = idx < sh.D ? qrow[idx] : 0.f;
+    }
+    RowState st;
+    st.m = -INFINITY;
+    st.l = 0.f;
+#pragma unroll
+    for (int i = 0; i < kMaxLatPerLane; ++i) st.o[i] = 0.f;
+    const T* cache = (const T*)a.cache_out + (size_t)b * sh.max_slots * sh.D;
+    const int nf = t / sh.s;
+    for (int j = 0; j < nf; ++j) row_visit<T>(st, q, cache + (size_t)j * sh.D, sh.D, sh.d_c, sh.scale);
+    {
+        // own partial slot, rounded to the storage type
+        const float* pp = P + ((size_t)b * a.T + t) * sh.D;
+        float x[kMaxPerLane];
+        float dot = 0.f;
+#pragma unroll
+        for (int i = 0; i < kMaxPerLane; ++i) {
+            const int idx = lane + 32 * i;
+            float v = 0.f;
+            if (idx < sh.D) v = round_to<T>(pp[idx]);
+            x[i] = v;
+            dot = fmaf(q[i], v, dot);
+        }
+        dot = warp_sum(dot) * sh.scale;
+        const float m_new = fmaxf(st.m, dot);
+        const float corr = (st.m == -INFINITY) ? 0.f : expf(st.m - m_new);
+        const float p = expf(dot - m_new);
+        st.l = st.l * corr + p;
+#pragma unroll
+        for (int i = 0; i < kMaxLatPerLane; ++i) {
+            const int idx = lane + 32 * i;
+            if (idx < sh.d_c) st.o[i] = st.o[i] * corr + p * x[i];
+        }
+        st.m = m_new;
+    }
+    const float inv_l = 1.f / st.l;
+    const T* W = (const T*)a.w_uv + (size_t)h * sh.d_h * sh.d_c;
+    T* out = (T*)a.out + (((size_t)b * a.T + t) * sh.H + h) * sh.d_h;
+    for (int i = 0; i < sh.d_h; ++i) {
+        float acc = 0.f;
+#pragma unroll
+        for (int k = 0; k < kMaxLatPerLane; ++k) {
+            const int idx = lane + 32 * k;
+            if (idx < sh.d_c) acc = fmaf(to_f<T>(W[(size_t)i * sh.d_c + idx]), st.o[k], acc);
+        }
+        acc = warp_sum(acc);
+        if (lane == 0) out[i] = from_f<T>(acc * inv_l);
+    }
+}
+
+void decode_plan(const Shape& sh, int* splits, int* chunk) {
+    int sp = (sh.max_slots + 63) / 64;
+    if (sp < 1) sp = 1;
+    if (sp > 32) sp = 32;
+    *splits = sp;
+    *chunk = (sh.max_slots + sp - 1) / sp;
+}
+
+template <typename T>
+cudaError_t decode_impl(const DecodeArgs& a, cudaStream_t st, uint64_t* launches) {
+    const Shape& sh = a.sh;
+    int splits, chunk;
+    decode_plan(sh, &splits, &chunk);
+    char* ws = (char*)a.workspace;
+    float* qt = (float*)ws;
+    float* part = (float*)(ws + align256((size_t)sh.B * sh.H * sh.D * sizeof(float)));
+    k_decode_update<T><<<sh.B, 128, 0, st>>>(a);
+    k_absorb_query<T><<<dim3(sh.B, sh.H), 128, 0, st>>>(sh, (const T*)a.q_c, (const T*)a.q_r,
+                                                         (const T*)a.w_uk, a.pos, 0, qt);
+    profile_begin(st);
+    k_decode_attn<T><<<dim3(splits, sh.B), 256, 0, st>>>(a, chunk, splits, qt, part);
+    profile_end(st);
+    k_decode_combine<T><<<dim3(sh.H, sh.B), 256, 0, st>>>(a, chunk, splits, part);
+    *launches += 4;
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t prefill_impl(const PrefillArgs& a, cudaStream_t st, uint64_t* launches) {
+    const Shape& sh = a.sh;
+    char* ws = (char*)a.workspace;
+    float* P = (float*)ws;
+    float* qt = (float*)(ws + align256((size_t)sh.B * a.T * sh.D * sizeof(float)));
+    const int n_slots = (a.T + sh.s - 1) / sh.s;
+    k_prefill_scan<T><<<dim3(n_slots, sh.B), 128, 0, st>>>(a, P);
+    k_absorb_query<T><<<dim3(sh.B * a.T, sh.H), 128, 0, st>>>(sh, (const T*)a.q_c, (const T*)a.q_r,
+                                                               (const T*)a.w_uk, nullptr, a.T, qt);
+    const int64_t rows = (int64_t)a.T * sh.H;
+    profile_begin(st);
+    k_prefill_attn<T><<<dim3((unsigned)((rows + 7) / 8), sh.B), 256, 0, st>>>(a, P, qt);
+    profile_end(st);
+    *launches += 3;
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t simt_decode_workspace(const Shape& sh) {
+    int splits, chunk;
+    decode_plan(sh, &splits, &chunk);
+    return align256((size_t)sh.B * sh.H * sh.D * sizeof(float)) +
+           align256((size_t)sh.B * splits * sh.H * (sh.d_c + 2) * sizeof(float));
+}
+
+size_t simt_prefill_workspace(const Shape& sh, int T) {
+    return align256((size_t)sh.B * T * sh.D * sizeof(float)) +
+           align256((size_t)sh.B * T * sh.H * sh.D * sizeof(float));
+}
+
+cudaError_t simt_decode(const DecodeArgs& a, bool fp32, cudaStream_t st, uint64_t* launches) {
+    return fp32 ? decode_impl<float>(a, st, launches) : decode_impl<bf16>(a, st, launches);
+}
+
+cudaError_t simt_prefill(const PrefillArgs& a, bool fp32, cudaStream_t st, uint64_t* launches) {
+    return fp32 ? prefill_impl<float>(a, st, launches) : prefill_impl<bf16>(a, st, launches);
+}
+
+}  // namespace mtla

@@ -1,0 +1,198 @@
+"""Python binding of libmtla.so (argument marshalling only).
+
+Every function here forwards torch tensors' device pointers to the C ABI in
+``include/mtla.h`` under the same name; all arithmetic runs in the library's
+CUDA kernels. If the shared library is missing this module raises at import
+of the first call -- there is no other implementation to fall back on.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmtla.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CAPACITY, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE = range(7)
+BF16, FP32 = 0, 1
+GATE_COMPUTED, GATE_SUPPLIED, GATE_UNIT = 0, 1, 2
+
+
+class MtlaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+class Config(ctypes.Structure):
+    """Mirror of ``mtla_config``."""
+    _fields_ = [
+        ("batch", ctypes.c_int32), ("heads", ctypes.c_int32), ("d_h", ctypes.c_int32),
+        ("d_c", ctypes.c_int32), ("d_r", ctypes.c_int32), ("stride", ctypes.c_int32),
+        ("dtype", ctypes.c_int32), ("gate_mode", ctypes.c_int32),
+        ("softmax_scale", ctypes.c_float), ("rope_base", ctypes.c_float),
+        ("max_slots", ctypes.c_int32),
+    ]
+
+    @property
+    def D(self) -> int:
+        return self.d_c + self.d_r
+
+    @property
+    def torch_dtype(self):
+        return torch.float32 if self.dtype == FP32 else torch.bfloat16
+
+
+def make_config(B, H, d_h, d_c, d_r, s, max_slots, dtype="bf16", gate_mode=GATE_COMPUTED,
+                softmax_scale=0.0, rope_base=10000.0) -> Config:
+    dt = FP32 if dtype in ("fp32", FP32, torch.float32) else BF16
+    return Config(B, H, d_h, d_c, d_r, s, dt, gate_mode, softmax_scale, rope_base, max_slots)
+
+
+_lib = None
+_vp = ctypes.c_void_p
+
+
+def load() -> ctypes.CDLL:
+    """Load libmtla.so (built by ``python -m kv_cache_mtla_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m kv_cache_mtla_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    cp = ctypes.POINTER(Config)
+    lib.mtla_workspace_size.argtypes = [cp, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)]
+    lib.mtla_workspace_size.restype = ctypes.c_int
+    lib.mtla_decode_step.argtypes = [cp] + [_vp] * 13 + [_vp, ctypes.c_size_t, _vp]
+    lib.mtla_decode_step.restype = ctypes.c_int
+    lib.mtla_prefill.argtypes = [cp, ctypes.c_int32] + [_vp] * 12 + [_vp, ctypes.c_size_t, _vp]
+    lib.mtla_prefill.restype = ctypes.c_int
+    lib.mtla_get_device_status.argtypes = [_vp]
+    lib.mtla_get_device_status.restype = ctypes.c_int
+    lib.mtla_status_string.argtypes = [ctypes.c_int]
+    lib.mtla_status_string.restype = ctypes.c_char_p
+    lib.mtla_kernel_launches.argtypes = []
+    lib.mtla_kernel_launches.restype = ctypes.c_uint64
+    lib.mtla_set_profile_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32]
+    lib.mtla_set_profile_events.restype = None
+    lib.mtla_profile_events_recorded.argtypes = []
+    lib.mtla_profile_events_recorded.restype = ctypes.c_int32
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load().mtla_status_string(int(status)).decode()
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libmtla must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def workspace_size(cfg: Config, max_tokens: int = 0) -> int:
+    n = ctypes.c_size_t(0)
+    st = load().mtla_workspace_size(ctypes.byref(cfg), int(max_tokens), ctypes.byref(n))
+    if st != OK:
+        raise MtlaError(st, "mtla_workspace_size")
+    return int(n.value)
+
+
+def decode_step(cfg, c_new, kr_new, q_c, q_r, w_uk, w_uv, gate_w, gate_b, gate_in, pos, cache,
+                open_slot, out, workspace, stream=None, check=True) -> int:
+    """Forward to ``mtla_decode_step``; returns the status (raises if check)."""
+    ws = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = load().mtla_decode_step(
+        ctypes.byref(cfg), _ptr(c_new), _ptr(kr_new), _ptr(q_c), _ptr(q_r), _ptr(w_uk),
+        _ptr(w_uv), _ptr(gate_w), _ptr(gate_b), _ptr(gate_in), _ptr(pos), _ptr(cache),
+        _ptr(open_slot), _ptr(out), _ptr(workspace), ws, _stream(stream))
+    if check and st != OK:
+        raise MtlaError(st, "mtla_decode_step")
+    return st
+
+
+def prefill(cfg, T, c, kr, q_c, q_r, w_uk, w_uv, gate_w, gate_b, gate_in, out, cache_out,
+            open_slot_out, workspace, stream=None, check=True) -> int:
+    """Forward to ``mtla_prefill``; returns the status (raises if check)."""
+    ws = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = load().mtla_prefill(
+        ctypes.byref(cfg), int(T), _ptr(c), _ptr(kr), _ptr(q_c), _ptr(q_r), _ptr(w_uk),
+        _ptr(w_uv), _ptr(gate_w), _ptr(gate_b), _ptr(gate_in), _ptr(out), _ptr(cache_out),
+        _ptr(open_slot_out), _ptr(workspace), ws, _stream(stream))
+    if check and st != OK:
+        raise MtlaError(st, "mtla_prefill")
+    return st
+
+
+def get_device_status(stream=None) -> int:
+    return int(load().mtla_get_device_status(_stream(stream)))
+
+
+def kernel_launches() -> int:
+    return int(load().mtla_kernel_launches())
+
+
+class ProfileEvents:
+    """Event pairs the library records around its main attention kernel
+    (``mtla_set_profile_events``); ``durations_ms()`` after a synchronize."""
+
+    def __init__(self, n_pairs: int):
+        self.events = [torch.cuda.Event(enable_timing=True) for _ in range(2 * n_pairs)]
+        self._arr = (ctypes.c_void_p * (2 * n_pairs))(*[e.cuda_event for e in self.events])
+        self.n = n_pairs
+
+    def __enter__(self):
+        load().mtla_set_profile_events(self._arr, self.n)
+        return self
+
+    def __exit__(self, *exc):
+        self.recorded = int(load().mtla_profile_events_recorded())
+        load().mtla_set_profile_events(None, 0)
+
+    def durations_ms(self):
+        return [self.events[2 * i].elapsed_time(self.events[2 * i + 1]) for i in range(self.recorded)]
+
+
+@dataclass
+class Buffers:
+    """Device buffers of one MTLA problem (weights, cache, open slot, scratch)."""
+    cfg: Config
+    w_uk: torch.Tensor
+    w_uv: torch.Tensor
+    gate_w: torch.Tensor
+    gate_b: torch.Tensor
+    cache: torch.Tensor
+    open_slot: torch.Tensor
+    workspace: torch.Tensor
+
+    @staticmethod
+    def allocate(cfg: Config, weights: dict, max_tokens: int = 0, device="cuda") -> "Buffers":
+        dt = cfg.torch_dtype
+        ws = workspace_size(cfg, max_tokens)
+        return Buffers(
+            cfg=cfg,
+            w_uk=weights["w_uk"].to(device=device, dtype=dt).contiguous(),
+            w_uv=weights["w_uv"].to(device=device, dtype=dt).contiguous(),
+            gate_w=weights["gate_w"].to(device=device, dtype=torch.float32).contiguous(),
+            gate_b=weights["gate_b"].to(device=device, dtype=torch.float32).contiguous(),
+            cache=torch.zeros(cfg.batch, cfg.max_slots, cfg.D, device=device, dtype=dt),
+            open_slot=torch.zeros(cfg.batch, cfg.D, device=device, dtype=torch.float32),
+            workspace=torch.empty(max(ws, 256), device=device, dtype=torch.uint8),
+        )

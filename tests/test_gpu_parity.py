@@ -1,0 +1,240 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 oracle on
+the same seeded inputs. Tolerances: max|gpu - ref| / max|ref| <= 2e-2 for bf16
+storage with fp32 accumulation, <= 1e-5 for the fp32 path; slot contents and
+the attended slot set exactly where the arithmetic is exact."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_harness import TOL, Problem, concat_tokens, np64, oracle_cfg, oracle_rows, rel_err
+from kv_cache_mtla_b200 import inputs, mtla
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _clean_status():
+    torch.cuda.synchronize()
+    mtla.get_device_status()
+    yield
+    assert mtla.get_device_status() == mtla.OK
+
+
+def _slots_from_P(P, T, s):
+    n = (T + s - 1) // s
+    idx = [min(j * s + s - 1, T - 1) for j in range(n)]
+    return P[:, idx]
+
+
+# ----------------------------------------------------------------- tiny fp32 (1e-5)
+
+@pytest.mark.parametrize("s", [1, 2, 3, 4])
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_tiny_prefill_and_decode(s, dtype):
+    """Prefill of T tokens and T decode steps from an empty cache both match the
+    oracle; decode equals prefill (the stride-aware mask reproduces incremental
+    decoding); the cache and the open slot match. T = 61 leaves a ragged tail."""
+    wl = inputs.TINY_FP32.with_(s=s, dtype=dtype)
+    T = 61 if s > 1 else 64
+    w = inputs.weights(wl)
+    toks = inputs.tokens(wl, T)
+    ref = oracle.prefill(oracle_cfg(wl), toks["c"], toks["kr"], toks["qc"], toks["qr"],
+                         w["w_uk"], w["w_uv"], w["gate_w"], w["gate_b"], toks["gate_in"])
+    n_slots = (T + s - 1) // s
+    tol = TOL[dtype]
+
+    pre = Problem(wl, max_slots=n_slots + 1, max_tokens=T, weights=w)
+    out_p = np64(pre.prefill(toks, T))
+    assert rel_err(out_p, ref["out"]) <= tol
+    assert rel_err(np64(pre.buf.cache[:, :n_slots]), ref["cache"]) <= (tol if dtype == "fp32" else 4e-3)
+    assert rel_err(np64(pre.buf.open_slot), ref["acc"]) <= 1e-5
+
+    dec = Problem(wl, max_slots=n_slots + 1, weights=w)
+    outs = []
+    for t in range(T):
+        outs.append(np64(dec.decode(toks, t, [t] * wl.B)))
+    out_d = np.stack(outs, axis=1)
+    assert rel_err(out_d, ref["out"]) <= tol
+    assert rel_err(out_d, out_p) <= tol
+    assert rel_err(np64(dec.buf.cache[:, :n_slots]), ref["cache"]) <= (tol if dtype == "fp32" else 4e-3)
+    assert rel_err(np64(dec.buf.open_slot), ref["acc"]) <= 1e-5
+
+
+@pytest.mark.parametrize("s", [1, 2, 3, 4])
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_mask_set_bit_exact(s, dtype):
+    """One-hot probe: zero queries and unit gates, W_UV = [I | 0]. Output entry j
+    of query t is nonzero exactly when slot j is attended, so the attended set
+    must equal {0..floor(t/s)} bit for bit, with weight 1/(floor(t/s)+1)."""
+    wl = inputs.TINY_FP32.with_(s=s, dtype=dtype, gate_mode=inputs.GATE_UNIT)
+    T = min(wl.s * wl.d_h, 61)
+    toks = inputs.one_hot_mask_probe(wl, T)
+    w = inputs.weights(wl)
+    eye = torch.zeros(wl.H, wl.d_h, wl.d_c)
+    eye[:, torch.arange(wl.d_h), torch.arange(wl.d_h)] = 1.0
+    w = dict(w, w_uv=eye, w_uk=torch.zeros_like(eye))
+    n_slots = (T + s - 1) // s
+    for mode in ("prefill", "decode"):
+        pb = Problem(wl, max_slots=n_slots, max_tokens=T, weights=w)
+        if mode == "prefill":
+            out = np64(pb.prefill(toks, T))[0]
+        else:
+            out = np.stack([np64(pb.decode(toks, t, [t]))[0] for t in range(T)])
+        for t in range(T):
+            for h in range(wl.H):
+                support = np.nonzero(out[t, h])[0].tolist()
+                assert support == list(range(t // s + 1)), (mode, t, h)
+                np.testing.assert_allclose(out[t, h, : t // s + 1], 1.0 / (t // s + 1),
+                                           rtol=TOL[dtype] if dtype == "fp32" else 4e-3)
+
+
+# ----------------------------------------------------------------- speech decode
+
+def test_speech_decode_prefix_then_steps():
+    """B=16, H=8, d_h=64, d_c=256, d_R=32, s=2: prefill a 1024-token prefix,
+    then 256 decode steps; sampled prefill rows and decode steps against the
+    oracle's parallel form over the whole 1280-token stream."""
+    wl = inputs.SPEECH_DECODE
+    T, S = wl.T, wl.steps
+    w = inputs.weights(wl)
+    pre_t = inputs.tokens(wl, T, stream=0)
+    dec_t = inputs.tokens(wl, S, stream=1)
+    max_slots = (T + S + wl.s - 1) // wl.s
+    pb = Problem(wl, max_slots=max_slots, max_tokens=T, weights=w)
+    out_p = np64(pb.prefill(pre_t, T))
+    outs = {}
+    keep = {0, 1, 2, 3, 100, 127, 254, 255}
+    for k in range(S):
+        o = pb.decode(dec_t, k, [T + k] * wl.B)
+        if k in keep:
+            outs[k] = np64(o)
+    allt = concat_tokens(pre_t, dec_t)
+    rows_p = [(b, t) for b in (0, 7, 15) for t in (0, 1, 2, 511, 512, 1022, 1023)]
+    rows_d = [(b, T + k) for b in range(wl.B) for k in sorted(keep)]
+    ref, P = oracle_rows(wl, w, allt, rows_p + rows_d)
+    ref_p = ref[: len(rows_p)]
+    got_p = np.stack([out_p[b, t] for b, t in rows_p])
+    assert rel_err(got_p, ref_p) <= TOL["bf16"]
+    ref_d = ref[len(rows_p):]
+    got_d = np.stack([outs[t - T][b] for b, t in rows_d])
+    assert rel_err(got_d, ref_d) <= TOL["bf16"]
+    slots = _slots_from_P(P, T + S, wl.s)
+    assert rel_err(np64(pb.buf.cache), slots) <= 4e-3
+    assert rel_err(np64(pb.buf.open_slot), P[:, T + S - 1]) <= 1e-5
+
+
+# ----------------------------------------------------------------- stride sweep
+
+@pytest.mark.parametrize("s", [1, 2, 3, 4])
+def test_stride_sweep_decode(s):
+    """B=64, N=4096 tokens after the step (s=3 leaves a one-token last slot):
+    synthetic cache of N-1 tokens, one decode step at pos = N-1, compared with
+    the oracle's incremental step on sampled sequences; plus mixed positions."""
+    wl = inputs.STRIDE_SWEEP.with_(s=s)
+    N = wl.T
+    max_slots = (N + s - 1) // s
+    w = inputs.weights(wl)
+    toks = inputs.tokens(wl, 1, stream=1)
+    cache0 = inputs.synthetic_cache(wl, N - 1, max_slots)
+    for variant in ("uniform", "mixed"):
+        if variant == "uniform":
+            pos = np.full(wl.B, N - 1)
+        else:
+            pos = np.array([(N - 1 - 61 * b) % N for b in range(wl.B)])
+            pos[5] = 0
+            pos[6] = s - 1
+        pb = Problem(wl, max_slots=max_slots, weights=w)
+        pb.buf.cache.copy_(cache0["cache"].to(pb.dt))
+        pb.buf.open_slot.copy_(cache0["acc"])
+        out = np64(pb.decode(toks, 0, pos))
+        sample = [0, 5, 6, 31, 63]
+        sub = lambda x: None if x is None else x[sample]
+        cfg = oracle_cfg(wl, B=len(sample))
+        cache_o = cache0["cache"][sample].double().numpy().copy()
+        acc_o = cache0["acc"][sample].double().numpy().copy()
+        ref = oracle.decode_step(cfg, sub(toks["c"][:, 0]), sub(toks["kr"][:, 0]),
+                                 sub(toks["qc"][:, 0]), sub(toks["qr"][:, 0]), w["w_uk"],
+                                 w["w_uv"], pos[sample], cache_o, acc_o, w["gate_w"], w["gate_b"])
+        assert rel_err(out[sample], ref["out"]) <= TOL["bf16"], variant
+        for i, b in enumerate(sample):
+            j = pos[b] // s
+            assert rel_err(np64(pb.buf.cache[b, j]), cache_o[i, j]) <= 4e-3
+        assert rel_err(np64(pb.buf.open_slot[sample]), acc_o) <= 1e-5
+
+
+# ----------------------------------------------------------------- prefill
+
+def test_prefill_full_size_sampled_rows():
+    """B=8, T=8192, H=8, d_h=64, d_c=256, d_R=32, s=2: the whole prefill on the
+    GPU; sampled rows (every sequence, block starts and ends, the first and last
+    rows) and all cache slots against the oracle."""
+    wl = inputs.PREFILL
+    T = wl.T
+    w = inputs.weights(wl)
+    toks = inputs.tokens(wl, T)
+    n_slots = T // wl.s
+    pb = Problem(wl, max_slots=n_slots, max_tokens=T, weights=w)
+    out = np64(pb.prefill(toks, T))
+    ts = [0, 1, 2, 3, 127, 128, 129, 1000, 4095, 4096, 6001, 8190, 8191]
+    rows = [(b, t) for b in range(wl.B) for t in ts]
+    ref, P = oracle_rows(wl, w, toks, rows)
+    got = np.stack([out[b, t] for b, t in rows])
+    assert rel_err(got, ref) <= TOL["bf16"]
+    assert rel_err(np64(pb.buf.cache), _slots_from_P(P, T, wl.s)) <= 4e-3
+    assert rel_err(np64(pb.buf.open_slot), P[:, T - 1]) <= 1e-5
+
+
+# ----------------------------------------------------------------- large latent
+
+def test_large_latent_decode():
+    """B=32, H=128, d_c=512, d_R=64 (absorbed width 576), s=4, N=65536 tokens
+    after the step (16384 slots per sequence), supplied gates sigmoid(N(0,1)):
+    one decode step at pos = N-1 on a synthetic cache; every head of sampled
+    sequences against the oracle's incremental step."""
+    wl = inputs.LARGE_LATENT
+    N = wl.T
+    max_slots = N // wl.s
+    w = inputs.weights(wl)
+    toks = inputs.tokens(wl, 1, stream=1)
+    cache0 = inputs.synthetic_cache(wl, N - 1, max_slots)
+    pb = Problem(wl, max_slots=max_slots, weights=w)
+    pb.buf.cache.copy_(cache0["cache"].to(pb.dt))
+    pb.buf.open_slot.copy_(cache0["acc"])
+    pos = np.full(wl.B, N - 1)
+    out = np64(pb.decode(toks, 0, pos))
+    sample = [0, 31]
+    sub = lambda x: x[sample]
+    cfg = oracle_cfg(wl, B=len(sample))
+    cache_o = cache0["cache"][sample].double().numpy().copy()
+    acc_o = cache0["acc"][sample].double().numpy().copy()
+    ref = oracle.decode_step(cfg, sub(toks["c"][:, 0]), sub(toks["kr"][:, 0]), sub(toks["qc"][:, 0]),
+                             sub(toks["qr"][:, 0]), w["w_uk"], w["w_uv"], pos[sample], cache_o, acc_o,
+                             gate_in=sub(toks["gate_in"][:, 0]))
+    assert rel_err(out[sample], ref["out"]) <= TOL["bf16"]
+    j = (N - 1) // wl.s
+    assert rel_err(np64(pb.buf.cache[sample, j]), cache_o[:, j]) <= 4e-3
+    assert rel_err(np64(pb.buf.open_slot[sample]), acc_o) <= 1e-5
+
+
+# ----------------------------------------------------------------- device-side errors
+
+def test_position_beyond_cache_latches_capacity():
+    """pos >= max_slots*s skips that sequence (its output untouched) and latches
+    CAPACITY; the other sequences are still computed correctly."""
+    wl = inputs.TINY_FP32.with_(B=3)
+    w = inputs.weights(wl)
+    toks = inputs.tokens(wl, 1)
+    pb = Problem(wl, max_slots=4, weights=w)
+    out = torch.full((wl.B, wl.H, wl.d_h), 7.0, device="cuda")
+    pos = torch.tensor([0, 8, 0], dtype=torch.int32, device="cuda")  # 8 >= 4*2
+    gw, gb = pb.gate_ptrs()
+    from gpu_harness import dev
+    mtla.decode_step(pb.cfg, dev(toks["c"][:, 0], pb.dt), dev(toks["kr"][:, 0], pb.dt),
+                     dev(toks["qc"][:, 0], pb.dt), dev(toks["qr"][:, 0], pb.dt), pb.buf.w_uk,
+                     pb.buf.w_uv, gw, gb, None, pos, pb.buf.cache, pb.buf.open_slot, out,
+                     pb.buf.workspace)
+    assert mtla.get_device_status() == mtla.ERR_CAPACITY
+    assert torch.all(out[1] == 7.0)
+    assert not torch.any(out[0] == 7.0)
+    assert mtla.get_device_status() == mtla.OK   # cleared by the read
