@@ -186,35 +186,38 @@ class Replica:
         return [(self.T + k) // self.wl.s + 1 for k in range(self.S)]
 
 
-def _cpu_sample(n_decode: int = 8):
-    """The oracle on a bounded sample of the workload: one of the B sequences,
-    the parallel prefill of its 1024-token prefix, then n_decode incremental
-    steps from the oracle's own cache. Returns (tokens, seconds, threads)."""
+def _cpu_step():
+    """The float64 oracle on one whole step of this workload for one replica:
+    the parallel prefill of the 1024-token prefix of all 16 sequences, then the
+    256 incremental decode steps from the oracle's own cache.
+    Returns (tokens, seconds, threads)."""
     import numpy as np
 
     import oracle
-    wl = WL.with_(B=1)
-    w = inputs.weights(WL)
-    pre = inputs.tokens(WL, WL.T, stream=0)
-    dec = inputs.tokens(WL, n_decode, stream=1)
-    one = lambda d: {k: (None if v is None else v[:1]) for k, v in d.items()}
-    pre, dec = one(pre), one(dec)
-    cfg = oracle.Cfg(1, wl.H, wl.d_h, wl.d_c, wl.d_r, wl.s, gate_mode=wl.gate_mode)
+    wl = WL
+    w = inputs.weights(wl)
+    pre = inputs.tokens(wl, wl.T, stream=0)
+    dec = inputs.tokens(wl, wl.steps, stream=1)
+    cfg = oracle.Cfg(wl.B, wl.H, wl.d_h, wl.d_c, wl.d_r, wl.s, gate_mode=wl.gate_mode)
     oracle.build()
     t0 = time.perf_counter()
     r = oracle.prefill(cfg, pre["c"], pre["kr"], pre["qc"], pre["qr"], w["w_uk"], w["w_uv"],
                        w["gate_w"], w["gate_b"])
-    max_slots = (WL.T + n_decode + wl.s - 1) // wl.s
-    cache = np.zeros((1, max_slots, wl.D))
-    n = r["cache"].shape[1]
-    cache[:, :n] = r["cache"]
+    max_slots = (wl.T + wl.steps + wl.s - 1) // wl.s
+    cache = np.zeros((wl.B, max_slots, wl.D))
+    cache[:, : r["cache"].shape[1]] = r["cache"]
     acc = r["acc"].copy()
-    for k in range(n_decode):
+    for k in range(wl.steps):
         oracle.decode_step(cfg, dec["c"][:, k], dec["kr"][:, k], dec["qc"][:, k], dec["qr"][:, k],
-                           w["w_uk"], w["w_uv"], [WL.T + k], cache, acc, w["gate_w"], w["gate_b"])
+                           w["w_uk"], w["w_uv"], np.full(wl.B, wl.T + k), cache, acc,
+                           w["gate_w"], w["gate_b"])
     dt = time.perf_counter() - t0
     threads = int(os.environ.get("OMP_NUM_THREADS", "0")) or len(os.sched_getaffinity(0))
-    return WL.T + n_decode, dt, threads
+    return wl.B * (wl.T + wl.steps), dt, threads
+
+
+CPU_SAMPLE = ("one whole step of one replica: parallel prefill of the 1024-token prefix of all 16 "
+              "sequences + 256 incremental decode steps (float64 C oracle, OpenMP)")
 
 
 def _config(ws: int):
@@ -230,7 +233,7 @@ def run_reference(args, ws, rank):
         return
     times, toks, threads = [], 0, 1
     for i in range(args.warmup + args.steps):
-        n, dt, threads = _cpu_sample()
+        n, dt, threads = _cpu_step()
         if i >= args.warmup:
             times.append(dt)
             toks += n
@@ -242,8 +245,7 @@ def run_reference(args, ws, rank):
         "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": _config(ws),
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                         "sample": "per step: 1 of 16 sequences, parallel prefill of 1024 tokens + "
-                                   "8 incremental decode steps (float64 C oracle, OpenMP)"},
+                         "sample": CPU_SAMPLE},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -334,10 +336,9 @@ def main():
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        n, dt, threads = _cpu_sample()
+        n, dt, threads = _cpu_step()
         cpu = {"value": n / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-               "sample": f"1 of 16 sequences: parallel prefill of {WL.T} tokens + 8 incremental "
-                         f"decode steps ({dt:.1f} s, float64 C oracle, OpenMP)"}
+               "sample": CPU_SAMPLE + f" ({dt:.1f} s)"}
 
     if rank == 0:
         line = {

@@ -24,15 +24,23 @@ static bool g_prof_open = false;
 void profile_begin(cudaStream_t st) {
     g_prof_open = false;
     if (g_prof_events && g_prof_next < g_prof_pairs) {
-        cudaEventRecord((cudaEvent_t)g_prof_events[2 * g_prof_next], st);
-        g_prof_open = true;
+        if (cudaEventRecord((cudaEvent_t)g_prof_events[2 * g_prof_next], st) == cudaSuccess) {
+            g_prof_open = true;
+        } else {
+            cudaGetLastError();            // a bad handle turns the hook off, not the call
+            g_prof_events = nullptr;
+        }
     }
 }
 
 void profile_end(cudaStream_t st) {
     if (g_prof_open) {
-        cudaEventRecord((cudaEvent_t)g_prof_events[2 * g_prof_next + 1], st);
-        ++g_prof_next;
+        if (cudaEventRecord((cudaEvent_t)g_prof_events[2 * g_prof_next + 1], st) == cudaSuccess) {
+            ++g_prof_next;
+        } else {
+            cudaGetLastError();
+            g_prof_events = nullptr;
+        }
         g_prof_open = false;
     }
 }

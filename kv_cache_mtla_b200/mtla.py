@@ -155,6 +155,9 @@ class ProfileEvents:
 
     def __init__(self, n_pairs: int):
         self.events = [torch.cuda.Event(enable_timing=True) for _ in range(2 * n_pairs)]
+        for e in self.events:          # torch creates the CUDA event at its first record
+            e.record()
+        torch.cuda.synchronize()
         self._arr = (ctypes.c_void_p * (2 * n_pairs))(*[e.cuda_event for e in self.events])
         self.n = n_pairs
 
