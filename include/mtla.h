@@ -157,6 +157,38 @@ mtla_status mtla_prefill(const mtla_config* cfg, int32_t T,
                          void* out, void* cache_out, float* open_slot_out,
                          void* workspace, size_t workspace_bytes, void* stream);
 
+/* Decode step without a workspace argument, for callers that cannot allocate
+ * device memory themselves: code inside a host framework whose pool allocator
+ * owns all device memory and forbids raw cudaMalloc, serving loops that cannot
+ * afford a cudaMalloc/cudaFree (which may synchronise the device) in the
+ * middle of a step, or plug-in hosts that hand over only input and output
+ * buffers. The pages describe no such interface: it has no counterpart in the
+ * paper.
+ *
+ * Same arguments, meaning and result as mtla_decode_step, minus `workspace`
+ * and `workspace_bytes`: the scratch comes from one array of
+ * MTLA_NOALLOC_SCRATCH_BYTES bytes in device memory that libmtla.so declares;
+ * every GPU that loads the library holds it until the process exits. The call
+ * allocates nothing (no cudaMalloc, cudaFree or allocating library routine).
+ *   - Limit: a config whose decode scratch (mtla_workspace_size with
+ *     max_tokens = 0) exceeds MTLA_NOALLOC_SCRATCH_BYTES is refused on the host
+ *     with MTLA_ERR_WORKSPACE before anything is launched.
+ *   - Set-up: the first call on a device looks up the array's device address
+ *     on that device (cudaGetSymbolAddress, with that device current); make
+ *     that first call before any stream capture.
+ *   - Sharing: all calls on a device share the one array, which keeps the last
+ *     call's contents. Calls whose kernels overlap on the GPU (different
+ *     streams with no ordering between them) race on it and give wrong
+ *     results; order them, or use mtla_decode_step with separate workspaces. */
+#define MTLA_NOALLOC_SCRATCH_BYTES (8u << 20)
+mtla_status mtla_decode_step_noalloc(const mtla_config* cfg,
+                                     const void* c_new, const void* kr_new,
+                                     const void* q_c, const void* q_r,
+                                     const void* w_uk, const void* w_uv,
+                                     const float* gate_w, const float* gate_b,
+                                     const float* gate_in, const int32_t* pos,
+                                     void* cache, float* open_slot, void* out, void* stream);
+
 /* Synchronises `stream`, then returns and clears the status latched by
  * device-side checks on the current device since the last call (OK if none). */
 mtla_status mtla_get_device_status(void* stream);

@@ -71,6 +71,8 @@ def load() -> ctypes.CDLL:
     lib.mtla_decode_step.restype = ctypes.c_int
     lib.mtla_prefill.argtypes = [cp, ctypes.c_int32] + [_vp] * 12 + [_vp, ctypes.c_size_t, _vp]
     lib.mtla_prefill.restype = ctypes.c_int
+    lib.mtla_decode_step_noalloc.argtypes = [cp] + [_vp] * 13 + [_vp]
+    lib.mtla_decode_step_noalloc.restype = ctypes.c_int
     lib.mtla_get_device_status.argtypes = [_vp]
     lib.mtla_get_device_status.restype = ctypes.c_int
     lib.mtla_status_string.argtypes = [ctypes.c_int]
@@ -126,6 +128,22 @@ def decode_step(cfg, c_new, kr_new, q_c, q_r, w_uk, w_uv, gate_w, gate_b, gate_i
     if check and st != OK:
         raise MtlaError(st, "mtla_decode_step")
     return st
+
+
+def decode_step_noalloc(cfg, c_new, kr_new, q_c, q_r, w_uk, w_uv, gate_w, gate_b, gate_in, pos,
+                        cache, open_slot, out, stream=None, check=True) -> int:
+    """Forward to ``mtla_decode_step_noalloc`` (no workspace: the library's
+    built-in scratch array is used); returns the status (raises if check)."""
+    st = load().mtla_decode_step_noalloc(
+        ctypes.byref(cfg), _ptr(c_new), _ptr(kr_new), _ptr(q_c), _ptr(q_r), _ptr(w_uk),
+        _ptr(w_uv), _ptr(gate_w), _ptr(gate_b), _ptr(gate_in), _ptr(pos), _ptr(cache),
+        _ptr(open_slot), _ptr(out), _stream(stream))
+    if check and st != OK:
+        raise MtlaError(st, "mtla_decode_step_noalloc")
+    return st
+
+
+NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
 def prefill(cfg, T, c, kr, q_c, q_r, w_uk, w_uv, gate_w, gate_b, gate_in, out, cache_out,
