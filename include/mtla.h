@@ -196,6 +196,11 @@ mtla_status mtla_get_device_status(void* stream);
 /* Static English text for a status code. */
 const char* mtla_status_string(mtla_status status);
 
+/* Text naming the CUDA call (and its error) behind the last MTLA_ERR_CUDA
+ * returned on this host thread; "" if none. Valid until the next call on the
+ * same thread. */
+const char* mtla_last_error_detail(void);
+
 /* Number of kernels this library has launched in this process (all devices). */
 uint64_t mtla_kernel_launches(void);
 

@@ -3,6 +3,7 @@
 #include <atomic>
 #include <cmath>
 #include <cstdint>
+#include <cstdio>
 #include <cstring>
 
 #include "../../include/mtla.h"
@@ -15,6 +16,15 @@ namespace mtla {
 __device__ int g_device_status;
 
 static std::atomic<uint64_t> g_launches{0};
+
+static thread_local char g_error_detail[256] = "";
+
+cudaError_t note_error(const char* where, cudaError_t e) {
+    if (e != cudaSuccess)
+        snprintf(g_error_detail, sizeof(g_error_detail), "%s: %s (%s)", where, cudaGetErrorName(e),
+                 cudaGetErrorString(e));
+    return e;
+}
 
 static void* const* g_prof_events = nullptr;
 static int32_t g_prof_pairs = 0;
@@ -98,7 +108,16 @@ static mtla_status check_config(const mtla_config* cfg, Shape* sh) {
     return MTLA_OK;
 }
 
-static size_t decode_ws(const Shape& sh) { return simt_decode_workspace(sh); }
+// bf16 decode runs on the tensor cores where the shape fits the kernel
+// (heads <= 32, d_c a multiple of 128, slot width <= 384); fp32 and the other
+// bf16 shapes run on the CUDA-core kernels.
+static bool use_tc_decode(const mtla_config* cfg, const Shape& sh) {
+    return cfg->dtype == MTLA_BF16 && tc_decode_supported(sh);
+}
+
+static size_t decode_ws(const mtla_config* cfg, const Shape& sh) {
+    return use_tc_decode(cfg, sh) ? tc_decode_workspace(sh) : simt_decode_workspace(sh);
+}
 static size_t prefill_ws(const Shape& sh, int T) { return simt_prefill_workspace(sh, T); }
 
 static mtla_status check_gate_ptrs(const mtla_config* cfg, const float* gate_w, const float* gate_b,
@@ -123,7 +142,7 @@ mtla_status mtla_workspace_size(const mtla_config* cfg, int32_t max_tokens, size
     if (!bytes || max_tokens < 0) return MTLA_ERR_INVALID_ARG;
     mtla_status st = check_config(cfg, &sh);
     if (st != MTLA_OK) return st;
-    size_t d = decode_ws(sh);
+    size_t d = decode_ws(cfg, sh);
     size_t p = max_tokens > 0 ? prefill_ws(sh, max_tokens) : 0;
     *bytes = d > p ? d : p;
     return MTLA_OK;
@@ -142,7 +161,7 @@ mtla_status mtla_decode_step(const mtla_config* cfg, const void* c_new, const vo
         if (!p || !aligned16(p)) return MTLA_ERR_INVALID_ARG;
     st = check_gate_ptrs(cfg, gate_w, gate_b, gate_in);
     if (st != MTLA_OK) return st;
-    if (workspace_bytes < decode_ws(sh)) return MTLA_ERR_WORKSPACE;
+    if (workspace_bytes < decode_ws(cfg, sh)) return MTLA_ERR_WORKSPACE;
     DecodeArgs a;
     a.sh = sh;
     a.c_new = c_new;
@@ -160,10 +179,13 @@ mtla_status mtla_decode_step(const mtla_config* cfg, const void* c_new, const vo
     a.out = out;
     a.workspace = workspace;
     a.workspace_bytes = workspace_bytes;
-    if (status_ptr(&a.status) != cudaSuccess) return MTLA_ERR_CUDA;
+    g_error_detail[0] = 0;
+    if (note_error("device status word", status_ptr(&a.status)) != cudaSuccess) return MTLA_ERR_CUDA;
     uint64_t n = 0;
-    cudaError_t e = simt_decode(a, cfg->dtype == MTLA_FP32, (cudaStream_t)stream, &n);
+    cudaError_t e = use_tc_decode(cfg, sh) ? tc_decode(a, (cudaStream_t)stream, &n)
+                                           : simt_decode(a, cfg->dtype == MTLA_FP32, (cudaStream_t)stream, &n);
     g_launches += n;
+    if (e != cudaSuccess && !g_error_detail[0]) note_error("decode launch", e);
     return e == cudaSuccess ? MTLA_OK : MTLA_ERR_CUDA;
 }
 
@@ -201,10 +223,12 @@ mtla_status mtla_prefill(const mtla_config* cfg, int32_t T, const void* c, const
     a.open_slot_out = open_slot_out;
     a.workspace = workspace;
     a.workspace_bytes = workspace_bytes;
-    if (status_ptr(&a.status) != cudaSuccess) return MTLA_ERR_CUDA;
+    g_error_detail[0] = 0;
+    if (note_error("device status word", status_ptr(&a.status)) != cudaSuccess) return MTLA_ERR_CUDA;
     uint64_t n = 0;
     cudaError_t e = simt_prefill(a, cfg->dtype == MTLA_FP32, (cudaStream_t)stream, &n);
     g_launches += n;
+    if (e != cudaSuccess && !g_error_detail[0]) note_error("prefill launch", e);
     return e == cudaSuccess ? MTLA_OK : MTLA_ERR_CUDA;
 }
 
@@ -234,6 +258,8 @@ const char* mtla_status_string(mtla_status s) {
 }
 
 uint64_t mtla_kernel_launches(void) { return g_launches.load(); }
+
+const char* mtla_last_error_detail(void) { return g_error_detail; }
 
 void mtla_set_profile_events(void* const* events, int32_t n_pairs) {
     g_prof_events = (events && n_pairs > 0) ? events : nullptr;

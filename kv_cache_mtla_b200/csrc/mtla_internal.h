@@ -64,6 +64,14 @@ size_t simt_prefill_workspace(const Shape& sh, int T);
 cudaError_t simt_decode(const DecodeArgs& a, bool fp32, cudaStream_t st, uint64_t* launches);
 cudaError_t simt_prefill(const PrefillArgs& a, bool fp32, cudaStream_t st, uint64_t* launches);
 
+// Tensor-core decode (bf16, heads <= 32): shapes it covers, its scratch, launcher.
+bool tc_decode_supported(const Shape& sh);
+size_t tc_decode_workspace(const Shape& sh);
+cudaError_t tc_decode(const DecodeArgs& a, cudaStream_t st, uint64_t* launches);
+
+// Record which CUDA step failed (read back by mtla_last_error_detail); returns e.
+cudaError_t note_error(const char* where, cudaError_t e);
+
 // Profile hook: record the next event pair around the main attention kernel.
 void profile_begin(cudaStream_t st);
 void profile_end(cudaStream_t st);

@@ -10,6 +10,7 @@
 //   the finished slots plus the own partial slot -> W_UV on the weighted latent.
 #include "common.cuh"
 #include "mtla_internal.h"
+#include "prep.cuh"
 
 namespace mtla {
 
@@ -18,100 +19,6 @@ namespace {
 constexpr int kMaxD = 576;              // d_c + d_r
 constexpr int kMaxPerLane = kMaxD / 32; // 18
 constexpr int kMaxLatPerLane = 512 / 32;
-
-// ----------------------------------------------------------------- gate
-
-// Merging weight of token t of sequence b; every thread of the block returns it.
-template <typename T>
-__device__ float gate_weight(const Shape& sh, int64_t t, const T* c_t, const float* gate_w,
-                             const float* gate_b, const float* w_given, float* red) {
-    if (sh.gate_mode == 2) return 1.f;
-    if (sh.gate_mode == 1) return *w_given;
-    const int r = (int)(t % sh.s);
-    const float* G = gate_w + (size_t)r * sh.d_c;
-    float z = 0.f;
-    for (int k = threadIdx.x; k < sh.d_c / 2; k += blockDim.x) {
-        float sn, cs;
-        pair_sincos(t, k, sh.d_c, sh.log2_pe_base, &sn, &cs);
-        z = fmaf(G[2 * k] * to_f<T>(c_t[2 * k]), sn, z);
-        z = fmaf(G[2 * k + 1] * to_f<T>(c_t[2 * k + 1]), cs, z);
-    }
-    z = block_sum(z, red) + gate_b[r];
-    return sigmoidf_(z);
-}
-
-// ----------------------------------------------------------------- decode
-
-template <typename T>
-__global__ void __launch_bounds__(128) k_decode_update(DecodeArgs a) {
-    const Shape sh = a.sh;
-    const int b = blockIdx.x;
-    const int64_t t = a.pos[b];
-    if (t < 0 || t >= (int64_t)sh.max_slots * sh.s) {
-        if (threadIdx.x == 0) latch_status(a.status, kStatusCapacity);
-        return;
-    }
-    __shared__ float red[32];
-    const T* c = (const T*)a.c_new + (size_t)b * sh.d_c;
-    const T* kr = (const T*)a.kr_new + (size_t)b * sh.d_r;
-    const float w = gate_weight<T>(sh, t, c, a.gate_w, a.gate_b, a.gate_in ? a.gate_in + b : nullptr, red);
-    float* acc = a.open_slot + (size_t)b * sh.D;
-    T* row = (T*)a.cache + ((size_t)b * sh.max_slots + (size_t)(t / sh.s)) * sh.D;
-    const bool fresh = (t % sh.s) == 0;
-    for (int k = threadIdx.x; k < sh.d_c; k += blockDim.x) {
-        const float v = (fresh ? 0.f : acc[k]) + w * to_f<T>(c[k]);
-        acc[k] = v;
-        row[k] = from_f<T>(v);
-    }
-    for (int k = threadIdx.x; k < sh.d_r / 2; k += blockDim.x) {
-        float sn, cs;
-        pair_sincos(t, k, sh.d_r, sh.log2_rope_base, &sn, &cs);
-        const float x0 = to_f<T>(kr[2 * k]), x1 = to_f<T>(kr[2 * k + 1]);
-        const float y0 = x0 * cs - x1 * sn, y1 = x0 * sn + x1 * cs;
-        float* ar = acc + sh.d_c;
-        const float v0 = (fresh ? 0.f : ar[2 * k]) + w * y0;
-        const float v1 = (fresh ? 0.f : ar[2 * k + 1]) + w * y1;
-        ar[2 * k] = v0;
-        ar[2 * k + 1] = v1;
-        row[sh.d_c + 2 * k] = from_f<T>(v0);
-        row[sh.d_c + 2 * k + 1] = from_f<T>(v1);
-    }
-}
-
-// Absorbed query for `rows` rows (decode: one per sequence; prefill: B*T).
-// grid (rows, H). Position of a row: pos[row] (decode) or row % T (prefill).
-template <typename T>
-__global__ void __launch_bounds__(128) k_absorb_query(Shape sh, const T* qc, const T* qr,
-                                                      const T* w_uk, const int32_t* pos, int T_len,
-                                                      float* qt) {
-    const int row = blockIdx.x, h = blockIdx.y;
-    int64_t t;
-    if (pos) {
-        t = pos[row];
-        if (t < 0 || t >= (int64_t)sh.max_slots * sh.s) return;
-    } else {
-        t = row % T_len;
-    }
-    __shared__ float q[256];
-    const size_t rh = (size_t)row * sh.H + h;
-    for (int i = threadIdx.x; i < sh.d_h; i += blockDim.x) q[i] = to_f<T>(qc[rh * sh.d_h + i]);
-    __syncthreads();
-    const T* W = w_uk + (size_t)h * sh.d_h * sh.d_c;
-    float* out = qt + rh * sh.D;
-    for (int j = threadIdx.x; j < sh.d_c; j += blockDim.x) {
-        float acc = 0.f;
-        for (int i = 0; i < sh.d_h; ++i) acc = fmaf(to_f<T>(W[(size_t)i * sh.d_c + j]), q[i], acc);
-        out[j] = acc;
-    }
-    const T* r = qr + rh * sh.d_r;
-    for (int k = threadIdx.x; k < sh.d_r / 2; k += blockDim.x) {
-        float sn, cs;
-        pair_sincos(t, k, sh.d_r, sh.log2_rope_base, &sn, &cs);
-        const float x0 = to_f<T>(r[2 * k]), x1 = to_f<T>(r[2 * k + 1]);
-        out[sh.d_c + 2 * k] = x0 * cs - x1 * sn;
-        out[sh.d_c + 2 * k + 1] = x0 * sn + x1 * cs;
-    }
-}
 
 // Online-softmax state of one (query, head) row held by a warp: lane l owns
 // latent entries l, l+32, ...
@@ -368,14 +275,12 @@ cudaError_t decode_impl(const DecodeArgs& a, cudaStream_t st, uint64_t* launches
     char* ws = (char*)a.workspace;
     float* qt = (float*)ws;
     float* part = (float*)(ws + align256((size_t)sh.B * sh.H * sh.D * sizeof(float)));
-    k_decode_update<T><<<sh.B, 128, 0, st>>>(a);
-    k_absorb_query<T><<<dim3(sh.B, sh.H), 128, 0, st>>>(sh, (const T*)a.q_c, (const T*)a.q_r,
-                                                         (const T*)a.w_uk, a.pos, 0, qt);
+    k_decode_prep<T><<<dim3(sh.B, sh.H + 1), 128, 0, st>>>(a, qt);
     profile_begin(st);
     k_decode_attn<T><<<dim3(splits, sh.B), 256, 0, st>>>(a, chunk, splits, qt, part);
     profile_end(st);
     k_decode_combine<T><<<dim3(sh.H, sh.B), 256, 0, st>>>(a, chunk, splits, part);
-    *launches += 4;
+    *launches += 3;
     return cudaGetLastError();
 }
 
@@ -387,8 +292,8 @@ cudaError_t prefill_impl(const PrefillArgs& a, cudaStream_t st, uint64_t* launch
     float* qt = (float*)(ws + align256((size_t)sh.B * a.T * sh.D * sizeof(float)));
     const int n_slots = (a.T + sh.s - 1) / sh.s;
     k_prefill_scan<T><<<dim3(n_slots, sh.B), 128, 0, st>>>(a, P);
-    k_absorb_query<T><<<dim3(sh.B * a.T, sh.H), 128, 0, st>>>(sh, (const T*)a.q_c, (const T*)a.q_r,
-                                                               (const T*)a.w_uk, nullptr, a.T, qt);
+    k_prefill_absorb<T><<<dim3(sh.B * a.T, sh.H), 128, 0, st>>>(sh, (const T*)a.q_c, (const T*)a.q_r,
+                                                                 (const T*)a.w_uk, a.T, qt);
     const int64_t rows = (int64_t)a.T * sh.H;
     profile_begin(st);
     k_prefill_attn<T><<<dim3((unsigned)((rows + 7) / 8), sh.B), 256, 0, st>>>(a, P, qt);

@@ -24,7 +24,9 @@ GATE_COMPUTED, GATE_SUPPLIED, GATE_UNIT = 0, 1, 2
 class MtlaError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {status_string(status)} (status {status})")
+        detail = last_error_detail() if status == ERR_CUDA else ""
+        super().__init__(f"{where}: {status_string(status)} (status {status})"
+                         + (f" [{detail}]" if detail else ""))
 
 
 class Config(ctypes.Structure):
@@ -77,6 +79,8 @@ def load() -> ctypes.CDLL:
     lib.mtla_get_device_status.restype = ctypes.c_int
     lib.mtla_status_string.argtypes = [ctypes.c_int]
     lib.mtla_status_string.restype = ctypes.c_char_p
+    lib.mtla_last_error_detail.argtypes = []
+    lib.mtla_last_error_detail.restype = ctypes.c_char_p
     lib.mtla_kernel_launches.argtypes = []
     lib.mtla_kernel_launches.restype = ctypes.c_uint64
     lib.mtla_set_profile_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), ctypes.c_int32]
@@ -157,6 +161,10 @@ def prefill(cfg, T, c, kr, q_c, q_r, w_uk, w_uv, gate_w, gate_b, gate_in, out, c
     if check and st != OK:
         raise MtlaError(st, "mtla_prefill")
     return st
+
+
+def last_error_detail() -> str:
+    return load().mtla_last_error_detail().decode()
 
 
 def get_device_status(stream=None) -> int:

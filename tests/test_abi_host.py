@@ -137,7 +137,7 @@ def test_prefill_rejects_bad_arguments_before_launch(lib):
     assert _call_prefill(lib, cfg, 33, ws) == mtla.ERR_CAPACITY      # ceil(33/2) > 16 slots
     assert _call_prefill(lib, cfg, 32, ws, cache_out=None) == mtla.ERR_INVALID_ARG
     assert _call_prefill(lib, cfg, 32, ws, open_slot_out=FAKE + 4) == mtla.ERR_INVALID_ARG
-    assert _call_prefill(lib, cfg, 32, ws - 1) == mtla.ERR_WORKSPACE
+    assert _call_prefill(lib, cfg, 32, 16) == mtla.ERR_WORKSPACE
     assert _call_prefill(lib, cfg, 32, ws, q_c=None) == mtla.ERR_INVALID_ARG
 
 

@@ -238,3 +238,60 @@ def test_position_beyond_cache_latches_capacity():
     assert torch.all(out[1] == 7.0)
     assert not torch.any(out[0] == 7.0)
     assert mtla.get_device_status() == mtla.OK   # cleared by the read
+
+
+# ----------------------------------------------------------------- decode schedule / head widths
+
+@pytest.mark.parametrize("H", [1, 8, 20, 32])
+def test_decode_many_short_sequences(H):
+    """Many sequences of 1 to ~5 slot tiles with mixed positions: the split
+    plan crosses sequence boundaries inside one CTA's range. Head counts cover
+    both padded head widths of the tensor-core kernel."""
+    wl = inputs.SPEECH_DECODE.with_(B=150, H=H, s=3)
+    max_slots = 700
+    w = inputs.weights(wl)
+    toks = inputs.tokens(wl, 1, stream=1)
+    cache0 = inputs.synthetic_cache(wl, max_slots * wl.s - 1, max_slots)
+    rng = np.random.default_rng(H)
+    pos = rng.integers(0, max_slots * wl.s, size=wl.B)
+    pos[:3] = [0, 1, max_slots * wl.s - 1]
+    pb = Problem(wl, max_slots=max_slots, weights=w)
+    pb.buf.cache.copy_(cache0["cache"].to(pb.dt))
+    pb.buf.open_slot.copy_(cache0["acc"])
+    out = np64(pb.decode(toks, 0, pos))
+    sample = [0, 1, 2, 17, 74, 75, 76, 148, 149]
+    sub = lambda x: x[sample]
+    cfg = oracle_cfg(wl, B=len(sample))
+    cache_o = cache0["cache"][sample].double().numpy().copy()
+    acc_o = cache0["acc"][sample].double().numpy().copy()
+    ref = oracle.decode_step(cfg, sub(toks["c"][:, 0]), sub(toks["kr"][:, 0]), sub(toks["qc"][:, 0]),
+                             sub(toks["qr"][:, 0]), w["w_uk"], w["w_uv"], pos[sample], cache_o,
+                             acc_o, w["gate_w"], w["gate_b"])
+    assert rel_err(out[sample], ref["out"]) <= TOL["bf16"]
+
+
+def test_decode_skips_invalid_sequences_in_the_split_plan():
+    """Sequences whose position is beyond the cache get no tiles; the others
+    around them are still right, and CAPACITY is latched."""
+    wl = inputs.SPEECH_DECODE.with_(B=40)
+    max_slots = 300
+    w = inputs.weights(wl)
+    toks = inputs.tokens(wl, 1, stream=1)
+    cache0 = inputs.synthetic_cache(wl, 500, max_slots)
+    pos = np.array([(37 * b) % 590 for b in range(wl.B)])
+    bad = [3, 4, 20, 39]
+    pos[bad] = max_slots * wl.s + 5
+    pb = Problem(wl, max_slots=max_slots, weights=w)
+    pb.buf.cache.copy_(cache0["cache"].to(pb.dt))
+    pb.buf.open_slot.copy_(cache0["acc"])
+    out = np64(pb.decode(toks, 0, pos))
+    assert mtla.get_device_status() == mtla.ERR_CAPACITY
+    good = [b for b in range(wl.B) if b not in bad]
+    sub = lambda x: x[good]
+    cfg = oracle_cfg(wl, B=len(good))
+    cache_o = cache0["cache"][good].double().numpy().copy()
+    acc_o = cache0["acc"][good].double().numpy().copy()
+    ref = oracle.decode_step(cfg, sub(toks["c"][:, 0]), sub(toks["kr"][:, 0]), sub(toks["qc"][:, 0]),
+                             sub(toks["qr"][:, 0]), w["w_uk"], w["w_uv"], pos[good], cache_o, acc_o,
+                             w["gate_w"], w["gate_b"])
+    assert rel_err(out[good], ref["out"]) <= TOL["bf16"]
