@@ -211,7 +211,8 @@ uint64_t mtla_kernel_launches(void);
  * `events` holds cudaEvent_t handles created and owned by the caller and must
  * stay valid while the hook is set. mtla_set_profile_events(NULL, 0) turns
  * the hook off. mtla_profile_events_recorded() returns how many pairs were
- * recorded since the hook was set. */
+ * recorded since the hook was set. Inside stream capture the records become
+ * event nodes of the graph (recorded at every replay). */
 void mtla_set_profile_events(void* const* events, int32_t n_pairs);
 int32_t mtla_profile_events_recorded(void);
 

@@ -70,6 +70,12 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
     return r;
 }
 
+// Two floats as bf16 (round to nearest even), `lo` at the lower address.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
 __device__ __forceinline__ float sigmoidf_(float z) { return 1.f / (1.f + expf(-z)); }
 
 }  // namespace mtla

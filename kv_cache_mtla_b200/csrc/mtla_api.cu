@@ -34,7 +34,8 @@ static bool g_prof_open = false;
 void profile_begin(cudaStream_t st) {
     g_prof_open = false;
     if (g_prof_events && g_prof_next < g_prof_pairs) {
-        if (cudaEventRecord((cudaEvent_t)g_prof_events[2 * g_prof_next], st) == cudaSuccess) {
+        if (cudaEventRecordWithFlags((cudaEvent_t)g_prof_events[2 * g_prof_next], st,
+                                      cudaEventRecordExternal) == cudaSuccess) {
             g_prof_open = true;
         } else {
             cudaGetLastError();            // a bad handle turns the hook off, not the call
@@ -45,7 +46,8 @@ void profile_begin(cudaStream_t st) {
 
 void profile_end(cudaStream_t st) {
     if (g_prof_open) {
-        if (cudaEventRecord((cudaEvent_t)g_prof_events[2 * g_prof_next + 1], st) == cudaSuccess) {
+        if (cudaEventRecordWithFlags((cudaEvent_t)g_prof_events[2 * g_prof_next + 1], st,
+                                      cudaEventRecordExternal) == cudaSuccess) {
             ++g_prof_next;
         } else {
             cudaGetLastError();
@@ -118,7 +120,15 @@ static bool use_tc_decode(const mtla_config* cfg, const Shape& sh) {
 static size_t decode_ws(const mtla_config* cfg, const Shape& sh) {
     return use_tc_decode(cfg, sh) ? tc_decode_workspace(sh) : simt_decode_workspace(sh);
 }
-static size_t prefill_ws(const Shape& sh, int T) { return simt_prefill_workspace(sh, T); }
+// bf16 prefill runs on the tensor cores where the shape fits the kernel
+// (d_h = 64, d_c <= 256, slot width <= 320); the rest on the CUDA cores.
+static bool use_tc_prefill(const mtla_config* cfg, const Shape& sh) {
+    return cfg->dtype == MTLA_BF16 && tc_prefill_supported(sh);
+}
+
+static size_t prefill_ws(const mtla_config* cfg, const Shape& sh, int T) {
+    return use_tc_prefill(cfg, sh) ? tc_prefill_workspace(sh, T) : simt_prefill_workspace(sh, T);
+}
 
 static mtla_status check_gate_ptrs(const mtla_config* cfg, const float* gate_w, const float* gate_b,
                                    const float* gate_in) {
@@ -143,7 +153,7 @@ mtla_status mtla_workspace_size(const mtla_config* cfg, int32_t max_tokens, size
     mtla_status st = check_config(cfg, &sh);
     if (st != MTLA_OK) return st;
     size_t d = decode_ws(cfg, sh);
-    size_t p = max_tokens > 0 ? prefill_ws(sh, max_tokens) : 0;
+    size_t p = max_tokens > 0 ? prefill_ws(cfg, sh, max_tokens) : 0;
     *bytes = d > p ? d : p;
     return MTLA_OK;
 }
@@ -205,7 +215,7 @@ mtla_status mtla_prefill(const mtla_config* cfg, int32_t T, const void* c, const
     st = check_gate_ptrs(cfg, gate_w, gate_b, gate_in);
     if (st != MTLA_OK) return st;
     if ((int64_t)(T + sh.s - 1) / sh.s > sh.max_slots) return MTLA_ERR_CAPACITY;
-    if (workspace_bytes < prefill_ws(sh, T)) return MTLA_ERR_WORKSPACE;
+    if (workspace_bytes < prefill_ws(cfg, sh, T)) return MTLA_ERR_WORKSPACE;
     PrefillArgs a;
     a.sh = sh;
     a.T = T;
@@ -226,7 +236,8 @@ mtla_status mtla_prefill(const mtla_config* cfg, int32_t T, const void* c, const
     g_error_detail[0] = 0;
     if (note_error("device status word", status_ptr(&a.status)) != cudaSuccess) return MTLA_ERR_CUDA;
     uint64_t n = 0;
-    cudaError_t e = simt_prefill(a, cfg->dtype == MTLA_FP32, (cudaStream_t)stream, &n);
+    cudaError_t e = use_tc_prefill(cfg, sh) ? tc_prefill(a, (cudaStream_t)stream, &n)
+                                            : simt_prefill(a, cfg->dtype == MTLA_FP32, (cudaStream_t)stream, &n);
     g_launches += n;
     if (e != cudaSuccess && !g_error_detail[0]) note_error("prefill launch", e);
     return e == cudaSuccess ? MTLA_OK : MTLA_ERR_CUDA;

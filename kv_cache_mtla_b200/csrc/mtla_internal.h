@@ -69,6 +69,16 @@ bool tc_decode_supported(const Shape& sh);
 size_t tc_decode_workspace(const Shape& sh);
 cudaError_t tc_decode(const DecodeArgs& a, cudaStream_t st, uint64_t* launches);
 
+// Tensor-core prefill (bf16, d_h = 64, d_c <= 256, slot width <= 320).
+bool tc_prefill_supported(const Shape& sh);
+size_t tc_prefill_workspace(const Shape& sh, int T);
+cudaError_t tc_prefill(const PrefillArgs& a, cudaStream_t st, uint64_t* launches);
+
+// Driver entry point cuTensorMapEncodeTiled (NULL if unavailable), looked up once.
+void* tensor_map_encoder();
+// Streaming multiprocessors of the current device (cached per device).
+int sm_count();
+
 // Record which CUDA step failed (read back by mtla_last_error_detail); returns e.
 cudaError_t note_error(const char* where, cudaError_t e);
 

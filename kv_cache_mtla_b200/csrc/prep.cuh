@@ -83,7 +83,13 @@ __device__ void absorb_query_body(const Shape& sh, const T* qc, const T* qr, con
     float* out = qt + rh * sh.D;
     for (int j = threadIdx.x; j < sh.d_c; j += blockDim.x) {
         float acc = 0.f;
-        for (int i = 0; i < sh.d_h; ++i) acc = fmaf(to_f<T>(W[(size_t)i * sh.d_c + j]), q[i], acc);
+        for (int i0 = 0; i0 < sh.d_h; i0 += 16) {      // d_h is a multiple of 16
+            float wv[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) wv[u] = to_f<T>(W[(size_t)(i0 + u) * sh.d_c + j]);
+#pragma unroll
+            for (int u = 0; u < 16; ++u) acc = fmaf(wv[u], q[i0 + u], acc);
+        }
         out[j] = acc;
     }
     const T* r = qr + rh * sh.d_r;
@@ -117,6 +123,122 @@ __global__ void __launch_bounds__(128) k_prefill_absorb(Shape sh, const T* qc, c
                                                         int T_len, float* qt) {
     const int64_t row = blockIdx.x;
     absorb_query_body<T>(sh, qc, qr, w_uk, row, blockIdx.y, row % T_len, qt);
+}
+
+// 8 consecutive values as float (T = float or bf16; 16-byte aligned address).
+template <typename T> __device__ __forceinline__ void load8(const T* p, float* v);
+template <> __device__ __forceinline__ void load8<float>(const float* p, float* v) {
+    const float4 a = *(const float4*)p, c = *(const float4*)(p + 4);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = c.x; v[5] = c.y; v[6] = c.z; v[7] = c.w;
+}
+template <> __device__ __forceinline__ void load8<bf16>(const bf16* p, float* v) {
+    const uint4 raw = *(const uint4*)p;
+    const bf16* h = (const bf16*)&raw;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __bfloat162float(h[i]);
+}
+template <typename T> __device__ __forceinline__ void store8(T* p, const float* v);
+template <> __device__ __forceinline__ void store8<float>(float* p, const float* v) {
+    *(float4*)p = make_float4(v[0], v[1], v[2], v[3]);
+    *(float4*)(p + 4) = make_float4(v[4], v[5], v[6], v[7]);
+}
+template <> __device__ __forceinline__ void store8<bf16>(bf16* p, const float* v) {
+    uint4 raw;
+    raw.x = pack_bf16x2(v[0], v[1]);
+    raw.y = pack_bf16x2(v[2], v[3]);
+    raw.z = pack_bf16x2(v[4], v[5]);
+    raw.w = pack_bf16x2(v[6], v[7]);
+    *(uint4*)p = raw;
+}
+
+// Block-prefix scan (MTLA Sec. 4.2): for slot j of sequence b, the merging
+// weights w_u (Sec. 4.1, Eq. 13) of its tokens u and the partial slots
+//   P_u = sum_{v = s*j}^{u} w_v [c_v ; RoPE_v(k_v)]
+// (stored as PT), the slot itself in the cache (rounded to T: finished, or the
+// last one) and, for the slot holding token T-1, the unrounded open slot.
+// One warp per slot: grid (ceil(ceil(T/s) / 8), B), 256 threads.
+template <typename T, typename PT>
+__global__ void __launch_bounds__(256) k_prefill_scan(PrefillArgs a, PT* P) {
+    const Shape sh = a.sh;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int b = blockIdx.y;
+    const int Tn = a.T;
+    __shared__ double pe_freq[256];     // PE frequencies, d_c / 2 <= 256
+    __shared__ double rope_freq[288];   // RoPE frequencies, d_r / 2 <= 280
+    for (int k = threadIdx.x; k < sh.d_c / 2; k += blockDim.x)
+        pe_freq[k] = exp2(-(2.0 * k / (double)sh.d_c) * sh.log2_pe_base);
+    for (int k = threadIdx.x; k < sh.d_r / 2; k += blockDim.x)
+        rope_freq[k] = exp2(-(2.0 * k / (double)sh.d_r) * sh.log2_rope_base);
+    __syncthreads();
+    const int n_slots = (Tn + sh.s - 1) / sh.s;
+    const int j = blockIdx.x * 8 + warp;
+    if (j >= n_slots) return;
+    const int u0 = j * sh.s, nu = min(sh.s, Tn - u0);
+    const T* c = (const T*)a.c + ((size_t)b * Tn + u0) * sh.d_c;
+    const T* kr = (const T*)a.kr + ((size_t)b * Tn + u0) * sh.d_r;
+    float wv[8];
+#pragma unroll
+    for (int uo = 0; uo < 8; ++uo) {
+        wv[uo] = 0.f;
+        if (uo >= nu) continue;
+        const int u = u0 + uo;
+        if (sh.gate_mode == 2) {
+            wv[uo] = 1.f;
+        } else if (sh.gate_mode == 1) {
+            wv[uo] = a.gate_in[(size_t)b * Tn + u];
+        } else {
+            const int r = u % sh.s;
+            const float* G = a.gate_w + (size_t)r * sh.d_c;
+            const T* cu = c + (size_t)uo * sh.d_c;
+            float z = 0.f;
+            for (int k = lane; k < sh.d_c / 2; k += 32) {
+                float sn, cs;
+                pair_sincos_f(u, pe_freq[k], &sn, &cs);
+                z = fmaf(G[2 * k] * to_f<T>(cu[2 * k]), sn, z);
+                z = fmaf(G[2 * k + 1] * to_f<T>(cu[2 * k + 1]), cs, z);
+            }
+            wv[uo] = sigmoidf_(warp_sum(z) + a.gate_b[r]);
+        }
+    }
+    T* slot = (T*)a.cache_out + ((size_t)b * sh.max_slots + j) * sh.D;
+    float* open = (u0 + nu == Tn && a.open_slot_out) ? a.open_slot_out + (size_t)b * sh.D : nullptr;
+    PT* Pj = P + ((size_t)b * Tn + u0) * sh.D;
+    for (int k0 = lane * 8; k0 < sh.d_c; k0 += 256) {
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int uo = 0; uo < 8; ++uo) {
+            if (uo >= nu) continue;
+            float x[8];
+            load8<T>(c + (size_t)uo * sh.d_c + k0, x);
+#pragma unroll
+            for (int v = 0; v < 8; ++v) acc[v] = fmaf(wv[uo], x[v], acc[v]);
+            store8<PT>(Pj + (size_t)uo * sh.D + k0, acc);
+        }
+        store8<T>(slot + k0, acc);
+        if (open) store8<float>(open + k0, acc);
+    }
+    for (int k = lane; k < sh.d_r / 2; k += 32) {
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+        for (int uo = 0; uo < 8; ++uo) {
+            if (uo >= nu) continue;
+            float sn, cs;
+            pair_sincos_f(u0 + uo, rope_freq[k], &sn, &cs);
+            const float x0 = to_f<T>(kr[(size_t)uo * sh.d_r + 2 * k]);
+            const float x1 = to_f<T>(kr[(size_t)uo * sh.d_r + 2 * k + 1]);
+            a0 = fmaf(wv[uo], x0 * cs - x1 * sn, a0);
+            a1 = fmaf(wv[uo], x0 * sn + x1 * cs, a1);
+            PT* pr = Pj + (size_t)uo * sh.D + sh.d_c;
+            pr[2 * k] = from_f<PT>(a0);
+            pr[2 * k + 1] = from_f<PT>(a1);
+        }
+        slot[sh.d_c + 2 * k] = from_f<T>(a0);
+        slot[sh.d_c + 2 * k + 1] = from_f<T>(a1);
+        if (open) {
+            open[sh.d_c + 2 * k] = a0;
+            open[sh.d_c + 2 * k + 1] = a1;
+        }
+    }
 }
 
 }  // namespace mtla

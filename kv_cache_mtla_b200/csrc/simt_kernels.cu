@@ -143,57 +143,6 @@ __global__ void __launch_bounds__(256) k_decode_combine(DecodeArgs a, int chunk,
 
 // ----------------------------------------------------------------- prefill
 
-// Block-prefix scan: block (j, b) computes the partial slots P_u of the
-// tokens u of slot j, the finished/last slot of the cache, and the open slot.
-template <typename T>
-__global__ void __launch_bounds__(128) k_prefill_scan(PrefillArgs a, float* P) {
-    const Shape sh = a.sh;
-    const int j = blockIdx.x, b = blockIdx.y;
-    const int Tn = a.T;
-    const int u0 = j * sh.s, u1 = min(u0 + sh.s, Tn);
-    __shared__ float red[32];
-    __shared__ float wsm[8];
-    const T* c = (const T*)a.c + (size_t)b * Tn * sh.d_c;
-    const T* kr = (const T*)a.kr + (size_t)b * Tn * sh.d_r;
-    for (int u = u0; u < u1; ++u) {
-        const float w = gate_weight<T>(sh, u, c + (size_t)u * sh.d_c, a.gate_w, a.gate_b,
-                                       a.gate_in ? a.gate_in + (size_t)b * Tn + u : nullptr, red);
-        if (threadIdx.x == 0) wsm[u - u0] = w;
-    }
-    __syncthreads();
-    T* slot = (T*)a.cache_out + ((size_t)b * sh.max_slots + j) * sh.D;
-    float* open = (u1 == Tn && a.open_slot_out) ? a.open_slot_out + (size_t)b * sh.D : nullptr;
-    for (int k = threadIdx.x; k < sh.d_c; k += blockDim.x) {
-        float acc = 0.f;
-        for (int u = u0; u < u1; ++u) {
-            acc += wsm[u - u0] * to_f<T>(c[(size_t)u * sh.d_c + k]);
-            P[((size_t)b * Tn + u) * sh.D + k] = acc;
-        }
-        slot[k] = from_f<T>(acc);
-        if (open) open[k] = acc;
-    }
-    for (int k = threadIdx.x; k < sh.d_r / 2; k += blockDim.x) {
-        float a0 = 0.f, a1 = 0.f;
-        for (int u = u0; u < u1; ++u) {
-            float sn, cs;
-            pair_sincos(u, k, sh.d_r, sh.log2_rope_base, &sn, &cs);
-            const float x0 = to_f<T>(kr[(size_t)u * sh.d_r + 2 * k]);
-            const float x1 = to_f<T>(kr[(size_t)u * sh.d_r + 2 * k + 1]);
-            a0 += wsm[u - u0] * (x0 * cs - x1 * sn);
-            a1 += wsm[u - u0] * (x0 * sn + x1 * cs);
-            float* pr = P + ((size_t)b * Tn + u) * sh.D + sh.d_c;
-            pr[2 * k] = a0;
-            pr[2 * k + 1] = a1;
-        }
-        slot[sh.d_c + 2 * k] = from_f<T>(a0);
-        slot[sh.d_c + 2 * k + 1] = from_f<T>(a1);
-        if (open) {
-            open[sh.d_c + 2 * k] = a0;
-            open[sh.d_c + 2 * k + 1] = a1;
-        }
-    }
-}
-
 // Masked attention: one warp per (t, h) row; keys are the finished slots
 // j < floor(t/s) (rounded cache) plus the own partial slot P_t (rounded).
 template <typename T>
@@ -291,7 +240,7 @@ cudaError_t prefill_impl(const PrefillArgs& a, cudaStream_t st, uint64_t* launch
     float* P = (float*)ws;
     float* qt = (float*)(ws + align256((size_t)sh.B * a.T * sh.D * sizeof(float)));
     const int n_slots = (a.T + sh.s - 1) / sh.s;
-    k_prefill_scan<T><<<dim3(n_slots, sh.B), 128, 0, st>>>(a, P);
+    k_prefill_scan<T, float><<<dim3((n_slots + 7) / 8, sh.B), 256, 0, st>>>(a, P);
     k_prefill_absorb<T><<<dim3(sh.B * a.T, sh.H), 128, 0, st>>>(sh, (const T*)a.q_c, (const T*)a.q_r,
                                                                  (const T*)a.w_uk, a.T, qt);
     const int64_t rows = (int64_t)a.T * sh.H;

@@ -7,8 +7,10 @@
 // Per-token decode work is O(N/s) slot reads (Sec. 6.1), so this kernel is a
 // streaming read of the bf16 latent cache.
 //
-// Launches per step:
-//   k_decode_prep   gate, RoPE, in-place slot update; absorbed queries (fp32)
+// Launches per step (the last two with programmatic dependent launch, so their
+// prologues overlap the previous kernel's tail):
+//   k_dec_prep_tc   gate, RoPE, in-place slot update; absorbed queries written
+//                   as a bf16 image already in the attention's SW128 layout
 //   k_dec_attn_sh   split-K attention over slot tiles (tcgen05 + TMEM + TMA)
 //   k_dec_combine   merge of the split partials and W_UV
 //
@@ -26,6 +28,7 @@
 
 #include <cstdio>
 #include <mutex>
+#include <utility>
 
 #include "common.cuh"
 #include "mtla_internal.h"
@@ -42,6 +45,9 @@ constexpr int kTileSlots = 128;
 constexpr int kThreads = 128;
 constexpr int kMaxGrid = 160;  // >= SMs of any sm_100 part; sizes the partial buffer
 constexpr int kMaxB = 2048;
+// S^T is accumulated in 4 independent TMEM accumulators (K-steps round robin)
+// so that the chain of dependent MMAs is a quarter as long; the softmax adds them.
+constexpr int kSAcc = 4;
 
 struct DecTC {
     int B, H, D, d_c, s, max_slots;
@@ -50,8 +56,9 @@ struct DecTC {
     int G;           // grid size
     float scale_log2;
     const int32_t* pos;
-    const float* qt;  // [B, H, D]
-    float* part;      // [(kMaxGrid + B), H, d_c + 2]
+    const uint8_t* qimg;  // [B] x n_chunks x [NH rows x 128 B]: q~ in bf16, SW128, zero padded
+    uint32_t qimg_bytes;  // per sequence
+    float* part;          // [(kMaxGrid + B), H, d_c + 2]
     int* status;
 };
 
@@ -72,6 +79,7 @@ struct Misc {
     uint64_t full[2];
     uint64_t bar_s;
     uint64_t bar_o;
+    uint64_t bar_q;
     uint32_t tmem_base;
     int fail;
     int rescale;
@@ -80,6 +88,80 @@ struct Misc {
     float m_run[NH];
     float fac[NH];
 };
+
+// Decode prep for the tensor-core path. grid (B, H + 1), 128 threads.
+// Block (b, h < H): absorbed query of head h, q~ = [W_UK[h]^T qC ; RoPE_t(qR)],
+// rounded to bf16 into row h of sequence b's query image (64-column SW128
+// chunks of NH rows, zero beyond D). Block (b, H): gate, RoPE and in-place
+// update of the open slot (MTLA Method (1)), and zero rows H..NH-1 of the image.
+__global__ void __launch_bounds__(128) k_dec_prep_tc(DecodeArgs a, uint8_t* qimg, int n_chunks, int NH) {
+    pdl_launch_dependents();   // the attention kernel may start its prologue now
+    const Shape& sh = a.sh;
+    const int b = blockIdx.x, h = blockIdx.y;
+    const uint32_t img_bytes = (uint32_t)n_chunks * NH * 128;
+    uint8_t* img = qimg + (size_t)b * img_bytes;
+    if (h == sh.H) {
+        decode_update_body<bf16>(a, b);
+        for (int e = threadIdx.x; e < n_chunks * (NH - sh.H) * 8; e += blockDim.x) {
+            const int c = e / ((NH - sh.H) * 8), rr = e % ((NH - sh.H) * 8);
+            *(uint4*)(img + (size_t)c * NH * 128 + (size_t)(sh.H + rr / 8) * 128 + (rr % 8) * 16) =
+                make_uint4(0, 0, 0, 0);
+        }
+        return;
+    }
+    const int64_t t = a.pos[b];
+    if (t < 0 || t >= (int64_t)sh.max_slots * sh.s) return;
+    __shared__ float q[256];
+    __shared__ float part_sum[8][512];     // [i-group][latent column]
+    const size_t rh = (size_t)b * sh.H + h;
+    const bf16* qc = (const bf16*)a.q_c + rh * sh.d_h;
+    for (int i = threadIdx.x; i < sh.d_h; i += blockDim.x) q[i] = __bfloat162float(qc[i]);
+    __syncthreads();
+    // thread (ig, jg): 8 latent columns [8 jg, 8 jg + 8) over rows i of group ig;
+    // all of its 16-byte loads of W_UK are issued before any product
+    const bf16* W = (const bf16*)a.w_uk + (size_t)h * sh.d_h * sh.d_c;
+    const int n_jg = sh.d_c / 8;
+    const int n_ig = max(1, min(8, (int)blockDim.x / n_jg));
+    const int rows_per = (sh.d_h + n_ig - 1) / n_ig;
+    for (int e = threadIdx.x; e < n_ig * n_jg; e += blockDim.x) {
+        const int ig = e / n_jg, jg = e % n_jg;
+        const int i0 = ig * rows_per, i1 = min(sh.d_h, i0 + rows_per);
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int ib = i0; ib < i1; ib += 16) {
+            uint4 raw[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u)
+                if (ib + u < i1) raw[u] = *(const uint4*)(W + (size_t)(ib + u) * sh.d_c + jg * 8);
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                if (ib + u < i1) {
+                    const bf16* wv = (const bf16*)&raw[u];
+                    const float qi = q[ib + u];
+#pragma unroll
+                    for (int v = 0; v < 8; ++v) acc[v] = fmaf(__bfloat162float(wv[v]), qi, acc[v]);
+                }
+            }
+        }
+#pragma unroll
+        for (int v = 0; v < 8; ++v) part_sum[ig][jg * 8 + v] = acc[v];
+    }
+    __syncthreads();
+    const bf16* qr = (const bf16*)a.q_r + rh * sh.d_r;
+    const int dpad = n_chunks * 64;
+    for (int j = threadIdx.x; j < dpad; j += blockDim.x) {
+        float v = 0.f;
+        if (j < sh.d_c) {
+            for (int ig = 0; ig < n_ig; ++ig) v += part_sum[ig][j];
+        } else if (j < sh.D) {
+            const int e = j - sh.d_c, k = e >> 1;
+            float sn, cs;
+            pair_sincos(t, k, sh.d_r, sh.log2_rope_base, &sn, &cs);
+            const float x0 = __bfloat162float(qr[2 * k]), x1 = __bfloat162float(qr[2 * k + 1]);
+            v = (e & 1) ? (x0 * sn + x1 * cs) : (x0 * cs - x1 * sn);
+        }
+        *(bf16*)(img + (size_t)(j >> 6) * NH * 128 + sw128_offset(h, j & 63)) = __float2bfloat16_rn(v);
+    }
+}
 
 template <int NH>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -123,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
     // ---- barriers and TMEM
-    const uint32_t tmem_cols_needed = (uint32_t)NH * (1 + p.lat_blocks);
+    const uint32_t tmem_cols_needed = (uint32_t)NH * (kSAcc + p.lat_blocks);
     uint32_t tmem_cols = 32;
     while (tmem_cols < tmem_cols_needed) tmem_cols <<= 1;
     if (tid == 0) {
@@ -131,10 +213,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&m.full[1], 1);
         mbar_init(&m.bar_s, 1);
         mbar_init(&m.bar_o, 1);
+        mbar_init(&m.bar_q, 1);
         m.fail = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmap);
     }
+    pdl_launch_dependents();
     if (warp == 0) {
         tmem_alloc(&m.tmem_base, tmem_cols);
         tmem_relinquish();
@@ -144,8 +228,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t tmem = m.tmem_base;
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    const uint32_t t_s = tmem;            // S^T: NH columns
-    const uint32_t t_o = tmem + NH;       // O^T: lat_blocks x NH columns
+    const uint32_t t_s = tmem;                // S^T: kSAcc partial sums of NH columns each
+    const uint32_t t_o = tmem + kSAcc * NH;   // O^T: lat_blocks x NH columns
 
     const int total = m.total;
     const int g = blockIdx.x;
@@ -173,6 +257,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t idesc_s = idesc_bf16_f32(128, NH, false, false);
     const uint32_t idesc_o = idesc_bf16_f32(128, NH, true, false);
 
+    // everything above only read pos; the cache row and q~ come from k_dec_prep_tc
+    pdl_wait();
     int loads_issued = 0;
     if (tid == 0) {
         for (int k = 0; k < 2 && gt0 + k < gt1; ++k) {
@@ -182,7 +268,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     float l_part[NH];
-    int seq_b = -1, seq_n = 0;
+    int seq_b = -1, seq_n = 0, q_phase = 0;
     bool first_o = true;
     bool failed = false;
     int it = 0;
@@ -191,17 +277,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         locate(gt, b, j);
         const int st = it & 1;
         if (b != seq_b) {
-            // new segment: this sequence's absorbed queries -> bf16, SW128, zero padded
+            // new segment: this sequence's query image (one bulk copy)
             seq_b = b;
             seq_n = seq_slots(p, b);
             first_o = true;
-            const float* q = p.qt + (size_t)b * p.H * p.D;
-            const int dpad = n_chunks * 64;
-            for (int e = tid; e < NH * dpad; e += kThreads) {
-                const int h = e / dpad, d = e - h * dpad;
-                const float v = (h < p.H && d < p.D) ? q[h * p.D + d] : 0.f;
-                *(bf16*)(q_s + (size_t)(d >> 6) * NH * 128 + sw128_offset(h, d & 63)) = __float2bfloat16_rn(v);
+            if (tid == 0) {
+                mbar_arrive_expect_tx(&m.bar_q, p.qimg_bytes);
+                bulk_load(q_s, p.qimg + (size_t)b * p.qimg_bytes, p.qimg_bytes, &m.bar_q);
             }
+            if (!mbar_wait(&m.bar_q, q_phase & 1)) m.fail = 1;
+            ++q_phase;
             if (tid < NH) m.m_run[tid] = -INFINITY;
 #pragma unroll
             for (int h = 0; h < NH; ++h) l_part[h] = 0.f;
@@ -236,9 +321,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t b0 = smem_u32(q_s);
             for (int c = 0; c < n_chunks; ++c)
                 for (int kk = 0; kk < 4; ++kk) {
+                    const int step = c * 4 + kk;
                     const uint64_t ad = sdesc_sw128(a0 + c * 16384 + kk * 32, 16, 1024);
                     const uint64_t bd = sdesc_sw128(b0 + c * NH * 128 + kk * 32, 16, 1024);
-                    umma_bf16(t_s, ad, bd, idesc_s, (c | kk) != 0);
+                    umma_bf16(t_s + (step % kSAcc) * NH, ad, bd, idesc_s, step >= kSAcc);
                 }
             umma_commit(&m.bar_s);
         }
@@ -246,19 +332,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         // (4) online softmax, thread = slot row
         float sv[NH];
-        tmem_ld16(t_s + lane_off, sv);
-        if (NH == 32) tmem_ld16(t_s + lane_off + 16, sv + 16);
-        tmem_wait_ld();
+        {
+            float part[kSAcc][NH];
+#pragma unroll
+            for (int q = 0; q < kSAcc; ++q) {
+                tmem_ld16(t_s + q * NH + lane_off, part[q]);
+                if (NH == 32) tmem_ld16(t_s + q * NH + lane_off + 16, part[q] + 16);
+            }
+            tmem_wait_ld();
+#pragma unroll
+            for (int h = 0; h < NH; ++h) sv[h] = (part[0][h] + part[1][h]) + (part[2][h] + part[3][h]);
+        }
         const bool row_ok = tid < valid;
 #pragma unroll
         for (int h = 0; h < NH; ++h) sv[h] = row_ok ? sv[h] * p.scale_log2 : -INFINITY;
 #pragma unroll
         for (int h = 0; h < NH; ++h) {
-            const float mx = warp_max(sv[h]);
-            if (lane == 0) m.red[warp][h] = mx;
+            if (h < p.H) {
+                const float mx = warp_max(sv[h]);
+                if (lane == 0) m.red[warp][h] = mx;
+            }
         }
         __syncthreads();
-        if (tid < NH) {
+        if (tid < p.H) {
             const float tile_max = fmaxf(fmaxf(m.red[0][tid], m.red[1][tid]), fmaxf(m.red[2][tid], m.red[3][tid]));
             const float old = m.m_run[tid];
             const float nm = fmaxf(old, tile_max);
@@ -271,8 +367,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         float pv[NH];
 #pragma unroll
         for (int h = 0; h < NH; ++h) {
-            pv[h] = (h < p.H) ? exp2f(sv[h] - m.m_run[h]) : 0.f;
-            l_part[h] = l_part[h] * m.fac[h] + pv[h];
+            pv[h] = 0.f;
+            if (h < p.H) {
+                pv[h] = exp2f(sv[h] - m.m_run[h]);
+                l_part[h] = l_part[h] * m.fac[h] + pv[h];
+            }
         }
         // P^T into shared memory as the K-major B operand [NH x 128 slots]
         {
@@ -320,8 +419,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_after();
 #pragma unroll
             for (int h = 0; h < NH; ++h) {
-                const float sum = warp_sum(l_part[h]);
-                if (lane == 0) m.red[warp][h] = sum;
+                if (h < p.H) {
+                    const float sum = warp_sum(l_part[h]);
+                    if (lane == 0) m.red[warp][h] = sum;
+                }
             }
             __syncthreads();
             if (m.fail) { failed = true; break; }
@@ -362,16 +463,24 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // Merge the partials of (b, h) and apply W_UV. grid (H, B), 256 threads.
+// W_UV[h] is staged in shared memory before the wait for the attention kernel;
+// after it, every partial value this block needs is read in one round.
 __global__ void __launch_bounds__(256) k_dec_combine(DecodeArgs a, DecTC p) {
     const int h = blockIdx.x, b = blockIdx.y;
     const Shape& sh = a.sh;
     if (seq_tiles(p, b) == 0) return;
     __shared__ float red[32];
-    __shared__ float wts[kMaxGrid];
     __shared__ int idx[kMaxGrid];
     __shared__ int n_part;
-    __shared__ float inv_l;
     __shared__ float olat[512];
+    extern __shared__ uint8_t dyn[];
+    bf16* Ws = (bf16*)dyn;                            // W_UV[h] [d_h x d_c]
+    {
+        const uint4* src = (const uint4*)((const bf16*)a.w_uv + (size_t)h * sh.d_h * sh.d_c);
+        uint4* dst = (uint4*)Ws;
+        const int n16 = sh.d_h * sh.d_c / 8;
+        for (int e = threadIdx.x; e < n16; e += blockDim.x) dst[e] = src[e];
+    }
     // this sequence's tile range and the total
     int before = 0, all = 0;
     for (int bb = threadIdx.x; bb < p.B; bb += blockDim.x) {
@@ -383,70 +492,71 @@ __global__ void __launch_bounds__(256) k_dec_combine(DecodeArgs a, DecTC p) {
     const int total = (int)block_sum((float)all, red);
     const int E_b = S_b + seq_tiles(p, b);
     if (threadIdx.x == 0) {
+        // CTA g covers tiles [lo(g), lo(g+1)) with lo(g) = floor(g*total/G). The
+        // CTAs touching [S_b, E_b) are g_first..g_last, the largest g with
+        // lo(g) <= S_b and lo(g) <= E_b - 1: g = ceil((x+1)*G/total) - 1 for x.
+        const int64_t G = p.G, tot = total;
+        const int g_first = (int)(((int64_t)(S_b + 1) * G + tot - 1) / tot) - 1;
+        const int g_last = (int)(((int64_t)E_b * G + tot - 1) / tot) - 1;
         int n = 0;
-        for (int g = 0; g < p.G; ++g) {
-            const int lo = (int)(((int64_t)g * total) / p.G);
-            const int hi = (int)(((int64_t)(g + 1) * total) / p.G);
-            if (hi > lo && lo < E_b && hi > S_b) idx[n++] = g + b;
+        int64_t lo = ((int64_t)g_first * tot) / G;
+        for (int g = g_first; g <= g_last; ++g) {
+            const int64_t hi = ((int64_t)(g + 1) * tot) / G;
+            if (hi > lo) idx[n++] = g + b;
+            lo = hi;
         }
         n_part = n;
-        const size_t stride = (size_t)p.H * (p.d_c + 2);
-        float M = -INFINITY;
-        for (int k = 0; k < n; ++k) M = fmaxf(M, p.part[idx[k] * stride + (size_t)h * (p.d_c + 2) + p.d_c]);
-        float L = 0.f;
-        for (int k = 0; k < n; ++k) {
-            const float* e = p.part + idx[k] * stride + (size_t)h * (p.d_c + 2);
-            const float w = exp2f(e[p.d_c] - M);
-            wts[k] = w;
-            L += w * e[p.d_c + 1];
-        }
-        inv_l = 1.f / L;
     }
     __syncthreads();
+    pdl_wait();   // the partials come from k_dec_attn_sh
+    const int n = n_part;
     const size_t stride = (size_t)p.H * (p.d_c + 2);
+    const size_t hoff = (size_t)h * (p.d_c + 2);
     for (int jj = threadIdx.x; jj < p.d_c; jj += blockDim.x) {
-        float acc = 0.f;
-        for (int k = 0; k < n_part; ++k) acc = fmaf(wts[k], p.part[idx[k] * stride + (size_t)h * (p.d_c + 2) + jj], acc);
-        olat[jj] = acc * inv_l;
+        // one round of loads: (m, l, o[jj]) of every partial
+        float mk[8], lk[8], ok[8];
+        float M = -INFINITY, L = 0.f, acc = 0.f;
+        for (int k0 = 0; k0 < n; k0 += 8) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                if (k0 + u < n) {
+                    const float* e = p.part + idx[k0 + u] * stride + hoff;
+                    mk[u] = e[p.d_c];
+                    lk[u] = e[p.d_c + 1];
+                    ok[u] = e[jj];
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                if (k0 + u < n) {
+                    const float Mn = fmaxf(M, mk[u]);
+                    const float c0 = exp2f(M - Mn), c1 = exp2f(mk[u] - Mn);
+                    L = L * c0 + lk[u] * c1;
+                    acc = acc * c0 + ok[u] * c1;
+                    M = Mn;
+                }
+            }
+        }
+        olat[jj] = acc / L;
     }
     __syncthreads();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const bf16* W = (const bf16*)a.w_uv + (size_t)h * sh.d_h * sh.d_c;
     bf16* out = (bf16*)a.out + ((size_t)b * sh.H + h) * sh.d_h;
     for (int i = warp; i < sh.d_h; i += 8) {
         float acc = 0.f;
-        for (int jj = lane; jj < sh.d_c; jj += 32) acc = fmaf(__bfloat162float(W[(size_t)i * sh.d_c + jj]), olat[jj], acc);
+        const bf16* Wi = Ws + (size_t)i * sh.d_c;
+        for (int c0 = lane * 8; c0 < sh.d_c; c0 += 256) {
+            const uint4 raw = *(const uint4*)(Wi + c0);
+            const bf16* wv = (const bf16*)&raw;
+#pragma unroll
+            for (int v = 0; v < 8; ++v) acc = fmaf(__bfloat162float(wv[v]), olat[c0 + v], acc);
+        }
         acc = warp_sum(acc);
         if (lane == 0) out[i] = __float2bfloat16_rn(acc);
     }
 }
 
 // ---------------------------------------------------------------- host side
-
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = (PFN_cuTensorMapEncodeTiled_v12000)ptr;
-    });
-    return fn;
-}
-
-int sm_count() {
-    static int cached[64] = {0};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-    if (!cached[dev]) {
-        int n = 0;
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-        cached[dev] = n;
-    }
-    return cached[dev];
-}
 
 int n_chunks_of(const Shape& sh) { return (sh.D + 63) / 64; }
 
@@ -480,6 +590,25 @@ cudaError_t ensure_smem(K kernel, size_t smem, size_t* done) {
     return e;
 }
 
+// Launch with programmatic stream serialization: the kernel may start while
+// the previous kernel in the stream finishes; it waits (griddepcontrol.wait)
+// before it reads that kernel's results.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 template <int NH>
 cudaError_t launch_attn(const CUtensorMap& map, const DecTC& p, size_t smem, cudaStream_t st) {
     static size_t done[64] = {0};
@@ -488,29 +617,59 @@ cudaError_t launch_attn(const CUtensorMap& map, const DecTC& p, size_t smem, cud
     if (dev < 0 || dev >= 64) dev = 0;
     cudaError_t e = ensure_smem(k_dec_attn_sh<NH>, smem, &done[dev]);
     if (e != cudaSuccess) return note_error("cudaFuncSetAttribute(k_dec_attn_sh)", e);
-    k_dec_attn_sh<NH><<<p.G, kThreads, smem, st>>>(map, p);
-    return note_error("k_dec_attn_sh launch", cudaGetLastError());
+    return note_error("k_dec_attn_sh launch", launch_pdl(k_dec_attn_sh<NH>, dim3(p.G), dim3(kThreads), smem, st, map, p));
 }
 
 }  // namespace
 
+void* tensor_map_encoder() {
+    static void* fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = ptr;
+    });
+    return fn;
+}
+
+int sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!cached[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
 bool tc_decode_supported(const Shape& sh) {
     return sh.H <= 32 && sh.d_c % 128 == 0 && n_chunks_of(sh) <= 6 && sh.B <= kMaxB &&
+           (size_t)sh.d_h * sh.d_c * sizeof(bf16) <= 160 * 1024 &&
            attn_smem_bytes(sh, sh.H <= 16 ? 16 : 32) <= 232448 - 1024;
 }
 
+static uint32_t qimg_bytes(const Shape& sh) {
+    return (uint32_t)n_chunks_of(sh) * (sh.H <= 16 ? 16 : 32) * 128;
+}
+
 size_t tc_decode_workspace(const Shape& sh) {
-    return align256((size_t)sh.B * sh.H * sh.D * sizeof(float)) +
+    return align256((size_t)sh.B * qimg_bytes(sh)) +
            align256((size_t)(kMaxGrid + sh.B) * sh.H * (sh.d_c + 2) * sizeof(float));
 }
 
 cudaError_t tc_decode(const DecodeArgs& a, cudaStream_t st, uint64_t* launches) {
     const Shape& sh = a.sh;
     char* ws = (char*)a.workspace;
-    float* qt = (float*)ws;
-    float* part = (float*)(ws + align256((size_t)sh.B * sh.H * sh.D * sizeof(float)));
+    uint8_t* qimg = (uint8_t*)ws;
+    float* part = (float*)(ws + align256((size_t)sh.B * qimg_bytes(sh)));
+    const int NH = sh.H <= 16 ? 16 : 32;
 
-    PFN_cuTensorMapEncodeTiled_v12000 encode = encode_fn();
+    auto encode = (PFN_cuTensorMapEncodeTiled_v12000)tensor_map_encoder();
     if (!encode) return note_error("cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", cudaErrorNotSupported);
     CUtensorMap map;
     cuuint64_t dims[3] = {(cuuint64_t)sh.D, (cuuint64_t)sh.max_slots, (cuuint64_t)sh.B};
@@ -539,22 +698,46 @@ cudaError_t tc_decode(const DecodeArgs& a, cudaStream_t st, uint64_t* launches) 
     p.G = (int)std::min<int64_t>(std::min(sm_count(), kMaxGrid), max_tiles);
     p.scale_log2 = sh.scale * 1.4426950408889634f;
     p.pos = a.pos;
-    p.qt = qt;
+    p.qimg = qimg;
+    p.qimg_bytes = qimg_bytes(sh);
     p.part = part;
     p.status = a.status;
 
-    k_decode_prep<bf16><<<dim3(sh.B, sh.H + 1), 128, 0, st>>>(a, qt);
+    {
+        // keep the SMs in the max-shared-memory configuration across the
+        // three kernels of a step (no carve-out switch between them)
+        static bool carve[64] = {false};
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (dev >= 0 && dev < 64 && !carve[dev]) {
+            cudaFuncSetAttribute(k_dec_prep_tc, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
+            cudaFuncSetAttribute(k_dec_combine, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 cudaSharedmemCarveoutMaxShared);
+            cudaGetLastError();
+            carve[dev] = true;
+        }
+    }
+    k_dec_prep_tc<<<dim3(sh.B, sh.H + 1), 128, 0, st>>>(a, qimg, p.n_chunks, NH);
     cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return note_error("k_decode_prep launch", e);
-    const int NH = sh.H <= 16 ? 16 : 32;
+    if (e != cudaSuccess) return note_error("k_dec_prep_tc launch", e);
     const size_t smem = attn_smem_bytes(sh, NH);
     profile_begin(st);
     e = NH == 16 ? launch_attn<16>(map, p, smem, st) : launch_attn<32>(map, p, smem, st);
     profile_end(st);
     if (e != cudaSuccess) return e;
-    k_dec_combine<<<dim3(sh.H, sh.B), 256, 0, st>>>(a, p);
+    const size_t comb_smem = (size_t)sh.d_h * sh.d_c * sizeof(bf16);
+    {
+        static size_t done[64] = {0};
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (dev < 0 || dev >= 64) dev = 0;
+        e = ensure_smem(k_dec_combine, comb_smem, &done[dev]);
+        if (e != cudaSuccess) return note_error("cudaFuncSetAttribute(k_dec_combine)", e);
+    }
+    e = launch_pdl(k_dec_combine, dim3(sh.H, sh.B), dim3(256), comb_smem, st, a, p);
     *launches += 3;
-    return note_error("k_dec_combine launch", cudaGetLastError());
+    return note_error("k_dec_combine launch", e);
 }
 
 }  // namespace mtla

@@ -1,0 +1,496 @@
+// tc_prefill.cu -- bf16 parallel (training-form) forward on the tensor cores.
+//
+// "Multi-head Temporal Latent Attention", Method (2)-(3), Sec. 4.2-4.3: with
+// the stride-aware causal mask, position t attends every finished slot
+// j < floor(t/s) plus its own block's partial slot
+//   P_t = sum_{u = s*floor(t/s)}^{t} w_u [c_u ; RoPE_u(k_u)],
+// which reproduces incremental decoding; W_UK is folded into the query and
+// W_UV applied to the weighted latent (absorption kept from MLA).
+//
+// Launches:
+//   k_prefill_scan<bf16, bf16>  gates, partial slots P (bf16, scratch),
+//                               finished slots (cache_out), open slot
+//   k_prefill_tc                one CTA per (query tile of 128 positions,
+//                               sequence, head), heaviest tiles first:
+//     absorption   q~ = qC . W_UK[h]          tcgen05 M=128 N=d_c K=d_h
+//     own partial  2 tiles of 64 rows of P     diagonal mask
+//     finished     64-slot tiles of cache_out  staircase mask on the last
+//                  S = q~ . K^T (M=128 N=64 K=D), online softmax (thread per
+//                  row, exp2, rescale only when a row max grows by > 2^8),
+//                  O += P . V (M=128 N=d_c K=64, V = the same smem tile)
+//     epilogue     out = (O / l) . W_UV[h]^T   tcgen05 M=128 N=d_h K=d_c
+// Warp roles: warp 0 TMA, warp 1 MMA issue and TMEM, warps 2-5 softmax. S is
+// double-buffered in TMEM so S(k+1) runs on the tensor cores while the
+// softmax of tile k runs; keys stream through a 3-stage TMA ring.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdio>
+
+#include "common.cuh"
+#include "mtla_internal.h"
+#include "prep.cuh"
+#include "tc_common.cuh"
+
+namespace mtla {
+
+namespace {
+
+using namespace tc;
+
+constexpr int kQ = 128;         // query positions per CTA
+constexpr int kKT = 64;         // keys per tile
+constexpr int kStages = 3;
+constexpr int kThreads = 192;   // 6 warps
+constexpr float kRescaleLog2 = 8.f;
+
+struct PreTC {
+    int B, T, H, d_h, d_c, d_r, D, s;
+    int n_chunks;     // slot width rounded up to 64, in 64-column chunks
+    int n_qtiles;     // ceil(T / 128)
+    float scale_log2;
+    double log2_rope_base;
+    const bf16* q_r;  // [B, T, H, d_r]
+    bf16* out;        // [B, T, H, d_h]
+    int* status;
+};
+
+struct Bars {
+    uint64_t full[kStages], empty[kStages];
+    uint64_t abs_full, abs_done, q_ready;
+    uint64_t s_full[2], s_empty[2];
+    uint64_t p_full, o_done, fin_s, wuv_full, olat_ready, out_done;
+    uint32_t tmem_base;
+    volatile int fail;
+};
+
+struct Maps {
+    CUtensorMap qc;     // (d_h, H, T, B)   box (64, 1, 128, 1)
+    CUtensorMap wuk;    // (d_c, d_h, H)    box (64, d_h, 1)
+    CUtensorMap wuv;    // (d_c, d_h, H)    box (64, d_h, 1)
+    CUtensorMap slots;  // (D, n_slots, B)  box (64, 64, 1)
+    CUtensorMap part;   // (D, T, B)        box (64, 64, 1)
+};
+
+__device__ __forceinline__ bool waitb(uint64_t* bar, uint32_t parity, Bars& bs) {
+    if (bs.fail) return false;
+    if (mbar_wait(bar, parity)) return true;
+    bs.fail = 1;
+    return false;
+}
+
+// Store 32 fp32 values as bf16 into row `row`, columns [col, col+32) of a
+// K-major SW128 operand made of [rows x 64] chunks spaced chunk_bytes apart.
+__device__ __forceinline__ void st_row32_bf16(uint8_t* base, uint32_t chunk_bytes, int row, int col,
+                                              const float* v) {
+    uint8_t* chunk = base + (size_t)(col >> 6) * chunk_bytes;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        uint4 pk;
+        pk.x = pack_bf16x2(v[8 * u + 0], v[8 * u + 1]);
+        pk.y = pack_bf16x2(v[8 * u + 2], v[8 * u + 3]);
+        pk.z = pack_bf16x2(v[8 * u + 4], v[8 * u + 5]);
+        pk.w = pack_bf16x2(v[8 * u + 6], v[8 * u + 7]);
+        *(uint4*)(chunk + sw128_offset(row, (col & 63) + 8 * u)) = pk;
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constant__ Maps maps, const PreTC p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    const int n_chunks = p.n_chunks;
+    const uint32_t chunk_k = kKT * 128;                                  // one 64-row chunk of a key tile
+    const uint32_t stage_bytes = (uint32_t)n_chunks * chunk_k;
+    uint8_t* ring = smem;                                                // kStages key tiles
+    uint8_t* q_s = ring + kStages * stage_bytes;                         // n_chunks x [128 x 128 B]
+    uint8_t* p_s = q_s + (size_t)n_chunks * kQ * 128;                    // [128 x 128 B]
+    Bars& bs = *(Bars*)(p_s + kQ * 128);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int per_qt = p.B * p.H;
+    const int qt = p.n_qtiles - 1 - (int)(blockIdx.x / per_qt);
+    const int rem = (int)(blockIdx.x % per_qt);
+    const int b = rem / p.H, h = rem % p.H;
+    const int p0 = qt * kQ;
+    const int last = min(p0 + kQ - 1, p.T - 1);
+    const int nft = (last / p.s + kKT - 1) / kKT;                        // finished-slot tiles
+    const int n_tiles = 2 + nft;
+    const int dc_chunks = p.d_c / 64;
+    const uint32_t wchunk = (uint32_t)p.d_h * 128;                       // one 64-column chunk of W
+
+    if (tid == 0) {
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&bs.full[i], 1);
+            mbar_init(&bs.empty[i], 1);
+        }
+        mbar_init(&bs.abs_full, 1);
+        mbar_init(&bs.abs_done, 1);
+        mbar_init(&bs.q_ready, 4);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bs.s_full[i], 1);
+            mbar_init(&bs.s_empty[i], 4);
+        }
+        mbar_init(&bs.p_full, 4);
+        mbar_init(&bs.o_done, 1);
+        mbar_init(&bs.fin_s, 1);
+        mbar_init(&bs.wuv_full, 1);
+        mbar_init(&bs.olat_ready, 4);
+        mbar_init(&bs.out_done, 1);
+        bs.fail = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&bs.tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bs.tmem_base;
+    const uint32_t t_s0 = tmem;            // S buffers: columns [0, 64) and [64, 128)
+    const uint32_t t_o = tmem + 128;       // q~, then O: columns [128, 128 + d_c)
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            tma_prefetch_desc(&maps.qc);
+            tma_prefetch_desc(&maps.slots);
+            tma_prefetch_desc(&maps.part);
+            mbar_arrive_expect_tx(&bs.abs_full, kQ * 128 + dc_chunks * wchunk);
+            tma_load_4d(p_s, &maps.qc, &bs.abs_full, 0, h, p0, b);
+            for (int n = 0; n < dc_chunks; ++n) tma_load_3d(q_s + n * wchunk, &maps.wuk, &bs.abs_full, n * 64, 0, h);
+            for (int k = 0; k < n_tiles; ++k) {
+                const int st = k % kStages;
+                if (k >= kStages && !waitb(&bs.empty[st], ((k / kStages) - 1) & 1, bs)) break;
+                mbar_arrive_expect_tx(&bs.full[st], stage_bytes);
+                uint8_t* dst = ring + st * stage_bytes;
+                if (k < 2) {
+                    for (int c = 0; c < n_chunks; ++c)
+                        tma_load_3d(dst + c * chunk_k, &maps.part, &bs.full[st], c * 64, p0 + kKT * k, b);
+                } else {
+                    for (int c = 0; c < n_chunks; ++c)
+                        tma_load_3d(dst + c * chunk_k, &maps.slots, &bs.full[st], c * 64, kKT * (k - 2), b);
+                }
+            }
+            if (waitb(&bs.fin_s, 0, bs)) {
+                mbar_arrive_expect_tx(&bs.wuv_full, dc_chunks * wchunk);
+                for (int n = 0; n < dc_chunks; ++n)
+                    tma_load_3d(q_s + n * wchunk, &maps.wuv, &bs.wuv_full, n * 64, 0, h);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issue
+        if (lane == 0) {
+            const uint32_t id_abs = idesc_bf16_f32(128, p.d_c, false, true);
+            const uint32_t id_s = idesc_bf16_f32(128, kKT, false, false);
+            const uint32_t id_o = idesc_bf16_f32(128, p.d_c, false, true);
+            const uint32_t id_out = idesc_bf16_f32(128, p.d_h, false, false);
+            const uint32_t ring_a = smem_u32(ring), q_a = smem_u32(q_s), p_a = smem_u32(p_s);
+            bool ok = waitb(&bs.abs_full, 0, bs);
+            if (ok) {
+                tc_fence_after();
+                // q~ = qC . W_UK[h]: A = qC [128 x d_h] K-major, B = W_UK[h] [d_h x d_c] MN-major
+                for (int kk = 0; kk < p.d_h / 16; ++kk)
+                    umma_bf16(t_o, sdesc_sw128(p_a + kk * 32, 16, 1024),
+                              sdesc_sw128(q_a + kk * 2048, wchunk, 1024), id_abs, kk > 0);
+                umma_commit(&bs.abs_done);
+                ok = waitb(&bs.q_ready, 0, bs);
+            }
+            auto issue_s = [&](int k) -> bool {
+                const int st = k % kStages;
+                if (!waitb(&bs.full[st], (k / kStages) & 1, bs)) return false;
+                if (k >= 2 && !waitb(&bs.s_empty[k & 1], ((k - 2) >> 1) & 1, bs)) return false;
+                tc_fence_after();
+                const uint32_t kb = ring_a + st * stage_bytes;
+                for (int c = 0; c < n_chunks; ++c)
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_bf16(t_s0 + (k & 1) * 64, sdesc_sw128(q_a + c * kQ * 128 + kk * 32, 16, 1024),
+                                  sdesc_sw128(kb + c * chunk_k + kk * 32, 16, 1024), id_s, (c | kk) != 0);
+                umma_commit(&bs.s_full[k & 1]);
+                return true;
+            };
+            if (ok) ok = issue_s(0);
+            for (int k = 0; ok && k < n_tiles; ++k) {
+                if (k + 1 < n_tiles) {
+                    if (!issue_s(k + 1)) break;
+                } else {
+                    umma_commit(&bs.fin_s);
+                }
+                if (!waitb(&bs.p_full, k & 1, bs)) break;
+                tc_fence_after();
+                const uint32_t kb = ring_a + (k % kStages) * stage_bytes;
+                // O += P . V: A = P [128 x 64] K-major, B = V = key tile latent [64 x d_c] MN-major
+                for (int kk = 0; kk < kKT / 16; ++kk)
+                    umma_bf16(t_o, sdesc_sw128(p_a + kk * 32, 16, 1024),
+                              sdesc_sw128(kb + kk * 2048, chunk_k, 1024), id_o, (k > 0 || kk > 0) ? 1u : 0u);
+                umma_commit(&bs.empty[k % kStages]);
+                umma_commit(&bs.o_done);
+            }
+            if (!bs.fail && waitb(&bs.olat_ready, 0, bs) && waitb(&bs.wuv_full, 0, bs)) {
+                tc_fence_after();
+                // out = O_lat . W_UV[h]^T: A = O_lat [128 x d_c] K-major (in the ring),
+                // B = W_UV[h] [d_h x d_c] K-major (in q_s)
+                for (int kk = 0; kk < p.d_c / 16; ++kk) {
+                    const int c = kk >> 2;
+                    umma_bf16(t_s0, sdesc_sw128(ring_a + c * kQ * 128 + (kk & 3) * 32, 16, 1024),
+                              sdesc_sw128(q_a + c * wchunk + (kk & 3) * 32, 16, 1024), id_out, kk > 0);
+                }
+                umma_commit(&bs.out_done);
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ softmax warps
+        const int quarter = warp & 3;                 // TMEM lanes this warp may access
+        const int r = quarter * 32 + lane;            // query row of this thread
+        const int pos = p0 + r;
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        float v[32];
+        // q~ (latent part) from TMEM, RoPE part from qR, into the K-major Q tile
+        if (waitb(&bs.abs_done, 0, bs)) {
+            tc_fence_after();
+            for (int cc = 0; cc < p.d_c / 32; ++cc) {
+                tmem_ld32(t_o + cc * 32 + lane_off, v);
+                tmem_wait_ld();
+                st_row32_bf16(q_s, kQ * 128, r, cc * 32, v);
+            }
+            const int dpad = n_chunks * 64;
+            for (int c0 = p.d_c; c0 < dpad; c0 += 32) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = 0.f;
+                if (pos < p.T) {
+                    const bf16* qr = p.q_r + (((size_t)b * p.T + pos) * p.H + h) * p.d_r;
+#pragma unroll
+                    for (int i = 0; i < 32; i += 2) {
+                        const int e = c0 - p.d_c + i;        // rope element index
+                        if (e < p.d_r) {
+                            float sn, cs;
+                            pair_sincos(pos, e >> 1, p.d_r, p.log2_rope_base, &sn, &cs);
+                            const float x0 = __bfloat162float(qr[e]), x1 = __bfloat162float(qr[e + 1]);
+                            v[i] = x0 * cs - x1 * sn;
+                            v[i + 1] = x0 * sn + x1 * cs;
+                        }
+                    }
+                }
+                st_row32_bf16(q_s, kQ * 128, r, c0, v);
+            }
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bs.q_ready);
+
+        float m_ref = -INFINITY, l = 0.f;
+        const int fin_lim = pos / p.s;                // finished slots this row may see
+        for (int k = 0; k < n_tiles; ++k) {
+            if (!waitb(&bs.s_full[k & 1], (k >> 1) & 1, bs)) break;
+            tc_fence_after();
+            float sv[kKT];
+            tmem_ld32(t_s0 + (k & 1) * 64 + lane_off, sv);
+            tmem_ld32(t_s0 + (k & 1) * 64 + 32 + lane_off, sv + 32);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bs.s_empty[k & 1]);
+            float mt = -INFINITY;
+            if (k < 2) {
+#pragma unroll
+                for (int c = 0; c < kKT; ++c) {
+                    sv[c] = (c + kKT * k == r) ? sv[c] * p.scale_log2 : -INFINITY;
+                    mt = fmaxf(mt, sv[c]);
+                }
+            } else {
+                const int j0 = kKT * (k - 2);
+#pragma unroll
+                for (int c = 0; c < kKT; ++c) {
+                    sv[c] = (j0 + c < fin_lim) ? sv[c] * p.scale_log2 : -INFINITY;
+                    mt = fmaxf(mt, sv[c]);
+                }
+            }
+            float m_new = m_ref, fac = 1.f;
+            if (mt > m_ref + kRescaleLog2 || (m_ref == -INFINITY && mt > -INFINITY)) {
+                m_new = mt;
+                fac = (m_ref == -INFINITY) ? 0.f : exp2f(m_ref - mt);
+            }
+            const float mu = (m_new == -INFINITY) ? 0.f : m_new;
+            float rs = 0.f;
+#pragma unroll
+            for (int c = 0; c < kKT; ++c) {
+                sv[c] = exp2f(sv[c] - mu);
+                rs += sv[c];
+            }
+            l = l * fac + rs;
+            if (k >= 1) {
+                if (!waitb(&bs.o_done, (k - 1) & 1, bs)) break;
+                tc_fence_after();
+                if (__any_sync(0xffffffffu, fac != 1.f)) {
+                    for (int cc = 0; cc < p.d_c / 32; ++cc) {
+                        tmem_ld32(t_o + cc * 32 + lane_off, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) v[i] *= fac;
+                        tmem_st32(t_o + cc * 32 + lane_off, v);
+                    }
+                    tmem_wait_st();
+                }
+            }
+            st_row32_bf16(p_s, 0, r, 0, sv);
+            st_row32_bf16(p_s, 0, r, 32, sv + 32);
+            fence_proxy_async();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bs.p_full);
+            m_ref = m_new;
+        }
+        // epilogue: O / l -> bf16 K-major O_lat (in the ring), then out
+        if (waitb(&bs.o_done, (n_tiles - 1) & 1, bs)) {
+            tc_fence_after();
+            const float inv = 1.f / l;
+            for (int cc = 0; cc < p.d_c / 32; ++cc) {
+                tmem_ld32(t_o + cc * 32 + lane_off, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] *= inv;
+                st_row32_bf16(ring, kQ * 128, r, cc * 32, v);
+            }
+        }
+        fence_proxy_async();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bs.olat_ready);
+        if (waitb(&bs.out_done, 0, bs)) {
+            tc_fence_after();
+            for (int cc = 0; cc < p.d_h / 32; ++cc) {
+                tmem_ld32(t_s0 + cc * 32 + lane_off, v);
+                tmem_wait_ld();
+                if (pos < p.T) {
+                    bf16* o = p.out + (((size_t)b * p.T + pos) * p.H + h) * p.d_h + cc * 32;
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        uint4 pk;
+                        pk.x = pack_bf16x2(v[8 * u + 0], v[8 * u + 1]);
+                        pk.y = pack_bf16x2(v[8 * u + 2], v[8 * u + 3]);
+                        pk.z = pack_bf16x2(v[8 * u + 4], v[8 * u + 5]);
+                        pk.w = pack_bf16x2(v[8 * u + 6], v[8 * u + 7]);
+                        *(uint4*)(o + 8 * u) = pk;
+                    }
+                }
+            }
+        }
+    }
+    if (bs.fail && tid == 0) latch_status(p.status, kStatusTimeout);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+// ---------------------------------------------------------------- host side
+
+int n_chunks_of(const Shape& sh) { return (sh.D + 63) / 64; }
+
+size_t prefill_smem_bytes(const Shape& sh) {
+    const size_t nc = n_chunks_of(sh);
+    return 1024 + kStages * nc * kKT * 128 + nc * kQ * 128 + kQ * 128 + ((sizeof(Bars) + 15) & ~(size_t)15);
+}
+
+cudaError_t make_map(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* m, const void* base, int rank,
+                     const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box, const char* what) {
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        char buf[128];
+        snprintf(buf, sizeof(buf), "cuTensorMapEncodeTiled(%s) (CUresult %d)", what, (int)r);
+        return note_error(buf, cudaErrorInvalidValue);
+    }
+    return cudaSuccess;
+}
+
+}  // namespace
+
+bool tc_prefill_supported(const Shape& sh) {
+    return sh.d_h == 64 && sh.d_c % 64 == 0 && sh.d_c <= 256 && n_chunks_of(sh) <= 5 &&
+           prefill_smem_bytes(sh) <= 232448 - 1024;
+}
+
+size_t tc_prefill_workspace(const Shape& sh, int T) {
+    return align256((size_t)sh.B * T * sh.D * sizeof(bf16));
+}
+
+cudaError_t tc_prefill(const PrefillArgs& a, cudaStream_t st, uint64_t* launches) {
+    const Shape& sh = a.sh;
+    const int T = a.T;
+    bf16* P = (bf16*)a.workspace;
+    auto enc = (PFN_cuTensorMapEncodeTiled_v12000)tensor_map_encoder();
+    if (!enc) return note_error("cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", cudaErrorNotSupported);
+    Maps maps;
+    const cuuint64_t E = 2;
+    {
+        cuuint64_t d[4] = {(cuuint64_t)sh.d_h, (cuuint64_t)sh.H, (cuuint64_t)T, (cuuint64_t)sh.B};
+        cuuint64_t s[3] = {E * sh.d_h, E * sh.H * sh.d_h, E * T * sh.H * sh.d_h};
+        cuuint32_t bx[4] = {64, 1, kQ, 1};
+        cudaError_t e = make_map(enc, &maps.qc, a.q_c, 4, d, s, bx, "q_c");
+        if (e != cudaSuccess) return e;
+    }
+    {
+        cuuint64_t d[3] = {(cuuint64_t)sh.d_c, (cuuint64_t)sh.d_h, (cuuint64_t)sh.H};
+        cuuint64_t s[2] = {E * sh.d_c, E * sh.d_h * sh.d_c};
+        cuuint32_t bx[3] = {64, (cuuint32_t)sh.d_h, 1};
+        cudaError_t e = make_map(enc, &maps.wuk, a.w_uk, 3, d, s, bx, "w_uk");
+        if (e == cudaSuccess) e = make_map(enc, &maps.wuv, a.w_uv, 3, d, s, bx, "w_uv");
+        if (e != cudaSuccess) return e;
+    }
+    {
+        const int n_slots = (T + sh.s - 1) / sh.s;
+        cuuint64_t d[3] = {(cuuint64_t)sh.D, (cuuint64_t)n_slots, (cuuint64_t)sh.B};
+        cuuint64_t s[2] = {E * sh.D, E * sh.max_slots * sh.D};
+        cuuint32_t bx[3] = {64, kKT, 1};
+        cudaError_t e = make_map(enc, &maps.slots, a.cache_out, 3, d, s, bx, "cache_out");
+        if (e != cudaSuccess) return e;
+        cuuint64_t d2[3] = {(cuuint64_t)sh.D, (cuuint64_t)T, (cuuint64_t)sh.B};
+        cuuint64_t s2[2] = {E * sh.D, E * T * sh.D};
+        e = make_map(enc, &maps.part, P, 3, d2, s2, bx, "partials");
+        if (e != cudaSuccess) return e;
+    }
+    PreTC p;
+    p.B = sh.B;
+    p.T = T;
+    p.H = sh.H;
+    p.d_h = sh.d_h;
+    p.d_c = sh.d_c;
+    p.d_r = sh.d_r;
+    p.D = sh.D;
+    p.s = sh.s;
+    p.n_chunks = n_chunks_of(sh);
+    p.n_qtiles = (T + kQ - 1) / kQ;
+    p.scale_log2 = sh.scale * 1.4426950408889634f;
+    p.log2_rope_base = sh.log2_rope_base;
+    p.q_r = (const bf16*)a.q_r;
+    p.out = (bf16*)a.out;
+    p.status = a.status;
+
+    const int n_slots = (T + sh.s - 1) / sh.s;
+    k_prefill_scan<bf16, bf16><<<dim3((n_slots + 7) / 8, sh.B), 256, 0, st>>>(a, P);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return note_error("k_prefill_scan launch", e);
+
+    const size_t smem = prefill_smem_bytes(sh);
+    static size_t done[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) dev = 0;
+    if (done[dev] < smem) {
+        e = cudaFuncSetAttribute(k_prefill_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return note_error("cudaFuncSetAttribute(k_prefill_tc)", e);
+        done[dev] = smem;
+    }
+    const unsigned grid = (unsigned)p.n_qtiles * sh.B * sh.H;
+    profile_begin(st);
+    k_prefill_tc<<<grid, kThreads, smem, st>>>(maps, p);
+    profile_end(st);
+    *launches += 2;
+    return note_error("k_prefill_tc launch", cudaGetLastError());
+}
+
+}  // namespace mtla

@@ -295,3 +295,49 @@ def test_decode_skips_invalid_sequences_in_the_split_plan():
                              sub(toks["qr"][:, 0]), w["w_uk"], w["w_uv"], pos[good], cache_o, acc_o,
                              w["gate_w"], w["gate_b"])
     assert rel_err(out[good], ref["out"]) <= TOL["bf16"]
+
+
+# ----------------------------------------------------------------- tensor-core prefill edges
+
+@pytest.mark.parametrize("s", [1, 2, 3, 4])
+@pytest.mark.parametrize("T", [1, 63, 129, 300])
+def test_prefill_ragged_lengths(s, T):
+    """Speech-decode widths (d_h=64, d_c=256, d_R=32), lengths around the
+    128-position query tiles and 64-slot key tiles, every row against the
+    oracle; the cache and open slot too."""
+    wl = inputs.SPEECH_DECODE.with_(B=2, H=3, s=s)
+    w = inputs.weights(wl)
+    toks = inputs.tokens(wl, T)
+    ref = oracle.prefill(oracle_cfg(wl), toks["c"], toks["kr"], toks["qc"], toks["qr"], w["w_uk"],
+                         w["w_uv"], w["gate_w"], w["gate_b"])
+    n_slots = (T + s - 1) // s
+    pb = Problem(wl, max_slots=n_slots + 3, max_tokens=T, weights=w)
+    out = np64(pb.prefill(toks, T))
+    assert rel_err(out, ref["out"]) <= TOL["bf16"]
+    assert rel_err(np64(pb.buf.cache[:, :n_slots]), ref["cache"]) <= 4e-3
+    assert rel_err(np64(pb.buf.open_slot), ref["acc"]) <= 1e-5
+
+
+@pytest.mark.parametrize("s", [1, 2, 3, 4])
+def test_mask_set_bit_exact_speech_widths(s):
+    """The one-hot mask probe at the speech-decode widths, where both the
+    decode and the prefill run on the tensor-core kernels."""
+    wl = inputs.SPEECH_DECODE.with_(B=1, H=2, s=s, gate_mode=inputs.GATE_UNIT)
+    T = min(wl.s * wl.d_h, 150)
+    toks = inputs.one_hot_mask_probe(wl, T)
+    w = inputs.weights(wl)
+    eye = torch.zeros(wl.H, wl.d_h, wl.d_c)
+    eye[:, torch.arange(wl.d_h), torch.arange(wl.d_h)] = 1.0
+    w = dict(w, w_uv=eye, w_uk=torch.zeros_like(eye))
+    n_slots = (T + s - 1) // s
+    for mode in ("prefill", "decode"):
+        pb = Problem(wl, max_slots=n_slots, max_tokens=T, weights=w)
+        if mode == "prefill":
+            out = np64(pb.prefill(toks, T))[0]
+        else:
+            out = np.stack([np64(pb.decode(toks, t, [t]))[0] for t in range(T)])
+        for t in range(T):
+            for h in range(wl.H):
+                support = np.nonzero(out[t, h])[0].tolist()
+                assert support == list(range(t // s + 1)), (mode, t, h)
+                np.testing.assert_allclose(out[t, h, : t // s + 1], 1.0 / (t // s + 1), rtol=4e-3)
