@@ -253,6 +253,85 @@ def run_reference(args, ws, rank):
     print(json.dumps(line), flush=True)
 
 
+def run_kernel_workload(args, ws, rank):
+    """Kernel-level measurement of one of the other workloads (not the contract
+    line): decode attention GB/s against the measured HBM copy bandwidth, or
+    prefill TFLOP/s against the measured bf16 peak. L2 flushed before every
+    timed call; each call bracketed by CUDA events on the launching stream."""
+    hbm, tflops_peak, peak_kind = _peaks()
+    flush = torch.empty(64 * 1024 * 1024, dtype=torch.float32, device="cuda")
+    st = torch.cuda.current_stream()
+    name = args.workload
+    wl = inputs.WORKLOADS[name.split(":")[0]]
+    if ":" in name:
+        wl = wl.with_(s=int(name.split(":")[1]))
+    w = inputs.weights(wl)
+    lines = []
+    if name.startswith("prefill"):
+        T = wl.T
+        cfg = mtla.make_config(wl.B, wl.H, wl.d_h, wl.d_c, wl.d_r, wl.s, (T + wl.s - 1) // wl.s,
+                               dtype=wl.dtype, gate_mode=wl.gate_mode)
+        buf = mtla.Buffers.allocate(cfg, w, max_tokens=T)
+        tk = inputs.tokens(wl, T)
+        d = {k: (None if v is None else v.to("cuda", torch.bfloat16).contiguous()) for k, v in tk.items()}
+        out = torch.empty(wl.B, T, wl.H, wl.d_h, device="cuda", dtype=torch.bfloat16)
+
+        def call():
+            mtla.prefill(cfg, T, d["c"], d["kr"], d["qc"], d["qr"], buf.w_uk, buf.w_uv, buf.gate_w,
+                         buf.gate_b, None, out, buf.cache, buf.open_slot, buf.workspace)
+        pairs = sum(t // wl.s + 1 for t in range(T))
+        flops = 2 * pairs * (wl.D + wl.d_c) * wl.B * wl.H
+        unit_fn = lambda ms: flops / (ms / 1e3) / 1e12
+        unit, peak, bound = "TFLOP/s", tflops_peak, "tensor"
+    else:
+        N = wl.T
+        max_slots = (N + wl.s - 1) // wl.s
+        cfg = mtla.make_config(wl.B, wl.H, wl.d_h, wl.d_c, wl.d_r, wl.s, max_slots, dtype=wl.dtype,
+                               gate_mode=wl.gate_mode)
+        buf = mtla.Buffers.allocate(cfg, w)
+        c0 = inputs.synthetic_cache(wl, N - 1, max_slots)
+        buf.cache.copy_(c0["cache"].to(torch.bfloat16))
+        buf.open_slot.copy_(c0["acc"])
+        del c0
+        tk = inputs.tokens(wl, 1, stream=1)
+        d = {k: (None if v is None else v[:, 0].to("cuda", torch.bfloat16 if k != "gate_in" else torch.float32).contiguous())
+             for k, v in tk.items()}
+        pos = torch.full((wl.B,), N - 1, dtype=torch.int32, device="cuda")
+        out = torch.empty(wl.B, wl.H, wl.d_h, device="cuda", dtype=torch.bfloat16)
+        gw, gb = (buf.gate_w, buf.gate_b) if wl.gate_mode == inputs.GATE_COMPUTED else (None, None)
+
+        def call():
+            mtla.decode_step(cfg, d["c"], d["kr"], d["qc"], d["qr"], buf.w_uk, buf.w_uv, gw, gb,
+                             d["gate_in"], pos, buf.cache, buf.open_slot, out, buf.workspace)
+        nbytes = wl.B * max_slots * wl.D * 2
+        unit_fn = lambda ms: nbytes / (ms / 1e3) / 1e9
+        unit, peak, bound = "GB/s", hbm, "hbm"
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    prof = mtla.ProfileEvents(args.steps)
+    with ClockSampler(torch.cuda.current_device()) as clk, prof:
+        for i in range(args.steps):
+            flush.zero_()
+            ev[i][0].record(st)
+            call()
+            ev[i][1].record(st)
+        torch.cuda.synchronize()
+    assert mtla.get_device_status() == mtla.OK
+    call_ms = statistics.median(a.elapsed_time(b_) for a, b_ in ev)
+    kern_ms = statistics.median(prof.durations_ms())
+    line = {"workload": name, "config": {"B": wl.B, "H": wl.H, "d_h": wl.d_h, "d_c": wl.d_c,
+                                         "d_R": wl.d_r, "s": wl.s, "T_or_N": wl.T},
+            "call_ms": call_ms, "attention_kernel_ms": kern_ms,
+            "call": {"value": unit_fn(call_ms), "unit": unit},
+            "roofline": {"kernel": "attention", "bound": bound, "achieved": unit_fn(kern_ms),
+                         "peak": peak, "unit": unit, "frac": unit_fn(kern_ms) / peak,
+                         "peak_source": f"{peak_kind} " + ("hbm_gbs" if bound == "hbm" else "bf16_tflops")},
+            "clocks": clk.summary(), "l2": "flushed (256 MiB write) before every timed call"}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -260,9 +339,18 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="mtla", choices=["mtla", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default="speech_decode",
+                    help="speech_decode (the contract line) or a kernel-level measurement of "
+                         "stride_sweep[:s], prefill or large_latent")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     ws, rank = _dist()
+    if args.workload != "speech_decode":
+        if rank == 0:
+            run_kernel_workload(args, ws, rank)
+        if ws > 1:
+            torch.distributed.destroy_process_group()
+        return
     if args.impl == "reference":
         run_reference(args, ws, rank)
         if ws > 1:

@@ -31,11 +31,20 @@ static int32_t g_prof_pairs = 0;
 static int32_t g_prof_next = 0;
 static bool g_prof_open = false;
 
+// Record a profile event: a plain record, or an event node while `st` is
+// being captured into a graph.
+static cudaError_t record_profile_event(void* ev, cudaStream_t st) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cs) != cudaSuccess) return cudaGetLastError();
+    if (cs == cudaStreamCaptureStatusActive)
+        return cudaEventRecordWithFlags((cudaEvent_t)ev, st, cudaEventRecordExternal);
+    return cudaEventRecord((cudaEvent_t)ev, st);
+}
+
 void profile_begin(cudaStream_t st) {
     g_prof_open = false;
     if (g_prof_events && g_prof_next < g_prof_pairs) {
-        if (cudaEventRecordWithFlags((cudaEvent_t)g_prof_events[2 * g_prof_next], st,
-                                      cudaEventRecordExternal) == cudaSuccess) {
+        if (record_profile_event(g_prof_events[2 * g_prof_next], st) == cudaSuccess) {
             g_prof_open = true;
         } else {
             cudaGetLastError();            // a bad handle turns the hook off, not the call
@@ -46,8 +55,7 @@ void profile_begin(cudaStream_t st) {
 
 void profile_end(cudaStream_t st) {
     if (g_prof_open) {
-        if (cudaEventRecordWithFlags((cudaEvent_t)g_prof_events[2 * g_prof_next + 1], st,
-                                      cudaEventRecordExternal) == cudaSuccess) {
+        if (record_profile_event(g_prof_events[2 * g_prof_next + 1], st) == cudaSuccess) {
             ++g_prof_next;
         } else {
             cudaGetLastError();
@@ -116,9 +124,15 @@ static mtla_status check_config(const mtla_config* cfg, Shape* sh) {
 static bool use_tc_decode(const mtla_config* cfg, const Shape& sh) {
     return cfg->dtype == MTLA_BF16 && tc_decode_supported(sh);
 }
+// bf16 with 32 < heads <= 128: the cluster kernel with all heads as M = 128.
+static bool use_tc_decode_lh(const mtla_config* cfg, const Shape& sh) {
+    return cfg->dtype == MTLA_BF16 && !tc_decode_supported(sh) && tc_decode_lh_supported(sh);
+}
 
 static size_t decode_ws(const mtla_config* cfg, const Shape& sh) {
-    return use_tc_decode(cfg, sh) ? tc_decode_workspace(sh) : simt_decode_workspace(sh);
+    if (use_tc_decode(cfg, sh)) return tc_decode_workspace(sh);
+    if (use_tc_decode_lh(cfg, sh)) return tc_decode_lh_workspace(sh);
+    return simt_decode_workspace(sh);
 }
 // bf16 prefill runs on the tensor cores where the shape fits the kernel
 // (d_h = 64, d_c <= 256, slot width <= 320); the rest on the CUDA cores.
@@ -192,8 +206,9 @@ mtla_status mtla_decode_step(const mtla_config* cfg, const void* c_new, const vo
     g_error_detail[0] = 0;
     if (note_error("device status word", status_ptr(&a.status)) != cudaSuccess) return MTLA_ERR_CUDA;
     uint64_t n = 0;
-    cudaError_t e = use_tc_decode(cfg, sh) ? tc_decode(a, (cudaStream_t)stream, &n)
-                                           : simt_decode(a, cfg->dtype == MTLA_FP32, (cudaStream_t)stream, &n);
+    cudaError_t e = use_tc_decode(cfg, sh)      ? tc_decode(a, (cudaStream_t)stream, &n)
+                    : use_tc_decode_lh(cfg, sh) ? tc_decode_lh(a, (cudaStream_t)stream, &n)
+                                                : simt_decode(a, cfg->dtype == MTLA_FP32, (cudaStream_t)stream, &n);
     g_launches += n;
     if (e != cudaSuccess && !g_error_detail[0]) note_error("decode launch", e);
     return e == cudaSuccess ? MTLA_OK : MTLA_ERR_CUDA;

@@ -69,6 +69,11 @@ bool tc_decode_supported(const Shape& sh);
 size_t tc_decode_workspace(const Shape& sh);
 cudaError_t tc_decode(const DecodeArgs& a, cudaStream_t st, uint64_t* launches);
 
+// Tensor-core decode for many heads (bf16, 32 < heads <= 128, 2-CTA clusters).
+bool tc_decode_lh_supported(const Shape& sh);
+size_t tc_decode_lh_workspace(const Shape& sh);
+cudaError_t tc_decode_lh(const DecodeArgs& a, cudaStream_t st, uint64_t* launches);
+
 // Tensor-core prefill (bf16, d_h = 64, d_c <= 256, slot width <= 320).
 bool tc_prefill_supported(const Shape& sh);
 size_t tc_prefill_workspace(const Shape& sh, int T);

@@ -42,15 +42,14 @@ namespace {
 using namespace tc;
 
 constexpr int kTileSlots = 128;
-constexpr int kThreads = 128;
+constexpr int kAttnThreads = 192;   // warps 0-3 softmax, 4 TMA, 5 MMA
+constexpr float kRescaleLog2 = 8.f;
 constexpr int kMaxGrid = 160;  // >= SMs of any sm_100 part; sizes the partial buffer
 constexpr int kMaxB = 2048;
-// S^T is accumulated in 4 independent TMEM accumulators (K-steps round robin)
-// so that the chain of dependent MMAs is a quarter as long; the softmax adds them.
-constexpr int kSAcc = 4;
 
 struct DecTC {
     int B, H, D, d_c, s, max_slots;
+    int Hp;          // H rounded up to 8: heads per partial row block
     int n_chunks;    // D rounded up to 64, in 64-column chunks
     int lat_blocks;  // d_c / 128
     int G;           // grid size
@@ -58,7 +57,7 @@ struct DecTC {
     const int32_t* pos;
     const uint8_t* qimg;  // [B] x n_chunks x [NH rows x 128 B]: q~ in bf16, SW128, zero padded
     uint32_t qimg_bytes;  // per sequence
-    float* part;          // [(kMaxGrid + B), H, d_c + 2]
+    float* part;          // [(kMaxGrid + B), Hp, d_c + 2]
     int* status;
 };
 
@@ -73,21 +72,6 @@ __device__ __forceinline__ int seq_slots(const DecTC& p, int b) {
     if (t < 0 || t >= (int64_t)p.max_slots * p.s) return 0;
     return (int)(t / p.s) + 1;
 }
-
-template <int NH>
-struct Misc {
-    uint64_t full[2];
-    uint64_t bar_s;
-    uint64_t bar_o;
-    uint64_t bar_q;
-    uint32_t tmem_base;
-    int fail;
-    int rescale;
-    int total;
-    float red[4][NH];
-    float m_run[NH];
-    float fac[NH];
-};
 
 // Decode prep for the tensor-core path. grid (B, H + 1), 128 threads.
 // Block (b, h < H): absorbed query of head h, q~ = [W_UK[h]^T qC ; RoPE_t(qR)],
@@ -163,23 +147,54 @@ __global__ void __launch_bounds__(128) k_dec_prep_tc(DecodeArgs a, uint8_t* qimg
     }
 }
 
-template <int NH>
-__global__ void __launch_bounds__(kThreads, 1)
+// Barriers and small shared state of k_dec_attn_sh.
+template <int HV>
+struct SmallBars {
+    uint64_t full[2], empty[2];          // slot-tile ring
+    uint64_t q_full, q_free;             // query image of the current segment
+    uint64_t s_full[2], s_empty[2];      // S^T buffers
+    uint64_t p_full[2];                  // P^T buffers (4 softmax warps arrive)
+    uint64_t o_done[2];                  // P.V of tiles with this parity completed
+    uint64_t drain;                      // MMAs in flight when a wait gave up
+    uint32_t tmem_base;
+    volatile int fail;
+    int total;
+    float4 red[2][HV];                   // per head: the 4 warps' tile maxima, by tile parity
+    float4 lsum[HV];                     // per head: the 4 warps' sums at a segment end
+    float msave[HV];
+};
+
+template <int HV>
+__device__ __forceinline__ bool sb_wait(uint64_t* bar, uint32_t parity, SmallBars<HV>& bs) {
+    if (bs.fail) return false;
+    if (mbar_wait(bar, parity)) return true;
+    bs.fail = 1;
+    return false;
+}
+
+// Split-K attention over 128-slot tiles, heads as the MMA's N (NH = 16 or 32).
+// Warps 0-3: online softmax, thread = slot row (its TMEM lane), over HV heads
+// (H rounded up to 8; a compile-time count, so every per-head loop is
+// straight-line code); warp 4: TMA; warp 5: MMA issue and TMEM. S^T and P^T
+// are double-buffered so MMA1 of the next tile overlaps this tile's softmax.
+template <int NH, int HV>
+__global__ void __launch_bounds__(kAttnThreads, 1)
     k_dec_attn_sh(const __grid_constant__ CUtensorMap tmap, const DecTC p) {
+    static_assert(HV % 8 == 0 && HV <= NH, "head count");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int n_chunks = p.n_chunks;
     const uint32_t stage_bytes = (uint32_t)n_chunks * 16384u;
-    uint8_t* stage_ptr[2] = {smem, smem + stage_bytes};
+    uint8_t* ring = smem;                                        // 2 stages
     uint8_t* q_s = smem + 2 * stage_bytes;                       // n_chunks x [NH x 128 B]
-    uint8_t* p_s = q_s + (size_t)n_chunks * NH * 128;            // 2 x [NH x 128 B]
-    Misc<NH>& m = *(Misc<NH>*)(p_s + 2 * NH * 128);
-    int* starts = (int*)((uint8_t*)&m + ((sizeof(Misc<NH>) + 15) & ~(size_t)15));   // [B + 1]
+    uint8_t* p_s = q_s + (size_t)n_chunks * NH * 128;            // 2 buffers x 2 chunks x [NH x 128 B]
+    SmallBars<HV>& bs = *(SmallBars<HV>*)(p_s + 4 * NH * 128);
+    int* starts = (int*)((uint8_t*)&bs + ((sizeof(SmallBars<HV>) + 15) & ~(size_t)15));   // [B + 1]
 
-    // ---- schedule: tiles per sequence and their exclusive prefix sum
+    // ---- schedule: tiles per sequence and their exclusive prefix sum (reads pos only)
     {
-        const int per = (p.B + kThreads - 1) / kThreads;
+        const int per = (p.B + kAttnThreads - 1) / kAttnThreads;
         const int b0 = tid * per, b1 = min(b0 + per, p.B);
         int local = 0;
         for (int b = b0; b < b1; ++b) local += seq_tiles(p, b);
@@ -189,56 +204,60 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int v = __shfl_up_sync(0xffffffffu, incl, o);
             if (lane >= o) incl += v;
         }
-        __shared__ int warp_tot[4];
+        __shared__ int warp_tot[kAttnThreads / 32];
         if (lane == 31) warp_tot[warp] = incl;
         __syncthreads();
-        int off = 0;
-        for (int w = 0; w < warp; ++w) off += warp_tot[w];
+        int off = 0, tot = 0;
+        for (int w = 0; w < kAttnThreads / 32; ++w) {
+            if (w < warp) off += warp_tot[w];
+            tot += warp_tot[w];
+        }
         int run = off + incl - local;
         for (int b = b0; b < b1; ++b) {
             starts[b] = run;
             run += seq_tiles(p, b);
         }
         if (tid == 0) {
-            m.total = warp_tot[0] + warp_tot[1] + warp_tot[2] + warp_tot[3];
-            starts[p.B] = m.total;
+            bs.total = tot;
+            starts[p.B] = tot;
         }
     }
-    // ---- barriers and TMEM
-    const uint32_t tmem_cols_needed = (uint32_t)NH * (kSAcc + p.lat_blocks);
+    const uint32_t tmem_cols_needed = (uint32_t)NH * (2 + p.lat_blocks);
     uint32_t tmem_cols = 32;
     while (tmem_cols < tmem_cols_needed) tmem_cols <<= 1;
     if (tid == 0) {
-        mbar_init(&m.full[0], 1);
-        mbar_init(&m.full[1], 1);
-        mbar_init(&m.bar_s, 1);
-        mbar_init(&m.bar_o, 1);
-        mbar_init(&m.bar_q, 1);
-        m.fail = 0;
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bs.full[i], 1);
+            mbar_init(&bs.empty[i], 1);
+            mbar_init(&bs.s_full[i], 1);
+            mbar_init(&bs.s_empty[i], 4);
+            mbar_init(&bs.p_full[i], 4);
+            mbar_init(&bs.o_done[i], 1);
+        }
+        mbar_init(&bs.q_full, 1);
+        mbar_init(&bs.q_free, 1);
+        mbar_init(&bs.drain, 1);
+        bs.fail = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmap);
     }
-    pdl_launch_dependents();
-    if (warp == 0) {
-        tmem_alloc(&m.tmem_base, tmem_cols);
+    if (warp == 5) {
+        tmem_alloc(&bs.tmem_base, tmem_cols);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = m.tmem_base;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-    const uint32_t t_s = tmem;                // S^T: kSAcc partial sums of NH columns each
-    const uint32_t t_o = tmem + kSAcc * NH;   // O^T: lat_blocks x NH columns
-
-    const int total = m.total;
+    pdl_launch_dependents();
+    const uint32_t tmem = bs.tmem_base;
+    const uint32_t t_s = tmem;                 // S^T buffers: 2 x NH columns
+    const uint32_t t_o = tmem + 2 * NH;        // O^T: lat_blocks x NH columns
+    const int total = bs.total;
     const int g = blockIdx.x;
     const int gt0 = (int)(((int64_t)g * total) / p.G);
     const int gt1 = (int)(((int64_t)(g + 1) * total) / p.G);
-
-    // global tile -> (sequence, tile within the sequence)
     auto locate = [&](int gt, int& b, int& j) {
-        int lo = 0, hi = p.B - 1;        // largest b with starts[b] <= gt
+        int lo = 0, hi = p.B - 1;            // largest b with starts[b] <= gt
         while (lo < hi) {
             const int mid = (lo + hi + 1) >> 1;
             if (starts[mid] <= gt) lo = mid; else hi = mid - 1;
@@ -246,220 +265,232 @@ __global__ void __launch_bounds__(kThreads, 1)
         b = lo;
         j = gt - starts[lo];
     };
-    auto issue_load = [&](int gt, int stage) {
-        int b, j;
-        locate(gt, b, j);
-        mbar_arrive_expect_tx(&m.full[stage], stage_bytes);
-        for (int c = 0; c < n_chunks; ++c)
-            tma_load_3d(stage_ptr[stage] + (size_t)c * 16384, &tmap, &m.full[stage], c * 64, j * kTileSlots, b);
-    };
+    pdl_wait();                              // the cache row and q~ come from k_dec_prep_tc
 
-    const uint32_t idesc_s = idesc_bf16_f32(128, NH, false, false);
-    const uint32_t idesc_o = idesc_bf16_f32(128, NH, true, false);
-
-    // everything above only read pos; the cache row and q~ come from k_dec_prep_tc
-    pdl_wait();
-    int loads_issued = 0;
-    if (tid == 0) {
-        for (int k = 0; k < 2 && gt0 + k < gt1; ++k) {
-            issue_load(gt0 + k, k);
-            ++loads_issued;
-        }
-    }
-
-    float l_part[NH];
-    int seq_b = -1, seq_n = 0, q_phase = 0;
-    bool first_o = true;
-    bool failed = false;
-    int it = 0;
-    for (int gt = gt0; gt < gt1; ++gt, ++it) {
-        int b, j;
-        locate(gt, b, j);
-        const int st = it & 1;
-        if (b != seq_b) {
-            // new segment: this sequence's query image (one bulk copy)
-            seq_b = b;
-            seq_n = seq_slots(p, b);
-            first_o = true;
-            if (tid == 0) {
-                mbar_arrive_expect_tx(&m.bar_q, p.qimg_bytes);
-                bulk_load(q_s, p.qimg + (size_t)b * p.qimg_bytes, p.qimg_bytes, &m.bar_q);
-            }
-            if (!mbar_wait(&m.bar_q, q_phase & 1)) m.fail = 1;
-            ++q_phase;
-            if (tid < NH) m.m_run[tid] = -INFINITY;
-#pragma unroll
-            for (int h = 0; h < NH; ++h) l_part[h] = 0.f;
-        }
-        // (1) previous PV done: its stage takes the tile after this one
-        if (it > 0) {
-            if (!mbar_wait(&m.bar_o, (it - 1) & 1)) m.fail = 1;
-            if (tid == 0 && !m.fail && gt + 1 < gt1) {
-                issue_load(gt + 1, (it + 1) & 1);
+    int loads_issued = 0, q_loads = 0;       // producer's copies, for the drain on failure
+    if (warp == 4) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int prev_b = -1;
+            for (int gt = gt0, it = 0; gt < gt1; ++gt, ++it) {
+                int b, j;
+                locate(gt, b, j);
+                if (b != prev_b) {
+                    prev_b = b;
+                    if (q_loads >= 1 && !sb_wait(&bs.q_free, (q_loads - 1) & 1, bs)) break;
+                    mbar_arrive_expect_tx(&bs.q_full, p.qimg_bytes);
+                    bulk_load(q_s, p.qimg + (size_t)b * p.qimg_bytes, p.qimg_bytes, &bs.q_full);
+                    ++q_loads;
+                }
+                const int st = it & 1;
+                if (it >= 2 && !sb_wait(&bs.empty[st], ((it >> 1) - 1) & 1, bs)) break;
+                mbar_arrive_expect_tx(&bs.full[st], stage_bytes);
+                for (int c = 0; c < n_chunks; ++c)
+                    tma_load_3d(ring + st * stage_bytes + (size_t)c * 16384, &tmap, &bs.full[st], c * 64,
+                                j * kTileSlots, b);
                 ++loads_issued;
             }
         }
-        // (2) this tile's slots
-        if (!mbar_wait(&m.full[st], (it >> 1) & 1)) m.fail = 1;
-        const int valid = min(kTileSlots, seq_n - j * kTileSlots);
-        if (valid < kTileSlots && tid >= valid) {
-            // stale rows past the sequence's last slot must not reach P.V
-            for (int c = 0; c < n_chunks; ++c) {
-                uint4* row = (uint4*)(stage_ptr[st] + (size_t)c * 16384 + (size_t)tid * 128);
+    } else if (warp == 5) {
+        // ------------------------------------------------------------ MMA issue
+        if (lane == 0) {
+            const uint32_t id_s = idesc_bf16_f32(128, NH, false, false);
+            const uint32_t id_o = idesc_bf16_f32(128, NH, true, false);
+            const uint64_t q_d = sdesc_sw128(smem_u32(q_s), 16, 1024);
+            const uint32_t ring_a = smem_u32(ring), p_a = smem_u32(p_s);
+            int seg = -1, prev_b = -1;
+            bool prev_first = true, ok = true;
+            int it = 0;
+            // O^T += V^T . P^T for tile k (A = the slot tile, MN-major; B = P^T, K-major)
+            auto issue_pv = [&](int k, bool first) -> bool {
+                if (!sb_wait(&bs.p_full[k & 1], (k >> 1) & 1, bs)) return false;
+                tc_fence_after();
+                const uint64_t a0 = sdesc_sw128(ring_a + (k & 1) * stage_bytes, 16384, 1024);
+                const uint64_t b0 = sdesc_sw128(p_a + (k & 1) * 2 * NH * 128, 16, 1024);
+                for (int lb = 0; lb < p.lat_blocks; ++lb) {
+                    const uint64_t al = desc_add(a0, 2 * lb * 16384);
 #pragma unroll
-                for (int u = 0; u < 8; ++u) row[u] = make_uint4(0, 0, 0, 0);
-            }
-        }
-        fence_proxy_async();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        if (m.fail) { failed = true; break; }
-        // (3) S^T = K_tile . q~^T
-        if (tid == 0) {
-            const uint32_t a0 = smem_u32(stage_ptr[st]);
-            const uint32_t b0 = smem_u32(q_s);
-            for (int c = 0; c < n_chunks; ++c)
-                for (int kk = 0; kk < 4; ++kk) {
-                    const int step = c * 4 + kk;
-                    const uint64_t ad = sdesc_sw128(a0 + c * 16384 + kk * 32, 16, 1024);
-                    const uint64_t bd = sdesc_sw128(b0 + c * NH * 128 + kk * 32, 16, 1024);
-                    umma_bf16(t_s + (step % kSAcc) * NH, ad, bd, idesc_s, step >= kSAcc);
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma_bf16(t_o + lb * NH, desc_add(al, kk * 2048),
+                                  desc_add(b0, (kk >> 2) * NH * 128 + (kk & 3) * 32), id_o,
+                                  (first && kk == 0) ? 0u : 1u);
                 }
-            umma_commit(&m.bar_s);
-        }
-        if (!mbar_wait(&m.bar_s, it & 1)) m.fail = 1;
-        tc_fence_after();
-        // (4) online softmax, thread = slot row
-        float sv[NH];
-        {
-            float part[kSAcc][NH];
+                umma_commit(&bs.empty[k & 1]);
+                umma_commit(&bs.o_done[k & 1]);
+                return true;
+            };
+            for (int gt = gt0; gt < gt1; ++gt, ++it) {
+                int b, j;
+                locate(gt, b, j);
+                const bool first = (b != prev_b);
+                if (first) {
+                    prev_b = b;
+                    ++seg;
+                    if (!sb_wait(&bs.q_full, seg & 1, bs)) { ok = false; break; }
+                }
+                const int st = it & 1;
+                if (!sb_wait(&bs.full[st], (it >> 1) & 1, bs)) { ok = false; break; }
+                if (it >= 2 && !sb_wait(&bs.s_empty[st], ((it >> 1) - 1) & 1, bs)) { ok = false; break; }
+                tc_fence_after();
+                // S^T = K_tile . q~^T (A = slot tile, B = q~ image; both K-major)
+                const uint64_t a0 = sdesc_sw128(ring_a + st * stage_bytes, 16, 1024);
+                for (int c = 0; c < n_chunks; ++c) {
+                    const uint64_t ac = desc_add(a0, c * 16384), bc = desc_add(q_d, c * NH * 128);
 #pragma unroll
-            for (int q = 0; q < kSAcc; ++q) {
-                tmem_ld16(t_s + q * NH + lane_off, part[q]);
-                if (NH == 32) tmem_ld16(t_s + q * NH + lane_off + 16, part[q] + 16);
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_bf16(t_s + st * NH, desc_add(ac, kk * 32), desc_add(bc, kk * 32), id_s, (c | kk) != 0);
+                }
+                umma_commit(&bs.s_full[st]);
+                const bool last = (gt + 1 == gt1) || (j + 1 == starts[b + 1] - starts[b]);
+                if (last) umma_commit(&bs.q_free);
+                if (it >= 1 && !issue_pv(it - 1, prev_first)) { ok = false; break; }
+                prev_first = first;
             }
+            if (ok && it >= 1) issue_pv(it - 1, prev_first);
+        }
+    } else {
+        // ------------------------------------------------------------ softmax (warps 0-3)
+        // No early exit: every softmax thread passes every named barrier even after a
+        // bounded wait gave up (later waits then return at once), so none can hang.
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        float m_ref[HV], l_part[HV];
+        int prev_b = -1, n_b = 0, k_in_seg = 0;
+        for (int gt = gt0, it = 0; gt < gt1; ++gt, ++it) {
+            int b, j;
+            locate(gt, b, j);
+            if (b != prev_b) {
+                prev_b = b;
+                n_b = seq_slots(p, b);
+                k_in_seg = 0;
+#pragma unroll
+                for (int h = 0; h < HV; ++h) {
+                    m_ref[h] = -INFINITY;
+                    l_part[h] = 0.f;
+                }
+            }
+            const int st = it & 1;
+            const int valid = min(kTileSlots, n_b - j * kTileSlots);
+            sb_wait(&bs.s_full[st], (it >> 1) & 1, bs);
+            tc_fence_after();
+            float sv[HV];
+            tmem_ld_cols<HV>(t_s + st * NH + lane_off, sv);
             tmem_wait_ld();
-#pragma unroll
-            for (int h = 0; h < NH; ++h) sv[h] = (part[0][h] + part[1][h]) + (part[2][h] + part[3][h]);
-        }
-        const bool row_ok = tid < valid;
-#pragma unroll
-        for (int h = 0; h < NH; ++h) sv[h] = row_ok ? sv[h] * p.scale_log2 : -INFINITY;
-#pragma unroll
-        for (int h = 0; h < NH; ++h) {
-            if (h < p.H) {
-                const float mx = warp_max(sv[h]);
-                if (lane == 0) m.red[warp][h] = mx;
-            }
-        }
-        __syncthreads();
-        if (tid < p.H) {
-            const float tile_max = fmaxf(fmaxf(m.red[0][tid], m.red[1][tid]), fmaxf(m.red[2][tid], m.red[3][tid]));
-            const float old = m.m_run[tid];
-            const float nm = fmaxf(old, tile_max);
-            m.fac[tid] = (old == -INFINITY) ? 0.f : exp2f(old - nm);
-            m.m_run[tid] = nm;
-        }
-        if (tid == 0) m.rescale = 0;
-        __syncthreads();
-        if (tid < p.H && m.fac[tid] != 1.f && !first_o) m.rescale = 1;
-        float pv[NH];
-#pragma unroll
-        for (int h = 0; h < NH; ++h) {
-            pv[h] = 0.f;
-            if (h < p.H) {
-                pv[h] = exp2f(sv[h] - m.m_run[h]);
-                l_part[h] = l_part[h] * m.fac[h] + pv[h];
-            }
-        }
-        // P^T into shared memory as the K-major B operand [NH x 128 slots]
-        {
-            uint8_t* pc = p_s + (size_t)(tid >> 6) * NH * 128;
-#pragma unroll
-            for (int h = 0; h < NH; ++h) *(bf16*)(pc + sw128_offset(h, tid & 63)) = __float2bfloat16_rn(pv[h]);
-        }
-        fence_proxy_async();
-        __syncthreads();
-        // (5) rescale the running O^T where a head's max moved
-        if (m.rescale) {
-            for (int lb = 0; lb < p.lat_blocks; ++lb) {
-                float ov[NH];
-                const uint32_t ta = t_o + lb * NH + lane_off;
-                tmem_ld16(ta, ov);
-                if (NH == 32) tmem_ld16(ta + 16, ov + 16);
-                tmem_wait_ld();
-#pragma unroll
-                for (int h = 0; h < NH; ++h) ov[h] *= m.fac[h];
-                tmem_st16(ta, ov);
-                if (NH == 32) tmem_st16(ta + 16, ov + 16);
-            }
-            tmem_wait_st();
-        }
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        // (6) O^T += V^T . P^T
-        if (tid == 0) {
-            const uint32_t a0 = smem_u32(stage_ptr[st]);
-            const uint32_t b0 = smem_u32(p_s);
-            for (int lb = 0; lb < p.lat_blocks; ++lb)
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t ad = sdesc_sw128(a0 + (2 * lb) * 16384 + kk * 2048, 16384, 1024);
-                    const uint64_t bd = sdesc_sw128(b0 + (kk >> 2) * NH * 128 + (kk & 3) * 32, 16, 1024);
-                    umma_bf16(t_o + lb * NH, ad, bd, idesc_o, (first_o && kk == 0) ? 0u : 1u);
-                }
-            umma_commit(&m.bar_o);
-        }
-        first_o = false;
-        // (7) end of this sequence's segment: write the partial (o, m, l)
-        const bool seg_end = (gt + 1 == gt1) || (j + 1 == starts[b + 1] - starts[b]);
-        if (seg_end) {
-            if (!mbar_wait(&m.bar_o, it & 1)) m.fail = 1;
-            tc_fence_after();
-#pragma unroll
-            for (int h = 0; h < NH; ++h) {
-                if (h < p.H) {
-                    const float sum = warp_sum(l_part[h]);
-                    if (lane == 0) m.red[warp][h] = sum;
-                }
-            }
-            __syncthreads();
-            if (m.fail) { failed = true; break; }
-            float* dst = p.part + (size_t)(g + b) * p.H * (p.d_c + 2);
-            for (int lb = 0; lb < p.lat_blocks; ++lb) {
-                float ov[NH];
-                const uint32_t ta = t_o + lb * NH + lane_off;
-                tmem_ld16(ta, ov);
-                if (NH == 32) tmem_ld16(ta + 16, ov + 16);
-                tmem_wait_ld();
-#pragma unroll
-                for (int h = 0; h < NH; ++h)
-                    if (h < p.H) dst[(size_t)h * (p.d_c + 2) + lb * 128 + tid] = ov[h];
-            }
-            if (tid < p.H) {
-                dst[(size_t)tid * (p.d_c + 2) + p.d_c] = m.m_run[tid];
-                dst[(size_t)tid * (p.d_c + 2) + p.d_c + 1] =
-                    m.red[0][tid] + m.red[1][tid] + m.red[2][tid] + m.red[3][tid];
-            }
             tc_fence_before();
-            __syncthreads();
-            tc_fence_after();
-        }
-    }
-    if (failed) {
-        // drain what is still in flight (bounded), then report
-        if (tid == 0) {
-            latch_status(p.status, kStatusTimeout);
-            for (int k = it; k < loads_issued && k < it + 2; ++k) mbar_wait(&m.full[k & 1], (k >> 1) & 1);
-            mbar_wait(&m.bar_s, it & 1);
-            if (it > 0) mbar_wait(&m.bar_o, (it - 1) & 1);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bs.s_empty[st]);
+            if (valid < kTileSlots) {
+                // stale rows past the sequence's last slot must not reach P.V
+                // (whole 128-byte rows, so the swizzle does not matter)
+                for (int c = 0; c < n_chunks; ++c) {
+                    uint8_t* base = ring + st * stage_bytes + (size_t)c * 16384;
+                    for (int off = valid * 128 + tid * 16; off < 16384; off += 128 * 16)
+                        *(uint4*)(base + off) = make_uint4(0, 0, 0, 0);
+                }
+            }
+            const bool row_ok = tid < valid;
+#pragma unroll
+            for (int h = 0; h < HV; ++h) {
+                sv[h] = row_ok ? sv[h] * p.scale_log2 : -INFINITY;
+                const float mx = warp_max_redux(sv[h]);
+                if (lane == 0) reinterpret_cast<float*>(&bs.red[st][h])[warp] = mx;
+            }
+            named_sync(1, 128);
+            // lazy rescale: a head's reference maximum moves only when the tile's
+            // maximum exceeds it by more than 2^8 (P stays <= 256 in bf16)
+            float fac[HV];
+            bool any_rescale = false;
+#pragma unroll
+            for (int h = 0; h < HV; ++h) {
+                const float4 r = bs.red[st][h];
+                const float tmax = fmaxf(fmaxf(r.x, r.y), fmaxf(r.z, r.w));
+                const bool upd = tmax > m_ref[h] + kRescaleLog2;
+                const float nm = upd ? tmax : m_ref[h];
+                fac[h] = exp2f(m_ref[h] - nm);     // 0 when m_ref was -inf, 1 when kept
+                any_rescale |= upd;
+                m_ref[h] = nm;
+                sv[h] = exp2f(sv[h] - nm);
+                l_part[h] = fmaf(l_part[h], fac[h], sv[h]);
+            }
+            any_rescale &= (k_in_seg > 0);
+            // P^T buffer st was last read by P.V of tile it-2
+            if (it >= 2) sb_wait(&bs.o_done[st], ((it >> 1) - 1) & 1, bs);
+            if (any_rescale) {
+                // the running O^T of this segment moves to the new reference maximum
+                sb_wait(&bs.o_done[st ^ 1], ((it - 1) >> 1) & 1, bs);
+                tc_fence_after();
+                for (int lb = 0; lb < p.lat_blocks; ++lb) {
+                    float ov[HV];
+                    const uint32_t ta = t_o + lb * NH + lane_off;
+                    tmem_ld_cols<HV>(ta, ov);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int h = 0; h < HV; ++h) ov[h] *= fac[h];
+                    tmem_st_cols<HV>(ta, ov);
+                }
+                tmem_wait_st();
+            }
+            {
+                uint8_t* pb = p_s + (size_t)st * 2 * NH * 128 + (size_t)(tid >> 6) * NH * 128;
+#pragma unroll
+                for (int h = 0; h < HV; ++h) *(bf16*)(pb + sw128_offset(h, tid & 63)) = __float2bfloat16_rn(sv[h]);
+            }
+            fence_proxy_async();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bs.p_full[st]);
+            ++k_in_seg;
+            const bool last = (gt + 1 == gt1) || (j + 1 == starts[b + 1] - starts[b]);
+            if (last) {
+                // partial (o, m, l) of this sequence segment: rows of HV heads
+                sb_wait(&bs.o_done[st], (it >> 1) & 1, bs);
+                tc_fence_after();
+#pragma unroll
+                for (int h = 0; h < HV; ++h) l_part[h] = warp_sum(l_part[h]);
+                if (lane == 0) {
+#pragma unroll
+                    for (int h = 0; h < HV; ++h) reinterpret_cast<float*>(&bs.lsum[h])[warp] = l_part[h];
+                }
+                if (tid == 0) {
+#pragma unroll
+                    for (int h = 0; h < HV; ++h) bs.msave[h] = m_ref[h];
+                }
+                named_sync(1, 128);
+                float* dst = p.part + (size_t)(g + b) * HV * (p.d_c + 2);
+                for (int lb = 0; lb < p.lat_blocks; ++lb) {
+                    float ov[HV];
+                    tmem_ld_cols<HV>(t_o + lb * NH + lane_off, ov);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int h = 0; h < HV; ++h) dst[(size_t)h * (p.d_c + 2) + lb * 128 + tid] = ov[h];
+                }
+                if (tid < HV) {
+                    const float4 l4 = bs.lsum[tid];
+                    dst[(size_t)tid * (p.d_c + 2) + p.d_c] = bs.msave[tid];
+                    dst[(size_t)tid * (p.d_c + 2) + p.d_c + 1] = (l4.x + l4.y) + (l4.z + l4.w);
+                }
+                named_sync(1, 128);          // lsum and msave are free for the next segment
+                tc_fence_before();
+            }
         }
     }
     tc_fence_before();
     __syncthreads();
+    if (bs.fail) {
+        // a bounded wait gave up: let this CTA's copies and MMAs land (bounded
+        // again) before the shared memory and TMEM are released, then report
+        if (warp == 4 && lane == 0) {
+            for (int k = max(0, loads_issued - 2); k < loads_issued; ++k) mbar_wait(&bs.full[k & 1], (k >> 1) & 1);
+            if (q_loads > 0) mbar_wait(&bs.q_full, (q_loads - 1) & 1);
+        }
+        if (warp == 5 && lane == 0) {
+            umma_commit(&bs.drain);
+            mbar_wait(&bs.drain, 0);
+        }
+        if (tid == 0) latch_status(p.status, kStatusTimeout);
+        __syncthreads();
+    }
     tc_fence_after();
-    if (warp == 0) tmem_dealloc(tmem, tmem_cols);
+    if (warp == 5) tmem_dealloc(tmem, tmem_cols);
 }
 
 // Merge the partials of (b, h) and apply W_UV. grid (H, B), 256 threads.
@@ -472,14 +503,23 @@ __global__ void __launch_bounds__(256) k_dec_combine(DecodeArgs a, DecTC p) {
     __shared__ float red[32];
     __shared__ int idx[kMaxGrid];
     __shared__ int n_part;
-    __shared__ float olat[512];
+    __shared__ __align__(16) float olat[512];
     extern __shared__ uint8_t dyn[];
     bf16* Ws = (bf16*)dyn;                            // W_UV[h] [d_h x d_c]
     {
+        // eight 16-byte loads in flight per thread before any store
         const uint4* src = (const uint4*)((const bf16*)a.w_uv + (size_t)h * sh.d_h * sh.d_c);
         uint4* dst = (uint4*)Ws;
         const int n16 = sh.d_h * sh.d_c / 8;
-        for (int e = threadIdx.x; e < n16; e += blockDim.x) dst[e] = src[e];
+        for (int e0 = threadIdx.x; e0 < n16; e0 += 8 * blockDim.x) {
+            uint4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (e0 + u * (int)blockDim.x < n16) v[u] = src[e0 + u * blockDim.x];
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (e0 + u * (int)blockDim.x < n16) dst[e0 + u * blockDim.x] = v[u];
+        }
     }
     // this sequence's tile range and the total
     int before = 0, all = 0;
@@ -510,7 +550,7 @@ __global__ void __launch_bounds__(256) k_dec_combine(DecodeArgs a, DecTC p) {
     __syncthreads();
     pdl_wait();   // the partials come from k_dec_attn_sh
     const int n = n_part;
-    const size_t stride = (size_t)p.H * (p.d_c + 2);
+    const size_t stride = (size_t)p.Hp * (p.d_c + 2);
     const size_t hoff = (size_t)h * (p.d_c + 2);
     for (int jj = threadIdx.x; jj < p.d_c; jj += blockDim.x) {
         // one round of loads: (m, l, o[jj]) of every partial
@@ -540,19 +580,34 @@ __global__ void __launch_bounds__(256) k_dec_combine(DecodeArgs a, DecTC p) {
         olat[jj] = acc / L;
     }
     __syncthreads();
+    // o = W_UV[h] o_lat: warp w takes rows w, w + 8, ... in groups of 8 rows whose
+    // dot products run side by side (8 independent chains, one reduction round)
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     bf16* out = (bf16*)a.out + ((size_t)b * sh.H + h) * sh.d_h;
-    for (int i = warp; i < sh.d_h; i += 8) {
-        float acc = 0.f;
-        const bf16* Wi = Ws + (size_t)i * sh.d_c;
+    for (int i0 = warp; i0 < sh.d_h; i0 += 64) {
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         for (int c0 = lane * 8; c0 < sh.d_c; c0 += 256) {
-            const uint4 raw = *(const uint4*)(Wi + c0);
-            const bf16* wv = (const bf16*)&raw;
+            const float4 o0 = *(const float4*)(olat + c0), o1 = *(const float4*)(olat + c0 + 4);
+            const float ov[8] = {o0.x, o0.y, o0.z, o0.w, o1.x, o1.y, o1.z, o1.w};
 #pragma unroll
-            for (int v = 0; v < 8; ++v) acc = fmaf(__bfloat162float(wv[v]), olat[c0 + v], acc);
+            for (int r = 0; r < 8; ++r) {
+                const int i = i0 + r * 8;
+                if (i < sh.d_h) {
+                    const uint4 raw = *(const uint4*)(Ws + (size_t)i * sh.d_c + c0);
+                    const bf16* wv = (const bf16*)&raw;
+#pragma unroll
+                    for (int v = 0; v < 8; ++v) acc[r] = fmaf(__bfloat162float(wv[v]), ov[v], acc[r]);
+                }
+            }
         }
-        acc = warp_sum(acc);
-        if (lane == 0) out[i] = __float2bfloat16_rn(acc);
+#pragma unroll
+        for (int r = 0; r < 8; ++r) acc[r] = warp_sum(acc[r]);
+        if (lane < 8 && i0 + lane * 8 < sh.d_h) {
+            float mine = acc[0];
+#pragma unroll
+            for (int r = 1; r < 8; ++r) mine = lane == r ? acc[r] : mine;
+            out[i0 + lane * 8] = __float2bfloat16_rn(mine);
+        }
     }
 }
 
@@ -565,8 +620,8 @@ size_t attn_smem_bytes(const Shape& sh, int NH) {
     size_t bytes = 1024;                          // alignment slack
     bytes += 2 * nc * 16384;                      // two stages
     bytes += nc * NH * 128;                       // q~
-    bytes += 2 * NH * 128;                        // P^T
-    bytes += 256 + 4 * (size_t)NH * 4 + 2 * (size_t)NH * 4;   // barriers, reductions
+    bytes += 4 * NH * 128;                        // P^T (2 buffers)
+    bytes += sizeof(SmallBars<32>);               // upper bound for every head count
     bytes += ((size_t)sh.B + 1) * 4 + 16;         // tile prefix sums
     return bytes;
 }
@@ -609,15 +664,25 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
-template <int NH>
+template <int NH, int HV>
 cudaError_t launch_attn(const CUtensorMap& map, const DecTC& p, size_t smem, cudaStream_t st) {
     static size_t done[64] = {0};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64) dev = 0;
-    cudaError_t e = ensure_smem(k_dec_attn_sh<NH>, smem, &done[dev]);
+    cudaError_t e = ensure_smem(k_dec_attn_sh<NH, HV>, smem, &done[dev]);
     if (e != cudaSuccess) return note_error("cudaFuncSetAttribute(k_dec_attn_sh)", e);
-    return note_error("k_dec_attn_sh launch", launch_pdl(k_dec_attn_sh<NH>, dim3(p.G), dim3(kThreads), smem, st, map, p));
+    return note_error("k_dec_attn_sh launch",
+                      launch_pdl(k_dec_attn_sh<NH, HV>, dim3(p.G), dim3(kAttnThreads), smem, st, map, p));
+}
+
+cudaError_t launch_attn_any(const CUtensorMap& map, const DecTC& p, size_t smem, cudaStream_t st) {
+    switch (p.Hp) {
+        case 8: return launch_attn<16, 8>(map, p, smem, st);
+        case 16: return launch_attn<16, 16>(map, p, smem, st);
+        case 24: return launch_attn<32, 24>(map, p, smem, st);
+        default: return launch_attn<32, 32>(map, p, smem, st);
+    }
 }
 
 }  // namespace
@@ -659,7 +724,7 @@ static uint32_t qimg_bytes(const Shape& sh) {
 
 size_t tc_decode_workspace(const Shape& sh) {
     return align256((size_t)sh.B * qimg_bytes(sh)) +
-           align256((size_t)(kMaxGrid + sh.B) * sh.H * (sh.d_c + 2) * sizeof(float));
+           align256((size_t)(kMaxGrid + sh.B) * ((sh.H + 7) & ~7) * (sh.d_c + 2) * sizeof(float));
 }
 
 cudaError_t tc_decode(const DecodeArgs& a, cudaStream_t st, uint64_t* launches) {
@@ -688,6 +753,7 @@ cudaError_t tc_decode(const DecodeArgs& a, cudaStream_t st, uint64_t* launches) 
     DecTC p;
     p.B = sh.B;
     p.H = sh.H;
+    p.Hp = (sh.H + 7) & ~7;
     p.D = sh.D;
     p.d_c = sh.d_c;
     p.s = sh.s;
@@ -723,7 +789,7 @@ cudaError_t tc_decode(const DecodeArgs& a, cudaStream_t st, uint64_t* launches) 
     if (e != cudaSuccess) return note_error("k_dec_prep_tc launch", e);
     const size_t smem = attn_smem_bytes(sh, NH);
     profile_begin(st);
-    e = NH == 16 ? launch_attn<16>(map, p, smem, st) : launch_attn<32>(map, p, smem, st);
+    e = launch_attn_any(map, p, smem, st);
     profile_end(st);
     if (e != cudaSuccess) return e;
     const size_t comb_smem = (size_t)sh.d_h * sh.d_c * sizeof(bf16);

@@ -186,13 +186,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
             const uint32_t id_o = idesc_bf16_f32(128, p.d_c, false, true);
             const uint32_t id_out = idesc_bf16_f32(128, p.d_h, false, false);
             const uint32_t ring_a = smem_u32(ring), q_a = smem_u32(q_s), p_a = smem_u32(p_s);
+            const uint64_t q_d = sdesc_sw128(q_a, 16, 1024), p_d = sdesc_sw128(p_a, 16, 1024);
             bool ok = waitb(&bs.abs_full, 0, bs);
             if (ok) {
                 tc_fence_after();
                 // q~ = qC . W_UK[h]: A = qC [128 x d_h] K-major, B = W_UK[h] [d_h x d_c] MN-major
+                const uint64_t wd = sdesc_sw128(q_a, wchunk, 1024);
                 for (int kk = 0; kk < p.d_h / 16; ++kk)
-                    umma_bf16(t_o, sdesc_sw128(p_a + kk * 32, 16, 1024),
-                              sdesc_sw128(q_a + kk * 2048, wchunk, 1024), id_abs, kk > 0);
+                    umma_bf16(t_o, desc_add(p_d, kk * 32), desc_add(wd, kk * 2048), id_abs, kk > 0);
                 umma_commit(&bs.abs_done);
                 ok = waitb(&bs.q_ready, 0, bs);
             }
@@ -201,11 +202,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
                 if (!waitb(&bs.full[st], (k / kStages) & 1, bs)) return false;
                 if (k >= 2 && !waitb(&bs.s_empty[k & 1], ((k - 2) >> 1) & 1, bs)) return false;
                 tc_fence_after();
-                const uint32_t kb = ring_a + st * stage_bytes;
-                for (int c = 0; c < n_chunks; ++c)
+                const uint64_t kd = sdesc_sw128(ring_a + st * stage_bytes, 16, 1024);
+                for (int c = 0; c < n_chunks; ++c) {
+                    const uint64_t qc = desc_add(q_d, c * kQ * 128), kc = desc_add(kd, c * chunk_k);
+#pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        umma_bf16(t_s0 + (k & 1) * 64, sdesc_sw128(q_a + c * kQ * 128 + kk * 32, 16, 1024),
-                                  sdesc_sw128(kb + c * chunk_k + kk * 32, 16, 1024), id_s, (c | kk) != 0);
+                        umma_bf16(t_s0 + (k & 1) * 64, desc_add(qc, kk * 32), desc_add(kc, kk * 32), id_s,
+                                  (c | kk) != 0);
+                }
                 umma_commit(&bs.s_full[k & 1]);
                 return true;
             };
@@ -218,11 +222,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
                 }
                 if (!waitb(&bs.p_full, k & 1, bs)) break;
                 tc_fence_after();
-                const uint32_t kb = ring_a + (k % kStages) * stage_bytes;
+                const uint64_t vd = sdesc_sw128(ring_a + (k % kStages) * stage_bytes, chunk_k, 1024);
                 // O += P . V: A = P [128 x 64] K-major, B = V = key tile latent [64 x d_c] MN-major
+#pragma unroll
                 for (int kk = 0; kk < kKT / 16; ++kk)
-                    umma_bf16(t_o, sdesc_sw128(p_a + kk * 32, 16, 1024),
-                              sdesc_sw128(kb + kk * 2048, chunk_k, 1024), id_o, (k > 0 || kk > 0) ? 1u : 0u);
+                    umma_bf16(t_o, desc_add(p_d, kk * 32), desc_add(vd, kk * 2048), id_o, (k > 0 || kk > 0) ? 1u : 0u);
                 umma_commit(&bs.empty[k % kStages]);
                 umma_commit(&bs.o_done);
             }
@@ -230,10 +234,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
                 tc_fence_after();
                 // out = O_lat . W_UV[h]^T: A = O_lat [128 x d_c] K-major (in the ring),
                 // B = W_UV[h] [d_h x d_c] K-major (in q_s)
+                const uint64_t od = sdesc_sw128(ring_a, 16, 1024);
                 for (int kk = 0; kk < p.d_c / 16; ++kk) {
                     const int c = kk >> 2;
-                    umma_bf16(t_s0, sdesc_sw128(ring_a + c * kQ * 128 + (kk & 3) * 32, 16, 1024),
-                              sdesc_sw128(q_a + c * wchunk + (kk & 3) * 32, 16, 1024), id_out, kk > 0);
+                    umma_bf16(t_s0, desc_add(od, c * kQ * 128 + (kk & 3) * 32),
+                              desc_add(q_d, c * wchunk + (kk & 3) * 32), id_out, kk > 0);
                 }
                 umma_commit(&bs.out_done);
             }

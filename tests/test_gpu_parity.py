@@ -341,3 +341,34 @@ def test_mask_set_bit_exact_speech_widths(s):
                 support = np.nonzero(out[t, h])[0].tolist()
                 assert support == list(range(t // s + 1)), (mode, t, h)
                 np.testing.assert_allclose(out[t, h, : t // s + 1], 1.0 / (t // s + 1), rtol=4e-3)
+
+
+# ----------------------------------------------------------------- many heads (cluster kernel)
+
+@pytest.mark.parametrize("H,s", [(33, 4), (64, 1), (128, 4), (128, 3)])
+def test_decode_many_heads(H, s):
+    """Large-latent widths (d_h=128, d_c=512, d_R=64) with 32 < H <= 128: the
+    decode runs on the two-CTA cluster kernel. Mixed positions put several
+    sequences in one cluster's range and one sequence across clusters."""
+    wl = inputs.LARGE_LATENT.with_(B=12, H=H, s=s)
+    max_slots = 1500
+    w = inputs.weights(wl)
+    toks = inputs.tokens(wl, 1, stream=1)
+    cache0 = inputs.synthetic_cache(wl, max_slots * s - 1, max_slots)
+    rng = np.random.default_rng(H + s)
+    pos = rng.integers(0, max_slots * s, size=wl.B)
+    pos[:4] = [0, s - 1, 63 * s, max_slots * s - 1]
+    pb = Problem(wl, max_slots=max_slots, weights=w)
+    pb.buf.cache.copy_(cache0["cache"].to(pb.dt))
+    pb.buf.open_slot.copy_(cache0["acc"])
+    out = np64(pb.decode(toks, 0, pos))
+    cfg = oracle_cfg(wl)
+    cache_o = cache0["cache"].double().numpy().copy()
+    acc_o = cache0["acc"].double().numpy().copy()
+    ref = oracle.decode_step(cfg, toks["c"][:, 0], toks["kr"][:, 0], toks["qc"][:, 0], toks["qr"][:, 0],
+                             w["w_uk"], w["w_uv"], pos, cache_o, acc_o, gate_in=toks["gate_in"][:, 0])
+    assert rel_err(out, ref["out"]) <= TOL["bf16"]
+    for b in range(wl.B):
+        j = pos[b] // s
+        assert rel_err(np64(pb.buf.cache[b, j]), cache_o[b, j]) <= 4e-3
+    assert rel_err(np64(pb.buf.open_slot), acc_o) <= 1e-5
