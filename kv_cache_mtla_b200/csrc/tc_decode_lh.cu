@@ -26,6 +26,7 @@
 #include <cudaTypedefs.h>
 
 #include <cstdio>
+#include <algorithm>
 #include <utility>
 
 #include <cuda_fp16.h>
@@ -42,8 +43,8 @@ namespace {
 using namespace tc;
 
 constexpr int kKT = 64;          // slots per key tile
-constexpr int kStages = 2;
-constexpr int kThreads = 192;    // warp 0 TMA, warp 1 MMA, warps 2-5 softmax
+constexpr int kStages = 3;
+constexpr int kThreads = 352;    // warp 0 TMA, 1 score MMAs, 2-9 softmax, 10 P.V MMAs
 constexpr int kMaxClusters = 80; // >= SMs/2 of any sm_100 part; sizes the partial buffer
 constexpr int kMaxB = 2048;
 constexpr float kRescaleLog2 = 8.f;
@@ -130,17 +131,41 @@ __global__ void __launch_bounds__(256) k_lh_prep(DecodeArgs a, uint8_t* qimg, in
     __syncthreads();
     bool w_ok = mbar_wait(bar, 0);
     if (!w_ok && threadIdx.x == 0) latch_status(a.status, kStatusTimeout);
+    __shared__ int64_t tpos[32];                                  // position, or -1 if invalid
     for (int c0 = 0; c0 < sh.B && w_ok; c0 += 32) {
-        __syncthreads();                                          // X free
-        for (int e = threadIdx.x; e < sh.d_h * 32; e += blockDim.x) {
-            const int k = e / 32, bb = e % 32, b = c0 + bb;
-            X[e] = b < sh.B ? __bfloat162float(((const bf16*)a.q_c)[((size_t)b * sh.H + h) * sh.d_h + k]) : 0.f;
+        __syncthreads();                                          // X, tpos free
+        if (threadIdx.x < 32) {
+            const int b = c0 + threadIdx.x;
+            const int64_t t = b < sh.B ? (int64_t)a.pos[b] : -1;
+            tpos[threadIdx.x] = lh_pos_ok(sh, t) ? t : -1;
+        }
+        {
+            // X[k][bb] = qC[c0 + bb, h, k]: lane = sequence, so the stores are
+            // conflict-free; every 16-byte load of a thread is issued first
+            const int n8 = sh.d_h / 8;                            // <= 64 -> <= 8 per thread
+            uint4 raw[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int e = threadIdx.x + u * blockDim.x, k8 = e / 32, bb = e % 32, b = c0 + bb;
+                raw[u] = make_uint4(0, 0, 0, 0);
+                if (k8 < n8 && b < sh.B)
+                    raw[u] = *(const uint4*)((const bf16*)a.q_c + ((size_t)b * sh.H + h) * sh.d_h + k8 * 8);
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int e = threadIdx.x + u * blockDim.x, k8 = e / 32, bb = e % 32;
+                if (k8 < n8) {
+                    const bf16* w = (const bf16*)&raw[u];
+#pragma unroll
+                    for (int v = 0; v < 8; ++v) X[(k8 * 8 + v) * 32 + bb] = __bfloat162float(w[v]);
+                }
+            }
         }
         __syncthreads();
         auto emit = [&](auto& acc, int b0, int j0, int bt) {
             for (int i = 0; i < bt; ++i) {
                 const int b = c0 + b0 + i;
-                if (b0 >= 32 || b >= sh.B || !lh_pos_ok(sh, a.pos[b])) continue;
+                if (b0 >= 32 || b >= sh.B || tpos[b0 + i] < 0) continue;
                 uint4 pk;
                 pk.x = pack_bf16x2(acc[i][0], acc[i][1]);
                 pk.y = pack_bf16x2(acc[i][2], acc[i][3]);
@@ -153,25 +178,33 @@ __global__ void __launch_bounds__(256) k_lh_prep(DecodeArgs a, uint8_t* qimg, in
         if (sh.d_c == 512) { float acc[8][8]; head_gemm_32<8>(X, Ws, sh.d_h, sh.d_c, acc, b0, j0); emit(acc, b0, j0, 8); }
         else if (sh.d_c == 256) { float acc[4][8]; head_gemm_32<4>(X, Ws, sh.d_h, sh.d_c, acc, b0, j0); emit(acc, b0, j0, 4); }
         else { float acc[2][8]; head_gemm_32<2>(X, Ws, sh.d_h, sh.d_c, acc, b0, j0); emit(acc, b0, j0, 2); }
-        // rotated part: columns [d_c, n_qchunks*64), zero past D
-        const int nrot = n_qchunks * 64 - sh.d_c;
-        for (int e = threadIdx.x; e < 32 * nrot; e += blockDim.x) {
-            const int bb = e / nrot, jr = e % nrot, b = c0 + bb;
-            if (b >= sh.B) continue;
-            const int64_t t = a.pos[b];
-            if (!lh_pos_ok(sh, t)) continue;
-            float v = 0.f;
-            if (jr < sh.d_r) {
-                const bf16* qr = (const bf16*)a.q_r + ((size_t)b * sh.H + h) * sh.d_r;
-                const int k = jr >> 1;
+        // rotated part: column pairs [d_c, n_qchunks*64), zero past D; a thread
+        // takes up to 4 (sequence, pair) items and issues their loads first
+        const int npair = (n_qchunks * 64 - sh.d_c) / 2;          // <= 32
+        uint32_t qv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int e = threadIdx.x + u * blockDim.x, bb = e / npair, k = e % npair, b = c0 + bb;
+            qv[u] = 0;
+            if (bb < 32 && b < sh.B && 2 * k < sh.d_r)
+                qv[u] = *(const uint32_t*)((const bf16*)a.q_r + ((size_t)b * sh.H + h) * sh.d_r + 2 * k);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int e = threadIdx.x + u * blockDim.x, bb = e / npair, k = e % npair, b = c0 + bb;
+            if (bb >= 32 || b >= sh.B || tpos[bb] < 0) continue;
+            float v0 = 0.f, v1 = 0.f;
+            if (2 * k < sh.d_r) {
                 float sn, cs;
-                pair_sincos(t, k, sh.d_r, sh.log2_rope_base, &sn, &cs);
-                const float x0 = __bfloat162float(qr[2 * k]), x1 = __bfloat162float(qr[2 * k + 1]);
-                v = (jr & 1) ? (x0 * sn + x1 * cs) : (x0 * cs - x1 * sn);
+                pair_sincos(tpos[bb], k, sh.d_r, sh.log2_rope_base, &sn, &cs);
+                const bf16* xq = (const bf16*)&qv[u];
+                const float x0 = __bfloat162float(xq[0]), x1 = __bfloat162float(xq[1]);
+                v0 = x0 * cs - x1 * sn;
+                v1 = x0 * sn + x1 * cs;
             }
-            const int j = sh.d_c + jr;
-            *(bf16*)(qimg + (size_t)b * img_bytes + (size_t)(j >> 6) * 128 * 128 + sw128_offset(h, j & 63)) =
-                __float2bfloat16_rn(v);
+            const int j = sh.d_c + 2 * k;
+            *(uint32_t*)(qimg + (size_t)b * img_bytes + (size_t)(j >> 6) * 128 * 128 + sw128_offset(h, j & 63)) =
+                pack_bf16x2(v0, v1);
         }
     }
     for (int b = h; b < sh.B; b += sh.H) {
@@ -190,14 +223,19 @@ __global__ void __launch_bounds__(256) k_lh_prep(DecodeArgs a, uint8_t* qimg, in
 // ---------------------------------------------------------------- attention
 
 struct LhBars {
-    uint64_t full[kStages], empty[kStages];
-    uint64_t q_full, q_free;
-    uint64_t s_full, s_empty;
-    uint64_t p_full, o_done;
-    uint64_t x_full, x_empty;
+    uint64_t full[kStages], empty[kStages];   // slot-tile ring
+    uint64_t q_full, q_free;                  // query image of the current segment
+    uint64_t s_full[2], s_empty[2];           // partial scores in TMEM, by tile parity
+    uint64_t p_full[2], o_done[2];            // P in TMEM; P.V of tiles with this parity completed
+    uint64_t x_full[2];                       // peer's partial scores landed in x_in[parity] (bulk copy)
+    uint64_t x_free[2];                       // peer has read the scores this CTA sent into its x_in[parity]
+    uint64_t qt_full;                         // query chunks of the segment written to TMEM (8 warps)
+    uint64_t drain[2];                        // MMAs in flight when a wait gave up (per issuing thread)
     uint32_t tmem_base;
     volatile int fail;
     int total;
+    float red[2][2][128];                     // [tile parity][column half][row]: half-row maxima
+    float lsum[2][128];                       // [column half][row]: half-row sums at a segment end
 };
 
 __device__ __forceinline__ bool lh_wait(uint64_t* bar, uint32_t parity, LhBars& bs) {
@@ -223,6 +261,15 @@ __device__ __forceinline__ int lh_chunk_id(int rank, int i, int lat_chunks, int 
 // (128 B), its 16-byte units XOR-swizzled by r mod 8 (conflict-free access).
 __device__ __forceinline__ uint32_t xoff(int r, int unit) { return (uint32_t)r * 128 + (((unit ^ r) & 7) << 4); }
 
+// Attention over 64-slot tiles for one cluster of two CTAs (see the top of the
+// file). Warp 0: TMA; warp 1: MMA issue and TMEM; warps 2-9: softmax, two
+// threads per head row (one per 32-slot half of a tile). The softmax of tile it
+// is split in two halves:
+//   A(it)  read this CTA's partial scores from TMEM, round them (scaled) to
+//          fp16 and send them to the peer (one bulk copy into its x_in);
+//   B(it)  add the peer's partial scores, online softmax, P into TMEM.
+// The order A(it+1), B(it) lets both copies of tile it+1 fly while the CTAs
+// do B(it). Scores, P and x_in are double-buffered; the ring has three stages.
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     k_lh_attn(const __grid_constant__ CUtensorMap tmap, const LhArgs p) {
     extern __shared__ uint8_t smem_raw[];
@@ -234,13 +281,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const int rope_first = p.d_c / 64;                   // first chunk of the RoPE columns
     const int max_chunks = lat_chunks + (p.n_qchunks - rope_first);
     const int my_chunks = rank == 0 ? max_chunks : lat_chunks;
+    // the last n_tq of this CTA's query chunks live in TMEM (the MMA's A from
+    // tensor memory), the first n_sq in shared memory
+    const int n_tq = min(2, my_chunks), n_sq = my_chunks - n_tq;
     const uint32_t stage_bytes = (uint32_t)max_chunks * kKT * 128;
-    uint8_t* q_s = smem;                                             // max_chunks x [128 x 128 B]
-    uint8_t* ring = q_s + (size_t)max_chunks * 128 * 128;            // kStages x stage_bytes
-    uint8_t* p_s = ring + (size_t)kStages * stage_bytes;             // P [128 x 128 B]
-    uint8_t* x_out = p_s + 128 * 128;                                // own scores, fp16 [128 x 128 B]
-    uint8_t* x_in = x_out + 128 * 128;                               // peer scores, fp16 [128 x 128 B]
-    LhBars& bs = *(LhBars*)(x_in + 128 * 128);
+    uint8_t* q_s = smem;                                             // (max_chunks - 2) x [128 x 128 B]
+    uint8_t* ring = q_s + (size_t)max(0, max_chunks - 2) * 128 * 128;   // kStages x stage_bytes
+    uint8_t* x_out = ring + (size_t)kStages * stage_bytes;           // own scores, fp16 [128 x 128 B]
+    uint8_t* x_in = x_out + 128 * 128;                               // peer's scores, 2 x [128 x 128 B]
+    LhBars& bs = *(LhBars*)(x_in + 2 * 128 * 128);
     int* starts = (int*)((uint8_t*)&bs + ((sizeof(LhBars) + 15) & ~(size_t)15));   // [B + 1]
 
     // ---- schedule over 64-slot tiles (reads pos only)
@@ -278,14 +327,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             mbar_init(&bs.full[i], 1);
             mbar_init(&bs.empty[i], 1);
         }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bs.s_full[i], 1);
+            mbar_init(&bs.s_empty[i], 8);
+            mbar_init(&bs.p_full[i], 8);
+            mbar_init(&bs.o_done[i], 1);
+        }
         mbar_init(&bs.q_full, 1);
         mbar_init(&bs.q_free, 1);
-        mbar_init(&bs.s_full, 1);
-        mbar_init(&bs.s_empty, 4);
-        mbar_init(&bs.p_full, 4);
-        mbar_init(&bs.o_done, 1);
-        mbar_init(&bs.x_full, 1);        // local expect_tx arrive; the peer's copy completes the bytes
-        mbar_init(&bs.x_empty, 1);       // one remote arrive per tile from the peer
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bs.x_full[i], 1);     // local expect_tx arrive; the peer's copy completes the bytes
+            mbar_init(&bs.x_free[i], 1);     // one remote arrive from the peer
+        }
+        mbar_init(&bs.qt_full, 8);
+        mbar_init(&bs.drain[0], 1);
+        mbar_init(&bs.drain[1], 1);
         bs.fail = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmap);
@@ -301,7 +357,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     pdl_launch_dependents();
     const uint32_t tmem = bs.tmem_base;
     const uint32_t t_o = tmem;                         // O_c: columns [0, lat_half)
-    const uint32_t t_s = tmem + 256;                   // S: 4 accumulators of 64 columns
+    const uint32_t t_s = tmem + 256;                   // partial scores: 2 x 64 columns
+    const uint32_t t_p = tmem + 384;                   // P (bf16 pairs): 2 x 32 columns
+    const uint32_t t_q = tmem + 448;                   // query chunks (bf16 pairs): 2 x 32 columns
     const int total = bs.total;
     const int gt0 = (int)(((int64_t)g * total) / p.G2);
     const int gt1 = (int)(((int64_t)(g + 1) * total) / p.G2);
@@ -316,23 +374,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     };
     pdl_wait();                          // cache row and query image come from k_lh_prep
 
+    int loads_issued = 0, q_loads = 0;   // producer's copies, for the drain on failure
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            int seg = -1, prev_b = -1;
+            int prev_b = -1;
             for (int gt = gt0, it = 0; gt < gt1; ++gt, ++it) {
                 int b, j;
                 locate(gt, b, j);
                 if (b != prev_b) {
                     prev_b = b;
-                    ++seg;
-                    if (seg >= 1 && !lh_wait(&bs.q_free, (seg - 1) & 1, bs)) break;
-                    mbar_arrive_expect_tx(&bs.q_full, (uint32_t)my_chunks * 128 * 128);
+                    if (q_loads >= 1 && !lh_wait(&bs.q_free, (q_loads - 1) & 1, bs)) break;
+                    mbar_arrive_expect_tx(&bs.q_full, (uint32_t)n_sq * 128 * 128);
                     const uint8_t* src = p.qimg + (size_t)b * p.n_qchunks * 128 * 128;
-                    for (int i = 0; i < my_chunks; ++i)
+                    for (int i = 0; i < n_sq; ++i)
                         bulk_load(q_s + (size_t)i * 128 * 128,
                                   src + (size_t)lh_chunk_id(rank, i, lat_chunks, rope_first) * 128 * 128,
                                   128 * 128, &bs.q_full);
+                    ++q_loads;
                 }
                 const int st = it % kStages;
                 if (it >= kStages && !lh_wait(&bs.empty[st], ((it / kStages) - 1) & 1, bs)) break;
@@ -340,72 +399,172 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 for (int i = 0; i < my_chunks; ++i)
                     tma_load_3d(ring + st * stage_bytes + (size_t)i * kKT * 128, &tmap, &bs.full[st],
                                 lh_chunk_id(rank, i, lat_chunks, rope_first) * 64, j * kKT, b);
+                ++loads_issued;
+                if (gt + kStages < gt1) {
+                    // the tile that takes this stage next: start its trip from HBM into L2
+                    int b2, j2;
+                    locate(gt + kStages, b2, j2);
+                    for (int i = 0; i < my_chunks; ++i)
+                        tma_prefetch_l2_3d(&tmap, lh_chunk_id(rank, i, lat_chunks, rope_first) * 64, j2 * kKT, b2);
+                }
             }
         }
     } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issue
+        // ------------------------------------------------------------ score MMAs
         if (lane == 0) {
             const uint32_t id_s = idesc_bf16_f32(128, kKT, false, false);
-            const uint32_t id_o = idesc_bf16_f32(128, lat_half, false, true);
             const uint32_t ring_a = smem_u32(ring);
-            const uint64_t q_d = sdesc_sw128(smem_u32(q_s), 16, 1024), p_d = sdesc_sw128(smem_u32(p_s), 16, 1024);
-            int seg = -1, prev_b = -1;
-            bool prev_first = true;          // first tile of its segment (for the pending P.V)
-            bool ok = true;
-            int it = 0;
-            auto issue_pv = [&](int k, bool first) -> bool {
-                if (!lh_wait(&bs.p_full, k & 1, bs)) return false;
-                tc_fence_after();
-                const uint64_t vd = sdesc_sw128(ring_a + (k % kStages) * stage_bytes, kKT * 128, 1024);
-#pragma unroll
-                for (int kk = 0; kk < kKT / 16; ++kk)
-                    umma_bf16(t_o, desc_add(p_d, kk * 32), desc_add(vd, kk * 2048), id_o, (first && kk == 0) ? 0u : 1u);
-                umma_commit(&bs.empty[k % kStages]);
-                umma_commit(&bs.o_done);
-                return true;
-            };
-            for (int gt = gt0; gt < gt1 && ok; ++gt, ++it) {
+            const uint64_t q_d = sdesc_sw128(smem_u32(q_s), 16, 1024);
+            int seg = -1, prev_b = -1, it = 0;
+            for (int gt = gt0; gt < gt1; ++gt, ++it) {
                 int b, j;
                 locate(gt, b, j);
-                const bool first = (b != prev_b);
-                if (first) {
+                if (b != prev_b) {
                     prev_b = b;
                     ++seg;
-                    if (!lh_wait(&bs.q_full, seg & 1, bs)) { ok = false; break; }
+                    if (!lh_wait(&bs.q_full, seg & 1, bs)) break;    // q~ chunks in smem
+                    if (!lh_wait(&bs.qt_full, seg & 1, bs)) break;   // q~ chunks in TMEM
                 }
                 const int st = it % kStages;
-                if (!lh_wait(&bs.full[st], (it / kStages) & 1, bs)) { ok = false; break; }
-                if (it >= 1 && !lh_wait(&bs.s_empty, (it - 1) & 1, bs)) { ok = false; break; }
+                if (!lh_wait(&bs.full[st], (it / kStages) & 1, bs)) break;
+                if (it >= 2 && !lh_wait(&bs.s_empty[it & 1], ((it >> 1) - 1) & 1, bs)) break;
                 tc_fence_after();
-                // S_c = q~_c . K_c^T into 4 accumulators (K-steps round robin)
+                // S_c = q~_c . K_c^T (M = 128 heads, N = 64 slots)
                 const uint64_t kd = sdesc_sw128(ring_a + st * stage_bytes, 16, 1024);
-                for (int i = 0; i < my_chunks; ++i) {
+                const uint32_t ts = t_s + (it & 1) * kKT;
+                for (int i = 0; i < n_sq; ++i) {
                     const uint64_t qi = desc_add(q_d, i * 128 * 128), ki = desc_add(kd, i * kKT * 128);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        umma_bf16(t_s + kk * kKT, desc_add(qi, kk * 32), desc_add(ki, kk * 32), id_s, i > 0);
+                        umma_bf16(ts, desc_add(qi, kk * 32), desc_add(ki, kk * 32), id_s, (i | kk) != 0);
                 }
-                umma_commit(&bs.s_full);
+                for (int i = 0; i < n_tq; ++i) {
+                    const uint64_t ki = desc_add(kd, (n_sq + i) * kKT * 128);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_bf16_ts(ts, t_q + i * 32 + kk * 8, desc_add(ki, kk * 32), id_s, (n_sq + i) + kk != 0);
+                }
+                umma_commit(&bs.s_full[it & 1]);
                 const bool last = (gt + 1 == gt1) || (j + 1 == starts[b + 1] - starts[b]);
                 if (last) umma_commit(&bs.q_free);
-                if (it >= 1 && !issue_pv(it - 1, prev_first)) { ok = false; break; }
-                prev_first = first;
             }
-            if (ok && it >= 1) issue_pv(it - 1, prev_first);
+        }
+    } else if (warp == 10) {
+        // ------------------------------------------------------------ P.V MMAs
+        // A second issuing thread, so that P.V (which frees ring stages) never
+        // waits behind score MMAs that wait for a load.
+        if (lane == 0) {
+            const uint32_t id_o = idesc_bf16_f32(128, lat_half, false, true);
+            const uint32_t ring_a = smem_u32(ring);
+            int prev_b = -1, it = 0;
+            for (int gt = gt0; gt < gt1; ++gt, ++it) {
+                int b, j;
+                locate(gt, b, j);
+                const bool first = (b != prev_b);
+                prev_b = b;
+                if (!lh_wait(&bs.p_full[it & 1], (it >> 1) & 1, bs)) break;
+                tc_fence_after();
+                // O_c += P . V_c: A = P in TMEM, B = the tile's latent columns (MN-major)
+                const uint64_t vd = sdesc_sw128(ring_a + (it % kStages) * stage_bytes, kKT * 128, 1024);
+#pragma unroll
+                for (int kk = 0; kk < kKT / 16; ++kk)
+                    umma_bf16_ts(t_o, t_p + (it & 1) * 32 + kk * 8, desc_add(vd, kk * 2048), id_o,
+                                 (first && kk == 0) ? 0u : 1u);
+                umma_commit(&bs.empty[it % kStages]);
+                umma_commit(&bs.o_done[it & 1]);
+            }
         }
     } else {
-        // ------------------------------------------------------------ softmax (thread = head row)
-        // No early exit: every softmax thread passes every named barrier even after a
-        // bounded wait gave up (later waits then return at once), so none can hang.
+        // ------------------------------------------------------------ softmax (two threads per head row)
+        // Warps 2-9: row r = (warp mod 4) * 32 + lane (the TMEM lane quarter a warp
+        // may access), column half hc = (warp - 2) / 4 of each 64-slot tile.
+        // The partial scores travel by one bulk copy per tile from x_out into the
+        // peer's x_in[tile parity]; the copy completes the bytes on the peer's
+        // x_full[parity]. No early exit from the loop: after a bounded wait gave
+        // up, later waits return at once, so no thread is left waiting.
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;
+        const int hc = (warp - 2) >> 2;
+        const int sidx = tid - 64;                     // 0..255 over the softmax warps
+        const bool leader = sidx == 0;
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const uint32_t x_in_peer = map_to_rank(x_in, peer);
-        const uint32_t xfull_peer = map_to_rank(&bs.x_full, peer);
-        const uint32_t xempty_peer = map_to_rank(&bs.x_empty, peer);
-        const bool leader = (tid == 64);
-        float m_ref = -INFINITY, l = 0.f;
+        const uint32_t xfull_peer = map_to_rank(&bs.x_full[0], peer);
+        const uint32_t xfree_peer = map_to_rank(&bs.x_free[0], peer);
+        uint32_t own[16];        // this thread's 32 scaled partial scores of the newest tile, fp16 pairs
+        uint32_t own_prev[16];   // ... of the tile B works on
+        // Query chunks n_sq.. of sequence b into TMEM: the thread of row r and
+        // half hc writes chunk n_sq + hc of row r (de-swizzled from the image).
+        auto load_qt = [&](int b) {
+            if (hc < n_tq) {
+                const uint8_t* src = p.qimg + (size_t)b * p.n_qchunks * 128 * 128 +
+                                     (size_t)lh_chunk_id(rank, n_sq + hc, lat_chunks, rope_first) * 128 * 128 +
+                                     (size_t)r * 128;
+                uint32_t w[32];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const uint4 v = *(const uint4*)(src + (((u ^ r) & 7) << 4));
+                    w[4 * u] = v.x;
+                    w[4 * u + 1] = v.y;
+                    w[4 * u + 2] = v.z;
+                    w[4 * u + 3] = v.w;
+                }
+                tmem_st32_u(t_q + hc * 32 + lane_off, w);
+                tmem_wait_st();
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bs.qt_full);
+        };
+        // A(k): partial scores of tile k -> own[], x_out, and the peer's x_in[k & 1]
+        auto half_a = [&](int k) {
+            lh_wait(&bs.s_full[k & 1], (k >> 1) & 1, bs);
+            tc_fence_after();
+            float sv[32];
+            tmem_ld32(t_s + (k & 1) * kKT + hc * 32 + lane_off, sv);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bs.s_empty[k & 1]);
+            if (gt0 + k + 1 < gt1) {
+                // S(k) is complete, so every score MMA that read the TMEM query chunks
+                // is done; if tile k+1 opens a new segment, bring in its query
+                int b1, j1;
+                locate(gt0 + k + 1, b1, j1);
+                if (j1 == 0) load_qt(b1);
+            }
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                const __half2 h2 = __floats2half2_rn(sv[2 * c] * p.scale_log2, sv[2 * c + 1] * p.scale_log2);
+                own[c] = *(const uint32_t*)&h2;
+            }
+            if (leader) {
+                bulk_wait_read_all();                               // the copy of tile k-1 has read x_out
+                if (!bs.fail) mbar_arrive_expect_tx(&bs.x_full[k & 1], 128 * 128);   // the peer's tile k
+            }
+            named_sync(1, 256);
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                *(uint4*)(x_out + xoff(r, 4 * hc + u)) =
+                    make_uint4(own[4 * u], own[4 * u + 1], own[4 * u + 2], own[4 * u + 3]);
+            fence_proxy_async();
+            named_sync(1, 256);
+            if (leader) {
+                // the peer's x_in[k & 1] was read by its B(k - 2)
+                if (k < 2 || lh_wait_cluster(&bs.x_free[k & 1], ((k >> 1) - 1) & 1, bs)) {
+                    bulk_copy_to_peer(x_in_peer + (k & 1) * 128 * 128, x_out, 128 * 128, xfull_peer + (k & 1) * 8);
+                    bulk_commit_group();
+                }
+            }
+        };
+        float m_ref = -INFINITY, l = 0.f;              // l: this thread's half of the row sum
         int prev_b = -1, n_b = 0, k_in_seg = 0;
+        if (gt0 < gt1) {
+            int b0, j0;
+            locate(gt0, b0, j0);
+            load_qt(b0);
+            half_a(0);
+        }
         for (int gt = gt0, it = 0; gt < gt1; ++gt, ++it) {
             int b, j;
             locate(gt, b, j);
@@ -416,160 +575,144 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 l = 0.f;
                 k_in_seg = 0;
             }
+#pragma unroll
+            for (int c = 0; c < 16; ++c) own_prev[c] = own[c];
+            if (gt + 1 < gt1) half_a(it + 1);       // the peer's copy of tile it+1 overlaps B(it)
             const int st = it % kStages;
-            const int valid = min(kKT, n_b - j * kKT);
-            if (leader && !bs.fail) mbar_arrive_expect_tx(&bs.x_full, 128 * 128);   // peer's scores, this tile
-            lh_wait(&bs.s_full, it & 1, bs);    // on a timeout: keep going, the status is latched
-            tc_fence_after();
-            float sv[kKT];
-            {
-                float tmp[32];
+            const int valid = min(kKT, n_b - j * kKT) - hc * 32;   // valid columns of this half
+            // B(it): add the peer's partial scores of this tile (a + b = b + a
+            // exactly, so both CTAs hold the same scores)
+            lh_wait(&bs.x_full[it & 1], (it >> 1) & 1, bs);
+            const uint8_t* xin = x_in + (it & 1) * 128 * 128;
+            uint4 th[4];
 #pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    tmem_ld32(t_s + h2 * 32 + lane_off, sv + h2 * 32);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int q = 1; q < 4; ++q) {
-                        tmem_ld32(t_s + q * kKT + h2 * 32 + lane_off, tmp);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) sv[h2 * 32 + i] += tmp[i];
-                    }
-                }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bs.s_empty);
-            // stale rows past the sequence's last slot must not reach P.V
-            if (valid < kKT) {
-                const int rows = kKT - valid;
-                uint8_t* stg = ring + st * stage_bytes;
-                for (int e = tid - 64; e < my_chunks * rows * 8; e += 128) {
-                    const int i = e / (rows * 8), rr = e % (rows * 8);
-                    *(uint4*)(stg + (size_t)i * kKT * 128 + (size_t)(valid + rr / 8) * 128 + (rr % 8) * 16) =
-                        make_uint4(0, 0, 0, 0);
-                }
-            }
-            // own scaled partial scores as fp16 (both CTAs use the rounded values)
-            if (it >= 1 && leader) bulk_wait_read_all();    // x_out free again
-            named_sync(1, 128);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                uint4 pk;
-                __half2 h0 = __floats2half2_rn(sv[8 * u + 0] * p.scale_log2, sv[8 * u + 1] * p.scale_log2);
-                __half2 h1 = __floats2half2_rn(sv[8 * u + 2] * p.scale_log2, sv[8 * u + 3] * p.scale_log2);
-                __half2 h2 = __floats2half2_rn(sv[8 * u + 4] * p.scale_log2, sv[8 * u + 5] * p.scale_log2);
-                __half2 h3 = __floats2half2_rn(sv[8 * u + 6] * p.scale_log2, sv[8 * u + 7] * p.scale_log2);
-                pk.x = *(uint32_t*)&h0;
-                pk.y = *(uint32_t*)&h1;
-                pk.z = *(uint32_t*)&h2;
-                pk.w = *(uint32_t*)&h3;
-                *(uint4*)(x_out + xoff(r, u)) = pk;
-            }
-            fence_proxy_async();
-            named_sync(1, 128);
-            if (leader) {
-                if (it == 0 || lh_wait_cluster(&bs.x_empty, (it - 1) & 1, bs)) {
-                    bulk_copy_to_peer(x_in_peer, x_out, 128 * 128, xfull_peer);
-                    bulk_commit_group();
-                }
-            }
-            lh_wait_cluster(&bs.x_full, it & 1, bs);
+            for (int u = 0; u < 4; ++u) th[u] = *(const uint4*)(xin + xoff(r, 4 * hc + u));
+            float sv[32];
             float mt = -INFINITY;
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const uint4 mine = *(const uint4*)(x_out + xoff(r, u));
-                const uint4 theirs = *(const uint4*)(x_in + xoff(r, u));
-                const __half2* hm = (const __half2*)&mine;
-                const __half2* ht = (const __half2*)&theirs;
+            for (int u = 0; u < 4; ++u) {
+                const uint32_t tw[4] = {th[u].x, th[u].y, th[u].z, th[u].w};
 #pragma unroll
                 for (int v = 0; v < 4; ++v) {
-                    const float2 fm = __half22float2(hm[v]), ft = __half22float2(ht[v]);
+                    const float2 fm = __half22float2(*(const __half2*)&own_prev[4 * u + v]);
+                    const float2 ft = __half22float2(*(const __half2*)&tw[v]);
                     const int c = 8 * u + 2 * v;
-                    const float s0 = rank == 0 ? fm.x + ft.x : ft.x + fm.x;
-                    const float s1 = rank == 0 ? fm.y + ft.y : ft.y + fm.y;
-                    sv[c] = (c < valid) ? s0 : -INFINITY;
-                    sv[c + 1] = (c + 1 < valid) ? s1 : -INFINITY;
+                    sv[c] = c < valid ? fm.x + ft.x : -INFINITY;
+                    sv[c + 1] = c + 1 < valid ? fm.y + ft.y : -INFINITY;
                     mt = fmaxf(mt, fmaxf(sv[c], sv[c + 1]));
                 }
             }
-            named_sync(1, 128);                              // every row of x_in read
-            if (leader) mbar_arrive_remote(xempty_peer);
-            float m_new = m_ref, fac = 1.f;
-            if (mt > m_ref + kRescaleLog2 || m_ref == -INFINITY) {
-                m_new = mt;
-                fac = (m_ref == -INFINITY) ? 0.f : exp2f(m_ref - mt);
-            }
+            bs.red[it & 1][hc][r] = mt;
+            named_sync(1, 256);                        // also: every thread has read x_in[it & 1]
+            if (leader) mbar_arrive_remote_relaxed(xfree_peer + (it & 1) * 8);
+            mt = fmaxf(mt, bs.red[it & 1][hc ^ 1][r]);
+            // lazy rescale: the reference maximum moves only when the tile's maximum
+            // exceeds it by more than 2^8 (P stays <= 256); both halves decide alike
+            const bool upd = mt > m_ref + kRescaleLog2;
+            const float nm = upd ? mt : m_ref;
+            const float fac = ex2_approx(m_ref - nm);    // 0 when m_ref was -inf, 1 when kept
             float rs = 0.f;
+            uint32_t pk[16];
 #pragma unroll
-            for (int c = 0; c < kKT; ++c) {
-                sv[c] = exp2f(sv[c] - m_new);
-                rs += sv[c];
+            for (int c = 0; c < 16; ++c) {
+                const float p0 = ex2_approx(sv[2 * c] - nm), p1 = ex2_approx(sv[2 * c + 1] - nm);
+                rs += p0 + p1;
+                pk[c] = pack_bf16x2(p0, p1);
             }
-            l = l * fac + rs;
-            if (it >= 1) {
-                lh_wait(&bs.o_done, (it - 1) & 1, bs);
+            l = fmaf(l, fac, rs);
+            m_ref = nm;
+            const bool need = upd && k_in_seg > 0;
+            if (__any_sync(0xffffffffu, need)) {
+                // this warp's rows of its half of O_c move to their new reference maxima
+                lh_wait(&bs.o_done[(it - 1) & 1], ((it - 1) >> 1) & 1, bs);
                 tc_fence_after();
-                if (k_in_seg > 0 && __any_sync(0xffffffffu, fac != 1.f)) {
-                    float v[32];
-                    for (int cc = 0; cc < lat_half / 32; ++cc) {
-                        tmem_ld32(t_o + cc * 32 + lane_off, v);
-                        tmem_wait_ld();
+                const float f = need ? fac : 1.f;
+                const int cols = lat_half / 2;
+                float v[32];
+                for (int cc = 0; cc < cols / 32; ++cc) {
+                    const uint32_t ta = t_o + hc * cols + cc * 32 + lane_off;
+                    tmem_ld32(ta, v);
+                    tmem_wait_ld();
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) v[i] *= fac;
-                        tmem_st32(t_o + cc * 32 + lane_off, v);
-                    }
-                    tmem_wait_st();
+                    for (int i = 0; i < 32; ++i) v[i] *= f;
+                    tmem_st32(ta, v);
+                }
+                tmem_wait_st();
+            }
+            if (valid + hc * 32 < kKT) {
+                // stale rows past the sequence's last slot must not reach P.V
+                const int v0 = valid + hc * 32, rows = kKT - v0;
+                uint8_t* stg = ring + st * stage_bytes;
+                for (int e = sidx; e < my_chunks * rows * 8; e += 256) {
+                    const int i = e / (rows * 8), rr = e % (rows * 8);
+                    *(uint4*)(stg + (size_t)i * kKT * 128 + (size_t)(v0 + rr / 8) * 128 + (rr % 8) * 16) =
+                        make_uint4(0, 0, 0, 0);
                 }
             }
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                uint4 pk;
-                pk.x = pack_bf16x2(sv[8 * u + 0], sv[8 * u + 1]);
-                pk.y = pack_bf16x2(sv[8 * u + 2], sv[8 * u + 3]);
-                pk.z = pack_bf16x2(sv[8 * u + 4], sv[8 * u + 5]);
-                pk.w = pack_bf16x2(sv[8 * u + 6], sv[8 * u + 7]);
-                *(uint4*)(p_s + sw128_offset(r, 8 * u)) = pk;
-            }
+            if (it >= 2) lh_wait(&bs.o_done[it & 1], ((it >> 1) - 1) & 1, bs);   // P.V of tile it-2 read this P buffer
+            tmem_st16_u(t_p + (it & 1) * 32 + hc * 16 + lane_off, pk);
+            tmem_wait_st();
             fence_proxy_async();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bs.p_full);
-            m_ref = m_new;
+            if (lane == 0) mbar_arrive(&bs.p_full[it & 1]);
             ++k_in_seg;
             const bool last = (gt + 1 == gt1) || (j + 1 == starts[b + 1] - starts[b]);
             if (last) {
                 // partial of this sequence segment: this CTA's half of O, plus (m, l)
-                lh_wait(&bs.o_done, it & 1, bs);
+                bs.lsum[hc][r] = l;
+                lh_wait(&bs.o_done[it & 1], (it >> 1) & 1, bs);
                 tc_fence_after();
+                named_sync(1, 256);
                 const size_t row = (size_t)p.d_c + 4;
                 float* dst = p.part + ((size_t)(g + b) * p.H + r) * row;
+                const int cols = lat_half / 2;
                 float v[32];
-                for (int cc = 0; cc < lat_half / 32; ++cc) {
-                    tmem_ld32(t_o + cc * 32 + lane_off, v);
+                for (int cc = 0; cc < cols / 32; ++cc) {
+                    tmem_ld32(t_o + hc * cols + cc * 32 + lane_off, v);
                     tmem_wait_ld();
                     if (r < p.H) {
 #pragma unroll
                         for (int u = 0; u < 8; ++u)
-                            *(float4*)(dst + rank * lat_half + cc * 32 + 4 * u) =
+                            *(float4*)(dst + rank * lat_half + hc * cols + cc * 32 + 4 * u) =
                                 make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
                     }
                 }
-                if (rank == 0 && r < p.H) {
+                if (rank == 0 && hc == 0 && r < p.H) {
                     dst[p.d_c] = m_ref;
-                    dst[p.d_c + 1] = l;
+                    dst[p.d_c + 1] = l + bs.lsum[1][r];
                 }
                 tc_fence_before();
             }
         }
-        if (leader) bulk_wait_read_all();
     }
-    if (bs.fail && (tid & 63) == 0) latch_status(p.status, kStatusTimeout);
     tc_fence_before();
     __syncthreads();
+    if (bs.fail) {
+        // a bounded wait gave up: let this CTA's copies and MMAs land (bounded
+        // again) before shared memory and TMEM are released, then report
+        if (warp == 0 && lane == 0) {
+            for (int k = max(0, loads_issued - kStages); k < loads_issued; ++k)
+                mbar_wait(&bs.full[k % kStages], (k / kStages) & 1);
+            if (q_loads > 0) mbar_wait(&bs.q_full, (q_loads - 1) & 1);
+        }
+        if ((warp == 1 || warp == 10) && lane == 0) {
+            uint64_t* d = &bs.drain[warp == 1 ? 0 : 1];
+            umma_commit(d);              // arrives when this thread's MMAs are done
+            mbar_wait(d, 0);
+        }
+        if (tid == 64) {
+            // the peer's score copies into this CTA, and this CTA's own copies
+            const int n = gt1 - gt0;
+            for (int k = max(0, n - 2); k < n; ++k) mbar_wait(&bs.x_full[k & 1], (k >> 1) & 1);
+            bulk_wait_read_all();
+        }
+        if (tid == 0) latch_status(p.status, kStatusTimeout);
+        __syncthreads();
+    }
     tc_fence_after();
     if (warp == 1) tmem_dealloc(tmem, 512);
-    cluster_sync();                      // the peer may still copy into / arrive on us until here
+    cluster_sync();                      // the peer may still store into / arrive on us until here
 }
 
 // ---------------------------------------------------------------- combine
@@ -621,7 +764,9 @@ __global__ void __launch_bounds__(256) k_lh_combine(DecodeArgs a, LhArgs p) {
     __shared__ float invl[32];
     __shared__ int maxn_s;
     {
-        // transpose W_UV[h] [d_h][d_c] into [d_c][d_h]; 8 loads in flight per thread
+        // transpose W_UV[h] [d_h][d_c] into [d_c][d_h]; 8 loads in flight per thread.
+        // Consecutive threads take consecutive rows i, so the 2-byte stores of a
+        // warp land in consecutive shared-memory words (no bank conflicts).
         const bf16* src = (const bf16*)a.w_uv + (size_t)h * sh.d_h * sh.d_c;
         const int n16 = sh.d_h * sh.d_c / 8;
         for (int e0 = threadIdx.x; e0 < n16; e0 += 8 * blockDim.x) {
@@ -629,13 +774,14 @@ __global__ void __launch_bounds__(256) k_lh_combine(DecodeArgs a, LhArgs p) {
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const int e = e0 + u * blockDim.x;
-                if (e < n16) raw[u] = *(const uint4*)(src + (size_t)e * 8);
+                const int i = e % sh.d_h, k0 = (e / sh.d_h) * 8;
+                if (e < n16) raw[u] = *(const uint4*)(src + (size_t)i * sh.d_c + k0);
             }
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const int e = e0 + u * blockDim.x;
                 if (e < n16) {
-                    const int i = (e * 8) / sh.d_c, k0 = (e * 8) % sh.d_c;
+                    const int i = e % sh.d_h, k0 = (e / sh.d_h) * 8;
                     const bf16* w = (const bf16*)&raw[u];
 #pragma unroll
                     for (int v = 0; v < 8; ++v) Wt[(size_t)(k0 + v) * sh.d_h + i] = w[v];
@@ -737,10 +883,9 @@ size_t lh_attn_smem(const Shape& sh) {
     const int lat_chunks = sh.d_c / 128;
     const int max_chunks = lat_chunks + (sh.D / 64 - sh.d_c / 64);
     size_t bytes = 1024;
-    bytes += (size_t)max_chunks * 128 * 128;            // q~ chunks
+    bytes += (size_t)std::max(0, max_chunks - 2) * 128 * 128;   // q~ chunks in shared memory
     bytes += (size_t)kStages * max_chunks * kKT * 128;  // key tiles
-    bytes += 128 * 128;                                 // P
-    bytes += 2 * 128 * 128;                             // exchanged scores (own, peer), fp16
+    bytes += 3 * 128 * 128;                             // exchanged scores (own; peer's x 2), fp16
     bytes += ((sizeof(LhBars) + 15) & ~(size_t)15) + ((size_t)sh.B + 1) * 4;
     return bytes;
 }
