@@ -43,6 +43,25 @@ METRIC = "decode latent-cache GB/s and tokens/s at N/s slots; prefill TFLOP/s; %
 WL = inputs.SPEECH_DECODE
 
 
+def _traffic(kernel):
+    """DRAM bytes (read + write) of one launch of `kernel` from the committed ncu
+    capture, or None when the kernel's sources changed since the capture."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)[kernel]
+        h = hashlib.sha256()
+        for src in rec["sources"]:
+            with open(os.path.join(ROOT, src), "rb") as f:
+                h.update(f.read())
+        if h.hexdigest() != rec["sources_sha256"]:
+            return None
+        return rec["dram_bytes_read"] + rec["dram_bytes_write"]
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def _peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -95,7 +114,7 @@ class ClockSampler:
         try:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=self.f, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
@@ -335,7 +354,7 @@ def run_kernel_workload(args, ws, rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=60)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="mtla", choices=["mtla", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -478,7 +497,7 @@ def main():
             "prefill": {"ms": statistics.mean(pre_ms), "attention_kernel_ms": statistics.mean(pre_attn),
                         "TFLOPs": pre_flops / (statistics.mean(pre_ms) / 1e3) / 1e12},
             "roofline": {"kernel": "decode attention", "bound": "hbm", "achieved": achieved,
-                         "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "traffic": None,
+                         "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "traffic": _traffic("k_dec_attn_sh"),
                          "peak_source": f"{peak_kind} hbm_gbs",
                          "bytes_per_launch": bytes_per_launch, "avg_launch_us": attn_ms * 1e3,
                          "timing": "CUDA event pairs recorded by the library around each of the "
