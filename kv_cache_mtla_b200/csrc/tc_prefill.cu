@@ -13,15 +13,19 @@
 //   k_prefill_tc                one CTA per (query tile of 128 positions,
 //                               sequence, head), heaviest tiles first:
 //     absorption   q~ = qC . W_UK[h]          tcgen05 M=128 N=d_c K=d_h
-//     own partial  2 tiles of 64 rows of P     diagonal mask
+//     own partial  one dot product q~ . P_t per row on the CUDA cores; it is
+//                  the softmax's starting point and its value P_t enters the
+//                  output at the end with the row's final weight
 //     finished     64-slot tiles of cache_out  staircase mask on the last
-//                  S = q~ . K^T (M=128 N=64 K=D), online softmax (thread per
-//                  row, exp2, rescale only when a row max grows by > 2^8),
-//                  O += P . V (M=128 N=d_c K=64, V = the same smem tile)
+//                  S = q~ . K^T (M=128 N=64 K=D), online softmax (two threads
+//                  per row, exp2, rescale only when a row max grows by > 2^8),
+//                  O += P . V (M=128 N=d_c K=64, P in TMEM, V = the same tile)
 //     epilogue     out = (O / l) . W_UV[h]^T   tcgen05 M=128 N=d_h K=d_c
-// Warp roles: warp 0 TMA, warp 1 MMA issue and TMEM, warps 2-5 softmax. S is
-// double-buffered in TMEM so S(k+1) runs on the tensor cores while the
-// softmax of tile k runs; keys stream through a 3-stage TMA ring.
+// Warp roles: warp 0 TMA, warp 1 absorption / score / output MMAs and TMEM,
+// warps 2-9 softmax, warp 10 P.V MMAs (so P.V, which frees ring stages, never
+// waits behind a score MMA that waits for a load). S and P are double-
+// buffered in TMEM, two query chunks live in TMEM (the MMA's A from tensor
+// memory), and keys stream through a 4-stage TMA ring.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -40,8 +44,8 @@ using namespace tc;
 
 constexpr int kQ = 128;         // query positions per CTA
 constexpr int kKT = 64;         // keys per tile
-constexpr int kStages = 3;
-constexpr int kThreads = 192;   // 6 warps
+constexpr int kStages = 4;
+constexpr int kThreads = 352;   // warp 0 TMA, 1 score MMAs, 2-9 softmax, 10 P.V MMAs
 constexpr float kRescaleLog2 = 8.f;
 
 struct PreTC {
@@ -51,6 +55,7 @@ struct PreTC {
     float scale_log2;
     double log2_rope_base;
     const bf16* q_r;  // [B, T, H, d_r]
+    const bf16* P;    // [B, T, D]: partial slots from the scan (the own-slot keys)
     bf16* out;        // [B, T, H, d_h]
     int* status;
 };
@@ -59,9 +64,13 @@ struct Bars {
     uint64_t full[kStages], empty[kStages];
     uint64_t abs_full, abs_done, q_ready;
     uint64_t s_full[2], s_empty[2];
-    uint64_t p_full, o_done, fin_s, wuv_full, olat_ready, out_done;
+    uint64_t p_full[2], o_done[2];
+    uint64_t fin_s, wuv_full, olat_ready, out_done;
+    uint64_t drain[2];
     uint32_t tmem_base;
     volatile int fail;
+    float red[2][2][kQ];      // [tile parity][column half][row]: half-row maxima
+    float xs[2][kQ];          // [column half][row]: own-slot score halves, then row-sum halves
 };
 
 struct Maps {
@@ -69,7 +78,6 @@ struct Maps {
     CUtensorMap wuk;    // (d_c, d_h, H)    box (64, d_h, 1)
     CUtensorMap wuv;    // (d_c, d_h, H)    box (64, d_h, 1)
     CUtensorMap slots;  // (D, n_slots, B)  box (64, 64, 1)
-    CUtensorMap part;   // (D, T, B)        box (64, 64, 1)
 };
 
 __device__ __forceinline__ bool waitb(uint64_t* bar, uint32_t parity, Bars& bs) {
@@ -95,16 +103,38 @@ __device__ __forceinline__ void st_row32_bf16(uint8_t* base, uint32_t chunk_byte
     }
 }
 
+// 32 values as 16 packed bf16 pairs (lower element in the lower half).
+__device__ __forceinline__ void pack32(const float* v, uint32_t* w) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+}
+
+// 32 bf16 of a global row (16-byte aligned) as fp32.
+__device__ __forceinline__ void ld_row32_bf16(const bf16* src, float* v) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const uint4 raw = *(const uint4*)(src + 8 * u);
+        const bf16* e = (const bf16*)&raw;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[8 * u + i] = __bfloat162float(e[i]);
+    }
+}
+
+// One CTA per (128 query positions, sequence, head), heaviest first. The own
+// partial slot of every row is handled on the CUDA cores (its score is one dot
+// product per row; its value enters the output at the end with the row's final
+// weight); the finished slots stream through the tensor cores in 64-slot tiles.
 __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constant__ Maps maps, const PreTC p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const int n_chunks = p.n_chunks;
+    const int n_sq = n_chunks - 2;                                       // query chunks in smem; 2 in TMEM
     const uint32_t chunk_k = kKT * 128;                                  // one 64-row chunk of a key tile
     const uint32_t stage_bytes = (uint32_t)n_chunks * chunk_k;
     uint8_t* ring = smem;                                                // kStages key tiles
-    uint8_t* q_s = ring + kStages * stage_bytes;                         // n_chunks x [128 x 128 B]
-    uint8_t* p_s = q_s + (size_t)n_chunks * kQ * 128;                    // [128 x 128 B]
-    Bars& bs = *(Bars*)(p_s + kQ * 128);
+    uint8_t* q_s = ring + kStages * stage_bytes;                         // n_sq x [128 x 128 B]; W_UK, W_UV
+    uint8_t* qc_s = ring + (kStages - 1) * stage_bytes;                  // qC tile, before key tile kStages-1
+    Bars& bs = *(Bars*)(q_s + (size_t)n_sq * kQ * 128);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int per_qt = p.B * p.H;
@@ -114,7 +144,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
     const int p0 = qt * kQ;
     const int last = min(p0 + kQ - 1, p.T - 1);
     const int nft = (last / p.s + kKT - 1) / kKT;                        // finished-slot tiles
-    const int n_tiles = 2 + nft;
     const int dc_chunks = p.d_c / 64;
     const uint32_t wchunk = (uint32_t)p.d_h * 128;                       // one 64-column chunk of W
 
@@ -125,16 +154,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
         }
         mbar_init(&bs.abs_full, 1);
         mbar_init(&bs.abs_done, 1);
-        mbar_init(&bs.q_ready, 4);
+        mbar_init(&bs.q_ready, 8);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bs.s_full[i], 1);
-            mbar_init(&bs.s_empty[i], 4);
+            mbar_init(&bs.s_empty[i], 8);
+            mbar_init(&bs.p_full[i], 8);
+            mbar_init(&bs.o_done[i], 1);
+            mbar_init(&bs.drain[i], 1);
         }
-        mbar_init(&bs.p_full, 4);
-        mbar_init(&bs.o_done, 1);
         mbar_init(&bs.fin_s, 1);
         mbar_init(&bs.wuv_full, 1);
-        mbar_init(&bs.olat_ready, 4);
+        mbar_init(&bs.olat_ready, 8);
         mbar_init(&bs.out_done, 1);
         bs.fail = 0;
         fence_mbar_init();
@@ -147,30 +177,27 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bs.tmem_base;
-    const uint32_t t_s0 = tmem;            // S buffers: columns [0, 64) and [64, 128)
-    const uint32_t t_o = tmem + 128;       // q~, then O: columns [128, 128 + d_c)
+    const uint32_t t_s0 = tmem;            // S buffers: columns [0, 64) and [64, 128); later the output
+    const uint32_t t_o = tmem + 128;       // q~ (absorption), then O: columns [128, 128 + d_c)
+    const uint32_t t_p = tmem + 384;       // P (bf16 pairs): 2 x 32 columns
+    const uint32_t t_q = tmem + 448;       // query chunks n_sq, n_sq + 1 (bf16 pairs): 2 x 32 columns
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             tma_prefetch_desc(&maps.qc);
             tma_prefetch_desc(&maps.slots);
-            tma_prefetch_desc(&maps.part);
             mbar_arrive_expect_tx(&bs.abs_full, kQ * 128 + dc_chunks * wchunk);
-            tma_load_4d(p_s, &maps.qc, &bs.abs_full, 0, h, p0, b);
+            tma_load_4d(qc_s, &maps.qc, &bs.abs_full, 0, h, p0, b);
             for (int n = 0; n < dc_chunks; ++n) tma_load_3d(q_s + n * wchunk, &maps.wuk, &bs.abs_full, n * 64, 0, h);
-            for (int k = 0; k < n_tiles; ++k) {
+            for (int k = 0; k < nft; ++k) {
                 const int st = k % kStages;
                 if (k >= kStages && !waitb(&bs.empty[st], ((k / kStages) - 1) & 1, bs)) break;
+                if (k == kStages - 1 && !waitb(&bs.abs_done, 0, bs)) break;    // qC has been read
                 mbar_arrive_expect_tx(&bs.full[st], stage_bytes);
                 uint8_t* dst = ring + st * stage_bytes;
-                if (k < 2) {
-                    for (int c = 0; c < n_chunks; ++c)
-                        tma_load_3d(dst + c * chunk_k, &maps.part, &bs.full[st], c * 64, p0 + kKT * k, b);
-                } else {
-                    for (int c = 0; c < n_chunks; ++c)
-                        tma_load_3d(dst + c * chunk_k, &maps.slots, &bs.full[st], c * 64, kKT * (k - 2), b);
-                }
+                for (int c = 0; c < n_chunks; ++c)
+                    tma_load_3d(dst + c * chunk_k, &maps.slots, &bs.full[st], c * 64, kKT * k, b);
             }
             if (waitb(&bs.fin_s, 0, bs)) {
                 mbar_arrive_expect_tx(&bs.wuv_full, dc_chunks * wchunk);
@@ -179,57 +206,47 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
             }
         }
     } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issue
+        // ------------------------------------------------------------ absorption, score and output MMAs
         if (lane == 0) {
             const uint32_t id_abs = idesc_bf16_f32(128, p.d_c, false, true);
             const uint32_t id_s = idesc_bf16_f32(128, kKT, false, false);
-            const uint32_t id_o = idesc_bf16_f32(128, p.d_c, false, true);
             const uint32_t id_out = idesc_bf16_f32(128, p.d_h, false, false);
-            const uint32_t ring_a = smem_u32(ring), q_a = smem_u32(q_s), p_a = smem_u32(p_s);
-            const uint64_t q_d = sdesc_sw128(q_a, 16, 1024), p_d = sdesc_sw128(p_a, 16, 1024);
+            const uint32_t ring_a = smem_u32(ring), q_a = smem_u32(q_s);
+            const uint64_t q_d = sdesc_sw128(q_a, 16, 1024), qc_d = sdesc_sw128(smem_u32(qc_s), 16, 1024);
             bool ok = waitb(&bs.abs_full, 0, bs);
             if (ok) {
                 tc_fence_after();
                 // q~ = qC . W_UK[h]: A = qC [128 x d_h] K-major, B = W_UK[h] [d_h x d_c] MN-major
                 const uint64_t wd = sdesc_sw128(q_a, wchunk, 1024);
                 for (int kk = 0; kk < p.d_h / 16; ++kk)
-                    umma_bf16(t_o, desc_add(p_d, kk * 32), desc_add(wd, kk * 2048), id_abs, kk > 0);
+                    umma_bf16(t_o, desc_add(qc_d, kk * 32), desc_add(wd, kk * 2048), id_abs, kk > 0);
                 umma_commit(&bs.abs_done);
                 ok = waitb(&bs.q_ready, 0, bs);
             }
-            auto issue_s = [&](int k) -> bool {
+            for (int k = 0; ok && k < nft; ++k) {
                 const int st = k % kStages;
-                if (!waitb(&bs.full[st], (k / kStages) & 1, bs)) return false;
-                if (k >= 2 && !waitb(&bs.s_empty[k & 1], ((k - 2) >> 1) & 1, bs)) return false;
+                if (!waitb(&bs.full[st], (k / kStages) & 1, bs)) break;
+                if (k >= 2 && !waitb(&bs.s_empty[k & 1], ((k >> 1) - 1) & 1, bs)) break;
                 tc_fence_after();
+                // S = q~ . K^T (M = 128 queries, N = 64 slots, K = D)
                 const uint64_t kd = sdesc_sw128(ring_a + st * stage_bytes, 16, 1024);
-                for (int c = 0; c < n_chunks; ++c) {
+                const uint32_t ts = t_s0 + (k & 1) * 64;
+                for (int c = 0; c < n_sq; ++c) {
                     const uint64_t qc = desc_add(q_d, c * kQ * 128), kc = desc_add(kd, c * chunk_k);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        umma_bf16(t_s0 + (k & 1) * 64, desc_add(qc, kk * 32), desc_add(kc, kk * 32), id_s,
-                                  (c | kk) != 0);
+                        umma_bf16(ts, desc_add(qc, kk * 32), desc_add(kc, kk * 32), id_s, (c | kk) != 0);
+                }
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    const uint64_t kc = desc_add(kd, (n_sq + c) * chunk_k);
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        umma_bf16_ts(ts, t_q + c * 32 + kk * 8, desc_add(kc, kk * 32), id_s, (n_sq + c) + kk != 0);
                 }
                 umma_commit(&bs.s_full[k & 1]);
-                return true;
-            };
-            if (ok) ok = issue_s(0);
-            for (int k = 0; ok && k < n_tiles; ++k) {
-                if (k + 1 < n_tiles) {
-                    if (!issue_s(k + 1)) break;
-                } else {
-                    umma_commit(&bs.fin_s);
-                }
-                if (!waitb(&bs.p_full, k & 1, bs)) break;
-                tc_fence_after();
-                const uint64_t vd = sdesc_sw128(ring_a + (k % kStages) * stage_bytes, chunk_k, 1024);
-                // O += P . V: A = P [128 x 64] K-major, B = V = key tile latent [64 x d_c] MN-major
-#pragma unroll
-                for (int kk = 0; kk < kKT / 16; ++kk)
-                    umma_bf16(t_o, desc_add(p_d, kk * 32), desc_add(vd, kk * 2048), id_o, (k > 0 || kk > 0) ? 1u : 0u);
-                umma_commit(&bs.empty[k % kStages]);
-                umma_commit(&bs.o_done);
             }
+            umma_commit(&bs.fin_s);      // every score MMA is done: q_s may take W_UV
             if (!bs.fail && waitb(&bs.olat_ready, 0, bs) && waitb(&bs.wuv_full, 0, bs)) {
                 tc_fence_after();
                 // out = O_lat . W_UV[h]^T: A = O_lat [128 x d_c] K-major (in the ring),
@@ -243,148 +260,224 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
                 umma_commit(&bs.out_done);
             }
         }
-    } else {
-        // ------------------------------------------------------------ softmax warps
-        const int quarter = warp & 3;                 // TMEM lanes this warp may access
-        const int r = quarter * 32 + lane;            // query row of this thread
-        const int pos = p0 + r;
-        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-        float v[32];
-        // q~ (latent part) from TMEM, RoPE part from qR, into the K-major Q tile
-        if (waitb(&bs.abs_done, 0, bs)) {
-            tc_fence_after();
-            for (int cc = 0; cc < p.d_c / 32; ++cc) {
-                tmem_ld32(t_o + cc * 32 + lane_off, v);
-                tmem_wait_ld();
-                st_row32_bf16(q_s, kQ * 128, r, cc * 32, v);
-            }
-            const int dpad = n_chunks * 64;
-            for (int c0 = p.d_c; c0 < dpad; c0 += 32) {
+    } else if (warp == 10) {
+        // ------------------------------------------------------------ P.V MMAs (own thread: they free
+        // ring stages, so they never wait behind a score MMA that waits for a load)
+        if (lane == 0) {
+            const uint32_t id_o = idesc_bf16_f32(128, p.d_c, false, true);
+            const uint32_t ring_a = smem_u32(ring);
+            for (int k = 0; k < nft; ++k) {
+                if (!waitb(&bs.p_full[k & 1], (k >> 1) & 1, bs)) break;
+                tc_fence_after();
+                // O += P . V: A = P [128 x 64] in TMEM, B = V = key tile latent [64 x d_c] MN-major
+                const uint64_t vd = sdesc_sw128(ring_a + (k % kStages) * stage_bytes, chunk_k, 1024);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] = 0.f;
-                if (pos < p.T) {
-                    const bf16* qr = p.q_r + (((size_t)b * p.T + pos) * p.H + h) * p.d_r;
-#pragma unroll
-                    for (int i = 0; i < 32; i += 2) {
-                        const int e = c0 - p.d_c + i;        // rope element index
-                        if (e < p.d_r) {
-                            float sn, cs;
-                            pair_sincos(pos, e >> 1, p.d_r, p.log2_rope_base, &sn, &cs);
-                            const float x0 = __bfloat162float(qr[e]), x1 = __bfloat162float(qr[e + 1]);
-                            v[i] = x0 * cs - x1 * sn;
-                            v[i + 1] = x0 * sn + x1 * cs;
-                        }
-                    }
-                }
-                st_row32_bf16(q_s, kQ * 128, r, c0, v);
+                for (int kk = 0; kk < kKT / 16; ++kk)
+                    umma_bf16_ts(t_o, t_p + (k & 1) * 32 + kk * 8, desc_add(vd, kk * 2048), id_o,
+                                 (k > 0 || kk > 0) ? 1u : 0u);
+                umma_commit(&bs.empty[k % kStages]);
+                umma_commit(&bs.o_done[k & 1]);
             }
         }
+    } else {
+        // ------------------------------------------------------------ softmax warps (2-9)
+        // Row r = (warp mod 4) * 32 + lane (the TMEM lane quarter a warp may
+        // access); hc = (warp - 2) / 4 picks the column half of every tile. No
+        // early exit: after a bounded wait gave up, later waits return at once and
+        // every thread still meets every named barrier.
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;
+        const int hc = (warp - 2) >> 2;
+        const int pos = p0 + r;
+        const bool row_ok = pos < p.T;
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        const bf16* prow = p.P + ((size_t)b * p.T + min(pos, p.T - 1)) * p.D;   // own partial slot
+        float v[32], pv[32];
+        uint32_t w[16];
+        // q~ row: latent part from TMEM (this thread's column half), RoPE part
+        // (hc = 1) from qR; rounded to bf16 into the smem or TMEM query chunks.
+        // The own-slot score q~ . P_pos uses the same rounded values.
+        auto put_q = [&](int col) {
+            const int c = col >> 6;
+            if (c < n_sq) {
+                st_row32_bf16(q_s, kQ * 128, r, col, v);
+            } else {
+                pack32(v, w);
+                tmem_st16_u(t_q + (c - n_sq) * 32 + (col & 63) / 2 + lane_off, w);
+            }
+        };
+        float e_own = 0.f;
+        waitb(&bs.abs_done, 0, bs);
+        tc_fence_after();
+        {
+            const int half = p.d_c / 2;
+            for (int cc = hc * half; cc < (hc + 1) * half; cc += 32) {
+                tmem_ld32(t_o + cc + lane_off, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = __bfloat162float(__float2bfloat16_rn(v[i]));
+                put_q(cc);
+                ld_row32_bf16(prow + cc, pv);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) e_own = fmaf(v[i], pv[i], e_own);
+            }
+            if (hc == 1) {
+                for (int c0 = p.d_c; c0 < n_chunks * 64; c0 += 32) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = 0.f;
+                    if (row_ok) {
+                        const bf16* qr = p.q_r + (((size_t)b * p.T + pos) * p.H + h) * p.d_r;
+#pragma unroll
+                        for (int i = 0; i < 32; i += 2) {
+                            const int e = c0 - p.d_c + i;        // RoPE element index
+                            if (e < p.d_r) {
+                                float sn, cs;
+                                pair_sincos(pos, e >> 1, p.d_r, p.log2_rope_base, &sn, &cs);
+                                const float x0 = __bfloat162float(qr[e]), x1 = __bfloat162float(qr[e + 1]);
+                                v[i] = __bfloat162float(__float2bfloat16_rn(x0 * cs - x1 * sn));
+                                v[i + 1] = __bfloat162float(__float2bfloat16_rn(x0 * sn + x1 * cs));
+                            }
+                        }
+                    }
+                    put_q(c0);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (c0 + i < p.D) e_own = fmaf(v[i], __bfloat162float(prow[c0 + i]), e_own);
+                }
+            }
+        }
+        tmem_wait_st();
         fence_proxy_async();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bs.q_ready);
-
-        float m_ref = -INFINITY, l = 0.f;
+        bs.xs[hc][r] = e_own;
+        named_sync(1, 256);
+        const float es = row_ok ? (bs.xs[0][r] + bs.xs[1][r]) * p.scale_log2 : 0.f;
+        named_sync(1, 256);                           // xs is free again
+        // online softmax over the finished-slot tiles; the own slot is the
+        // starting point (reference maximum es, weight 1 in the row sum)
+        float m_ref = es, l = hc == 0 ? 1.f : 0.f;    // l: this thread's half of the row sum
         const int fin_lim = pos / p.s;                // finished slots this row may see
-        for (int k = 0; k < n_tiles; ++k) {
-            if (!waitb(&bs.s_full[k & 1], (k >> 1) & 1, bs)) break;
+        for (int k = 0; k < nft; ++k) {
+            waitb(&bs.s_full[k & 1], (k >> 1) & 1, bs);
             tc_fence_after();
-            float sv[kKT];
-            tmem_ld32(t_s0 + (k & 1) * 64 + lane_off, sv);
-            tmem_ld32(t_s0 + (k & 1) * 64 + 32 + lane_off, sv + 32);
+            float sv[32];
+            tmem_ld32(t_s0 + (k & 1) * 64 + hc * 32 + lane_off, sv);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bs.s_empty[k & 1]);
+            const int j0 = kKT * k + 32 * hc;
             float mt = -INFINITY;
-            if (k < 2) {
 #pragma unroll
-                for (int c = 0; c < kKT; ++c) {
-                    sv[c] = (c + kKT * k == r) ? sv[c] * p.scale_log2 : -INFINITY;
-                    mt = fmaxf(mt, sv[c]);
-                }
-            } else {
-                const int j0 = kKT * (k - 2);
-#pragma unroll
-                for (int c = 0; c < kKT; ++c) {
-                    sv[c] = (j0 + c < fin_lim) ? sv[c] * p.scale_log2 : -INFINITY;
-                    mt = fmaxf(mt, sv[c]);
-                }
+            for (int c = 0; c < 32; ++c) {
+                sv[c] = (j0 + c < fin_lim) ? sv[c] * p.scale_log2 : -INFINITY;
+                mt = fmaxf(mt, sv[c]);
             }
-            float m_new = m_ref, fac = 1.f;
-            if (mt > m_ref + kRescaleLog2 || (m_ref == -INFINITY && mt > -INFINITY)) {
-                m_new = mt;
-                fac = (m_ref == -INFINITY) ? 0.f : exp2f(m_ref - mt);
-            }
-            const float mu = (m_new == -INFINITY) ? 0.f : m_new;
+            bs.red[k & 1][hc][r] = mt;
+            named_sync(1, 256);
+            mt = fmaxf(mt, bs.red[k & 1][hc ^ 1][r]);
+            // lazy rescale: the reference maximum moves only when the tile's maximum
+            // exceeds it by more than 2^8 (P stays <= 256); both halves decide alike
+            const bool upd = mt > m_ref + kRescaleLog2;
+            const float nm = upd ? mt : m_ref;
+            const float fac = ex2_approx(m_ref - nm);
             float rs = 0.f;
 #pragma unroll
-            for (int c = 0; c < kKT; ++c) {
-                sv[c] = exp2f(sv[c] - mu);
-                rs += sv[c];
+            for (int c = 0; c < 16; ++c) {
+                const float q0 = ex2_approx(sv[2 * c] - nm), q1 = ex2_approx(sv[2 * c + 1] - nm);
+                rs += q0 + q1;
+                w[c] = pack_bf16x2(q0, q1);
             }
-            l = l * fac + rs;
-            if (k >= 1) {
-                if (!waitb(&bs.o_done, (k - 1) & 1, bs)) break;
+            l = fmaf(l, fac, rs);
+            const bool need = upd && k > 0;           // O holds tiles 0..k-1
+            if (__any_sync(0xffffffffu, need)) {
+                waitb(&bs.o_done[(k - 1) & 1], ((k - 1) >> 1) & 1, bs);
                 tc_fence_after();
-                if (__any_sync(0xffffffffu, fac != 1.f)) {
-                    for (int cc = 0; cc < p.d_c / 32; ++cc) {
-                        tmem_ld32(t_o + cc * 32 + lane_off, v);
-                        tmem_wait_ld();
+                const float f = need ? fac : 1.f;
+                const int half = p.d_c / 2;
+                for (int cc = hc * half; cc < (hc + 1) * half; cc += 32) {
+                    tmem_ld32(t_o + cc + lane_off, v);
+                    tmem_wait_ld();
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) v[i] *= fac;
-                        tmem_st32(t_o + cc * 32 + lane_off, v);
-                    }
-                    tmem_wait_st();
+                    for (int i = 0; i < 32; ++i) v[i] *= f;
+                    tmem_st32(t_o + cc + lane_off, v);
                 }
+                tmem_wait_st();
             }
-            st_row32_bf16(p_s, 0, r, 0, sv);
-            st_row32_bf16(p_s, 0, r, 32, sv + 32);
-            fence_proxy_async();
+            if (k >= 2) waitb(&bs.o_done[k & 1], ((k >> 1) - 1) & 1, bs);   // P.V of tile k-2 read this P buffer
+            tmem_st16_u(t_p + (k & 1) * 32 + hc * 16 + lane_off, w);
+            tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bs.p_full);
-            m_ref = m_new;
+            if (lane == 0) mbar_arrive(&bs.p_full[k & 1]);
+            m_ref = nm;
         }
-        // epilogue: O / l -> bf16 K-major O_lat (in the ring), then out
-        if (waitb(&bs.o_done, (n_tiles - 1) & 1, bs)) {
-            tc_fence_after();
-            const float inv = 1.f / l;
-            for (int cc = 0; cc < p.d_c / 32; ++cc) {
-                tmem_ld32(t_o + cc * 32 + lane_off, v);
-                tmem_wait_ld();
+        // epilogue: O_lat = (O + w_own P_pos[:d_c]) / l -> bf16 K-major (in the ring), then out
+        if (nft > 0) waitb(&bs.o_done[(nft - 1) & 1], ((nft - 1) >> 1) & 1, bs);
+        tc_fence_after();
+        bs.xs[hc][r] = l;
+        named_sync(1, 256);
+        const float inv = 1.f / (bs.xs[0][r] + bs.xs[1][r]);
+        const float w_own = ex2_approx(es - m_ref);
+        {
+            const int half = p.d_c / 2;
+            for (int cc = hc * half; cc < (hc + 1) * half; cc += 32) {
+                if (nft > 0) {
+                    tmem_ld32(t_o + cc + lane_off, v);
+                    tmem_wait_ld();
+                } else {
 #pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] *= inv;
-                st_row32_bf16(ring, kQ * 128, r, cc * 32, v);
+                    for (int i = 0; i < 32; ++i) v[i] = 0.f;
+                }
+                ld_row32_bf16(prow + cc, pv);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = fmaf(w_own, pv[i], v[i]) * inv;
+                st_row32_bf16(ring, kQ * 128, r, cc, v);
             }
         }
         fence_proxy_async();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bs.olat_ready);
-        if (waitb(&bs.out_done, 0, bs)) {
-            tc_fence_after();
-            for (int cc = 0; cc < p.d_h / 32; ++cc) {
-                tmem_ld32(t_s0 + cc * 32 + lane_off, v);
-                tmem_wait_ld();
-                if (pos < p.T) {
-                    bf16* o = p.out + (((size_t)b * p.T + pos) * p.H + h) * p.d_h + cc * 32;
+        waitb(&bs.out_done, 0, bs);
+        tc_fence_after();
+        for (int cc = hc * (p.d_h / 2); cc < (hc + 1) * (p.d_h / 2); cc += 32) {
+            tmem_ld32(t_s0 + cc + lane_off, v);
+            tmem_wait_ld();
+            if (row_ok) {
+                bf16* o = p.out + (((size_t)b * p.T + pos) * p.H + h) * p.d_h + cc;
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        uint4 pk;
-                        pk.x = pack_bf16x2(v[8 * u + 0], v[8 * u + 1]);
-                        pk.y = pack_bf16x2(v[8 * u + 2], v[8 * u + 3]);
-                        pk.z = pack_bf16x2(v[8 * u + 4], v[8 * u + 5]);
-                        pk.w = pack_bf16x2(v[8 * u + 6], v[8 * u + 7]);
-                        *(uint4*)(o + 8 * u) = pk;
-                    }
+                for (int u = 0; u < 4; ++u) {
+                    uint4 pk;
+                    pk.x = pack_bf16x2(v[8 * u + 0], v[8 * u + 1]);
+                    pk.y = pack_bf16x2(v[8 * u + 2], v[8 * u + 3]);
+                    pk.z = pack_bf16x2(v[8 * u + 4], v[8 * u + 5]);
+                    pk.w = pack_bf16x2(v[8 * u + 6], v[8 * u + 7]);
+                    *(uint4*)(o + 8 * u) = pk;
                 }
             }
         }
     }
-    if (bs.fail && tid == 0) latch_status(p.status, kStatusTimeout);
     tc_fence_before();
     __syncthreads();
+    if (bs.fail) {
+        // a bounded wait gave up: let the copies and MMAs in flight land (bounded
+        // again) before shared memory and TMEM are released, then report
+        if ((warp == 1 || warp == 10) && lane == 0) {
+            uint64_t* d = &bs.drain[warp == 1 ? 0 : 1];
+            umma_commit(d);
+            mbar_wait(d, 0);
+        }
+        if (warp == 0 && lane == 0) {
+            for (int k = max(0, nft - kStages); k < nft; ++k) mbar_wait(&bs.full[k % kStages], (k / kStages) & 1);
+            mbar_wait(&bs.abs_full, 0);
+            mbar_wait(&bs.wuv_full, 0);
+        }
+        if (tid == 0) latch_status(p.status, kStatusTimeout);
+        __syncthreads();
+    }
     tc_fence_after();
     if (warp == 1) tmem_dealloc(tmem, 512);
 }
@@ -395,7 +488,7 @@ int n_chunks_of(const Shape& sh) { return (sh.D + 63) / 64; }
 
 size_t prefill_smem_bytes(const Shape& sh) {
     const size_t nc = n_chunks_of(sh);
-    return 1024 + kStages * nc * kKT * 128 + nc * kQ * 128 + kQ * 128 + ((sizeof(Bars) + 15) & ~(size_t)15);
+    return 1024 + kStages * nc * kKT * 128 + (nc - 2) * kQ * 128 + ((sizeof(Bars) + 15) & ~(size_t)15);
 }
 
 cudaError_t make_map(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* m, const void* base, int rank,
@@ -415,7 +508,8 @@ cudaError_t make_map(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* m, cons
 }  // namespace
 
 bool tc_prefill_supported(const Shape& sh) {
-    return sh.d_h == 64 && sh.d_c % 64 == 0 && sh.d_c <= 256 && n_chunks_of(sh) <= 5 &&
+    // d_c >= 128: the smem query chunks also hold W_UK and W_UV
+    return sh.d_h == 64 && sh.d_c % 64 == 0 && sh.d_c >= 128 && sh.d_c <= 256 && n_chunks_of(sh) <= 5 &&
            prefill_smem_bytes(sh) <= 232448 - 1024;
 }
 
@@ -453,10 +547,6 @@ cudaError_t tc_prefill(const PrefillArgs& a, cudaStream_t st, uint64_t* launches
         cuuint32_t bx[3] = {64, kKT, 1};
         cudaError_t e = make_map(enc, &maps.slots, a.cache_out, 3, d, s, bx, "cache_out");
         if (e != cudaSuccess) return e;
-        cuuint64_t d2[3] = {(cuuint64_t)sh.D, (cuuint64_t)T, (cuuint64_t)sh.B};
-        cuuint64_t s2[2] = {E * sh.D, E * T * sh.D};
-        e = make_map(enc, &maps.part, P, 3, d2, s2, bx, "partials");
-        if (e != cudaSuccess) return e;
     }
     PreTC p;
     p.B = sh.B;
@@ -472,6 +562,7 @@ cudaError_t tc_prefill(const PrefillArgs& a, cudaStream_t st, uint64_t* launches
     p.scale_log2 = sh.scale * 1.4426950408889634f;
     p.log2_rope_base = sh.log2_rope_base;
     p.q_r = (const bf16*)a.q_r;
+    p.P = P;
     p.out = (bf16*)a.out;
     p.status = a.status;
 
