@@ -298,6 +298,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const uint32_t id_o = idesc_bf16_f32(128, NH, true, false);
             const uint64_t q_d = sdesc_sw128(smem_u32(q_s), 16, 1024);
             const uint32_t ring_a = smem_u32(ring), p_a = smem_u32(p_s);
+            const int last_ksteps = (p.D - 64 * (n_chunks - 1)) / 16;   // D is a multiple of 16
             int seg = -1, prev_b = -1;
             bool prev_first = true, ok = true;
             int it = 0;
@@ -336,9 +337,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 const uint64_t a0 = sdesc_sw128(ring_a + st * stage_bytes, 16, 1024);
                 for (int c = 0; c < n_chunks; ++c) {
                     const uint64_t ac = desc_add(a0, c * 16384), bc = desc_add(q_d, c * NH * 128);
+                    // K-steps past D (the zero-filled tail of the last chunk) are skipped
+                    const int kst = c == n_chunks - 1 ? last_ksteps : 4;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        umma_bf16(t_s + st * NH, desc_add(ac, kk * 32), desc_add(bc, kk * 32), id_s, (c | kk) != 0);
+                        if (kk < kst)
+                            umma_bf16(t_s + st * NH, desc_add(ac, kk * 32), desc_add(bc, kk * 32), id_s, (c | kk) != 0);
                 }
                 umma_commit(&bs.s_full[st]);
                 const bool last = (gt + 1 == gt1) || (j + 1 == starts[b + 1] - starts[b]);

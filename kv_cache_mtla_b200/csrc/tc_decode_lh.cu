@@ -415,6 +415,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const uint32_t id_s = idesc_bf16_f32(128, kKT, false, false);
             const uint32_t ring_a = smem_u32(ring);
             const uint64_t q_d = sdesc_sw128(smem_u32(q_s), 16, 1024);
+            const int last_ksteps = (p.D - 64 * (p.n_qchunks - 1)) / 16;   // D is a multiple of 16
             int seg = -1, prev_b = -1, it = 0;
             for (int gt = gt0; gt < gt1; ++gt, ++it) {
                 int b, j;
@@ -440,9 +441,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 }
                 for (int i = 0; i < n_tq; ++i) {
                     const uint64_t ki = desc_add(kd, (n_sq + i) * kKT * 128);
+                    // K-steps past D (the zero-filled tail of the last chunk) are skipped
+                    const int kst = lh_chunk_id(rank, n_sq + i, lat_chunks, rope_first) == p.n_qchunks - 1 ? last_ksteps : 4;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        umma_bf16_ts(ts, t_q + i * 32 + kk * 8, desc_add(ki, kk * 32), id_s, (n_sq + i) + kk != 0);
+                        if (kk < kst)
+                            umma_bf16_ts(ts, t_q + i * 32 + kk * 8, desc_add(ki, kk * 32), id_s, (n_sq + i) + kk != 0);
                 }
                 umma_commit(&bs.s_full[it & 1]);
                 const bool last = (gt + 1 == gt1) || (j + 1 == starts[b + 1] - starts[b]);

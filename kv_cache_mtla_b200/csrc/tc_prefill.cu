@@ -213,6 +213,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
             const uint32_t id_out = idesc_bf16_f32(128, p.d_h, false, false);
             const uint32_t ring_a = smem_u32(ring), q_a = smem_u32(q_s);
             const uint64_t q_d = sdesc_sw128(q_a, 16, 1024), qc_d = sdesc_sw128(smem_u32(qc_s), 16, 1024);
+            const int last_ksteps = (p.D - 64 * (n_chunks - 1)) / 16;   // D is a multiple of 16
             bool ok = waitb(&bs.abs_full, 0, bs);
             if (ok) {
                 tc_fence_after();
@@ -240,9 +241,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
 #pragma unroll
                 for (int c = 0; c < 2; ++c) {
                     const uint64_t kc = desc_add(kd, (n_sq + c) * chunk_k);
+                    // K-steps past D (the zero-filled tail of the last chunk) are skipped
+                    const int kst = c == 1 ? last_ksteps : 4;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        umma_bf16_ts(ts, t_q + c * 32 + kk * 8, desc_add(kc, kk * 32), id_s, (n_sq + c) + kk != 0);
+                        if (kk < kst)
+                            umma_bf16_ts(ts, t_q + c * 32 + kk * 8, desc_add(kc, kk * 32), id_s, (n_sq + c) + kk != 0);
                 }
                 umma_commit(&bs.s_full[k & 1]);
             }
