@@ -86,9 +86,11 @@ def _dist():
 
 
 def _max_over_ranks(x: float, ws: int) -> float:
+    """The largest of every rank's x (all ranks call it, in the same order)."""
     if ws == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.cuda.is_available() else "cpu"   # cpu: gloo process groups
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
 
@@ -96,7 +98,14 @@ def _max_over_ranks(x: float, ws: int) -> float:
 def _barrier(ws: int):
     if ws > 1:
         torch.distributed.barrier()
-    torch.cuda.synchronize()
+    if torch.cuda.is_available():
+        torch.cuda.synchronize()
+
+
+def job_value(units_per_rank_step: float, ws: int, steps: int, max_ms: float) -> float:
+    """Whole-job throughput: the units all ranks processed over the slowest
+    rank's device time (weak scaling: every rank has the same per-step work)."""
+    return units_per_rank_step * ws * steps / (max_ms / 1e3)
 
 
 class ClockSampler:
@@ -440,7 +449,7 @@ def main():
     pre_ms = [a.elapsed_time(b) for a, b, c in evs]
     dec_ms = [b.elapsed_time(c) for a, b, c in evs]
     total_ms = _max_over_ranks(sum(step_ms), ws)
-    value = rep.tokens_per_step * ws * args.steps / (total_ms / 1e3)
+    value = job_value(rep.tokens_per_step, ws, args.steps, total_ms)
 
     # dominant kernel: decode attention, from the profiled replay's event pairs
     durs = prof.durations_ms()
