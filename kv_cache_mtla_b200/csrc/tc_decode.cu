@@ -42,7 +42,7 @@ namespace {
 using namespace tc;
 
 constexpr int kTileSlots = 128;
-constexpr int kAttnThreads = 192;   // warps 0-3 softmax, 4 TMA, 5 MMA
+constexpr int kAttnThreads = 224;   // warps 0-3 softmax, 4 TMA, 5 score MMAs, 6 P.V MMAs
 constexpr float kRescaleLog2 = 8.f;
 constexpr int kMaxGrid = 160;  // >= SMs of any sm_100 part; sizes the partial buffer
 constexpr int kMaxB = 2048;
@@ -155,7 +155,7 @@ struct SmallBars {
     uint64_t s_full[2], s_empty[2];      // S^T buffers
     uint64_t p_full[2];                  // P^T buffers (4 softmax warps arrive)
     uint64_t o_done[2];                  // P.V of tiles with this parity completed
-    uint64_t drain;                      // MMAs in flight when a wait gave up
+    uint64_t drain[2];                   // MMAs in flight when a wait gave up (per issuing thread)
     uint32_t tmem_base;
     volatile int fail;
     int total;
@@ -236,7 +236,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         mbar_init(&bs.q_full, 1);
         mbar_init(&bs.q_free, 1);
-        mbar_init(&bs.drain, 1);
+        mbar_init(&bs.drain[0], 1);
+        mbar_init(&bs.drain[1], 1);
         bs.fail = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmap);
@@ -289,49 +290,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     tma_load_3d(ring + st * stage_bytes + (size_t)c * 16384, &tmap, &bs.full[st], c * 64,
                                 j * kTileSlots, b);
                 ++loads_issued;
+
             }
         }
     } else if (warp == 5) {
-        // ------------------------------------------------------------ MMA issue
+        // ------------------------------------------------------------ score MMAs
         if (lane == 0) {
             const uint32_t id_s = idesc_bf16_f32(128, NH, false, false);
-            const uint32_t id_o = idesc_bf16_f32(128, NH, true, false);
             const uint64_t q_d = sdesc_sw128(smem_u32(q_s), 16, 1024);
-            const uint32_t ring_a = smem_u32(ring), p_a = smem_u32(p_s);
+            const uint32_t ring_a = smem_u32(ring);
             const int last_ksteps = (p.D - 64 * (n_chunks - 1)) / 16;   // D is a multiple of 16
-            int seg = -1, prev_b = -1;
-            bool prev_first = true, ok = true;
-            int it = 0;
-            // O^T += V^T . P^T for tile k (A = the slot tile, MN-major; B = P^T, K-major)
-            auto issue_pv = [&](int k, bool first) -> bool {
-                if (!sb_wait(&bs.p_full[k & 1], (k >> 1) & 1, bs)) return false;
-                tc_fence_after();
-                const uint64_t a0 = sdesc_sw128(ring_a + (k & 1) * stage_bytes, 16384, 1024);
-                const uint64_t b0 = sdesc_sw128(p_a + (k & 1) * 2 * NH * 128, 16, 1024);
-                for (int lb = 0; lb < p.lat_blocks; ++lb) {
-                    const uint64_t al = desc_add(a0, 2 * lb * 16384);
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        umma_bf16(t_o + lb * NH, desc_add(al, kk * 2048),
-                                  desc_add(b0, (kk >> 2) * NH * 128 + (kk & 3) * 32), id_o,
-                                  (first && kk == 0) ? 0u : 1u);
-                }
-                umma_commit(&bs.empty[k & 1]);
-                umma_commit(&bs.o_done[k & 1]);
-                return true;
-            };
+            int seg = -1, prev_b = -1, it = 0;
             for (int gt = gt0; gt < gt1; ++gt, ++it) {
                 int b, j;
                 locate(gt, b, j);
-                const bool first = (b != prev_b);
-                if (first) {
+                if (b != prev_b) {
                     prev_b = b;
                     ++seg;
-                    if (!sb_wait(&bs.q_full, seg & 1, bs)) { ok = false; break; }
+                    if (!sb_wait(&bs.q_full, seg & 1, bs)) break;
                 }
                 const int st = it & 1;
-                if (!sb_wait(&bs.full[st], (it >> 1) & 1, bs)) { ok = false; break; }
-                if (it >= 2 && !sb_wait(&bs.s_empty[st], ((it >> 1) - 1) & 1, bs)) { ok = false; break; }
+                if (!sb_wait(&bs.full[st], (it >> 1) & 1, bs)) break;
+                if (it >= 2 && !sb_wait(&bs.s_empty[st], ((it >> 1) - 1) & 1, bs)) break;
                 tc_fence_after();
                 // S^T = K_tile . q~^T (A = slot tile, B = q~ image; both K-major)
                 const uint64_t a0 = sdesc_sw128(ring_a + st * stage_bytes, 16, 1024);
@@ -347,10 +327,36 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 umma_commit(&bs.s_full[st]);
                 const bool last = (gt + 1 == gt1) || (j + 1 == starts[b + 1] - starts[b]);
                 if (last) umma_commit(&bs.q_free);
-                if (it >= 1 && !issue_pv(it - 1, prev_first)) { ok = false; break; }
-                prev_first = first;
             }
-            if (ok && it >= 1) issue_pv(it - 1, prev_first);
+        }
+    } else if (warp == 6) {
+        // ------------------------------------------------------------ P.V MMAs (own thread: they free
+        // ring stages, so they never wait behind a score MMA that waits for a load)
+        if (lane == 0) {
+            const uint32_t id_o = idesc_bf16_f32(128, NH, true, false);
+            const uint32_t ring_a = smem_u32(ring), p_a = smem_u32(p_s);
+            int prev_b = -1, k = 0;
+            for (int gt = gt0; gt < gt1; ++gt, ++k) {
+                int b, j;
+                locate(gt, b, j);
+                const bool first = (b != prev_b);
+                prev_b = b;
+                if (!sb_wait(&bs.p_full[k & 1], (k >> 1) & 1, bs)) break;
+                tc_fence_after();
+                // O^T += V^T . P^T (A = the slot tile, MN-major; B = P^T, K-major)
+                const uint64_t a0 = sdesc_sw128(ring_a + (k & 1) * stage_bytes, 16384, 1024);
+                const uint64_t b0 = sdesc_sw128(p_a + (k & 1) * 2 * NH * 128, 16, 1024);
+                for (int lb = 0; lb < p.lat_blocks; ++lb) {
+                    const uint64_t al = desc_add(a0, 2 * lb * 16384);
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk)
+                        umma_bf16(t_o + lb * NH, desc_add(al, kk * 2048),
+                                  desc_add(b0, (kk >> 2) * NH * 128 + (kk & 3) * 32), id_o,
+                                  (first && kk == 0) ? 0u : 1u);
+                }
+                umma_commit(&bs.empty[k & 1]);
+                umma_commit(&bs.o_done[k & 1]);
+            }
         }
     } else {
         // ------------------------------------------------------------ softmax (warps 0-3)
@@ -486,9 +492,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             for (int k = max(0, loads_issued - 2); k < loads_issued; ++k) mbar_wait(&bs.full[k & 1], (k >> 1) & 1);
             if (q_loads > 0) mbar_wait(&bs.q_full, (q_loads - 1) & 1);
         }
-        if (warp == 5 && lane == 0) {
-            umma_commit(&bs.drain);
-            mbar_wait(&bs.drain, 0);
+        if ((warp == 5 || warp == 6) && lane == 0) {
+            uint64_t* d = &bs.drain[warp - 5];
+            umma_commit(d);              // arrives when this thread's MMAs are done
+            mbar_wait(d, 0);
         }
         if (tid == 0) latch_status(p.status, kStatusTimeout);
         __syncthreads();

@@ -400,13 +400,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     tma_load_3d(ring + st * stage_bytes + (size_t)i * kKT * 128, &tmap, &bs.full[st],
                                 lh_chunk_id(rank, i, lat_chunks, rope_first) * 64, j * kKT, b);
                 ++loads_issued;
-                if (gt + kStages < gt1) {
-                    // the tile that takes this stage next: start its trip from HBM into L2
-                    int b2, j2;
-                    locate(gt + kStages, b2, j2);
-                    for (int i = 0; i < my_chunks; ++i)
-                        tma_prefetch_l2_3d(&tmap, lh_chunk_id(rank, i, lat_chunks, rope_first) * 64, j2 * kKT, b2);
-                }
+
             }
         }
     } else if (warp == 1) {
