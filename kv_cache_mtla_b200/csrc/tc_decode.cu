@@ -266,12 +266,30 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         b = lo;
         j = gt - starts[lo];
     };
-    pdl_wait();                              // the cache row and q~ come from k_dec_prep_tc
-
+    // Only the producer waits for k_dec_prep_tc (programmatic dependent launch):
+    // the query image and each sequence's last tile (which holds the slot the
+    // prep kernel updates) come from it; the tiles of finished slots do not,
+    // so the first of those are already in flight while the prep kernel runs.
     int loads_issued = 0, q_loads = 0;       // producer's copies, for the drain on failure
     if (warp == 4) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
+            auto load_tile = [&](int st, int b, int j) {
+                mbar_arrive_expect_tx(&bs.full[st], stage_bytes);
+                for (int c = 0; c < n_chunks; ++c)
+                    tma_load_3d(ring + st * stage_bytes + (size_t)c * 16384, &tmap, &bs.full[st], c * 64,
+                                j * kTileSlots, b);
+                ++loads_issued;
+            };
+            int early = 0;                   // tiles 0..early-1 issued before the wait
+            for (int gt = gt0; gt < gt1 && early < 2; ++gt) {
+                int b, j;
+                locate(gt, b, j);
+                if (j + 1 == starts[b + 1] - starts[b]) break;    // holds the open slot
+                load_tile(early, b, j);
+                ++early;
+            }
+            pdl_wait();
             int prev_b = -1;
             for (int gt = gt0, it = 0; gt < gt1; ++gt, ++it) {
                 int b, j;
@@ -283,14 +301,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     bulk_load(q_s, p.qimg + (size_t)b * p.qimg_bytes, p.qimg_bytes, &bs.q_full);
                     ++q_loads;
                 }
+                if (it < early) continue;
                 const int st = it & 1;
                 if (it >= 2 && !sb_wait(&bs.empty[st], ((it >> 1) - 1) & 1, bs)) break;
-                mbar_arrive_expect_tx(&bs.full[st], stage_bytes);
-                for (int c = 0; c < n_chunks; ++c)
-                    tma_load_3d(ring + st * stage_bytes + (size_t)c * 16384, &tmap, &bs.full[st], c * 64,
-                                j * kTileSlots, b);
-                ++loads_issued;
-
+                load_tile(st, b, j);
             }
         }
     } else if (warp == 5) {
