@@ -10,62 +10,128 @@
 
 namespace mtla {
 
-// Merging weight of token t: sigmoid(G[t mod s] . (c_t * PE_t) + g[t mod s])
-// (computed), the supplied value, or 1. Every thread of the block returns it;
-// all threads must call it (block reduction inside).
-template <typename T>
-__device__ float gate_weight(const Shape& sh, int64_t t, const T* c_t, const float* gate_w,
-                             const float* gate_b, const float* w_given, float* red) {
-    if (sh.gate_mode == 2) return 1.f;
-    if (sh.gate_mode == 1) return *w_given;
-    const int r = (int)(t % sh.s);
-    const float* G = gate_w + (size_t)r * sh.d_c;
-    float z = 0.f;
-    for (int k = threadIdx.x; k < sh.d_c / 2; k += blockDim.x) {
-        float sn, cs;
-        pair_sincos(t, k, sh.d_c, sh.log2_pe_base, &sn, &cs);
-        z = fmaf(G[2 * k] * to_f<T>(c_t[2 * k]), sn, z);
-        z = fmaf(G[2 * k + 1] * to_f<T>(c_t[2 * k + 1]), cs, z);
-    }
-    z = block_sum(z, red) + gate_b[r];
-    return sigmoidf_(z);
-}
-
-// Decode: gate, RoPE and in-place update of sequence b's open slot; writes
-// the rounded row into the cache. Returns false (and latches CAPACITY) if
-// pos[b] does not fit the cache.
+// Decode: gate (the merging weight of token t: sigmoid(G[t mod s] .
+// (c_t * PE_t) + g[t mod s]) computed, the supplied value, or 1), RoPE and
+// in-place update of sequence b's open slot; writes the rounded row into the
+// cache. Every thread of the block must call it (block reduction inside).
+// Returns false (and latches CAPACITY) if pos[b] does not fit the cache.
 template <typename T>
 __device__ bool decode_update_body(const DecodeArgs& a, int b) {
     const Shape& sh = a.sh;
+    __shared__ float red[32];
+    constexpr int kMaxPer = 4;                    // latent pairs per thread (d_c / 2 <= 4 * blockDim)
+    constexpr int kMaxPairs = 3;                  // RoPE pairs per thread (d_r / 2 <= 3 * blockDim)
+    const int nt = blockDim.x, tid = threadIdx.x;
+    const T* c = (const T*)a.c_new + (size_t)b * sh.d_c;
+    const T* kr = (const T*)a.kr_new + (size_t)b * sh.d_r;
+    float* acc = a.open_slot + (size_t)b * sh.D;
+    // every load that does not depend on the position first (one round trip
+    // with the position itself): latent pairs (2kp, 2kp+1), open-slot values,
+    // RoPE key pairs
     const int64_t t = a.pos[b];
+    float c0[kMaxPer], c1[kMaxPer], a0[kMaxPer], a1[kMaxPer];
+#pragma unroll
+    for (int i = 0; i < kMaxPer; ++i) {
+        const int kp = tid + i * nt;
+        c0[i] = c1[i] = a0[i] = a1[i] = 0.f;
+        if (kp < sh.d_c / 2) {
+            c0[i] = to_f<T>(c[2 * kp]);
+            c1[i] = to_f<T>(c[2 * kp + 1]);
+            a0[i] = acc[2 * kp];
+            a1[i] = acc[2 * kp + 1];
+        }
+    }
+    float x0[kMaxPairs], x1[kMaxPairs], ar0[kMaxPairs], ar1[kMaxPairs];
+#pragma unroll
+    for (int i = 0; i < kMaxPairs; ++i) {
+        const int kp = tid + i * nt;
+        x0[i] = x1[i] = ar0[i] = ar1[i] = 0.f;
+        if (kp < sh.d_r / 2) {
+            x0[i] = to_f<T>(kr[2 * kp]);
+            x1[i] = to_f<T>(kr[2 * kp + 1]);
+            ar0[i] = acc[sh.d_c + 2 * kp];
+            ar1[i] = acc[sh.d_c + 2 * kp + 1];
+        }
+    }
     if (t < 0 || t >= (int64_t)sh.max_slots * sh.s) {
         if (threadIdx.x == 0) latch_status(a.status, kStatusCapacity);
         return false;
     }
-    __shared__ float red[32];
-    const T* c = (const T*)a.c_new + (size_t)b * sh.d_c;
-    const T* kr = (const T*)a.kr_new + (size_t)b * sh.d_r;
-    const float w = gate_weight<T>(sh, t, c, a.gate_w, a.gate_b, a.gate_in ? a.gate_in + b : nullptr, red);
-    float* acc = a.open_slot + (size_t)b * sh.D;
     T* row = (T*)a.cache + ((size_t)b * sh.max_slots + (size_t)(t / sh.s)) * sh.D;
-    const bool fresh = (t % sh.s) == 0;
-    for (int k = threadIdx.x; k < sh.d_c; k += blockDim.x) {
-        const float v = (fresh ? 0.f : acc[k]) + w * to_f<T>(c[k]);
-        acc[k] = v;
-        row[k] = from_f<T>(v);
+    const bool fresh = (t % sh.s) == 0;           // a new slot opens: the accumulator restarts
+    const int r = (int)(t % sh.s);
+    if (fresh) {
+#pragma unroll
+        for (int i = 0; i < kMaxPer; ++i) a0[i] = a1[i] = 0.f;
+#pragma unroll
+        for (int i = 0; i < kMaxPairs; ++i) ar0[i] = ar1[i] = 0.f;
     }
-    for (int k = threadIdx.x; k < sh.d_r / 2; k += blockDim.x) {
-        float sn, cs;
-        pair_sincos(t, k, sh.d_r, sh.log2_rope_base, &sn, &cs);
-        const float x0 = to_f<T>(kr[2 * k]), x1 = to_f<T>(kr[2 * k + 1]);
-        const float y0 = x0 * cs - x1 * sn, y1 = x0 * sn + x1 * cs;
-        float* ar = acc + sh.d_c;
-        const float v0 = (fresh ? 0.f : ar[2 * k]) + w * y0;
-        const float v1 = (fresh ? 0.f : ar[2 * k + 1]) + w * y1;
-        ar[2 * k] = v0;
-        ar[2 * k + 1] = v1;
-        row[sh.d_c + 2 * k] = from_f<T>(v0);
-        row[sh.d_c + 2 * k + 1] = from_f<T>(v1);
+    // RoPE of the key at position t (independent of the gate)
+    float y0[kMaxPairs], y1[kMaxPairs];
+#pragma unroll
+    for (int i = 0; i < kMaxPairs; ++i) {
+        const int kp = tid + i * nt;
+        y0[i] = y1[i] = 0.f;
+        if (kp < sh.d_r / 2) {
+            float sn, cs;
+            pair_sincos(t, kp, sh.d_r, sh.log2_rope_base, &sn, &cs);
+            y0[i] = x0[i] * cs - x1[i] * sn;
+            y1[i] = x0[i] * sn + x1[i] * cs;
+        }
+    }
+    // gate (Eq. 13): w = sigmoid(G[t mod s] . (c_t * PE_t) + g[t mod s])
+    float w;
+    if (sh.gate_mode == 2) {
+        w = 1.f;
+    } else if (sh.gate_mode == 1) {
+        w = a.gate_in[b];
+    } else {
+        float g0[kMaxPer], g1[kMaxPer];
+#pragma unroll
+        for (int i = 0; i < kMaxPer; ++i) {
+            const int kp = tid + i * nt;
+            g0[i] = g1[i] = 0.f;
+            if (kp < sh.d_c / 2) {
+                g0[i] = a.gate_w[(size_t)r * sh.d_c + 2 * kp];
+                g1[i] = a.gate_w[(size_t)r * sh.d_c + 2 * kp + 1];
+            }
+        }
+        float z = 0.f;
+#pragma unroll
+        for (int i = 0; i < kMaxPer; ++i) {
+            const int kp = tid + i * nt;
+            if (kp < sh.d_c / 2) {
+                float sn, cs;
+                pair_sincos(t, kp, sh.d_c, sh.log2_pe_base, &sn, &cs);   // PE_t[2kp], PE_t[2kp+1]
+                z = fmaf(g0[i] * c0[i], sn, z);
+                z = fmaf(g1[i] * c1[i], cs, z);
+            }
+        }
+        z = block_sum(z, red) + a.gate_b[r];
+        w = sigmoidf_(z);
+    }
+    // in-place update of the open slot; its bf16 rounding is the cache row
+#pragma unroll
+    for (int i = 0; i < kMaxPer; ++i) {
+        const int kp = tid + i * nt;
+        if (kp < sh.d_c / 2) {
+            const float v0 = a0[i] + w * c0[i], v1 = a1[i] + w * c1[i];
+            acc[2 * kp] = v0;
+            acc[2 * kp + 1] = v1;
+            row[2 * kp] = from_f<T>(v0);
+            row[2 * kp + 1] = from_f<T>(v1);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < kMaxPairs; ++i) {
+        const int kp = tid + i * nt;
+        if (kp < sh.d_r / 2) {
+            const float v0 = ar0[i] + w * y0[i], v1 = ar1[i] + w * y1[i];
+            acc[sh.d_c + 2 * kp] = v0;
+            acc[sh.d_c + 2 * kp + 1] = v1;
+            row[sh.d_c + 2 * kp] = from_f<T>(v0);
+            row[sh.d_c + 2 * kp + 1] = from_f<T>(v1);
+        }
     }
     return true;
 }

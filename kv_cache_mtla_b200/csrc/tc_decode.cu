@@ -44,6 +44,7 @@ using namespace tc;
 constexpr int kTileSlots = 128;
 constexpr int kAttnThreads = 224;   // warps 0-3 softmax, 4 TMA, 5 score MMAs, 6 P.V MMAs
 constexpr float kRescaleLog2 = 8.f;
+constexpr int kPrepAbsThreads = 128;   // prep: W_UK product threads (plus one RoPE warp)
 constexpr int kMaxGrid = 160;  // >= SMs of any sm_100 part; sizes the partial buffer
 constexpr int kMaxB = 2048;
 
@@ -73,12 +74,12 @@ __device__ __forceinline__ int seq_slots(const DecTC& p, int b) {
     return (int)(t / p.s) + 1;
 }
 
-// Decode prep for the tensor-core path. grid (B, H + 1), 128 threads.
+// Decode prep for the tensor-core path. grid (B, H + 1), 160 threads.
 // Block (b, h < H): absorbed query of head h, q~ = [W_UK[h]^T qC ; RoPE_t(qR)],
 // rounded to bf16 into row h of sequence b's query image (64-column SW128
 // chunks of NH rows, zero beyond D). Block (b, H): gate, RoPE and in-place
 // update of the open slot (MTLA Method (1)), and zero rows H..NH-1 of the image.
-__global__ void __launch_bounds__(128) k_dec_prep_tc(DecodeArgs a, uint8_t* qimg, int n_chunks, int NH) {
+__global__ void __launch_bounds__(kPrepAbsThreads + 32) k_dec_prep_tc(DecodeArgs a, uint8_t* qimg, int n_chunks, int NH) {
     pdl_launch_dependents();   // the attention kernel may start its prologue now
     const Shape& sh = a.sh;
     const int b = blockIdx.x, h = blockIdx.y;
@@ -94,33 +95,53 @@ __global__ void __launch_bounds__(128) k_dec_prep_tc(DecodeArgs a, uint8_t* qimg
         return;
     }
     const int64_t t = a.pos[b];
-    if (t < 0 || t >= (int64_t)sh.max_slots * sh.s) return;
-    __shared__ float q[256];
+    const bool t_ok = t >= 0 && t < (int64_t)sh.max_slots * sh.s;
     __shared__ float part_sum[8][512];     // [i-group][latent column]
     const size_t rh = (size_t)b * sh.H + h;
     const bf16* qc = (const bf16*)a.q_c + rh * sh.d_h;
-    for (int i = threadIdx.x; i < sh.d_h; i += blockDim.x) q[i] = __bfloat162float(qc[i]);
-    __syncthreads();
+    const bf16* qr = (const bf16*)a.q_r + rh * sh.d_r;
+    const int dpad = n_chunks * 64;
+    if (threadIdx.x >= kPrepAbsThreads) {
+        // the last warp: RoPE part of q~ (columns d_c .. D-1) and the zero padding
+        // up to the chunk boundary, independent of the W_UK product
+        if (!t_ok) return;
+        for (int j = sh.d_c + (int)threadIdx.x - kPrepAbsThreads; j < dpad; j += 32) {
+            float v = 0.f;
+            if (j < sh.D) {
+                const int e = j - sh.d_c, k = e >> 1;
+                const float x0 = __bfloat162float(qr[2 * k]), x1 = __bfloat162float(qr[2 * k + 1]);
+                float sn, cs;
+                pair_sincos(t, k, sh.d_r, sh.log2_rope_base, &sn, &cs);
+                v = (e & 1) ? (x0 * sn + x1 * cs) : (x0 * cs - x1 * sn);
+            }
+            *(bf16*)(img + (size_t)(j >> 6) * NH * 128 + sw128_offset(h, j & 63)) = __float2bfloat16_rn(v);
+        }
+        return;
+    }
     // thread (ig, jg): 8 latent columns [8 jg, 8 jg + 8) over rows i of group ig;
-    // all of its 16-byte loads of W_UK are issued before any product
+    // its 16-byte loads of W_UK and of qC are all issued before any product
     const bf16* W = (const bf16*)a.w_uk + (size_t)h * sh.d_h * sh.d_c;
     const int n_jg = sh.d_c / 8;
-    const int n_ig = max(1, min(8, (int)blockDim.x / n_jg));
-    const int rows_per = (sh.d_h + n_ig - 1) / n_ig;
-    for (int e = threadIdx.x; e < n_ig * n_jg; e += blockDim.x) {
+    const int n_ig = max(1, min(8, kPrepAbsThreads / n_jg));
+    const int rows_per = (((sh.d_h + n_ig - 1) / n_ig) + 15) & ~15;   // 16-row batches, aligned
+    for (int e = threadIdx.x; e < n_ig * n_jg; e += kPrepAbsThreads) {
         const int ig = e / n_jg, jg = e % n_jg;
         const int i0 = ig * rows_per, i1 = min(sh.d_h, i0 + rows_per);
         float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         for (int ib = i0; ib < i1; ib += 16) {
-            uint4 raw[16];
+            uint4 raw[16], qraw[2];
 #pragma unroll
             for (int u = 0; u < 16; ++u)
                 if (ib + u < i1) raw[u] = *(const uint4*)(W + (size_t)(ib + u) * sh.d_c + jg * 8);
 #pragma unroll
+            for (int u = 0; u < 2; ++u)
+                if (ib + 8 * u < i1) qraw[u] = *(const uint4*)(qc + ib + 8 * u);   // d_h % 16 == 0
+            const bf16* qv = (const bf16*)qraw;
+#pragma unroll
             for (int u = 0; u < 16; ++u) {
                 if (ib + u < i1) {
                     const bf16* wv = (const bf16*)&raw[u];
-                    const float qi = q[ib + u];
+                    const float qi = __bfloat162float(qv[u]);
 #pragma unroll
                     for (int v = 0; v < 8; ++v) acc[v] = fmaf(__bfloat162float(wv[v]), qi, acc[v]);
                 }
@@ -129,20 +150,11 @@ __global__ void __launch_bounds__(128) k_dec_prep_tc(DecodeArgs a, uint8_t* qimg
 #pragma unroll
         for (int v = 0; v < 8; ++v) part_sum[ig][jg * 8 + v] = acc[v];
     }
-    __syncthreads();
-    const bf16* qr = (const bf16*)a.q_r + rh * sh.d_r;
-    const int dpad = n_chunks * 64;
-    for (int j = threadIdx.x; j < dpad; j += blockDim.x) {
+    named_sync(1, kPrepAbsThreads);      // the W_UK threads only
+    if (!t_ok) return;                   // (the loads above do not depend on the position)
+    for (int j = threadIdx.x; j < sh.d_c; j += kPrepAbsThreads) {
         float v = 0.f;
-        if (j < sh.d_c) {
-            for (int ig = 0; ig < n_ig; ++ig) v += part_sum[ig][j];
-        } else if (j < sh.D) {
-            const int e = j - sh.d_c, k = e >> 1;
-            float sn, cs;
-            pair_sincos(t, k, sh.d_r, sh.log2_rope_base, &sn, &cs);
-            const float x0 = __bfloat162float(qr[2 * k]), x1 = __bfloat162float(qr[2 * k + 1]);
-            v = (e & 1) ? (x0 * sn + x1 * cs) : (x0 * cs - x1 * sn);
-        }
+        for (int ig = 0; ig < n_ig; ++ig) v += part_sum[ig][j];
         *(bf16*)(img + (size_t)(j >> 6) * NH * 128 + sw128_offset(h, j & 63)) = __float2bfloat16_rn(v);
     }
 }
@@ -809,7 +821,7 @@ cudaError_t tc_decode(const DecodeArgs& a, cudaStream_t st, uint64_t* launches) 
             carve[dev] = true;
         }
     }
-    k_dec_prep_tc<<<dim3(sh.B, sh.H + 1), 128, 0, st>>>(a, qimg, p.n_chunks, NH);
+    k_dec_prep_tc<<<dim3(sh.B, sh.H + 1), kPrepAbsThreads + 32, 0, st>>>(a, qimg, p.n_chunks, NH);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return note_error("k_dec_prep_tc launch", e);
     const size_t smem = attn_smem_bytes(sh, NH);
