@@ -745,134 +745,197 @@ __device__ void lh_tile_starts(const LhArgs& p, int* starts, int* warp_tot) {
     __syncthreads();
 }
 
-// grid (H), 256 threads. Block h: W_UV[h] staged transposed ([d_c][d_h]); for
-// every 32 sequences, the partials of head h are merged by the online-softmax
-// rule into o_lat [d_c][32], then out[b, h] = W_UV[h] o_lat[b] by head_gemm_32.
-__global__ void __launch_bounds__(256) k_lh_combine(DecodeArgs a, LhArgs p) {
+// Merge and W_UV on the tensor cores. grid (H, ceil(B / 32)), 512 threads.
+// Block (h, group of 32 sequences):
+//   A. per sequence, one warp turns the partial maxima and sums (m_i, l_i)
+//      into merge weights 2^(m_i - M) / L (lane i: partial i);
+//   B. thread (column quad, sequence octet) sums the weighted partial rows,
+//      writing o_lat as bf16 into a K-major operand;
+//   C. out^T [d_h x 32] = W_UV[h] [d_h x d_c] . o_lat^T  (tcgen05, M = 128, N = 32)
+//      with W_UV[h] brought in by TMA before the wait for the attention kernel.
+constexpr int kCombThreads = 512;
+__global__ void __launch_bounds__(kCombThreads, 1)
+    k_lh_combine(const __grid_constant__ CUtensorMap wuv_map, DecodeArgs a, LhArgs p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const Shape& sh = a.sh;
-    const int h = blockIdx.x;
-    extern __shared__ uint8_t dyn[];
-    bf16* Wt = (bf16*)dyn;                                                    // [d_c][d_h]
-    float* X = (float*)(dyn + (size_t)sh.d_h * sh.d_c * sizeof(bf16));       // [d_c][32]
-    int* idx = (int*)(X + (size_t)sh.d_c * 32);                               // [32][kMaxClusters]
-    int* npart = idx + 32 * kMaxClusters;                                     // [32]
-    int* starts = npart + 32;                                                 // [B + 1]
-    float* wts = (float*)(starts + sh.B + 1);                                 // [32][kMaxClusters]
-    __shared__ int warp_tot[8];
-    __shared__ float invl[32];
-    __shared__ int maxn_s;
-    {
-        // transpose W_UV[h] [d_h][d_c] into [d_c][d_h]; 8 loads in flight per thread.
-        // Consecutive threads take consecutive rows i, so the 2-byte stores of a
-        // warp land in consecutive shared-memory words (no bank conflicts).
-        const bf16* src = (const bf16*)a.w_uv + (size_t)h * sh.d_h * sh.d_c;
-        const int n16 = sh.d_h * sh.d_c / 8;
-        for (int e0 = threadIdx.x; e0 < n16; e0 += 8 * blockDim.x) {
-            uint4 raw[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int e = e0 + u * blockDim.x;
-                const int i = e % sh.d_h, k0 = (e / sh.d_h) * 8;
-                if (e < n16) raw[u] = *(const uint4*)(src + (size_t)i * sh.d_c + k0);
-            }
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int e = e0 + u * blockDim.x;
-                if (e < n16) {
-                    const int i = e % sh.d_h, k0 = (e / sh.d_h) * 8;
-                    const bf16* w = (const bf16*)&raw[u];
-#pragma unroll
-                    for (int v = 0; v < 8; ++v) Wt[(size_t)(k0 + v) * sh.d_h + i] = w[v];
-                }
-            }
-        }
+    const int h = blockIdx.x, c0 = blockIdx.y * 32;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int n_kc = p.d_c / 64, n_mb = (sh.d_h + 127) / 128;
+    uint8_t* w_s = smem;                                  // n_kc x [128 W_UV rows x 128 B]
+    uint8_t* o_s = w_s + (size_t)n_kc * 16384;            // n_kc x [32 sequences x 128 B]
+    float* wts = (float*)(o_s + (size_t)n_kc * 4096);     // [32][kMaxClusters] merge weights
+    int* pidx = (int*)(wts + 32 * kMaxClusters);          // [32][kMaxClusters] partial index or -1
+    int* npart = pidx + 32 * kMaxClusters;                // [32]
+    uint64_t* bars = (uint64_t*)(npart + 32);             // [0] W landed, [1] MMAs done
+    uint32_t* tmem_slot = (uint32_t*)(bars + 2);
+    int* starts = (int*)(bars + 4);                       // [B + 1]
+    __shared__ int warp_tot[kCombThreads / 32];
+    const uint32_t w_bytes = (uint32_t)n_kc * 16384;
+    if (tid == 0) {
+        mbar_init(&bars[0], 1);
+        mbar_init(&bars[1], 1);
+        fence_mbar_init();
+        tma_prefetch_desc(&wuv_map);
+        mbar_arrive_expect_tx(&bars[0], w_bytes);
+        for (int kc = 0; kc < n_kc; ++kc) tma_load_2d(w_s + kc * 16384, &wuv_map, &bars[0], kc * 64, h * sh.d_h);
     }
-    lh_tile_starts(p, starts, warp_tot);
-    pdl_wait();                          // the partials come from k_lh_attn
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 128);
+        tmem_relinquish();
+    }
+    lh_tile_starts(p, starts, warp_tot);                  // reads pos only; ends with a block barrier
+    tc_fence_after();
+    const uint32_t t_d = *tmem_slot;
     const int total = starts[p.B];
     const size_t row = (size_t)p.d_c + 4;
-    for (int c0 = 0; c0 < sh.B; c0 += 32) {
-        __syncthreads();                 // X, idx free
-        if (threadIdx.x < 32) {
-            const int b = c0 + threadIdx.x;
-            int n = 0;
-            if (b < sh.B && starts[b + 1] > starts[b] && total > 0) {
-                const int S_b = starts[b], E_b = starts[b + 1];
-                const int64_t G = p.G2, tot = total;
-                const int g_first = (int)(((int64_t)(S_b + 1) * G + tot - 1) / tot) - 1;
-                const int g_last = (int)(((int64_t)E_b * G + tot - 1) / tot) - 1;
-                int64_t lo = ((int64_t)g_first * tot) / G;
-                for (int gg = g_first; gg <= g_last; ++gg) {
-                    const int64_t hi = ((int64_t)(gg + 1) * tot) / G;
-                    if (hi > lo && n < kMaxClusters) idx[threadIdx.x * kMaxClusters + n++] = gg + b;
-                    lo = hi;
-                }
-            }
-            npart[threadIdx.x] = n;
-            // merge weights 2^(m_i - M) and 1 / sum_i 2^(m_i - M) l_i
+    pdl_wait();                                           // the partials come from k_lh_attn
+    // ---- A: merge weights
+    for (int bb = warp; bb < 32; bb += kCombThreads / 32) {
+        const int b = c0 + bb;
+        int n = 0;
+        if (b < sh.B && starts[b + 1] > starts[b] && total > 0) {
+            // the clusters g_first..g_last touching this sequence's tiles [S_b, E_b)
+            const int S_b = starts[b], E_b = starts[b + 1];
+            const int64_t G = p.G2, tot = total;
+            const int g_first = (int)(((int64_t)(S_b + 1) * G + tot - 1) / tot) - 1;
+            const int g_last = (int)(((int64_t)E_b * G + tot - 1) / tot) - 1;
+            n = min(g_last - g_first + 1, kMaxClusters);
+            float mv[3], lv[3];                           // n <= kMaxClusters <= 96 = 3 x 32
             float M = -INFINITY;
-            for (int i = 0; i < n; ++i)
-                M = fmaxf(M, p.part[((size_t)idx[threadIdx.x * kMaxClusters + i] * p.H + h) * row + p.d_c]);
-            float L = 0.f;
-            for (int i = 0; i < n; ++i) {
-                const float* ep = p.part + ((size_t)idx[threadIdx.x * kMaxClusters + i] * p.H + h) * row;
-                const float w = exp2f(ep[p.d_c] - M);
-                wts[threadIdx.x * kMaxClusters + i] = w;
-                L += w * ep[p.d_c + 1];
-            }
-            invl[threadIdx.x] = n > 0 ? 1.f / L : 0.f;
-            int mx = n;
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-            if (threadIdx.x == 0) maxn_s = mx;
-        }
-        __syncthreads();
-        // o_lat[k][bb] = sum_i w_i o_i[k] / L: 32 partial values in flight per round
-        for (int k = threadIdx.x; k < sh.d_c; k += blockDim.x) {
-            for (int g8 = 0; g8 < 4; ++g8) {
-                float acc8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                for (int kk0 = 0; kk0 < maxn_s; kk0 += 4) {
-                    float o[8][4];
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int bb = 8 * g8 + i;
-                            o[i][u] = (kk0 + u < npart[bb])
-                                          ? p.part[((size_t)idx[bb * kMaxClusters + kk0 + u] * p.H + h) * row + k]
-                                          : 0.f;
-                        }
-#pragma unroll
-                    for (int i = 0; i < 8; ++i)
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int bb = 8 * g8 + i;
-                            if (kk0 + u < npart[bb]) acc8[i] = fmaf(wts[bb * kMaxClusters + kk0 + u], o[i][u], acc8[i]);
-                        }
+            for (int r = 0; r < 3; ++r) {
+                const int i = r * 32 + lane, g = g_first + i;
+                mv[r] = -INFINITY;
+                lv[r] = 0.f;
+                if (i < n) {
+                    const int64_t lo = ((int64_t)g * tot) / G, hi = ((int64_t)(g + 1) * tot) / G;
+                    if (hi > lo) {
+                        const float* e = p.part + ((size_t)(g + b) * p.H + h) * row;
+                        mv[r] = e[p.d_c];
+                        lv[r] = e[p.d_c + 1];
+                    }
                 }
+                M = fmaxf(M, mv[r]);
+            }
+            M = warp_max(M);
+            float L = 0.f;
 #pragma unroll
-                for (int i = 0; i < 8; ++i) X[(size_t)k * 32 + 8 * g8 + i] = acc8[i] * invl[8 * g8 + i];
+            for (int r = 0; r < 3; ++r) L += (mv[r] == -INFINITY) ? 0.f : exp2f(mv[r] - M) * lv[r];
+            const float inv = 1.f / warp_sum(L);
+#pragma unroll
+            for (int r = 0; r < 3; ++r) {
+                const int i = r * 32 + lane;
+                if (i < n) {
+                    const bool live = mv[r] != -INFINITY;
+                    wts[bb * kMaxClusters + i] = live ? exp2f(mv[r] - M) * inv : 0.f;
+                    pidx[bb * kMaxClusters + i] = live ? g_first + i + b : -1;
+                }
             }
         }
-        __syncthreads();
-        auto emit = [&](auto& acc, int b0, int j0, int bt) {
-            for (int i = 0; i < bt; ++i) {
-                const int b = c0 + b0 + i;
-                if (b0 >= 32 || b >= sh.B || npart[b0 + i] == 0) continue;
-                uint4 pk;
-                pk.x = pack_bf16x2(acc[i][0], acc[i][1]);
-                pk.y = pack_bf16x2(acc[i][2], acc[i][3]);
-                pk.z = pack_bf16x2(acc[i][4], acc[i][5]);
-                pk.w = pack_bf16x2(acc[i][6], acc[i][7]);
-                *(uint4*)((bf16*)a.out + ((size_t)b * sh.H + h) * sh.d_h + j0) = pk;
-            }
-        };
-        int b0, j0;
-        if (sh.d_h == 512) { float acc[8][8]; head_gemm_32<8>(X, Wt, sh.d_c, sh.d_h, acc, b0, j0); emit(acc, b0, j0, 8); }
-        else if (sh.d_h == 256) { float acc[4][8]; head_gemm_32<4>(X, Wt, sh.d_c, sh.d_h, acc, b0, j0); emit(acc, b0, j0, 4); }
-        else if (sh.d_h == 128) { float acc[2][8]; head_gemm_32<2>(X, Wt, sh.d_c, sh.d_h, acc, b0, j0); emit(acc, b0, j0, 2); }
-        else { float acc[1][8]; head_gemm_32<1>(X, Wt, sh.d_c, sh.d_h, acc, b0, j0); emit(acc, b0, j0, 1); }
+        if (lane == 0) npart[bb] = n;
     }
+    __syncthreads();
+    // ---- B: weighted sums, thread = (column quad cq, octet of sequences so)
+    {
+        const int cq = tid & 127, so = tid >> 7;
+        const int k = cq * 4;
+        for (int bb = so * 8; bb < so * 8 + 8; bb += 2) {
+            float o[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+            const int nmax = max(npart[bb], npart[bb + 1]);
+            for (int i0 = 0; i0 < nmax; i0 += 4) {
+                float4 v[2][4];
+                float wv[2][4];
+#pragma unroll
+                for (int s2 = 0; s2 < 2; ++s2)
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int i = i0 + u, q = bb + s2;
+                        v[s2][u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                        wv[s2][u] = 0.f;
+                        if (k < p.d_c && i < npart[q]) {
+                            const int pi = pidx[q * kMaxClusters + i];
+                            if (pi >= 0) {
+                                wv[s2][u] = wts[q * kMaxClusters + i];
+                                v[s2][u] = *(const float4*)(p.part + ((size_t)pi * p.H + h) * row + k);
+                            }
+                        }
+                    }
+#pragma unroll
+                for (int s2 = 0; s2 < 2; ++s2)
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        o[s2][0] = fmaf(wv[s2][u], v[s2][u].x, o[s2][0]);
+                        o[s2][1] = fmaf(wv[s2][u], v[s2][u].y, o[s2][1]);
+                        o[s2][2] = fmaf(wv[s2][u], v[s2][u].z, o[s2][2]);
+                        o[s2][3] = fmaf(wv[s2][u], v[s2][u].w, o[s2][3]);
+                    }
+            }
+            if (k < p.d_c) {
+#pragma unroll
+                for (int s2 = 0; s2 < 2; ++s2) {
+                    uint2 pk;
+                    pk.x = pack_bf16x2(o[s2][0], o[s2][1]);
+                    pk.y = pack_bf16x2(o[s2][2], o[s2][3]);
+                    *(uint2*)(o_s + (size_t)(k >> 6) * 4096 + sw128_offset(bb + s2, k & 63)) = pk;
+                }
+            }
+        }
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    // ---- C: out^T = W_UV[h] . o_lat^T, 128 output rows at a time
+    if (tid == 0) {
+        bool ok = true;
+        for (int mb = 0; mb < n_mb && ok; ++mb) {
+            if (mb > 0) {
+                // the next 128 rows of W_UV[h] into the same buffer, once the previous
+                // block's MMAs have read it
+                ok = mbar_wait(&bars[1], (mb - 1) & 1);
+                if (!ok) break;
+                mbar_arrive_expect_tx(&bars[0], w_bytes);
+                for (int kc = 0; kc < n_kc; ++kc)
+                    tma_load_2d(w_s + kc * 16384, &wuv_map, &bars[0], kc * 64, h * sh.d_h + mb * 128);
+            }
+            ok = mbar_wait(&bars[0], mb & 1);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t idesc = idesc_bf16_f32(128, 32, false, false);
+            const uint64_t ad = sdesc_sw128(smem_u32(w_s), 16, 1024), bd = sdesc_sw128(smem_u32(o_s), 16, 1024);
+            for (int kc = 0; kc < n_kc; ++kc) {
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_bf16(t_d + mb * 32, desc_add(ad, kc * 16384 + kk * 32), desc_add(bd, kc * 4096 + kk * 32),
+                              idesc, (kc | kk) != 0);
+            }
+            umma_commit(&bars[1]);
+        }
+        if (!ok) latch_status(a.status, kStatusTimeout);
+    }
+    // every thread: the last block's MMAs (they complete in order); warp w reads
+    // TMEM lane quarter w mod 4, sequences 8 (w / 4) .. 8 (w / 4) + 7
+    const bool done = mbar_wait(&bars[1], (n_mb - 1) & 1);
+    tc_fence_after();
+    const int quarter = warp & 3, oct = warp >> 2;
+    for (int mb = 0; mb < n_mb; ++mb) {
+        float v[8];
+        tmem_ld8(t_d + mb * 32 + oct * 8 + ((uint32_t)(quarter * 32) << 16), v);
+        tmem_wait_ld();
+        const int i = mb * 128 + quarter * 32 + lane;       // output dimension (W_UV row)
+        if (done && i < sh.d_h) {
+#pragma unroll
+            for (int s8 = 0; s8 < 8; ++s8) {
+                const int b = c0 + oct * 8 + s8;
+                if (b < sh.B && starts[b + 1] > starts[b])
+                    ((bf16*)a.out)[((size_t)b * sh.H + h) * sh.d_h + i] = __float2bfloat16_rn(v[s8]);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(t_d, 128);
 }
 
 // ---------------------------------------------------------------- host side
@@ -891,7 +954,8 @@ size_t lh_attn_smem(const Shape& sh) {
 size_t lh_stage_smem(const Shape& sh) { return (size_t)sh.d_h * sh.d_c * sizeof(bf16); }
 size_t lh_prep_smem(const Shape& sh) { return lh_stage_smem(sh) + (size_t)sh.d_h * 32 * 4 + 16; }
 size_t lh_comb_smem(const Shape& sh) {
-    return lh_stage_smem(sh) + (size_t)sh.d_c * 32 * 4 + (2 * 32 * kMaxClusters + 32 + (size_t)sh.B + 1) * 4;
+    const size_t n_kc = sh.d_c / 64;
+    return 1024 + n_kc * 16384 + n_kc * 4096 + (2 * 32 * kMaxClusters + 32) * 4 + 32 + ((size_t)sh.B + 1) * 4;
 }
 
 template <typename... KArgs, typename... Args>
@@ -952,6 +1016,23 @@ cudaError_t tc_decode_lh(const DecodeArgs& a, cudaStream_t st, uint64_t* launche
         snprintf(buf, sizeof(buf), "cuTensorMapEncodeTiled (CUresult %d)", (int)r);
         return note_error(buf, cudaErrorInvalidValue);
     }
+    CUtensorMap wuv_map;
+    {
+        // W_UV as [H * d_h rows][d_c] bf16, 128-row x 64-column boxes (rows past
+        // the last head read as zero)
+        cuuint64_t d2[2] = {(cuuint64_t)sh.d_c, (cuuint64_t)sh.H * sh.d_h};
+        cuuint64_t s2[1] = {(cuuint64_t)sh.d_c * 2};
+        cuuint32_t b2[2] = {64, 128};
+        cuuint32_t e2[2] = {1, 1};
+        r = encode(&wuv_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a.w_uv), d2, s2, b2, e2,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) {
+            char buf[96];
+            snprintf(buf, sizeof(buf), "cuTensorMapEncodeTiled W_UV (CUresult %d)", (int)r);
+            return note_error(buf, cudaErrorInvalidValue);
+        }
+    }
     LhArgs p;
     p.B = sh.B;
     p.H = sh.H;
@@ -1001,7 +1082,7 @@ cudaError_t tc_decode_lh(const DecodeArgs& a, cudaStream_t st, uint64_t* launche
     e = launch_pdl_lh(k_lh_attn, dim3(2 * p.G2), dim3(kThreads), attn_smem, st, map, p);
     profile_end(st);
     if (e != cudaSuccess) return note_error("k_lh_attn launch", e);
-    e = launch_pdl_lh(k_lh_combine, dim3(sh.H), dim3(256), comb_smem, st, a, p);
+    e = launch_pdl_lh(k_lh_combine, dim3(sh.H, (sh.B + 31) / 32), dim3(kCombThreads), comb_smem, st, wuv_map, a, p);
     *launches += 3;
     return note_error("k_lh_combine launch", e);
 }
