@@ -69,136 +69,105 @@ __device__ __forceinline__ int lh_tiles(const LhArgs& p, int b) { return (lh_slo
 
 // ---------------------------------------------------------------- prep
 
-// Register-blocked product for one head, 32 sequences at a time, CUDA cores:
-//   acc[i][jj] = sum_k X[k][b0 + i] * W[k][j0 + jj]     (i < BT, jj < 8)
-// with X fp32 [K][32] and W bf16 [K][N] in shared memory. The 256 threads
-// tile the [32 x N] output as (32 / BT) sequence groups x (N / 8) column
-// groups, BT = N / 64 (N in {64, 128, 256, 512}).
-template <int BT>
-__device__ __forceinline__ void head_gemm_32(const float* X, const bf16* W, int K, int N, float (&acc)[BT][8],
-                                             int& b0, int& j0) {
-    const int n_jg = N / 8;
-    const int t = threadIdx.x;
-    j0 = 8 * (t % n_jg);
-    b0 = BT * (t / n_jg);
-#pragma unroll
-    for (int i = 0; i < BT; ++i)
-#pragma unroll
-        for (int jj = 0; jj < 8; ++jj) acc[i][jj] = 0.f;
-    if (b0 >= 32) return;
-    for (int k = 0; k < K; ++k) {
-        const uint4 raw = *(const uint4*)(W + (size_t)k * N + j0);
-        const bf16* w = (const bf16*)&raw;
-        float wf[8];
-#pragma unroll
-        for (int jj = 0; jj < 8; ++jj) wf[jj] = __bfloat162float(w[jj]);
-#pragma unroll
-        for (int i = 0; i < BT; ++i) {
-            const float x = X[k * 32 + b0 + i];
-#pragma unroll
-            for (int jj = 0; jj < 8; ++jj) acc[i][jj] = fmaf(x, wf[jj], acc[i][jj]);
-        }
-    }
-}
-
 __device__ __forceinline__ bool lh_pos_ok(const Shape& sh, int64_t t) {
     return t >= 0 && t < (int64_t)sh.max_slots * sh.s;
 }
 
-// grid (H), 256 threads. Block h: W_UK[h] staged by one bulk copy; for every
-// 32 sequences, q~ = W_UK[h]^T qC[b, h] (latent part) by head_gemm_32 and
-// RoPE_t(qR[b, h]) (rotated part), rounded to bf16 into row h of sequence b's
-// image. Then the in-place slot updates of sequences b = h, h + H, ... (gate,
-// RoPE, open slot; MTLA Method (1)) and the zero rows H..127 of their images.
-__global__ void __launch_bounds__(256) k_lh_prep(DecodeArgs a, uint8_t* qimg, int n_qchunks) {
+// Decode prep for many heads on the tensor cores. grid (H, ceil(B / 32)),
+// 256 threads. Block (h, group of 32 sequences):
+//   q~^T [d_c x 32] = W_UK[h]^T [d_c x d_h] . qC^T [d_h x 32]   (tcgen05,
+//   M = 128 latent columns per block, N = 32, A = W_UK[h] by TMA, MN-major)
+// rounded to bf16 into row h of each sequence's query image; the RoPE part
+// RoPE_t(qR) and the zero tail on the CUDA cores; then the in-place slot
+// updates (gate, RoPE key, open slot; MTLA Method (1)) of the group's
+// sequences b with b mod H = h, and the zero rows H..127 of their images.
+constexpr int kPrepThreads = 256;
+__global__ void __launch_bounds__(kPrepThreads, 1)
+    k_lh_prep(const __grid_constant__ CUtensorMap wuk_map, DecodeArgs a, uint8_t* qimg, int n_qchunks) {
     pdl_launch_dependents();
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const Shape& sh = a.sh;
-    const int h = blockIdx.x;
+    const int h = blockIdx.x, c0 = blockIdx.y * 32;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t img_bytes = (uint32_t)n_qchunks * 128 * 128;
-    extern __shared__ uint8_t dyn[];
-    bf16* Ws = (bf16*)dyn;                                                   // [d_h][d_c]
-    float* X = (float*)(dyn + (size_t)sh.d_h * sh.d_c * sizeof(bf16));      // [d_h][32]
-    uint64_t* bar = (uint64_t*)(X + (size_t)sh.d_h * 32);
-    const uint32_t w_bytes = (uint32_t)sh.d_h * sh.d_c * sizeof(bf16);
-    if (threadIdx.x == 0) {
-        mbar_init(bar, 1);
+    const int n_kc = sh.d_c / 64;                          // 64-column chunks of W_UK rows (= latent)
+    const int n_kb = (sh.d_h + 127) / 128;                 // 128-row blocks of W_UK (= K)
+    const int n_qc = (sh.d_h + 63) / 64;                   // 64-column chunks of qC
+    uint8_t* w_s = smem;                                   // n_kc x [128 k-rows x 128 B]
+    uint8_t* x_s = w_s + (size_t)n_kc * 16384;             // n_qc x [32 sequences x 128 B]: qC rows
+    uint64_t* bars = (uint64_t*)(x_s + (size_t)n_qc * 4096);   // [0] W landed, [1] MMAs done
+    uint32_t* tmem_slot = (uint32_t*)(bars + 2);
+    const uint32_t w_bytes = (uint32_t)n_kc * 16384;
+    if (tid == 0) {
+        mbar_init(&bars[0], 1);
+        mbar_init(&bars[1], 1);
         fence_mbar_init();
-        mbar_arrive_expect_tx(bar, w_bytes);
-        const uint8_t* src = (const uint8_t*)((const bf16*)a.w_uk + (size_t)h * sh.d_h * sh.d_c);
-        for (uint32_t off = 0; off < w_bytes; off += 32768)
-            bulk_load((uint8_t*)Ws + off, src + off, min(32768u, w_bytes - off), bar);
+        mbar_arrive_expect_tx(&bars[0], w_bytes);
+        for (int kc = 0; kc < n_kc; ++kc) tma_load_2d(w_s + kc * 16384, &wuk_map, &bars[0], kc * 64, h * sh.d_h);
     }
+    if (warp == 0) {
+        tmem_alloc(tmem_slot, 128);
+        tmem_relinquish();
+    }
+    // qC rows of the 32 sequences (zero past B) as the K-major B operand
+    for (int e = tid; e < 32 * n_qc * 8; e += kPrepThreads) {
+        const int bb = e / (n_qc * 8), rem = e % (n_qc * 8), c = rem >> 3, u = rem & 7;
+        const int b = c0 + bb, col = c * 64 + u * 8;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (b < sh.B && col < sh.d_h) v = *(const uint4*)((const bf16*)a.q_c + ((size_t)b * sh.H + h) * sh.d_h + col);
+        *(uint4*)(x_s + (size_t)c * 4096 + sw128_offset(bb, u * 8)) = v;
+    }
+    fence_proxy_async();
+    tc_fence_before();
     __syncthreads();
-    bool w_ok = mbar_wait(bar, 0);
-    if (!w_ok && threadIdx.x == 0) latch_status(a.status, kStatusTimeout);
-    __shared__ int64_t tpos[32];                                  // position, or -1 if invalid
-    for (int c0 = 0; c0 < sh.B && w_ok; c0 += 32) {
-        __syncthreads();                                          // X, tpos free
-        if (threadIdx.x < 32) {
-            const int b = c0 + threadIdx.x;
-            const int64_t t = b < sh.B ? (int64_t)a.pos[b] : -1;
-            tpos[threadIdx.x] = lh_pos_ok(sh, t) ? t : -1;
-        }
-        {
-            // X[k][bb] = qC[c0 + bb, h, k]: lane = sequence, so the stores are
-            // conflict-free; every 16-byte load of a thread is issued first
-            const int n8 = sh.d_h / 8;                            // <= 64 -> <= 8 per thread
-            uint4 raw[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int e = threadIdx.x + u * blockDim.x, k8 = e / 32, bb = e % 32, b = c0 + bb;
-                raw[u] = make_uint4(0, 0, 0, 0);
-                if (k8 < n8 && b < sh.B)
-                    raw[u] = *(const uint4*)((const bf16*)a.q_c + ((size_t)b * sh.H + h) * sh.d_h + k8 * 8);
+    tc_fence_after();
+    const uint32_t t_d = *tmem_slot;
+    if (tid == 0) {
+        bool ok = true;
+        const uint32_t idesc = idesc_bf16_f32(128, 32, true, false);
+        const uint64_t ad = sdesc_sw128(smem_u32(w_s), 16384, 1024), bd = sdesc_sw128(smem_u32(x_s), 16, 1024);
+        for (int kb = 0; kb < n_kb && ok; ++kb) {
+            if (kb > 0) {
+                // the next 128 rows of W_UK[h] into the same buffer once the MMAs read it
+                ok = mbar_wait(&bars[1], (kb - 1) & 1);
+                if (!ok) break;
+                mbar_arrive_expect_tx(&bars[0], w_bytes);
+                for (int kc = 0; kc < n_kc; ++kc)
+                    tma_load_2d(w_s + kc * 16384, &wuk_map, &bars[0], kc * 64, h * sh.d_h + kb * 128);
             }
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int e = threadIdx.x + u * blockDim.x, k8 = e / 32, bb = e % 32;
-                if (k8 < n8) {
-                    const bf16* w = (const bf16*)&raw[u];
-#pragma unroll
-                    for (int v = 0; v < 8; ++v) X[(k8 * 8 + v) * 32 + bb] = __bfloat162float(w[v]);
+            ok = mbar_wait(&bars[0], kb & 1);
+            if (!ok) break;
+            tc_fence_after();
+            const int ksteps = min(128, sh.d_h - kb * 128) / 16;
+            for (int mb = 0; mb < n_kc / 2; ++mb) {
+                // A = W_UK[h]^T block mb: latent 128 mb.. as M (two 64-column chunks), k rows as K
+                const uint64_t am = desc_add(ad, mb * 2 * 16384);
+                for (int kk = 0; kk < ksteps; ++kk) {
+                    const int kg = kb * 8 + kk;                // global 16-row K step
+                    umma_bf16(t_d + mb * 32, desc_add(am, kk * 2048),
+                              desc_add(bd, (kg >> 2) * 4096 + (kg & 3) * 32), idesc, (kg > 0) ? 1u : 0u);
                 }
             }
+            umma_commit(&bars[1]);
         }
-        __syncthreads();
-        auto emit = [&](auto& acc, int b0, int j0, int bt) {
-            for (int i = 0; i < bt; ++i) {
-                const int b = c0 + b0 + i;
-                if (b0 >= 32 || b >= sh.B || tpos[b0 + i] < 0) continue;
-                uint4 pk;
-                pk.x = pack_bf16x2(acc[i][0], acc[i][1]);
-                pk.y = pack_bf16x2(acc[i][2], acc[i][3]);
-                pk.z = pack_bf16x2(acc[i][4], acc[i][5]);
-                pk.w = pack_bf16x2(acc[i][6], acc[i][7]);
-                *(uint4*)(qimg + (size_t)b * img_bytes + (size_t)(j0 >> 6) * 128 * 128 + sw128_offset(h, j0 & 63)) = pk;
-            }
-        };
-        int b0, j0;
-        if (sh.d_c == 512) { float acc[8][8]; head_gemm_32<8>(X, Ws, sh.d_h, sh.d_c, acc, b0, j0); emit(acc, b0, j0, 8); }
-        else if (sh.d_c == 256) { float acc[4][8]; head_gemm_32<4>(X, Ws, sh.d_h, sh.d_c, acc, b0, j0); emit(acc, b0, j0, 4); }
-        else { float acc[2][8]; head_gemm_32<2>(X, Ws, sh.d_h, sh.d_c, acc, b0, j0); emit(acc, b0, j0, 2); }
-        // rotated part: column pairs [d_c, n_qchunks*64), zero past D; a thread
-        // takes up to 4 (sequence, pair) items and issues their loads first
-        const int npair = (n_qchunks * 64 - sh.d_c) / 2;          // <= 32
-        uint32_t qv[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int e = threadIdx.x + u * blockDim.x, bb = e / npair, k = e % npair, b = c0 + bb;
-            qv[u] = 0;
-            if (bb < 32 && b < sh.B && 2 * k < sh.d_r)
-                qv[u] = *(const uint32_t*)((const bf16*)a.q_r + ((size_t)b * sh.H + h) * sh.d_r + 2 * k);
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int e = threadIdx.x + u * blockDim.x, bb = e / npair, k = e % npair, b = c0 + bb;
-            if (bb >= 32 || b >= sh.B || tpos[bb] < 0) continue;
+        if (!ok) latch_status(a.status, kStatusTimeout);
+    }
+    // RoPE part of q~ and the zero tail (columns d_c .. n_qchunks * 64) meanwhile
+    {
+        const int nrot = n_qchunks * 64 - sh.d_c;            // even
+        for (int e = tid; e < 32 * (nrot / 2); e += kPrepThreads) {
+            const int bb = e / (nrot / 2), k = e % (nrot / 2), b = c0 + bb;
+            if (b >= sh.B) continue;
+            const int64_t t = a.pos[b];
+            if (!lh_pos_ok(sh, t)) continue;
             float v0 = 0.f, v1 = 0.f;
             if (2 * k < sh.d_r) {
-                float sn, cs;
-                pair_sincos(tpos[bb], k, sh.d_r, sh.log2_rope_base, &sn, &cs);
-                const bf16* xq = (const bf16*)&qv[u];
+                const uint32_t qv = *(const uint32_t*)((const bf16*)a.q_r + ((size_t)b * sh.H + h) * sh.d_r + 2 * k);
+                const bf16* xq = (const bf16*)&qv;
                 const float x0 = __bfloat162float(xq[0]), x1 = __bfloat162float(xq[1]);
+                float sn, cs;
+                pair_sincos(t, k, sh.d_r, sh.log2_rope_base, &sn, &cs);
                 v0 = x0 * cs - x1 * sn;
                 v1 = x0 * sn + x1 * cs;
             }
@@ -207,12 +176,36 @@ __global__ void __launch_bounds__(256) k_lh_prep(DecodeArgs a, uint8_t* qimg, in
                 pack_bf16x2(v0, v1);
         }
     }
-    for (int b = h; b < sh.B; b += sh.H) {
+    // latent part: warp w reads TMEM lane quarter w mod 4 (latent rows), sequences
+    // 16 (w / 4) .. 16 (w / 4) + 15
+    const bool done = mbar_wait(&bars[1], (n_kb - 1) & 1);
+    tc_fence_after();
+    {
+        const int quarter = warp & 3, half = warp >> 2;
+        for (int mb = 0; mb < n_kc / 2; ++mb) {
+            float v[16];
+            tmem_ld16(t_d + mb * 32 + half * 16 + ((uint32_t)(quarter * 32) << 16), v);
+            tmem_wait_ld();
+            const int j = mb * 128 + quarter * 32 + lane;      // latent column
+#pragma unroll
+            for (int s = 0; s < 16; ++s) {
+                const int b = c0 + half * 16 + s;
+                if (done && b < sh.B && lh_pos_ok(sh, a.pos[b]))
+                    *(bf16*)(qimg + (size_t)b * img_bytes + (size_t)(j >> 6) * 128 * 128 + sw128_offset(h, j & 63)) =
+                        __float2bfloat16_rn(v[s]);
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(t_d, 128);
+    // in-place slot updates of this group's sequences b with b mod H = h
+    for (int b = c0 + ((h - c0 % sh.H) % sh.H + sh.H) % sh.H; b < min(sh.B, c0 + 32); b += sh.H) {
         __syncthreads();
         decode_update_body<bf16>(a, b);
         uint8_t* img = qimg + (size_t)b * img_bytes;
         const int pad_rows = 128 - sh.H;
-        for (int e = threadIdx.x; e < n_qchunks * pad_rows * 8; e += blockDim.x) {
+        for (int e = tid; e < n_qchunks * pad_rows * 8; e += kPrepThreads) {
             const int c = e / (pad_rows * 8), rr = e % (pad_rows * 8);
             *(uint4*)(img + (size_t)c * 128 * 128 + (size_t)(sh.H + rr / 8) * 128 + (rr % 8) * 16) =
                 make_uint4(0, 0, 0, 0);
@@ -951,8 +944,9 @@ size_t lh_attn_smem(const Shape& sh) {
     return bytes;
 }
 
-size_t lh_stage_smem(const Shape& sh) { return (size_t)sh.d_h * sh.d_c * sizeof(bf16); }
-size_t lh_prep_smem(const Shape& sh) { return lh_stage_smem(sh) + (size_t)sh.d_h * 32 * 4 + 16; }
+size_t lh_prep_smem(const Shape& sh) {
+    return 1024 + (size_t)(sh.d_c / 64) * 16384 + (size_t)((sh.d_h + 63) / 64) * 4096 + 32;
+}
 size_t lh_comb_smem(const Shape& sh) {
     const size_t n_kc = sh.d_c / 64;
     return 1024 + n_kc * 16384 + n_kc * 4096 + (2 * 32 * kMaxClusters + 32) * 4 + 32 + ((size_t)sh.B + 1) * 4;
@@ -1016,20 +1010,20 @@ cudaError_t tc_decode_lh(const DecodeArgs& a, cudaStream_t st, uint64_t* launche
         snprintf(buf, sizeof(buf), "cuTensorMapEncodeTiled (CUresult %d)", (int)r);
         return note_error(buf, cudaErrorInvalidValue);
     }
-    CUtensorMap wuv_map;
-    {
-        // W_UV as [H * d_h rows][d_c] bf16, 128-row x 64-column boxes (rows past
-        // the last head read as zero)
+    // W_UK and W_UV as [H * d_h rows][d_c] bf16, 128-row x 64-column boxes
+    // (rows past the last head read as zero)
+    CUtensorMap wuk_map, wuv_map;
+    for (int w = 0; w < 2; ++w) {
         cuuint64_t d2[2] = {(cuuint64_t)sh.d_c, (cuuint64_t)sh.H * sh.d_h};
         cuuint64_t s2[1] = {(cuuint64_t)sh.d_c * 2};
         cuuint32_t b2[2] = {64, 128};
         cuuint32_t e2[2] = {1, 1};
-        r = encode(&wuv_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a.w_uv), d2, s2, b2, e2,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        r = encode(w == 0 ? &wuk_map : &wuv_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                   const_cast<void*>(w == 0 ? a.w_uk : a.w_uv), d2, s2, b2, e2, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) {
             char buf[96];
-            snprintf(buf, sizeof(buf), "cuTensorMapEncodeTiled W_UV (CUresult %d)", (int)r);
+            snprintf(buf, sizeof(buf), "cuTensorMapEncodeTiled %s (CUresult %d)", w == 0 ? "W_UK" : "W_UV", (int)r);
             return note_error(buf, cudaErrorInvalidValue);
         }
     }
@@ -1075,7 +1069,7 @@ cudaError_t tc_decode_lh(const DecodeArgs& a, cudaStream_t st, uint64_t* launche
     p.part = part;
     p.status = a.status;
 
-    k_lh_prep<<<sh.H, 256, prep_smem, st>>>(a, qimg, p.n_qchunks);
+    k_lh_prep<<<dim3(sh.H, (sh.B + 31) / 32), kPrepThreads, prep_smem, st>>>(wuk_map, a, qimg, p.n_qchunks);
     e = cudaGetLastError();
     if (e != cudaSuccess) return note_error("k_lh_prep launch", e);
     profile_begin(st);
