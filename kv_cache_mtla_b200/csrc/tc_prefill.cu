@@ -65,7 +65,7 @@ struct Bars {
     uint64_t abs_full, abs_done, q_ready;
     uint64_t s_full[2], s_empty[2];
     uint64_t p_full[2], o_done[2];
-    uint64_t fin_s, wuv_full, olat_ready, out_done;
+    uint64_t wuv_full, olat_ready, out_done;
     uint64_t drain[2];
     uint32_t tmem_base;
     volatile int fail;
@@ -128,12 +128,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const int n_chunks = p.n_chunks;
-    const int n_sq = n_chunks - 2;                                       // query chunks in smem; 2 in TMEM
+    const int n_sq = 1;                                                  // query chunk 0 in smem, 1.. in TMEM
     const uint32_t chunk_k = kKT * 128;                                  // one 64-row chunk of a key tile
     const uint32_t stage_bytes = (uint32_t)n_chunks * chunk_k;
     uint8_t* ring = smem;                                                // kStages key tiles
-    uint8_t* q_s = ring + kStages * stage_bytes;                         // n_sq x [128 x 128 B]; W_UK, W_UV
-    uint8_t* qc_s = ring + (kStages - 1) * stage_bytes;                  // qC tile, before key tile kStages-1
+    uint8_t* q_s = ring + kStages * stage_bytes;                         // query chunk 0 [128 x 128 B]
+    // staging in ring stages the key tiles do not use at the time: qC and W_UK
+    // (stages 3 and 2, before key tiles 2 and 3), W_UV (stage 3, after the last
+    // P.V), O_lat (stages 0-1, after the last P.V)
+    uint8_t* qc_s = ring + 3 * stage_bytes;
+    uint8_t* wk_s = ring + 2 * stage_bytes;
+    uint8_t* wv_s = ring + 3 * stage_bytes;
     Bars& bs = *(Bars*)(q_s + (size_t)n_sq * kQ * 128);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -157,12 +162,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
         mbar_init(&bs.q_ready, 8);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bs.s_full[i], 1);
-            mbar_init(&bs.s_empty[i], 8);
+            mbar_init(&bs.s_empty[i], 1);    // P.V of the tile two back is done (P lives in S)
             mbar_init(&bs.p_full[i], 8);
             mbar_init(&bs.o_done[i], 1);
             mbar_init(&bs.drain[i], 1);
         }
-        mbar_init(&bs.fin_s, 1);
         mbar_init(&bs.wuv_full, 1);
         mbar_init(&bs.olat_ready, 8);
         mbar_init(&bs.out_done, 1);
@@ -179,8 +183,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
     const uint32_t tmem = bs.tmem_base;
     const uint32_t t_s0 = tmem;            // S buffers: columns [0, 64) and [64, 128); later the output
     const uint32_t t_o = tmem + 128;       // q~ (absorption), then O: columns [128, 128 + d_c)
-    const uint32_t t_p = tmem + 384;       // P (bf16 pairs): 2 x 32 columns
-    const uint32_t t_q = tmem + 448;       // query chunks n_sq, n_sq + 1 (bf16 pairs): 2 x 32 columns
+    // P (bf16 pairs) of tile k overwrites the first 32 columns of S buffer k & 1
+    const uint32_t t_q = tmem + 384;       // query chunks 1 .. n_chunks-1 (bf16 pairs): 4 x 32 columns
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -189,20 +193,24 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
             tma_prefetch_desc(&maps.slots);
             mbar_arrive_expect_tx(&bs.abs_full, kQ * 128 + dc_chunks * wchunk);
             tma_load_4d(qc_s, &maps.qc, &bs.abs_full, 0, h, p0, b);
-            for (int n = 0; n < dc_chunks; ++n) tma_load_3d(q_s + n * wchunk, &maps.wuk, &bs.abs_full, n * 64, 0, h);
+            for (int n = 0; n < dc_chunks; ++n) tma_load_3d(wk_s + n * wchunk, &maps.wuk, &bs.abs_full, n * 64, 0, h);
             for (int k = 0; k < nft; ++k) {
                 const int st = k % kStages;
                 if (k >= kStages && !waitb(&bs.empty[st], ((k / kStages) - 1) & 1, bs)) break;
-                if (k == kStages - 1 && !waitb(&bs.abs_done, 0, bs)) break;    // qC has been read
+                if (k == 2 && !waitb(&bs.abs_done, 0, bs)) break;    // qC and W_UK have been read
                 mbar_arrive_expect_tx(&bs.full[st], stage_bytes);
                 uint8_t* dst = ring + st * stage_bytes;
                 for (int c = 0; c < n_chunks; ++c)
                     tma_load_3d(dst + c * chunk_k, &maps.slots, &bs.full[st], c * 64, kKT * k, b);
             }
-            if (waitb(&bs.fin_s, 0, bs)) {
+            // W_UV into stage 3 once nothing reads it: after the absorption and every
+            // P.V. olat_ready (one phase) is the safe signal: the softmax warps arrive
+            // on it after the last P.V, and a parity wait on an o_done barrier that
+            // may be phases ahead of this thread could pass or block wrongly.
+            if (waitb(&bs.abs_done, 0, bs) && waitb(&bs.olat_ready, 0, bs)) {
                 mbar_arrive_expect_tx(&bs.wuv_full, dc_chunks * wchunk);
                 for (int n = 0; n < dc_chunks; ++n)
-                    tma_load_3d(q_s + n * wchunk, &maps.wuv, &bs.wuv_full, n * 64, 0, h);
+                    tma_load_3d(wv_s + n * wchunk, &maps.wuv, &bs.wuv_full, n * 64, 0, h);
             }
         }
     } else if (warp == 1) {
@@ -218,7 +226,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
             if (ok) {
                 tc_fence_after();
                 // q~ = qC . W_UK[h]: A = qC [128 x d_h] K-major, B = W_UK[h] [d_h x d_c] MN-major
-                const uint64_t wd = sdesc_sw128(q_a, wchunk, 1024);
+                const uint64_t wd = sdesc_sw128(smem_u32(wk_s), wchunk, 1024);
                 for (int kk = 0; kk < p.d_h / 16; ++kk)
                     umma_bf16(t_o, desc_add(qc_d, kk * 32), desc_add(wd, kk * 2048), id_abs, kk > 0);
                 umma_commit(&bs.abs_done);
@@ -238,11 +246,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
                     for (int kk = 0; kk < 4; ++kk)
                         umma_bf16(ts, desc_add(qc, kk * 32), desc_add(kc, kk * 32), id_s, (c | kk) != 0);
                 }
-#pragma unroll
-                for (int c = 0; c < 2; ++c) {
+                for (int c = 0; c < n_chunks - n_sq; ++c) {
                     const uint64_t kc = desc_add(kd, (n_sq + c) * chunk_k);
                     // K-steps past D (the zero-filled tail of the last chunk) are skipped
-                    const int kst = c == 1 ? last_ksteps : 4;
+                    const int kst = c == n_chunks - n_sq - 1 ? last_ksteps : 4;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         if (kk < kst)
@@ -250,16 +257,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
                 }
                 umma_commit(&bs.s_full[k & 1]);
             }
-            umma_commit(&bs.fin_s);      // every score MMA is done: q_s may take W_UV
             if (!bs.fail && waitb(&bs.olat_ready, 0, bs) && waitb(&bs.wuv_full, 0, bs)) {
                 tc_fence_after();
                 // out = O_lat . W_UV[h]^T: A = O_lat [128 x d_c] K-major (in the ring),
-                // B = W_UV[h] [d_h x d_c] K-major (in q_s)
-                const uint64_t od = sdesc_sw128(ring_a, 16, 1024);
+                // B = W_UV[h] [d_h x d_c] K-major (in ring stage 3)
+                const uint64_t od = sdesc_sw128(ring_a, 16, 1024), wv_d = sdesc_sw128(smem_u32(wv_s), 16, 1024);
                 for (int kk = 0; kk < p.d_c / 16; ++kk) {
                     const int c = kk >> 2;
                     umma_bf16(t_s0, desc_add(od, c * kQ * 128 + (kk & 3) * 32),
-                              desc_add(q_d, c * wchunk + (kk & 3) * 32), id_out, kk > 0);
+                              desc_add(wv_d, c * wchunk + (kk & 3) * 32), id_out, kk > 0);
                 }
                 umma_commit(&bs.out_done);
             }
@@ -277,10 +283,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
                 const uint64_t vd = sdesc_sw128(ring_a + (k % kStages) * stage_bytes, chunk_k, 1024);
 #pragma unroll
                 for (int kk = 0; kk < kKT / 16; ++kk)
-                    umma_bf16_ts(t_o, t_p + (k & 1) * 32 + kk * 8, desc_add(vd, kk * 2048), id_o,
+                    umma_bf16_ts(t_o, t_s0 + (k & 1) * 64 + kk * 8, desc_add(vd, kk * 2048), id_o,
                                  (k > 0 || kk > 0) ? 1u : 0u);
                 umma_commit(&bs.empty[k % kStages]);
                 umma_commit(&bs.o_done[k & 1]);
+                umma_commit(&bs.s_empty[k & 1]);   // S buffer k & 1 (which held P) is free
             }
         }
     } else {
@@ -371,7 +378,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bs.s_empty[k & 1]);
             const int j0 = kKT * k + 32 * hc;
             float mt = -INFINITY;
 #pragma unroll
@@ -381,6 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
             }
             bs.red[k & 1][hc][r] = mt;
             named_sync(1, 256);
+            tc_fence_after();                         // the other half's TMEM reads are done
             mt = fmaxf(mt, bs.red[k & 1][hc ^ 1][r]);
             // lazy rescale: the reference maximum moves only when the tile's maximum
             // exceeds it by more than 2^8 (P stays <= 256); both halves decide alike
@@ -410,8 +417,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
                 }
                 tmem_wait_st();
             }
-            if (k >= 2) waitb(&bs.o_done[k & 1], ((k >> 1) - 1) & 1, bs);   // P.V of tile k-2 read this P buffer
-            tmem_st16_u(t_p + (k & 1) * 32 + hc * 16 + lane_off, w);
+            // P over the first 32 columns of this tile's S buffer (both halves have
+            // read their scores: the barrier above)
+            tmem_st16_u(t_s0 + (k & 1) * 64 + hc * 16 + lane_off, w);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
@@ -492,7 +500,7 @@ int n_chunks_of(const Shape& sh) { return (sh.D + 63) / 64; }
 
 size_t prefill_smem_bytes(const Shape& sh) {
     const size_t nc = n_chunks_of(sh);
-    return 1024 + kStages * nc * kKT * 128 + (nc - 2) * kQ * 128 + ((sizeof(Bars) + 15) & ~(size_t)15);
+    return 1024 + kStages * nc * kKT * 128 + kQ * 128 + ((sizeof(Bars) + 15) & ~(size_t)15);
 }
 
 cudaError_t make_map(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* m, const void* base, int rank,
