@@ -372,3 +372,59 @@ def test_decode_many_heads(H, s):
         j = pos[b] // s
         assert rel_err(np64(pb.buf.cache[b, j]), cache_o[b, j]) <= 4e-3
     assert rel_err(np64(pb.buf.open_slot), acc_o) <= 1e-5
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("B,N", [(1, 65536), (40, 4096)])
+def test_large_head_decode_split_extremes(B, N):
+    """The large-head decode where one sequence is split over every cluster
+    (B=1: more partials per sequence than a warp has lanes) and where the
+    batch spans two 32-sequence groups of the prep and combine blocks (B=40)."""
+    wl = inputs.LARGE_LATENT.with_(B=B)
+    max_slots = N // wl.s
+    w = inputs.weights(wl)
+    toks = inputs.tokens(wl, 1, stream=2)
+    cache0 = inputs.synthetic_cache(wl, N - 1, max_slots)
+    pb = Problem(wl, max_slots=max_slots, weights=w)
+    pb.buf.cache.copy_(cache0["cache"].to(pb.dt))
+    pb.buf.open_slot.copy_(cache0["acc"])
+    rng = np.random.default_rng(B)
+    pos = np.full(B, N - 1) if B == 1 else rng.integers(0, N, size=B)
+    out = np64(pb.decode(toks, 0, pos))
+    sample = [0] if B == 1 else [0, 31, 32, 39]
+    sub = lambda x: x[sample]
+    cfg = oracle_cfg(wl, B=len(sample))
+    cache_o = cache0["cache"][sample].double().numpy().copy()
+    acc_o = cache0["acc"][sample].double().numpy().copy()
+    ref = oracle.decode_step(cfg, sub(toks["c"][:, 0]), sub(toks["kr"][:, 0]), sub(toks["qc"][:, 0]),
+                             sub(toks["qr"][:, 0]), w["w_uk"], w["w_uv"], pos[sample], cache_o, acc_o,
+                             gate_in=sub(toks["gate_in"][:, 0]))
+    assert rel_err(out[sample], ref["out"]) <= TOL["bf16"]
+    for i, b in enumerate(sample):
+        j = pos[b] // wl.s
+        assert rel_err(np64(pb.buf.cache[b, j]), cache_o[i, j]) <= 4e-3
+    assert rel_err(np64(pb.buf.open_slot[sample]), acc_o) <= 1e-5
+
+
+@pytest.mark.gpu
+def test_small_head_decode_one_long_sequence():
+    """Speech-decode widths with B=1 and 32768 slots: the one sequence is split
+    over every CTA of the grid, and the combine merges all of their partials."""
+    wl = inputs.SPEECH_DECODE.with_(B=1)
+    N = 65536
+    max_slots = N // wl.s
+    w = inputs.weights(wl)
+    toks = inputs.tokens(wl, 1, stream=2)
+    cache0 = inputs.synthetic_cache(wl, N - 1, max_slots)
+    pb = Problem(wl, max_slots=max_slots, weights=w)
+    pb.buf.cache.copy_(cache0["cache"].to(pb.dt))
+    pb.buf.open_slot.copy_(cache0["acc"])
+    pos = np.array([N - 1])
+    out = np64(pb.decode(toks, 0, pos))
+    cfg = oracle_cfg(wl)
+    cache_o = cache0["cache"].double().numpy().copy()
+    acc_o = cache0["acc"].double().numpy().copy()
+    ref = oracle.decode_step(cfg, toks["c"][:, 0], toks["kr"][:, 0], toks["qc"][:, 0], toks["qr"][:, 0],
+                             w["w_uk"], w["w_uv"], pos, cache_o, acc_o, G=w["gate_w"], g=w["gate_b"])
+    assert rel_err(out, ref["out"]) <= TOL["bf16"]
+    assert rel_err(np64(pb.buf.open_slot), acc_o) <= 1e-5
