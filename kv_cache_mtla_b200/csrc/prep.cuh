@@ -224,7 +224,7 @@ template <> __device__ __forceinline__ void store8<bf16>(bf16* p, const float* v
 // last one) and, for the slot holding token T-1, the unrounded open slot.
 // One warp per slot: grid (ceil(ceil(T/s) / 8), B), 256 threads.
 template <typename T, typename PT>
-__global__ void __launch_bounds__(256) k_prefill_scan(PrefillArgs a, PT* P) {
+__global__ void __launch_bounds__(256) k_prefill_scan(PrefillArgs a, PT* P, float2* rope_tab = nullptr) {
     const Shape sh = a.sh;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int b = blockIdx.y;
@@ -290,6 +290,8 @@ __global__ void __launch_bounds__(256) k_prefill_scan(PrefillArgs a, PT* P) {
             if (uo >= nu) continue;
             float sn, cs;
             pair_sincos_f(u0 + uo, rope_freq[k], &sn, &cs);
+            // (cos, sin) of every position for the queries' RoPE (sequence 0 writes it)
+            if (rope_tab && b == 0) rope_tab[(size_t)(u0 + uo) * (sh.d_r / 2) + k] = make_float2(cs, sn);
             const float x0 = to_f<T>(kr[(size_t)uo * sh.d_r + 2 * k]);
             const float x1 = to_f<T>(kr[(size_t)uo * sh.d_r + 2 * k + 1]);
             a0 = fmaf(wv[uo], x0 * cs - x1 * sn, a0);

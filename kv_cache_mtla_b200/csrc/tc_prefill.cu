@@ -56,6 +56,7 @@ struct PreTC {
     double log2_rope_base;
     const bf16* q_r;  // [B, T, H, d_r]
     const bf16* P;    // [B, T, D]: partial slots from the scan (the own-slot keys)
+    const float2* rope_tab;   // [T, d_r / 2]: (cos, sin) of every position, from the scan
     bf16* out;        // [B, T, H, d_h]
     int* status;
 };
@@ -203,11 +204,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
                 for (int c = 0; c < n_chunks; ++c)
                     tma_load_3d(dst + c * chunk_k, &maps.slots, &bs.full[st], c * 64, kKT * k, b);
             }
-            // W_UV into stage 3 once nothing reads it: after the absorption and every
-            // P.V. olat_ready (one phase) is the safe signal: the softmax warps arrive
-            // on it after the last P.V, and a parity wait on an o_done barrier that
-            // may be phases ahead of this thread could pass or block wrongly.
-            if (waitb(&bs.abs_done, 0, bs) && waitb(&bs.olat_ready, 0, bs)) {
+            // W_UV into stage 3 as soon as nothing reads it: after the absorption (qC)
+            // and the P.V of the last tile in stage 3. This thread waited the previous
+            // phase of empty[3] when it loaded that tile, so the parity wait is exact.
+            const int t3 = nft >= 4 ? nft - 1 - ((nft - 4) & 3) : -1;   // last tile in stage 3
+            if (waitb(&bs.abs_done, 0, bs) && (t3 < 0 || waitb(&bs.empty[3], (t3 >> 2) & 1, bs))) {
                 mbar_arrive_expect_tx(&bs.wuv_full, dc_chunks * wchunk);
                 for (int n = 0; n < dc_chunks; ++n)
                     tma_load_3d(wv_s + n * wchunk, &maps.wuv, &bs.wuv_full, n * 64, 0, h);
@@ -318,42 +319,71 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
             }
         };
         float e_own = 0.f;
+        // the own slot's latent half of this thread (<= 128 columns), loaded while
+        // the absorption runs
+        uint4 prow_v[16];
+        {
+            const int half = p.d_c / 2;
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                prow_v[u] = make_uint4(0, 0, 0, 0);
+                if (8 * u < half) prow_v[u] = *(const uint4*)(prow + hc * half + 8 * u);
+            }
+        }
         waitb(&bs.abs_done, 0, bs);
         tc_fence_after();
         {
             const int half = p.d_c / 2;
-            for (int cc = hc * half; cc < (hc + 1) * half; cc += 32) {
-                tmem_ld32(t_o + cc + lane_off, v);
-                tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] = __bfloat162float(__float2bfloat16_rn(v[i]));
-                put_q(cc);
-                ld_row32_bf16(prow + cc, pv);
+            for (int q = 0; q < 4; ++q) {
+                const int cc = hc * half + 32 * q;
+                if (32 * q < half) {
+                    tmem_ld32(t_o + cc + lane_off, v);
+                    tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 32; ++i) e_own = fmaf(v[i], pv[i], e_own);
+                    for (int i = 0; i < 32; ++i) v[i] = __bfloat162float(__float2bfloat16_rn(v[i]));
+                    put_q(cc);
+                    const bf16* pe = (const bf16*)&prow_v[4 * q];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) e_own = fmaf(v[i], __bfloat162float(pe[i]), e_own);
+                }
             }
             if (hc == 1) {
+                const bf16* qr = p.q_r + (((size_t)b * p.T + min(pos, p.T - 1)) * p.H + h) * p.d_r;
+                const float2* cs_row = p.rope_tab + (size_t)min(pos, p.T - 1) * (p.d_r / 2);
                 for (int c0 = p.d_c; c0 < n_chunks * 64; c0 += 32) {
+                    // this block's 32 RoPE columns (zero past d_r): qR, P_pos and the
+                    // (cos, sin) pairs as 16-byte vectors
+                    const int e0 = c0 - p.d_c;
+                    uint4 qv[4], pv4[4];
+                    float4 cs4[8];
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) v[i] = 0.f;
-                    if (row_ok) {
-                        const bf16* qr = p.q_r + (((size_t)b * p.T + pos) * p.H + h) * p.d_r;
+                    for (int u = 0; u < 4; ++u) {
+                        qv[u] = pv4[u] = make_uint4(0, 0, 0, 0);
+                        if (e0 + 8 * u < p.d_r) qv[u] = *(const uint4*)(qr + e0 + 8 * u);
+                        if (c0 + 8 * u < p.D) pv4[u] = *(const uint4*)(prow + c0 + 8 * u);
+                    }
 #pragma unroll
-                        for (int i = 0; i < 32; i += 2) {
-                            const int e = c0 - p.d_c + i;        // RoPE element index
-                            if (e < p.d_r) {
-                                float sn, cs;
-                                pair_sincos(pos, e >> 1, p.d_r, p.log2_rope_base, &sn, &cs);
-                                const float x0 = __bfloat162float(qr[e]), x1 = __bfloat162float(qr[e + 1]);
-                                v[i] = __bfloat162float(__float2bfloat16_rn(x0 * cs - x1 * sn));
-                                v[i + 1] = __bfloat162float(__float2bfloat16_rn(x0 * sn + x1 * cs));
-                            }
+                    for (int u = 0; u < 8; ++u) {
+                        cs4[u] = make_float4(1.f, 0.f, 1.f, 0.f);
+                        if (e0 + 4 * u < p.d_r) cs4[u] = *(const float4*)(cs_row + e0 / 2 + 2 * u);
+                    }
+                    const bf16* qe = (const bf16*)qv;
+                    const bf16* pe = (const bf16*)pv4;
+                    const float* csv = (const float*)cs4;      // cos, sin of pair i / 2
+#pragma unroll
+                    for (int i = 0; i < 32; i += 2) {
+                        v[i] = v[i + 1] = 0.f;
+                        if (row_ok && e0 + i < p.d_r) {
+                            const float cs = csv[i], sn = csv[i + 1];
+                            const float x0 = __bfloat162float(qe[i]), x1 = __bfloat162float(qe[i + 1]);
+                            v[i] = __bfloat162float(__float2bfloat16_rn(x0 * cs - x1 * sn));
+                            v[i + 1] = __bfloat162float(__float2bfloat16_rn(x0 * sn + x1 * cs));
                         }
                     }
                     put_q(c0);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        if (c0 + i < p.D) e_own = fmaf(v[i], __bfloat162float(prow[c0 + i]), e_own);
+                    for (int i = 0; i < 32; ++i) e_own = fmaf(v[i], __bfloat162float(pe[i]), e_own);
                 }
             }
         }
@@ -435,18 +465,22 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
         const float w_own = ex2_approx(es - m_ref);
         {
             const int half = p.d_c / 2;
-            for (int cc = hc * half; cc < (hc + 1) * half; cc += 32) {
-                if (nft > 0) {
-                    tmem_ld32(t_o + cc + lane_off, v);
-                    tmem_wait_ld();
-                } else {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) v[i] = 0.f;
+            for (int q = 0; q < 4; ++q) {
+                const int cc = hc * half + 32 * q;
+                if (32 * q < half) {
+                    if (nft > 0) {
+                        tmem_ld32(t_o + cc + lane_off, v);
+                        tmem_wait_ld();
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) v[i] = 0.f;
+                    }
+                    ld_row32_bf16(prow + cc, pv);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) v[i] = fmaf(w_own, pv[i], v[i]) * inv;
+                    st_row32_bf16(ring, kQ * 128, r, cc, v);
                 }
-                ld_row32_bf16(prow + cc, pv);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] = fmaf(w_own, pv[i], v[i]) * inv;
-                st_row32_bf16(ring, kQ * 128, r, cc, v);
             }
         }
         fence_proxy_async();
@@ -520,13 +554,13 @@ cudaError_t make_map(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* m, cons
 }  // namespace
 
 bool tc_prefill_supported(const Shape& sh) {
-    // d_c >= 128: the smem query chunks also hold W_UK and W_UV
+    // d_c >= 128 and at most 5 slot chunks: 4 query chunks fit in TMEM beside S and O
     return sh.d_h == 64 && sh.d_c % 64 == 0 && sh.d_c >= 128 && sh.d_c <= 256 && n_chunks_of(sh) <= 5 &&
            prefill_smem_bytes(sh) <= 232448 - 1024;
 }
 
 size_t tc_prefill_workspace(const Shape& sh, int T) {
-    return align256((size_t)sh.B * T * sh.D * sizeof(bf16));
+    return align256((size_t)sh.B * T * sh.D * sizeof(bf16)) + align256((size_t)T * (sh.d_r / 2) * sizeof(float2));
 }
 
 cudaError_t tc_prefill(const PrefillArgs& a, cudaStream_t st, uint64_t* launches) {
@@ -575,11 +609,12 @@ cudaError_t tc_prefill(const PrefillArgs& a, cudaStream_t st, uint64_t* launches
     p.log2_rope_base = sh.log2_rope_base;
     p.q_r = (const bf16*)a.q_r;
     p.P = P;
+    p.rope_tab = (const float2*)((char*)a.workspace + align256((size_t)sh.B * T * sh.D * sizeof(bf16)));
     p.out = (bf16*)a.out;
     p.status = a.status;
 
     const int n_slots = (T + sh.s - 1) / sh.s;
-    k_prefill_scan<bf16, bf16><<<dim3((n_slots + 7) / 8, sh.B), 256, 0, st>>>(a, P);
+    k_prefill_scan<bf16, bf16><<<dim3((n_slots + 7) / 8, sh.B), 256, 0, st>>>(a, P, (float2*)p.rope_tab);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return note_error("k_prefill_scan launch", e);
 
