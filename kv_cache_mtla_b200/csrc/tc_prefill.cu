@@ -319,49 +319,46 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
             }
         };
         float e_own = 0.f;
-        // the own slot's latent half of this thread (<= 128 columns), loaded while
-        // the absorption runs
-        uint4 prow_v[16];
-        {
-            const int half = p.d_c / 2;
+        // q~ row in 32-column blocks, the first half of the blocks for hc = 0 and
+        // the rest for hc = 1 (which therefore holds the RoPE part): latent blocks
+        // from TMEM, RoPE blocks rotated with the scan's (cos, sin) table; all
+        // rounded to bf16 into the smem or TMEM query chunks. The own-slot score
+        // q~ . P_pos uses the same rounded values. Every global load of a block is
+        // issued before the wait for the absorption.
+        const int n_blk = n_chunks * 2, nb0 = (n_blk + 1) / 2;
+        const int blk0 = hc == 0 ? 0 : nb0, blk1 = hc == 0 ? nb0 : n_blk;   // <= 5 blocks each
+        const bf16* qr = p.q_r + (((size_t)b * p.T + min(pos, p.T - 1)) * p.H + h) * p.d_r;
+        const float2* cs_row = p.rope_tab + (size_t)min(pos, p.T - 1) * (p.d_r / 2);
+        uint4 pv4[5][4];
 #pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                prow_v[u] = make_uint4(0, 0, 0, 0);
-                if (8 * u < half) prow_v[u] = *(const uint4*)(prow + hc * half + 8 * u);
+        for (int q = 0; q < 5; ++q) {
+            const int c0 = (blk0 + q) * 32;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                pv4[q][u] = make_uint4(0, 0, 0, 0);
+                if (blk0 + q < blk1 && c0 + 8 * u < p.D) pv4[q][u] = *(const uint4*)(prow + c0 + 8 * u);
             }
         }
         waitb(&bs.abs_done, 0, bs);
         tc_fence_after();
-        {
-            const int half = p.d_c / 2;
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int cc = hc * half + 32 * q;
-                if (32 * q < half) {
-                    tmem_ld32(t_o + cc + lane_off, v);
+        for (int q = 0; q < 5; ++q) {
+            const int c0 = (blk0 + q) * 32;
+            if (blk0 + q < blk1) {
+                if (c0 < p.d_c) {
+                    tmem_ld32(t_o + c0 + lane_off, v);
                     tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 32; ++i) v[i] = __bfloat162float(__float2bfloat16_rn(v[i]));
-                    put_q(cc);
-                    const bf16* pe = (const bf16*)&prow_v[4 * q];
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) e_own = fmaf(v[i], __bfloat162float(pe[i]), e_own);
-                }
-            }
-            if (hc == 1) {
-                const bf16* qr = p.q_r + (((size_t)b * p.T + min(pos, p.T - 1)) * p.H + h) * p.d_r;
-                const float2* cs_row = p.rope_tab + (size_t)min(pos, p.T - 1) * (p.d_r / 2);
-                for (int c0 = p.d_c; c0 < n_chunks * 64; c0 += 32) {
-                    // this block's 32 RoPE columns (zero past d_r): qR, P_pos and the
-                    // (cos, sin) pairs as 16-byte vectors
+                } else {
+                    // RoPE columns (zero past d_r): qR and the (cos, sin) pairs as vectors
                     const int e0 = c0 - p.d_c;
-                    uint4 qv[4], pv4[4];
+                    uint4 qv[4];
                     float4 cs4[8];
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
-                        qv[u] = pv4[u] = make_uint4(0, 0, 0, 0);
+                        qv[u] = make_uint4(0, 0, 0, 0);
                         if (e0 + 8 * u < p.d_r) qv[u] = *(const uint4*)(qr + e0 + 8 * u);
-                        if (c0 + 8 * u < p.D) pv4[u] = *(const uint4*)(prow + c0 + 8 * u);
                     }
 #pragma unroll
                     for (int u = 0; u < 8; ++u) {
@@ -369,7 +366,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
                         if (e0 + 4 * u < p.d_r) cs4[u] = *(const float4*)(cs_row + e0 / 2 + 2 * u);
                     }
                     const bf16* qe = (const bf16*)qv;
-                    const bf16* pe = (const bf16*)pv4;
                     const float* csv = (const float*)cs4;      // cos, sin of pair i / 2
 #pragma unroll
                     for (int i = 0; i < 32; i += 2) {
@@ -381,10 +377,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
                             v[i + 1] = __bfloat162float(__float2bfloat16_rn(x0 * sn + x1 * cs));
                         }
                     }
-                    put_q(c0);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) e_own = fmaf(v[i], __bfloat162float(pe[i]), e_own);
                 }
+                put_q(c0);
+                const bf16* pe = (const bf16*)pv4[q];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) e_own = fmaf(v[i], __bfloat162float(pe[i]), e_own);
             }
         }
         tmem_wait_st();
