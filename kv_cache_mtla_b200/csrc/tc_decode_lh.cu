@@ -110,6 +110,9 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
         tmem_alloc(tmem_slot, 128);
         tmem_relinquish();
     }
+    __shared__ double rope_freq[64];                      // base^(-2k / d_r), d_r / 2 <= 64
+    for (int k = tid; k < sh.d_r / 2; k += kPrepThreads)
+        rope_freq[k] = exp2(-(2.0 * k / (double)sh.d_r) * sh.log2_rope_base);
     // qC rows of the 32 sequences (zero past B) as the K-major B operand
     for (int e = tid; e < 32 * n_qc * 8; e += kPrepThreads) {
         const int bb = e / (n_qc * 8), rem = e % (n_qc * 8), c = rem >> 3, u = rem & 7;
@@ -153,21 +156,34 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
         }
         if (!ok) latch_status(a.status, kStatusTimeout);
     }
-    // RoPE part of q~ and the zero tail (columns d_c .. n_qchunks * 64) meanwhile
+    // RoPE part of q~ and the zero tail (columns d_c .. n_qchunks * 64) meanwhile:
+    // every load of a thread's (up to 4) pairs first, frequencies from a table
     {
-        const int nrot = n_qchunks * 64 - sh.d_c;            // even
-        for (int e = tid; e < 32 * (nrot / 2); e += kPrepThreads) {
-            const int bb = e / (nrot / 2), k = e % (nrot / 2), b = c0 + bb;
-            if (b >= sh.B) continue;
-            const int64_t t = a.pos[b];
-            if (!lh_pos_ok(sh, t)) continue;
+        const int nrot = n_qchunks * 64 - sh.d_c;            // even, <= 128
+        const int npair = nrot / 2;
+        constexpr int kPer = 8;                              // 32 * 64 pairs / 256 threads
+        int64_t tv[kPer];
+        uint32_t qv[kPer];
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+            const int e = tid + i * kPrepThreads, bb = e / npair, k = e % npair, b = c0 + bb;
+            tv[i] = -1;
+            qv[i] = 0;
+            if (bb < 32 && b < sh.B) {
+                tv[i] = a.pos[b];
+                if (2 * k < sh.d_r) qv[i] = *(const uint32_t*)((const bf16*)a.q_r + ((size_t)b * sh.H + h) * sh.d_r + 2 * k);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+            const int e = tid + i * kPrepThreads, bb = e / npair, k = e % npair, b = c0 + bb;
+            if (bb >= 32 || b >= sh.B || !lh_pos_ok(sh, tv[i])) continue;
             float v0 = 0.f, v1 = 0.f;
             if (2 * k < sh.d_r) {
-                const uint32_t qv = *(const uint32_t*)((const bf16*)a.q_r + ((size_t)b * sh.H + h) * sh.d_r + 2 * k);
-                const bf16* xq = (const bf16*)&qv;
+                const bf16* xq = (const bf16*)&qv[i];
                 const float x0 = __bfloat162float(xq[0]), x1 = __bfloat162float(xq[1]);
                 float sn, cs;
-                pair_sincos(t, k, sh.d_r, sh.log2_rope_base, &sn, &cs);
+                pair_sincos_f(tv[i], rope_freq[k], &sn, &cs);
                 v0 = x0 * cs - x1 * sn;
                 v1 = x0 * sn + x1 * cs;
             }
@@ -979,7 +995,7 @@ cudaError_t lh_set_smem(K kernel, size_t smem, size_t* done) {
 }  // namespace
 
 bool tc_decode_lh_supported(const Shape& sh) {
-    return sh.H > 32 && sh.H <= 128 && sh.d_c % 128 == 0 && sh.d_c <= 512 && sh.D % 64 == 0 &&
+    return sh.H > 32 && sh.H <= 128 && sh.d_c % 128 == 0 && sh.d_c <= 512 && sh.D % 64 == 0 && sh.d_r <= 128 &&
            (sh.d_h == 64 || sh.d_h == 128 || sh.d_h == 256 || sh.d_h == 512) &&
            (sh.d_c == 128 || sh.d_c == 256 || sh.d_c == 512) && sh.B <= kMaxB && lh_comb_smem(sh) <= 227 * 1024 &&
            lh_prep_smem(sh) <= 227 * 1024 &&
