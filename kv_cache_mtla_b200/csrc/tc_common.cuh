@@ -361,6 +361,18 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
     return d;
 }
 
+// The same for a K-major operand in the 64-byte swizzle (rows of 64 bytes,
+// 8-row groups 512 bytes apart): layout type 4.
+__device__ __forceinline__ uint64_t sdesc_sw64(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1 << 16;
+    d |= (uint64_t)(512u >> 4) << 32;
+    d |= (uint64_t)1 << 46;
+    d |= (uint64_t)4 << 61;
+    return d;
+}
+
 // Advance a descriptor's start address by `bytes` (a multiple of 16): the
 // address field sits in the low bits, so this is one 64-bit add (shared
 // addresses stay below 2^18, no carry out of the 14-bit field).
@@ -411,6 +423,13 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
 // columns (row pitch 128 B; 16-byte units XOR-ed with row mod 8).
 __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t col) {
     return row * 128u + ((((col >> 3) ^ (row & 7u)) & 7u) << 4) + ((col & 7u) << 1);
+}
+
+// Byte offset of bf16 element (row, col) in a K-major tile of 64-byte rows in
+// the 64-byte swizzle (what a TMA load with SWIZZLE_64B writes): the 16-byte
+// unit index is XORed with bits 1-2 of the row.
+__device__ __forceinline__ uint32_t sw64_offset(uint32_t row, uint32_t col) {
+    return row * 64u + ((((col >> 3) ^ (row >> 1)) & 3u) << 4) + ((col & 7u) << 1);
 }
 
 }  // namespace tc

@@ -16,16 +16,21 @@
 //     own partial  one dot product q~ . P_t per row on the CUDA cores; it is
 //                  the softmax's starting point and its value P_t enters the
 //                  output at the end with the row's final weight
-//     finished     64-slot tiles of cache_out  staircase mask on the last
-//                  S = q~ . K^T (M=128 N=64 K=D), online softmax (two threads
+//     finished     128-slot tiles of cache_out  staircase mask on the last
+//                  S = q~ . K^T (M=128 N=128 K=D), online softmax (two threads
 //                  per row, exp2, rescale only when a row max grows by > 2^8),
-//                  O += P . V (M=128 N=d_c K=64, P in TMEM, V = the same tile)
+//                  O += P . V (M=128 N=d_c K=128, P in TMEM, V = the same tile)
 //     epilogue     out = (O / l) . W_UV[h]^T   tcgen05 M=128 N=d_h K=d_c
 // Warp roles: warp 0 TMA, warp 1 absorption / score / output MMAs and TMEM,
 // warps 2-9 softmax, warp 10 P.V MMAs (so P.V, which frees ring stages, never
-// waits behind a score MMA that waits for a load). S and P are double-
-// buffered in TMEM, two query chunks live in TMEM (the MMA's A from tensor
-// memory), and keys stream through a 4-stage TMA ring.
+// waits behind a score MMA that waits for a load). S is double-buffered in
+// TMEM beside O and P (bf16) is written over its own tile's scores. The query
+// image and the keys are shared-memory operands: the latent columns in 64-
+// column chunks with the 128-byte swizzle, the 32 RoPE columns as one chunk
+// with the 64-byte swizzle, so that a 128-slot key tile takes 72 KB and two
+// of them fit beside the query image. 128-slot tiles (N=128 score MMAs, K=128
+// P.V MMAs) halve the per-tile costs of the pipeline (commits, barrier round
+// trips) against 64-slot tiles.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -43,14 +48,15 @@ namespace {
 using namespace tc;
 
 constexpr int kQ = 128;         // query positions per CTA
-constexpr int kKT = 64;         // keys per tile
-constexpr int kStages = 4;
+constexpr int kKT = 128;        // keys per tile
+constexpr int kStages = 2;
+constexpr int kDr = 32;         // RoPE width d_R of this kernel (one 64-byte-swizzled chunk)
 constexpr int kThreads = 352;   // warp 0 TMA, 1 score MMAs, 2-9 softmax, 10 P.V MMAs
 constexpr float kRescaleLog2 = 8.f;
+constexpr int kDh = 64;         // head width d_h of this kernel
 
 struct PreTC {
     int B, T, H, d_h, d_c, d_r, D, s;
-    int n_chunks;     // slot width rounded up to 64, in 64-column chunks
     int n_qtiles;     // ceil(T / 128)
     float scale_log2;
     double log2_rope_base;
@@ -78,7 +84,8 @@ struct Maps {
     CUtensorMap qc;     // (d_h, H, T, B)   box (64, 1, 128, 1)
     CUtensorMap wuk;    // (d_c, d_h, H)    box (64, d_h, 1)
     CUtensorMap wuv;    // (d_c, d_h, H)    box (64, d_h, 1)
-    CUtensorMap slots;  // (D, n_slots, B)  box (64, 64, 1)
+    CUtensorMap slots;  // (D, n_slots, B)  box (64, 128, 1), 128-byte swizzle: latent chunks
+    CUtensorMap slots_r;  // (D, n_slots, B)  box (32, 128, 1), 64-byte swizzle: the RoPE chunk
 };
 
 __device__ __forceinline__ bool waitb(uint64_t* bar, uint32_t parity, Bars& bs) {
@@ -104,10 +111,18 @@ __device__ __forceinline__ void st_row32_bf16(uint8_t* base, uint32_t chunk_byte
     }
 }
 
-// 32 values as 16 packed bf16 pairs (lower element in the lower half).
-__device__ __forceinline__ void pack32(const float* v, uint32_t* w) {
+// Store 32 fp32 values as bf16 into row `row` of a K-major tile of 32 columns
+// (64-byte rows, 64-byte swizzle).
+__device__ __forceinline__ void st_row32_bf16_sw64(uint8_t* base, int row, const float* v) {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+    for (int u = 0; u < 4; ++u) {
+        uint4 pk;
+        pk.x = pack_bf16x2(v[8 * u + 0], v[8 * u + 1]);
+        pk.y = pack_bf16x2(v[8 * u + 2], v[8 * u + 3]);
+        pk.z = pack_bf16x2(v[8 * u + 4], v[8 * u + 5]);
+        pk.w = pack_bf16x2(v[8 * u + 6], v[8 * u + 7]);
+        *(uint4*)(base + sw64_offset(row, 8 * u)) = pk;
+    }
 }
 
 // 32 bf16 of a global row (16-byte aligned) as fp32.
@@ -124,23 +139,28 @@ __device__ __forceinline__ void ld_row32_bf16(const bf16* src, float* v) {
 // One CTA per (128 query positions, sequence, head), heaviest first. The own
 // partial slot of every row is handled on the CUDA cores (its score is one dot
 // product per row; its value enters the output at the end with the row's final
-// weight); the finished slots stream through the tensor cores in 64-slot tiles.
+// weight); the finished slots stream through the tensor cores in 128-slot
+// tiles. DC = d_c (d_h = 64 and d_R = 32 are fixed): every MMA sequence is
+// unrolled at compile time (a runtime loop or branch between tcgen05.mma
+// instructions halves their issue rate).
+template <int DC>
 __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constant__ Maps maps, const PreTC p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    const int n_chunks = p.n_chunks;
-    const int n_sq = 1;                                                  // query chunk 0 in smem, 1.. in TMEM
-    const uint32_t chunk_k = kKT * 128;                                  // one 64-row chunk of a key tile
-    const uint32_t stage_bytes = (uint32_t)n_chunks * chunk_k;
+    constexpr int NL = DC / 64;                                          // latent chunks
+    constexpr uint32_t chunk_k = kKT * 128;                              // one latent chunk of a key tile
+    constexpr uint32_t rope_k = kKT * 64;                                // its RoPE chunk (64-byte rows)
+    constexpr uint32_t stage_bytes = NL * chunk_k + rope_k;
+    constexpr uint32_t q_bytes = NL * kQ * 128 + kQ * 64;
     uint8_t* ring = smem;                                                // kStages key tiles
-    uint8_t* q_s = ring + kStages * stage_bytes;                         // query chunk 0 [128 x 128 B]
+    uint8_t* q_s = ring + kStages * stage_bytes;                         // the query image, same layout
     // staging in ring stages the key tiles do not use at the time: qC and W_UK
-    // (stages 3 and 2, before key tiles 2 and 3), W_UV (stage 3, after the last
-    // P.V), O_lat (stages 0-1, after the last P.V)
-    uint8_t* qc_s = ring + 3 * stage_bytes;
-    uint8_t* wk_s = ring + 2 * stage_bytes;
-    uint8_t* wv_s = ring + 3 * stage_bytes;
-    Bars& bs = *(Bars*)(q_s + (size_t)n_sq * kQ * 128);
+    // (stage 1, before key tile 1), W_UV (stage 1, after the last P.V of a tile
+    // in stage 1), O_lat (stage 0, after the last P.V)
+    uint8_t* qc_s = ring + stage_bytes;
+    uint8_t* wk_s = ring + stage_bytes + kQ * 128;
+    uint8_t* wv_s = ring + stage_bytes;
+    Bars& bs = *(Bars*)(q_s + q_bytes);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int per_qt = p.B * p.H;
@@ -150,8 +170,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
     const int p0 = qt * kQ;
     const int last = min(p0 + kQ - 1, p.T - 1);
     const int nft = (last / p.s + kKT - 1) / kKT;                        // finished-slot tiles
-    const int dc_chunks = p.d_c / 64;
-    const uint32_t wchunk = (uint32_t)p.d_h * 128;                       // one 64-column chunk of W
+    constexpr int dc_chunks = DC / 64;
+    constexpr uint32_t wchunk = (uint32_t)kDh * 128;                     // one 64-column chunk of W
 
     if (tid == 0) {
         for (int i = 0; i < kStages; ++i) {
@@ -182,33 +202,35 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bs.tmem_base;
-    const uint32_t t_s0 = tmem;            // S buffers: columns [0, 64) and [64, 128); later the output
-    const uint32_t t_o = tmem + 128;       // q~ (absorption), then O: columns [128, 128 + d_c)
-    // P (bf16 pairs) of tile k overwrites the first 32 columns of S buffer k & 1
-    const uint32_t t_q = tmem + 384;       // query chunks 1 .. n_chunks-1 (bf16 pairs): 4 x 32 columns
+    const uint32_t t_s0 = tmem;            // S buffers: columns [0, 128) and [128, 256); later the output
+    const uint32_t t_o = tmem + 256;       // q~ (absorption), then O: columns [256, 256 + d_c)
+    // P (bf16 pairs) of tile k overwrites the first 64 columns of S buffer k & 1
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             tma_prefetch_desc(&maps.qc);
             tma_prefetch_desc(&maps.slots);
+            tma_prefetch_desc(&maps.slots_r);
             mbar_arrive_expect_tx(&bs.abs_full, kQ * 128 + dc_chunks * wchunk);
             tma_load_4d(qc_s, &maps.qc, &bs.abs_full, 0, h, p0, b);
             for (int n = 0; n < dc_chunks; ++n) tma_load_3d(wk_s + n * wchunk, &maps.wuk, &bs.abs_full, n * 64, 0, h);
             for (int k = 0; k < nft; ++k) {
-                const int st = k % kStages;
-                if (k >= kStages && !waitb(&bs.empty[st], ((k / kStages) - 1) & 1, bs)) break;
-                if (k == 2 && !waitb(&bs.abs_done, 0, bs)) break;    // qC and W_UK have been read
+                const int st = k & 1;
+                if (k >= kStages && !waitb(&bs.empty[st], ((k >> 1) - 1) & 1, bs)) break;
+                if (k == 1 && !waitb(&bs.abs_done, 0, bs)) break;    // qC and W_UK have been read
                 mbar_arrive_expect_tx(&bs.full[st], stage_bytes);
                 uint8_t* dst = ring + st * stage_bytes;
-                for (int c = 0; c < n_chunks; ++c)
+#pragma unroll
+                for (int c = 0; c < NL; ++c)
                     tma_load_3d(dst + c * chunk_k, &maps.slots, &bs.full[st], c * 64, kKT * k, b);
+                tma_load_3d(dst + NL * chunk_k, &maps.slots_r, &bs.full[st], DC, kKT * k, b);
             }
-            // W_UV into stage 3 as soon as nothing reads it: after the absorption (qC)
-            // and the P.V of the last tile in stage 3. This thread waited the previous
-            // phase of empty[3] when it loaded that tile, so the parity wait is exact.
-            const int t3 = nft >= 4 ? nft - 1 - ((nft - 4) & 3) : -1;   // last tile in stage 3
-            if (waitb(&bs.abs_done, 0, bs) && (t3 < 0 || waitb(&bs.empty[3], (t3 >> 2) & 1, bs))) {
+            // W_UV into stage 1 as soon as nothing reads it: after the absorption (qC)
+            // and the P.V of the last tile in stage 1. This thread waited the previous
+            // phase of empty[1] when it loaded that tile, so the parity wait is exact.
+            const int t1 = nft >= 2 ? ((nft - 1) & 1 ? nft - 1 : nft - 2) : -1;   // last tile in stage 1
+            if (waitb(&bs.abs_done, 0, bs) && (t1 < 0 || waitb(&bs.empty[1], (t1 >> 1) & 1, bs))) {
                 mbar_arrive_expect_tx(&bs.wuv_full, dc_chunks * wchunk);
                 for (int n = 0; n < dc_chunks; ++n)
                     tma_load_3d(wv_s + n * wchunk, &maps.wuv, &bs.wuv_full, n * 64, 0, h);
@@ -217,53 +239,52 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
     } else if (warp == 1) {
         // ------------------------------------------------------------ absorption, score and output MMAs
         if (lane == 0) {
-            const uint32_t id_abs = idesc_bf16_f32(128, p.d_c, false, true);
+            const uint32_t id_abs = idesc_bf16_f32(128, DC, false, true);
             const uint32_t id_s = idesc_bf16_f32(128, kKT, false, false);
-            const uint32_t id_out = idesc_bf16_f32(128, p.d_h, false, false);
+            const uint32_t id_out = idesc_bf16_f32(128, kDh, false, false);
             const uint32_t ring_a = smem_u32(ring), q_a = smem_u32(q_s);
-            const uint64_t q_d = sdesc_sw128(q_a, 16, 1024), qc_d = sdesc_sw128(smem_u32(qc_s), 16, 1024);
-            const int last_ksteps = (p.D - 64 * (n_chunks - 1)) / 16;   // D is a multiple of 16
+            const uint64_t q_d = sdesc_sw128(q_a, 16, 1024), q_r = sdesc_sw64(q_a + NL * kQ * 128);
+            const uint64_t qc_d = sdesc_sw128(smem_u32(qc_s), 16, 1024);
             bool ok = waitb(&bs.abs_full, 0, bs);
             if (ok) {
                 tc_fence_after();
                 // q~ = qC . W_UK[h]: A = qC [128 x d_h] K-major, B = W_UK[h] [d_h x d_c] MN-major
                 const uint64_t wd = sdesc_sw128(smem_u32(wk_s), wchunk, 1024);
-                for (int kk = 0; kk < p.d_h / 16; ++kk)
+#pragma unroll
+                for (int kk = 0; kk < kDh / 16; ++kk)
                     umma_bf16(t_o, desc_add(qc_d, kk * 32), desc_add(wd, kk * 2048), id_abs, kk > 0);
                 umma_commit(&bs.abs_done);
                 ok = waitb(&bs.q_ready, 0, bs);
             }
             for (int k = 0; ok && k < nft; ++k) {
-                const int st = k % kStages;
-                if (!waitb(&bs.full[st], (k / kStages) & 1, bs)) break;
+                const int st = k & 1;
+                if (!waitb(&bs.full[st], (k >> 1) & 1, bs)) break;
                 if (k >= 2 && !waitb(&bs.s_empty[k & 1], ((k >> 1) - 1) & 1, bs)) break;
                 tc_fence_after();
-                // S = q~ . K^T (M = 128 queries, N = 64 slots, K = D)
-                const uint64_t kd = sdesc_sw128(ring_a + st * stage_bytes, 16, 1024);
-                const uint32_t ts = t_s0 + (k & 1) * 64;
-                for (int c = 0; c < n_sq; ++c) {
+                // S = q~ . K^T (M = 128 queries, N = 128 slots, K = D): the latent
+                // chunks, then the two K-steps of the RoPE chunk
+                const uint32_t stage_a = ring_a + st * stage_bytes;
+                const uint64_t kd = sdesc_sw128(stage_a, 16, 1024), kr = sdesc_sw64(stage_a + NL * chunk_k);
+                const uint32_t ts = t_s0 + (k & 1) * kKT;
+#pragma unroll
+                for (int c = 0; c < NL; ++c) {
                     const uint64_t qc = desc_add(q_d, c * kQ * 128), kc = desc_add(kd, c * chunk_k);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         umma_bf16(ts, desc_add(qc, kk * 32), desc_add(kc, kk * 32), id_s, (c | kk) != 0);
                 }
-                for (int c = 0; c < n_chunks - n_sq; ++c) {
-                    const uint64_t kc = desc_add(kd, (n_sq + c) * chunk_k);
-                    // K-steps past D (the zero-filled tail of the last chunk) are skipped
-                    const int kst = c == n_chunks - n_sq - 1 ? last_ksteps : 4;
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        if (kk < kst)
-                            umma_bf16_ts(ts, t_q + c * 32 + kk * 8, desc_add(kc, kk * 32), id_s, (n_sq + c) + kk != 0);
-                }
+                for (int kk = 0; kk < kDr / 16; ++kk)
+                    umma_bf16(ts, desc_add(q_r, kk * 32), desc_add(kr, kk * 32), id_s, 1u);
                 umma_commit(&bs.s_full[k & 1]);
             }
             if (!bs.fail && waitb(&bs.olat_ready, 0, bs) && waitb(&bs.wuv_full, 0, bs)) {
                 tc_fence_after();
-                // out = O_lat . W_UV[h]^T: A = O_lat [128 x d_c] K-major (in the ring),
-                // B = W_UV[h] [d_h x d_c] K-major (in ring stage 3)
+                // out = O_lat . W_UV[h]^T: A = O_lat [128 x d_c] K-major (ring stage 0),
+                // B = W_UV[h] [d_h x d_c] K-major (ring stage 1)
                 const uint64_t od = sdesc_sw128(ring_a, 16, 1024), wv_d = sdesc_sw128(smem_u32(wv_s), 16, 1024);
-                for (int kk = 0; kk < p.d_c / 16; ++kk) {
+#pragma unroll
+                for (int kk = 0; kk < DC / 16; ++kk) {
                     const int c = kk >> 2;
                     umma_bf16(t_s0, desc_add(od, c * kQ * 128 + (kk & 3) * 32),
                               desc_add(wv_d, c * wchunk + (kk & 3) * 32), id_out, kk > 0);
@@ -275,18 +296,18 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
         // ------------------------------------------------------------ P.V MMAs (own thread: they free
         // ring stages, so they never wait behind a score MMA that waits for a load)
         if (lane == 0) {
-            const uint32_t id_o = idesc_bf16_f32(128, p.d_c, false, true);
+            const uint32_t id_o = idesc_bf16_f32(128, DC, false, true);
             const uint32_t ring_a = smem_u32(ring);
             for (int k = 0; k < nft; ++k) {
                 if (!waitb(&bs.p_full[k & 1], (k >> 1) & 1, bs)) break;
                 tc_fence_after();
-                // O += P . V: A = P [128 x 64] in TMEM, B = V = key tile latent [64 x d_c] MN-major
-                const uint64_t vd = sdesc_sw128(ring_a + (k % kStages) * stage_bytes, chunk_k, 1024);
+                // O += P . V: A = P [128 x 128] in TMEM, B = V = key tile latent [128 x d_c] MN-major
+                const uint64_t vd = sdesc_sw128(ring_a + (k & 1) * stage_bytes, chunk_k, 1024);
 #pragma unroll
                 for (int kk = 0; kk < kKT / 16; ++kk)
-                    umma_bf16_ts(t_o, t_s0 + (k & 1) * 64 + kk * 8, desc_add(vd, kk * 2048), id_o,
+                    umma_bf16_ts(t_o, t_s0 + (k & 1) * kKT + kk * 8, desc_add(vd, kk * 2048), id_o,
                                  (k > 0 || kk > 0) ? 1u : 0u);
-                umma_commit(&bs.empty[k % kStages]);
+                umma_commit(&bs.empty[k & 1]);
                 umma_commit(&bs.o_done[k & 1]);
                 umma_commit(&bs.s_empty[k & 1]);   // S buffer k & 1 (which held P) is free
             }
@@ -305,27 +326,21 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
         const bf16* prow = p.P + ((size_t)b * p.T + min(pos, p.T - 1)) * p.D;   // own partial slot
         float v[32], pv[32];
-        uint32_t w[16];
-        // q~ row: latent part from TMEM (this thread's column half), RoPE part
-        // (hc = 1) from qR; rounded to bf16 into the smem or TMEM query chunks.
-        // The own-slot score q~ . P_pos uses the same rounded values.
+        uint32_t w[32];
+        // q~ row block of 32 columns into the query image: latent columns into the
+        // 128-byte-swizzled chunks, the RoPE block into the 64-byte-swizzled one
         auto put_q = [&](int col) {
-            const int c = col >> 6;
-            if (c < n_sq) {
-                st_row32_bf16(q_s, kQ * 128, r, col, v);
-            } else {
-                pack32(v, w);
-                tmem_st16_u(t_q + (c - n_sq) * 32 + (col & 63) / 2 + lane_off, w);
-            }
+            if (col < DC) st_row32_bf16(q_s, kQ * 128, r, col, v);
+            else st_row32_bf16_sw64(q_s + NL * kQ * 128, r, v);
         };
         float e_own = 0.f;
         // q~ row in 32-column blocks, the first half of the blocks for hc = 0 and
-        // the rest for hc = 1 (which therefore holds the RoPE part): latent blocks
-        // from TMEM, RoPE blocks rotated with the scan's (cos, sin) table; all
-        // rounded to bf16 into the smem or TMEM query chunks. The own-slot score
-        // q~ . P_pos uses the same rounded values. Every global load of a block is
-        // issued before the wait for the absorption.
-        const int n_blk = n_chunks * 2, nb0 = (n_blk + 1) / 2;
+        // the rest for hc = 1 (which therefore holds the RoPE block): latent blocks
+        // from TMEM, the RoPE block rotated with the scan's (cos, sin) table; all
+        // rounded to bf16 into the query image. The own-slot score q~ . P_pos uses
+        // the same rounded values. Every global load of a block is issued before
+        // the wait for the absorption.
+        constexpr int n_blk = NL * 2 + 1, nb0 = (n_blk + 1) / 2;
         const int blk0 = hc == 0 ? 0 : nb0, blk1 = hc == 0 ? nb0 : n_blk;   // <= 5 blocks each
         const bf16* qr = p.q_r + (((size_t)b * p.T + min(pos, p.T - 1)) * p.H + h) * p.d_r;
         const float2* cs_row = p.rope_tab + (size_t)min(pos, p.T - 1) * (p.d_r / 2);
@@ -345,14 +360,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
         for (int q = 0; q < 5; ++q) {
             const int c0 = (blk0 + q) * 32;
             if (blk0 + q < blk1) {
-                if (c0 < p.d_c) {
+                if (c0 < DC) {
                     tmem_ld32(t_o + c0 + lane_off, v);
                     tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < 32; ++i) v[i] = __bfloat162float(__float2bfloat16_rn(v[i]));
                 } else {
                     // RoPE columns (zero past d_r): qR and the (cos, sin) pairs as vectors
-                    const int e0 = c0 - p.d_c;
+                    const int e0 = c0 - DC;
                     uint4 qv[4];
                     float4 cs4[8];
 #pragma unroll
@@ -384,7 +399,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
                 for (int i = 0; i < 32; ++i) e_own = fmaf(v[i], __bfloat162float(pe[i]), e_own);
             }
         }
-        tmem_wait_st();
         fence_proxy_async();
         tc_fence_before();
         __syncwarp();
@@ -400,15 +414,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
         for (int k = 0; k < nft; ++k) {
             waitb(&bs.s_full[k & 1], (k >> 1) & 1, bs);
             tc_fence_after();
-            float sv[32];
-            tmem_ld32(t_s0 + (k & 1) * 64 + hc * 32 + lane_off, sv);
+            float sv[64];
+            tmem_ld32(t_s0 + (k & 1) * kKT + hc * 64 + lane_off, sv);
+            tmem_ld32(t_s0 + (k & 1) * kKT + hc * 64 + 32 + lane_off, sv + 32);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
-            const int j0 = kKT * k + 32 * hc;
+            const int j0 = kKT * k + 64 * hc;
             float mt = -INFINITY;
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
+            for (int c = 0; c < 64; ++c) {
                 sv[c] = (j0 + c < fin_lim) ? sv[c] * p.scale_log2 : -INFINITY;
                 mt = fmaxf(mt, sv[c]);
             }
@@ -423,7 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
             const float fac = ex2_approx(m_ref - nm);
             float rs = 0.f;
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
+            for (int c = 0; c < 32; ++c) {
                 const float q0 = ex2_approx(sv[2 * c] - nm), q1 = ex2_approx(sv[2 * c + 1] - nm);
                 rs += q0 + q1;
                 w[c] = pack_bf16x2(q0, q1);
@@ -434,7 +449,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
                 waitb(&bs.o_done[(k - 1) & 1], ((k - 1) >> 1) & 1, bs);
                 tc_fence_after();
                 const float f = need ? fac : 1.f;
-                const int half = p.d_c / 2;
+                constexpr int half = DC / 2;
                 for (int cc = hc * half; cc < (hc + 1) * half; cc += 32) {
                     tmem_ld32(t_o + cc + lane_off, v);
                     tmem_wait_ld();
@@ -444,16 +459,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
                 }
                 tmem_wait_st();
             }
-            // P over the first 32 columns of this tile's S buffer (both halves have
+            // P over the first 64 columns of this tile's S buffer (both halves have
             // read their scores: the barrier above)
-            tmem_st16_u(t_s0 + (k & 1) * 64 + hc * 16 + lane_off, w);
+            tmem_st32_u(t_s0 + (k & 1) * kKT + hc * 32 + lane_off, w);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bs.p_full[k & 1]);
             m_ref = nm;
         }
-        // epilogue: O_lat = (O + w_own P_pos[:d_c]) / l -> bf16 K-major (in the ring), then out
+        // epilogue: O_lat = (O + w_own P_pos[:d_c]) / l -> bf16 K-major (ring stage 0), then out
         if (nft > 0) waitb(&bs.o_done[(nft - 1) & 1], ((nft - 1) >> 1) & 1, bs);
         tc_fence_after();
         bs.xs[hc][r] = l;
@@ -461,7 +476,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
         const float inv = 1.f / (bs.xs[0][r] + bs.xs[1][r]);
         const float w_own = ex2_approx(es - m_ref);
         {
-            const int half = p.d_c / 2;
+            constexpr int half = DC / 2;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const int cc = hc * half + 32 * q;
@@ -486,11 +501,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
         if (lane == 0) mbar_arrive(&bs.olat_ready);
         waitb(&bs.out_done, 0, bs);
         tc_fence_after();
-        for (int cc = hc * (p.d_h / 2); cc < (hc + 1) * (p.d_h / 2); cc += 32) {
+        for (int cc = hc * (kDh / 2); cc < (hc + 1) * (kDh / 2); cc += 32) {
             tmem_ld32(t_s0 + cc + lane_off, v);
             tmem_wait_ld();
             if (row_ok) {
-                bf16* o = p.out + (((size_t)b * p.T + pos) * p.H + h) * p.d_h + cc;
+                bf16* o = p.out + (((size_t)b * p.T + pos) * p.H + h) * kDh + cc;
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
                     uint4 pk;
@@ -527,18 +542,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
 
 // ---------------------------------------------------------------- host side
 
-int n_chunks_of(const Shape& sh) { return (sh.D + 63) / 64; }
-
+// Key tile and query image: d_c / 64 latent chunks of 128 rows x 128 B plus a
+// RoPE chunk of 128 rows x 64 B.
 size_t prefill_smem_bytes(const Shape& sh) {
-    const size_t nc = n_chunks_of(sh);
-    return 1024 + kStages * nc * kKT * 128 + kQ * 128 + ((sizeof(Bars) + 15) & ~(size_t)15);
+    const size_t tile = (size_t)(sh.d_c / 64) * kKT * 128 + kKT * 64;
+    return 1024 + (kStages + 1) * tile + ((sizeof(Bars) + 15) & ~(size_t)15);
 }
 
 cudaError_t make_map(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* m, const void* base, int rank,
-                     const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box, const char* what) {
+                     const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box, const char* what,
+                     CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
     cuuint32_t estr[5] = {1, 1, 1, 1, 1};
     CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides, box, estr,
-                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {
         char buf[128];
@@ -548,12 +564,20 @@ cudaError_t make_map(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* m, cons
     return cudaSuccess;
 }
 
+// The compiled instances: d_h = 64, d_R = 32 and d_c = 256 or 128. Other
+// widths take the CUDA-core prefill.
+using PrefillKernel = void (*)(Maps, PreTC);
+PrefillKernel prefill_kernel(const Shape& sh) {
+    if (sh.d_h != kDh || sh.d_r != kDr) return nullptr;
+    if (sh.d_c == 256) return k_prefill_tc<256>;
+    if (sh.d_c == 128) return k_prefill_tc<128>;
+    return nullptr;
+}
+
 }  // namespace
 
 bool tc_prefill_supported(const Shape& sh) {
-    // d_c >= 128 and at most 5 slot chunks: 4 query chunks fit in TMEM beside S and O
-    return sh.d_h == 64 && sh.d_c % 64 == 0 && sh.d_c >= 128 && sh.d_c <= 256 && n_chunks_of(sh) <= 5 &&
-           prefill_smem_bytes(sh) <= 232448 - 1024;
+    return prefill_kernel(sh) != nullptr && prefill_smem_bytes(sh) <= 232448 - 1024;
 }
 
 size_t tc_prefill_workspace(const Shape& sh, int T) {
@@ -589,6 +613,9 @@ cudaError_t tc_prefill(const PrefillArgs& a, cudaStream_t st, uint64_t* launches
         cuuint64_t s[2] = {E * sh.D, E * sh.max_slots * sh.D};
         cuuint32_t bx[3] = {64, kKT, 1};
         cudaError_t e = make_map(enc, &maps.slots, a.cache_out, 3, d, s, bx, "cache_out");
+        cuuint32_t bxr[3] = {kDr, kKT, 1};
+        if (e == cudaSuccess)
+            e = make_map(enc, &maps.slots_r, a.cache_out, 3, d, s, bxr, "cache_out RoPE", CU_TENSOR_MAP_SWIZZLE_64B);
         if (e != cudaSuccess) return e;
     }
     PreTC p;
@@ -600,7 +627,6 @@ cudaError_t tc_prefill(const PrefillArgs& a, cudaStream_t st, uint64_t* launches
     p.d_r = sh.d_r;
     p.D = sh.D;
     p.s = sh.s;
-    p.n_chunks = n_chunks_of(sh);
     p.n_qtiles = (T + kQ - 1) / kQ;
     p.scale_log2 = sh.scale * 1.4426950408889634f;
     p.log2_rope_base = sh.log2_rope_base;
@@ -616,18 +642,14 @@ cudaError_t tc_prefill(const PrefillArgs& a, cudaStream_t st, uint64_t* launches
     if (e != cudaSuccess) return note_error("k_prefill_scan launch", e);
 
     const size_t smem = prefill_smem_bytes(sh);
-    static size_t done[64] = {0};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev < 0 || dev >= 64) dev = 0;
-    if (done[dev] < smem) {
-        e = cudaFuncSetAttribute(k_prefill_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return note_error("cudaFuncSetAttribute(k_prefill_tc)", e);
-        done[dev] = smem;
-    }
+    const PrefillKernel kern = prefill_kernel(sh);
+    if (!kern) return note_error("tc_prefill: no compiled instance for these widths", cudaErrorInvalidValue);
+    // the attribute is set on every call: it is per kernel instance and device
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return note_error("cudaFuncSetAttribute(k_prefill_tc)", e);
     const unsigned grid = (unsigned)p.n_qtiles * sh.B * sh.H;
     profile_begin(st);
-    k_prefill_tc<<<grid, kThreads, smem, st>>>(maps, p);
+    kern<<<grid, kThreads, smem, st>>>(maps, p);
     profile_end(st);
     *launches += 2;
     return note_error("k_prefill_tc launch", cudaGetLastError());
