@@ -411,6 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
         // starting point (reference maximum es, weight 1 in the row sum)
         float m_ref = es, l = hc == 0 ? 1.f : 0.f;    // l: this thread's half of the row sum
         const int fin_lim = pos / p.s;                // finished slots this row may see
+        const int min_fin = p0 / p.s;                 // ... and the first row of the tile
         for (int k = 0; k < nft; ++k) {
             waitb(&bs.s_full[k & 1], (k >> 1) & 1, bs);
             tc_fence_after();
@@ -420,13 +421,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
+            // raw scores: the scale is folded into the exponent below. The slot mask
+            // only matters on tiles that reach past the first row's limit (a test
+            // uniform across the CTA). Maxima and sums in four independent chains.
             const int j0 = kKT * k + 64 * hc;
-            float mt = -INFINITY;
+            if (kKT * (k + 1) > min_fin) {
 #pragma unroll
-            for (int c = 0; c < 64; ++c) {
-                sv[c] = (j0 + c < fin_lim) ? sv[c] * p.scale_log2 : -INFINITY;
-                mt = fmaxf(mt, sv[c]);
+                for (int c = 0; c < 64; ++c)
+                    if (j0 + c >= fin_lim) sv[c] = -INFINITY;
             }
+            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+            for (int c = 0; c < 64; ++c) m4[c & 3] = fmaxf(m4[c & 3], sv[c]);
+            float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * p.scale_log2;
             bs.red[k & 1][hc][r] = mt;
             named_sync(1, 256);
             tc_fence_after();                         // the other half's TMEM reads are done
@@ -436,14 +443,15 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
             const bool upd = mt > m_ref + kRescaleLog2;
             const float nm = upd ? mt : m_ref;
             const float fac = ex2_approx(m_ref - nm);
-            float rs = 0.f;
+            float rs4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int c = 0; c < 32; ++c) {
-                const float q0 = ex2_approx(sv[2 * c] - nm), q1 = ex2_approx(sv[2 * c + 1] - nm);
-                rs += q0 + q1;
+                const float q0 = ex2_approx(fmaf(sv[2 * c], p.scale_log2, -nm));
+                const float q1 = ex2_approx(fmaf(sv[2 * c + 1], p.scale_log2, -nm));
+                rs4[c & 3] += q0 + q1;
                 w[c] = pack_bf16x2(q0, q1);
             }
-            l = fmaf(l, fac, rs);
+            l = fmaf(l, fac, (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
             const bool need = upd && k > 0;           // O holds tiles 0..k-1
             if (__any_sync(0xffffffffu, need)) {
                 waitb(&bs.o_done[(k - 1) & 1], ((k - 1) >> 1) & 1, bs);
