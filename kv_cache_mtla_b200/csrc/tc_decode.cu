@@ -47,6 +47,8 @@ constexpr float kRescaleLog2 = 8.f;
 constexpr int kPrepAbsThreads = 128;   // prep: W_UK product threads (plus one RoPE warp)
 constexpr int kMaxGrid = 160;  // >= SMs of any sm_100 part; sizes the partial buffer
 constexpr int kMaxB = 2048;
+constexpr int kMaxChunks = 6;     // 64-column chunks of the slot width (supported shapes)
+constexpr int kMaxLatBlocks = 3;  // 128-column latent blocks (d_c <= 384 follows from the above)
 
 struct DecTC {
     int B, H, D, d_c, s, max_slots;
@@ -340,15 +342,44 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 if (it >= 2 && !sb_wait(&bs.s_empty[st], ((it >> 1) - 1) & 1, bs)) break;
                 tc_fence_after();
                 // S^T = K_tile . q~^T (A = slot tile, B = q~ image; both K-major)
+                // The MMAs go out in straight-line groups (one test per group of
+                // four): a runtime loop or a test per MMA halves their issue rate.
                 const uint64_t a0 = sdesc_sw128(ring_a + st * stage_bytes, 16, 1024);
-                for (int c = 0; c < n_chunks; ++c) {
-                    const uint64_t ac = desc_add(a0, c * 16384), bc = desc_add(q_d, c * NH * 128);
-                    // K-steps past D (the zero-filled tail of the last chunk) are skipped
-                    const int kst = c == n_chunks - 1 ? last_ksteps : 4;
+                const uint32_t ts = t_s + st * NH;
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        if (kk < kst)
-                            umma_bf16(t_s + st * NH, desc_add(ac, kk * 32), desc_add(bc, kk * 32), id_s, (c | kk) != 0);
+                for (int c = 0; c < kMaxChunks - 1; ++c) {
+                    if (c < n_chunks - 1) {
+                        const uint64_t ac = desc_add(a0, c * 16384), bc = desc_add(q_d, c * NH * 128);
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            umma_bf16(ts, desc_add(ac, kk * 32), desc_add(bc, kk * 32), id_s, (c | kk) != 0);
+                    }
+                }
+                {
+                    // the last chunk: its K-steps up to D (the zero-filled tail is skipped)
+                    const int cl = n_chunks - 1;
+                    const uint64_t ac = desc_add(a0, cl * 16384), bc = desc_add(q_d, cl * NH * 128);
+                    const uint32_t acc0 = cl > 0 ? 1u : 0u;
+                    switch (last_ksteps) {
+                        case 4:
+                            umma_bf16(ts, ac, bc, id_s, acc0);
+                            umma_bf16(ts, desc_add(ac, 32), desc_add(bc, 32), id_s, 1u);
+                            umma_bf16(ts, desc_add(ac, 64), desc_add(bc, 64), id_s, 1u);
+                            umma_bf16(ts, desc_add(ac, 96), desc_add(bc, 96), id_s, 1u);
+                            break;
+                        case 3:
+                            umma_bf16(ts, ac, bc, id_s, acc0);
+                            umma_bf16(ts, desc_add(ac, 32), desc_add(bc, 32), id_s, 1u);
+                            umma_bf16(ts, desc_add(ac, 64), desc_add(bc, 64), id_s, 1u);
+                            break;
+                        case 2:
+                            umma_bf16(ts, ac, bc, id_s, acc0);
+                            umma_bf16(ts, desc_add(ac, 32), desc_add(bc, 32), id_s, 1u);
+                            break;
+                        default:
+                            umma_bf16(ts, ac, bc, id_s, acc0);
+                            break;
+                    }
                 }
                 umma_commit(&bs.s_full[st]);
                 const bool last = (gt + 1 == gt1) || (j + 1 == starts[b + 1] - starts[b]);
@@ -372,13 +403,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 // O^T += V^T . P^T (A = the slot tile, MN-major; B = P^T, K-major)
                 const uint64_t a0 = sdesc_sw128(ring_a + (k & 1) * stage_bytes, 16384, 1024);
                 const uint64_t b0 = sdesc_sw128(p_a + (k & 1) * 2 * NH * 128, 16, 1024);
-                for (int lb = 0; lb < p.lat_blocks; ++lb) {
-                    const uint64_t al = desc_add(a0, 2 * lb * 16384);
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk)
-                        umma_bf16(t_o + lb * NH, desc_add(al, kk * 2048),
-                                  desc_add(b0, (kk >> 2) * NH * 128 + (kk & 3) * 32), id_o,
-                                  (first && kk == 0) ? 0u : 1u);
+                for (int lb = 0; lb < kMaxLatBlocks; ++lb) {
+                    if (lb < p.lat_blocks) {
+                        const uint64_t al = desc_add(a0, 2 * lb * 16384);
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk)
+                            umma_bf16(t_o + lb * NH, desc_add(al, kk * 2048),
+                                      desc_add(b0, (kk >> 2) * NH * 128 + (kk & 3) * 32), id_o,
+                                      (first && kk == 0) ? 0u : 1u);
+                    }
                 }
                 umma_commit(&bs.empty[k & 1]);
                 umma_commit(&bs.o_done[k & 1]);

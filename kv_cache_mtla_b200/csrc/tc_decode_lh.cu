@@ -44,6 +44,7 @@ using namespace tc;
 
 constexpr int kKT = 64;          // slots per key tile
 constexpr int kStages = 3;
+constexpr int kMaxSq = 4;         // query chunks in shared memory: at most 4 latent + 2 RoPE - 2 in TMEM
 constexpr int kThreads = 352;    // warp 0 TMA, 1 score MMAs, 2-9 softmax, 10 P.V MMAs
 constexpr int kMaxClusters = 80; // >= SMs/2 of any sm_100 part; sizes the partial buffer
 constexpr int kMaxB = 2048;
@@ -418,7 +419,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const uint32_t id_s = idesc_bf16_f32(128, kKT, false, false);
             const uint32_t ring_a = smem_u32(ring);
             const uint64_t q_d = sdesc_sw128(smem_u32(q_s), 16, 1024);
-            const int last_ksteps = (p.D - 64 * (p.n_qchunks - 1)) / 16;   // D is a multiple of 16
             int seg = -1, prev_b = -1, it = 0;
             for (int gt = gt0; gt < gt1; ++gt, ++it) {
                 int b, j;
@@ -436,20 +436,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 // S_c = q~_c . K_c^T (M = 128 heads, N = 64 slots)
                 const uint64_t kd = sdesc_sw128(ring_a + st * stage_bytes, 16, 1024);
                 const uint32_t ts = t_s + (it & 1) * kKT;
-                for (int i = 0; i < n_sq; ++i) {
-                    const uint64_t qi = desc_add(q_d, i * 128 * 128), ki = desc_add(kd, i * kKT * 128);
+                // Straight-line groups of four MMAs with one test per group (a
+                // runtime loop or a test per MMA halves their issue rate). Every
+                // chunk is a full 64 columns (D is a multiple of 64).
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        umma_bf16(ts, desc_add(qi, kk * 32), desc_add(ki, kk * 32), id_s, (i | kk) != 0);
+                for (int i = 0; i < kMaxSq; ++i) {
+                    if (i < n_sq) {
+                        const uint64_t qi = desc_add(q_d, i * 128 * 128), ki = desc_add(kd, i * kKT * 128);
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            umma_bf16(ts, desc_add(qi, kk * 32), desc_add(ki, kk * 32), id_s, (i | kk) != 0);
+                    }
                 }
-                for (int i = 0; i < n_tq; ++i) {
-                    const uint64_t ki = desc_add(kd, (n_sq + i) * kKT * 128);
-                    // K-steps past D (the zero-filled tail of the last chunk) are skipped
-                    const int kst = lh_chunk_id(rank, n_sq + i, lat_chunks, rope_first) == p.n_qchunks - 1 ? last_ksteps : 4;
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        if (kk < kst)
-                            umma_bf16_ts(ts, t_q + i * 32 + kk * 8, desc_add(ki, kk * 32), id_s, (n_sq + i) + kk != 0);
+                for (int i = 0; i < 2; ++i) {
+                    if (i < n_tq) {
+                        const uint64_t ki = desc_add(kd, (n_sq + i) * kKT * 128);
+                        const uint32_t acc0 = (n_sq + i) != 0 ? 1u : 0u;
+                        umma_bf16_ts(ts, t_q + i * 32, ki, id_s, acc0);
+#pragma unroll
+                        for (int kk = 1; kk < 4; ++kk)
+                            umma_bf16_ts(ts, t_q + i * 32 + kk * 8, desc_add(ki, kk * 32), id_s, 1u);
+                    }
                 }
                 umma_commit(&bs.s_full[it & 1]);
                 const bool last = (gt + 1 == gt1) || (j + 1 == starts[b + 1] - starts[b]);
