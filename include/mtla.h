@@ -45,6 +45,13 @@
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy
  *     default stream) and allocate nothing: scratch comes from `workspace`,
  *     whose size mtla_workspace_size() reports.
+ *   - Stream order: the first kernel of a bf16 decode step is launched as a
+ *     programmatic dependent of the kernel before it, so consecutive steps
+ *     overlap. It reads only the absorbed projection W_UK before that kernel
+ *     finishes. That holds for any kernel that does not trigger its
+ *     dependents early (ordinary kernels never do). A caller kernel that does
+ *     trigger early must write the step's inputs before it triggers. Those
+ *     inputs are the positions, latents, queries and gates.
  *   - Argument errors are found on the host before anything is launched and
  *     returned as a status; nothing is written then. Errors found on the
  *     device (a position beyond the cache, a bounded wait that ran out) skip

@@ -81,6 +81,14 @@ __device__ __forceinline__ int seq_slots(const DecTC& p, int b) {
 // rounded to bf16 into row h of sequence b's query image (64-column SW128
 // chunks of NH rows, zero beyond D). Block (b, H): gate, RoPE and in-place
 // update of the open slot (MTLA Method (1)), and zero rows H..NH-1 of the image.
+// Launched as a programmatic dependent of the previous kernel in the stream:
+// only the W_UK rows (weights, constant across steps) are read before the
+// wait for that kernel; every input of the step and every write come after it.
+// The attention kernel may start at once: it reads the positions and finished
+// slots before its own wait. Those are safe to read early because this kernel
+// starts before its predecessor ends only when that predecessor triggers its
+// dependents early, which the library's own kernels alone do (a step's combine
+// kernel, which writes neither); the C-ABI header states this for callers.
 __global__ void __launch_bounds__(kPrepAbsThreads + 32) k_dec_prep_tc(DecodeArgs a, uint8_t* qimg, int n_chunks, int NH) {
     pdl_launch_dependents();   // the attention kernel may start its prologue now
     const Shape& sh = a.sh;
@@ -88,6 +96,7 @@ __global__ void __launch_bounds__(kPrepAbsThreads + 32) k_dec_prep_tc(DecodeArgs
     const uint32_t img_bytes = (uint32_t)n_chunks * NH * 128;
     uint8_t* img = qimg + (size_t)b * img_bytes;
     if (h == sh.H) {
+        pdl_wait();
         decode_update_body<bf16>(a, b);
         for (int e = threadIdx.x; e < n_chunks * (NH - sh.H) * 8; e += blockDim.x) {
             const int c = e / ((NH - sh.H) * 8), rr = e % ((NH - sh.H) * 8);
@@ -96,8 +105,6 @@ __global__ void __launch_bounds__(kPrepAbsThreads + 32) k_dec_prep_tc(DecodeArgs
         }
         return;
     }
-    const int64_t t = a.pos[b];
-    const bool t_ok = t >= 0 && t < (int64_t)sh.max_slots * sh.s;
     __shared__ float part_sum[8][512];     // [i-group][latent column]
     const size_t rh = (size_t)b * sh.H + h;
     const bf16* qc = (const bf16*)a.q_c + rh * sh.d_h;
@@ -106,7 +113,9 @@ __global__ void __launch_bounds__(kPrepAbsThreads + 32) k_dec_prep_tc(DecodeArgs
     if (threadIdx.x >= kPrepAbsThreads) {
         // the last warp: RoPE part of q~ (columns d_c .. D-1) and the zero padding
         // up to the chunk boundary, independent of the W_UK product
-        if (!t_ok) return;
+        pdl_wait();
+        const int64_t t = a.pos[b];
+        if (t < 0 || t >= (int64_t)sh.max_slots * sh.s) return;
         for (int j = sh.d_c + (int)threadIdx.x - kPrepAbsThreads; j < dpad; j += 32) {
             float v = 0.f;
             if (j < sh.D) {
@@ -126,15 +135,32 @@ __global__ void __launch_bounds__(kPrepAbsThreads + 32) k_dec_prep_tc(DecodeArgs
     const int n_jg = sh.d_c / 8;
     const int n_ig = max(1, min(8, kPrepAbsThreads / n_jg));
     const int rows_per = (((sh.d_h + n_ig - 1) / n_ig) + 15) & ~15;   // 16-row batches, aligned
+    // this thread's first batch of W_UK rows is in flight before the wait
+    uint4 raw[16];
+    {
+        const int e = threadIdx.x;
+        if (e < n_ig * n_jg) {
+            const int ig = e / n_jg, jg = e % n_jg;
+            const int i0 = ig * rows_per, i1 = min(sh.d_h, i0 + rows_per);
+#pragma unroll
+            for (int u = 0; u < 16; ++u)
+                if (i0 + u < i1) raw[u] = *(const uint4*)(W + (size_t)(i0 + u) * sh.d_c + jg * 8);
+        }
+    }
+    pdl_wait();
+    const int64_t t = a.pos[b];
+    const bool t_ok = t >= 0 && t < (int64_t)sh.max_slots * sh.s;
     for (int e = threadIdx.x; e < n_ig * n_jg; e += kPrepAbsThreads) {
         const int ig = e / n_jg, jg = e % n_jg;
         const int i0 = ig * rows_per, i1 = min(sh.d_h, i0 + rows_per);
         float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         for (int ib = i0; ib < i1; ib += 16) {
-            uint4 raw[16], qraw[2];
+            uint4 qraw[2];
+            if (e != (int)threadIdx.x || ib != i0) {
 #pragma unroll
-            for (int u = 0; u < 16; ++u)
-                if (ib + u < i1) raw[u] = *(const uint4*)(W + (size_t)(ib + u) * sh.d_c + jg * 8);
+                for (int u = 0; u < 16; ++u)
+                    if (ib + u < i1) raw[u] = *(const uint4*)(W + (size_t)(ib + u) * sh.d_c + jg * 8);
+            }
 #pragma unroll
             for (int u = 0; u < 2; ++u)
                 if (ib + 8 * u < i1) qraw[u] = *(const uint4*)(qc + ib + 8 * u);   // d_h % 16 == 0
@@ -568,6 +594,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 // W_UV[h] is staged in shared memory before the wait for the attention kernel;
 // after it, every partial value this block needs is read in one round.
 __global__ void __launch_bounds__(256) k_dec_combine(DecodeArgs a, DecTC p) {
+    pdl_launch_dependents();   // the next step's prep may stage its W_UK rows now
     const int h = blockIdx.x, b = blockIdx.y;
     const Shape& sh = a.sh;
     if (seq_tiles(p, b) == 0) return;
@@ -855,8 +882,8 @@ cudaError_t tc_decode(const DecodeArgs& a, cudaStream_t st, uint64_t* launches) 
             carve[dev] = true;
         }
     }
-    k_dec_prep_tc<<<dim3(sh.B, sh.H + 1), kPrepAbsThreads + 32, 0, st>>>(a, qimg, p.n_chunks, NH);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(k_dec_prep_tc, dim3(sh.B, sh.H + 1), dim3(kPrepAbsThreads + 32), 0, st, a, qimg,
+                               p.n_chunks, NH);
     if (e != cudaSuccess) return note_error("k_dec_prep_tc launch", e);
     const size_t smem = attn_smem_bytes(sh, NH);
     profile_begin(st);
