@@ -58,6 +58,7 @@ constexpr int kDh = 64;         // head width d_h of this kernel
 struct PreTC {
     int B, T, H, d_h, d_c, d_r, D, s;
     int n_qtiles;     // ceil(T / 128)
+    int n_items;      // n_qtiles * B * H
     float scale_log2;
     double log2_rope_base;
     const bf16* q_r;  // [B, T, H, d_r]
@@ -68,11 +69,11 @@ struct PreTC {
 };
 
 struct Bars {
-    uint64_t full[kStages], empty[kStages];
-    uint64_t abs_full, abs_done, q_ready;
+    uint64_t full[kStages], empty[kStages];      // ring: key tiles and each item's W_UV
+    uint64_t abs_full, abs_done, q_ready, q_free;
     uint64_t s_full[2], s_empty[2];
     uint64_t p_full[2], o_done[2];
-    uint64_t wuv_full, olat_ready, out_done;
+    uint64_t olat_ready, out_done, tail_free;
     uint64_t drain[2];
     uint32_t tmem_base;
     volatile int fail;
@@ -136,13 +137,49 @@ __device__ __forceinline__ void ld_row32_bf16(const bf16* src, float* v) {
     }
 }
 
-// One CTA per (128 query positions, sequence, head), heaviest first. The own
-// partial slot of every row is handled on the CUDA cores (its score is one dot
-// product per row; its value enters the output at the end with the row's final
-// weight); the finished slots stream through the tensor cores in 128-slot
+// Work item idx (heaviest first): query tile qt = n_qtiles - 1 - idx / (B H),
+// then sequence and head.
+struct Item {
+    int b, h, p0, nft;    // nft: finished-slot tiles of 128 slots this query tile attends
+};
+__device__ __forceinline__ Item decode_item(const PreTC& p, int idx) {
+    const int per_qt = p.B * p.H;
+    const int qt = p.n_qtiles - 1 - idx / per_qt;
+    const int rem = idx % per_qt;
+    Item it;
+    it.b = rem / p.H;
+    it.h = rem % p.H;
+    it.p0 = qt * kQ;
+    const int last = min(it.p0 + kQ - 1, p.T - 1);
+    it.nft = (last / p.s + kKT - 1) / kKT;
+    return it;
+}
+// The j-th item of this CTA, or -1 past the end: round j of gridDim.x items,
+// walked forwards on even rounds and backwards on odd ones.
+__device__ __forceinline__ int item_at(const PreTC& p, int j) {
+    const int g = (int)gridDim.x, c = (int)blockIdx.x;
+    const int idx = j * g + ((j & 1) ? g - 1 - c : c);
+    return idx < p.n_items ? idx : -1;
+}
+
+// One work item = (128 query positions, sequence, head), heaviest first. The
+// own partial slot of every row is handled on the CUDA cores (its score is one
+// dot product per row; its value enters the output at the end with the row's
+// final weight); the finished slots stream through the tensor cores in 128-slot
 // tiles. DC = d_c (d_h = 64 and d_R = 32 are fixed): every MMA sequence is
 // unrolled at compile time (a runtime loop or branch between tcgen05.mma
 // instructions halves their issue rate).
+//
+// Persistent: CTA c takes items c, 2G-1-c, 2G+c, ... (a snake over rounds of G
+// = gridDim.x items, so the heavy and light items of each round spread evenly),
+// and the next item's set-up overlaps this one's end:
+//   - qC and W_UK of item j+1 load into the query region once the score MMAs
+//     of item j are done (q_free);
+//   - item j's W_UV loads into the ring as one more "tile" after its key tiles,
+//     so the ring's empty/full barriers order it with the tiles around it;
+//   - O_lat of item j goes to TMEM (bf16, the output MMA's A operand), so the
+//     absorption of item j+1 into the O columns starts as soon as O is read;
+//   - item j+1's key tiles load as soon as the P.V of item j frees the stages.
 template <int DC>
 __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constant__ Maps maps, const PreTC p) {
     extern __shared__ uint8_t smem_raw[];
@@ -152,26 +189,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
     constexpr uint32_t rope_k = kKT * 64;                                // its RoPE chunk (64-byte rows)
     constexpr uint32_t stage_bytes = NL * chunk_k + rope_k;
     constexpr uint32_t q_bytes = NL * kQ * 128 + kQ * 64;
+    constexpr int dc_chunks = DC / 64;
+    constexpr uint32_t wchunk = (uint32_t)kDh * 128;                     // one 64-column chunk of W
+    static_assert(kQ * 128 + dc_chunks * wchunk <= q_bytes, "qC and W_UK staging fits the query region");
+    static_assert(dc_chunks * wchunk <= stage_bytes, "W_UV fits a ring stage");
     uint8_t* ring = smem;                                                // kStages key tiles
     uint8_t* q_s = ring + kStages * stage_bytes;                         // the query image, same layout
-    // staging in ring stages the key tiles do not use at the time: qC and W_UK
-    // (stage 1, before key tile 1), W_UV (stage 1, after the last P.V of a tile
-    // in stage 1), O_lat (stage 0, after the last P.V)
-    uint8_t* qc_s = ring + stage_bytes;
-    uint8_t* wk_s = ring + stage_bytes + kQ * 128;
-    uint8_t* wv_s = ring + stage_bytes;
+    // qC and W_UK of the next item are staged in the query region (free once the
+    // score MMAs of the current item are done)
+    uint8_t* qc_s = q_s;
+    uint8_t* wk_s = q_s + kQ * 128;
     Bars& bs = *(Bars*)(q_s + q_bytes);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int per_qt = p.B * p.H;
-    const int qt = p.n_qtiles - 1 - (int)(blockIdx.x / per_qt);
-    const int rem = (int)(blockIdx.x % per_qt);
-    const int b = rem / p.H, h = rem % p.H;
-    const int p0 = qt * kQ;
-    const int last = min(p0 + kQ - 1, p.T - 1);
-    const int nft = (last / p.s + kKT - 1) / kKT;                        // finished-slot tiles
-    constexpr int dc_chunks = DC / 64;
-    constexpr uint32_t wchunk = (uint32_t)kDh * 128;                     // one 64-column chunk of W
 
     if (tid == 0) {
         for (int i = 0; i < kStages; ++i) {
@@ -181,6 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
         mbar_init(&bs.abs_full, 1);
         mbar_init(&bs.abs_done, 1);
         mbar_init(&bs.q_ready, 8);
+        mbar_init(&bs.q_free, 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bs.s_full[i], 1);
             mbar_init(&bs.s_empty[i], 1);    // P.V of the tile two back is done (P lives in S)
@@ -188,9 +219,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
             mbar_init(&bs.o_done[i], 1);
             mbar_init(&bs.drain[i], 1);
         }
-        mbar_init(&bs.wuv_full, 1);
         mbar_init(&bs.olat_ready, 8);
         mbar_init(&bs.out_done, 1);
+        mbar_init(&bs.tail_free, 8);
         bs.fail = 0;
         fence_mbar_init();
     }
@@ -202,9 +233,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bs.tmem_base;
-    const uint32_t t_s0 = tmem;            // S buffers: columns [0, 128) and [128, 256); later the output
+    const uint32_t t_s0 = tmem;            // S buffers: columns [0, 128) and [128, 256)
     const uint32_t t_o = tmem + 256;       // q~ (absorption), then O: columns [256, 256 + d_c)
-    // P (bf16 pairs) of tile k overwrites the first 64 columns of S buffer k & 1
+    // P (bf16 pairs) of a tile overwrites the first 64 columns of its S buffer;
+    // at an item's end O_lat (bf16 pairs) takes columns [0, d_c / 2) and the
+    // output columns [128, 128 + d_h)
+    const uint32_t t_olat = tmem, t_out = tmem + 128;
+
+    // every role walks the same items and counts ring positions R (key tiles
+    // plus one W_UV position per item) and key tiles G (S buffers) alike
+    int loads_R = 0, loads_q = 0;          // the producer's copies, for the drain on failure
 
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
@@ -212,28 +250,51 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
             tma_prefetch_desc(&maps.qc);
             tma_prefetch_desc(&maps.slots);
             tma_prefetch_desc(&maps.slots_r);
-            mbar_arrive_expect_tx(&bs.abs_full, kQ * 128 + dc_chunks * wchunk);
-            tma_load_4d(qc_s, &maps.qc, &bs.abs_full, 0, h, p0, b);
-            for (int n = 0; n < dc_chunks; ++n) tma_load_3d(wk_s + n * wchunk, &maps.wuk, &bs.abs_full, n * 64, 0, h);
-            for (int k = 0; k < nft; ++k) {
-                const int st = k & 1;
-                if (k >= kStages && !waitb(&bs.empty[st], ((k >> 1) - 1) & 1, bs)) break;
-                if (k == 1 && !waitb(&bs.abs_done, 0, bs)) break;    // qC and W_UK have been read
-                mbar_arrive_expect_tx(&bs.full[st], stage_bytes);
-                uint8_t* dst = ring + st * stage_bytes;
-#pragma unroll
-                for (int c = 0; c < NL; ++c)
-                    tma_load_3d(dst + c * chunk_k, &maps.slots, &bs.full[st], c * 64, kKT * k, b);
-                tma_load_3d(dst + NL * chunk_k, &maps.slots_r, &bs.full[st], DC, kKT * k, b);
-            }
-            // W_UV into stage 1 as soon as nothing reads it: after the absorption (qC)
-            // and the P.V of the last tile in stage 1. This thread waited the previous
-            // phase of empty[1] when it loaded that tile, so the parity wait is exact.
-            const int t1 = nft >= 2 ? ((nft - 1) & 1 ? nft - 1 : nft - 2) : -1;   // last tile in stage 1
-            if (waitb(&bs.abs_done, 0, bs) && (t1 < 0 || waitb(&bs.empty[1], (t1 >> 1) & 1, bs))) {
-                mbar_arrive_expect_tx(&bs.wuv_full, dc_chunks * wchunk);
+            auto load_qw = [&](const Item& it) {
+                mbar_arrive_expect_tx(&bs.abs_full, kQ * 128 + dc_chunks * wchunk);
+                tma_load_4d(qc_s, &maps.qc, &bs.abs_full, 0, it.h, it.p0, it.b);
                 for (int n = 0; n < dc_chunks; ++n)
-                    tma_load_3d(wv_s + n * wchunk, &maps.wuv, &bs.wuv_full, n * 64, 0, h);
+                    tma_load_3d(wk_s + n * wchunk, &maps.wuk, &bs.abs_full, n * 64, 0, it.h);
+                ++loads_q;
+            };
+            // ring position `pos` is free once the consumer of position pos - 2 released it
+            auto ring_free = [&](int pos) {
+                return pos < kStages || waitb(&bs.empty[pos & 1], ((pos >> 1) - 1) & 1, bs);
+            };
+            int R = 0;
+            int idx = item_at(p, 0);
+            if (idx >= 0) load_qw(decode_item(p, idx));
+            for (int j = 0; idx >= 0 && !bs.fail; ++j) {
+                const Item it = decode_item(p, idx);
+                const int nidx = item_at(p, j + 1);
+                bool ok = true;
+                for (int k = 0; k < it.nft && ok; ++k) {
+                    const int pos = R++;
+                    if (!(ok = ring_free(pos))) break;
+                    uint8_t* dst = ring + (pos & 1) * stage_bytes;
+                    mbar_arrive_expect_tx(&bs.full[pos & 1], stage_bytes);
+#pragma unroll
+                    for (int c = 0; c < NL; ++c)
+                        tma_load_3d(dst + c * chunk_k, &maps.slots, &bs.full[pos & 1], c * 64, kKT * k, it.b);
+                    tma_load_3d(dst + NL * chunk_k, &maps.slots_r, &bs.full[pos & 1], DC, kKT * k, it.b);
+                    loads_R = R;
+                }
+                if (!ok) break;
+                // the next item's qC and W_UK into the query region once this item's
+                // score MMAs have read it
+                if (nidx >= 0) {
+                    if (!waitb(&bs.q_free, j & 1, bs)) break;
+                    load_qw(decode_item(p, nidx));
+                }
+                // this item's W_UV as one more ring position
+                const int pos = R++;
+                if (!ring_free(pos)) break;
+                mbar_arrive_expect_tx(&bs.full[pos & 1], dc_chunks * wchunk);
+                for (int n = 0; n < dc_chunks; ++n)
+                    tma_load_3d(ring + (pos & 1) * stage_bytes + n * wchunk, &maps.wuv, &bs.full[pos & 1], n * 64, 0,
+                                it.h);
+                loads_R = R;
+                idx = nidx;
             }
         }
     } else if (warp == 1) {
@@ -245,51 +306,63 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
             const uint32_t ring_a = smem_u32(ring), q_a = smem_u32(q_s);
             const uint64_t q_d = sdesc_sw128(q_a, 16, 1024), q_r = sdesc_sw64(q_a + NL * kQ * 128);
             const uint64_t qc_d = sdesc_sw128(smem_u32(qc_s), 16, 1024);
-            bool ok = waitb(&bs.abs_full, 0, bs);
-            if (ok) {
+            const uint64_t wd = sdesc_sw128(smem_u32(wk_s), wchunk, 1024);
+            int R = 0, G = 0, wpos = -1;     // wpos: ring position of the previous item's W_UV
+            for (int j = 0; !bs.fail; ++j) {
+                const int idx = item_at(p, j);
+                if (j > 0) {
+                    // out = O_lat . W_UV[h]^T of the previous item: A = O_lat [128 x d_c]
+                    // (bf16 pairs in TMEM), B = W_UV[h] [d_h x d_c] K-major (ring)
+                    if (!waitb(&bs.olat_ready, (j - 1) & 1, bs)) break;
+                    if (!waitb(&bs.full[wpos & 1], (wpos >> 1) & 1, bs)) break;
+                    tc_fence_after();
+                    const uint64_t wv_d = sdesc_sw128(ring_a + (wpos & 1) * stage_bytes, 16, 1024);
+#pragma unroll
+                    for (int kk = 0; kk < DC / 16; ++kk)
+                        umma_bf16_ts(t_out, t_olat + kk * 8, desc_add(wv_d, (kk >> 2) * wchunk + (kk & 3) * 32),
+                                     id_out, kk > 0);
+                    umma_commit(&bs.out_done);
+                    umma_commit(&bs.empty[wpos & 1]);   // the W_UV position of the ring is free
+                }
+                if (idx < 0) break;
+                const Item it = decode_item(p, idx);
+                // q~ = qC . W_UK[h]: A = qC [128 x d_h] K-major, B = W_UK[h] [d_h x d_c]
+                // MN-major; into the O columns, free since the previous item's O was read
+                if (!waitb(&bs.abs_full, j & 1, bs)) break;
                 tc_fence_after();
-                // q~ = qC . W_UK[h]: A = qC [128 x d_h] K-major, B = W_UK[h] [d_h x d_c] MN-major
-                const uint64_t wd = sdesc_sw128(smem_u32(wk_s), wchunk, 1024);
 #pragma unroll
                 for (int kk = 0; kk < kDh / 16; ++kk)
                     umma_bf16(t_o, desc_add(qc_d, kk * 32), desc_add(wd, kk * 2048), id_abs, kk > 0);
                 umma_commit(&bs.abs_done);
-                ok = waitb(&bs.q_ready, 0, bs);
-            }
-            for (int k = 0; ok && k < nft; ++k) {
-                const int st = k & 1;
-                if (!waitb(&bs.full[st], (k >> 1) & 1, bs)) break;
-                if (k >= 2 && !waitb(&bs.s_empty[k & 1], ((k >> 1) - 1) & 1, bs)) break;
-                tc_fence_after();
-                // S = q~ . K^T (M = 128 queries, N = 128 slots, K = D): the latent
-                // chunks, then the two K-steps of the RoPE chunk
-                const uint32_t stage_a = ring_a + st * stage_bytes;
-                const uint64_t kd = sdesc_sw128(stage_a, 16, 1024), kr = sdesc_sw64(stage_a + NL * chunk_k);
-                const uint32_t ts = t_s0 + (k & 1) * kKT;
+                if (!waitb(&bs.q_ready, j & 1, bs)) break;
+                // the S columns held the previous item's O_lat and output until read
+                if (j > 0 && !waitb(&bs.tail_free, (j - 1) & 1, bs)) break;
+                bool ok = true;
+                for (int k = 0; k < it.nft; ++k, ++G) {
+                    const int pos = R++;
+                    if (!(ok = waitb(&bs.full[pos & 1], (pos >> 1) & 1, bs))) break;
+                    if (G >= 2 && !(ok = waitb(&bs.s_empty[G & 1], ((G >> 1) - 1) & 1, bs))) break;
+                    tc_fence_after();
+                    // S = q~ . K^T (M = 128 queries, N = 128 slots, K = D): the latent
+                    // chunks, then the two K-steps of the RoPE chunk
+                    const uint32_t stage_a = ring_a + (pos & 1) * stage_bytes;
+                    const uint64_t kd = sdesc_sw128(stage_a, 16, 1024), kr = sdesc_sw64(stage_a + NL * chunk_k);
+                    const uint32_t ts = t_s0 + (G & 1) * kKT;
 #pragma unroll
-                for (int c = 0; c < NL; ++c) {
-                    const uint64_t qc = desc_add(q_d, c * kQ * 128), kc = desc_add(kd, c * chunk_k);
+                    for (int c = 0; c < NL; ++c) {
+                        const uint64_t qc = desc_add(q_d, c * kQ * 128), kc = desc_add(kd, c * chunk_k);
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        umma_bf16(ts, desc_add(qc, kk * 32), desc_add(kc, kk * 32), id_s, (c | kk) != 0);
+                        for (int kk = 0; kk < 4; ++kk)
+                            umma_bf16(ts, desc_add(qc, kk * 32), desc_add(kc, kk * 32), id_s, (c | kk) != 0);
+                    }
+#pragma unroll
+                    for (int kk = 0; kk < kDr / 16; ++kk)
+                        umma_bf16(ts, desc_add(q_r, kk * 32), desc_add(kr, kk * 32), id_s, 1u);
+                    umma_commit(&bs.s_full[G & 1]);
                 }
-#pragma unroll
-                for (int kk = 0; kk < kDr / 16; ++kk)
-                    umma_bf16(ts, desc_add(q_r, kk * 32), desc_add(kr, kk * 32), id_s, 1u);
-                umma_commit(&bs.s_full[k & 1]);
-            }
-            if (!bs.fail && waitb(&bs.olat_ready, 0, bs) && waitb(&bs.wuv_full, 0, bs)) {
-                tc_fence_after();
-                // out = O_lat . W_UV[h]^T: A = O_lat [128 x d_c] K-major (ring stage 0),
-                // B = W_UV[h] [d_h x d_c] K-major (ring stage 1)
-                const uint64_t od = sdesc_sw128(ring_a, 16, 1024), wv_d = sdesc_sw128(smem_u32(wv_s), 16, 1024);
-#pragma unroll
-                for (int kk = 0; kk < DC / 16; ++kk) {
-                    const int c = kk >> 2;
-                    umma_bf16(t_s0, desc_add(od, c * kQ * 128 + (kk & 3) * 32),
-                              desc_add(wv_d, c * wchunk + (kk & 3) * 32), id_out, kk > 0);
-                }
-                umma_commit(&bs.out_done);
+                if (!ok) break;
+                umma_commit(&bs.q_free);             // the query region may take the next item's qC
+                wpos = R++;
             }
         }
     } else if (warp == 10) {
@@ -298,18 +371,27 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
         if (lane == 0) {
             const uint32_t id_o = idesc_bf16_f32(128, DC, false, true);
             const uint32_t ring_a = smem_u32(ring);
-            for (int k = 0; k < nft; ++k) {
-                if (!waitb(&bs.p_full[k & 1], (k >> 1) & 1, bs)) break;
-                tc_fence_after();
-                // O += P . V: A = P [128 x 128] in TMEM, B = V = key tile latent [128 x d_c] MN-major
-                const uint64_t vd = sdesc_sw128(ring_a + (k & 1) * stage_bytes, chunk_k, 1024);
+            int R = 0, G = 0;
+            bool ok = true;
+            for (int j = 0; ok; ++j) {
+                const int idx = item_at(p, j);
+                if (idx < 0) break;
+                const Item it = decode_item(p, idx);
+                for (int k = 0; k < it.nft; ++k, ++G) {
+                    const int pos = R++;
+                    if (!(ok = waitb(&bs.p_full[G & 1], (G >> 1) & 1, bs))) break;
+                    tc_fence_after();
+                    // O += P . V: A = P [128 x 128] in TMEM, B = V = key tile latent [128 x d_c] MN-major
+                    const uint64_t vd = sdesc_sw128(ring_a + (pos & 1) * stage_bytes, chunk_k, 1024);
 #pragma unroll
-                for (int kk = 0; kk < kKT / 16; ++kk)
-                    umma_bf16_ts(t_o, t_s0 + (k & 1) * kKT + kk * 8, desc_add(vd, kk * 2048), id_o,
-                                 (k > 0 || kk > 0) ? 1u : 0u);
-                umma_commit(&bs.empty[k & 1]);
-                umma_commit(&bs.o_done[k & 1]);
-                umma_commit(&bs.s_empty[k & 1]);   // S buffer k & 1 (which held P) is free
+                    for (int kk = 0; kk < kKT / 16; ++kk)
+                        umma_bf16_ts(t_o, t_s0 + (G & 1) * kKT + kk * 8, desc_add(vd, kk * 2048), id_o,
+                                     (k > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit(&bs.empty[pos & 1]);
+                    umma_commit(&bs.o_done[G & 1]);
+                    umma_commit(&bs.s_empty[G & 1]);   // S buffer G & 1 (which held P) is free
+                }
+                ++R;                                   // the item's W_UV position
             }
         }
     } else {
@@ -321,170 +403,176 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;
         const int hc = (warp - 2) >> 2;
-        const int pos = p0 + r;
-        const bool row_ok = pos < p.T;
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-        const bf16* prow = p.P + ((size_t)b * p.T + min(pos, p.T - 1)) * p.D;   // own partial slot
-        float v[32], pv[32];
+        constexpr int half = DC / 2;
+        float v[32];
         uint32_t w[32];
-        // q~ row block of 32 columns into the query image: latent columns into the
-        // 128-byte-swizzled chunks, the RoPE block into the 64-byte-swizzled one
-        auto put_q = [&](int col) {
-            if (col < DC) st_row32_bf16(q_s, kQ * 128, r, col, v);
-            else st_row32_bf16_sw64(q_s + NL * kQ * 128, r, v);
-        };
-        float e_own = 0.f;
-        // q~ row in 32-column blocks, the first half of the blocks for hc = 0 and
-        // the rest for hc = 1 (which therefore holds the RoPE block): latent blocks
-        // from TMEM, the RoPE block rotated with the scan's (cos, sin) table; all
-        // rounded to bf16 into the query image. The own-slot score q~ . P_pos uses
-        // the same rounded values. Every global load of a block is issued before
-        // the wait for the absorption.
-        constexpr int n_blk = NL * 2 + 1, nb0 = (n_blk + 1) / 2;
-        const int blk0 = hc == 0 ? 0 : nb0, blk1 = hc == 0 ? nb0 : n_blk;   // <= 5 blocks each
-        const bf16* qr = p.q_r + (((size_t)b * p.T + min(pos, p.T - 1)) * p.H + h) * p.d_r;
-        const float2* cs_row = p.rope_tab + (size_t)min(pos, p.T - 1) * (p.d_r / 2);
-        uint4 pv4[5][4];
+        int G = 0;
+        for (int j = 0;; ++j) {
+            const int idx = item_at(p, j);
+            if (idx < 0) break;
+            const Item it = decode_item(p, idx);
+            const int b = it.b, h = it.h, p0 = it.p0, nft = it.nft;
+            const int pos = p0 + r;
+            const bool row_ok = pos < p.T;
+            const bf16* prow = p.P + ((size_t)b * p.T + min(pos, p.T - 1)) * p.D;   // own partial slot
+            // q~ row block of 32 columns into the query image: latent columns into the
+            // 128-byte-swizzled chunks, the RoPE block into the 64-byte-swizzled one
+            auto put_q = [&](int col) {
+                if (col < DC) st_row32_bf16(q_s, kQ * 128, r, col, v);
+                else st_row32_bf16_sw64(q_s + NL * kQ * 128, r, v);
+            };
+            float e_own = 0.f;
+            // q~ row in 32-column blocks, the first half of the blocks for hc = 0 and
+            // the rest for hc = 1 (which therefore holds the RoPE block): latent blocks
+            // from TMEM, the RoPE block rotated with the scan's (cos, sin) table; all
+            // rounded to bf16 into the query image. The own-slot score q~ . P_pos uses
+            // the same rounded values. Every global load of a block is issued before
+            // the wait for the absorption.
+            constexpr int n_blk = NL * 2 + 1, nb0 = (n_blk + 1) / 2;
+            const int blk0 = hc == 0 ? 0 : nb0, blk1 = hc == 0 ? nb0 : n_blk;   // <= 5 blocks each
+            const bf16* qr = p.q_r + (((size_t)b * p.T + min(pos, p.T - 1)) * p.H + h) * p.d_r;
+            const float2* cs_row = p.rope_tab + (size_t)min(pos, p.T - 1) * (p.d_r / 2);
+            uint4 pv4[5][4];
 #pragma unroll
-        for (int q = 0; q < 5; ++q) {
-            const int c0 = (blk0 + q) * 32;
+            for (int q = 0; q < 5; ++q) {
+                const int c0 = (blk0 + q) * 32;
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                pv4[q][u] = make_uint4(0, 0, 0, 0);
-                if (blk0 + q < blk1 && c0 + 8 * u < p.D) pv4[q][u] = *(const uint4*)(prow + c0 + 8 * u);
+                for (int u = 0; u < 4; ++u) {
+                    pv4[q][u] = make_uint4(0, 0, 0, 0);
+                    if (blk0 + q < blk1 && c0 + 8 * u < p.D) pv4[q][u] = *(const uint4*)(prow + c0 + 8 * u);
+                }
             }
-        }
-        waitb(&bs.abs_done, 0, bs);
-        tc_fence_after();
+            waitb(&bs.abs_done, j & 1, bs);
+            tc_fence_after();
 #pragma unroll
-        for (int q = 0; q < 5; ++q) {
-            const int c0 = (blk0 + q) * 32;
-            if (blk0 + q < blk1) {
-                if (c0 < DC) {
-                    tmem_ld32(t_o + c0 + lane_off, v);
-                    tmem_wait_ld();
+            for (int q = 0; q < 5; ++q) {
+                const int c0 = (blk0 + q) * 32;
+                if (blk0 + q < blk1) {
+                    if (c0 < DC) {
+                        tmem_ld32(t_o + c0 + lane_off, v);
+                        tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) v[i] = __bfloat162float(__float2bfloat16_rn(v[i]));
-                } else {
-                    // RoPE columns (zero past d_r): qR and the (cos, sin) pairs as vectors
-                    const int e0 = c0 - DC;
-                    uint4 qv[4];
-                    float4 cs4[8];
+                        for (int i = 0; i < 32; ++i) v[i] = __bfloat162float(__float2bfloat16_rn(v[i]));
+                    } else {
+                        // RoPE columns (zero past d_r): qR and the (cos, sin) pairs as vectors
+                        const int e0 = c0 - DC;
+                        uint4 qv[4];
+                        float4 cs4[8];
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        qv[u] = make_uint4(0, 0, 0, 0);
-                        if (e0 + 8 * u < p.d_r) qv[u] = *(const uint4*)(qr + e0 + 8 * u);
-                    }
+                        for (int u = 0; u < 4; ++u) {
+                            qv[u] = make_uint4(0, 0, 0, 0);
+                            if (e0 + 8 * u < p.d_r) qv[u] = *(const uint4*)(qr + e0 + 8 * u);
+                        }
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        cs4[u] = make_float4(1.f, 0.f, 1.f, 0.f);
-                        if (e0 + 4 * u < p.d_r) cs4[u] = *(const float4*)(cs_row + e0 / 2 + 2 * u);
-                    }
-                    const bf16* qe = (const bf16*)qv;
-                    const float* csv = (const float*)cs4;      // cos, sin of pair i / 2
+                        for (int u = 0; u < 8; ++u) {
+                            cs4[u] = make_float4(1.f, 0.f, 1.f, 0.f);
+                            if (e0 + 4 * u < p.d_r) cs4[u] = *(const float4*)(cs_row + e0 / 2 + 2 * u);
+                        }
+                        const bf16* qe = (const bf16*)qv;
+                        const float* csv = (const float*)cs4;      // cos, sin of pair i / 2
 #pragma unroll
-                    for (int i = 0; i < 32; i += 2) {
-                        v[i] = v[i + 1] = 0.f;
-                        if (row_ok && e0 + i < p.d_r) {
-                            const float cs = csv[i], sn = csv[i + 1];
-                            const float x0 = __bfloat162float(qe[i]), x1 = __bfloat162float(qe[i + 1]);
-                            v[i] = __bfloat162float(__float2bfloat16_rn(x0 * cs - x1 * sn));
-                            v[i + 1] = __bfloat162float(__float2bfloat16_rn(x0 * sn + x1 * cs));
+                        for (int i = 0; i < 32; i += 2) {
+                            v[i] = v[i + 1] = 0.f;
+                            if (row_ok && e0 + i < p.d_r) {
+                                const float cs = csv[i], sn = csv[i + 1];
+                                const float x0 = __bfloat162float(qe[i]), x1 = __bfloat162float(qe[i + 1]);
+                                v[i] = __bfloat162float(__float2bfloat16_rn(x0 * cs - x1 * sn));
+                                v[i + 1] = __bfloat162float(__float2bfloat16_rn(x0 * sn + x1 * cs));
+                            }
                         }
                     }
-                }
-                put_q(c0);
-                const bf16* pe = (const bf16*)pv4[q];
+                    put_q(c0);
+                    const bf16* pe = (const bf16*)pv4[q];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) e_own = fmaf(v[i], __bfloat162float(pe[i]), e_own);
+                    for (int i = 0; i < 32; ++i) e_own = fmaf(v[i], __bfloat162float(pe[i]), e_own);
+                }
             }
-        }
-        fence_proxy_async();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bs.q_ready);
-        bs.xs[hc][r] = e_own;
-        named_sync(1, 256);
-        const float es = row_ok ? (bs.xs[0][r] + bs.xs[1][r]) * p.scale_log2 : 0.f;
-        named_sync(1, 256);                           // xs is free again
-        // online softmax over the finished-slot tiles; the own slot is the
-        // starting point (reference maximum es, weight 1 in the row sum)
-        float m_ref = es, l = hc == 0 ? 1.f : 0.f;    // l: this thread's half of the row sum
-        const int fin_lim = pos / p.s;                // finished slots this row may see
-        const int min_fin = p0 / p.s;                 // ... and the first row of the tile
-        for (int k = 0; k < nft; ++k) {
-            waitb(&bs.s_full[k & 1], (k >> 1) & 1, bs);
-            tc_fence_after();
-            float sv[64];
-            tmem_ld32(t_s0 + (k & 1) * kKT + hc * 64 + lane_off, sv);
-            tmem_ld32(t_s0 + (k & 1) * kKT + hc * 64 + 32 + lane_off, sv + 32);
-            tmem_wait_ld();
+            fence_proxy_async();
             tc_fence_before();
             __syncwarp();
-            // raw scores: the scale is folded into the exponent below. The slot mask
-            // only matters on tiles that reach past the first row's limit (a test
-            // uniform across the CTA). Maxima and sums in four independent chains.
-            const int j0 = kKT * k + 64 * hc;
-            if (kKT * (k + 1) > min_fin) {
-#pragma unroll
-                for (int c = 0; c < 64; ++c)
-                    if (j0 + c >= fin_lim) sv[c] = -INFINITY;
-            }
-            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-            for (int c = 0; c < 64; ++c) m4[c & 3] = fmaxf(m4[c & 3], sv[c]);
-            float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * p.scale_log2;
-            bs.red[k & 1][hc][r] = mt;
+            if (lane == 0) mbar_arrive(&bs.q_ready);
+            bs.xs[hc][r] = e_own;
             named_sync(1, 256);
-            tc_fence_after();                         // the other half's TMEM reads are done
-            mt = fmaxf(mt, bs.red[k & 1][hc ^ 1][r]);
-            // lazy rescale: the reference maximum moves only when the tile's maximum
-            // exceeds it by more than 2^8 (P stays <= 256); both halves decide alike
-            const bool upd = mt > m_ref + kRescaleLog2;
-            const float nm = upd ? mt : m_ref;
-            const float fac = ex2_approx(m_ref - nm);
-            float rs4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                const float q0 = ex2_approx(fmaf(sv[2 * c], p.scale_log2, -nm));
-                const float q1 = ex2_approx(fmaf(sv[2 * c + 1], p.scale_log2, -nm));
-                rs4[c & 3] += q0 + q1;
-                w[c] = pack_bf16x2(q0, q1);
-            }
-            l = fmaf(l, fac, (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
-            const bool need = upd && k > 0;           // O holds tiles 0..k-1
-            if (__any_sync(0xffffffffu, need)) {
-                waitb(&bs.o_done[(k - 1) & 1], ((k - 1) >> 1) & 1, bs);
+            const float es = row_ok ? (bs.xs[0][r] + bs.xs[1][r]) * p.scale_log2 : 0.f;
+            named_sync(1, 256);                           // xs is free again
+            // online softmax over the finished-slot tiles; the own slot is the
+            // starting point (reference maximum es, weight 1 in the row sum)
+            float m_ref = es, l = hc == 0 ? 1.f : 0.f;    // l: this thread's half of the row sum
+            const int fin_lim = pos / p.s;                // finished slots this row may see
+            const int min_fin = p0 / p.s;                 // ... and the first row of the tile
+            for (int k = 0; k < nft; ++k, ++G) {
+                waitb(&bs.s_full[G & 1], (G >> 1) & 1, bs);
                 tc_fence_after();
-                const float f = need ? fac : 1.f;
-                constexpr int half = DC / 2;
-                for (int cc = hc * half; cc < (hc + 1) * half; cc += 32) {
-                    tmem_ld32(t_o + cc + lane_off, v);
-                    tmem_wait_ld();
+                float sv[64];
+                tmem_ld32(t_s0 + (G & 1) * kKT + hc * 64 + lane_off, sv);
+                tmem_ld32(t_s0 + (G & 1) * kKT + hc * 64 + 32 + lane_off, sv + 32);
+                tmem_wait_ld();
+                tc_fence_before();
+                __syncwarp();
+                // raw scores: the scale is folded into the exponent below. The slot mask
+                // only matters on tiles that reach past the first row's limit (a test
+                // uniform across the CTA). Maxima and sums in four independent chains.
+                const int j0 = kKT * k + 64 * hc;
+                if (kKT * (k + 1) > min_fin) {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) v[i] *= f;
-                    tmem_st32(t_o + cc + lane_off, v);
+                    for (int c = 0; c < 64; ++c)
+                        if (j0 + c >= fin_lim) sv[c] = -INFINITY;
                 }
+                float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                for (int c = 0; c < 64; ++c) m4[c & 3] = fmaxf(m4[c & 3], sv[c]);
+                float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * p.scale_log2;
+                bs.red[G & 1][hc][r] = mt;
+                named_sync(1, 256);
+                tc_fence_after();                         // the other half's TMEM reads are done
+                mt = fmaxf(mt, bs.red[G & 1][hc ^ 1][r]);
+                // lazy rescale: the reference maximum moves only when the tile's maximum
+                // exceeds it by more than 2^8 (P stays <= 256); both halves decide alike
+                const bool upd = mt > m_ref + kRescaleLog2;
+                const float nm = upd ? mt : m_ref;
+                const float fac = ex2_approx(m_ref - nm);
+                float rs4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    const float q0 = ex2_approx(fmaf(sv[2 * c], p.scale_log2, -nm));
+                    const float q1 = ex2_approx(fmaf(sv[2 * c + 1], p.scale_log2, -nm));
+                    rs4[c & 3] += q0 + q1;
+                    w[c] = pack_bf16x2(q0, q1);
+                }
+                l = fmaf(l, fac, (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
+                const bool need = upd && k > 0;           // O holds this item's tiles 0..k-1
+                if (__any_sync(0xffffffffu, need)) {
+                    waitb(&bs.o_done[(G - 1) & 1], ((G - 1) >> 1) & 1, bs);
+                    tc_fence_after();
+                    const float f = need ? fac : 1.f;
+                    for (int cc = hc * half; cc < (hc + 1) * half; cc += 32) {
+                        tmem_ld32(t_o + cc + lane_off, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) v[i] *= f;
+                        tmem_st32(t_o + cc + lane_off, v);
+                    }
+                    tmem_wait_st();
+                }
+                // P over the first 64 columns of this tile's S buffer (both halves have
+                // read their scores: the barrier above)
+                tmem_st32_u(t_s0 + (G & 1) * kKT + hc * 32 + lane_off, w);
                 tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bs.p_full[G & 1]);
+                m_ref = nm;
             }
-            // P over the first 64 columns of this tile's S buffer (both halves have
-            // read their scores: the barrier above)
-            tmem_st32_u(t_s0 + (k & 1) * kKT + hc * 32 + lane_off, w);
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bs.p_full[k & 1]);
-            m_ref = nm;
-        }
-        // epilogue: O_lat = (O + w_own P_pos[:d_c]) / l -> bf16 K-major (ring stage 0), then out
-        if (nft > 0) waitb(&bs.o_done[(nft - 1) & 1], ((nft - 1) >> 1) & 1, bs);
-        tc_fence_after();
-        bs.xs[hc][r] = l;
-        named_sync(1, 256);
-        const float inv = 1.f / (bs.xs[0][r] + bs.xs[1][r]);
-        const float w_own = ex2_approx(es - m_ref);
-        {
-            constexpr int half = DC / 2;
+            // epilogue: O_lat = (O + w_own P_pos[:d_c]) / l as bf16 pairs into the S
+            // columns (the output MMA's A operand), then out = O_lat . W_UV^T
+            if (nft > 0) waitb(&bs.o_done[(G - 1) & 1], ((G - 1) >> 1) & 1, bs);
+            tc_fence_after();
+            bs.xs[hc][r] = l;
+            named_sync(1, 256);
+            const float inv = 1.f / (bs.xs[0][r] + bs.xs[1][r]);
+            const float w_own = ex2_approx(es - m_ref);
+            named_sync(1, 256);                           // xs is free again
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const int cc = hc * half + 32 * q;
@@ -496,34 +584,40 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
 #pragma unroll
                         for (int i = 0; i < 32; ++i) v[i] = 0.f;
                     }
+                    float pv[32];
                     ld_row32_bf16(prow + cc, pv);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) v[i] = fmaf(w_own, pv[i], v[i]) * inv;
-                    st_row32_bf16(ring, kQ * 128, r, cc, v);
+                    for (int i = 0; i < 16; ++i)
+                        w[i] = pack_bf16x2(fmaf(w_own, pv[2 * i], v[2 * i]) * inv,
+                                           fmaf(w_own, pv[2 * i + 1], v[2 * i + 1]) * inv);
+                    tmem_st16_u(t_olat + cc / 2 + lane_off, w);
                 }
             }
-        }
-        fence_proxy_async();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bs.olat_ready);
-        waitb(&bs.out_done, 0, bs);
-        tc_fence_after();
-        for (int cc = hc * (kDh / 2); cc < (hc + 1) * (kDh / 2); cc += 32) {
-            tmem_ld32(t_s0 + cc + lane_off, v);
-            tmem_wait_ld();
-            if (row_ok) {
-                bf16* o = p.out + (((size_t)b * p.T + pos) * p.H + h) * kDh + cc;
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bs.olat_ready);   // also: O has been read
+            waitb(&bs.out_done, j & 1, bs);
+            tc_fence_after();
+            for (int cc = hc * (kDh / 2); cc < (hc + 1) * (kDh / 2); cc += 32) {
+                tmem_ld32(t_out + cc + lane_off, v);
+                tmem_wait_ld();
+                if (row_ok) {
+                    bf16* o = p.out + (((size_t)b * p.T + pos) * p.H + h) * kDh + cc;
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    uint4 pk;
-                    pk.x = pack_bf16x2(v[8 * u + 0], v[8 * u + 1]);
-                    pk.y = pack_bf16x2(v[8 * u + 2], v[8 * u + 3]);
-                    pk.z = pack_bf16x2(v[8 * u + 4], v[8 * u + 5]);
-                    pk.w = pack_bf16x2(v[8 * u + 6], v[8 * u + 7]);
-                    *(uint4*)(o + 8 * u) = pk;
+                    for (int u = 0; u < 4; ++u) {
+                        uint4 pk;
+                        pk.x = pack_bf16x2(v[8 * u + 0], v[8 * u + 1]);
+                        pk.y = pack_bf16x2(v[8 * u + 2], v[8 * u + 3]);
+                        pk.z = pack_bf16x2(v[8 * u + 4], v[8 * u + 5]);
+                        pk.w = pack_bf16x2(v[8 * u + 6], v[8 * u + 7]);
+                        *(uint4*)(o + 8 * u) = pk;
+                    }
                 }
             }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bs.tail_free);    // the S columns are free
         }
     }
     tc_fence_before();
@@ -537,9 +631,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
             mbar_wait(d, 0);
         }
         if (warp == 0 && lane == 0) {
-            for (int k = max(0, nft - kStages); k < nft; ++k) mbar_wait(&bs.full[k % kStages], (k / kStages) & 1);
-            mbar_wait(&bs.abs_full, 0);
-            mbar_wait(&bs.wuv_full, 0);
+            for (int pos = max(0, loads_R - kStages); pos < loads_R; ++pos)
+                mbar_wait(&bs.full[pos & 1], (pos >> 1) & 1);
+            if (loads_q > 0) mbar_wait(&bs.abs_full, (loads_q - 1) & 1);
         }
         if (tid == 0) latch_status(p.status, kStatusTimeout);
         __syncthreads();
@@ -636,6 +730,7 @@ cudaError_t tc_prefill(const PrefillArgs& a, cudaStream_t st, uint64_t* launches
     p.D = sh.D;
     p.s = sh.s;
     p.n_qtiles = (T + kQ - 1) / kQ;
+    p.n_items = p.n_qtiles * sh.B * sh.H;
     p.scale_log2 = sh.scale * 1.4426950408889634f;
     p.log2_rope_base = sh.log2_rope_base;
     p.q_r = (const bf16*)a.q_r;
@@ -655,7 +750,9 @@ cudaError_t tc_prefill(const PrefillArgs& a, cudaStream_t st, uint64_t* launches
     // the attribute is set on every call: it is per kernel instance and device
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return note_error("cudaFuncSetAttribute(k_prefill_tc)", e);
-    const unsigned grid = (unsigned)p.n_qtiles * sh.B * sh.H;
+    // persistent: one CTA per SM (the shared memory allows no second), each
+    // walking its share of the items
+    const unsigned grid = (unsigned)std::min(p.n_items, sm_count());
     profile_begin(st);
     kern<<<grid, kThreads, smem, st>>>(maps, p);
     profile_end(st);
