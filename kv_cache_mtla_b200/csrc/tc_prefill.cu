@@ -62,7 +62,6 @@ struct PreTC {
     float scale_log2;
     double log2_rope_base;
     const bf16* q_r;  // [B, T, H, d_r]
-    const bf16* P;    // [B, T, D]: partial slots from the scan (the own-slot keys)
     const float2* rope_tab;   // [T, d_r / 2]: (cos, sin) of every position, from the scan
     bf16* out;        // [B, T, H, d_h]
     int* status;
@@ -87,6 +86,8 @@ struct Maps {
     CUtensorMap wuv;    // (d_c, d_h, H)    box (64, d_h, 1)
     CUtensorMap slots;  // (D, n_slots, B)  box (64, 128, 1), 128-byte swizzle: latent chunks
     CUtensorMap slots_r;  // (D, n_slots, B)  box (32, 128, 1), 64-byte swizzle: the RoPE chunk
+    CUtensorMap prow;   // (D, T, B)        box (64, 128, 1): the scan's partial slots, latent chunks
+    CUtensorMap prow_r; // (D, T, B)        box (32, 128, 1): their RoPE chunk
 };
 
 __device__ __forceinline__ bool waitb(uint64_t* bar, uint32_t parity, Bars& bs) {
@@ -126,17 +127,6 @@ __device__ __forceinline__ void st_row32_bf16_sw64(uint8_t* base, int row, const
     }
 }
 
-// 32 bf16 of a global row (16-byte aligned) as fp32.
-__device__ __forceinline__ void ld_row32_bf16(const bf16* src, float* v) {
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-        const uint4 raw = *(const uint4*)(src + 8 * u);
-        const bf16* e = (const bf16*)&raw;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) v[8 * u + i] = __bfloat162float(e[i]);
-    }
-}
-
 // Work item idx (heaviest first): query tile qt = n_qtiles - 1 - idx / (B H),
 // then sequence and head.
 struct Item {
@@ -163,9 +153,10 @@ __device__ __forceinline__ int item_at(const PreTC& p, int j) {
 }
 
 // One work item = (128 query positions, sequence, head), heaviest first. The
-// own partial slot of every row is handled on the CUDA cores (its score is one
-// dot product per row; its value enters the output at the end with the row's
-// final weight); the finished slots stream through the tensor cores in 128-slot
+// own partial slots of the item's rows come into the ring as one tile; each
+// row's score against its own slot is one dot product on the CUDA cores, and O
+// starts as that slot's latent part (weight 1 at the starting reference
+// maximum); the finished slots stream through the tensor cores in 128-slot
 // tiles. DC = d_c (d_h = 64 and d_R = 32 are fixed): every MMA sequence is
 // unrolled at compile time (a runtime loop or branch between tcgen05.mma
 // instructions halves their issue rate).
@@ -267,6 +258,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
             for (int j = 0; idx >= 0 && !bs.fail; ++j) {
                 const Item it = decode_item(p, idx);
                 const int nidx = item_at(p, j + 1);
+                {
+                    // the item's own partial slots P[b, p0 .. p0+127] as one ring position
+                    // (same layout as a key tile; rows past T read as zeros)
+                    const int pos = R++;
+                    if (!ring_free(pos)) break;
+                    uint8_t* dst = ring + (pos & 1) * stage_bytes;
+                    mbar_arrive_expect_tx(&bs.full[pos & 1], stage_bytes);
+#pragma unroll
+                    for (int c = 0; c < NL; ++c)
+                        tma_load_3d(dst + c * chunk_k, &maps.prow, &bs.full[pos & 1], c * 64, it.p0, it.b);
+                    tma_load_3d(dst + NL * chunk_k, &maps.prow_r, &bs.full[pos & 1], DC, it.p0, it.b);
+                    loads_R = R;
+                }
                 bool ok = true;
                 for (int k = 0; k < it.nft && ok; ++k) {
                     const int pos = R++;
@@ -337,6 +341,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
                 if (!waitb(&bs.q_ready, j & 1, bs)) break;
                 // the S columns held the previous item's O_lat and output until read
                 if (j > 0 && !waitb(&bs.tail_free, (j - 1) & 1, bs)) break;
+                ++R;                                 // the item's own partial slots (the softmax reads them)
                 bool ok = true;
                 for (int k = 0; k < it.nft; ++k, ++G) {
                     const int pos = R++;
@@ -377,6 +382,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
                 const int idx = item_at(p, j);
                 if (idx < 0) break;
                 const Item it = decode_item(p, idx);
+                ++R;                                   // the item's own partial slots
                 for (int k = 0; k < it.nft; ++k, ++G) {
                     const int pos = R++;
                     if (!(ok = waitb(&bs.p_full[G & 1], (G >> 1) & 1, bs))) break;
@@ -385,8 +391,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
                     const uint64_t vd = sdesc_sw128(ring_a + (pos & 1) * stage_bytes, chunk_k, 1024);
 #pragma unroll
                     for (int kk = 0; kk < kKT / 16; ++kk)
-                        umma_bf16_ts(t_o, t_s0 + (G & 1) * kKT + kk * 8, desc_add(vd, kk * 2048), id_o,
-                                     (k > 0 || kk > 0) ? 1u : 0u);
+                        umma_bf16_ts(t_o, t_s0 + (G & 1) * kKT + kk * 8, desc_add(vd, kk * 2048), id_o, 1u);
                     umma_commit(&bs.empty[pos & 1]);
                     umma_commit(&bs.o_done[G & 1]);
                     umma_commit(&bs.s_empty[G & 1]);   // S buffer G & 1 (which held P) is free
@@ -407,7 +412,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
         constexpr int half = DC / 2;
         float v[32];
         uint32_t w[32];
-        int G = 0;
+        int G = 0, R = 0;
         for (int j = 0;; ++j) {
             const int idx = item_at(p, j);
             if (idx < 0) break;
@@ -415,7 +420,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
             const int b = it.b, h = it.h, p0 = it.p0, nft = it.nft;
             const int pos = p0 + r;
             const bool row_ok = pos < p.T;
-            const bf16* prow = p.P + ((size_t)b * p.T + min(pos, p.T - 1)) * p.D;   // own partial slot
+            // ring positions of this item: own partial slots, key tiles, W_UV
+            const int ppos = R;
+            R += nft + 2;
+            const uint8_t* pst = ring + (ppos & 1) * stage_bytes;   // row r: this row's own partial slot
             // q~ row block of 32 columns into the query image: latent columns into the
             // 128-byte-swizzled chunks, the RoPE block into the 64-byte-swizzled one
             auto put_q = [&](int col) {
@@ -423,27 +431,22 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
                 else st_row32_bf16_sw64(q_s + NL * kQ * 128, r, v);
             };
             float e_own = 0.f;
+            // 8 columns [c, c + 8) of this row's own partial slot, from the ring
+            auto own8 = [&](int c) -> uint4 {
+                return c < DC ? *(const uint4*)(pst + (c >> 6) * chunk_k + sw128_offset(r, c & 63))
+                              : *(const uint4*)(pst + NL * chunk_k + sw64_offset(r, c - DC));
+            };
             // q~ row in 32-column blocks, the first half of the blocks for hc = 0 and
             // the rest for hc = 1 (which therefore holds the RoPE block): latent blocks
             // from TMEM, the RoPE block rotated with the scan's (cos, sin) table; all
             // rounded to bf16 into the query image. The own-slot score q~ . P_pos uses
-            // the same rounded values. Every global load of a block is issued before
-            // the wait for the absorption.
+            // the same rounded values.
             constexpr int n_blk = NL * 2 + 1, nb0 = (n_blk + 1) / 2;
             const int blk0 = hc == 0 ? 0 : nb0, blk1 = hc == 0 ? nb0 : n_blk;   // <= 5 blocks each
             const bf16* qr = p.q_r + (((size_t)b * p.T + min(pos, p.T - 1)) * p.H + h) * p.d_r;
             const float2* cs_row = p.rope_tab + (size_t)min(pos, p.T - 1) * (p.d_r / 2);
-            uint4 pv4[5][4];
-#pragma unroll
-            for (int q = 0; q < 5; ++q) {
-                const int c0 = (blk0 + q) * 32;
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    pv4[q][u] = make_uint4(0, 0, 0, 0);
-                    if (blk0 + q < blk1 && c0 + 8 * u < p.D) pv4[q][u] = *(const uint4*)(prow + c0 + 8 * u);
-                }
-            }
             waitb(&bs.abs_done, j & 1, bs);
+            waitb(&bs.full[ppos & 1], (ppos >> 1) & 1, bs);
             tc_fence_after();
 #pragma unroll
             for (int q = 0; q < 5; ++q) {
@@ -483,9 +486,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
                         }
                     }
                     put_q(c0);
-                    const bf16* pe = (const bf16*)pv4[q];
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) e_own = fmaf(v[i], __bfloat162float(pe[i]), e_own);
+                    for (int u = 0; u < 4; ++u) {
+                        const uint4 raw = own8(c0 + 8 * u);
+                        const bf16* pe = (const bf16*)&raw;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) e_own = fmaf(v[8 * u + i], __bfloat162float(pe[i]), e_own);
+                    }
                 }
             }
             fence_proxy_async();
@@ -493,9 +500,29 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
             __syncwarp();
             if (lane == 0) mbar_arrive(&bs.q_ready);
             bs.xs[hc][r] = e_own;
-            named_sync(1, 256);
+            named_sync(1, 256);                           // also: every q~ read of TMEM is done
+            tc_fence_after();
             const float es = row_ok ? (bs.xs[0][r] + bs.xs[1][r]) * p.scale_log2 : 0.f;
-            named_sync(1, 256);                           // xs is free again
+            // O starts as the own slot's latent part, with weight 1 at the starting
+            // reference maximum es (its TMEM columns held q~, read above)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int cc = hc * half + 32 * q;
+                if (32 * q < half) {
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const uint4 raw = own8(cc + 8 * u);
+                        const bf16* pe = (const bf16*)&raw;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) v[8 * u + i] = __bfloat162float(pe[i]);
+                    }
+                    tmem_st32(t_o + cc + lane_off, v);
+                }
+            }
+            tmem_wait_st();
+            fence_proxy_async();
+            named_sync(1, 256);                           // xs is free again; the own slots are read
+            if (tid == 64) mbar_arrive(&bs.empty[ppos & 1]);   // their ring position is free
             // online softmax over the finished-slot tiles; the own slot is the
             // starting point (reference maximum es, weight 1 in the row sum)
             float m_ref = es, l = hc == 0 ? 1.f : 0.f;    // l: this thread's half of the row sum
@@ -541,11 +568,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
                     w[c] = pack_bf16x2(q0, q1);
                 }
                 l = fmaf(l, fac, (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
-                const bool need = upd && k > 0;           // O holds this item's tiles 0..k-1
-                if (__any_sync(0xffffffffu, need)) {
-                    waitb(&bs.o_done[(G - 1) & 1], ((G - 1) >> 1) & 1, bs);
+                // O holds the own slot and this item's tiles 0..k-1
+                if (__any_sync(0xffffffffu, upd)) {
+                    if (k > 0) waitb(&bs.o_done[(G - 1) & 1], ((G - 1) >> 1) & 1, bs);
                     tc_fence_after();
-                    const float f = need ? fac : 1.f;
+                    const float f = upd ? fac : 1.f;
                     for (int cc = hc * half; cc < (hc + 1) * half; cc += 32) {
                         tmem_ld32(t_o + cc + lane_off, v);
                         tmem_wait_ld();
@@ -564,32 +591,22 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
                 if (lane == 0) mbar_arrive(&bs.p_full[G & 1]);
                 m_ref = nm;
             }
-            // epilogue: O_lat = (O + w_own P_pos[:d_c]) / l as bf16 pairs into the S
-            // columns (the output MMA's A operand), then out = O_lat . W_UV^T
+            // epilogue: O_lat = O / l as bf16 pairs into the S columns (the output
+            // MMA's A operand), then out = O_lat . W_UV^T
             if (nft > 0) waitb(&bs.o_done[(G - 1) & 1], ((G - 1) >> 1) & 1, bs);
             tc_fence_after();
             bs.xs[hc][r] = l;
             named_sync(1, 256);
             const float inv = 1.f / (bs.xs[0][r] + bs.xs[1][r]);
-            const float w_own = ex2_approx(es - m_ref);
             named_sync(1, 256);                           // xs is free again
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const int cc = hc * half + 32 * q;
                 if (32 * q < half) {
-                    if (nft > 0) {
-                        tmem_ld32(t_o + cc + lane_off, v);
-                        tmem_wait_ld();
-                    } else {
+                    tmem_ld32(t_o + cc + lane_off, v);
+                    tmem_wait_ld();
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) v[i] = 0.f;
-                    }
-                    float pv[32];
-                    ld_row32_bf16(prow + cc, pv);
-#pragma unroll
-                    for (int i = 0; i < 16; ++i)
-                        w[i] = pack_bf16x2(fmaf(w_own, pv[2 * i], v[2 * i]) * inv,
-                                           fmaf(w_own, pv[2 * i + 1], v[2 * i + 1]) * inv);
+                    for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(v[2 * i] * inv, v[2 * i + 1] * inv);
                     tmem_st16_u(t_olat + cc / 2 + lane_off, w);
                 }
             }
@@ -720,6 +737,17 @@ cudaError_t tc_prefill(const PrefillArgs& a, cudaStream_t st, uint64_t* launches
             e = make_map(enc, &maps.slots_r, a.cache_out, 3, d, s, bxr, "cache_out RoPE", CU_TENSOR_MAP_SWIZZLE_64B);
         if (e != cudaSuccess) return e;
     }
+    {
+        // the own partial slots P [B, T, D] as 128-row tiles of the same layout
+        cuuint64_t d[3] = {(cuuint64_t)sh.D, (cuuint64_t)T, (cuuint64_t)sh.B};
+        cuuint64_t s[2] = {E * sh.D, E * T * sh.D};
+        cuuint32_t bx[3] = {64, kQ, 1};
+        cuuint32_t bxr[3] = {kDr, kQ, 1};
+        cudaError_t e = make_map(enc, &maps.prow, P, 3, d, s, bx, "partial slots");
+        if (e == cudaSuccess)
+            e = make_map(enc, &maps.prow_r, P, 3, d, s, bxr, "partial slots RoPE", CU_TENSOR_MAP_SWIZZLE_64B);
+        if (e != cudaSuccess) return e;
+    }
     PreTC p;
     p.B = sh.B;
     p.T = T;
@@ -734,7 +762,6 @@ cudaError_t tc_prefill(const PrefillArgs& a, cudaStream_t st, uint64_t* launches
     p.scale_log2 = sh.scale * 1.4426950408889634f;
     p.log2_rope_base = sh.log2_rope_base;
     p.q_r = (const bf16*)a.q_r;
-    p.P = P;
     p.rope_tab = (const float2*)((char*)a.workspace + align256((size_t)sh.B * T * sh.D * sizeof(bf16)));
     p.out = (bf16*)a.out;
     p.status = a.status;
