@@ -97,35 +97,22 @@ __device__ __forceinline__ bool waitb(uint64_t* bar, uint32_t parity, Bars& bs) 
     return false;
 }
 
-// Store 32 fp32 values as bf16 into row `row`, columns [col, col+32) of a
-// K-major SW128 operand made of [rows x 64] chunks spaced chunk_bytes apart.
-__device__ __forceinline__ void st_row32_bf16(uint8_t* base, uint32_t chunk_bytes, int row, int col,
-                                              const float* v) {
-    uint8_t* chunk = base + (size_t)(col >> 6) * chunk_bytes;
+// Store 16 packed bf16 pairs (32 columns from `col`) into row `row` of a K-major
+// SW128 operand made of [rows x 64] chunks spaced chunk_bytes apart, or of the
+// 64-byte-swizzled chunk when sw64 (col is then relative to that chunk).
+__device__ __forceinline__ void st_row32_packed(uint8_t* base, uint32_t chunk_bytes, int row, int col,
+                                                const uint32_t* pk, bool sw64) {
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-        uint4 pk;
-        pk.x = pack_bf16x2(v[8 * u + 0], v[8 * u + 1]);
-        pk.y = pack_bf16x2(v[8 * u + 2], v[8 * u + 3]);
-        pk.z = pack_bf16x2(v[8 * u + 4], v[8 * u + 5]);
-        pk.w = pack_bf16x2(v[8 * u + 6], v[8 * u + 7]);
-        *(uint4*)(chunk + sw128_offset(row, (col & 63) + 8 * u)) = pk;
+        const uint4 q = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+        if (sw64) *(uint4*)(base + sw64_offset(row, col + 8 * u)) = q;
+        else *(uint4*)(base + (size_t)(col >> 6) * chunk_bytes + sw128_offset(row, (col & 63) + 8 * u)) = q;
     }
 }
 
-// Store 32 fp32 values as bf16 into row `row` of a K-major tile of 32 columns
-// (64-byte rows, 64-byte swizzle).
-__device__ __forceinline__ void st_row32_bf16_sw64(uint8_t* base, int row, const float* v) {
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-        uint4 pk;
-        pk.x = pack_bf16x2(v[8 * u + 0], v[8 * u + 1]);
-        pk.y = pack_bf16x2(v[8 * u + 2], v[8 * u + 3]);
-        pk.z = pack_bf16x2(v[8 * u + 4], v[8 * u + 5]);
-        pk.w = pack_bf16x2(v[8 * u + 6], v[8 * u + 7]);
-        *(uint4*)(base + sw64_offset(row, 8 * u)) = pk;
-    }
-}
+// bf16 halves of a packed pair as fp32 (exact: bf16 is the top half of fp32).
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
 // Work item idx (heaviest first): query tile qt = n_qtiles - 1 - idx / (B H),
 // then sequence and head.
@@ -426,9 +413,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
             const uint8_t* pst = ring + (ppos & 1) * stage_bytes;   // row r: this row's own partial slot
             // q~ row block of 32 columns into the query image: latent columns into the
             // 128-byte-swizzled chunks, the RoPE block into the 64-byte-swizzled one
+            // (v holds the block in fp32; it is rounded once, into packed pairs w)
             auto put_q = [&](int col) {
-                if (col < DC) st_row32_bf16(q_s, kQ * 128, r, col, v);
-                else st_row32_bf16_sw64(q_s + NL * kQ * 128, r, v);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+                if (col < DC) st_row32_packed(q_s, kQ * 128, r, col, w, false);
+                else st_row32_packed(q_s + NL * kQ * 128, 0, r, col - DC, w, true);
             };
             float e_own = 0.f;
             // 8 columns [c, c + 8) of this row's own partial slot, from the ring
@@ -455,8 +445,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
                     if (c0 < DC) {
                         tmem_ld32(t_o + c0 + lane_off, v);
                         tmem_wait_ld();
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) v[i] = __bfloat162float(__float2bfloat16_rn(v[i]));
                     } else {
                         // RoPE columns (zero past d_r): qR and the (cos, sin) pairs as vectors
                         const int e0 = c0 - DC;
@@ -480,19 +468,24 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
                             if (row_ok && e0 + i < p.d_r) {
                                 const float cs = csv[i], sn = csv[i + 1];
                                 const float x0 = __bfloat162float(qe[i]), x1 = __bfloat162float(qe[i + 1]);
-                                v[i] = __bfloat162float(__float2bfloat16_rn(x0 * cs - x1 * sn));
-                                v[i + 1] = __bfloat162float(__float2bfloat16_rn(x0 * sn + x1 * cs));
+                                v[i] = x0 * cs - x1 * sn;
+                                v[i + 1] = x0 * sn + x1 * cs;
                             }
                         }
                     }
                     put_q(c0);
+                    float e2[2] = {0.f, 0.f};
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
                         const uint4 raw = own8(c0 + 8 * u);
-                        const bf16* pe = (const bf16*)&raw;
+                        const uint32_t rw[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) e_own = fmaf(v[8 * u + i], __bfloat162float(pe[i]), e_own);
+                        for (int i = 0; i < 4; ++i) {
+                            e2[0] = fmaf(bf16_lo(w[4 * u + i]), bf16_lo(rw[i]), e2[0]);
+                            e2[1] = fmaf(bf16_hi(w[4 * u + i]), bf16_hi(rw[i]), e2[1]);
+                        }
                     }
+                    e_own += e2[0] + e2[1];
                 }
             }
             fence_proxy_async();
