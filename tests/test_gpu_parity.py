@@ -303,7 +303,7 @@ def test_decode_skips_invalid_sequences_in_the_split_plan():
 @pytest.mark.parametrize("T", [1, 63, 129, 300])
 def test_prefill_ragged_lengths(s, T):
     """Speech-decode widths (d_h=64, d_c=256, d_R=32), lengths around the
-    128-position query tiles and 64-slot key tiles, every row against the
+    128-position query tiles and 128-slot key tiles, every row against the
     oracle; the cache and open slot too."""
     wl = inputs.SPEECH_DECODE.with_(B=2, H=3, s=s)
     w = inputs.weights(wl)
@@ -316,6 +316,24 @@ def test_prefill_ragged_lengths(s, T):
     assert rel_err(out, ref["out"]) <= TOL["bf16"]
     assert rel_err(np64(pb.buf.cache[:, :n_slots]), ref["cache"]) <= 4e-3
     assert rel_err(np64(pb.buf.open_slot), ref["acc"]) <= 1e-5
+
+
+@pytest.mark.parametrize("d_c, s, T, B, H", [(256, 2, 2500, 2, 8), (128, 2, 1100, 2, 10), (128, 3, 300, 1, 3)])
+def test_prefill_many_items_per_cta(d_c, s, T, B, H):
+    """More work items (128 positions x sequence x head) than SMs, so every
+    persistent CTA walks several items and the ring, the query region and the
+    TMEM columns pass from one item to the next; both compiled widths
+    (d_c = 256 and 128, d_h = 64, d_R = 32). Every row against the oracle."""
+    wl = inputs.SPEECH_DECODE.with_(B=B, H=H, s=s, d_c=d_c)
+    w = inputs.weights(wl)
+    toks = inputs.tokens(wl, T)
+    ref = oracle.prefill(oracle_cfg(wl), toks["c"], toks["kr"], toks["qc"], toks["qr"], w["w_uk"],
+                         w["w_uv"], w["gate_w"], w["gate_b"])
+    n_slots = (T + s - 1) // s
+    pb = Problem(wl, max_slots=n_slots + 1, max_tokens=T, weights=w)
+    out = np64(pb.prefill(toks, T))
+    assert rel_err(out, ref["out"]) <= TOL["bf16"]
+    assert rel_err(np64(pb.buf.cache[:, :n_slots]), ref["cache"]) <= 4e-3
 
 
 @pytest.mark.parametrize("s", [1, 2, 3, 4])
