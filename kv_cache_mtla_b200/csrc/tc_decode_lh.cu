@@ -603,7 +603,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int u = 0; u < 4; ++u) th[u] = *(const uint4*)(xin + xoff(r, 4 * hc + u));
             float sv[32];
-            float mt = -INFINITY;
+            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // four independent chains
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const uint32_t tw[4] = {th[u].x, th[u].y, th[u].z, th[u].w};
@@ -614,9 +614,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     const int c = 8 * u + 2 * v;
                     sv[c] = c < valid ? fm.x + ft.x : -INFINITY;
                     sv[c + 1] = c + 1 < valid ? fm.y + ft.y : -INFINITY;
-                    mt = fmaxf(mt, fmaxf(sv[c], sv[c + 1]));
+                    m4[v] = fmaxf(m4[v], fmaxf(sv[c], sv[c + 1]));
                 }
             }
+            float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
             bs.red[it & 1][hc][r] = mt;
             named_sync(1, 256);                        // also: every thread has read x_in[it & 1]
             if (leader) mbar_arrive_remote_relaxed(xfree_peer + (it & 1) * 8);
@@ -626,15 +627,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             const bool upd = mt > m_ref + kRescaleLog2;
             const float nm = upd ? mt : m_ref;
             const float fac = ex2_approx(m_ref - nm);    // 0 when m_ref was -inf, 1 when kept
-            float rs = 0.f;
+            float rs4[4] = {0.f, 0.f, 0.f, 0.f};
             uint32_t pk[16];
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
                 const float p0 = ex2_approx(sv[2 * c] - nm), p1 = ex2_approx(sv[2 * c + 1] - nm);
-                rs += p0 + p1;
+                rs4[c & 3] += p0 + p1;
                 pk[c] = pack_bf16x2(p0, p1);
             }
-            l = fmaf(l, fac, rs);
+            l = fmaf(l, fac, (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
             m_ref = nm;
             const bool need = upd && k_in_seg > 0;
             if (__any_sync(0xffffffffu, need)) {
