@@ -10,17 +10,19 @@
 // Launches:
 //   k_prefill_scan<bf16, bf16>  gates, partial slots P (bf16, scratch),
 //                               finished slots (cache_out), open slot
-//   k_prefill_tc                one CTA per (query tile of 128 positions,
-//                               sequence, head), heaviest tiles first:
+//   k_prefill_tc                persistent, one CTA per SM walking work items
+//                               (query tile of 128 positions, sequence, head),
+//                               heaviest first:
 //     absorption   q~ = qC . W_UK[h]          tcgen05 M=128 N=d_c K=d_h
-//     own partial  one dot product q~ . P_t per row on the CUDA cores; it is
-//                  the softmax's starting point and its value P_t enters the
-//                  output at the end with the row's final weight
+//     own partial  the rows' partial slots P_t arrive as one tile; each row's
+//                  score q~ . P_t is one dot product on the CUDA cores and the
+//                  softmax's starting point; O starts as P_t's latent part
 //     finished     128-slot tiles of cache_out  staircase mask on the last
 //                  S = q~ . K^T (M=128 N=128 K=D), online softmax (two threads
 //                  per row, exp2, rescale only when a row max grows by > 2^8),
 //                  O += P . V (M=128 N=d_c K=128, P in TMEM, V = the same tile)
-//     epilogue     out = (O / l) . W_UV[h]^T   tcgen05 M=128 N=d_h K=d_c
+//     epilogue     out = (O / l) . W_UV[h]^T   tcgen05 M=128 N=d_h K=d_c, with
+//                  O / l as bf16 in TMEM (the MMA's A operand)
 // Warp roles: warp 0 TMA, warp 1 absorption / score / output MMAs and TMEM,
 // warps 2-9 softmax, warp 10 P.V MMAs (so P.V, which frees ring stages, never
 // waits behind a score MMA that waits for a load). S is double-buffered in
