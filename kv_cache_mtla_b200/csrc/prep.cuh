@@ -5,6 +5,8 @@
 // kept from MLA). Device functions shared by the CUDA-core and tensor-core
 // decode paths and by the prefill.
 #pragma once
+#include <type_traits>
+
 #include "common.cuh"
 #include "mtla_internal.h"
 
@@ -223,8 +225,22 @@ template <> __device__ __forceinline__ void store8<bf16>(bf16* p, const float* v
 // (stored as PT), the slot itself in the cache (rounded to T: finished, or the
 // last one) and, for the slot holding token T-1, the unrounded open slot.
 // One warp per slot: grid (ceil(ceil(T/s) / 8), B), 256 threads.
+// With bf16 partial slots (the tensor-core prefill) the sine and cosine of the
+// angle, reduced to [-pi, pi] in double as everywhere, come from the special-
+// function unit (absolute error about 2^-21 there, far below the bf16 rounding
+// of the slots); the fp32 partial slots of the CUDA-core path keep sincosf.
 template <typename T, typename PT>
 __global__ void __launch_bounds__(256) k_prefill_scan(PrefillArgs a, PT* P, float2* rope_tab = nullptr) {
+    constexpr bool kFastSinCos = std::is_same<PT, bf16>::value;
+    auto sincos_at = [](int64_t t, double inv_freq, float* sn, float* cs) {
+        if constexpr (kFastSinCos) {
+            double ang = (double)t * inv_freq;
+            ang = fma(-6.283185307179586476925, rint(ang * 0.15915494309189533577), ang);
+            __sincosf((float)ang, sn, cs);
+        } else {
+            pair_sincos_f(t, inv_freq, sn, cs);
+        }
+    };
     const Shape sh = a.sh;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int b = blockIdx.y;
@@ -259,7 +275,7 @@ __global__ void __launch_bounds__(256) k_prefill_scan(PrefillArgs a, PT* P, floa
             float z = 0.f;
             for (int k = lane; k < sh.d_c / 2; k += 32) {
                 float sn, cs;
-                pair_sincos_f(u, pe_freq[k], &sn, &cs);
+                sincos_at(u, pe_freq[k], &sn, &cs);
                 z = fmaf(G[2 * k] * to_f<T>(cu[2 * k]), sn, z);
                 z = fmaf(G[2 * k + 1] * to_f<T>(cu[2 * k + 1]), cs, z);
             }
@@ -289,7 +305,7 @@ __global__ void __launch_bounds__(256) k_prefill_scan(PrefillArgs a, PT* P, floa
         for (int uo = 0; uo < 8; ++uo) {
             if (uo >= nu) continue;
             float sn, cs;
-            pair_sincos_f(u0 + uo, rope_freq[k], &sn, &cs);
+            sincos_at(u0 + uo, rope_freq[k], &sn, &cs);
             // (cos, sin) of every position for the queries' RoPE (sequence 0 writes it)
             if (rope_tab && b == 0) rope_tab[(size_t)(u0 + uo) * (sh.d_r / 2) + k] = make_float2(cs, sn);
             const float x0 = to_f<T>(kr[(size_t)uo * sh.d_r + 2 * k]);
