@@ -155,8 +155,9 @@ __device__ __forceinline__ int item_at(const PreTC& p, int j) {
 // and the next item's set-up overlaps this one's end:
 //   - qC and W_UK of item j+1 load into the query region once the score MMAs
 //     of item j are done (q_free);
-//   - item j's W_UV loads into the ring as one more "tile" after its key tiles,
-//     so the ring's empty/full barriers order it with the tiles around it;
+//   - the ring carries, per item, its own partial slots (one tile, read by the
+//     softmax warps), its key tiles and its W_UV (one more position), so the
+//     ring's empty/full barriers order each with the tiles around it;
 //   - O_lat of item j goes to TMEM (bf16, the output MMA's A operand), so the
 //     absorption of item j+1 into the O columns starts as soon as O is read;
 //   - item j+1's key tiles load as soon as the P.V of item j frees the stages.
