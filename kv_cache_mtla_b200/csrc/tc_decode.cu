@@ -27,6 +27,7 @@
 #include <cudaTypedefs.h>
 
 #include <cstdio>
+#include <cstring>
 #include <mutex>
 #include <utility>
 
@@ -54,11 +55,14 @@ struct DecTC {
     int B, H, D, d_c, s, max_slots;
     int Hp;          // H rounded up to 8: heads per partial row block
     int n_chunks;    // D rounded up to 64, in 64-column chunks
+    int n_lat;       // d_c / 64 latent chunks
+    int compact;     // the RoPE chunk is 32 columns wide (64-byte rows, SW64)
+    uint32_t stage_bytes;   // one slot tile in shared memory
     int lat_blocks;  // d_c / 128
     int G;           // grid size
     float scale_log2;
     const int32_t* pos;
-    const uint8_t* qimg;  // [B] x n_chunks x [NH rows x 128 B]: q~ in bf16, SW128, zero padded
+    const uint8_t* qimg;  // [B] x image: q~ in bf16, the slot tile's chunk layout, zero padded
     uint32_t qimg_bytes;  // per sequence
     float* part;          // [(kMaxGrid + B), Hp, d_c + 2]
     int* status;
@@ -78,9 +82,11 @@ __device__ __forceinline__ int seq_slots(const DecTC& p, int b) {
 
 // Decode prep for the tensor-core path. grid (B, H + 1), 160 threads.
 // Block (b, h < H): absorbed query of head h, q~ = [W_UK[h]^T qC ; RoPE_t(qR)],
-// rounded to bf16 into row h of sequence b's query image (64-column SW128
-// chunks of NH rows, zero beyond D). Block (b, H): gate, RoPE and in-place
-// update of the open slot (MTLA Method (1)), and zero rows H..NH-1 of the image.
+// rounded to bf16 into row h of sequence b's query image: 64-column SW128
+// chunks of NH rows, zero beyond D; in the compact layout (d_R = 32) the RoPE
+// part is one 32-column chunk of 64-byte SW64 rows after the latent chunks.
+// Block (b, H): gate, RoPE and in-place update of the open slot (MTLA Method
+// (1)), and zero rows H..NH-1 of the image.
 // Launched as a programmatic dependent of the previous kernel in the stream:
 // only the W_UK rows (weights, constant across steps) are read before the
 // wait for that kernel; every input of the step and every write come after it.
@@ -89,27 +95,32 @@ __device__ __forceinline__ int seq_slots(const DecTC& p, int b) {
 // starts before its predecessor ends only when that predecessor triggers its
 // dependents early, which the library's own kernels alone do (a step's combine
 // kernel, which writes neither); the C-ABI header states this for callers.
-__global__ void __launch_bounds__(kPrepAbsThreads + 32) k_dec_prep_tc(DecodeArgs a, uint8_t* qimg, int n_chunks, int NH) {
+__global__ void __launch_bounds__(kPrepAbsThreads + 32) k_dec_prep_tc(DecodeArgs a, uint8_t* qimg, uint32_t img_bytes, int n_chunks, int NH, int compact) {
     pdl_launch_dependents();   // the attention kernel may start its prologue now
     const Shape& sh = a.sh;
     const int b = blockIdx.x, h = blockIdx.y;
-    const uint32_t img_bytes = (uint32_t)n_chunks * NH * 128;
     uint8_t* img = qimg + (size_t)b * img_bytes;
+    const int n_wide = compact ? n_chunks - 1 : n_chunks;     // chunks of 128-byte rows
+    uint8_t* rope_img = img + (size_t)n_wide * NH * 128;     // compact: [NH x 64 B]
     if (h == sh.H) {
         pdl_wait();
         decode_update_body<bf16>(a, b);
-        for (int e = threadIdx.x; e < n_chunks * (NH - sh.H) * 8; e += blockDim.x) {
-            const int c = e / ((NH - sh.H) * 8), rr = e % ((NH - sh.H) * 8);
+        const int pad = NH - sh.H;
+        for (int e = threadIdx.x; e < n_wide * pad * 8; e += blockDim.x) {
+            const int c = e / (pad * 8), rr = e % (pad * 8);
             *(uint4*)(img + (size_t)c * NH * 128 + (size_t)(sh.H + rr / 8) * 128 + (rr % 8) * 16) =
                 make_uint4(0, 0, 0, 0);
         }
+        if (compact)
+            for (int e = threadIdx.x; e < pad * 4; e += blockDim.x)
+                *(uint4*)(rope_img + (size_t)(sh.H + e / 4) * 64 + (e % 4) * 16) = make_uint4(0, 0, 0, 0);
         return;
     }
     __shared__ float part_sum[8][512];     // [i-group][latent column]
     const size_t rh = (size_t)b * sh.H + h;
     const bf16* qc = (const bf16*)a.q_c + rh * sh.d_h;
     const bf16* qr = (const bf16*)a.q_r + rh * sh.d_r;
-    const int dpad = n_chunks * 64;
+    const int dpad = compact ? sh.D : n_chunks * 64;
     if (threadIdx.x >= kPrepAbsThreads) {
         // the last warp: RoPE part of q~ (columns d_c .. D-1) and the zero padding
         // up to the chunk boundary, independent of the W_UK product
@@ -125,7 +136,9 @@ __global__ void __launch_bounds__(kPrepAbsThreads + 32) k_dec_prep_tc(DecodeArgs
                 pair_sincos(t, k, sh.d_r, sh.log2_rope_base, &sn, &cs);
                 v = (e & 1) ? (x0 * sn + x1 * cs) : (x0 * cs - x1 * sn);
             }
-            *(bf16*)(img + (size_t)(j >> 6) * NH * 128 + sw128_offset(h, j & 63)) = __float2bfloat16_rn(v);
+            bf16* dst = compact ? (bf16*)(rope_img + sw64_offset(h, j - sh.d_c))
+                                : (bf16*)(img + (size_t)(j >> 6) * NH * 128 + sw128_offset(h, j & 63));
+            *dst = __float2bfloat16_rn(v);
         }
         return;
     }
@@ -190,7 +203,7 @@ __global__ void __launch_bounds__(kPrepAbsThreads + 32) k_dec_prep_tc(DecodeArgs
 // Barriers and small shared state of k_dec_attn_sh.
 template <int HV>
 struct SmallBars {
-    uint64_t full[2], empty[2];          // slot-tile ring
+    uint64_t full[3], empty[3];          // slot-tile ring (2 or 3 stages)
     uint64_t q_full, q_free;             // query image of the current segment
     uint64_t s_full[2], s_empty[2];      // S^T buffers
     uint64_t p_full[2];                  // P^T buffers (4 softmax warps arrive)
@@ -212,24 +225,41 @@ __device__ __forceinline__ bool sb_wait(uint64_t* bar, uint32_t parity, SmallBar
     return false;
 }
 
+// The slot cache as TMA sees it: 64-column SW128 boxes of 128 slots, and (the
+// compact layout) the 32-column RoPE part as one SW64 box.
+struct DecMaps {
+    CUtensorMap lat, rope;
+};
+
 // Split-K attention over 128-slot tiles, heads as the MMA's N (NH = 16 or 32).
 // Warps 0-3: online softmax, thread = slot row (its TMEM lane), over HV heads
 // (H rounded up to 8; a compile-time count, so every per-head loop is
-// straight-line code); warp 4: TMA; warp 5: MMA issue and TMEM. S^T and P^T
-// are double-buffered so MMA1 of the next tile overlaps this tile's softmax.
-template <int NH, int HV>
+// straight-line code); warp 4: TMA; warp 5: score MMAs; warp 6: P.V MMAs. S^T
+// is double-buffered in TMEM so the scores of the next tile overlap this
+// tile's softmax.
+// ST = 2: a tile is n_chunks 64-column SW128 chunks (the RoPE part padded to a
+// whole chunk) and P^T has two buffers of its own.
+// ST = 3 (d_R = 32, NH = 16): the compact layout -- the latent chunks, then the
+// RoPE part as 128 rows of 64 bytes (SW64), 72 KB per tile for d_c = 256 -- and
+// P^T of a tile is written over its RoPE part, which only the score MMAs read
+// and which is free once they are done; that leaves room for a third stage,
+// so two loads stay in flight while a tile is worked on.
+template <int NH, int HV, int ST>
 __global__ void __launch_bounds__(kAttnThreads, 1)
-    k_dec_attn_sh(const __grid_constant__ CUtensorMap tmap, const DecTC p) {
+    k_dec_attn_sh(const __grid_constant__ DecMaps maps, const DecTC p) {
     static_assert(HV % 8 == 0 && HV <= NH, "head count");
+    static_assert(ST == 2 || (ST == 3 && NH == 16), "ring");
+    constexpr bool kCompact = ST == 3;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int n_chunks = p.n_chunks;
-    const uint32_t stage_bytes = (uint32_t)n_chunks * 16384u;
-    uint8_t* ring = smem;                                        // 2 stages
-    uint8_t* q_s = smem + 2 * stage_bytes;                       // n_chunks x [NH x 128 B]
-    uint8_t* p_s = q_s + (size_t)n_chunks * NH * 128;            // 2 buffers x 2 chunks x [NH x 128 B]
-    SmallBars<HV>& bs = *(SmallBars<HV>*)(p_s + 4 * NH * 128);
+    const int n_chunks = p.n_chunks, n_lat = p.n_lat;
+    const uint32_t stage_bytes = p.stage_bytes;
+    const uint32_t pt_off = (uint32_t)n_lat * 16384u;           // compact: P^T over the RoPE part
+    uint8_t* ring = smem;                                        // ST stages
+    uint8_t* q_s = smem + ST * stage_bytes;                      // the query image (qimg_bytes)
+    uint8_t* p_s = q_s + p.qimg_bytes;                           // ST = 2: 2 buffers x 2 chunks x [NH x 128 B]
+    SmallBars<HV>& bs = *(SmallBars<HV>*)(p_s + (kCompact ? 0 : 4 * NH * 128));
     int* starts = (int*)((uint8_t*)&bs + ((sizeof(SmallBars<HV>) + 15) & ~(size_t)15));   // [B + 1]
 
     // ---- schedule: tiles per sequence and their exclusive prefix sum (reads pos only)
@@ -266,9 +296,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     uint32_t tmem_cols = 32;
     while (tmem_cols < tmem_cols_needed) tmem_cols <<= 1;
     if (tid == 0) {
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < ST; ++i) {
             mbar_init(&bs.full[i], 1);
             mbar_init(&bs.empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
             mbar_init(&bs.s_full[i], 1);
             mbar_init(&bs.s_empty[i], 4);
             mbar_init(&bs.p_full[i], 4);
@@ -280,7 +312,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         mbar_init(&bs.drain[1], 1);
         bs.fail = 0;
         fence_mbar_init();
-        tma_prefetch_desc(&tmap);
+        tma_prefetch_desc(&maps.lat);
+        if (kCompact) tma_prefetch_desc(&maps.rope);
     }
     if (warp == 5) {
         tmem_alloc(&bs.tmem_base, tmem_cols);
@@ -315,14 +348,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             auto load_tile = [&](int st, int b, int j) {
+                uint8_t* dst = ring + st * stage_bytes;
                 mbar_arrive_expect_tx(&bs.full[st], stage_bytes);
-                for (int c = 0; c < n_chunks; ++c)
-                    tma_load_3d(ring + st * stage_bytes + (size_t)c * 16384, &tmap, &bs.full[st], c * 64,
-                                j * kTileSlots, b);
+                for (int c = 0; c < (kCompact ? n_lat : n_chunks); ++c)
+                    tma_load_3d(dst + (size_t)c * 16384, &maps.lat, &bs.full[st], c * 64, j * kTileSlots, b);
+                if (kCompact)
+                    tma_load_3d(dst + pt_off, &maps.rope, &bs.full[st], p.d_c, j * kTileSlots, b);
                 ++loads_issued;
             };
             int early = 0;                   // tiles 0..early-1 issued before the wait
-            for (int gt = gt0; gt < gt1 && early < 2; ++gt) {
+            for (int gt = gt0; gt < gt1 && early < ST; ++gt) {
                 int b, j;
                 locate(gt, b, j);
                 if (j + 1 == starts[b + 1] - starts[b]) break;    // holds the open slot
@@ -342,8 +377,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     ++q_loads;
                 }
                 if (it < early) continue;
-                const int st = it & 1;
-                if (it >= 2 && !sb_wait(&bs.empty[st], ((it >> 1) - 1) & 1, bs)) break;
+                const int st = it % ST;
+                if (it >= ST && !sb_wait(&bs.empty[st], ((it / ST) - 1) & 1, bs)) break;
                 load_tile(st, b, j);
             }
         }
@@ -363,15 +398,35 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     ++seg;
                     if (!sb_wait(&bs.q_full, seg & 1, bs)) break;
                 }
-                const int st = it & 1;
-                if (!sb_wait(&bs.full[st], (it >> 1) & 1, bs)) break;
-                if (it >= 2 && !sb_wait(&bs.s_empty[st], ((it >> 1) - 1) & 1, bs)) break;
+                const int rs = it % ST, sb = it & 1;      // ring stage, S^T buffer
+                if (!sb_wait(&bs.full[rs], (it / ST) & 1, bs)) break;
+                if (it >= 2 && !sb_wait(&bs.s_empty[sb], ((it >> 1) - 1) & 1, bs)) break;
                 tc_fence_after();
                 // S^T = K_tile . q~^T (A = slot tile, B = q~ image; both K-major)
                 // The MMAs go out in straight-line groups (one test per group of
                 // four): a runtime loop or a test per MMA halves their issue rate.
-                const uint64_t a0 = sdesc_sw128(ring_a + st * stage_bytes, 16, 1024);
-                const uint32_t ts = t_s + st * NH;
+                const uint64_t a0 = sdesc_sw128(ring_a + rs * stage_bytes, 16, 1024);
+                const uint32_t ts = t_s + sb * NH;
+                if (kCompact) {
+                    // the latent chunks, then the two K-steps of the 64-byte RoPE rows
+#pragma unroll
+                    for (int c = 0; c < kMaxLatBlocks * 2; ++c) {
+                        if (c < n_lat) {
+                            const uint64_t ac = desc_add(a0, c * 16384), bc = desc_add(q_d, c * NH * 128);
+#pragma unroll
+                            for (int kk = 0; kk < 4; ++kk)
+                                umma_bf16(ts, desc_add(ac, kk * 32), desc_add(bc, kk * 32), id_s, (c | kk) != 0);
+                        }
+                    }
+                    const uint64_t ar = sdesc_sw64(ring_a + rs * stage_bytes + pt_off);
+                    const uint64_t br = sdesc_sw64(smem_u32(q_s) + n_lat * NH * 128);
+                    umma_bf16(ts, ar, br, id_s, 1u);
+                    umma_bf16(ts, desc_add(ar, 32), desc_add(br, 32), id_s, 1u);
+                    umma_commit(&bs.s_full[sb]);
+                    const bool last = (gt + 1 == gt1) || (j + 1 == starts[b + 1] - starts[b]);
+                    if (last) umma_commit(&bs.q_free);
+                    continue;
+                }
 #pragma unroll
                 for (int c = 0; c < kMaxChunks - 1; ++c) {
                     if (c < n_chunks - 1) {
@@ -407,7 +462,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                             break;
                     }
                 }
-                umma_commit(&bs.s_full[st]);
+                umma_commit(&bs.s_full[sb]);
                 const bool last = (gt + 1 == gt1) || (j + 1 == starts[b + 1] - starts[b]);
                 if (last) umma_commit(&bs.q_free);
             }
@@ -427,8 +482,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 if (!sb_wait(&bs.p_full[k & 1], (k >> 1) & 1, bs)) break;
                 tc_fence_after();
                 // O^T += V^T . P^T (A = the slot tile, MN-major; B = P^T, K-major)
-                const uint64_t a0 = sdesc_sw128(ring_a + (k & 1) * stage_bytes, 16384, 1024);
-                const uint64_t b0 = sdesc_sw128(p_a + (k & 1) * 2 * NH * 128, 16, 1024);
+                const uint32_t stage_a = ring_a + (k % ST) * stage_bytes;
+                const uint64_t a0 = sdesc_sw128(stage_a, 16384, 1024);
+                const uint64_t b0 = sdesc_sw128(kCompact ? stage_a + pt_off : p_a + (k & 1) * 2 * NH * 128, 16, 1024);
 #pragma unroll
                 for (int lb = 0; lb < kMaxLatBlocks; ++lb) {
                     if (lb < p.lat_blocks) {
@@ -440,7 +496,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                                       (first && kk == 0) ? 0u : 1u);
                     }
                 }
-                umma_commit(&bs.empty[k & 1]);
+                umma_commit(&bs.empty[k % ST]);
                 umma_commit(&bs.o_done[k & 1]);
             }
         }
@@ -464,7 +520,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                     l_part[h] = 0.f;
                 }
             }
-            const int st = it & 1;
+            const int st = it & 1;                  // S^T and P^T buffer parity
+            uint8_t* stage = ring + (it % ST) * stage_bytes;
             const int valid = min(kTileSlots, n_b - j * kTileSlots);
             sb_wait(&bs.s_full[st], (it >> 1) & 1, bs);
             tc_fence_after();
@@ -476,9 +533,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             if (lane == 0) mbar_arrive(&bs.s_empty[st]);
             if (valid < kTileSlots) {
                 // stale rows past the sequence's last slot must not reach P.V
-                // (whole 128-byte rows, so the swizzle does not matter)
-                for (int c = 0; c < n_chunks; ++c) {
-                    uint8_t* base = ring + st * stage_bytes + (size_t)c * 16384;
+                // (whole 128-byte rows of the latent chunks, so the swizzle does
+                // not matter)
+                for (int c = 0; c < n_lat; ++c) {
+                    uint8_t* base = stage + (size_t)c * 16384;
                     for (int off = valid * 128 + tid * 16; off < 16384; off += 128 * 16)
                         *(uint4*)(base + off) = make_uint4(0, 0, 0, 0);
                 }
@@ -508,7 +566,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 l_part[h] = fmaf(l_part[h], fac[h], sv[h]);
             }
             any_rescale &= (k_in_seg > 0);
-            // P^T buffer st was last read by P.V of tile it-2
+            // P.V of tile it-2 is done: it read P^T buffer st (in the compact
+            // layout P^T sits in this tile's own stage instead), and the P.V
+            // thread has taken p_full[st]'s previous phase, so this tile's
+            // arrivals cannot run a whole phase ahead of it
             if (it >= 2) sb_wait(&bs.o_done[st], ((it >> 1) - 1) & 1, bs);
             if (any_rescale) {
                 // the running O^T of this segment moves to the new reference maximum
@@ -526,7 +587,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 tmem_wait_st();
             }
             {
-                uint8_t* pb = p_s + (size_t)st * 2 * NH * 128 + (size_t)(tid >> 6) * NH * 128;
+                uint8_t* pb = (kCompact ? stage + pt_off : p_s + (size_t)st * 2 * NH * 128) +
+                              (size_t)(tid >> 6) * NH * 128;
 #pragma unroll
                 for (int h = 0; h < HV; ++h) *(bf16*)(pb + sw128_offset(h, tid & 63)) = __float2bfloat16_rn(sv[h]);
             }
@@ -575,7 +637,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // a bounded wait gave up: let this CTA's copies and MMAs land (bounded
         // again) before the shared memory and TMEM are released, then report
         if (warp == 4 && lane == 0) {
-            for (int k = max(0, loads_issued - 2); k < loads_issued; ++k) mbar_wait(&bs.full[k & 1], (k >> 1) & 1);
+            for (int k = max(0, loads_issued - ST); k < loads_issued; ++k) mbar_wait(&bs.full[k % ST], (k / ST) & 1);
             if (q_loads > 0) mbar_wait(&bs.q_full, (q_loads - 1) & 1);
         }
         if ((warp == 5 || warp == 6) && lane == 0) {
@@ -713,15 +775,55 @@ __global__ void __launch_bounds__(256) k_dec_combine(DecodeArgs a, DecTC p) {
 
 int n_chunks_of(const Shape& sh) { return (sh.D + 63) / 64; }
 
-size_t attn_smem_bytes(const Shape& sh, int NH) {
-    const size_t nc = n_chunks_of(sh);
-    size_t bytes = 1024;                          // alignment slack
-    bytes += 2 * nc * 16384;                      // two stages
-    bytes += nc * NH * 128;                       // q~
-    bytes += 4 * NH * 128;                        // P^T (2 buffers)
-    bytes += sizeof(SmallBars<32>);               // upper bound for every head count
-    bytes += ((size_t)sh.B + 1) * 4 + 16;         // tile prefix sums
+int heads_padded(const Shape& sh) { return (sh.H + 7) & ~7; }
+int nh_of(const Shape& sh) { return sh.H <= 16 ? 16 : 32; }
+
+// One slot tile in shared memory: whole 64-column chunks, or (compact) the
+// latent chunks and 128 RoPE rows of 64 bytes.
+uint32_t stage_bytes_of(const Shape& sh, bool compact) {
+    return compact ? (uint32_t)(sh.d_c / 64) * 16384u + (uint32_t)kTileSlots * 64u
+                   : (uint32_t)n_chunks_of(sh) * 16384u;
+}
+
+// The query image of one sequence in the tile's chunk layout (NH rows).
+uint32_t qimg_bytes_of(const Shape& sh, bool compact) {
+    const uint32_t nh = (uint32_t)nh_of(sh);
+    return compact ? (uint32_t)(sh.d_c / 64) * nh * 128u + nh * 64u : (uint32_t)n_chunks_of(sh) * nh * 128u;
+}
+
+size_t small_bars_bytes(int HV) {
+    switch (HV) {
+        case 8: return sizeof(SmallBars<8>);
+        case 16: return sizeof(SmallBars<16>);
+        case 24: return sizeof(SmallBars<24>);
+        default: return sizeof(SmallBars<32>);
+    }
+}
+
+// Dynamic shared memory of k_dec_attn_sh with `stages` ring stages (3 means
+// the compact layout); the kernel's static shared memory comes on top.
+size_t attn_smem_bytes(const Shape& sh, int stages) {
+    const bool compact = stages == 3;
+    size_t bytes = 1024;                                   // alignment slack
+    bytes += (size_t)stages * stage_bytes_of(sh, compact); // the ring
+    bytes += qimg_bytes_of(sh, compact);                   // q~
+    if (!compact) bytes += 4 * (size_t)nh_of(sh) * 128;    // P^T (2 buffers)
+    bytes += (small_bars_bytes(heads_padded(sh)) + 15) & ~(size_t)15;
+    bytes += ((size_t)sh.B + 1) * 4 + 16;                  // tile prefix sums
     return bytes;
+}
+
+constexpr size_t kSmemOptin = 232448;      // per-block opt-in limit of sm_100
+constexpr size_t kStaticMargin = 64;       // >= the kernel's static shared memory (32 B)
+
+// The compact three-stage ring: 32 RoPE columns, at most 16 heads, room for
+// it, and CTAs that may get more than two tiles (with two or fewer, both sit
+// in a two-stage ring at once, and the smaller kernel leaves room on its SM
+// for the prep and combine kernels that overlap it).
+bool use_three_stages(const Shape& sh, int grid) {
+    const int64_t max_tiles = (int64_t)sh.B * ((sh.max_slots + kTileSlots - 1) / kTileSlots);
+    return sh.d_r == 32 && sh.d_c % 64 == 0 && sh.H <= 16 && max_tiles > 2 * (int64_t)grid &&
+           attn_smem_bytes(sh, 3) + kStaticMargin <= kSmemOptin;
 }
 
 // Opt the kernel into `smem` bytes of dynamic shared memory (once per device
@@ -762,24 +864,28 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
-template <int NH, int HV>
-cudaError_t launch_attn(const CUtensorMap& map, const DecTC& p, size_t smem, cudaStream_t st) {
+template <int NH, int HV, int ST>
+cudaError_t launch_attn(const DecMaps& maps, const DecTC& p, size_t smem, cudaStream_t st) {
     static size_t done[64] = {0};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64) dev = 0;
-    cudaError_t e = ensure_smem(k_dec_attn_sh<NH, HV>, smem, &done[dev]);
+    cudaError_t e = ensure_smem(k_dec_attn_sh<NH, HV, ST>, smem, &done[dev]);
     if (e != cudaSuccess) return note_error("cudaFuncSetAttribute(k_dec_attn_sh)", e);
     return note_error("k_dec_attn_sh launch",
-                      launch_pdl(k_dec_attn_sh<NH, HV>, dim3(p.G), dim3(kAttnThreads), smem, st, map, p));
+                      launch_pdl(k_dec_attn_sh<NH, HV, ST>, dim3(p.G), dim3(kAttnThreads), smem, st, maps, p));
 }
 
-cudaError_t launch_attn_any(const CUtensorMap& map, const DecTC& p, size_t smem, cudaStream_t st) {
+cudaError_t launch_attn_any(const DecMaps& maps, const DecTC& p, size_t smem, cudaStream_t st) {
+    if (p.compact) {
+        if (p.Hp == 8) return launch_attn<16, 8, 3>(maps, p, smem, st);
+        return launch_attn<16, 16, 3>(maps, p, smem, st);
+    }
     switch (p.Hp) {
-        case 8: return launch_attn<16, 8>(map, p, smem, st);
-        case 16: return launch_attn<16, 16>(map, p, smem, st);
-        case 24: return launch_attn<32, 24>(map, p, smem, st);
-        default: return launch_attn<32, 32>(map, p, smem, st);
+        case 8: return launch_attn<16, 8, 2>(maps, p, smem, st);
+        case 16: return launch_attn<16, 16, 2>(maps, p, smem, st);
+        case 24: return launch_attn<32, 24, 2>(maps, p, smem, st);
+        default: return launch_attn<32, 32, 2>(maps, p, smem, st);
     }
 }
 
@@ -813,15 +919,15 @@ int sm_count() {
 bool tc_decode_supported(const Shape& sh) {
     return sh.H <= 32 && sh.d_c % 128 == 0 && n_chunks_of(sh) <= 6 && sh.B <= kMaxB &&
            (size_t)sh.d_h * sh.d_c * sizeof(bf16) <= 160 * 1024 &&
-           attn_smem_bytes(sh, sh.H <= 16 ? 16 : 32) <= 232448 - 1024;
+           attn_smem_bytes(sh, 2) + kStaticMargin <= kSmemOptin;
 }
 
-static uint32_t qimg_bytes(const Shape& sh) {
-    return (uint32_t)n_chunks_of(sh) * (sh.H <= 16 ? 16 : 32) * 128;
-}
+// Workspace layout: the query images (sized for the larger, padded layout),
+// then the split partials.
+static size_t qimg_region(const Shape& sh) { return align256((size_t)sh.B * qimg_bytes_of(sh, false)); }
 
 size_t tc_decode_workspace(const Shape& sh) {
-    return align256((size_t)sh.B * qimg_bytes(sh)) +
+    return qimg_region(sh) +
            align256((size_t)(kMaxGrid + sh.B) * ((sh.H + 7) & ~7) * (sh.d_c + 2) * sizeof(float));
 }
 
@@ -829,23 +935,32 @@ cudaError_t tc_decode(const DecodeArgs& a, cudaStream_t st, uint64_t* launches) 
     const Shape& sh = a.sh;
     char* ws = (char*)a.workspace;
     uint8_t* qimg = (uint8_t*)ws;
-    float* part = (float*)(ws + align256((size_t)sh.B * qimg_bytes(sh)));
-    const int NH = sh.H <= 16 ? 16 : 32;
+    float* part = (float*)(ws + qimg_region(sh));
+    const int NH = nh_of(sh);
+    const int grid = (int)std::min<int64_t>(std::min(sm_count(), kMaxGrid),
+                                            (int64_t)sh.B * ((sh.max_slots + kTileSlots - 1) / kTileSlots));
+    const bool compact = use_three_stages(sh, grid);
 
     auto encode = (PFN_cuTensorMapEncodeTiled_v12000)tensor_map_encoder();
     if (!encode) return note_error("cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", cudaErrorNotSupported);
-    CUtensorMap map;
+    DecMaps maps;
+    memset(&maps, 0, sizeof(maps));
     cuuint64_t dims[3] = {(cuuint64_t)sh.D, (cuuint64_t)sh.max_slots, (cuuint64_t)sh.B};
     cuuint64_t strides[2] = {(cuuint64_t)sh.D * 2, (cuuint64_t)sh.max_slots * sh.D * 2};
-    cuuint32_t box[3] = {64, (cuuint32_t)kTileSlots, 1};
     cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.cache, dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) {
-        char buf[96];
-        snprintf(buf, sizeof(buf), "cuTensorMapEncodeTiled (CUresult %d)", (int)r);
-        return note_error(buf, cudaErrorInvalidValue);
+    for (int m = 0; m < (compact ? 2 : 1); ++m) {
+        // the latent map (64-column SW128 boxes), then the RoPE map (one
+        // 32-column SW64 box starting at column d_c: 2 * d_c bytes, 16-aligned)
+        cuuint32_t box[3] = {m == 0 ? 64u : 32u, (cuuint32_t)kTileSlots, 1};
+        CUresult r = encode(m == 0 ? &maps.lat : &maps.rope, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.cache, dims,
+                            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                            m == 0 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) {
+            char buf[96];
+            snprintf(buf, sizeof(buf), "cuTensorMapEncodeTiled (CUresult %d)", (int)r);
+            return note_error(buf, cudaErrorInvalidValue);
+        }
     }
 
     DecTC p;
@@ -857,13 +972,15 @@ cudaError_t tc_decode(const DecodeArgs& a, cudaStream_t st, uint64_t* launches) 
     p.s = sh.s;
     p.max_slots = sh.max_slots;
     p.n_chunks = n_chunks_of(sh);
+    p.n_lat = sh.d_c / 64;
+    p.compact = compact ? 1 : 0;
+    p.stage_bytes = stage_bytes_of(sh, compact);
     p.lat_blocks = sh.d_c / 128;
-    const int64_t max_tiles = (int64_t)sh.B * ((sh.max_slots + kTileSlots - 1) / kTileSlots);
-    p.G = (int)std::min<int64_t>(std::min(sm_count(), kMaxGrid), max_tiles);
+    p.G = grid;
     p.scale_log2 = sh.scale * 1.4426950408889634f;
     p.pos = a.pos;
     p.qimg = qimg;
-    p.qimg_bytes = qimg_bytes(sh);
+    p.qimg_bytes = qimg_bytes_of(sh, compact);
     p.part = part;
     p.status = a.status;
 
@@ -883,11 +1000,11 @@ cudaError_t tc_decode(const DecodeArgs& a, cudaStream_t st, uint64_t* launches) 
         }
     }
     cudaError_t e = launch_pdl(k_dec_prep_tc, dim3(sh.B, sh.H + 1), dim3(kPrepAbsThreads + 32), 0, st, a, qimg,
-                               p.n_chunks, NH);
+                               p.qimg_bytes, p.n_chunks, NH, p.compact);
     if (e != cudaSuccess) return note_error("k_dec_prep_tc launch", e);
-    const size_t smem = attn_smem_bytes(sh, NH);
+    const size_t smem = attn_smem_bytes(sh, compact ? 3 : 2);
     profile_begin(st);
-    e = launch_attn_any(map, p, smem, st);
+    e = launch_attn_any(maps, p, smem, st);
     profile_end(st);
     if (e != cudaSuccess) return e;
     const size_t comb_smem = (size_t)sh.d_h * sh.d_c * sizeof(bf16);

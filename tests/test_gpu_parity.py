@@ -270,6 +270,34 @@ def test_decode_many_short_sequences(H):
     assert rel_err(out[sample], ref["out"]) <= TOL["bf16"]
 
 
+@pytest.mark.parametrize("H,d_c,d_r,B", [(12, 256, 32, 24), (16, 128, 32, 30), (3, 256, 32, 40),
+                                          (8, 256, 64, 20), (8, 128, 16, 20)])
+def test_small_head_decode_ring_layouts(H, d_c, d_r, B):
+    """Both slot-tile layouts of the small-head tensor-core kernel: the compact
+    three-stage ring (32 RoPE columns in 64-byte rows, P^T over them; 8 and 16
+    padded heads, d_c 128 and 256) and the padded two-stage ring (RoPE widths
+    64 and 16). Up to 32 tiles per sequence, so CTAs take several tiles and
+    their ranges cross sequences."""
+    wl = inputs.SPEECH_DECODE.with_(B=B, H=H, d_c=d_c, d_r=d_r, s=2)
+    max_slots = 4096
+    w = inputs.weights(wl)
+    toks = inputs.tokens(wl, 1, stream=3)
+    cache0 = inputs.synthetic_cache(wl, max_slots * wl.s - 1, max_slots)
+    rng = np.random.default_rng(1000 + H + d_c + d_r)
+    pos = rng.integers(0, max_slots * wl.s, size=wl.B)
+    pos[:3] = [0, 255, max_slots * wl.s - 1]       # one slot; a whole tile (128 slots); full cache
+    pb = Problem(wl, max_slots=max_slots, weights=w)
+    pb.buf.cache.copy_(cache0["cache"].to(pb.dt))
+    pb.buf.open_slot.copy_(cache0["acc"])
+    out = np64(pb.decode(toks, 0, pos))
+    cfg = oracle_cfg(wl)
+    cache_o = cache0["cache"].double().numpy().copy()
+    acc_o = cache0["acc"].double().numpy().copy()
+    ref = oracle.decode_step(cfg, toks["c"][:, 0], toks["kr"][:, 0], toks["qc"][:, 0], toks["qr"][:, 0],
+                             w["w_uk"], w["w_uv"], pos, cache_o, acc_o, w["gate_w"], w["gate_b"])
+    assert rel_err(out, ref["out"]) <= TOL["bf16"]
+
+
 def test_decode_skips_invalid_sequences_in_the_split_plan():
     """Sequences whose position is beyond the cache get no tiles; the others
     around them are still right, and CAPACITY is latched."""
