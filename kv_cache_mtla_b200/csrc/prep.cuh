@@ -12,17 +12,44 @@
 
 namespace mtla {
 
+constexpr int kUpdMaxPer = 4;     // latent pairs per thread of the slot update (d_c / 2 <= 4 * blockDim)
+constexpr int kUpdMaxPairs = 3;   // RoPE pairs per thread (d_r / 2 <= 3 * blockDim)
+
+// Inverse frequencies base^(-2k/d) of this thread's sinusoidal-PE pairs (over
+// d_c) and RoPE pairs (over d_R) in the slot update: position independent, so
+// a kernel may compute them before it waits for the step's inputs.
+struct UpdateFreqs {
+    double pe[kUpdMaxPer];
+    double rope[kUpdMaxPairs];
+};
+
+__device__ __forceinline__ void update_freqs(const Shape& sh, UpdateFreqs& f) {
+    const int nt = blockDim.x, tid = threadIdx.x;
+#pragma unroll
+    for (int i = 0; i < kUpdMaxPer; ++i) {
+        const int kp = tid + i * nt;
+        f.pe[i] = kp < sh.d_c / 2 ? exp2(-(2.0 * kp / (double)sh.d_c) * sh.log2_pe_base) : 0.0;
+    }
+#pragma unroll
+    for (int i = 0; i < kUpdMaxPairs; ++i) {
+        const int kp = tid + i * nt;
+        f.rope[i] = kp < sh.d_r / 2 ? exp2(-(2.0 * kp / (double)sh.d_r) * sh.log2_rope_base) : 0.0;
+    }
+}
+
 // Decode: gate (the merging weight of token t: sigmoid(G[t mod s] .
 // (c_t * PE_t) + g[t mod s]) computed, the supplied value, or 1), RoPE and
 // in-place update of sequence b's open slot; writes the rounded row into the
 // cache. Every thread of the block must call it (block reduction inside).
 // Returns false (and latches CAPACITY) if pos[b] does not fit the cache.
+// `gate_w` is G [s x d_c] (global memory, or a copy in shared memory) and `f`
+// the frequencies from update_freqs.
 template <typename T>
-__device__ bool decode_update_body(const DecodeArgs& a, int b) {
+__device__ bool decode_update_body(const DecodeArgs& a, int b, const float* gate_w, const UpdateFreqs& f) {
     const Shape& sh = a.sh;
     __shared__ float red[32];
-    constexpr int kMaxPer = 4;                    // latent pairs per thread (d_c / 2 <= 4 * blockDim)
-    constexpr int kMaxPairs = 3;                  // RoPE pairs per thread (d_r / 2 <= 3 * blockDim)
+    constexpr int kMaxPer = kUpdMaxPer;
+    constexpr int kMaxPairs = kUpdMaxPairs;
     const int nt = blockDim.x, tid = threadIdx.x;
     const T* c = (const T*)a.c_new + (size_t)b * sh.d_c;
     const T* kr = (const T*)a.kr_new + (size_t)b * sh.d_r;
@@ -76,7 +103,7 @@ __device__ bool decode_update_body(const DecodeArgs& a, int b) {
         y0[i] = y1[i] = 0.f;
         if (kp < sh.d_r / 2) {
             float sn, cs;
-            pair_sincos(t, kp, sh.d_r, sh.log2_rope_base, &sn, &cs);
+            pair_sincos_f(t, f.rope[i], &sn, &cs);
             y0[i] = x0[i] * cs - x1[i] * sn;
             y1[i] = x0[i] * sn + x1[i] * cs;
         }
@@ -94,8 +121,8 @@ __device__ bool decode_update_body(const DecodeArgs& a, int b) {
             const int kp = tid + i * nt;
             g0[i] = g1[i] = 0.f;
             if (kp < sh.d_c / 2) {
-                g0[i] = a.gate_w[(size_t)r * sh.d_c + 2 * kp];
-                g1[i] = a.gate_w[(size_t)r * sh.d_c + 2 * kp + 1];
+                g0[i] = gate_w[(size_t)r * sh.d_c + 2 * kp];
+                g1[i] = gate_w[(size_t)r * sh.d_c + 2 * kp + 1];
             }
         }
         float z = 0.f;
@@ -104,7 +131,7 @@ __device__ bool decode_update_body(const DecodeArgs& a, int b) {
             const int kp = tid + i * nt;
             if (kp < sh.d_c / 2) {
                 float sn, cs;
-                pair_sincos(t, kp, sh.d_c, sh.log2_pe_base, &sn, &cs);   // PE_t[2kp], PE_t[2kp+1]
+                pair_sincos_f(t, f.pe[i], &sn, &cs);   // PE_t[2kp], PE_t[2kp+1]
                 z = fmaf(g0[i] * c0[i], sn, z);
                 z = fmaf(g1[i] * c1[i], cs, z);
             }
@@ -136,6 +163,13 @@ __device__ bool decode_update_body(const DecodeArgs& a, int b) {
         }
     }
     return true;
+}
+
+template <typename T>
+__device__ bool decode_update_body(const DecodeArgs& a, int b) {
+    UpdateFreqs f;
+    update_freqs(a.sh, f);
+    return decode_update_body<T>(a, b, a.gate_w, f);
 }
 
 // Absorbed query of (row, head h) at position t into qt[(row*H + h)*D ...]

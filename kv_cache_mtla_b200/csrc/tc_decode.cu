@@ -102,9 +102,21 @@ __global__ void __launch_bounds__(kPrepAbsThreads + 32) k_dec_prep_tc(DecodeArgs
     uint8_t* img = qimg + (size_t)b * img_bytes;
     const int n_wide = compact ? n_chunks - 1 : n_chunks;     // chunks of 128-byte rows
     uint8_t* rope_img = img + (size_t)n_wide * NH * 128;     // compact: [NH x 64 B]
+    __shared__ float part_sum[8][512];     // W_UK blocks: [i-group][latent column]; update block: G
     if (h == sh.H) {
+        // weights first (G into shared memory, the PE and RoPE frequencies),
+        // then the wait, then the step's inputs
+        UpdateFreqs f;
+        update_freqs(sh, f);
+        const float* gw = a.gate_w;
+        if (sh.gate_mode == 0 && sh.s * sh.d_c <= 8 * 512) {
+            float* gs = &part_sum[0][0];
+            for (int e = threadIdx.x; e < sh.s * sh.d_c; e += blockDim.x) gs[e] = a.gate_w[e];
+            __syncthreads();
+            gw = gs;
+        }
         pdl_wait();
-        decode_update_body<bf16>(a, b);
+        decode_update_body<bf16>(a, b, gw, f);
         const int pad = NH - sh.H;
         for (int e = threadIdx.x; e < n_wide * pad * 8; e += blockDim.x) {
             const int c = e / (pad * 8), rr = e % (pad * 8);
@@ -116,7 +128,6 @@ __global__ void __launch_bounds__(kPrepAbsThreads + 32) k_dec_prep_tc(DecodeArgs
                 *(uint4*)(rope_img + (size_t)(sh.H + e / 4) * 64 + (e % 4) * 16) = make_uint4(0, 0, 0, 0);
         return;
     }
-    __shared__ float part_sum[8][512];     // [i-group][latent column]
     const size_t rh = (size_t)b * sh.H + h;
     const bf16* qc = (const bf16*)a.q_c + rh * sh.d_h;
     const bf16* qr = (const bf16*)a.q_r + rh * sh.d_r;
