@@ -47,8 +47,8 @@
  *     whose size mtla_workspace_size() reports.
  *   - Stream order: the first kernel of a bf16 decode step is launched as a
  *     programmatic dependent of the kernel before it, so consecutive steps
- *     overlap. It reads only the absorbed projection W_UK before that kernel
- *     finishes. That holds for any kernel that does not trigger its
+ *     overlap. It reads only weights (the absorbed projection W_UK and the
+ *     gate's G) before that kernel finishes. That holds for any kernel that does not trigger its
  *     dependents early (ordinary kernels never do). A caller kernel that does
  *     trigger early must write the step's inputs before it triggers. Those
  *     inputs are the positions, latents, queries and gates.

@@ -88,8 +88,8 @@ __device__ __forceinline__ int seq_slots(const DecTC& p, int b) {
 // Block (b, H): gate, RoPE and in-place update of the open slot (MTLA Method
 // (1)), and zero rows H..NH-1 of the image.
 // Launched as a programmatic dependent of the previous kernel in the stream:
-// only the W_UK rows (weights, constant across steps) are read before the
-// wait for that kernel; every input of the step and every write come after it.
+// only weights (the W_UK rows, G) are read before the wait for that kernel;
+// every input of the step and every write come after it.
 // The attention kernel may start at once: it reads the positions and finished
 // slots before its own wait. Those are safe to read early because this kernel
 // starts before its predecessor ends only when that predecessor triggers its
