@@ -572,7 +572,7 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) inputs, random-init weights)",
             "config": _config(ws),
-            "decode": {"tokens_per_s": dec_tokens * ws / dec_s,
+            "decode": {"tokens_per_s": dec_tokens * ws * args.steps / dec_s,
                        "ms_per_token_step": 1e3 * dec_s / (rep.S * args.steps),
                        "latent_cache_GBps": wl.B * slot_bytes * sum(slots) * args.steps / dec_s / 1e9,
                        "slots_per_seq": [slots[0], slots[-1]]},
