@@ -312,6 +312,70 @@ def run_reference(args, ws, rank):
     print(json.dumps(line), flush=True)
 
 
+def run_reorder_workload(args):
+    """Beam-search reorder of the cache (``mtla_reorder_cache``): 64 sequences of
+    4096 tokens at the stride-sweep widths with s = 2, i.e. 2048 filled slots of
+    576 B each, parents a seeded random permutation. Algorithmic bytes = read +
+    write of the filled slots and the fp32 open slots, against the measured
+    HBM copy bandwidth (which counts read + write too). L2 flushed before every
+    timed call; each call (one kernel) bracketed by CUDA events. The oracle's
+    reorder of the same arrays is timed on the host beside it."""
+    import numpy as np
+    hbm, _, peak_kind = _peaks()
+    wl = inputs.WORKLOADS["stride_sweep"].with_(s=2)
+    B, N, s = wl.B, wl.T, wl.s
+    max_slots = N // s
+    cfg = mtla.make_config(B, wl.H, wl.d_h, wl.d_c, wl.d_r, s, max_slots)
+    g = torch.Generator().manual_seed(0)
+    h_cache = torch.randn(B, max_slots, cfg.D, generator=g).to(torch.bfloat16)
+    h_open = torch.randn(B, cfg.D, generator=g)
+    h_src = torch.randperm(B, generator=g).to(torch.int32)
+    cache_in, open_in = h_cache.cuda(), h_open.cuda()
+    cache_out, open_out = torch.empty_like(cache_in), torch.empty_like(open_in)
+    src = h_src.cuda()
+    n_tok = torch.full((B,), N, dtype=torch.int32, device="cuda")
+    nbytes = 2 * (B * max_slots * cfg.D * 2 + B * cfg.D * 4)
+    flush = L2Flush()
+    st = torch.cuda.current_stream()
+
+    def call():
+        mtla.reorder_cache(cfg, src, n_tok, cache_in, open_in, cache_out, open_out)
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for i in range(args.steps):
+            flush()
+            ev[i][0].record(st)
+            call()
+            ev[i][1].record(st)
+        torch.cuda.synchronize()
+    assert mtla.get_device_status() == mtla.OK
+    ms = statistics.median(a.elapsed_time(b) for a, b in ev)
+    achieved = nbytes / (ms / 1e3) / 1e9
+    cpu = None
+    if not args.no_cpu_baseline:
+        import oracle
+        c_in = h_cache.view(torch.int16).numpy().view(np.uint16)
+        c_out = np.empty_like(c_in)
+        o_in, o_out = h_open.numpy(), np.empty_like(h_open.numpy())
+        t0 = time.perf_counter()
+        oracle.reorder_cache(s, h_src.numpy(), np.full(B, N, np.int32), c_in, o_in, c_out, o_out)
+        dt = time.perf_counter() - t0
+        cpu = {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+               "sample": f"the whole reorder, once ({dt:.3f} s)"}
+    line = {"workload": "beam_reorder",
+            "config": {"B": B, "d_c": wl.d_c, "d_R": wl.d_r, "s": s, "tokens": N, "slots": max_slots,
+                       "parents": "random permutation"},
+            "kernel_ms": ms,
+            "roofline": {"kernel": "k_reorder_cache", "bound": "hbm", "achieved": achieved, "peak": hbm,
+                         "unit": "GB/s", "frac": achieved / hbm, "bytes_per_launch": nbytes,
+                         "peak_source": f"{peak_kind} hbm_gbs"},
+            "cpu_baseline": cpu, "clocks": clk.summary(), "l2": L2Flush.desc + " call"}
+    print(json.dumps(line), flush=True)
+
+
 def run_kernel_workload(args, ws, rank):
     """Kernel-level measurement of one of the other workloads (not the contract
     line): decode attention GB/s against the measured HBM copy bandwidth, or
@@ -400,10 +464,16 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default="speech_decode",
                     help="speech_decode (the contract line) or a kernel-level measurement of "
-                         "stride_sweep[:s], prefill or large_latent")
+                         "stride_sweep[:s], prefill, large_latent or beam_reorder")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     ws, rank = _dist()
+    if args.workload == "beam_reorder":
+        if rank == 0:
+            run_reorder_workload(args)
+        if ws > 1:
+            torch.distributed.destroy_process_group()
+        return
     if args.workload != "speech_decode":
         if rank == 0:
             run_kernel_workload(args, ws, rank)

@@ -196,6 +196,30 @@ mtla_status mtla_decode_step_noalloc(const mtla_config* cfg,
                                      const float* gate_in, const int32_t* pos,
                                      void* cache, float* open_slot, void* out, void* stream);
 
+/* Beam-search reorder of the cache, between decode steps. The authors'
+ * toolkit decodes with parallel beam search (its project page on
+ * sourcepulse.org, "Highlighted Details"); after a step each surviving beam b
+ * continues from a parent beam j = src[b], whose cache it must take over:
+ *   cache_out[b, 0:n) = cache_in[j, 0:n),  n = ceil(n_tokens[j] / s)
+ *   open_out[b]       = open_in[j]
+ * The copy is byte exact. Slots n .. max_slots-1 of cache_out[b] are left as
+ * they were. Out of place: the caller keeps two caches and swaps them.
+ *
+ *   src       [B] int32, device: parent of each destination, 0 <= src[b] < B
+ *             (duplicates allowed); an index outside skips destination b and
+ *             latches INVALID_ARG.
+ *   n_tokens  [B] int32, device, indexed by parent: tokens cached in it (its
+ *             next decode position); above max_slots * s skips the
+ *             destinations that take that parent and latches CAPACITY.
+ *   cache_in, cache_out   [B, max_slots, d_c + d_r] dtype; must not overlap.
+ *   open_in, open_out     [B, d_c + d_r] fp32; must not overlap.
+ * Only cfg's batch, d_c, d_r, stride, dtype and max_slots matter. All
+ * pointers 16-byte aligned; INVALID_ARG (nothing launched) otherwise or if
+ * the buffers overlap. Returns OK once the work is enqueued. */
+mtla_status mtla_reorder_cache(const mtla_config* cfg, const int32_t* src, const int32_t* n_tokens,
+                               const void* cache_in, const float* open_in,
+                               void* cache_out, float* open_out, void* stream);
+
 /* Synchronises `stream`, then returns and clears the status latched by
  * device-side checks on the current device since the last call (OK if none). */
 mtla_status mtla_get_device_status(void* stream);

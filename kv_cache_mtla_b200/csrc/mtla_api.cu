@@ -283,6 +283,34 @@ const char* mtla_status_string(mtla_status s) {
     return "unknown status";
 }
 
+mtla_status mtla_reorder_cache(const mtla_config* cfg, const int32_t* src, const int32_t* n_tokens,
+                               const void* cache_in, const float* open_in, void* cache_out,
+                               float* open_out, void* stream) {
+    Shape sh;
+    mtla_status st = check_config(cfg, &sh);
+    if (st != MTLA_OK) return st;
+    const void* req[] = {src, n_tokens, cache_in, open_in, cache_out, open_out};
+    for (const void* p : req)
+        if (!p || !aligned16(p)) return MTLA_ERR_INVALID_ARG;
+    const size_t esize = cfg->dtype == MTLA_FP32 ? 4 : 2;
+    const size_t cache_bytes = (size_t)sh.B * sh.max_slots * sh.D * esize;
+    const size_t open_bytes = (size_t)sh.B * sh.D * sizeof(float);
+    auto overlap = [](const void* a, size_t na, const void* b, size_t nb) {
+        const uintptr_t x = (uintptr_t)a, y = (uintptr_t)b;
+        return x < y + nb && y < x + na;
+    };
+    if (overlap(cache_in, cache_bytes, cache_out, cache_bytes) || overlap(open_in, open_bytes, open_out, open_bytes))
+        return MTLA_ERR_INVALID_ARG;
+    g_error_detail[0] = 0;
+    int* status = nullptr;
+    if (note_error("device status word", status_ptr(&status)) != cudaSuccess) return MTLA_ERR_CUDA;
+    uint64_t n = 0;
+    cudaError_t e = reorder_cache(sh, esize, src, n_tokens, cache_in, open_in, cache_out, open_out, status,
+                                  (cudaStream_t)stream, &n);
+    g_launches += n;
+    return e == cudaSuccess ? MTLA_OK : MTLA_ERR_CUDA;
+}
+
 uint64_t mtla_kernel_launches(void) { return g_launches.load(); }
 
 const char* mtla_last_error_detail(void) { return g_error_detail; }

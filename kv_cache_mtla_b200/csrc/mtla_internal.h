@@ -79,6 +79,11 @@ bool tc_prefill_supported(const Shape& sh);
 size_t tc_prefill_workspace(const Shape& sh, int T);
 cudaError_t tc_prefill(const PrefillArgs& a, cudaStream_t st, uint64_t* launches);
 
+// Beam-search reorder of the slot cache and open slots (cache_ops.cu).
+cudaError_t reorder_cache(const Shape& sh, size_t elem_bytes, const int32_t* src, const int32_t* n_tokens,
+                          const void* cache_in, const float* open_in, void* cache_out, float* open_out,
+                          int* status, cudaStream_t st, uint64_t* launches);
+
 // Driver entry point cuTensorMapEncodeTiled (NULL if unavailable), looked up once.
 void* tensor_map_encoder();
 // Streaming multiprocessors of the current device (cached per device).

@@ -75,6 +75,8 @@ def load() -> ctypes.CDLL:
     lib.mtla_prefill.restype = ctypes.c_int
     lib.mtla_decode_step_noalloc.argtypes = [cp] + [_vp] * 13 + [_vp]
     lib.mtla_decode_step_noalloc.restype = ctypes.c_int
+    lib.mtla_reorder_cache.argtypes = [cp] + [_vp] * 6 + [_vp]
+    lib.mtla_reorder_cache.restype = ctypes.c_int
     lib.mtla_get_device_status.argtypes = [_vp]
     lib.mtla_get_device_status.restype = ctypes.c_int
     lib.mtla_status_string.argtypes = [ctypes.c_int]
@@ -160,6 +162,17 @@ def prefill(cfg, T, c, kr, q_c, q_r, w_uk, w_uv, gate_w, gate_b, gate_in, out, c
         _ptr(open_slot_out), _ptr(workspace), ws, _stream(stream))
     if check and st != OK:
         raise MtlaError(st, "mtla_prefill")
+    return st
+
+
+def reorder_cache(cfg, src, n_tokens, cache_in, open_in, cache_out, open_out, stream=None,
+                  check=True) -> int:
+    """Forward to ``mtla_reorder_cache`` (beam-search reorder of the cache and
+    open slots, out of place); returns the status (raises if check)."""
+    st = load().mtla_reorder_cache(ctypes.byref(cfg), _ptr(src), _ptr(n_tokens), _ptr(cache_in),
+                                   _ptr(open_in), _ptr(cache_out), _ptr(open_out), _stream(stream))
+    if check and st != OK:
+        raise MtlaError(st, "mtla_reorder_cache")
     return st
 
 

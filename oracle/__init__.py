@@ -100,6 +100,8 @@ def _load():
                                          + [_PI] + [_P] * 5)
         _lib.orc_prefill_explicit.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int32] + [_P] * 10
         _lib.orc_set_fault.argtypes = [ctypes.c_int]
+        _lib.orc_reorder_cache.argtypes = [ctypes.c_int32] * 5 + [ctypes.c_void_p] * 6
+        _lib.orc_reorder_cache.restype = ctypes.c_int
     return _lib
 
 
@@ -211,3 +213,21 @@ def prefill_explicit(cfg: Cfg, c, kr, qc, qr, w_uk, w_uv, G=None, g=None, gate_i
     _load().orc_prefill_explicit(ctypes.byref(cfg.c()), T, _p(c), _p(kr), _p(qc), _p(qr),
                                  _p(w_uk), _p(w_uv), _p(G), _p(g), _p(gate_in), _p(out))
     return out
+
+
+def reorder_cache(s: int, src, n_tokens, cache_in, open_in, cache_out, open_out) -> int:
+    """Beam-search reorder: destination b takes the filled slots and the open
+    slot of parent src[b] (``orc_reorder_cache``). ``cache_in``/``cache_out``
+    [B,max_slots,D] of any element type (copied as bytes; pass bf16 as its
+    uint16 bits), ``open_in``/``open_out`` [B,D] float32; the outputs are
+    numpy arrays updated in place. Returns the status (0, 1 or 3)."""
+    for a in (cache_in, cache_out, open_in, open_out):
+        assert isinstance(a, np.ndarray) and a.flags.c_contiguous
+    assert cache_in.dtype == cache_out.dtype and cache_in.shape == cache_out.shape
+    assert open_in.dtype == np.float32 and open_out.dtype == np.float32
+    B, max_slots, D = cache_in.shape
+    src = np.ascontiguousarray(src, dtype=np.int32)
+    n_tokens = np.ascontiguousarray(n_tokens, dtype=np.int32)
+    return int(_load().orc_reorder_cache(B, max_slots, D, int(s), cache_in.itemsize,
+                                         src.ctypes.data, n_tokens.ctypes.data, cache_in.ctypes.data,
+                                         open_in.ctypes.data, cache_out.ctypes.data, open_out.ctypes.data))

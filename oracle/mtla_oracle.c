@@ -408,3 +408,37 @@ void orc_prefill_explicit(const orc_cfg* cfg, int32_t T, const double* c, const 
     free(w);
     free(P);
 }
+
+/* Beam-search reorder of the cache (the authors' toolkit decodes with
+ * parallel beam search: its project page on sourcepulse.org, "Highlighted
+ * Details"). Destination b takes over the cache of its parent j = src[b]:
+ * the ceil(n_tokens[j] / s) slots j has filled (slot count of n tokens, as
+ * above) and j's open-slot accumulator, both copied byte for byte (values of
+ * `elem_bytes` bytes in the cache, float32 in the open slot); the other slots
+ * of the destination keep their contents. A parent outside [0, B) leaves the
+ * destination unchanged and gives status 1, a parent with more tokens than
+ * the cache holds gives 3 (the first in b order is returned, 0 if none). */
+int orc_reorder_cache(int32_t B, int32_t max_slots, int32_t D, int32_t s, int32_t elem_bytes,
+                      const int32_t* src, const int32_t* n_tokens, const unsigned char* cache_in,
+                      const float* open_in, unsigned char* cache_out, float* open_out) {
+    int status = 0;
+    const size_t row_bytes = (size_t)D * (size_t)elem_bytes;
+    for (int32_t b = 0; b < B; ++b) {
+        const int32_t j = src[b];
+        if (j < 0 || j >= B) {
+            if (!status) status = 1;
+            continue;
+        }
+        const int64_t n = n_tokens[j];
+        if (n < 0 || n > (int64_t)max_slots * s) {
+            if (!status) status = 3;
+            continue;
+        }
+        const int64_t slots = (n + s - 1) / s;
+        for (int64_t k = 0; k < slots; ++k)
+            memcpy(cache_out + ((size_t)b * max_slots + (size_t)k) * row_bytes,
+                   cache_in + ((size_t)j * max_slots + (size_t)k) * row_bytes, row_bytes);
+        for (int32_t e = 0; e < D; ++e) open_out[(size_t)b * D + e] = open_in[(size_t)j * D + e];
+    }
+    return status;
+}

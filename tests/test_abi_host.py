@@ -141,6 +141,29 @@ def test_prefill_rejects_bad_arguments_before_launch(lib):
     assert _call_prefill(lib, cfg, 32, ws, q_c=None) == mtla.ERR_INVALID_ARG
 
 
+def test_reorder_rejects_bad_arguments_before_launch(lib):
+    """Null or unaligned pointers and overlapping input/output buffers are
+    refused on the host, before any CUDA call."""
+    cfg = _cfg(B=4, max_slots=16)
+    cache_bytes = 4 * 16 * (256 + 32) * 2
+    base = dict(src=FAKE, n_tokens=FAKE + 256, cache_in=FAKE + 0x100000, open_in=FAKE + 0x400000,
+                cache_out=FAKE + 0x800000, open_out=FAKE + 0xC00000)
+
+    def call(**over):
+        a = dict(base)
+        a.update(over)
+        return lib.mtla_reorder_cache(ctypes.byref(cfg), a["src"], a["n_tokens"], a["cache_in"],
+                                      a["open_in"], a["cache_out"], a["open_out"], None)
+    for name in base:
+        assert call(**{name: None}) == mtla.ERR_INVALID_ARG, name
+        assert call(**{name: base[name] + 8}) == mtla.ERR_INVALID_ARG, name
+    # the output cache starting inside the input cache, and the open slots in place
+    assert call(cache_out=base["cache_in"] + cache_bytes - 16) == mtla.ERR_INVALID_ARG
+    assert call(open_out=base["open_in"]) == mtla.ERR_INVALID_ARG
+    bad = _cfg(B=4, max_slots=0)
+    assert lib.mtla_reorder_cache(ctypes.byref(bad), *base.values(), None) == mtla.ERR_INVALID_ARG
+
+
 def test_product_imports_nothing_from_the_oracle():
     """The product package must not import, link or call the oracle."""
     pkg = os.path.join(ROOT, "kv_cache_mtla_b200")

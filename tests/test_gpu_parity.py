@@ -474,3 +474,79 @@ def test_small_head_decode_one_long_sequence():
                              w["w_uk"], w["w_uv"], pos, cache_o, acc_o, G=w["gate_w"], g=w["gate_b"])
     assert rel_err(out, ref["out"]) <= TOL["bf16"]
     assert rel_err(np64(pb.buf.open_slot), acc_o) <= 1e-5
+
+
+# ----------------------------------------------------------------- beam-search cache reorder
+
+
+def _bits(t):
+    """A tensor's bytes as a C-contiguous numpy array of its shape (bf16 as uint16)."""
+    t = t.detach().cpu().contiguous()
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).numpy().view(np.uint16)
+    return t.numpy()
+
+
+def _reorder_case(B, max_slots, s, dtype, src, n_tok, seed):
+    cfg = mtla.make_config(B, 8, 64, 256, 32, s, max_slots, dtype=dtype)
+    g = torch.Generator().manual_seed(seed)
+    dt = torch.float32 if dtype == "fp32" else torch.bfloat16
+    cache_in = torch.randn(B, max_slots, cfg.D, generator=g).to(dt)
+    cache_out0 = torch.randn(B, max_slots, cfg.D, generator=g).to(dt)
+    open_in = torch.randn(B, cfg.D, generator=g)
+    open_out0 = torch.randn(B, cfg.D, generator=g)
+    dev = lambda t: t.to("cuda").contiguous()
+    co, oo = dev(cache_out0), dev(open_out0)
+    mtla.reorder_cache(cfg, dev(src), dev(n_tok), dev(cache_in), dev(open_in), co, oo)
+    status = mtla.get_device_status()
+    want_c, want_o = _bits(cache_out0).copy(), open_out0.numpy().copy()
+    want_status = oracle.reorder_cache(s, src.numpy(), n_tok.numpy(), _bits(cache_in), open_in.numpy(),
+                                       want_c, want_o)
+    return status, want_status, _bits(co), want_c, oo.cpu().numpy(), want_o
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp32"])
+def test_reorder_cache_matches_oracle(dtype):
+    """Beam-search reorder against the oracle, byte for byte: parents with
+    duplicates, token counts from 0 to a full cache (s = 3, so slot counts end
+    inside a block), destination slots past the parent's count untouched."""
+    B, max_slots, s = 37, 150, 3
+    g = torch.Generator().manual_seed(5)
+    src = torch.randint(0, B, (B,), generator=g, dtype=torch.int32)
+    n_tok = torch.randint(0, max_slots * s + 1, (B,), generator=g, dtype=torch.int32)
+    n_tok[:5] = torch.tensor([0, 1, s, s + 1, max_slots * s], dtype=torch.int32)
+    src[:10] = torch.tensor([0, 1, 2, 3, 4, 4, 3, 2, 1, 0], dtype=torch.int32)
+    st, want_st, c, want_c, o, want_o = _reorder_case(B, max_slots, s, dtype, src, n_tok, 11)
+    assert st == mtla.OK and want_st == 0
+    assert np.array_equal(c, want_c)
+    assert np.array_equal(o, want_o)
+
+
+def test_reorder_cache_full_size():
+    """The benchmarked size: 64 sequences of 2048 filled slots (576 bytes),
+    a random permutation of parents; byte for byte."""
+    B, max_slots, s = 64, 2048, 2
+    g = torch.Generator().manual_seed(6)
+    src = torch.randperm(B, generator=g).to(torch.int32)
+    n_tok = torch.full((B,), max_slots * s, dtype=torch.int32)
+    st, want_st, c, want_c, o, want_o = _reorder_case(B, max_slots, s, "bf16", src, n_tok, 12)
+    assert st == mtla.OK and want_st == 0
+    assert np.array_equal(c, want_c)
+    assert np.array_equal(o, want_o)
+
+
+def test_reorder_cache_bad_parent_and_capacity():
+    """A parent index outside [0, B) latches INVALID_ARG, a parent holding more
+    tokens than the cache latches CAPACITY; the affected destinations keep
+    their contents and every other destination is still copied."""
+    B, max_slots, s = 8, 40, 2
+    src = torch.tensor([1, 0, 3, B, 2, 5, 7, 6], dtype=torch.int32)
+    n_tok = torch.tensor([80, 7, 1, 0, 33, 12, 79, 2], dtype=torch.int32)
+    st, want_st, c, want_c, o, want_o = _reorder_case(B, max_slots, s, "bf16", src, n_tok, 13)
+    assert want_st == 1 and st == mtla.ERR_INVALID_ARG
+    assert np.array_equal(c, want_c) and np.array_equal(o, want_o)
+    n_tok[2] = max_slots * s + 1                 # parent of destination 4
+    src[3] = 4
+    st, want_st, c, want_c, o, want_o = _reorder_case(B, max_slots, s, "bf16", src, n_tok, 14)
+    assert want_st == 3 and st == mtla.ERR_CAPACITY
+    assert np.array_equal(c, want_c) and np.array_equal(o, want_o)

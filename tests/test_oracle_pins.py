@@ -323,3 +323,81 @@ def test_mask_probe_support():
             support = np.nonzero(olat[t, 0])[0]
             assert list(support) == list(range(t // s + 1))
             assert np.allclose(olat[t, 0, support], 1.0 / (t // s + 1), atol=1e-15)
+
+
+# ----------------------------------------------------------------- beam-search reorder
+
+
+def test_reorder_worked_example():
+    """Hand-worked case: 3 sequences, 3 slots of width 2, s = 2. Parents
+    src = [2, 2, 0] (a duplicate, a cycle-free gather); n_tokens indexed by
+    parent = [1, 4, 3]. Destination 0 and 1 take parent 2's ceil(3/2) = 2
+    slots, destination 2 takes parent 0's ceil(1/2) = 1 slot; the rest of
+    each destination keeps its old value (999). A scatter instead of a gather,
+    a token count read at the destination, or floor instead of ceil each
+    change this result."""
+    ci = np.arange(18, dtype=np.uint16).reshape(3, 3, 2)
+    co = np.full_like(ci, 999)
+    oi = np.arange(6, dtype=np.float32).reshape(3, 2)
+    oo = np.zeros_like(oi)
+    assert oracle.reorder_cache(2, [2, 2, 0], [1, 4, 3], ci, oi, co, oo) == 0
+    want = np.array([[[12, 13], [14, 15], [999, 999]],
+                     [[12, 13], [14, 15], [999, 999]],
+                     [[0, 1], [999, 999], [999, 999]]], dtype=np.uint16)
+    assert np.array_equal(co, want)
+    assert np.array_equal(oo, np.array([[4, 5], [4, 5], [0, 1]], dtype=np.float32))
+
+
+def test_reorder_slot_count_is_ceil():
+    """n tokens fill ceil(n/s) slots: 0, 1, s, s+1 and a full cache."""
+    s, max_slots = 3, 4
+    for n, slots in ((0, 0), (1, 1), (3, 1), (4, 2), (12, 4)):
+        ci = np.arange(max_slots * 2, dtype=np.float32).reshape(1, max_slots, 2) + 1
+        co = np.zeros_like(ci)
+        oo = np.zeros((1, 2), np.float32)
+        assert oracle.reorder_cache(s, [0], [n], ci, np.ones((1, 2), np.float32), co, oo) == 0
+        copied = int((co[0] != 0).any(axis=1).sum())
+        assert copied == slots, (n, copied)
+
+
+def test_reorder_composes_like_a_gather():
+    """Reordering by p and then by q (token counts follow the first reorder)
+    equals one reorder by p[q]; a permutation followed by its inverse restores
+    every filled slot."""
+    rng = np.random.default_rng(7)
+    B, max_slots, D, s = 9, 11, 4, 2
+    ci = rng.standard_normal((B, max_slots, D)).astype(np.float32)
+    oi = rng.standard_normal((B, D)).astype(np.float32)
+    n = rng.integers(0, max_slots * s + 1, size=B).astype(np.int32)
+    p = rng.integers(0, B, size=B)
+    q = rng.integers(0, B, size=B)
+    c1, o1 = np.zeros_like(ci), np.zeros_like(oi)
+    oracle.reorder_cache(s, p, n, ci, oi, c1, o1)
+    c2, o2 = np.zeros_like(ci), np.zeros_like(oi)
+    oracle.reorder_cache(s, q, n[p], c1, o1, c2, o2)
+    c3, o3 = np.zeros_like(ci), np.zeros_like(oi)
+    oracle.reorder_cache(s, p[q], n, ci, oi, c3, o3)
+    assert np.array_equal(c2, c3) and np.array_equal(o2, o3)
+    perm = rng.permutation(B)
+    back = np.argsort(perm)
+    c4, o4 = np.zeros_like(ci), np.zeros_like(oi)
+    oracle.reorder_cache(s, perm, n, ci, oi, c4, o4)
+    c5, o5 = np.zeros_like(ci), np.zeros_like(oi)
+    oracle.reorder_cache(s, back, n[perm], c4, o4, c5, o5)
+    for b in range(B):
+        k = (n[b] + s - 1) // s
+        assert np.array_equal(c5[b, :k], ci[b, :k])
+    assert np.array_equal(o5, oi)
+
+
+def test_reorder_bad_parent_and_capacity():
+    """A parent outside [0, B) gives status 1 and leaves its destination
+    alone; a parent holding more tokens than the cache gives status 3."""
+    ci = np.ones((2, 2, 2), np.float32)
+    oi = np.ones((2, 2), np.float32)
+    co, oo = np.zeros_like(ci), np.zeros_like(oi)
+    assert oracle.reorder_cache(2, [0, 2], [4, 4], ci, oi, co, oo) == 1
+    assert co[1].sum() == 0 and oo[1].sum() == 0 and co[0].sum() == 4
+    co, oo = np.zeros_like(ci), np.zeros_like(oi)
+    assert oracle.reorder_cache(2, [1, 0], [4, 5], ci, oi, co, oo) == 3
+    assert co[0].sum() == 0 and co[1].sum() == 4
