@@ -21,6 +21,7 @@ namespace mtla {
 
 namespace {
 
+constexpr int kStatusInvalidArg = 1;   // device status word value of MTLA_ERR_INVALID_ARG
 constexpr int kReorderThreads = 256;
 constexpr int kRowsPerBlock = 16;   // slot rows of one sequence per block
 constexpr int kUnroll = 4;          // 16-byte loads in flight per thread before its stores

@@ -7,7 +7,7 @@
 namespace mtla {
 
 // Device-side status codes (same values as mtla_status).
-enum : int { kStatusOk = 0, kStatusInvalidArg = 1, kStatusCapacity = 3, kStatusTimeout = 5 };
+enum : int { kStatusOk = 0, kStatusCapacity = 3, kStatusTimeout = 5 };
 
 // Record the first device-side error; later ones keep the first.
 __device__ __forceinline__ void latch_status(int* status, int code) {
