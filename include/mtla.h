@@ -213,9 +213,10 @@ mtla_status mtla_decode_step_noalloc(const mtla_config* cfg,
  *             destinations that take that parent and latches CAPACITY.
  *   cache_in, cache_out   [B, max_slots, d_c + d_r] dtype; must not overlap.
  *   open_in, open_out     [B, d_c + d_r] fp32; must not overlap.
- * Only cfg's batch, d_c, d_r, stride, dtype and max_slots matter. All
- * pointers 16-byte aligned; INVALID_ARG (nothing launched) otherwise or if
- * the buffers overlap. Returns OK once the work is enqueued. */
+ * cfg must pass the same checks as for the other calls, but only its batch,
+ * d_c, d_r, stride, dtype and max_slots are used. All pointers 16-byte
+ * aligned; INVALID_ARG (nothing launched) otherwise or if the buffers
+ * overlap. Returns OK once the work is enqueued. */
 mtla_status mtla_reorder_cache(const mtla_config* cfg, const int32_t* src, const int32_t* n_tokens,
                                const void* cache_in, const float* open_in,
                                void* cache_out, float* open_out, void* stream);
