@@ -35,6 +35,11 @@ FAULT_SCAN_NO_RESET = 5
 FAULT_DROP_ROPE_KEY = 6
 FAULT_GATE_WRONG_ROW = 7
 FAULT_SCALE = 8
+FAULT_FREQ_EXPONENT = 9
+FAULT_PE_BASE = 10
+FAULT_PAIR_ORDER = 11
+FAULT_ROPE_HALF_SPLIT = 12
+FAULT_PE_SWAP = 13
 
 
 def build(force: bool = False) -> str:

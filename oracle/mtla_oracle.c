@@ -38,8 +38,10 @@
  *     theirs;
  *   - scores use scale 1/sqrt(d_h + d_R) unless a scale is given;
  *   - the merged sum is not normalised.
- * Parity unpinned: the PE, RoPE-frequency and gate conventions above are
- * readings only; the pins check their invariants, not the conventions.
+ * The PE, RoPE-frequency and gate conventions above are readings (the pages
+ * print no worked example of them); the pins hold this file to the exact
+ * values those readings give at small sizes (frequencies 1, 0.1, 0.01, 0.001
+ * at width 8, a gate value worked by hand), besides their invariants.
  *
  * Everything is float64, written as the definitions read, with no blocking,
  * fusion or reordering. Layouts are row-major:
@@ -76,6 +78,11 @@ enum {
     ORC_FAULT_DROP_ROPE_KEY = 6,     /* score only the latent part          */
     ORC_FAULT_GATE_WRONG_ROW = 7,    /* use gate row (t+1) mod s            */
     ORC_FAULT_SCALE = 8,             /* scale by 1/sqrt(d_h)                */
+    ORC_FAULT_FREQ_EXPONENT = 9,     /* PE and RoPE frequencies base^(-k/d)  */
+    ORC_FAULT_PE_BASE = 10,          /* PE with base 1000                    */
+    ORC_FAULT_PAIR_ORDER = 11,       /* frequencies of pairs k >= 1 reversed */
+    ORC_FAULT_ROPE_HALF_SPLIT = 12,  /* RoPE pairs (x_k, x_{k+d/2})          */
+    ORC_FAULT_PE_SWAP = 13,          /* PE with cos at even, sin at odd      */
 };
 static int orc_fault = ORC_FAULT_NONE;
 void orc_set_fault(int f) { orc_fault = f; }
@@ -85,24 +92,37 @@ static double orc_scale(const orc_cfg* cfg) {
     return cfg->scale != 0.0 ? cfg->scale : 1.0 / sqrt((double)(cfg->d_h + cfg->d_r));
 }
 
+/* Inverse frequency base^(-2k/d) of rotation pair k (the reading of the
+ * PE and of RoPE), with the planted schedule mistakes of the tests. */
+static double orc_inv_freq(int32_t k, int32_t d, double base) {
+    if (orc_fault == ORC_FAULT_PAIR_ORDER && k >= 1) k = d / 2 - k;
+    double e = (orc_fault == ORC_FAULT_FREQ_EXPONENT) ? -(double)k / d : -2.0 * k / d;
+    return pow(base, e);
+}
+
 /* Sinusoidal positional embedding of width d at position t. */
 void orc_pe(int64_t t, int32_t d, double base, double* pe) {
+    if (orc_fault == ORC_FAULT_PE_BASE) base = 1000.0;
     for (int32_t k = 0; 2 * k < d; ++k) {
-        double ang = (double)t * pow(base, -2.0 * k / (double)d);
-        pe[2 * k] = sin(ang);
-        if (2 * k + 1 < d) pe[2 * k + 1] = cos(ang);
+        double ang = (double)t * orc_inv_freq(k, d, base);
+        double even = sin(ang), odd = cos(ang);
+        if (orc_fault == ORC_FAULT_PE_SWAP) even = cos(ang), odd = sin(ang);
+        pe[2 * k] = even;
+        if (2 * k + 1 < d) pe[2 * k + 1] = odd;
     }
 }
 
 /* Rotary embedding of a d-vector at position t (interleaved pairs). */
 void orc_rope(int64_t t, int32_t d, double base, const double* x, double* y) {
     for (int32_t k = 0; k < d / 2; ++k) {
-        double ang = (double)t * pow(base, -2.0 * k / (double)d);
+        double ang = (double)t * orc_inv_freq(k, d, base);
         if (orc_fault == ORC_FAULT_ROPE_SIGN) ang = -ang;
         double cs = cos(ang), sn = sin(ang);
-        double x0 = x[2 * k], x1 = x[2 * k + 1];
-        y[2 * k] = x0 * cs - x1 * sn;
-        y[2 * k + 1] = x0 * sn + x1 * cs;
+        int32_t i0 = 2 * k, i1 = 2 * k + 1;
+        if (orc_fault == ORC_FAULT_ROPE_HALF_SPLIT) i0 = k, i1 = k + d / 2;
+        double x0 = x[i0], x1 = x[i1];
+        y[i0] = x0 * cs - x1 * sn;
+        y[i1] = x0 * sn + x1 * cs;
     }
 }
 

@@ -11,7 +11,9 @@ mathematics fix, none of which retypes the oracle's own formulas.
   absorption identities);
 - invariant: incremental decoding == parallel masked forward (Sec. 4.2);
 - brute force: dense enumerated mask over per-token partial slots (tests/brute_force.py);
-- closed forms of the scan, the gate modes, PE and RoPE.
+- closed forms of the scan, the gate modes, PE and RoPE;
+- exact values of the adopted PE / RoPE readings at width 8 (pair frequencies
+  exactly 1, 0.1, 0.01, 0.001 at base 10000) and one gate worked by hand.
 Finally, each planted mistake in the oracle must trip at least one pin.
 """
 import math
@@ -261,6 +263,55 @@ def pin_pe():
     return True
 
 
+def pin_pe_values():
+    """Exact values of the adopted PE reading: interleaved (sin, cos) pairs,
+    pair k turning at base^(-2k/d) with base 10000. At width 8 the four pair
+    frequencies are exactly 1, 0.1, 0.01 and 0.001; at width 4 they are 1 and
+    0.01. Expected values are written from those literals, not from the
+    oracle's formula."""
+    t = 10
+    want8 = [math.sin(10.0), math.cos(10.0), math.sin(1.0), math.cos(1.0),
+             math.sin(0.1), math.cos(0.1), math.sin(0.01), math.cos(0.01)]
+    if np.max(np.abs(oracle.pe(t, 8) - np.array(want8))) > 1e-14:
+        return False
+    want4 = [math.sin(3.0), math.cos(3.0), math.sin(0.03), math.cos(0.03)]
+    return np.max(np.abs(oracle.pe(3, 4) - np.array(want4))) < 1e-14
+
+
+def pin_rope_values():
+    """Exact values of the adopted RoPE reading at width 8, t = 10: the unit
+    vector e_2k comes out as (cos a_k, sin a_k) in pair k and e_2k+1 as
+    (-sin a_k, cos a_k), with a_k = 10 * 10^-k (frequencies 1, 0.1, 0.01,
+    0.001 of base 10000), and nothing leaks into the other pairs."""
+    d, t = 8, 10
+    for k in range(d // 2):
+        a = t * 10.0 ** (-k)
+        for which, pair in ((0, (math.cos(a), math.sin(a))), (1, (-math.sin(a), math.cos(a)))):
+            e = np.zeros(d)
+            e[2 * k + which] = 1.0
+            want = np.zeros(d)
+            want[2 * k], want[2 * k + 1] = pair
+            if np.max(np.abs(oracle.rope(t, e) - want)) > 1e-14:
+                return False
+    return True
+
+
+def pin_gate_value():
+    """One gate worked by hand (Eq. 13 under the adopted reading): t = 3,
+    s = 2, d_c = 4 takes row r = 3 mod 2 = 1; PE_3 at width 4 is
+    (sin 3, cos 3, sin 0.03, cos 0.03); with c = (1, 2, 3, 4),
+    G[1] = (0.5, -1, 0.25, 2), g[1] = 0.1:
+      z = 0.1 + 0.5 sin 3 - 2 cos 3 + 0.75 sin 0.03 + 8 cos 0.03,
+      w = 1 / (1 + e^-z)."""
+    cfg = oracle.Cfg(1, 1, 4, 4, 4, 2)
+    c = np.array([1.0, 2.0, 3.0, 4.0])
+    G = np.array([[9.0, -7.0, 5.0, 3.0], [0.5, -1.0, 0.25, 2.0]])
+    g = np.array([-4.0, 0.1])
+    z = (0.1 + 0.5 * math.sin(3.0) - 2.0 * math.cos(3.0) + 0.75 * math.sin(0.03)
+         + 8.0 * math.cos(0.03))
+    return abs(oracle.gate(cfg, 3, c, G, g) - 1.0 / (1.0 + math.exp(-z))) < 1e-14
+
+
 PINS = {
     "cache_footprint": pin_cache_footprint,
     "s1_is_mla_sdpa": pin_s1_is_mla_sdpa,
@@ -271,6 +322,9 @@ PINS = {
     "gate_modes": pin_gate_modes,
     "rope": pin_rope,
     "pe": pin_pe,
+    "pe_values": pin_pe_values,
+    "rope_values": pin_rope_values,
+    "gate_value": pin_gate_value,
 }
 
 
@@ -295,6 +349,11 @@ FAULTS = {
     "drop_rope_key": oracle.FAULT_DROP_ROPE_KEY,
     "gate_wrong_row": oracle.FAULT_GATE_WRONG_ROW,
     "scale": oracle.FAULT_SCALE,
+    "freq_exponent": oracle.FAULT_FREQ_EXPONENT,
+    "pe_base": oracle.FAULT_PE_BASE,
+    "pair_order": oracle.FAULT_PAIR_ORDER,
+    "rope_half_split": oracle.FAULT_ROPE_HALF_SPLIT,
+    "pe_swap": oracle.FAULT_PE_SWAP,
 }
 
 
