@@ -57,6 +57,11 @@
  *     device (a position beyond the cache, a bounded wait that ran out) skip
  *     the affected work and are latched in a device status word that
  *     mtla_get_device_status() reads.
+ *   - The library looks up the device addresses of its own device variables
+ *     (the status word, the no-allocation scratch array) once per device and
+ *     keeps them for the life of the process. A cudaDeviceReset() on a device
+ *     invalidates them: calls on that device after such a reset are not
+ *     supported.
  */
 #ifndef MTLA_H_
 #define MTLA_H_

@@ -1,5 +1,6 @@
 // mtla_api.cu -- the C ABI of libmtla.so: argument checks, scratch layout,
 // device status word and dispatch to the kernels. See include/mtla.h.
+#include <mutex>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
@@ -67,11 +68,13 @@ void profile_end(cudaStream_t st) {
 
 // Address of g_device_status on the current device (looked up once per device).
 static cudaError_t status_ptr(int** out) {
+    static std::mutex mu;
     static int* cached[64] = {nullptr};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
     if (!cached[dev]) {
         void* p = nullptr;
         e = cudaGetSymbolAddress(&p, g_device_status);

@@ -173,3 +173,12 @@ def test_product_imports_nothing_from_the_oracle():
         text = open(path, errors="ignore").read()
         assert "import oracle" not in text and "from oracle" not in text, path
         assert "mtla_oracle" not in text and "orc_" not in text, path
+
+
+def test_noalloc_limit_matches_header():
+    """The binding's copy of MTLA_NOALLOC_SCRATCH_BYTES equals the macro in
+    include/mtla.h, so the two cannot drift apart silently."""
+    text = open(os.path.join(ROOT, "include", "mtla.h")).read()
+    m = re.search(r"#define\s+MTLA_NOALLOC_SCRATCH_BYTES\s+\((\d+)u\s*<<\s*(\d+)\)", text)
+    assert m, "MTLA_NOALLOC_SCRATCH_BYTES not found in include/mtla.h"
+    assert mtla.NOALLOC_SCRATCH_BYTES == int(m.group(1)) << int(m.group(2))
