@@ -3,26 +3,34 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mtla|reference]
 
-Workload (per rank; weak scaling, every rank runs an independent replica):
-the speech-model-scale decode -- B=16 sequences, H=8, d_h=64, d_c=256,
-d_R=32, s=2 -- one step = the parallel prefill of a 1024-token prefix
-(512 slots) followed by 256 incremental decode steps (513..640 slots), i.e.
-every stage of the path: gate, RoPE, block-prefix scan / in-place slot update,
-query absorption, stride-aware masked attention, split merge, output
-absorption. Inputs are seeded synthetic draws (kv_cache_mtla_b200.inputs).
+Contract line (per rank; weak scaling, every rank runs an independent replica):
+the large-latent decode -- B=32 sequences, H=128, d_h=128, d_c=512, d_R=64
+(slot width 576, 1152 bytes), s=4, supplied gates sigmoid(N(0,1)). One step =
+256 consecutive incremental decode steps of every sequence at positions
+65280..65535, so each decode step attends 16321..16384 slots per sequence and
+the cache ends holding N=65536 tokens: gate, RoPE of the new key, in-place
+update of the slot being filled, query absorption through W_UK, stride-aware
+masked attention over the slots (split over the SMs), merge of the splits and
+output absorption through W_UV. The 604 MB cache is larger than the 126 MB L2,
+and the L2 is also flushed before every step (outside the timed events).
 
-`value` = tokens processed (prefix + decoded) per second over all ranks, from
-CUDA events around each step on the launching stream, the L2 flushed (a
-256 MiB write, then a 256 MiB read) before every step outside the events. The step runs as two
-CUDA graphs captured through the public API (the prefill; the 256 decode
-steps), so host launch overhead is not part of the number. `e2e` times the same
-steps through the public API with every step's inputs copied from pinned host
-memory and its outputs copied back inside one timed region, the copies of the
-next step's inputs and of the previous step's outputs overlapping the current
-step on a copy stream (two device input/output sets). `roofline` reports
-the dominant kernel (decode attention) timed by event pairs the library
-records around it. `cpu_baseline` / `--impl reference` time the float64 CPU
-oracle on a bounded sample of the same workload.
+`value` = latent-cache bytes read by the attention (slots attended x 1152 B)
+per second over all ranks, from CUDA events around each step on the launching
+stream; the 256 decode steps run as one CUDA graph captured through the public
+API. `decode` gives the same run in tokens/s. `roofline` is the dominant kernel
+(the decode attention) timed by event pairs the library records around each of
+its launches in one profiled replay. `e2e` times the same steps through the
+public API with every step's inputs (the 256 tokens' latents, keys, queries,
+gates and positions) copied from pinned host memory and its outputs copied
+back inside one timed region, pipelined on a copy stream.
+
+Sub-objects measure the other workloads, each over its own clock-sampled timed
+region: `prefill` (B=8, T=8192, s=2: TFLOP/s of the masked attention),
+`speech_decode` (B=16, H=8, a 1024-token prefix then 256 decode steps:
+decode tokens/s separately from the prefix), `stride_sweep` (B=64, N=4096,
+s=1..4: latent-cache GB/s of one decode step). `cpu_baseline` and
+`--impl reference` time the float64 CPU oracle on a bounded sample of the
+contract workload (a few of its sequences, one decode step each).
 """
 from __future__ import annotations
 
@@ -42,12 +50,15 @@ sys.path.insert(0, ROOT)
 from kv_cache_mtla_b200 import inputs, mtla  # noqa: E402
 
 METRIC = "decode latent-cache GB/s and tokens/s at N/s slots; prefill TFLOP/s; % roofline"
-WL = inputs.SPEECH_DECODE
+WL = inputs.LARGE_LATENT
+GEN_STEPS = 256          # decode steps per sequence in one contract step
 
 
-def _traffic(kernel):
+def _traffic(kernel, launch_scale=1.0):
     """DRAM bytes (read + write) of one launch of `kernel` from the committed ncu
-    capture, or None when the kernel's sources changed since the capture."""
+    capture, scaled by `launch_scale` (units of the timed launch over units of
+    the captured one), or None when the kernel's sources changed since the
+    capture."""
     import hashlib
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
@@ -59,7 +70,7 @@ def _traffic(kernel):
                 h.update(f.read())
         if h.hexdigest() != rec["sources_sha256"]:
             return None
-        return rec["dram_bytes_read"] + rec["dram_bytes_write"]
+        return (rec["dram_bytes_read"] + rec["dram_bytes_write"]) * launch_scale
     except (OSError, KeyError, ValueError):
         return None
 
@@ -130,7 +141,10 @@ def job_value(units_per_rank_step: float, ws: int, steps: int, max_ms: float) ->
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples during the timed region."""
+    """nvidia-smi clock / throttle-reason samples during the timed region. The
+    sampler is started before the region and the region begins only once the
+    first sample has arrived (or after 3 s), so a region of T seconds holds
+    about T / 50 ms samples."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -138,7 +152,7 @@ class ClockSampler:
     def __init__(self, dev_index: int):
         self.dev = dev_index
         self.proc = None
-        self.path = f"/tmp/mtla_clocks_{os.getpid()}.csv"
+        self.path = f"/tmp/mtla_clocks_{os.getpid()}_{id(self)}.csv"
 
     def __enter__(self):
         try:
@@ -148,6 +162,10 @@ class ClockSampler:
                                          stdout=self.f, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
+            return self
+        t0 = time.time()
+        while time.time() - t0 < 3.0 and os.path.getsize(self.path) == 0:
+            time.sleep(0.02)
         return self
 
     def __exit__(self, *exc):
@@ -161,7 +179,8 @@ class ClockSampler:
 
     def summary(self):
         if self.proc is None or not os.path.exists(self.path):
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"],
+                    "samples": 0}
         sms, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in open(self.path):
@@ -184,132 +203,476 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sms)}
 
 
-class Replica:
-    """One rank's problem: weights, cache, inputs of a whole step on the device."""
+def _events(n, k=2):
+    return [tuple(torch.cuda.Event(enable_timing=True) for _ in range(k)) for _ in range(n)]
+
+
+# --------------------------------------------------------------------- contract
+
+
+class LargeLatentReplica:
+    """One rank's large-latent decode: weights, a cache holding 65280 tokens,
+    and the inputs of 256 decode steps of every sequence, on the device."""
 
     def __init__(self, rank: int):
         wl = WL.with_(seed=WL.seed + 1000 * rank)
         self.wl = wl
-        self.T, self.S = wl.T, wl.steps
-        self.max_slots = (self.T + self.S + wl.s - 1) // wl.s
+        self.S = GEN_STEPS
+        self.N0 = wl.T - self.S                           # tokens cached before the step
+        self.max_slots = (wl.T + wl.s - 1) // wl.s        # 16384
         self.cfg = mtla.make_config(wl.B, wl.H, wl.d_h, wl.d_c, wl.d_r, wl.s, self.max_slots,
                                     dtype=wl.dtype, gate_mode=wl.gate_mode)
-        self.buf = mtla.Buffers.allocate(self.cfg, inputs.weights(wl), max_tokens=self.T)
+        self.buf = mtla.Buffers.allocate(self.cfg, inputs.weights(wl))
+        c0 = inputs.synthetic_cache(wl, self.N0, self.max_slots)
+        self.buf.cache.copy_(c0["cache"].to(torch.bfloat16))
+        self.buf.open_slot.copy_(c0["acc"])
+        del c0
         bf = torch.bfloat16
-        pre = inputs.tokens(wl, self.T, stream=0)
-        dec = inputs.tokens(wl, self.S, stream=1)
-        # host copies (pinned) of one step's inputs, and their device twins
-        self.h = {k: pre[k].to(bf).contiguous().pin_memory() for k in ("c", "kr", "qc", "qr")}
-        for k in ("c", "kr", "qc", "qr"):      # decode tokens, step-major [S, B, ...]
-            self.h["d_" + k] = dec[k].transpose(0, 1).to(bf).contiguous().pin_memory()
+        tk = inputs.tokens(wl, self.S, stream=1)
+        # host copies (pinned) of one step's inputs, step-major [S, B, ...]
+        self.h = {k: tk[k].transpose(0, 1).to(bf).contiguous().pin_memory()
+                  for k in ("c", "kr", "qc", "qr")}
+        self.h["gate_in"] = tk["gate_in"].transpose(0, 1).contiguous().pin_memory()
+        self.h["pos"] = (self.N0 + torch.arange(self.S, dtype=torch.int32)).repeat_interleave(
+            wl.B).view(self.S, wl.B).contiguous().pin_memory()
         self.d = {k: v.to("cuda") for k, v in self.h.items()}
-        self.pos = (self.T + torch.arange(self.S, dtype=torch.int32)).repeat_interleave(wl.B)
-        self.pos = self.pos.view(self.S, wl.B).contiguous().to("cuda")
-        self.out_p = torch.empty(wl.B, self.T, wl.H, wl.d_h, device="cuda", dtype=bf)
-        self.out_d = torch.empty(self.S, wl.B, wl.H, wl.d_h, device="cuda", dtype=bf)
-        self.h_out_p = torch.empty(self.out_p.shape, dtype=bf).pin_memory()
-        self.h_out_d = torch.empty(self.out_d.shape, dtype=bf).pin_memory()
+        self.out = torch.empty(self.S, wl.B, wl.H, wl.d_h, device="cuda", dtype=bf)
+        self.h_out = torch.empty(self.out.shape, dtype=bf).pin_memory()
         self.h2d_bytes = sum(v.numel() * v.element_size() for v in self.h.values())
-        self.d2h_bytes = (self.out_p.numel() + self.out_d.numel()) * 2
-        self.tokens_per_step = wl.B * (self.T + self.S)
-        # device input/output sets: set 1 (added by add_set) lets the end-to-end
-        # loop copy one step's inputs while the other set's step computes
-        self.sets = [(self.d, self.out_p, self.out_d)]
+        self.d2h_bytes = self.out.numel() * 2
+        self.tokens_per_step = wl.B * self.S
+        self.slots = [(self.N0 + k) // wl.s + 1 for k in range(self.S)]
+        self.slot_bytes = wl.D * 2
+        self.bytes_per_step = wl.B * self.slot_bytes * sum(self.slots)
+        self.sets = [(self.d, self.out)]
 
     def add_set(self):
-        d = {k: torch.empty_like(v) for k, v in self.d.items()}
-        self.sets.append((d, torch.empty_like(self.out_p), torch.empty_like(self.out_d)))
+        self.sets.append(({k: torch.empty_like(v) for k, v in self.d.items()},
+                          torch.empty_like(self.out)))
 
     def use(self, j: int):
-        self.d, self.out_p, self.out_d = self.sets[j]
-
-    def prefill(self):
-        b = self.buf
-        mtla.prefill(self.cfg, self.T, self.d["c"], self.d["kr"], self.d["qc"], self.d["qr"],
-                     b.w_uk, b.w_uv, b.gate_w, b.gate_b, None, self.out_p, b.cache, b.open_slot,
-                     b.workspace)
+        self.d, self.out = self.sets[j]
 
     def decode(self, k: int):
         b, d = self.buf, self.d
-        mtla.decode_step(self.cfg, d["d_c"][k], d["d_kr"][k], d["d_qc"][k], d["d_qr"][k], b.w_uk,
-                         b.w_uv, b.gate_w, b.gate_b, None, self.pos[k], b.cache, b.open_slot,
-                         self.out_d[k], b.workspace)
+        mtla.decode_step(self.cfg, d["c"][k], d["kr"][k], d["qc"][k], d["qr"][k], b.w_uk, b.w_uv,
+                         None, None, d["gate_in"][k], d["pos"][k], b.cache, b.open_slot,
+                         self.out[k], b.workspace)
 
-    def step(self, ev=None):
-        self.prefill()
-        if ev is not None:
-            ev.record()
+    def step(self):
         for k in range(self.S):
             self.decode(k)
 
-    def slots_read_per_decode(self):
-        """Slots the k-th decode step attends per sequence: floor(t/s) + 1."""
-        return [(self.T + k) // self.wl.s + 1 for k in range(self.S)]
+
+def _capture(fn, stream):
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    return g
 
 
-def _cpu_step():
-    """The float64 oracle on one whole step of this workload for one replica:
-    the parallel prefill of the 1024-token prefix of all 16 sequences, then the
-    256 incremental decode steps from the oracle's own cache.
-    Returns (tokens, seconds, threads)."""
-    import numpy as np
+def measure_contract(args, ws, rank):
+    """The large-latent decode: device-timed steps, the profiled attention
+    launches, and the end-to-end pipeline with host buffers."""
+    rep = LargeLatentReplica(rank)
+    flush = L2Flush()
+    st = torch.cuda.current_stream()
+    rep.step()                                     # eager warm-up, sets up per-device state
+    torch.cuda.synchronize()
+    assert mtla.get_device_status() == mtla.OK
 
-    import oracle
-    wl = WL
-    w = inputs.weights(wl)
-    pre = inputs.tokens(wl, wl.T, stream=0)
-    dec = inputs.tokens(wl, wl.steps, stream=1)
-    cfg = oracle.Cfg(wl.B, wl.H, wl.d_h, wl.d_c, wl.d_r, wl.s, gate_mode=wl.gate_mode)
-    oracle.build()
-    t0 = time.perf_counter()
-    r = oracle.prefill(cfg, pre["c"], pre["kr"], pre["qc"], pre["qr"], w["w_uk"], w["w_uv"],
-                       w["gate_w"], w["gate_b"])
-    max_slots = (wl.T + wl.steps + wl.s - 1) // wl.s
-    cache = np.zeros((wl.B, max_slots, wl.D))
-    cache[:, : r["cache"].shape[1]] = r["cache"]
-    acc = r["acc"].copy()
-    for k in range(wl.steps):
-        oracle.decode_step(cfg, dec["c"][:, k], dec["kr"][:, k], dec["qc"][:, k], dec["qr"][:, k],
-                           w["w_uk"], w["w_uv"], np.full(wl.B, wl.T + k), cache, acc,
-                           w["gate_w"], w["gate_b"])
-    dt = time.perf_counter() - t0
-    threads = int(os.environ.get("OMP_NUM_THREADS", "0")) or len(os.sched_getaffinity(0))
-    return wl.B * (wl.T + wl.steps), dt, threads
+    cap = torch.cuda.Stream()
+    cap.wait_stream(st)
+    n0 = mtla.kernel_launches()
+    g0 = _capture(rep.step, cap)
+    kernels_per_step = mtla.kernel_launches() - n0
+    prof = mtla.ProfileEvents(rep.S)
+    with prof:
+        g_prof = _capture(rep.step, cap)
+    rep.add_set()
+    rep.use(1)
+    g1 = _capture(rep.step, cap)
+    rep.use(0)
+    st.wait_stream(cap)
+    graphs = (g0, g1)
+
+    for i in range(args.warmup):
+        flush()
+        graphs[i & 1].replay()
+    flush()
+    g_prof.replay()
+    torch.cuda.synchronize()
+    assert mtla.get_device_status() == mtla.OK
+
+    # ---- device-timed steps
+    evs = _events(args.steps)
+    _barrier(ws)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for i in range(args.steps):
+            flush()
+            evs[i][0].record(st)
+            g0.replay()
+            evs[i][1].record(st)
+        torch.cuda.synchronize()
+    clocks = clk.summary()
+    _barrier(ws)
+    assert mtla.get_device_status() == mtla.OK
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    total_ms = _max_over_ranks(sum(step_ms), ws)
+    value = job_value(rep.bytes_per_step / 1e9, ws, args.steps, total_ms)
+    tokens_s = job_value(rep.tokens_per_step, ws, args.steps, total_ms)
+
+    # ---- dominant kernel: the decode attention, from the profiled replay
+    attn_ms = statistics.mean(prof.durations_ms())
+    hbm, _, peak_kind = _peaks()
+    attn_bytes = rep.bytes_per_step / rep.S
+    achieved = attn_bytes / (attn_ms / 1e3) / 1e9
+    traffic = _traffic("k_lh_attn", launch_scale=statistics.mean(rep.slots) / rep.max_slots)
+
+    # ---- end to end through the public API with host buffers
+    e2e_ms = _e2e(rep, graphs, flush, args.steps, ws)
+    e2e_value = job_value(rep.bytes_per_step / 1e9, ws, args.steps, e2e_ms)
+    wl = rep.wl
+    return {
+        "value": value, "ms_per_step": total_ms / args.steps, "clocks": clocks,
+        "gpu_launches": kernels_per_step * args.steps,
+        "decode": {"tokens_per_s": tokens_s,
+                   "ms_per_token_step": total_ms / args.steps / rep.S,
+                   "latent_cache_GBps": value, "slots_per_seq": [rep.slots[0], rep.slots[-1]],
+                   "kernels_per_token_step": kernels_per_step // rep.S},
+        "roofline": {"kernel": "k_lh_attn (decode attention)", "bound": "hbm",
+                     "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                     "traffic": traffic, "peak_source": f"{peak_kind} hbm_gbs (burst copy)",
+                     "bytes_per_launch": attn_bytes, "avg_launch_us": attn_ms * 1e3,
+                     "timing": f"CUDA event pairs recorded by the library around each of the "
+                               f"{rep.S} attention launches of one profiled replay of the step "
+                               f"(not counted in value)"},
+        "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": rep.h2d_bytes,
+                "d2h_bytes_per_step": rep.d2h_bytes,
+                "tokens_per_s": job_value(rep.tokens_per_step, ws, args.steps, e2e_ms),
+                "pipeline": "one timed region over all steps: inputs of step i+1 copied in "
+                            "(pinned, copy stream) while step i computes, outputs of step i "
+                            "copied out while step i+1 computes; L2 flush before each step "
+                            "inside the region"},
+        "config": {"workload": f"large_latent decode: B={wl.B}/rank, H={wl.H}, d_h={wl.d_h}, "
+                               f"d_c={wl.d_c}, d_R={wl.d_r}, s={wl.s}, supplied gates; "
+                               f"{rep.S} decode steps per sequence at positions "
+                               f"{rep.N0}..{wl.T - 1} ({rep.slots[0]}..{rep.slots[-1]} slots)",
+                   "global_batch": wl.B * ws, "seq_len": wl.T, "decode_steps_per_step": rep.S,
+                   "parallelism": f"replicas x{ws} (independent sequences)",
+                   "l2": "cache (604 MB) larger than L2; also " + L2Flush.desc + " step"},
+    }
 
 
-CPU_SAMPLE = ("one whole step of one replica: parallel prefill of the 1024-token prefix of all 16 "
-              "sequences + 256 incremental decode steps (float64 C oracle, OpenMP)")
+def _e2e(rep, graphs, flush, K, ws):
+    """One timed region over K steps: every step's inputs copied from pinned
+    host memory into one of two device sets and its outputs copied back, on a
+    copy stream, overlapping the neighbouring steps' compute."""
+    st = torch.cuda.current_stream()
+    cs = torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event(enable_timing=False)
+    e_beg, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    in_done, comp_done, out_done = [ev() for _ in range(K)], [ev() for _ in range(K)], [ev() for _ in range(K)]
+
+    def copy_in(i):
+        d = rep.sets[i & 1][0]
+        for k, v in rep.h.items():
+            d[k].copy_(v, non_blocking=True)
+        in_done[i].record(cs)
+
+    _barrier(ws)
+    torch.cuda.synchronize()
+    e_beg.record(st)
+    cs.wait_event(e_beg)
+    with torch.cuda.stream(cs):
+        copy_in(0)
+    for i in range(K):
+        j = i & 1
+        if i + 1 < K:
+            with torch.cuda.stream(cs):
+                if i >= 1:
+                    cs.wait_event(comp_done[i - 1])     # step i-1 read the set step i+1 uses
+                copy_in(i + 1)
+        if i >= 2:
+            st.wait_event(out_done[i - 2])               # outputs of step i-2 (same set) copied out
+        st.wait_event(in_done[i])
+        flush()
+        graphs[j].replay()
+        comp_done[i].record(st)
+        with torch.cuda.stream(cs):
+            cs.wait_event(comp_done[i])
+            rep.h_out.copy_(rep.sets[j][1], non_blocking=True)
+            out_done[i].record(cs)
+    st.wait_event(out_done[K - 1])
+    e_end.record(st)
+    torch.cuda.synchronize()
+    _barrier(ws)
+    assert mtla.get_device_status() == mtla.OK
+    return _max_over_ranks(e_beg.elapsed_time(e_end), ws)
 
 
-def _config(ws: int):
-    return {"workload": "speech_decode: B=16/rank, H=8, d_h=64, d_c=256, d_R=32, s=2; "
-                        "prefill 1024 tokens then 256 decode steps",
-            "global_batch": WL.B * ws, "prefix_tokens": WL.T, "decode_steps": WL.steps,
-            "seq_len": WL.T + WL.steps, "parallelism": f"replicas x{ws} (independent sequences)",
+# ------------------------------------------------------------- other workloads
+
+
+def _timed_calls(call, n, flush, ws, profile=True):
+    """n calls, each after an L2 flush, each between CUDA events; returns
+    (median call ms, median attention-kernel ms or None, clocks), the
+    medians taken as the max over ranks."""
+    st = torch.cuda.current_stream()
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    evs = _events(n)
+    prof = mtla.ProfileEvents(n) if profile else None
+    _barrier(ws)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        if prof:
+            prof.__enter__()
+        for i in range(n):
+            flush()
+            evs[i][0].record(st)
+            call()
+            evs[i][1].record(st)
+        torch.cuda.synchronize()
+        if prof:
+            prof.__exit__(None, None, None)
+    assert mtla.get_device_status() == mtla.OK
+    call_ms = _max_over_ranks(statistics.median(a.elapsed_time(b) for a, b in evs), ws)
+    kern_ms = _max_over_ranks(statistics.median(prof.durations_ms()), ws) if prof else None
+    return call_ms, kern_ms, clk.summary()
+
+
+def measure_prefill(n, flush, ws, rank):
+    """Parallel prefill B=8, T=8192, s=2: the block-prefix scan and the
+    stride-aware masked attention with absorption on both sides."""
+    _, tflops_peak, peak_kind = _peaks()
+    wl = inputs.PREFILL.with_(seed=inputs.PREFILL.seed + 1000 * rank)
+    T = wl.T
+    cfg = mtla.make_config(wl.B, wl.H, wl.d_h, wl.d_c, wl.d_r, wl.s, (T + wl.s - 1) // wl.s,
+                           dtype=wl.dtype, gate_mode=wl.gate_mode)
+    buf = mtla.Buffers.allocate(cfg, inputs.weights(wl), max_tokens=T)
+    tk = inputs.tokens(wl, T)
+    d = {k: tk[k].to("cuda", torch.bfloat16).contiguous() for k in ("c", "kr", "qc", "qr")}
+    out = torch.empty(wl.B, T, wl.H, wl.d_h, device="cuda", dtype=torch.bfloat16)
+
+    def call():
+        mtla.prefill(cfg, T, d["c"], d["kr"], d["qc"], d["qr"], buf.w_uk, buf.w_uv, buf.gate_w,
+                     buf.gate_b, None, out, buf.cache, buf.open_slot, buf.workspace)
+    call_ms, kern_ms, clocks = _timed_calls(call, n, flush, ws)
+    pairs = sum(t // wl.s + 1 for t in range(T))
+    flops = 2 * pairs * (wl.D + wl.d_c) * wl.B * wl.H
+    kern = flops / (kern_ms / 1e3) / 1e12
+    return {"workload": f"prefill: B={wl.B}/rank, T={T}, H={wl.H}, d_h={wl.d_h}, d_c={wl.d_c}, "
+                        f"d_R={wl.d_r}, s={wl.s}, computed gates",
+            "TFLOPs": flops * ws / (call_ms / 1e3) / 1e12, "call_ms": call_ms,
+            "attention_flops_per_call": flops, "calls": n,
+            "roofline": {"kernel": "k_prefill_tc (masked attention with absorption)",
+                         "bound": "tensor", "achieved": kern, "peak": tflops_peak,
+                         "unit": "TFLOP/s", "frac": kern / tflops_peak,
+                         "traffic": _traffic("k_prefill_tc"),
+                         "peak_source": f"{peak_kind} bf16_tflops (burst)",
+                         "avg_launch_us": kern_ms * 1e3},
+            "clocks": clocks, "l2": L2Flush.desc + " call"}
+
+
+def measure_speech(n, flush, ws, rank):
+    """Speech-model-scale decode B=16, H=8, s=2: a 1024-token prefix by the
+    prefill, then 256 decode steps (513..640 slots), as two CUDA graphs."""
+    wl = inputs.SPEECH_DECODE.with_(seed=inputs.SPEECH_DECODE.seed + 1000 * rank)
+    T, S = wl.T, wl.steps
+    max_slots = (T + S + wl.s - 1) // wl.s
+    cfg = mtla.make_config(wl.B, wl.H, wl.d_h, wl.d_c, wl.d_r, wl.s, max_slots, dtype=wl.dtype,
+                           gate_mode=wl.gate_mode)
+    buf = mtla.Buffers.allocate(cfg, inputs.weights(wl), max_tokens=T)
+    bf = torch.bfloat16
+    pre = inputs.tokens(wl, T, stream=0)
+    dec = inputs.tokens(wl, S, stream=1)
+    dp = {k: pre[k].to("cuda", bf).contiguous() for k in ("c", "kr", "qc", "qr")}
+    dd = {k: dec[k].transpose(0, 1).to("cuda", bf).contiguous() for k in ("c", "kr", "qc", "qr")}
+    pos = (T + torch.arange(S, dtype=torch.int32)).repeat_interleave(wl.B).view(S, wl.B).cuda()
+    out_p = torch.empty(wl.B, T, wl.H, wl.d_h, device="cuda", dtype=bf)
+    out_d = torch.empty(S, wl.B, wl.H, wl.d_h, device="cuda", dtype=bf)
+
+    def prefill():
+        mtla.prefill(cfg, T, dp["c"], dp["kr"], dp["qc"], dp["qr"], buf.w_uk, buf.w_uv,
+                     buf.gate_w, buf.gate_b, None, out_p, buf.cache, buf.open_slot, buf.workspace)
+
+    def decode():
+        for k in range(S):
+            mtla.decode_step(cfg, dd["c"][k], dd["kr"][k], dd["qc"][k], dd["qr"][k], buf.w_uk,
+                             buf.w_uv, buf.gate_w, buf.gate_b, None, pos[k], buf.cache,
+                             buf.open_slot, out_d[k], buf.workspace)
+    st = torch.cuda.current_stream()
+    prefill()
+    decode()
+    torch.cuda.synchronize()
+    cap = torch.cuda.Stream()
+    cap.wait_stream(st)
+    g_pre, g_dec = _capture(prefill, cap), _capture(decode, cap)
+    prof = mtla.ProfileEvents(S)
+    with prof:
+        g_prof = _capture(decode, cap)
+    st.wait_stream(cap)
+    for _ in range(3):
+        flush()
+        g_pre.replay()
+        g_dec.replay()
+    flush()
+    g_pre.replay()
+    g_prof.replay()
+    torch.cuda.synchronize()
+    evs = _events(n, 3)
+    _barrier(ws)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for i in range(n):
+            flush()
+            evs[i][0].record(st)
+            g_pre.replay()
+            evs[i][1].record(st)
+            g_dec.replay()
+            evs[i][2].record(st)
+        torch.cuda.synchronize()
+    assert mtla.get_device_status() == mtla.OK
+    pre_ms = _max_over_ranks(sum(a.elapsed_time(b) for a, b, c in evs), ws)
+    dec_ms = _max_over_ranks(sum(b.elapsed_time(c) for a, b, c in evs), ws)
+    slots = [(T + k) // wl.s + 1 for k in range(S)]
+    hbm, _, peak_kind = _peaks()
+    attn_ms = statistics.mean(prof.durations_ms())
+    attn_bytes = wl.B * wl.D * 2 * statistics.mean(slots)
+    return {"workload": f"speech_decode: B={wl.B}/rank, H={wl.H}, d_h={wl.d_h}, d_c={wl.d_c}, "
+                        f"d_R={wl.d_r}, s={wl.s}; prefill {T} tokens then {S} decode steps",
+            "decode_tokens_per_s": wl.B * S * ws * n / (dec_ms / 1e3),
+            "ms_per_token_step": dec_ms / n / S,
+            "decode_latent_cache_GBps": wl.B * wl.D * 2 * sum(slots) * ws * n / (dec_ms / 1e3) / 1e9,
+            "prefix_prefill_ms": pre_ms / n,
+            "prefix_tokens_per_s": wl.B * T * ws * n / (pre_ms / 1e3),
+            "steps": n, "slots_per_seq": [slots[0], slots[-1]],
+            "roofline": {"kernel": "k_dec_attn_sh (decode attention)", "bound": "hbm",
+                         "achieved": attn_bytes / (attn_ms / 1e3) / 1e9, "peak": hbm,
+                         "unit": "GB/s", "frac": attn_bytes / (attn_ms / 1e3) / 1e9 / hbm,
+                         "traffic": _traffic("k_dec_attn_sh"),
+                         "peak_source": f"{peak_kind} hbm_gbs", "avg_launch_us": attn_ms * 1e3},
+            "clocks": clk.summary(), "cuda_graphs": "prefill graph + 256-step decode graph",
             "l2": L2Flush.desc + " step"}
 
 
+def _decode_call(wl, N, max_slots=None):
+    """A decode step at position N-1 over a cache drawn directly (N-1 tokens)."""
+    max_slots = max_slots or (N + wl.s - 1) // wl.s
+    cfg = mtla.make_config(wl.B, wl.H, wl.d_h, wl.d_c, wl.d_r, wl.s, max_slots, dtype=wl.dtype,
+                           gate_mode=wl.gate_mode)
+    buf = mtla.Buffers.allocate(cfg, inputs.weights(wl))
+    c0 = inputs.synthetic_cache(wl, N - 1, max_slots)
+    buf.cache.copy_(c0["cache"].to(torch.bfloat16))
+    buf.open_slot.copy_(c0["acc"])
+    del c0
+    tk = inputs.tokens(wl, 1, stream=1)
+    d = {k: (None if v is None else
+             v[:, 0].to("cuda", torch.bfloat16 if k != "gate_in" else torch.float32).contiguous())
+         for k, v in tk.items()}
+    pos = torch.full((wl.B,), N - 1, dtype=torch.int32, device="cuda")
+    out = torch.empty(wl.B, wl.H, wl.d_h, device="cuda", dtype=torch.bfloat16)
+    gw, gb = (buf.gate_w, buf.gate_b) if wl.gate_mode == inputs.GATE_COMPUTED else (None, None)
+
+    def call():
+        mtla.decode_step(cfg, d["c"], d["kr"], d["qc"], d["qr"], buf.w_uk, buf.w_uv, gw, gb,
+                         d["gate_in"], pos, buf.cache, buf.open_slot, out, buf.workspace)
+    nbytes = wl.B * ((N - 1) // wl.s + 1) * wl.D * 2
+    return call, nbytes
+
+
+def measure_stride(n, flush, ws, rank):
+    """Stride sweep B=64, H=8, N=4096, s=1..4: one decode step at position
+    4095 over a cache of 4095 tokens (s=3: the last slot holds one token)."""
+    hbm, _, peak_kind = _peaks()
+    res = {"workload": "stride_sweep: B=64/rank, H=8, d_h=64, d_c=256, d_R=32, N=4096, "
+                       "one decode step at position 4095", "per_s": {}}
+    for s in (1, 2, 3, 4):
+        wl = inputs.STRIDE_SWEEP.with_(s=s, seed=inputs.STRIDE_SWEEP.seed + 1000 * rank)
+        call, nbytes = _decode_call(wl, wl.T)
+        call_ms, kern_ms, clocks = _timed_calls(call, n, flush, ws)
+        kern = nbytes / (kern_ms / 1e3) / 1e9
+        res["per_s"][str(s)] = {
+            "latent_cache_bytes": nbytes, "call_us": call_ms * 1e3,
+            "call_GBps": nbytes * ws / (call_ms / 1e3) / 1e9,
+            "roofline": {"kernel": "k_dec_attn_sh", "bound": "hbm", "achieved": kern, "peak": hbm,
+                         "unit": "GB/s", "frac": kern / hbm, "avg_launch_us": kern_ms * 1e3,
+                         "peak_source": f"{peak_kind} hbm_gbs"},
+            "clocks": clocks}
+        torch.cuda.empty_cache()
+    res["l2"] = L2Flush.desc + " call"
+    return res
+
+
+# ------------------------------------------------------------------ CPU oracle
+
+
+_CPU_DATA = {}
+
+
+def _cpu_sample(n_seq: int, min_s: float = 0.0, max_reps: int = 1):
+    """The float64 oracle on one decode step (position 65535, 16384 slots) of
+    `n_seq` sequences of the contract workload, repeated until `min_s` seconds
+    or `max_reps` calls. Returns (latent-cache bytes, seconds, threads, reps)."""
+    import numpy as np
+
+    import oracle
+    wl = WL.with_(B=n_seq)
+    N = wl.T
+    max_slots = (N + wl.s - 1) // wl.s
+    if n_seq not in _CPU_DATA:
+        c0 = inputs.synthetic_cache(wl, N - 1, max_slots)
+        _CPU_DATA[n_seq] = (inputs.weights(wl), inputs.tokens(wl, 1, stream=1),
+                            c0["cache"].double().numpy(), c0["acc"].double().numpy())
+        oracle.build()
+    w, tk, cache0, acc0 = _CPU_DATA[n_seq]
+    cfg = oracle.Cfg(wl.B, wl.H, wl.d_h, wl.d_c, wl.d_r, wl.s, gate_mode=wl.gate_mode)
+    reps, dt = 0, 0.0
+    while reps < max_reps and (reps == 0 or dt < min_s):
+        cache, acc = cache0.copy(), acc0.copy()
+        t0 = time.perf_counter()
+        oracle.decode_step(cfg, tk["c"][:, 0], tk["kr"][:, 0], tk["qc"][:, 0], tk["qr"][:, 0],
+                           w["w_uk"], w["w_uv"], np.full(wl.B, N - 1), cache, acc,
+                           gate_in=tk["gate_in"][:, 0])
+        dt += time.perf_counter() - t0
+        reps += 1
+    threads = int(os.environ.get("OMP_NUM_THREADS", "0")) or len(os.sched_getaffinity(0))
+    return wl.B * max_slots * wl.D * 2 * reps, dt, threads, reps
+
+
 def run_reference(args, ws, rank):
+    """The oracle arm: each step one oracle decode step of 2 of the 32
+    sequences at full length, in the contract line's unit (latent-cache GB/s)."""
     if rank != 0:
         return
-    times, toks, threads = [], 0, 1
+    n_seq = 2
+    times, nbytes, threads = [], 0, 1
     for i in range(args.warmup + args.steps):
-        n, dt, threads = _cpu_step()
+        b, dt, threads, _ = _cpu_sample(n_seq)
         if i >= args.warmup:
             times.append(dt)
-            toks += n
+            nbytes += b
     total = sum(times)
-    value = toks / total
+    value = nbytes / total / 1e9
+    wl = WL
+    sample = (f"one decode step (position {wl.T - 1}, {wl.T // wl.s} slots) of {n_seq} of the "
+              f"{wl.B} sequences per step, float64 C oracle with OpenMP over (sequence, head)")
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": _config(ws),
-        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                         "sample": CPU_SAMPLE},
-        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"large_latent decode: B={wl.B}, H={wl.H}, d_h={wl.d_h}, "
+                               f"d_c={wl.d_c}, d_R={wl.d_r}, s={wl.s}, supplied gates "
+                               f"(oracle sample: {n_seq} sequences per step)"},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------- kernel lines
 
 
 def run_reorder_workload(args):
@@ -336,23 +699,10 @@ def run_reorder_workload(args):
     n_tok = torch.full((B,), N, dtype=torch.int32, device="cuda")
     nbytes = 2 * (B * max_slots * cfg.D * 2 + B * cfg.D * 4)
     flush = L2Flush()
-    st = torch.cuda.current_stream()
 
     def call():
         mtla.reorder_cache(cfg, src, n_tok, cache_in, open_in, cache_out, open_out)
-    for _ in range(args.warmup):
-        call()
-    torch.cuda.synchronize()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    with ClockSampler(torch.cuda.current_device()) as clk:
-        for i in range(args.steps):
-            flush()
-            ev[i][0].record(st)
-            call()
-            ev[i][1].record(st)
-        torch.cuda.synchronize()
-    assert mtla.get_device_status() == mtla.OK
-    ms = statistics.median(a.elapsed_time(b) for a, b in ev)
+    ms, _, clocks = _timed_calls(call, args.steps, flush, 1, profile=False)
     achieved = nbytes / (ms / 1e3) / 1e9
     cpu = None
     if not args.no_cpu_baseline:
@@ -372,303 +722,102 @@ def run_reorder_workload(args):
             "roofline": {"kernel": "k_reorder_cache", "bound": "hbm", "achieved": achieved, "peak": hbm,
                          "unit": "GB/s", "frac": achieved / hbm, "bytes_per_launch": nbytes,
                          "peak_source": f"{peak_kind} hbm_gbs"},
-            "cpu_baseline": cpu, "clocks": clk.summary(), "l2": L2Flush.desc + " call"}
+            "cpu_baseline": cpu, "clocks": clocks, "l2": L2Flush.desc + " call"}
     print(json.dumps(line), flush=True)
 
 
-def run_kernel_workload(args, ws, rank):
-    """Kernel-level measurement of one of the other workloads (not the contract
-    line): decode attention GB/s against the measured HBM copy bandwidth, or
-    prefill TFLOP/s against the measured bf16 peak. L2 flushed before every
-    timed call; each call bracketed by CUDA events on the launching stream."""
-    hbm, tflops_peak, peak_kind = _peaks()
+def run_kernel_workload(args):
+    """Kernel-level line of one workload (not the contract line), for profiling
+    runs: decode attention GB/s or prefill TFLOP/s against the measured peaks."""
     flush = L2Flush()
-    st = torch.cuda.current_stream()
     name = args.workload
+    if name.startswith("prefill"):
+        print(json.dumps(measure_prefill(args.steps, flush, 1, 0)), flush=True)
+        return
+    if name.startswith("speech_decode"):
+        print(json.dumps(measure_speech(args.steps, flush, 1, 0)), flush=True)
+        return
+    hbm, _, peak_kind = _peaks()
     wl = inputs.WORKLOADS[name.split(":")[0]]
     if ":" in name:
         wl = wl.with_(s=int(name.split(":")[1]))
-    w = inputs.weights(wl)
-    lines = []
-    if name.startswith("prefill"):
-        T = wl.T
-        cfg = mtla.make_config(wl.B, wl.H, wl.d_h, wl.d_c, wl.d_r, wl.s, (T + wl.s - 1) // wl.s,
-                               dtype=wl.dtype, gate_mode=wl.gate_mode)
-        buf = mtla.Buffers.allocate(cfg, w, max_tokens=T)
-        tk = inputs.tokens(wl, T)
-        d = {k: (None if v is None else v.to("cuda", torch.bfloat16).contiguous()) for k, v in tk.items()}
-        out = torch.empty(wl.B, T, wl.H, wl.d_h, device="cuda", dtype=torch.bfloat16)
-
-        def call():
-            mtla.prefill(cfg, T, d["c"], d["kr"], d["qc"], d["qr"], buf.w_uk, buf.w_uv, buf.gate_w,
-                         buf.gate_b, None, out, buf.cache, buf.open_slot, buf.workspace)
-        pairs = sum(t // wl.s + 1 for t in range(T))
-        flops = 2 * pairs * (wl.D + wl.d_c) * wl.B * wl.H
-        unit_fn = lambda ms: flops / (ms / 1e3) / 1e12
-        unit, peak, bound = "TFLOP/s", tflops_peak, "tensor"
-    else:
-        N = wl.T
-        max_slots = (N + wl.s - 1) // wl.s
-        cfg = mtla.make_config(wl.B, wl.H, wl.d_h, wl.d_c, wl.d_r, wl.s, max_slots, dtype=wl.dtype,
-                               gate_mode=wl.gate_mode)
-        buf = mtla.Buffers.allocate(cfg, w)
-        c0 = inputs.synthetic_cache(wl, N - 1, max_slots)
-        buf.cache.copy_(c0["cache"].to(torch.bfloat16))
-        buf.open_slot.copy_(c0["acc"])
-        del c0
-        tk = inputs.tokens(wl, 1, stream=1)
-        d = {k: (None if v is None else v[:, 0].to("cuda", torch.bfloat16 if k != "gate_in" else torch.float32).contiguous())
-             for k, v in tk.items()}
-        pos = torch.full((wl.B,), N - 1, dtype=torch.int32, device="cuda")
-        out = torch.empty(wl.B, wl.H, wl.d_h, device="cuda", dtype=torch.bfloat16)
-        gw, gb = (buf.gate_w, buf.gate_b) if wl.gate_mode == inputs.GATE_COMPUTED else (None, None)
-
-        def call():
-            mtla.decode_step(cfg, d["c"], d["kr"], d["qc"], d["qr"], buf.w_uk, buf.w_uv, gw, gb,
-                             d["gate_in"], pos, buf.cache, buf.open_slot, out, buf.workspace)
-        nbytes = wl.B * max_slots * wl.D * 2
-        unit_fn = lambda ms: nbytes / (ms / 1e3) / 1e9
-        unit, peak, bound = "GB/s", hbm, "hbm"
-    for _ in range(args.warmup):
-        call()
-    torch.cuda.synchronize()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    prof = mtla.ProfileEvents(args.steps)
-    with ClockSampler(torch.cuda.current_device()) as clk, prof:
-        for i in range(args.steps):
-            flush()
-            ev[i][0].record(st)
-            call()
-            ev[i][1].record(st)
-        torch.cuda.synchronize()
-    assert mtla.get_device_status() == mtla.OK
-    call_ms = statistics.median(a.elapsed_time(b_) for a, b_ in ev)
-    kern_ms = statistics.median(prof.durations_ms())
-    line = {"workload": name, "config": {"B": wl.B, "H": wl.H, "d_h": wl.d_h, "d_c": wl.d_c,
-                                         "d_R": wl.d_r, "s": wl.s, "T_or_N": wl.T},
-            "call_ms": call_ms, "attention_kernel_ms": kern_ms,
-            "call": {"value": unit_fn(call_ms), "unit": unit},
-            "roofline": {"kernel": "attention", "bound": bound, "achieved": unit_fn(kern_ms),
-                         "peak": peak, "unit": unit, "frac": unit_fn(kern_ms) / peak,
-                         "peak_source": f"{peak_kind} " + ("hbm_gbs" if bound == "hbm" else "bf16_tflops")},
-            "clocks": clk.summary(), "l2": L2Flush.desc + " call"}
-    print(json.dumps(line), flush=True)
+    call, nbytes = _decode_call(wl, wl.T)
+    call_ms, kern_ms, clocks = _timed_calls(call, args.steps, flush, 1)
+    kern = nbytes / (kern_ms / 1e3) / 1e9
+    print(json.dumps({"workload": name, "config": {"B": wl.B, "H": wl.H, "d_h": wl.d_h,
+                                                   "d_c": wl.d_c, "d_R": wl.d_r, "s": wl.s,
+                                                   "N": wl.T},
+                      "call_ms": call_ms, "attention_kernel_ms": kern_ms,
+                      "call": {"value": nbytes / (call_ms / 1e3) / 1e9, "unit": "GB/s"},
+                      "roofline": {"kernel": "decode attention", "bound": "hbm", "achieved": kern,
+                                   "peak": hbm, "unit": "GB/s", "frac": kern / hbm,
+                                   "peak_source": f"{peak_kind} hbm_gbs"},
+                      "clocks": clocks, "l2": L2Flush.desc + " call"}), flush=True)
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=60)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="mtla", choices=["mtla", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="speech_decode",
-                    help="speech_decode (the contract line) or a kernel-level measurement of "
-                         "stride_sweep[:s], prefill, large_latent or beam_reorder")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="contract line only (no prefill / speech / stride-sweep sub-objects)")
+    ap.add_argument("--workload", default="large_latent",
+                    help="large_latent (the contract line), or a kernel-level line of "
+                         "stride_sweep[:s], prefill, speech_decode or beam_reorder")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     ws, rank = _dist()
-    if args.workload == "beam_reorder":
-        if rank == 0:
-            run_reorder_workload(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, ws, rank)
+        elif args.workload == "beam_reorder":
+            if rank == 0:
+                run_reorder_workload(args)
+        elif args.workload != "large_latent":
+            if rank == 0:
+                run_kernel_workload(args)
+        else:
+            run_contract(args, ws, rank)
+    finally:
         if ws > 1:
             torch.distributed.destroy_process_group()
-        return
-    if args.workload != "speech_decode":
-        if rank == 0:
-            run_kernel_workload(args, ws, rank)
-        if ws > 1:
-            torch.distributed.destroy_process_group()
-        return
-    if args.impl == "reference":
-        run_reference(args, ws, rank)
-        if ws > 1:
-            torch.distributed.destroy_process_group()
-        return
 
-    rep = Replica(rank)
-    flush = L2Flush()
-    st = torch.cuda.current_stream()
 
-    # eager warm-up (also sets up every per-device cache inside the library)
-    rep.step()
-    torch.cuda.synchronize()
-    assert mtla.get_device_status() == mtla.OK
-
-    # the step as two CUDA graphs (prefill; 256 decode steps), captured through
-    # the public API. A third graph -- the decode steps again, with the event
-    # pairs the library records around each attention launch as graph nodes --
-    # is replayed once inside the timed region for the kernel's own time (the
-    # event nodes would otherwise sit between the step's kernels).
-    g_pre, g_dec, g_prof = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-    cap = torch.cuda.Stream()
-    cap.wait_stream(st)
-    n0 = mtla.kernel_launches()
-    with torch.cuda.graph(g_pre, stream=cap):
-        rep.prefill()
-    with torch.cuda.graph(g_dec, stream=cap):
-        for k in range(rep.S):
-            rep.decode(k)
-    kernels_per_step = mtla.kernel_launches() - n0
-    prof = mtla.ProfileEvents(1 + rep.S)
-    with prof:
-        with torch.cuda.graph(g_prof, stream=cap):
-            rep.prefill()
-            for k in range(rep.S):
-                rep.decode(k)
-    # the same step on input/output set 1, for the end-to-end pipeline
-    rep.add_set()
-    rep.use(1)
-    g_pre1, g_dec1 = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_pre1, stream=cap):
-        rep.prefill()
-    with torch.cuda.graph(g_dec1, stream=cap):
-        for k in range(rep.S):
-            rep.decode(k)
-    rep.use(0)
-    st.wait_stream(cap)
-
-    def step(j=0):
-        (g_pre, g_pre1)[j].replay()
-        (g_dec, g_dec1)[j].replay()
-
-    for i in range(args.warmup):
-        step(i & 1)
-    g_prof.replay()
-    torch.cuda.synchronize()
-    assert mtla.get_device_status() == mtla.OK
-
-    # ---- device-timed steps
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-            torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    _barrier(ws)
-    with ClockSampler(torch.cuda.current_device()) as clk:
-        for i in range(args.steps):
-            flush()
-            evs[i][0].record(st)
-            g_pre.replay()
-            evs[i][1].record(st)
-            g_dec.replay()
-            evs[i][2].record(st)
-        flush()
-        g_prof.replay()
-        torch.cuda.synchronize()
-    _barrier(ws)
-    launches = kernels_per_step * args.steps
-    assert mtla.get_device_status() == mtla.OK
-    step_ms = [a.elapsed_time(c) for a, b, c in evs]
-    pre_ms = [a.elapsed_time(b) for a, b, c in evs]
-    dec_ms = [b.elapsed_time(c) for a, b, c in evs]
-    total_ms = _max_over_ranks(sum(step_ms), ws)
-    value = job_value(rep.tokens_per_step, ws, args.steps, total_ms)
-
-    # dominant kernel: decode attention, from the profiled replay's event pairs
-    durs = prof.durations_ms()
-    attn = durs[1:]
-    pre_attn = durs[:1]
-    slot_bytes = rep.wl.D * 2
-    slots = rep.slots_read_per_decode()
-    bytes_per_launch = rep.wl.B * slot_bytes * sum(slots) / len(slots)
-    attn_ms = statistics.mean(attn)
-    hbm, tflops_peak, peak_kind = _peaks()
-    achieved = bytes_per_launch / (attn_ms / 1e3) / 1e9
-    # prefill attention flops: 2 * allowed pairs * (D + d_c) * B * H
-    wl = rep.wl
-    pairs = sum(t // wl.s + 1 for t in range(rep.T))
-    pre_flops = 2 * pairs * (wl.D + wl.d_c) * wl.B * wl.H
-    dec_tokens = wl.B * rep.S
-    dec_s = _max_over_ranks(sum(dec_ms), ws) / 1e3
-
-    # ---- end to end through the public API with host buffers: one timed region
-    # over all steps. Every step's inputs are copied from pinned host memory and
-    # its outputs copied back inside it, on a copy stream: the inputs of step
-    # i+1 (into the other device set) while step i computes, the outputs of
-    # step i while step i+1 computes; the first copy in and the last copy out
-    # are not overlapped. The L2 flush before each step is inside the region.
-    cs = torch.cuda.Stream()
-    ev = lambda: torch.cuda.Event(enable_timing=False)
-    e_beg, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    K = args.steps
-    in_done, comp_done, out_done = [ev() for _ in range(K)], [ev() for _ in range(K)], [ev() for _ in range(K)]
-
-    def copy_in(i):
-        d = rep.sets[i & 1][0]
-        for k, v in rep.h.items():
-            d[k].copy_(v, non_blocking=True)
-        in_done[i].record(cs)
-
-    _barrier(ws)
-    torch.cuda.synchronize()
-    e_beg.record(st)
-    cs.wait_event(e_beg)
-    with torch.cuda.stream(cs):
-        copy_in(0)
-    for i in range(K):
-        j = i & 1
-        if i + 1 < K:
-            with torch.cuda.stream(cs):
-                if i >= 1:
-                    cs.wait_event(comp_done[i - 1])     # step i-1 read the set step i+1 uses
-                copy_in(i + 1)
-        if i >= 2:
-            st.wait_event(out_done[i - 2])               # outputs of step i-2 (same set) copied out
-        st.wait_event(in_done[i])
-        flush()
-        step(j)
-        comp_done[i].record(st)
-        with torch.cuda.stream(cs):
-            cs.wait_event(comp_done[i])
-            _, out_p, out_d = rep.sets[j]
-            rep.h_out_p.copy_(out_p, non_blocking=True)
-            rep.h_out_d.copy_(out_d, non_blocking=True)
-            out_done[i].record(cs)
-    st.wait_event(out_done[K - 1])
-    e_end.record(st)
-    torch.cuda.synchronize()
-    _barrier(ws)
-    e2e_ms = _max_over_ranks(e_beg.elapsed_time(e_end), ws)
-    e2e_value = rep.tokens_per_step * ws * K / (e2e_ms / 1e3)
-
+def run_contract(args, ws, rank):
+    res = measure_contract(args, ws, rank)
+    torch.cuda.empty_cache()
+    extras = {}
+    if not args.no_extras:
+        flush = L2Flush()
+        extras["prefill"] = measure_prefill(900, flush, ws, rank)
+        torch.cuda.empty_cache()
+        extras["speech_decode"] = measure_speech(320, flush, ws, rank)
+        torch.cuda.empty_cache()
+        extras["stride_sweep"] = measure_stride(6000, flush, ws, rank)
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        n, dt, threads = _cpu_step()
-        cpu = {"value": n / dt, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-               "sample": CPU_SAMPLE + f" ({dt:.1f} s)"}
-
+        n_seq = 8
+        b, dt, threads, reps = _cpu_sample(n_seq, min_s=10.0, max_reps=4)
+        cpu = {"value": b / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+               "sample": f"{reps} x one decode step (position {WL.T - 1}, {WL.T // WL.s} slots) "
+                         f"of {n_seq} of the {WL.B} sequences, float64 C oracle with OpenMP "
+                         f"over (sequence, head) ({dt:.1f} s)"}
     if rank == 0:
         line = {
-            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+            "metric": METRIC, "value": res["value"], "unit": "GB/s", "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": res["ms_per_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic (seeded N(0,1) inputs, random-init weights)",
-            "config": _config(ws),
-            "decode": {"tokens_per_s": dec_tokens * ws * args.steps / dec_s,
-                       "ms_per_token_step": 1e3 * dec_s / (rep.S * args.steps),
-                       "latent_cache_GBps": wl.B * slot_bytes * sum(slots) * args.steps / dec_s / 1e9,
-                       "slots_per_seq": [slots[0], slots[-1]]},
-            "prefill": {"ms": statistics.mean(pre_ms), "attention_kernel_ms": statistics.mean(pre_attn),
-                        "TFLOPs": pre_flops / (statistics.mean(pre_ms) / 1e3) / 1e12},
-            "roofline": {"kernel": "decode attention", "bound": "hbm", "achieved": achieved,
-                         "peak": hbm, "unit": "GB/s", "frac": achieved / hbm, "traffic": _traffic("k_dec_attn_sh"),
-                         "peak_source": f"{peak_kind} hbm_gbs",
-                         "bytes_per_launch": bytes_per_launch, "avg_launch_us": attn_ms * 1e3,
-                         "timing": "CUDA event pairs recorded by the library around each of the "
-                                   "256 decode attention launches of one profiled replay of the "
-                                   "step inside the timed region (not counted in value)"},
-            "cpu_baseline": cpu,
-            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": rep.h2d_bytes,
-                    "d2h_bytes_per_step": rep.d2h_bytes,
-                    "pipeline": "one timed region over all steps: inputs of step i+1 copied in "
-                                "(pinned, copy stream) while step i computes, outputs of step i "
-                                "copied out while step i+1 computes; L2 flush before each step "
-                                "inside the region"},
-            "gpu_launches": launches,
-            "cuda_graphs": "prefill graph + 256-step decode graph, replayed per step",
-            "clocks": clk.summary(),
+            "data": "synthetic (seeded N(0,1) inputs and cache, random-init weights)",
+            "config": res["config"], "decode": res["decode"], "roofline": res["roofline"],
+            "cpu_baseline": cpu, "e2e": res["e2e"], "gpu_launches": res["gpu_launches"],
+            "cuda_graphs": f"{GEN_STEPS} decode steps per graph, one replay per step",
+            "clocks": res["clocks"],
         }
+        line.update(extras)
         print(json.dumps(line), flush=True)
-    if ws > 1:
-        torch.distributed.destroy_process_group()
 
 
 if __name__ == "__main__":
