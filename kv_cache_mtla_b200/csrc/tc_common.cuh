@@ -34,14 +34,18 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                  : "memory");
 }
+// The suspend-time hint lets a waiting thread sleep until the phase completes
+// (or 1 ms passes) instead of polling the barrier, which would take shared
+// memory cycles from the TMA writes and the tensor cores.
+constexpr uint32_t kSuspendHintNs = 1000000;
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}\n"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendHintNs)
         : "memory");
     return ok != 0;
 }
@@ -66,7 +70,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
-        for (int i = 0; i < 64; ++i)
+        for (int i = 0; i < 8; ++i)
             if (mbar_try_wait(bar, parity)) return true;
         if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
     }
@@ -230,6 +234,15 @@ __device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const float* v) {
     for (int c = 0; c + 16 <= N; c += 16) tmem_st16(taddr + c, v + c);
     if (N % 16) tmem_st8(taddr + (N & ~15), v + (N & ~15));
 }
+// One 32-bit column of this thread's lane.
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, float v) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(__float_as_uint(v)) : "memory");
+}
+__device__ __forceinline__ float tmem_ld1(uint32_t taddr) {
+    uint32_t r;
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
+    return __uint_as_float(r);
+}
 // Maximum over the warp in one instruction (sm_100a); -inf stays -inf.
 __device__ __forceinline__ float warp_max_redux(float v) {
     float r;
@@ -288,6 +301,14 @@ __device__ __forceinline__ void st_cluster_u4(uint32_t addr, uint4 v) {
                  "r"(v.w)
                  : "memory");
 }
+__device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+// Make this thread's generic-proxy writes to shared memory anywhere in the
+// cluster visible to the async proxy (the tensor cores of the CTA that owns it).
+__device__ __forceinline__ void fence_proxy_async_cluster() {
+    asm volatile("fence.proxy.async.shared::cluster;" ::: "memory");
+}
 // Bulk copy from this CTA's shared memory to another CTA's shared memory in
 // the cluster (16-byte aligned, size a multiple of 16); the bytes complete on
 // the destination CTA's mbarrier `remote_bar` (a cluster address).
@@ -308,6 +329,20 @@ __device__ __forceinline__ void bulk_wait_read_all() {
 __device__ __forceinline__ void named_sync(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
+// Named barrier that also returns the AND of `pred` over the `count` threads,
+// so that they all take the same branch afterwards.
+__device__ __forceinline__ bool named_sync_and(int id, int count, bool pred) {
+    uint32_t out;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %3, 0;\n\t"
+        "bar.red.and.pred q, %1, %2, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}\n"
+        : "=r"(out)
+        : "r"(id), "r"(count), "r"((uint32_t)pred)
+        : "memory");
+    return out != 0;
+}
 // Arrive on an mbarrier of another CTA of the cluster without release
 // semantics: for signalling that reads (already consumed) are done.
 __device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t bar_cluster_addr) {
@@ -324,10 +359,10 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}\n"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendHintNs)
         : "memory");
     return ok != 0;
 }
@@ -335,7 +370,7 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity
     if (mbar_try_wait_cluster(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
-        for (int i = 0; i < 64; ++i)
+        for (int i = 0; i < 8; ++i)
             if (mbar_try_wait_cluster(bar, parity)) return true;
         if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
     }
@@ -417,6 +452,17 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                      smem_u32(bar))
                  : "memory");
+}
+
+// Arrive on the mbarrier at the same shared-memory offset as `bar` in every
+// CTA of the cluster named by `cta_mask`, once all previously issued
+// tcgen05.mma of this thread completed (a completion signal, not a load).
+__device__ __forceinline__ void umma_commit_to(uint64_t* bar, uint16_t cta_mask) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"(cta_mask)
+        : "memory");
 }
 
 // Byte offset of element (row, col) inside a K-major SW128 chunk of 64 bf16

@@ -7,15 +7,17 @@
 // latent cache is streamed once from HBM.
 //
 // The output accumulator O [128 heads x d_c] fp32 fills the whole tensor
-// memory at d_c = 512, so the work of a slot range is split over a cluster of
-// two CTAs by slot columns: CTA 0 holds latent columns [0, d_c/2) plus the
-// RoPE part, CTA 1 latent columns [d_c/2, d_c). Each CTA
-//   - loads only its columns of every 64-slot tile (TMA, no duplication),
-//   - computes its partial scores S_c = q~_c . K_c^T       (M=128, N=64),
-//   - sends S_c to the peer through distributed shared memory and adds the
-//     peer's part, so both hold S and run the same softmax (thread per head),
-//   - accumulates its half O_c += P . V_c                 (M=128, N=d_c/2),
-// Tensor memory per CTA: O_c (d_c/2 columns) + two S buffers (64 each).
+// memory at d_c = 512, so a cluster of two CTAs splits the work by role:
+//   - rank 0 holds the absorbed queries in tensor memory and computes the
+//     scores of every 128-slot tile over the whole slot width (M = 128 heads,
+//     N = 128 slots), runs the online softmax and writes P (bf16) straight
+//     into rank 1's shared memory;
+//   - rank 1 holds O and accumulates O += P . V over the latent columns
+//     (M = 128 heads, N = 256 columns), reading each tile a second time (from
+//     L2: the two CTAs stream the same tiles a few microseconds apart).
+// No partial scores are exchanged; the tensor pipes of the two CTAs take
+// about the same time per tile (36 score MMAs of N = 128 against 16 P.V MMAs
+// of N = 256).
 //
 // Launches per step:
 //   k_lh_prep      gate, RoPE and in-place slot update; absorbed queries for
@@ -42,11 +44,13 @@ namespace {
 
 using namespace tc;
 
-constexpr int kKT = 64;          // slots per key tile
-constexpr int kStages = 3;
-constexpr int kMaxSq = 4;         // query chunks in shared memory: at most 4 latent + 2 RoPE - 2 in TMEM
-constexpr int kThreads = 352;    // warp 0 TMA, 1 score MMAs, 2-9 softmax, 10 P.V MMAs
-constexpr int kMaxClusters = 80; // >= SMs/2 of any sm_100 part; sizes the partial buffer
+constexpr int kKT = 128;          // slots per tile
+constexpr int kHalf = 64;         // slots per half tile (one P buffer, one P.V block)
+constexpr int kMaxRing = 8;       // ring stages of either CTA
+constexpr int kMaxQChunks = 10;   // 64-column chunks of a slot (D <= 640)
+constexpr int kChunksPerStage = 3;  // 64-column chunks per score-ring stage (one TMA box)
+constexpr int kThreads = 320;     // warp 0 TMA, 1 MMA issue, 2-9 softmax / events
+constexpr int kMaxClusters = 80;  // >= SMs/2 of any sm_100 part; sizes the partial buffer
 constexpr int kMaxB = 2048;
 constexpr float kRescaleLog2 = 8.f;
 
@@ -54,10 +58,12 @@ struct LhArgs {
     int B, H, D, d_c, d_r, s, max_slots;
     int G2;                 // clusters in the grid
     int n_qchunks;          // D / 64
+    int unit_cols;          // latent columns per P.V MMA (N): min(256, d_c)
+    uint32_t smem_bytes;    // dynamic shared memory of the attention kernel
     float scale_log2;
     const int32_t* pos;
     const uint8_t* qimg;    // [B] x n_qchunks x [128 heads x 128 B]
-    float* part;            // [(kMaxClusters + B), H, d_c + 2]
+    float* part;            // [(kMaxClusters + B), H, d_c + 4]
     int* status;
 };
 
@@ -232,500 +238,553 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
 
 // ---------------------------------------------------------------- attention
 
-struct LhBars {
-    uint64_t full[kStages], empty[kStages];   // slot-tile ring
-    uint64_t q_full, q_free;                  // query image of the current segment
-    uint64_t s_full[2], s_empty[2];           // partial scores in TMEM, by tile parity
-    uint64_t p_full[2], o_done[2];            // P in TMEM; P.V of tiles with this parity completed
-    uint64_t x_full[2];                       // peer's partial scores landed in x_in[parity] (bulk copy)
-    uint64_t x_free[2];                       // peer has read the scores this CTA sent into its x_in[parity]
-    uint64_t qt_full;                         // query chunks of the segment written to TMEM (8 warps)
-    uint64_t drain[2];                        // MMAs in flight when a wait gave up (per issuing thread)
-    uint32_t tmem_base;
-    volatile int fail;
-    int total;
-    float red[2][2][128];                     // [tile parity][column half][row]: half-row maxima
-    float lsum[2][128];                       // [column half][row]: half-row sums at a segment end
+// Per-tile side information rank 0 sends with P half 0: the factor each row
+// of O must be scaled by before this tile adds to it (1 if none), and whether
+// any row of a TMEM lane quarter needs it.
+struct __align__(16) LhSide {
+    float fac[128];
+    int flag[4];
 };
 
-__device__ __forceinline__ bool lh_wait(uint64_t* bar, uint32_t parity, LhBars& bs) {
-    if (bs.fail) return false;
+// Shared-memory control block at the (1024-aligned) start of both CTAs' shared
+// memory. The barriers a peer arrives on and the side information sit at the
+// same offset in both CTAs.
+struct LhCtl {
+    uint64_t full[kMaxRing], empty[kMaxRing];   // this CTA's ring of landed tiles
+    uint64_t s_full, s_empty, qt_full;          // rank 0: scores in TMEM; query chunks in TMEM
+    uint64_t p_free[2];                         // rank 0: rank 1's P.V has read P half h
+    uint64_t p_full[2];                         // rank 1: P half h (and the side information) copied in
+    uint64_t o_done, ev_full, ev_done;          // rank 1: P.V complete; event posted / handled
+    uint64_t drain;                             // MMAs in flight when a wait gave up
+    uint32_t tmem_base;
+    volatile int fail;
+    int b0, j0, n_tiles;                        // the cluster's first tile and tile count
+    volatile int ev[2];                         // rank 1: event type and argument
+    volatile int ev_arg[2];
+    LhSide side;                                // rank 0: staged for the copy; rank 1: received
+};
+constexpr uint32_t kCtlBytes = 1024;
+static_assert(sizeof(LhCtl) <= kCtlBytes, "control block");
+
+enum { kEvEnd = 0, kEvRescale = 1, kEvZero = 2, kEvSegEnd = 3 };
+
+__device__ __forceinline__ bool lh_wait(uint64_t* bar, uint32_t parity, LhCtl& cs) {
+    if (cs.fail) return false;
     if (mbar_wait(bar, parity)) return true;
-    bs.fail = 1;
+    cs.fail = 1;
     return false;
 }
-__device__ __forceinline__ bool lh_wait_cluster(uint64_t* bar, uint32_t parity, LhBars& bs) {
-    if (bs.fail) return false;
+__device__ __forceinline__ bool lh_wait_cluster(uint64_t* bar, uint32_t parity, LhCtl& cs) {
+    if (cs.fail) return false;
     if (mbar_wait_cluster(bar, parity)) return true;
-    bs.fail = 1;
+    cs.fail = 1;
     return false;
 }
 
-// Chunk i of this CTA's slot columns -> 64-column chunk index of the slot.
-__device__ __forceinline__ int lh_chunk_id(int rank, int i, int lat_chunks, int rope_first) {
-    if (rank == 1) return lat_chunks + i;
-    return i < lat_chunks ? i : rope_first + (i - lat_chunks);
-}
+// Walk over the cluster's tiles in order: sequence b, tile j of nt, nb slots.
+struct LhWalk {
+    int b, j, nb, nt;
+    __device__ void start(const LhArgs& p, int b0, int j0) {
+        b = b0;
+        j = j0;
+        nb = b < p.B ? lh_slots(p, b) : 0;
+        nt = (nb + kKT - 1) / kKT;
+    }
+    __device__ void next(const LhArgs& p) {
+        if (++j < nt) return;
+        j = 0;
+        do {
+            ++b;
+            nb = b < p.B ? lh_slots(p, b) : 0;
+        } while (b < p.B && nb == 0);
+        nt = (nb + kKT - 1) / kKT;
+    }
+    __device__ bool last_of_seq() const { return j == nt - 1; }
+};
 
-// Exchange buffer: row r holds the 64 scaled partial scores of head r as fp16
-// (128 B), its 16-byte units XOR-swizzled by r mod 8 (conflict-free access).
-__device__ __forceinline__ uint32_t xoff(int r, int unit) { return (uint32_t)r * 128 + (((unit ^ r) & 7) << 4); }
-
-// Attention over 64-slot tiles for one cluster of two CTAs (see the top of the
-// file). Warp 0: TMA; warp 1: MMA issue and TMEM; warps 2-9: softmax, two
-// threads per head row (one per 32-slot half of a tile). The softmax of tile it
-// is split in two halves:
-//   A(it)  read this CTA's partial scores from TMEM, round them (scaled) to
-//          fp16 and send them to the peer (one bulk copy into its x_in);
-//   B(it)  add the peer's partial scores, online softmax, P into TMEM.
-// The order A(it+1), B(it) lets both copies of tile it+1 fly while the CTAs
-// do B(it). Scores, P and x_in are double-buffered; the ring has three stages.
+// Decode attention for one cluster of two CTAs over a contiguous range of
+// 128-slot tiles (the grid is balanced over all tiles of the batch):
+//   rank 0 (scorer): the absorbed queries of all heads in TMEM as the MMA's A
+//     operand; S = q~ K^T over the whole slot width (M = 128 heads, N = 128
+//     slots) from 64-column chunks of the tile streamed through a 14-stage
+//     ring; online softmax (two threads per head row, one per 64-slot half);
+//     P (bf16) written straight into rank 1's shared memory;
+//   rank 1 (accumulator): O [128 heads x d_c] fp32 in all of its TMEM;
+//     O += P V from the tile's latent columns (N = 256) streamed through its
+//     own ring (the second read of each tile, served by L2).
+// Warp 0: TMA; warp 1: MMA issue; warps 2-9: softmax (rank 0) or the event
+// handlers of rank 1 (rescale of O when a row's reference maximum moves,
+// zeroing of cache rows past a sequence's last slot, writing O at the end of a
+// sequence segment). One partial (O, m, l) per sequence segment.
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-    k_lh_attn(const __grid_constant__ CUtensorMap tmap, const LhArgs p) {
+    k_lh_attn(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v, const LhArgs p) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t* base = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    const uint32_t pad = (uint32_t)(base - smem_raw);
+    LhCtl& cs = *(LhCtl*)base;
+    uint8_t* region = base + kCtlBytes;
+    const uint32_t region_bytes = p.smem_bytes - pad - kCtlBytes;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int rank = (int)cluster_rank(), peer = rank ^ 1;
-    const int g = blockIdx.x >> 1;                       // cluster index
-    const int lat_half = p.d_c / 2, lat_chunks = lat_half / 64;
-    const int rope_first = p.d_c / 64;                   // first chunk of the RoPE columns
-    const int max_chunks = lat_chunks + (p.n_qchunks - rope_first);
-    const int my_chunks = rank == 0 ? max_chunks : lat_chunks;
-    // the last n_tq of this CTA's query chunks live in TMEM (the MMA's A from
-    // tensor memory), the first n_sq in shared memory
-    const int n_tq = min(2, my_chunks), n_sq = my_chunks - n_tq;
-    const uint32_t stage_bytes = (uint32_t)max_chunks * kKT * 128;
-    uint8_t* q_s = smem;                                             // (max_chunks - 2) x [128 x 128 B]
-    uint8_t* ring = q_s + (size_t)max(0, max_chunks - 2) * 128 * 128;   // kStages x stage_bytes
-    uint8_t* x_out = ring + (size_t)kStages * stage_bytes;           // own scores, fp16 [128 x 128 B]
-    uint8_t* x_in = x_out + 128 * 128;                               // peer's scores, 2 x [128 x 128 B]
-    LhBars& bs = *(LhBars*)(x_in + 2 * 128 * 128);
-    int* starts = (int*)((uint8_t*)&bs + ((sizeof(LhBars) + 15) & ~(size_t)15));   // [B + 1]
+    const int rank = (int)cluster_rank();
+    const int g = blockIdx.x >> 1;                        // cluster index
+    const int nq = p.n_qchunks;                           // 64-column chunks of a slot
+    const uint32_t unit_bytes = (uint32_t)p.unit_cols * kHalf * 2;
+    const int n_units = p.d_c / p.unit_cols;              // P.V units per 64-slot half
+    const int n_kst = (nq + kChunksPerStage - 1) / kChunksPerStage;   // score stages per tile
+    // both CTAs: two P halves [128 heads x 64 slots] bf16 (rank 0 stages them,
+    // rank 1 receives them), then the ring: rank 0 stages of three 64-column
+    // chunks [128 slots x 64 columns] each, rank 1 units [64 slots x unit_cols]
+    const uint32_t stage_bytes = rank == 0 ? (uint32_t)kChunksPerStage * 16384 : unit_bytes;
+    const int ring = min(kMaxRing, (int)((region_bytes - 2 * 16384) / stage_bytes));
+    uint8_t* ring_base = region + 2 * 16384;
 
-    // ---- schedule over 64-slot tiles (reads pos only)
-    {
-        const int per = (p.B + kThreads - 1) / kThreads;
-        const int b0 = tid * per, b1 = min(b0 + per, p.B);
-        int local = 0;
-        for (int b = b0; b < b1; ++b) local += lh_tiles(p, b);
-        int incl = local;
+    // ---- the cluster's tile range (reads pos only)
+    if (warp == 0) {
+        int total = 0;
+        for (int c = 0; c < p.B; c += 32) {
+            const int b = c + lane;
+            int t = b < p.B ? (lh_slots(p, b) + kKT - 1) / kKT : 0;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += v;
+            for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+            total += t;
         }
-        __shared__ int warp_tot[kThreads / 32];
-        if (lane == 31) warp_tot[warp] = incl;
-        __syncthreads();
-        int off = 0, tot = 0;
-        for (int w = 0; w < kThreads / 32; ++w) {
-            if (w < warp) off += warp_tot[w];
-            tot += warp_tot[w];
+        const int gt0 = (int)(((int64_t)g * total) / p.G2);
+        const int gt1 = (int)(((int64_t)(g + 1) * total) / p.G2);
+        // the sequence holding tile gt0: first b whose inclusive tile prefix exceeds gt0
+        int run = 0, b0 = p.B, j0 = 0;
+        for (int c = 0; c < p.B && b0 == p.B; c += 32) {
+            const int b = c + lane;
+            const int t = b < p.B ? (lh_slots(p, b) + kKT - 1) / kKT : 0;
+            int incl = t;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += v;
+            }
+            const unsigned hit = __ballot_sync(0xffffffffu, run + incl > gt0);
+            if (hit) {
+                const int l0 = __ffs(hit) - 1;
+                const int excl = __shfl_sync(0xffffffffu, incl - t, l0);
+                b0 = c + l0;
+                j0 = gt0 - (run + excl);
+            }
+            run += __shfl_sync(0xffffffffu, incl, 31);
         }
-        int run = off + incl - local;
-        for (int b = b0; b < b1; ++b) {
-            starts[b] = run;
-            run += lh_tiles(p, b);
-        }
-        if (tid == 0) {
-            bs.total = tot;
-            starts[p.B] = tot;
+        if (lane == 0) {
+            cs.b0 = b0;
+            cs.j0 = j0;
+            cs.n_tiles = gt1 - gt0;
         }
     }
     if (tid == 0) {
-        for (int i = 0; i < kStages; ++i) {
-            mbar_init(&bs.full[i], 1);
-            mbar_init(&bs.empty[i], 1);
+        for (int i = 0; i < kMaxRing; ++i) {
+            mbar_init(&cs.full[i], 1);
+            mbar_init(&cs.empty[i], 1);
         }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&bs.s_full[i], 1);
-            mbar_init(&bs.s_empty[i], 8);
-            mbar_init(&bs.p_full[i], 8);
-            mbar_init(&bs.o_done[i], 1);
+        mbar_init(&cs.s_full, 1);
+        mbar_init(&cs.s_empty, 8);
+        mbar_init(&cs.qt_full, 8);
+        for (int h = 0; h < 2; ++h) {
+            mbar_init(&cs.p_free[h], 1);
+            mbar_init(&cs.p_full[h], 1);
         }
-        mbar_init(&bs.q_full, 1);
-        mbar_init(&bs.q_free, 1);
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(&bs.x_full[i], 1);     // local expect_tx arrive; the peer's copy completes the bytes
-            mbar_init(&bs.x_free[i], 1);     // one remote arrive from the peer
-        }
-        mbar_init(&bs.qt_full, 8);
-        mbar_init(&bs.drain[0], 1);
-        mbar_init(&bs.drain[1], 1);
-        bs.fail = 0;
+        mbar_init(&cs.o_done, 1);
+        mbar_init(&cs.ev_full, 1);
+        mbar_init(&cs.ev_done, 1);
+        mbar_init(&cs.drain, 1);
+        cs.fail = 0;
         fence_mbar_init();
-        tma_prefetch_desc(&tmap);
+        tma_prefetch_desc(rank == 0 ? &map_k : &map_v);
     }
     if (warp == 1) {
-        tmem_alloc(&bs.tmem_base, 512);
+        tmem_alloc(&cs.tmem_base, 512);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    cluster_sync();                      // peer barriers exist before any remote operation
+    cluster_sync();                      // the peer's barriers exist before any remote operation
     pdl_launch_dependents();
-    const uint32_t tmem = bs.tmem_base;
-    const uint32_t t_o = tmem;                         // O_c: columns [0, lat_half)
-    const uint32_t t_s = tmem + 256;                   // partial scores: 2 x 64 columns
-    const uint32_t t_p = tmem + 384;                   // P (bf16 pairs): 2 x 32 columns
-    const uint32_t t_q = tmem + 448;                   // query chunks (bf16 pairs): 2 x 32 columns
-    const int total = bs.total;
-    const int gt0 = (int)(((int64_t)g * total) / p.G2);
-    const int gt1 = (int)(((int64_t)(g + 1) * total) / p.G2);
-    auto locate = [&](int gt, int& b, int& j) {
-        int lo = 0, hi = p.B - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (starts[mid] <= gt) lo = mid; else hi = mid - 1;
-        }
-        b = lo;
-        j = gt - starts[lo];
-    };
-    pdl_wait();                          // cache row and query image come from k_lh_prep
+    const uint32_t tmem = cs.tmem_base;
+    const int n = cs.n_tiles;
+    LhWalk w0;
+    w0.start(p, cs.b0, cs.j0);
 
-    int loads_issued = 0, q_loads = 0;   // producer's copies, for the drain on failure
+    int loads_issued = 0;                // producer: ring fills, for the drain after a failure
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
+        // Tiles before a sequence's last one do not hold the slot k_lh_prep
+        // updates, so their loads start before the wait for that kernel.
         if (lane == 0) {
-            int prev_b = -1;
-            for (int gt = gt0, it = 0; gt < gt1; ++gt, ++it) {
-                int b, j;
-                locate(gt, b, j);
-                if (b != prev_b) {
-                    prev_b = b;
-                    if (q_loads >= 1 && !lh_wait(&bs.q_free, (q_loads - 1) & 1, bs)) break;
-                    mbar_arrive_expect_tx(&bs.q_full, (uint32_t)n_sq * 128 * 128);
-                    const uint8_t* src = p.qimg + (size_t)b * p.n_qchunks * 128 * 128;
-                    for (int i = 0; i < n_sq; ++i)
-                        bulk_load(q_s + (size_t)i * 128 * 128,
-                                  src + (size_t)lh_chunk_id(rank, i, lat_chunks, rope_first) * 128 * 128,
-                                  128 * 128, &bs.q_full);
-                    ++q_loads;
+            LhWalk w = w0;
+            bool waited = false;
+            for (int k = 0; k < n && !cs.fail; ++k, w.next(p)) {
+                if (!waited && w.last_of_seq()) {
+                    pdl_wait();
+                    waited = true;
                 }
-                const int st = it % kStages;
-                if (it >= kStages && !lh_wait(&bs.empty[st], ((it / kStages) - 1) & 1, bs)) break;
-                mbar_arrive_expect_tx(&bs.full[st], (uint32_t)my_chunks * kKT * 128);
-                for (int i = 0; i < my_chunks; ++i)
-                    tma_load_3d(ring + st * stage_bytes + (size_t)i * kKT * 128, &tmap, &bs.full[st],
-                                lh_chunk_id(rank, i, lat_chunks, rope_first) * 64, j * kKT, b);
-                ++loads_issued;
-
+                if (rank == 0) {
+                    // one box per stage: chunks 3i .. 3i+2 of 128 slots (a chunk past
+                    // the slot width reads as zero)
+                    for (int i = 0; i < n_kst; ++i, ++loads_issued) {
+                        const int st = loads_issued % ring;
+                        if (loads_issued >= ring && !lh_wait(&cs.empty[st], ((loads_issued / ring) - 1) & 1, cs)) break;
+                        mbar_arrive_expect_tx(&cs.full[st], stage_bytes);
+                        tma_load_4d(ring_base + (size_t)st * stage_bytes, &map_k, &cs.full[st], 0, w.j * kKT,
+                                    i * kChunksPerStage, w.b);
+                    }
+                } else {
+                    for (int h = 0; h < 2; ++h)
+                        for (int u = 0; u < n_units; ++u, ++loads_issued) {
+                            const int st = loads_issued % ring;
+                            if (loads_issued >= ring &&
+                                !lh_wait(&cs.empty[st], ((loads_issued / ring) - 1) & 1, cs))
+                                break;
+                            mbar_arrive_expect_tx(&cs.full[st], unit_bytes);
+                            tma_load_4d(ring_base + (size_t)st * unit_bytes, &map_v, &cs.full[st], 0,
+                                        w.j * kKT + h * kHalf, u * (p.unit_cols / 64), w.b);
+                        }
+                }
+            }
+            if (cs.fail) {
+                // let the loads in flight land before shared memory is released
+                for (int k = max(0, loads_issued - ring); k < loads_issued; ++k)
+                    mbar_wait(&cs.full[k % ring], (k / ring) & 1);
             }
         }
     } else if (warp == 1) {
-        // ------------------------------------------------------------ score MMAs
         if (lane == 0) {
-            const uint32_t id_s = idesc_bf16_f32(128, kKT, false, false);
-            const uint32_t ring_a = smem_u32(ring);
-            const uint64_t q_d = sdesc_sw128(smem_u32(q_s), 16, 1024);
-            int seg = -1, prev_b = -1, it = 0;
-            for (int gt = gt0; gt < gt1; ++gt, ++it) {
-                int b, j;
-                locate(gt, b, j);
-                if (b != prev_b) {
-                    prev_b = b;
-                    ++seg;
-                    if (!lh_wait(&bs.q_full, seg & 1, bs)) break;    // q~ chunks in smem
-                    if (!lh_wait(&bs.qt_full, seg & 1, bs)) break;   // q~ chunks in TMEM
+            if (rank == 0) {
+                // -------------------------------------------------------- score MMAs
+                const uint32_t id_s = idesc_bf16_f32(128, kKT, false, false);
+                const uint32_t t_s = tmem, t_q = tmem + 128;
+                LhWalk w = w0;
+                int it = 0, seg = -1;
+                for (int k = 0; k < n; ++k, w.next(p)) {
+                    if (k == 0 || w.j == 0) {
+                        ++seg;
+                        if (!lh_wait(&cs.qt_full, seg & 1, cs)) break;    // query chunks in TMEM
+                    }
+                    if (k >= 1 && !lh_wait(&cs.s_empty, (k - 1) & 1, cs)) break;   // S(k-1) read out
+                    tc_fence_after();
+                    bool ok = true;
+                    // straight-line groups of four MMAs, one wait per stage of three chunks
+#pragma unroll
+                    for (int c = 0; c < kMaxQChunks; ++c) {
+                        if (c < nq && ok) {
+                            const int st = it % ring;
+                            const int cs3 = c % kChunksPerStage;
+                            if (cs3 == 0) {
+                                ok = lh_wait(&cs.full[st], (it / ring) & 1, cs);
+                                tc_fence_after();
+                            }
+                            if (ok) {
+                                const uint64_t kd = sdesc_sw128(
+                                    smem_u32(ring_base + (size_t)st * stage_bytes + cs3 * 16384), 16, 1024);
+                                umma_bf16_ts(t_s, t_q + c * 32, kd, id_s, c != 0 ? 1u : 0u);
+                                umma_bf16_ts(t_s, t_q + c * 32 + 8, desc_add(kd, 32), id_s, 1u);
+                                umma_bf16_ts(t_s, t_q + c * 32 + 16, desc_add(kd, 64), id_s, 1u);
+                                umma_bf16_ts(t_s, t_q + c * 32 + 24, desc_add(kd, 96), id_s, 1u);
+                                if (cs3 == kChunksPerStage - 1 || c == nq - 1) {
+                                    umma_commit(&cs.empty[st]);
+                                    ++it;
+                                }
+                            }
+                        }
+                    }
+                    if (!ok) break;
+                    umma_commit(&cs.s_full);
                 }
-                const int st = it % kStages;
-                if (!lh_wait(&bs.full[st], (it / kStages) & 1, bs)) break;
-                if (it >= 2 && !lh_wait(&bs.s_empty[it & 1], ((it >> 1) - 1) & 1, bs)) break;
-                tc_fence_after();
-                // S_c = q~_c . K_c^T (M = 128 heads, N = 64 slots)
-                const uint64_t kd = sdesc_sw128(ring_a + st * stage_bytes, 16, 1024);
-                const uint32_t ts = t_s + (it & 1) * kKT;
-                // Straight-line groups of four MMAs with one test per group (a
-                // runtime loop or a test per MMA halves their issue rate). Every
-                // chunk is a full 64 columns (D is a multiple of 64).
-#pragma unroll
-                for (int i = 0; i < kMaxSq; ++i) {
-                    if (i < n_sq) {
-                        const uint64_t qi = desc_add(q_d, i * 128 * 128), ki = desc_add(kd, i * kKT * 128);
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            umma_bf16(ts, desc_add(qi, kk * 32), desc_add(ki, kk * 32), id_s, (i | kk) != 0);
+                if (cs.fail) {
+                    umma_commit(&cs.drain);
+                    mbar_wait(&cs.drain, 0);
+                }
+            } else {
+                // -------------------------------------------------------- P.V MMAs
+                const uint32_t id_o = idesc_bf16_f32(128, p.unit_cols, false, true);
+                LhWalk w = w0;
+                int it = 0, ev = 0, ocnt = 0;
+                auto post = [&](int type, int arg) -> bool {
+                    cs.ev[0] = type;
+                    cs.ev_arg[0] = arg;
+                    mbar_arrive(&cs.ev_full);
+                    const bool ok = lh_wait(&cs.ev_done, ev & 1, cs);
+                    ++ev;
+                    return ok;
+                };
+                auto o_settle = [&]() -> bool {      // every P.V issued so far is complete
+                    umma_commit(&cs.o_done);
+                    ++ocnt;
+                    return lh_wait(&cs.o_done, (ocnt - 1) & 1, cs);
+                };
+                bool ok = true;
+                for (int k = 0; k < n && ok; ++k, w.next(p)) {
+                    const bool first = (k == 0) || (w.j == 0);
+                    for (int h = 0; h < 2 && ok; ++h) {
+                        // rank 0's bulk copy of P half h (and, with half 0, the side
+                        // information) completes its bytes on p_full[h]
+                        mbar_arrive_expect_tx(&cs.p_full[h], h == 0 ? 16384u + (uint32_t)sizeof(LhSide) : 16384u);
+                        ok = lh_wait_cluster(&cs.p_full[h], k & 1, cs);
+                        if (!ok) break;
+                        tc_fence_after();
+                        const volatile int* fl = cs.side.flag;
+                        if (h == 0 && !first && (fl[0] | fl[1] | fl[2] | fl[3])) {
+                            // a row's reference maximum moved: O rows scaled before this tile adds to them
+                            ok = o_settle() && post(kEvRescale, 0);
+                            if (!ok) break;
+                            tc_fence_after();
+                        }
+                        const int s0 = w.j * kKT + h * kHalf;
+                        const int v0 = max(0, min(kHalf, w.nb - s0));          // valid slots of this half
+                        const int vend = min(kHalf, p.max_slots - s0);         // rows inside the cache buffer
+                        if (v0 < vend) {
+                            // rows past the sequence's last slot hold stale bytes: zeroed before P.V
+                            ok = post(kEvZero, (it << 8) | v0);
+                            if (!ok) break;
+                        }
+                        const uint64_t pd = sdesc_sw128(smem_u32(region + h * 16384), 16, 1024);
+                        for (int u = 0; u < n_units; ++u) {
+                            const int st = it % ring;
+                            ok = lh_wait(&cs.full[st], (it / ring) & 1, cs);
+                            if (!ok) break;
+                            tc_fence_after();
+                            const uint64_t vd = sdesc_sw128(smem_u32(ring_base + (size_t)st * unit_bytes), 8192, 1024);
+                            const uint32_t t_o = tmem + u * p.unit_cols;
+                            umma_bf16(t_o, pd, vd, id_o, (first && h == 0) ? 0u : 1u);
+                            umma_bf16(t_o, desc_add(pd, 32), desc_add(vd, 2048), id_o, 1u);
+                            umma_bf16(t_o, desc_add(pd, 64), desc_add(vd, 4096), id_o, 1u);
+                            umma_bf16(t_o, desc_add(pd, 96), desc_add(vd, 6144), id_o, 1u);
+                            umma_commit(&cs.empty[st]);
+                            ++it;
+                        }
+                        if (!ok) break;
+                        umma_commit_to(&cs.p_free[h], 0x1);                    // rank 0 may write P half h again
+                    }
+                    if (ok && (k == n - 1 || w.last_of_seq())) {
+                        ok = o_settle() && post(kEvSegEnd, g + w.b);
                     }
                 }
-#pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    if (i < n_tq) {
-                        const uint64_t ki = desc_add(kd, (n_sq + i) * kKT * 128);
-                        const uint32_t acc0 = (n_sq + i) != 0 ? 1u : 0u;
-                        umma_bf16_ts(ts, t_q + i * 32, ki, id_s, acc0);
-#pragma unroll
-                        for (int kk = 1; kk < 4; ++kk)
-                            umma_bf16_ts(ts, t_q + i * 32 + kk * 8, desc_add(ki, kk * 32), id_s, 1u);
-                    }
+                cs.ev[0] = kEvEnd;
+                mbar_arrive(&cs.ev_full);
+                if (cs.fail) {
+                    umma_commit(&cs.drain);
+                    mbar_wait(&cs.drain, 0);
                 }
-                umma_commit(&bs.s_full[it & 1]);
-                const bool last = (gt + 1 == gt1) || (j + 1 == starts[b + 1] - starts[b]);
-                if (last) umma_commit(&bs.q_free);
             }
         }
-    } else if (warp == 10) {
-        // ------------------------------------------------------------ P.V MMAs
-        // A second issuing thread, so that P.V (which frees ring stages) never
-        // waits behind score MMAs that wait for a load.
-        if (lane == 0) {
-            const uint32_t id_o = idesc_bf16_f32(128, lat_half, false, true);
-            const uint32_t ring_a = smem_u32(ring);
-            int prev_b = -1, it = 0;
-            for (int gt = gt0; gt < gt1; ++gt, ++it) {
-                int b, j;
-                locate(gt, b, j);
-                const bool first = (b != prev_b);
-                prev_b = b;
-                if (!lh_wait(&bs.p_full[it & 1], (it >> 1) & 1, bs)) break;
-                tc_fence_after();
-                // O_c += P . V_c: A = P in TMEM, B = the tile's latent columns (MN-major)
-                const uint64_t vd = sdesc_sw128(ring_a + (it % kStages) * stage_bytes, kKT * 128, 1024);
-#pragma unroll
-                for (int kk = 0; kk < kKT / 16; ++kk)
-                    umma_bf16_ts(t_o, t_p + (it & 1) * 32 + kk * 8, desc_add(vd, kk * 2048), id_o,
-                                 (first && kk == 0) ? 0u : 1u);
-                umma_commit(&bs.empty[it % kStages]);
-                umma_commit(&bs.o_done[it & 1]);
-            }
-        }
-    } else {
+    } else if (rank == 0) {
         // ------------------------------------------------------------ softmax (two threads per head row)
-        // Warps 2-9: row r = (warp mod 4) * 32 + lane (the TMEM lane quarter a warp
-        // may access), column half hc = (warp - 2) / 4 of each 64-slot tile.
-        // The partial scores travel by one bulk copy per tile from x_out into the
-        // peer's x_in[tile parity]; the copy completes the bytes on the peer's
-        // x_full[parity]. No early exit from the loop: after a bounded wait gave
-        // up, later waits return at once, so no thread is left waiting.
+        // Warps 2-9: row r = (warp mod 4) * 32 + lane (the TMEM lane quarter a
+        // warp may access), slot half hc = (warp - 2) / 4 of each tile. No early
+        // exit from the loop: after a bounded wait gave up, later waits return
+        // at once, so every thread reaches every named barrier.
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;
         const int hc = (warp - 2) >> 2;
-        const int sidx = tid - 64;                     // 0..255 over the softmax warps
-        const bool leader = sidx == 0;
         const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
-        const uint32_t x_in_peer = map_to_rank(x_in, peer);
-        const uint32_t xfull_peer = map_to_rank(&bs.x_full[0], peer);
-        const uint32_t xfree_peer = map_to_rank(&bs.x_free[0], peer);
-        uint32_t own[16];        // this thread's 32 scaled partial scores of the newest tile, fp16 pairs
-        uint32_t own_prev[16];   // ... of the tile B works on
-        // Query chunks n_sq.. of sequence b into TMEM: the thread of row r and
-        // half hc writes chunk n_sq + hc of row r (de-swizzled from the image).
+        const uint32_t t_s = tmem, t_q = tmem + 128;
+        // columns 480..484: the two half-row maxima by tile parity, and the
+        // second half's row sum at a segment end, exchanged between the two
+        // threads of a row (same TMEM lane quarter)
+        const uint32_t t_x = tmem + 480 + lane_off;
+        uint8_t* prow = region + hc * 16384 + r * 128;            // staging of P half hc, row r
+        const uint32_t p_peer = map_to_rank(region + hc * 16384, 1);
+        const uint32_t side_peer = map_to_rank(&cs.side, 1);
+        const uint32_t pfull_peer = map_to_rank(&cs.p_full[hc], 1);
+        const bool elected = (warp == 2 + 4 * hc) && lane == 0;   // issues the half's copies
+        // query chunks c = hc, hc + 2, ... of sequence b into TMEM (row r de-swizzled from the image)
         auto load_qt = [&](int b) {
-            if (hc < n_tq) {
-                const uint8_t* src = p.qimg + (size_t)b * p.n_qchunks * 128 * 128 +
-                                     (size_t)lh_chunk_id(rank, n_sq + hc, lat_chunks, rope_first) * 128 * 128 +
-                                     (size_t)r * 128;
-                uint32_t w[32];
+            const uint8_t* img = p.qimg + (size_t)b * nq * 16384 + (size_t)r * 128;
+            for (int c = hc; c < nq; c += 2) {
+                uint32_t wv[32];
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
-                    const uint4 v = *(const uint4*)(src + (((u ^ r) & 7) << 4));
-                    w[4 * u] = v.x;
-                    w[4 * u + 1] = v.y;
-                    w[4 * u + 2] = v.z;
-                    w[4 * u + 3] = v.w;
+                    const uint4 v = *(const uint4*)(img + (size_t)c * 16384 + (((u ^ r) & 7) << 4));
+                    wv[4 * u] = v.x;
+                    wv[4 * u + 1] = v.y;
+                    wv[4 * u + 2] = v.z;
+                    wv[4 * u + 3] = v.w;
                 }
-                tmem_st32_u(t_q + hc * 32 + lane_off, w);
-                tmem_wait_st();
+                tmem_st32_u(t_q + c * 32 + lane_off, wv);
             }
+            tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bs.qt_full);
+            if (lane == 0) mbar_arrive(&cs.qt_full);
         };
-        // A(k): partial scores of tile k -> own[], x_out, and the peer's x_in[k & 1]
-        auto half_a = [&](int k) {
-            lh_wait(&bs.s_full[k & 1], (k >> 1) & 1, bs);
-            tc_fence_after();
-            float sv[32];
-            tmem_ld32(t_s + (k & 1) * kKT + hc * 32 + lane_off, sv);
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bs.s_empty[k & 1]);
-            if (gt0 + k + 1 < gt1) {
-                // S(k) is complete, so every score MMA that read the TMEM query chunks
-                // is done; if tile k+1 opens a new segment, bring in its query
-                int b1, j1;
-                locate(gt0 + k + 1, b1, j1);
-                if (j1 == 0) load_qt(b1);
-            }
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-                const __half2 h2 = __floats2half2_rn(sv[2 * c] * p.scale_log2, sv[2 * c + 1] * p.scale_log2);
-                own[c] = *(const uint32_t*)&h2;
-            }
-            if (leader) {
-                bulk_wait_read_all();                               // the copy of tile k-1 has read x_out
-                if (!bs.fail) mbar_arrive_expect_tx(&bs.x_full[k & 1], 128 * 128);   // the peer's tile k
-            }
-            named_sync(1, 256);
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-                *(uint4*)(x_out + xoff(r, 4 * hc + u)) =
-                    make_uint4(own[4 * u], own[4 * u + 1], own[4 * u + 2], own[4 * u + 3]);
-            fence_proxy_async();
-            named_sync(1, 256);
-            if (leader) {
-                // the peer's x_in[k & 1] was read by its B(k - 2)
-                if (k < 2 || lh_wait_cluster(&bs.x_free[k & 1], ((k >> 1) - 1) & 1, bs)) {
-                    bulk_copy_to_peer(x_in_peer + (k & 1) * 128 * 128, x_out, 128 * 128, xfull_peer + (k & 1) * 8);
-                    bulk_commit_group();
-                }
-            }
-        };
-        float m_ref = -INFINITY, l = 0.f;              // l: this thread's half of the row sum
-        int prev_b = -1, n_b = 0, k_in_seg = 0;
-        if (gt0 < gt1) {
-            int b0, j0;
-            locate(gt0, b0, j0);
-            load_qt(b0);
-            half_a(0);
-        }
-        for (int gt = gt0, it = 0; gt < gt1; ++gt, ++it) {
-            int b, j;
-            locate(gt, b, j);
-            if (b != prev_b) {
-                prev_b = b;
-                n_b = lh_slots(p, b);
+        pdl_wait();                      // the query images come from k_lh_prep
+        if (n > 0) load_qt(w0.b);
+        float m_ref = -INFINITY, l = 0.f;   // l: this thread's half of the row sum
+        int k_in_seg = 0;
+        LhWalk w = w0;
+        for (int k = 0; k < n; ++k) {
+            if (k > 0 && w.j == 0) {
                 m_ref = -INFINITY;
                 l = 0.f;
                 k_in_seg = 0;
             }
+            lh_wait(&cs.s_full, k & 1, cs);
+            tc_fence_after();
+            float sv[64];
+            tmem_ld32(t_s + hc * 64 + lane_off, sv);
+            tmem_ld32(t_s + hc * 64 + 32 + lane_off, sv + 32);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&cs.s_empty);
+            LhWalk nx = w;
+            nx.next(p);
+            // S(k) complete: every score MMA that read the query chunks is done
+            if (k + 1 < n && nx.j == 0) load_qt(nx.b);
+            const int valid = min(kKT, w.nb - w.j * kKT) - hc * kHalf;   // valid slots of this half
+            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // four independent chains
 #pragma unroll
-            for (int c = 0; c < 16; ++c) own_prev[c] = own[c];
-            if (gt + 1 < gt1) half_a(it + 1);       // the peer's copy of tile it+1 overlaps B(it)
-            const int st = it % kStages;
-            const int valid = min(kKT, n_b - j * kKT) - hc * 32;   // valid columns of this half
-            // B(it): add the peer's partial scores of this tile (a + b = b + a
-            // exactly, so both CTAs hold the same scores)
-            lh_wait(&bs.x_full[it & 1], (it >> 1) & 1, bs);
-            const uint8_t* xin = x_in + (it & 1) * 128 * 128;
-            uint4 th[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) th[u] = *(const uint4*)(xin + xoff(r, 4 * hc + u));
-            float sv[32];
-            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // four independent chains
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const uint32_t tw[4] = {th[u].x, th[u].y, th[u].z, th[u].w};
-#pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                    const float2 fm = __half22float2(*(const __half2*)&own_prev[4 * u + v]);
-                    const float2 ft = __half22float2(*(const __half2*)&tw[v]);
-                    const int c = 8 * u + 2 * v;
-                    sv[c] = c < valid ? fm.x + ft.x : -INFINITY;
-                    sv[c + 1] = c + 1 < valid ? fm.y + ft.y : -INFINITY;
-                    m4[v] = fmaxf(m4[v], fmaxf(sv[c], sv[c + 1]));
-                }
+            for (int c = 0; c < 64; ++c) {
+                sv[c] = c < valid ? sv[c] : -INFINITY;
+                m4[c & 3] = fmaxf(m4[c & 3], sv[c]);
             }
-            float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-            bs.red[it & 1][hc][r] = mt;
-            named_sync(1, 256);                        // also: every thread has read x_in[it & 1]
-            if (leader) mbar_arrive_remote_relaxed(xfree_peer + (it & 1) * 8);
-            mt = fmaxf(mt, bs.red[it & 1][hc ^ 1][r]);
+            float mt = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * p.scale_log2;
+            tmem_st1(t_x + (k & 1) * 2 + hc, mt);
+            tmem_wait_st();
+            tc_fence_before();
+            named_sync(1, 256);
+            tc_fence_after();
+            mt = fmaxf(mt, tmem_ld1(t_x + (k & 1) * 2 + (hc ^ 1)));
+            tmem_wait_ld();
             // lazy rescale: the reference maximum moves only when the tile's maximum
             // exceeds it by more than 2^8 (P stays <= 256); both halves decide alike
             const bool upd = mt > m_ref + kRescaleLog2;
             const float nm = upd ? mt : m_ref;
             const float fac = ex2_approx(m_ref - nm);    // 0 when m_ref was -inf, 1 when kept
             float rs4[4] = {0.f, 0.f, 0.f, 0.f};
-            uint32_t pk[16];
+            uint32_t pk[32];
 #pragma unroll
-            for (int c = 0; c < 16; ++c) {
-                const float p0 = ex2_approx(sv[2 * c] - nm), p1 = ex2_approx(sv[2 * c + 1] - nm);
+            for (int c = 0; c < 32; ++c) {
+                const float p0 = ex2_approx(fmaf(sv[2 * c], p.scale_log2, -nm));
+                const float p1 = ex2_approx(fmaf(sv[2 * c + 1], p.scale_log2, -nm));
                 rs4[c & 3] += p0 + p1;
                 pk[c] = pack_bf16x2(p0, p1);
             }
             l = fmaf(l, fac, (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
             m_ref = nm;
             const bool need = upd && k_in_seg > 0;
-            if (__any_sync(0xffffffffu, need)) {
-                // this warp's rows of its half of O_c move to their new reference maxima
-                lh_wait(&bs.o_done[(it - 1) & 1], ((it - 1) >> 1) & 1, bs);
-                tc_fence_after();
-                const float f = need ? fac : 1.f;
-                const int cols = lat_half / 2;
-                float v[32];
-                for (int cc = 0; cc < cols / 32; ++cc) {
-                    const uint32_t ta = t_o + hc * cols + cc * 32 + lane_off;
-                    tmem_ld32(ta, v);
-                    tmem_wait_ld();
+            // P half hc of tile k: staged here (the copy of tile k-1 has read the
+            // staging), then one bulk copy into rank 1 once its P.V of tile k-1
+            // has read the destination; the copy completes on rank 1's p_full[hc]
+            if (elected) bulk_wait_read_all();
+            named_sync(2 + hc, 128);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) v[i] *= f;
-                    tmem_st32(ta, v);
-                }
-                tmem_wait_st();
+            for (int u = 0; u < 8; ++u)
+                *(uint4*)(prow + (((u ^ r) & 7) << 4)) = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+            if (hc == 0) {
+                cs.side.fac[r] = need ? fac : 1.f;
+                const bool any = __any_sync(0xffffffffu, need);
+                if (lane == 0) cs.side.flag[quarter] = any ? 1 : 0;
             }
-            if (valid + hc * 32 < kKT) {
-                // stale rows past the sequence's last slot must not reach P.V
-                const int v0 = valid + hc * 32, rows = kKT - v0;
-                uint8_t* stg = ring + st * stage_bytes;
-                for (int e = sidx; e < my_chunks * rows * 8; e += 256) {
-                    const int i = e / (rows * 8), rr = e % (rows * 8);
-                    *(uint4*)(stg + (size_t)i * kKT * 128 + (size_t)(v0 + rr / 8) * 128 + (rr % 8) * 16) =
-                        make_uint4(0, 0, 0, 0);
-                }
-            }
-            if (it >= 2) lh_wait(&bs.o_done[it & 1], ((it >> 1) - 1) & 1, bs);   // P.V of tile it-2 read this P buffer
-            tmem_st16_u(t_p + (it & 1) * 32 + hc * 16 + lane_off, pk);
-            tmem_wait_st();
             fence_proxy_async();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bs.p_full[it & 1]);
+            named_sync(2 + hc, 128);
+            if (elected) {
+                if (k >= 1) lh_wait(&cs.p_free[hc], (k - 1) & 1, cs);
+                if (!cs.fail) {
+                    bulk_copy_to_peer(p_peer, region + hc * 16384, 16384, pfull_peer);
+                    if (hc == 0) bulk_copy_to_peer(side_peer, &cs.side, (uint32_t)sizeof(LhSide), pfull_peer);
+                    bulk_commit_group();
+                }
+            }
             ++k_in_seg;
-            const bool last = (gt + 1 == gt1) || (j + 1 == starts[b + 1] - starts[b]);
-            if (last) {
-                // partial of this sequence segment: this CTA's half of O, plus (m, l)
-                bs.lsum[hc][r] = l;
-                lh_wait(&bs.o_done[it & 1], (it >> 1) & 1, bs);
-                tc_fence_after();
+            if (k == n - 1 || w.last_of_seq()) {
+                // (m, l) of this sequence segment; rank 1 writes its O
+                if (hc == 1) {
+                    tmem_st1(t_x + 4, l);
+                    tmem_wait_st();
+                }
+                tc_fence_before();
                 named_sync(1, 256);
-                const size_t row = (size_t)p.d_c + 4;
-                float* dst = p.part + ((size_t)(g + b) * p.H + r) * row;
-                const int cols = lat_half / 2;
-                float v[32];
+                tc_fence_after();
+                if (hc == 0) {
+                    const float l1 = tmem_ld1(t_x + 4);
+                    tmem_wait_ld();
+                    if (r < p.H) {
+                        float* dst = p.part + ((size_t)(g + w.b) * p.H + r) * ((size_t)p.d_c + 4);
+                        dst[p.d_c] = m_ref;
+                        dst[p.d_c + 1] = l + l1;
+                    }
+                }
+            }
+            w = nx;
+        }
+        if (elected) bulk_wait_read_all();
+    } else {
+        // ------------------------------------------------------------ rank 1 events
+        // Warps 2-9 take the events the MMA thread posts, in order: thread
+        // (row r, column half hc) of O.
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;
+        const int hc = (warp - 2) >> 2;
+        const uint32_t lane_off = (uint32_t)(quarter * 32) << 16;
+        const int cols = p.d_c / 2;
+        const int sidx = tid - 64;
+        for (int ev = 0;; ++ev) {
+            const bool got = mbar_wait(&cs.ev_full, ev & 1);
+            if (!named_sync_and(1, 256, got)) break;
+            const int type = cs.ev[0], arg = cs.ev_arg[0];
+            if (type == kEvEnd) break;
+            tc_fence_after();
+            if (type == kEvRescale) {
+                const float f = cs.side.fac[r];
+                if (__any_sync(0xffffffffu, f != 1.f)) {
+                    for (int cc = 0; cc < cols / 32; ++cc) {
+                        const uint32_t ta = tmem + hc * cols + cc * 32 + lane_off;
+                        float v[32];
+                        tmem_ld32(ta, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) v[i] *= f;
+                        tmem_st32(ta, v);
+                    }
+                    tmem_wait_st();
+                }
+            } else if (type == kEvZero) {
+                // rows v0.. of the units it0 .. it0 + n_units - 1 (one 64-slot half)
+                const int it0 = arg >> 8, v0 = arg & 255;
+                const int rows = kHalf - v0, per_unit = rows * (p.unit_cols / 8);
+                bool landed = true;
+                for (int u = 0; u < n_units; ++u)
+                    landed &= mbar_wait(&cs.full[(it0 + u) % ring], ((it0 + u) / ring) & 1);
+                if (landed) {
+                    for (int e = sidx; e < n_units * per_unit; e += 256) {
+                        const int u = e / per_unit, rem = e % per_unit;
+                        const int row = v0 + rem / (p.unit_cols / 8), q16 = rem % (p.unit_cols / 8);
+                        uint8_t* unit = ring_base + (size_t)((it0 + u) % ring) * unit_bytes;
+                        *(uint4*)(unit + (size_t)(q16 >> 3) * 8192 + (size_t)row * 128 + (q16 & 7) * 16) =
+                            make_uint4(0, 0, 0, 0);
+                    }
+                    fence_proxy_async();
+                } else {
+                    cs.fail = 1;
+                }
+            } else if (type == kEvSegEnd) {
+                // TMEM loads are warp-collective: every lane loads, rows past H drop theirs
+                float* dst = p.part + ((size_t)arg * p.H + r) * ((size_t)p.d_c + 4) + hc * cols;
                 for (int cc = 0; cc < cols / 32; ++cc) {
-                    tmem_ld32(t_o + hc * cols + cc * 32 + lane_off, v);
+                    float v[32];
+                    tmem_ld32(tmem + hc * cols + cc * 32 + lane_off, v);
                     tmem_wait_ld();
                     if (r < p.H) {
 #pragma unroll
                         for (int u = 0; u < 8; ++u)
-                            *(float4*)(dst + rank * lat_half + hc * cols + cc * 32 + 4 * u) =
-                                make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+                            *(float4*)(dst + cc * 32 + 4 * u) = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
                     }
                 }
-                if (rank == 0 && hc == 0 && r < p.H) {
-                    dst[p.d_c] = m_ref;
-                    dst[p.d_c + 1] = l + bs.lsum[1][r];
-                }
-                tc_fence_before();
             }
+            tc_fence_before();
+            named_sync(1, 256);
+            if (sidx == 0) mbar_arrive(&cs.ev_done);
         }
     }
     tc_fence_before();
     __syncthreads();
-    if (bs.fail) {
-        // a bounded wait gave up: let this CTA's copies and MMAs land (bounded
-        // again) before shared memory and TMEM are released, then report
-        if (warp == 0 && lane == 0) {
-            for (int k = max(0, loads_issued - kStages); k < loads_issued; ++k)
-                mbar_wait(&bs.full[k % kStages], (k / kStages) & 1);
-            if (q_loads > 0) mbar_wait(&bs.q_full, (q_loads - 1) & 1);
-        }
-        if ((warp == 1 || warp == 10) && lane == 0) {
-            uint64_t* d = &bs.drain[warp == 1 ? 0 : 1];
-            umma_commit(d);              // arrives when this thread's MMAs are done
-            mbar_wait(d, 0);
-        }
-        if (tid == 64) {
-            // the peer's score copies into this CTA, and this CTA's own copies
-            const int n = gt1 - gt0;
-            for (int k = max(0, n - 2); k < n; ++k) mbar_wait(&bs.x_full[k & 1], (k >> 1) & 1);
-            bulk_wait_read_all();
-        }
-        if (tid == 0) latch_status(p.status, kStatusTimeout);
-        __syncthreads();
-    }
+    if (cs.fail && tid == 0) latch_status(p.status, kStatusTimeout);
     tc_fence_after();
     if (warp == 1) tmem_dealloc(tmem, 512);
     cluster_sync();                      // the peer may still store into / arrive on us until here
@@ -958,15 +1017,23 @@ __global__ void __launch_bounds__(kCombThreads, 1)
 
 // ---------------------------------------------------------------- host side
 
-size_t lh_attn_smem(const Shape& sh) {
-    const int lat_chunks = sh.d_c / 128;
-    const int max_chunks = lat_chunks + (sh.D / 64 - sh.d_c / 64);
-    size_t bytes = 1024;
-    bytes += (size_t)std::max(0, max_chunks - 2) * 128 * 128;   // q~ chunks in shared memory
-    bytes += (size_t)kStages * max_chunks * kKT * 128;  // key tiles
-    bytes += 3 * 128 * 128;                             // exchanged scores (own; peer's x 2), fp16
-    bytes += ((sizeof(LhBars) + 15) & ~(size_t)15) + ((size_t)sh.B + 1) * 4;
-    return bytes;
+// The attention kernel takes all the shared memory a block may opt into: its
+// rings are sized from what it gets (at least two P.V units on rank 1).
+size_t lh_attn_smem() {
+    static int optin = 0;
+    if (!optin) {
+        int dev = 0, v = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess &&
+            cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) == cudaSuccess && v > 0)
+            optin = v;
+        else
+            optin = 232448;
+    }
+    return (size_t)optin;
+}
+size_t lh_attn_smem_min(const Shape& sh) {
+    const size_t unit = (size_t)std::min(256, sh.d_c) * kHalf * 2;
+    return 1023 + kCtlBytes + 2 * 16384 + 2 * std::max(unit, (size_t)kChunksPerStage * 16384);
 }
 
 size_t lh_prep_smem(const Shape& sh) {
@@ -1007,8 +1074,7 @@ bool tc_decode_lh_supported(const Shape& sh) {
     return sh.H > 32 && sh.H <= 128 && sh.d_c % 128 == 0 && sh.d_c <= 512 && sh.D % 64 == 0 && sh.d_r <= 128 &&
            (sh.d_h == 64 || sh.d_h == 128 || sh.d_h == 256 || sh.d_h == 512) &&
            (sh.d_c == 128 || sh.d_c == 256 || sh.d_c == 512) && sh.B <= kMaxB && lh_comb_smem(sh) <= 227 * 1024 &&
-           lh_prep_smem(sh) <= 227 * 1024 &&
-           lh_attn_smem(sh) <= 232448 - 1024;
+           lh_prep_smem(sh) <= 227 * 1024 && sh.D / 64 <= kMaxQChunks && lh_attn_smem_min(sh) <= 232448 - 16384;
 }
 
 size_t tc_decode_lh_workspace(const Shape& sh) {
@@ -1022,18 +1088,29 @@ cudaError_t tc_decode_lh(const DecodeArgs& a, cudaStream_t st, uint64_t* launche
     float* part = (float*)((char*)a.workspace + align256((size_t)sh.B * (sh.D / 64) * 128 * 128));
     auto encode = (PFN_cuTensorMapEncodeTiled_v12000)tensor_map_encoder();
     if (!encode) return note_error("cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", cudaErrorNotSupported);
-    CUtensorMap map;
-    cuuint64_t dims[3] = {(cuuint64_t)sh.D, (cuuint64_t)sh.max_slots, (cuuint64_t)sh.B};
-    cuuint64_t strides[2] = {(cuuint64_t)sh.D * 2, (cuuint64_t)sh.max_slots * sh.D * 2};
-    cuuint32_t box[3] = {64, (cuuint32_t)kKT, 1};
-    cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.cache, dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) {
-        char buf[96];
-        snprintf(buf, sizeof(buf), "cuTensorMapEncodeTiled (CUresult %d)", (int)r);
-        return note_error(buf, cudaErrorInvalidValue);
+    // the cache viewed as {64 columns, max_slots, D / 64 chunks, B} (chunk
+    // stride 128 B), so that one box brings several 64-column chunks, each
+    // laid out as its own SW128 operand: three chunks x 128 slots for the
+    // scores (rank 0), unit_cols / 64 chunks x 64 slots for P.V (rank 1).
+    // Slots past max_slots and chunks past D / 64 read as zero. A TMA engine
+    // completes about as many boxes per second whatever their size up to
+    // 16 KB, so few large boxes keep one SM at the HBM share it needs.
+    CUtensorMap map_k, map_v;
+    CUresult r = CUDA_SUCCESS;
+    for (int m = 0; m < 2; ++m) {
+        cuuint64_t dims[4] = {64, (cuuint64_t)sh.max_slots, (cuuint64_t)(sh.D / 64), (cuuint64_t)sh.B};
+        cuuint64_t strides[3] = {(cuuint64_t)sh.D * 2, 128, (cuuint64_t)sh.max_slots * sh.D * 2};
+        cuuint32_t box[4] = {64, (cuuint32_t)(m == 0 ? kKT : kHalf),
+                             (cuuint32_t)(m == 0 ? kChunksPerStage : std::min(256, sh.d_c) / 64), 1};
+        cuuint32_t estr[4] = {1, 1, 1, 1};
+        r = encode(m == 0 ? &map_k : &map_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.cache, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) {
+            char buf[96];
+            snprintf(buf, sizeof(buf), "cuTensorMapEncodeTiled cache (CUresult %d)", (int)r);
+            return note_error(buf, cudaErrorInvalidValue);
+        }
     }
     // W_UK and W_UV as [H * d_h rows][d_c] bf16, 128-row x 64-column boxes
     // (rows past the last head read as zero)
@@ -1061,13 +1138,15 @@ cudaError_t tc_decode_lh(const DecodeArgs& a, cudaStream_t st, uint64_t* launche
     p.s = sh.s;
     p.max_slots = sh.max_slots;
     p.n_qchunks = sh.D / 64;
+    p.unit_cols = std::min(256, sh.d_c);
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64) dev = 0;
     static size_t done_prep[64] = {0}, done_attn[64] = {0}, done_comb[64] = {0};
     static int co_resident[64] = {0};
     const size_t prep_smem = lh_prep_smem(sh);
-    const size_t attn_smem = lh_attn_smem(sh);
+    const size_t attn_smem = lh_attn_smem();
+    p.smem_bytes = (uint32_t)attn_smem;
     const size_t comb_smem = lh_comb_smem(sh);
     cudaError_t e = lh_set_smem(k_lh_prep, prep_smem, &done_prep[dev]);
     if (e == cudaSuccess) e = lh_set_smem(k_lh_attn, attn_smem, &done_attn[dev]);
@@ -1098,7 +1177,7 @@ cudaError_t tc_decode_lh(const DecodeArgs& a, cudaStream_t st, uint64_t* launche
     e = cudaGetLastError();
     if (e != cudaSuccess) return note_error("k_lh_prep launch", e);
     profile_begin(st);
-    e = launch_pdl_lh(k_lh_attn, dim3(2 * p.G2), dim3(kThreads), attn_smem, st, map, p);
+    e = launch_pdl_lh(k_lh_attn, dim3(2 * p.G2), dim3(kThreads), attn_smem, st, map_k, map_v, p);
     profile_end(st);
     if (e != cudaSuccess) return note_error("k_lh_attn launch", e);
     e = launch_pdl_lh(k_lh_combine, dim3(sh.H, (sh.B + 31) / 32), dim3(kCombThreads), comb_smem, st, wuv_map, a, p);
