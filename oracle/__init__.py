@@ -40,6 +40,8 @@ FAULT_PE_BASE = 10
 FAULT_PAIR_ORDER = 11
 FAULT_ROPE_HALF_SPLIT = 12
 FAULT_PE_SWAP = 13
+FAULT_CHUNK_NO_SEED = 14
+FAULT_CHUNK_LOCAL_POS = 15
 
 
 def build(force: bool = False) -> str:
@@ -104,6 +106,7 @@ def _load():
         _lib.orc_decode_step.argtypes = ([ctypes.POINTER(_Cfg), ctypes.c_int32] + [_P] * 9
                                          + [_PI] + [_P] * 5)
         _lib.orc_prefill_explicit.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int32] + [_P] * 10
+        _lib.orc_prefill_from.argtypes = [ctypes.POINTER(_Cfg)] + [ctypes.c_int32] * 3 + [_P] * 15
         _lib.orc_set_fault.argtypes = [ctypes.c_int]
         _lib.orc_reorder_cache.argtypes = [ctypes.c_int32] * 5 + [ctypes.c_void_p] * 6
         _lib.orc_reorder_cache.restype = ctypes.c_int
@@ -184,6 +187,28 @@ def prefill(cfg: Cfg, c, kr, qc, qr, w_uk, w_uv, G=None, g=None, gate_in=None):
     acc = np.zeros((cfg.B, cfg.D))
     _load().orc_prefill(ctypes.byref(cfg.c()), T, _p(c), _p(kr), _p(qc), _p(qr), _p(w_uk),
                         _p(w_uv), _p(G), _p(g), _p(gate_in), _p(out), _p(w), _p(cache), _p(acc))
+    return dict(out=out, w=w, cache=cache, acc=acc)
+
+
+def prefill_from(cfg: Cfg, t0: int, cache_in, acc_in, c, kr, qc, qr, w_uk, w_uv, G=None, g=None,
+                 gate_in=None):
+    """Chunked prefill: T new tokens at positions t0.. continuing from the state
+    after t0 tokens (``cache_in`` [B, >= floor(t0/s), D], ``acc_in`` [B, D]).
+    Returns dict(out [B,T,H,d_h], w [B,T], cache [B, ceil((t0+T)/s), D], acc [B,D])."""
+    c, kr, qc, qr, w_uk, w_uv = map(_d, (c, kr, qc, qr, w_uk, w_uv))
+    G, g, gate_in = _d(G), _d(g), _d(gate_in)
+    cache_in, acc_in = _d(cache_in), _d(acc_in)
+    T = c.shape[1]
+    n_in = cache_in.shape[1]
+    assert n_in >= t0 // cfg.s
+    n_out = (t0 + T + cfg.s - 1) // cfg.s
+    out = np.zeros((cfg.B, T, cfg.H, cfg.d_h))
+    w = np.zeros((cfg.B, T))
+    cache = np.zeros((cfg.B, n_out, cfg.D))
+    acc = np.zeros((cfg.B, cfg.D))
+    _load().orc_prefill_from(ctypes.byref(cfg.c()), int(t0), T, n_in, _p(cache_in), _p(acc_in), _p(c),
+                             _p(kr), _p(qc), _p(qr), _p(w_uk), _p(w_uv), _p(G), _p(g), _p(gate_in),
+                             _p(out), _p(w), _p(cache), _p(acc))
     return dict(out=out, w=w, cache=cache, acc=acc)
 
 

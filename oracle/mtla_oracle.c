@@ -83,6 +83,8 @@ enum {
     ORC_FAULT_PAIR_ORDER = 11,       /* frequencies of pairs k >= 1 reversed */
     ORC_FAULT_ROPE_HALF_SPLIT = 12,  /* RoPE pairs (x_k, x_{k+d/2})          */
     ORC_FAULT_PE_SWAP = 13,          /* PE with cos at even, sin at odd      */
+    ORC_FAULT_CHUNK_NO_SEED = 14,    /* chunked prefill: open block restarts  */
+    ORC_FAULT_CHUNK_LOCAL_POS = 15,  /* chunked prefill: positions from 0     */
 };
 static int orc_fault = ORC_FAULT_NONE;
 void orc_set_fault(int f) { orc_fault = f; }
@@ -314,6 +316,94 @@ void orc_prefill(const orc_cfg* cfg, int32_t T, const double* c, const double* k
             memcpy(&acc[(int64_t)b * D], &P[((int64_t)b * T + T - 1) * D], sizeof(double) * D);
     }
     free(rows);
+    free(P);
+}
+
+/* Parallel forward over T new tokens at positions t0 .. t0+T-1 that continues
+ * from the state after t0 tokens (chunked prefill): the finished slots
+ * F_0 .. F_{floor(t0/s)-1} are cache_in's, and the block open at t0 (when t0 is
+ * not a multiple of s) continues from acc_in = P_{t0-1}:
+ *   P_i = [s*floor(i/s) < t0 ? acc_in : 0] + sum_{u = max(t0, s*floor(i/s))}^{i} w_u x_u.
+ * Query i attends F_j, j < floor(i/s) (cache_in's for j < floor(t0/s), the new
+ * block ends otherwise), plus P_i -- the same mask and the same sums as the
+ * parallel form over all t0+T tokens (MTLA Sec. 4.2).
+ *   cache_in [B,n_in,D] (n_in >= floor(t0/s))   acc_in [B,D]
+ *   c [B,T,d_c] kr [B,T,d_r] qc [B,T,H,d_h] qr [B,T,H,d_r] gate_in [B,T]: the new tokens
+ *   out [B,T,H,d_h]; w [B,T]; cache_out [B,ceil((t0+T)/s),D] = the cache after
+ *   t0+T tokens (cache_in's finished slots, then the new ones); acc_out [B,D]. */
+void orc_prefill_from(const orc_cfg* cfg, int32_t t0, int32_t T, int32_t n_in, const double* cache_in,
+                      const double* acc_in, const double* c, const double* kr, const double* qc,
+                      const double* qr, const double* w_uk, const double* w_uv, const double* G,
+                      const double* g, const double* gate_in, double* out, double* w, double* cache_out,
+                      double* acc_out) {
+    const int32_t B = cfg->B, H = cfg->H, d_h = cfg->d_h, d_c = cfg->d_c, d_r = cfg->d_r, s = cfg->s;
+    const int32_t D = d_c + d_r;
+    const int32_t nf0 = t0 / s;                         /* finished slots before the chunk */
+    const int32_t n_out = (t0 + T + s - 1) / s;
+    double* P = (double*)malloc(sizeof(double) * (size_t)B * T * D);
+    /* gates, then the partial slots of the new positions (local index i - t0) */
+    for (int32_t b = 0; b < B; ++b)
+        for (int32_t li = 0; li < T; ++li) {
+            const double* wg = gate_in ? &gate_in[(int64_t)b * T + li] : NULL;
+            w[(int64_t)b * T + li] = orc_gate(cfg, t0 + li, &c[((int64_t)b * T + li) * d_c], G, g, wg);
+        }
+#pragma omp parallel for schedule(static)
+    for (int64_t bl = 0; bl < (int64_t)B * T; ++bl) {
+        const int32_t b = (int32_t)(bl / T), li = (int32_t)(bl % T), i = t0 + li;
+        double* x = (double*)malloc(sizeof(double) * D);
+        double* o = &P[bl * D];
+        int32_t u0 = s * (i / s);
+        if (orc_fault == ORC_FAULT_SCAN_NO_RESET) u0 = 0;
+        const int seeded = u0 < t0 && orc_fault != ORC_FAULT_CHUNK_NO_SEED;
+        for (int32_t k = 0; k < D; ++k) o[k] = seeded ? acc_in[(int64_t)b * D + k] : 0.0;
+        for (int32_t u = u0 < t0 ? t0 : u0; u <= i; ++u) {
+            const int64_t bu = (int64_t)b * T + (u - t0);
+            const int32_t tu = orc_fault == ORC_FAULT_CHUNK_LOCAL_POS ? u - t0 : u;
+            orc_token_vector(cfg, tu, &c[bu * d_c], &kr[bu * d_r], x);
+            for (int32_t k = 0; k < D; ++k) o[k] += w[bu] * x[k];
+        }
+        free(x);
+    }
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t blh = 0; blh < (int64_t)B * T * H; ++blh) {
+        const int32_t h = (int32_t)(blh % H), li = (int32_t)((blh / H) % T), b = (int32_t)(blh / ((int64_t)H * T));
+        const int32_t i = t0 + li;
+        double* qt = (double*)malloc(sizeof(double) * D);
+        double* olat = (double*)malloc(sizeof(double) * d_c);
+        const double** keys = (const double**)malloc(sizeof(double*) * (size_t)(i / s + 2));
+        int64_t n = 0;
+        int32_t nf = i / s;
+        if (orc_fault == ORC_FAULT_MASK_OFF_BY_ONE) nf = i / s + 1;
+        for (int32_t j = 0; j < nf; ++j) {
+            if (j < nf0) {
+                keys[n++] = &cache_in[((int64_t)b * n_in + j) * D];
+            } else {
+                int32_t u = j * s + s - 1;
+                if (u > t0 + T - 1) u = t0 + T - 1;
+                keys[n++] = &P[((int64_t)b * T + (u - t0)) * D];
+            }
+        }
+        if (orc_fault != ORC_FAULT_DROP_OWN_PARTIAL) keys[n++] = &P[((int64_t)b * T + li) * D];
+        orc_absorb_query(cfg, i, h, &qc[blh * d_h], &qr[blh * d_r], w_uk, qt);
+        orc_attend_keys(cfg, qt, n, keys, olat);
+        orc_output(cfg, h, olat, w_uv, &out[blh * d_h]);
+        free(keys);
+        free(olat);
+        free(qt);
+    }
+    for (int32_t b = 0; b < B; ++b) {
+        for (int32_t j = 0; j < n_out; ++j) {
+            double* dst = &cache_out[((int64_t)b * n_out + j) * D];
+            if (j < nf0) {
+                memcpy(dst, &cache_in[((int64_t)b * n_in + j) * D], sizeof(double) * D);
+            } else {
+                int32_t u = j * s + s - 1;
+                if (u > t0 + T - 1) u = t0 + T - 1;
+                memcpy(dst, &P[((int64_t)b * T + (u - t0)) * D], sizeof(double) * D);
+            }
+        }
+        memcpy(&acc_out[(int64_t)b * D], &P[((int64_t)b * T + T - 1) * D], sizeof(double) * D);
+    }
     free(P);
 }
 

@@ -13,7 +13,10 @@ mathematics fix, none of which retypes the oracle's own formulas.
 - brute force: dense enumerated mask over per-token partial slots (tests/brute_force.py);
 - closed forms of the scan, the gate modes, PE and RoPE;
 - exact values of the adopted PE / RoPE readings at width 8 (pair frequencies
-  exactly 1, 0.1, 0.01, 0.001 at base 10000) and one gate worked by hand.
+  exactly 1, 0.1, 0.01, 0.001 at base 10000) and one gate worked by hand;
+- chunked prefill: from position 0 it is the parallel forward; a prefix then a
+  chunk equals one prefill (split points inside a block included); a chunk
+  equals the same number of incremental decode steps.
 Finally, each planted mistake in the oracle must trip at least one pin.
 """
 import math
@@ -312,6 +315,80 @@ def pin_gate_value():
     return abs(oracle.gate(cfg, 3, c, G, g) - 1.0 / (1.0 + math.exp(-z))) < 1e-14
 
 
+def _prefix_state(cfg, p, t0):
+    """Cache and open slot after the first t0 tokens (parallel form)."""
+    if t0 == 0:
+        return np.zeros((cfg.B, 0, cfg.D)), np.zeros((cfg.B, cfg.D))
+    r = oracle.prefill(cfg, p["c"][:, :t0], p["kr"][:, :t0], p["qc"][:, :t0], p["qr"][:, :t0],
+                       p["w_uk"], p["w_uv"], p["G"], p["g"])
+    return r["cache"], r["acc"]
+
+
+def _chunk(p, t0):
+    return {k: p[k][:, t0:] for k in ("c", "kr", "qc", "qr")}
+
+
+def pin_prefill_from_start_is_prefill():
+    """Chunked prefill from t0 = 0 is the parallel forward itself."""
+    for s in (1, 3):
+        cfg, p = _rand_problem(2, 2, 8, 16, 4, s, 10, seed=70 + s)
+        ref = oracle.prefill(cfg, p["c"], p["kr"], p["qc"], p["qr"], p["w_uk"], p["w_uv"], p["G"], p["g"])
+        cache0, acc0 = _prefix_state(cfg, p, 0)
+        got = oracle.prefill_from(cfg, 0, cache0, acc0, p["c"], p["kr"], p["qc"], p["qr"], p["w_uk"],
+                                  p["w_uv"], p["G"], p["g"])
+        for k in ("out", "cache", "acc", "w"):
+            if not np.max(np.abs(got[k] - ref[k])) < 1e-12:
+                return False
+    return True
+
+
+def pin_prefill_chunks_compose():
+    """Prefill of t0 tokens, then a chunk of T tokens from the resulting cache
+    and open slot, equals one prefill of t0 + T tokens (its last T rows, its
+    cache and open slot): the stride-aware mask makes the parallel form
+    split anywhere, inside a block included (MTLA Sec. 4.2)."""
+    for s in (1, 2, 3, 4):
+        total = 17
+        cfg, p = _rand_problem(2, 2, 8, 16, 4, s, total, seed=80 + s)
+        full = oracle.prefill(cfg, p["c"], p["kr"], p["qc"], p["qr"], p["w_uk"], p["w_uv"], p["G"], p["g"])
+        for t0 in sorted({1, s, 2 * s + 1, 7, 16}):
+            cache0, acc0 = _prefix_state(cfg, p, t0)
+            ch = _chunk(p, t0)
+            got = oracle.prefill_from(cfg, t0, cache0, acc0, ch["c"], ch["kr"], ch["qc"], ch["qr"],
+                                      p["w_uk"], p["w_uv"], p["G"], p["g"])
+            if not (np.max(np.abs(got["out"] - full["out"][:, t0:])) < 1e-12
+                    and np.max(np.abs(got["cache"] - full["cache"])) < 1e-12
+                    and np.max(np.abs(got["acc"] - full["acc"])) < 1e-12):
+                return False
+    return True
+
+
+def pin_prefill_from_equals_decode_steps():
+    """A chunk of T tokens from a cache state equals T incremental decode steps
+    from the same state (outputs, cache, open slot)."""
+    for s in (2, 3):
+        t0, T = 5, 8
+        cfg, p = _rand_problem(2, 2, 8, 16, 4, s, t0 + T, seed=90 + s)
+        cache0, acc0 = _prefix_state(cfg, p, t0)
+        ch = _chunk(p, t0)
+        got = oracle.prefill_from(cfg, t0, cache0, acc0, ch["c"], ch["kr"], ch["qc"], ch["qr"],
+                                  p["w_uk"], p["w_uv"], p["G"], p["g"])
+        max_slots = (t0 + T + s - 1) // s
+        cache = np.zeros((cfg.B, max_slots, cfg.D))
+        cache[:, :cache0.shape[1]] = cache0
+        acc = acc0.copy()
+        outs = []
+        for k in range(T):
+            r = oracle.decode_step(cfg, ch["c"][:, k], ch["kr"][:, k], ch["qc"][:, k], ch["qr"][:, k],
+                                   p["w_uk"], p["w_uv"], np.full(cfg.B, t0 + k), cache, acc, p["G"], p["g"])
+            outs.append(r["out"])
+        if not (np.max(np.abs(np.stack(outs, axis=1) - got["out"])) < 1e-12
+                and np.max(np.abs(cache - got["cache"])) < 1e-12
+                and np.max(np.abs(acc - got["acc"])) < 1e-12):
+            return False
+    return True
+
+
 PINS = {
     "cache_footprint": pin_cache_footprint,
     "s1_is_mla_sdpa": pin_s1_is_mla_sdpa,
@@ -325,6 +402,9 @@ PINS = {
     "pe_values": pin_pe_values,
     "rope_values": pin_rope_values,
     "gate_value": pin_gate_value,
+    "prefill_from_start_is_prefill": pin_prefill_from_start_is_prefill,
+    "prefill_chunks_compose": pin_prefill_chunks_compose,
+    "prefill_from_equals_decode_steps": pin_prefill_from_equals_decode_steps,
 }
 
 
@@ -354,6 +434,8 @@ FAULTS = {
     "pair_order": oracle.FAULT_PAIR_ORDER,
     "rope_half_split": oracle.FAULT_ROPE_HALF_SPLIT,
     "pe_swap": oracle.FAULT_PE_SWAP,
+    "chunk_no_seed": oracle.FAULT_CHUNK_NO_SEED,
+    "chunk_local_pos": oracle.FAULT_CHUNK_LOCAL_POS,
 }
 
 
