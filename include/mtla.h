@@ -169,6 +169,36 @@ mtla_status mtla_prefill(const mtla_config* cfg, int32_t T,
                          void* out, void* cache_out, float* open_slot_out,
                          void* workspace, size_t workspace_bytes, void* stream);
 
+/* Chunked prefill: the parallel forward over T new tokens at positions
+ * t0 .. t0+T-1 of every sequence, continuing from the cache state after t0
+ * tokens (a long prompt processed in chunks, or a prompt appended to a
+ * conversation whose cache exists). MTLA Method (1)-(3): the stride-aware
+ * mask lets position i see every finished slot j < floor(i/s) -- those already
+ * in the cache and those this chunk completes -- plus its own partial slot; a
+ * slot left open at t0 (t0 mod s != 0) continues from the open-slot
+ * accumulator, exactly as the in-place update of decoding would continue it.
+ * The result equals T calls of mtla_decode_step from the same state, and
+ * mtla_prefill over t0+T tokens equals mtla_prefill over t0 followed by this.
+ *
+ *   t0        tokens already in the cache, the same for every sequence (>= 0)
+ *   c, kr, q_c, q_r, gate_in   the new tokens only: [B,T,...] as for mtla_prefill
+ *   cache     [B, max_slots, d_c+d_r] dtype, in/out: slots 0 .. ceil(t0/s)-1
+ *             hold the state after t0 tokens; slots floor(t0/s) ..
+ *             ceil((t0+T)/s)-1 are written (the first may be the open one);
+ *             requires ceil((t0+T)/s) <= max_slots (else CAPACITY).
+ *   open_slot [B, d_c+d_r] fp32, in/out, not NULL: the accumulator after t0
+ *             tokens (read when t0 mod s != 0), then after t0+T tokens.
+ *   out, weights, workspace: as for mtla_prefill (mtla_workspace_size with
+ *             max_tokens >= T covers it).
+ * t0 = 0 is mtla_prefill with cache_out = cache. Returns OK once enqueued. */
+mtla_status mtla_prefill_from(const mtla_config* cfg, int32_t t0, int32_t T,
+                              const void* c, const void* kr,
+                              const void* q_c, const void* q_r,
+                              const void* w_uk, const void* w_uv,
+                              const float* gate_w, const float* gate_b, const float* gate_in,
+                              void* out, void* cache, float* open_slot,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
 /* Decode step without a workspace argument, for callers that cannot allocate
  * device memory themselves: code inside a host framework whose pool allocator
  * owns all device memory and forbids raw cudaMalloc, serving loops that cannot

@@ -158,6 +158,16 @@ static mtla_status check_gate_ptrs(const mtla_config* cfg, const float* gate_w, 
     return MTLA_OK;
 }
 
+size_t prefill_seed_bytes(const Shape& sh) { return align256((size_t)sh.B * sh.D * sizeof(float)); }
+
+cudaError_t prefill_seed(PrefillArgs& a, void* seed_ws, cudaStream_t st) {
+    if (!a.open_slot_in) return cudaSuccess;
+    cudaError_t e = cudaMemcpyAsync(seed_ws, a.open_slot_in, (size_t)a.sh.B * a.sh.D * sizeof(float),
+                                    cudaMemcpyDeviceToDevice, st);
+    a.open_slot_in = (const float*)seed_ws;
+    return note_error("prefill open-slot copy", e);
+}
+
 }  // namespace mtla
 
 using namespace mtla;
@@ -217,26 +227,29 @@ mtla_status mtla_decode_step(const mtla_config* cfg, const void* c_new, const vo
     return e == cudaSuccess ? MTLA_OK : MTLA_ERR_CUDA;
 }
 
-mtla_status mtla_prefill(const mtla_config* cfg, int32_t T, const void* c, const void* kr,
-                         const void* q_c, const void* q_r, const void* w_uk, const void* w_uv,
-                         const float* gate_w, const float* gate_b, const float* gate_in, void* out,
-                         void* cache_out, float* open_slot_out, void* workspace,
-                         size_t workspace_bytes, void* stream) {
+static mtla_status prefill_common(const mtla_config* cfg, int32_t t0, int32_t T, const void* c, const void* kr,
+                                  const void* q_c, const void* q_r, const void* w_uk, const void* w_uv,
+                                  const float* gate_w, const float* gate_b, const float* gate_in, void* out,
+                                  void* cache, const float* open_in, float* open_out, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
     Shape sh;
     mtla_status st = check_config(cfg, &sh);
     if (st != MTLA_OK) return st;
-    if (T <= 0) return MTLA_ERR_INVALID_ARG;
-    const void* req[] = {c, kr, q_c, q_r, w_uk, w_uv, out, cache_out, workspace};
+    if (T <= 0 || t0 < 0) return MTLA_ERR_INVALID_ARG;
+    const void* req[] = {c, kr, q_c, q_r, w_uk, w_uv, out, cache, workspace};
     for (const void* p : req)
         if (!p || !aligned16(p)) return MTLA_ERR_INVALID_ARG;
-    if (open_slot_out && !aligned16(open_slot_out)) return MTLA_ERR_INVALID_ARG;
+    if (open_out && !aligned16(open_out)) return MTLA_ERR_INVALID_ARG;
+    if (t0 % sh.s != 0 && (!open_in || !aligned16(open_in))) return MTLA_ERR_INVALID_ARG;
     st = check_gate_ptrs(cfg, gate_w, gate_b, gate_in);
     if (st != MTLA_OK) return st;
-    if ((int64_t)(T + sh.s - 1) / sh.s > sh.max_slots) return MTLA_ERR_CAPACITY;
+    if (((int64_t)t0 + T + sh.s - 1) / sh.s > sh.max_slots) return MTLA_ERR_CAPACITY;
     if (workspace_bytes < prefill_ws(cfg, sh, T)) return MTLA_ERR_WORKSPACE;
     PrefillArgs a;
     a.sh = sh;
     a.T = T;
+    a.t0 = t0;
+    a.open_slot_in = t0 % sh.s != 0 ? open_in : nullptr;
     a.c = c;
     a.kr = kr;
     a.q_c = q_c;
@@ -247,8 +260,8 @@ mtla_status mtla_prefill(const mtla_config* cfg, int32_t T, const void* c, const
     a.gate_b = gate_b;
     a.gate_in = gate_in;
     a.out = out;
-    a.cache_out = cache_out;
-    a.open_slot_out = open_slot_out;
+    a.cache_out = cache;
+    a.open_slot_out = open_out;
     a.workspace = workspace;
     a.workspace_bytes = workspace_bytes;
     g_error_detail[0] = 0;
@@ -259,6 +272,25 @@ mtla_status mtla_prefill(const mtla_config* cfg, int32_t T, const void* c, const
     g_launches += n;
     if (e != cudaSuccess && !g_error_detail[0]) note_error("prefill launch", e);
     return e == cudaSuccess ? MTLA_OK : MTLA_ERR_CUDA;
+}
+
+mtla_status mtla_prefill(const mtla_config* cfg, int32_t T, const void* c, const void* kr,
+                         const void* q_c, const void* q_r, const void* w_uk, const void* w_uv,
+                         const float* gate_w, const float* gate_b, const float* gate_in, void* out,
+                         void* cache_out, float* open_slot_out, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+    return prefill_common(cfg, 0, T, c, kr, q_c, q_r, w_uk, w_uv, gate_w, gate_b, gate_in, out, cache_out,
+                          nullptr, open_slot_out, workspace, workspace_bytes, stream);
+}
+
+mtla_status mtla_prefill_from(const mtla_config* cfg, int32_t t0, int32_t T, const void* c, const void* kr,
+                              const void* q_c, const void* q_r, const void* w_uk, const void* w_uv,
+                              const float* gate_w, const float* gate_b, const float* gate_in, void* out,
+                              void* cache, float* open_slot, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+    if (!open_slot) return MTLA_ERR_INVALID_ARG;
+    return prefill_common(cfg, t0, T, c, kr, q_c, q_r, w_uk, w_uv, gate_w, gate_b, gate_in, out, cache,
+                          open_slot, open_slot, workspace, workspace_bytes, stream);
 }
 
 mtla_status mtla_get_device_status(void* stream) {

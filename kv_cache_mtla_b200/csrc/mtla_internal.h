@@ -38,6 +38,8 @@ struct DecodeArgs {
 struct PrefillArgs {
     Shape sh;
     int T;
+    int t0;                     // position of the first token (tokens already cached)
+    const float* open_slot_in;  // [B, D] the open-slot accumulator after t0 tokens (t0 mod s != 0)
     const void* c;
     const void* kr;
     const void* q_c;
@@ -54,6 +56,13 @@ struct PrefillArgs {
     size_t workspace_bytes;
     int* status;
 };
+
+// Chunked prefill (t0 mod s != 0): the open-slot accumulator the chunk starts
+// from is copied into `seed_ws` (the last region of the prefill workspace,
+// prefill_seed_bytes long) before the scan, which may overwrite the caller's
+// open slot; a.open_slot_in then points at the copy. No-op otherwise.
+size_t prefill_seed_bytes(const Shape& sh);
+cudaError_t prefill_seed(PrefillArgs& a, void* seed_ws, cudaStream_t st);
 
 // Scratch layouts (bytes), each region 256-byte aligned.
 size_t simt_decode_workspace(const Shape& sh);

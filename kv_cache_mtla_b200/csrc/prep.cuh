@@ -219,12 +219,12 @@ __global__ void __launch_bounds__(128) k_decode_prep(DecodeArgs a, float* qt) {
     absorb_query_body<T>(sh, (const T*)a.q_c, (const T*)a.q_r, (const T*)a.w_uk, b, h, t, qt);
 }
 
-// Prefill absorption: grid (B*T, H); row = b*T + t.
+// Prefill absorption: grid (B*T, H); row = b*T + t, position t0 + t.
 template <typename T>
 __global__ void __launch_bounds__(128) k_prefill_absorb(Shape sh, const T* qc, const T* qr, const T* w_uk,
-                                                        int T_len, float* qt) {
+                                                        int T_len, int t0, float* qt) {
     const int64_t row = blockIdx.x;
-    absorb_query_body<T>(sh, qc, qr, w_uk, row, blockIdx.y, row % T_len, qt);
+    absorb_query_body<T>(sh, qc, qr, w_uk, row, blockIdx.y, t0 + row % T_len, qt);
 }
 
 // 8 consecutive values as float (T = float or bf16; 16-byte aligned address).
@@ -257,8 +257,12 @@ template <> __device__ __forceinline__ void store8<bf16>(bf16* p, const float* v
 // weights w_u (Sec. 4.1, Eq. 13) of its tokens u and the partial slots
 //   P_u = sum_{v = s*j}^{u} w_v [c_v ; RoPE_v(k_v)]
 // (stored as PT), the slot itself in the cache (rounded to T: finished, or the
-// last one) and, for the slot holding token T-1, the unrounded open slot.
-// One warp per slot: grid (ceil(ceil(T/s) / 8), B), 256 threads.
+// last one) and, for the slot holding the last token, the unrounded open slot.
+// The tokens are t0 .. t0+T-1 (absolute positions; inputs, P and the (cos,
+// sin) table are indexed from t0): the slots are floor(t0/s) .. and the one
+// open at t0, if t0 is not a multiple of s, starts from open_slot_in (the
+// accumulator after t0 tokens) instead of 0.
+// One warp per slot: grid (ceil(n / 8), B), n = slots touched, 256 threads.
 // With bf16 partial slots (the tensor-core prefill) the sine and cosine of the
 // angle, reduced to [-pi, pi] in double as everywhere, come from the special-
 // function unit (absolute error about 2^-21 there, far below the bf16 rounding
@@ -286,22 +290,26 @@ __global__ void __launch_bounds__(256) k_prefill_scan(PrefillArgs a, PT* P, floa
     for (int k = threadIdx.x; k < sh.d_r / 2; k += blockDim.x)
         rope_freq[k] = exp2(-(2.0 * k / (double)sh.d_r) * sh.log2_rope_base);
     __syncthreads();
-    const int n_slots = (Tn + sh.s - 1) / sh.s;
-    const int j = blockIdx.x * 8 + warp;
-    if (j >= n_slots) return;
-    const int u0 = j * sh.s, nu = min(sh.s, Tn - u0);
-    const T* c = (const T*)a.c + ((size_t)b * Tn + u0) * sh.d_c;
-    const T* kr = (const T*)a.kr + ((size_t)b * Tn + u0) * sh.d_r;
+    const int t0 = a.t0;
+    const int j_first = t0 / sh.s, j_end = (t0 + Tn - 1) / sh.s + 1;
+    const int j = j_first + blockIdx.x * 8 + warp;
+    if (j >= j_end) return;
+    // this slot's new tokens: absolute positions ua .. ua + nu - 1, local index lu0 ..
+    const int ua = max(j * sh.s, t0), nu = min((j + 1) * sh.s, t0 + Tn) - ua;
+    const int lu0 = ua - t0;
+    const float* seed = (j * sh.s < t0 && a.open_slot_in) ? a.open_slot_in + (size_t)b * sh.D : nullptr;
+    const T* c = (const T*)a.c + ((size_t)b * Tn + lu0) * sh.d_c;
+    const T* kr = (const T*)a.kr + ((size_t)b * Tn + lu0) * sh.d_r;
     float wv[8];
 #pragma unroll
     for (int uo = 0; uo < 8; ++uo) {
         wv[uo] = 0.f;
         if (uo >= nu) continue;
-        const int u = u0 + uo;
+        const int u = ua + uo;
         if (sh.gate_mode == 2) {
             wv[uo] = 1.f;
         } else if (sh.gate_mode == 1) {
-            wv[uo] = a.gate_in[(size_t)b * Tn + u];
+            wv[uo] = a.gate_in[(size_t)b * Tn + lu0 + uo];
         } else {
             const int r = u % sh.s;
             const float* G = a.gate_w + (size_t)r * sh.d_c;
@@ -317,10 +325,11 @@ __global__ void __launch_bounds__(256) k_prefill_scan(PrefillArgs a, PT* P, floa
         }
     }
     T* slot = (T*)a.cache_out + ((size_t)b * sh.max_slots + j) * sh.D;
-    float* open = (u0 + nu == Tn && a.open_slot_out) ? a.open_slot_out + (size_t)b * sh.D : nullptr;
-    PT* Pj = P + ((size_t)b * Tn + u0) * sh.D;
+    float* open = (ua + nu == t0 + Tn && a.open_slot_out) ? a.open_slot_out + (size_t)b * sh.D : nullptr;
+    PT* Pj = P + ((size_t)b * Tn + lu0) * sh.D;
     for (int k0 = lane * 8; k0 < sh.d_c; k0 += 256) {
         float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        if (seed) load8<float>(seed + k0, acc);
 #pragma unroll
         for (int uo = 0; uo < 8; ++uo) {
             if (uo >= nu) continue;
@@ -334,14 +343,14 @@ __global__ void __launch_bounds__(256) k_prefill_scan(PrefillArgs a, PT* P, floa
         if (open) store8<float>(open + k0, acc);
     }
     for (int k = lane; k < sh.d_r / 2; k += 32) {
-        float a0 = 0.f, a1 = 0.f;
+        float a0 = seed ? seed[sh.d_c + 2 * k] : 0.f, a1 = seed ? seed[sh.d_c + 2 * k + 1] : 0.f;
 #pragma unroll
         for (int uo = 0; uo < 8; ++uo) {
             if (uo >= nu) continue;
             float sn, cs;
-            sincos_at(u0 + uo, rope_freq[k], &sn, &cs);
+            sincos_at(ua + uo, rope_freq[k], &sn, &cs);
             // (cos, sin) of every position for the queries' RoPE (sequence 0 writes it)
-            if (rope_tab && b == 0) rope_tab[(size_t)(u0 + uo) * (sh.d_r / 2) + k] = make_float2(cs, sn);
+            if (rope_tab && b == 0) rope_tab[(size_t)(lu0 + uo) * (sh.d_r / 2) + k] = make_float2(cs, sn);
             const float x0 = to_f<T>(kr[(size_t)uo * sh.d_r + 2 * k]);
             const float x1 = to_f<T>(kr[(size_t)uo * sh.d_r + 2 * k + 1]);
             a0 = fmaf(wv[uo], x0 * cs - x1 * sn, a0);

@@ -166,7 +166,7 @@ __global__ void __launch_bounds__(256) k_prefill_attn(PrefillArgs a, const float
 #pragma unroll
     for (int i = 0; i < kMaxLatPerLane; ++i) st.o[i] = 0.f;
     const T* cache = (const T*)a.cache_out + (size_t)b * sh.max_slots * sh.D;
-    const int nf = t / sh.s;
+    const int nf = (a.t0 + t) / sh.s;          // finished slots: the cache's and this chunk's
     for (int j = 0; j < nf; ++j) row_visit<T>(st, q, cache + (size_t)j * sh.D, sh.D, sh.d_c, sh.scale);
     {
         // own partial slot, rounded to the storage type
@@ -234,15 +234,19 @@ cudaError_t decode_impl(const DecodeArgs& a, cudaStream_t st, uint64_t* launches
 }
 
 template <typename T>
-cudaError_t prefill_impl(const PrefillArgs& a, cudaStream_t st, uint64_t* launches) {
+cudaError_t prefill_impl(const PrefillArgs& a_in, cudaStream_t st, uint64_t* launches) {
+    PrefillArgs a = a_in;
     const Shape& sh = a.sh;
     char* ws = (char*)a.workspace;
     float* P = (float*)ws;
-    float* qt = (float*)(ws + align256((size_t)sh.B * a.T * sh.D * sizeof(float)));
-    const int n_slots = (a.T + sh.s - 1) / sh.s;
+    const size_t p_bytes = align256((size_t)sh.B * a.T * sh.D * sizeof(float));
+    float* qt = (float*)(ws + p_bytes);
+    cudaError_t e = prefill_seed(a, ws + p_bytes + align256((size_t)sh.B * a.T * sh.H * sh.D * sizeof(float)), st);
+    if (e != cudaSuccess) return e;
+    const int n_slots = (a.t0 + a.T - 1) / sh.s - a.t0 / sh.s + 1;    // slots the chunk touches
     k_prefill_scan<T, float><<<dim3((n_slots + 7) / 8, sh.B), 256, 0, st>>>(a, P);
     k_prefill_absorb<T><<<dim3(sh.B * a.T, sh.H), 128, 0, st>>>(sh, (const T*)a.q_c, (const T*)a.q_r,
-                                                                 (const T*)a.w_uk, a.T, qt);
+                                                                 (const T*)a.w_uk, a.T, a.t0, qt);
     const int64_t rows = (int64_t)a.T * sh.H;
     profile_begin(st);
     k_prefill_attn<T><<<dim3((unsigned)((rows + 7) / 8), sh.B), 256, 0, st>>>(a, P, qt);
@@ -262,7 +266,7 @@ size_t simt_decode_workspace(const Shape& sh) {
 
 size_t simt_prefill_workspace(const Shape& sh, int T) {
     return align256((size_t)sh.B * T * sh.D * sizeof(float)) +
-           align256((size_t)sh.B * T * sh.H * sh.D * sizeof(float));
+           align256((size_t)sh.B * T * sh.H * sh.D * sizeof(float)) + prefill_seed_bytes(sh);
 }
 
 cudaError_t simt_decode(const DecodeArgs& a, bool fp32, cudaStream_t st, uint64_t* launches) {

@@ -60,6 +60,7 @@ constexpr int kDh = 64;         // head width d_h of this kernel
 struct PreTC {
     int B, T, H, d_h, d_c, d_r, D, s;
     int n_qtiles;     // ceil(T / 128)
+    int t0;           // position of the first query (tokens already cached)
     int n_items;      // n_qtiles * B * H
     float scale_log2;
     double log2_rope_base;
@@ -130,7 +131,7 @@ __device__ __forceinline__ Item decode_item(const PreTC& p, int idx) {
     it.h = rem % p.H;
     it.p0 = qt * kQ;
     const int last = min(it.p0 + kQ - 1, p.T - 1);
-    it.nft = (last / p.s + kKT - 1) / kKT;
+    it.nft = ((p.t0 + last) / p.s + kKT - 1) / kKT;
     return it;
 }
 // The j-th item of this CTA, or -1 past the end: round j of gridDim.x items,
@@ -522,8 +523,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
             // online softmax over the finished-slot tiles; the own slot is the
             // starting point (reference maximum es, weight 1 in the row sum)
             float m_ref = es, l = hc == 0 ? 1.f : 0.f;    // l: this thread's half of the row sum
-            const int fin_lim = pos / p.s;                // finished slots this row may see
-            const int min_fin = p0 / p.s;                 // ... and the first row of the tile
+            const int fin_lim = (p.t0 + pos) / p.s;       // finished slots this row may see
+            const int min_fin = (p.t0 + p0) / p.s;        // ... and the first row of the tile
             for (int k = 0; k < nft; ++k, ++G) {
                 waitb(&bs.s_full[G & 1], (G >> 1) & 1, bs);
                 tc_fence_after();
@@ -696,13 +697,21 @@ bool tc_prefill_supported(const Shape& sh) {
 }
 
 size_t tc_prefill_workspace(const Shape& sh, int T) {
-    return align256((size_t)sh.B * T * sh.D * sizeof(bf16)) + align256((size_t)T * (sh.d_r / 2) * sizeof(float2));
+    return align256((size_t)sh.B * T * sh.D * sizeof(bf16)) + align256((size_t)T * (sh.d_r / 2) * sizeof(float2)) +
+           prefill_seed_bytes(sh);
 }
 
-cudaError_t tc_prefill(const PrefillArgs& a, cudaStream_t st, uint64_t* launches) {
+cudaError_t tc_prefill(const PrefillArgs& a_in, cudaStream_t st, uint64_t* launches) {
+    PrefillArgs a = a_in;
     const Shape& sh = a.sh;
     const int T = a.T;
     bf16* P = (bf16*)a.workspace;
+    {
+        const size_t off = align256((size_t)sh.B * T * sh.D * sizeof(bf16)) +
+                           align256((size_t)T * (sh.d_r / 2) * sizeof(float2));
+        cudaError_t e = prefill_seed(a, (char*)a.workspace + off, st);
+        if (e != cudaSuccess) return e;
+    }
     auto enc = (PFN_cuTensorMapEncodeTiled_v12000)tensor_map_encoder();
     if (!enc) return note_error("cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", cudaErrorNotSupported);
     Maps maps;
@@ -723,7 +732,8 @@ cudaError_t tc_prefill(const PrefillArgs& a, cudaStream_t st, uint64_t* launches
         if (e != cudaSuccess) return e;
     }
     {
-        const int n_slots = (T + sh.s - 1) / sh.s;
+        // the cache through slot ceil((t0 + T) / s) - 1: the earlier chunks' and this one's
+        const int n_slots = (a.t0 + T + sh.s - 1) / sh.s;
         cuuint64_t d[3] = {(cuuint64_t)sh.D, (cuuint64_t)n_slots, (cuuint64_t)sh.B};
         cuuint64_t s[2] = {E * sh.D, E * sh.max_slots * sh.D};
         cuuint32_t bx[3] = {64, kKT, 1};
@@ -754,6 +764,7 @@ cudaError_t tc_prefill(const PrefillArgs& a, cudaStream_t st, uint64_t* launches
     p.D = sh.D;
     p.s = sh.s;
     p.n_qtiles = (T + kQ - 1) / kQ;
+    p.t0 = a.t0;
     p.n_items = p.n_qtiles * sh.B * sh.H;
     p.scale_log2 = sh.scale * 1.4426950408889634f;
     p.log2_rope_base = sh.log2_rope_base;
@@ -762,7 +773,7 @@ cudaError_t tc_prefill(const PrefillArgs& a, cudaStream_t st, uint64_t* launches
     p.out = (bf16*)a.out;
     p.status = a.status;
 
-    const int n_slots = (T + sh.s - 1) / sh.s;
+    const int n_slots = (a.t0 + T - 1) / sh.s - a.t0 / sh.s + 1;    // slots the chunk touches
     k_prefill_scan<bf16, bf16><<<dim3((n_slots + 7) / 8, sh.B), 256, 0, st>>>(a, P, (float2*)p.rope_tab);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return note_error("k_prefill_scan launch", e);

@@ -73,6 +73,8 @@ def load() -> ctypes.CDLL:
     lib.mtla_decode_step.restype = ctypes.c_int
     lib.mtla_prefill.argtypes = [cp, ctypes.c_int32] + [_vp] * 12 + [_vp, ctypes.c_size_t, _vp]
     lib.mtla_prefill.restype = ctypes.c_int
+    lib.mtla_prefill_from.argtypes = [cp, ctypes.c_int32, ctypes.c_int32] + [_vp] * 12 + [_vp, ctypes.c_size_t, _vp]
+    lib.mtla_prefill_from.restype = ctypes.c_int
     lib.mtla_decode_step_noalloc.argtypes = [cp] + [_vp] * 13 + [_vp]
     lib.mtla_decode_step_noalloc.restype = ctypes.c_int
     lib.mtla_reorder_cache.argtypes = [cp] + [_vp] * 6 + [_vp]
@@ -162,6 +164,21 @@ def prefill(cfg, T, c, kr, q_c, q_r, w_uk, w_uv, gate_w, gate_b, gate_in, out, c
         _ptr(open_slot_out), _ptr(workspace), ws, _stream(stream))
     if check and st != OK:
         raise MtlaError(st, "mtla_prefill")
+    return st
+
+
+def prefill_from(cfg, t0, T, c, kr, q_c, q_r, w_uk, w_uv, gate_w, gate_b, gate_in, out, cache,
+                 open_slot, workspace, stream=None, check=True) -> int:
+    """Forward to ``mtla_prefill_from`` (chunked prefill of T tokens at
+    positions t0.. continuing from ``cache`` / ``open_slot``, both in/out);
+    returns the status (raises if check)."""
+    ws = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = load().mtla_prefill_from(
+        ctypes.byref(cfg), int(t0), int(T), _ptr(c), _ptr(kr), _ptr(q_c), _ptr(q_r), _ptr(w_uk),
+        _ptr(w_uv), _ptr(gate_w), _ptr(gate_b), _ptr(gate_in), _ptr(out), _ptr(cache),
+        _ptr(open_slot), _ptr(workspace), ws, _stream(stream))
+    if check and st != OK:
+        raise MtlaError(st, "mtla_prefill_from")
     return st
 
 

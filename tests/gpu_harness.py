@@ -2,6 +2,8 @@
 through the binding, and compare with the oracle."""
 from __future__ import annotations
 
+import os
+
 import numpy as np
 import torch
 
@@ -11,12 +13,32 @@ from kv_cache_mtla_b200 import inputs, mtla
 TOL = {"bf16": 2e-2, "fp32": 1e-5}
 
 
+# (test, max-relative error, elementwise error) of every comparison, written
+# out by conftest.py when MTLA_PARITY_LOG names a file
+MARGINS = []
+
+
 def rel_err(gpu, ref) -> float:
-    """max |gpu - ref| / max |ref| over the whole tensor."""
+    """max |gpu - ref| / max |ref| over the whole tensor. Also records the
+    elementwise relative error max |gpu - ref| / max(|ref|, 1e-3 max |ref|)."""
     gpu = np.asarray(gpu, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     denom = np.max(np.abs(ref))
-    return float(np.max(np.abs(gpu - ref)) / (denom if denom > 0 else 1.0))
+    denom = denom if denom > 0 else 1.0
+    diff = np.abs(gpu - ref)
+    rel = float(np.max(diff) / denom)
+    elem = float(np.max(diff / np.maximum(np.abs(ref), 1e-3 * denom)))
+    MARGINS.append((os.environ.get("PYTEST_CURRENT_TEST", "").split(" ")[0], rel, elem))
+    return rel
+
+
+def elem_err(gpu, ref) -> float:
+    """Elementwise relative error max |gpu - ref| / max(|ref|, 1e-3 max |ref|)."""
+    gpu = np.asarray(gpu, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    denom = np.max(np.abs(ref))
+    denom = denom if denom > 0 else 1.0
+    return float(np.max(np.abs(gpu - ref) / np.maximum(np.abs(ref), 1e-3 * denom)))
 
 
 def oracle_cfg(wl: inputs.Workload, B: int | None = None) -> oracle.Cfg:
@@ -59,6 +81,21 @@ class Problem:
                      self.buf.w_uk, self.buf.w_uv, gw, gb,
                      dev(toks["gate_in"][:, :T], torch.float32) if toks["gate_in"] is not None else None,
                      out, self.buf.cache, self.buf.open_slot, self.buf.workspace)
+        return out
+
+    def prefill_from(self, toks: dict, t0: int, t1: int):
+        """Chunked prefill of tokens t0 .. t1-1 (indices into toks) continuing from
+        the current cache and open slot."""
+        B, wl = self.B, self.wl
+        T = t1 - t0
+        out = torch.empty(B, T, wl.H, wl.d_h, device="cuda", dtype=self.dt)
+        gw, gb = self.gate_ptrs()
+        gin = toks["gate_in"]
+        mtla.prefill_from(self.cfg, t0, T, dev(toks["c"][:, t0:t1], self.dt), dev(toks["kr"][:, t0:t1], self.dt),
+                          dev(toks["qc"][:, t0:t1], self.dt), dev(toks["qr"][:, t0:t1], self.dt),
+                          self.buf.w_uk, self.buf.w_uv, gw, gb,
+                          dev(gin[:, t0:t1], torch.float32) if gin is not None else None,
+                          out, self.buf.cache, self.buf.open_slot, self.buf.workspace)
         return out
 
     def decode(self, toks: dict, k: int, pos):

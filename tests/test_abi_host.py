@@ -182,3 +182,19 @@ def test_noalloc_limit_matches_header():
     m = re.search(r"#define\s+MTLA_NOALLOC_SCRATCH_BYTES\s+\((\d+)u\s*<<\s*(\d+)\)", text)
     assert m, "MTLA_NOALLOC_SCRATCH_BYTES not found in include/mtla.h"
     assert mtla.NOALLOC_SCRATCH_BYTES == int(m.group(1)) << int(m.group(2))
+
+
+def test_prefill_from_rejects_bad_arguments_on_the_host(lib):
+    """mtla_prefill_from: a NULL open slot, a negative start and a chunk past
+    the cache are refused before anything touches the device (the pointers
+    below are never dereferenced)."""
+    cfg = _cfg(max_slots=16)           # s = 2: 32 tokens fit
+    fake = 0x10000
+    args = [fake] * 4 + [fake, fake, None, None, None, fake, fake]
+    ws = 1 << 30
+    st = lambda t0, T, open_slot: lib.mtla_prefill_from(
+        ctypes.byref(cfg), t0, T, *args, open_slot, fake, ws, None)
+    cfg.gate_mode = mtla.GATE_UNIT
+    assert st(3, 4, None) == mtla.ERR_INVALID_ARG
+    assert st(-1, 4, fake) == mtla.ERR_INVALID_ARG
+    assert st(30, 4, fake) == mtla.ERR_CAPACITY      # ceil(34 / 2) = 17 slots > 16
