@@ -25,6 +25,7 @@ _SRC = os.path.join(_HERE, "mtla_oracle.c")
 _LIB = os.path.join(_HERE, "libmtla_oracle.so")
 
 GATE_COMPUTED, GATE_SUPPLIED, GATE_UNIT = 0, 1, 2
+GATE_CHANNEL_COMPUTED, GATE_CHANNEL_SUPPLIED = 3, 4
 
 FAULT_NONE = 0
 FAULT_DROP_OWN_PARTIAL = 1
@@ -42,6 +43,7 @@ FAULT_ROPE_HALF_SPLIT = 12
 FAULT_PE_SWAP = 13
 FAULT_CHUNK_NO_SEED = 14
 FAULT_CHUNK_LOCAL_POS = 15
+FAULT_CHANNEL_TRANSPOSE = 16
 
 
 def build(force: bool = False) -> str:
@@ -99,6 +101,7 @@ def _load():
         _lib.orc_rope.argtypes = [ctypes.c_int64, ctypes.c_int32, ctypes.c_double, _P, _P]
         _lib.orc_gate.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int64, _P, _P, _P, _P]
         _lib.orc_gate.restype = ctypes.c_double
+        _lib.orc_gate_channels.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int64, _P, _P, _P, _P, _P]
         _lib.orc_partials.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int32] + [_P] * 7
         _lib.orc_attend_rows.argtypes = ([ctypes.POINTER(_Cfg), ctypes.c_int32] + [_P] * 5
                                          + [ctypes.c_int64, _PI, _P, _P])
@@ -148,6 +151,16 @@ def gate(cfg: Cfg, t: int, c_t, G=None, g=None, w_given=None) -> float:
     c_t = _d(c_t)
     wg = None if w_given is None else np.array([w_given], dtype=np.float64)
     return _load().orc_gate(ctypes.byref(cfg.c()), t, _p(c_t), _p(_d(G)), _p(_d(g)), _p(wg))
+
+
+def gate_channels(cfg: Cfg, t: int, c_t, G=None, g=None, w_given=None) -> np.ndarray:
+    """The D merging weights of token t (per-channel modes; the scalar modes
+    repeat their one weight)."""
+    c_t = _d(c_t)
+    wv = np.zeros(cfg.D)
+    wg = None if w_given is None else _d(np.atleast_1d(w_given))
+    _load().orc_gate_channels(ctypes.byref(cfg.c()), t, _p(c_t), _p(_d(G)), _p(_d(g)), _p(wg), _p(wv))
+    return wv
 
 
 def partials(cfg: Cfg, c, kr, G=None, g=None, gate_in=None):

@@ -38,6 +38,10 @@
  *     theirs;
  *   - scores use scale 1/sqrt(d_h + d_R) unless a scale is given;
  *   - the merged sum is not normalised.
+ * Per-channel variant (reading of W_t (.) x_t with W_t a vector): one weight
+ * per slot channel, w_t[k] = sigmoid((c_t (.) PE_t) . G[t mod s][:, k] +
+ * g[t mod s][k]) with G [s, d_c, D], or the D weights given per token; the
+ * scalar modes are the case of equal channels.
  * The PE, RoPE-frequency and gate conventions above are readings (the pages
  * print no worked example of them); the pins hold this file to the exact
  * values those readings give at small sizes (frequencies 1, 0.1, 0.01, 0.001
@@ -57,6 +61,8 @@
 #define ORC_GATE_COMPUTED 0
 #define ORC_GATE_SUPPLIED 1
 #define ORC_GATE_UNIT 2
+#define ORC_GATE_CHANNEL_COMPUTED 3
+#define ORC_GATE_CHANNEL_SUPPLIED 4
 
 typedef struct {
     int32_t B, H, d_h, d_c, d_r, s;
@@ -85,6 +91,7 @@ enum {
     ORC_FAULT_PE_SWAP = 13,          /* PE with cos at even, sin at odd      */
     ORC_FAULT_CHUNK_NO_SEED = 14,    /* chunked prefill: open block restarts  */
     ORC_FAULT_CHUNK_LOCAL_POS = 15,  /* chunked prefill: positions from 0     */
+    ORC_FAULT_CHANNEL_TRANSPOSE = 16, /* per-channel gate read as G [s,D,d_c] */
 };
 static int orc_fault = ORC_FAULT_NONE;
 void orc_set_fault(int f) { orc_fault = f; }
@@ -128,12 +135,23 @@ void orc_rope(int64_t t, int32_t d, double base, const double* x, double* y) {
     }
 }
 
+void orc_gate_channels(const orc_cfg* cfg, int64_t t, const double* c_t, const double* G,
+                       const double* g, const double* w_given, double* wv);
+
 /* Merging weight of token t (MTLA Sec. 4.1, Eq. 13, under the reading above).
  * w_given points at the supplied weight in SUPPLIED mode. */
 double orc_gate(const orc_cfg* cfg, int64_t t, const double* c_t, const double* G,
                 const double* g, const double* w_given) {
     if (cfg->gate_mode == ORC_GATE_UNIT) return 1.0;
     if (cfg->gate_mode == ORC_GATE_SUPPLIED) return *w_given;
+    if (cfg->gate_mode >= ORC_GATE_CHANNEL_COMPUTED) {
+        /* the per-channel modes: the weight of channel 0 (the w outputs below) */
+        double* wv = (double*)malloc(sizeof(double) * (cfg->d_c + cfg->d_r));
+        orc_gate_channels(cfg, t, c_t, G, g, w_given, wv);
+        double w0 = wv[0];
+        free(wv);
+        return w0;
+    }
     int32_t d_c = cfg->d_c;
     int64_t r = t % cfg->s;
     if (orc_fault == ORC_FAULT_GATE_WRONG_ROW) r = (t + 1) % cfg->s;
@@ -143,6 +161,49 @@ double orc_gate(const orc_cfg* cfg, int64_t t, const double* c_t, const double* 
     for (int32_t i = 0; i < d_c; ++i) z += G[r * d_c + i] * (c_t[i] * pe[i]);
     free(pe);
     return 1.0 / (1.0 + exp(-z));
+}
+
+/* Per-channel merging weights: the reading of W_t (.) x_t with one weight per
+ * slot channel (the latent and the rotated key alike):
+ *   w_t[k] = sigmoid( sum_i (c_t (.) PE_t)[i] G[r][i][k] + g[r][k] ),  r = t mod s,
+ * G [s, d_c, D], g [s, D] (CHANNEL_COMPUTED), or the D given weights
+ * (CHANNEL_SUPPLIED). The scalar modes give their one weight in every channel. */
+void orc_gate_channels(const orc_cfg* cfg, int64_t t, const double* c_t, const double* G,
+                       const double* g, const double* w_given, double* wv) {
+    const int32_t d_c = cfg->d_c, D = cfg->d_c + cfg->d_r;
+    if (cfg->gate_mode == ORC_GATE_CHANNEL_SUPPLIED) {
+        for (int32_t k = 0; k < D; ++k) wv[k] = w_given[k];
+        return;
+    }
+    if (cfg->gate_mode != ORC_GATE_CHANNEL_COMPUTED) {
+        double w = orc_gate(cfg, t, c_t, G, g, w_given);
+        for (int32_t k = 0; k < D; ++k) wv[k] = w;
+        return;
+    }
+    int64_t r = t % cfg->s;
+    if (orc_fault == ORC_FAULT_GATE_WRONG_ROW) r = (t + 1) % cfg->s;
+    double* pe = (double*)malloc(sizeof(double) * d_c);
+    orc_pe(t, d_c, cfg->pe_base, pe);
+    for (int32_t k = 0; k < D; ++k) {
+        double z = g[r * D + k];
+        for (int32_t i = 0; i < d_c; ++i) {
+            double gik = G[(r * d_c + i) * D + k];
+            if (orc_fault == ORC_FAULT_CHANNEL_TRANSPOSE) {
+                int64_t flat = (int64_t)i * D + k;          /* read as if stored [D, d_c] */
+                gik = G[r * d_c * D + (flat % d_c) * D + flat / d_c];
+            }
+            z += (c_t[i] * pe[i]) * gik;
+        }
+        wv[k] = 1.0 / (1.0 + exp(-z));
+    }
+    free(pe);
+}
+
+/* Where the supplied weights of token (b, t) start in gate_in: [B,T] scalars
+ * or [B,T,D] per-channel weights. */
+static const double* orc_given(const orc_cfg* cfg, const double* gate_in, int64_t bt) {
+    if (!gate_in) return NULL;
+    return cfg->gate_mode == ORC_GATE_CHANNEL_SUPPLIED ? &gate_in[bt * (cfg->d_c + cfg->d_r)] : &gate_in[bt];
 }
 
 /* x_t = [c_t ; RoPE_t(k_t)], the vector a token contributes to its slot. */
@@ -162,13 +223,14 @@ void orc_partials(const orc_cfg* cfg, int32_t T, const double* c, const double* 
     const int32_t D = d_c + d_r;
     for (int32_t b = 0; b < B; ++b)
         for (int32_t t = 0; t < T; ++t) {
-            const double* wg = gate_in ? &gate_in[(int64_t)b * T + t] : NULL;
-            w[(int64_t)b * T + t] = orc_gate(cfg, t, &c[((int64_t)b * T + t) * d_c], G, g, wg);
+            const int64_t bt = (int64_t)b * T + t;
+            w[bt] = orc_gate(cfg, t, &c[bt * d_c], G, g, orc_given(cfg, gate_in, bt));
         }
 #pragma omp parallel for schedule(static)
     for (int64_t bt = 0; bt < (int64_t)B * T; ++bt) {
         int32_t b = (int32_t)(bt / T), t = (int32_t)(bt % T);
         double* x = (double*)malloc(sizeof(double) * D);
+        double* wv = (double*)malloc(sizeof(double) * D);
         double* out = &P[bt * D];
         for (int32_t k = 0; k < D; ++k) out[k] = 0.0;
         int32_t u0 = s * (t / s);
@@ -176,8 +238,10 @@ void orc_partials(const orc_cfg* cfg, int32_t T, const double* c, const double* 
         for (int32_t u = u0; u <= t; ++u) {
             int64_t bu = (int64_t)b * T + u;
             orc_token_vector(cfg, u, &c[bu * d_c], &kr[bu * d_r], x);
-            for (int32_t k = 0; k < D; ++k) out[k] += w[bu] * x[k];
+            orc_gate_channels(cfg, u, &c[bu * d_c], G, g, orc_given(cfg, gate_in, bu), wv);
+            for (int32_t k = 0; k < D; ++k) out[k] += wv[k] * x[k];
         }
+        free(wv);
         free(x);
     }
 }
@@ -344,13 +408,14 @@ void orc_prefill_from(const orc_cfg* cfg, int32_t t0, int32_t T, int32_t n_in, c
     /* gates, then the partial slots of the new positions (local index i - t0) */
     for (int32_t b = 0; b < B; ++b)
         for (int32_t li = 0; li < T; ++li) {
-            const double* wg = gate_in ? &gate_in[(int64_t)b * T + li] : NULL;
-            w[(int64_t)b * T + li] = orc_gate(cfg, t0 + li, &c[((int64_t)b * T + li) * d_c], G, g, wg);
+            const int64_t bl = (int64_t)b * T + li;
+            w[bl] = orc_gate(cfg, t0 + li, &c[bl * d_c], G, g, orc_given(cfg, gate_in, bl));
         }
 #pragma omp parallel for schedule(static)
     for (int64_t bl = 0; bl < (int64_t)B * T; ++bl) {
         const int32_t b = (int32_t)(bl / T), li = (int32_t)(bl % T), i = t0 + li;
         double* x = (double*)malloc(sizeof(double) * D);
+        double* wv = (double*)malloc(sizeof(double) * D);
         double* o = &P[bl * D];
         int32_t u0 = s * (i / s);
         if (orc_fault == ORC_FAULT_SCAN_NO_RESET) u0 = 0;
@@ -360,8 +425,10 @@ void orc_prefill_from(const orc_cfg* cfg, int32_t t0, int32_t T, int32_t n_in, c
             const int64_t bu = (int64_t)b * T + (u - t0);
             const int32_t tu = orc_fault == ORC_FAULT_CHUNK_LOCAL_POS ? u - t0 : u;
             orc_token_vector(cfg, tu, &c[bu * d_c], &kr[bu * d_r], x);
-            for (int32_t k = 0; k < D; ++k) o[k] += w[bu] * x[k];
+            orc_gate_channels(cfg, tu, &c[bu * d_c], G, g, orc_given(cfg, gate_in, bu), wv);
+            for (int32_t k = 0; k < D; ++k) o[k] += wv[k] * x[k];
         }
+        free(wv);
         free(x);
     }
 #pragma omp parallel for schedule(dynamic, 1)
@@ -424,17 +491,19 @@ void orc_decode_step(const orc_cfg* cfg, int32_t max_slots, const double* c_new,
     for (int32_t b = 0; b < B; ++b) {
         int64_t t = pos[b];
         int64_t j = t / s;
-        const double* wg = gate_in ? &gate_in[b] : NULL;
-        double w = orc_gate(cfg, t, &c_new[(int64_t)b * d_c], G, g, wg);
-        if (w_out) w_out[b] = w;
+        const double* wg = orc_given(cfg, gate_in, b);
+        double* wv = (double*)malloc(sizeof(double) * D);
+        orc_gate_channels(cfg, t, &c_new[(int64_t)b * d_c], G, g, wg, wv);
+        if (w_out) w_out[b] = wv[0];
         double* x = (double*)malloc(sizeof(double) * D);
         orc_token_vector(cfg, t, &c_new[(int64_t)b * d_c], &kr_new[(int64_t)b * d_r], x);
         double* a = &acc[(int64_t)b * D];
         int fresh = (t % s == 0);
         if (orc_fault == ORC_FAULT_SCAN_NO_RESET) fresh = (t == 0);
-        for (int32_t k = 0; k < D; ++k) a[k] = (fresh ? 0.0 : a[k]) + w * x[k];
+        for (int32_t k = 0; k < D; ++k) a[k] = (fresh ? 0.0 : a[k]) + wv[k] * x[k];
         memcpy(&cache[((int64_t)b * max_slots + j) * D], a, sizeof(double) * D);
         free(x);
+        free(wv);
     }
 #pragma omp parallel for schedule(dynamic, 1)
     for (int64_t bh = 0; bh < (int64_t)B * H; ++bh) {

@@ -16,7 +16,10 @@ mathematics fix, none of which retypes the oracle's own formulas.
   exactly 1, 0.1, 0.01, 0.001 at base 10000) and one gate worked by hand;
 - chunked prefill: from position 0 it is the parallel forward; a prefix then a
   chunk equals one prefill (split points inside a block included); a chunk
-  equals the same number of incremental decode steps.
+  equals the same number of incremental decode steps;
+- per-channel gate: equal channels reduce it to the scalar gate (computed and
+  supplied); G = 0 gives a closed form; one value worked by hand; decoding
+  equals the parallel form.
 Finally, each planted mistake in the oracle must trip at least one pin.
 """
 import math
@@ -389,6 +392,101 @@ def pin_prefill_from_equals_decode_steps():
     return True
 
 
+def _channel_problem(s, T, seed, B=2, H=2, d_h=8, d_c=16, d_r=4):
+    """A problem with per-channel gate parameters G [s, d_c, D], g [s, D] and
+    supplied per-channel weights [B, T, D]."""
+    cfg, p = _rand_problem(B, H, d_h, d_c, d_r, s, T, seed)
+    rng = np.random.default_rng(seed + 1000)
+    D = d_c + d_r
+    p["Gc"] = rng.standard_normal((s, d_c, D)) / math.sqrt(d_c)
+    p["gc"] = rng.standard_normal((s, D)) * 0.5
+    p["gate_in_c"] = 1.0 / (1.0 + np.exp(-rng.standard_normal((B, T, D))))
+    return cfg, p
+
+
+def pin_channel_gate_equal_columns_is_scalar():
+    """Per-channel gate whose D columns are all the scalar gate's row (and
+    biases equal) reproduces the scalar-gate forward; supplied per-channel
+    weights equal across channels reproduce the scalar supplied gate."""
+    for s in (1, 3):
+        cfg, p = _channel_problem(s, 11, seed=100 + s)
+        D = cfg.D
+        ref = oracle.prefill(cfg, p["c"], p["kr"], p["qc"], p["qr"], p["w_uk"], p["w_uv"], p["G"], p["g"])
+        cc = oracle.Cfg(cfg.B, cfg.H, cfg.d_h, cfg.d_c, cfg.d_r, s, gate_mode=oracle.GATE_CHANNEL_COMPUTED)
+        Gc = np.repeat(p["G"][:, :, None], D, axis=2)
+        gc = np.repeat(p["g"][:, None], D, axis=1)
+        got = oracle.prefill(cc, p["c"], p["kr"], p["qc"], p["qr"], p["w_uk"], p["w_uv"], Gc, gc)
+        if not (np.max(np.abs(got["out"] - ref["out"])) < 1e-12 and np.max(np.abs(got["cache"] - ref["cache"])) < 1e-12):
+            return False
+        cs = oracle.Cfg(cfg.B, cfg.H, cfg.d_h, cfg.d_c, cfg.d_r, s, gate_mode=oracle.GATE_SUPPLIED)
+        ref = oracle.prefill(cs, p["c"], p["kr"], p["qc"], p["qr"], p["w_uk"], p["w_uv"], gate_in=p["gate_in"])
+        cq = oracle.Cfg(cfg.B, cfg.H, cfg.d_h, cfg.d_c, cfg.d_r, s, gate_mode=oracle.GATE_CHANNEL_SUPPLIED)
+        got = oracle.prefill(cq, p["c"], p["kr"], p["qc"], p["qr"], p["w_uk"], p["w_uv"],
+                             gate_in=np.repeat(p["gate_in"][:, :, None], D, axis=2))
+        if not np.max(np.abs(got["out"] - ref["out"])) < 1e-12:
+            return False
+    return True
+
+
+def pin_channel_gate_closed_form():
+    """G = 0: token t's weights are sigmoid(g[t mod s][k]) in channel k, so with
+    all-ones latents and zero keys the partial slot of position t holds, in
+    latent channel k, the sum of sigmoid(g[u mod s][k]) over its block's
+    tokens u <= t, and zeros in the key channels."""
+    s, T, d_c, d_r = 3, 10, 8, 4
+    D = d_c + d_r
+    cfg = oracle.Cfg(1, 1, 4, d_c, d_r, s, gate_mode=oracle.GATE_CHANNEL_COMPUTED)
+    g = np.arange(s * D, dtype=float).reshape(s, D) * 0.1 - 1.0
+    sig = 1.0 / (1.0 + np.exp(-g))
+    _, P = oracle.partials(cfg, np.ones((1, T, d_c)), np.zeros((1, T, d_r)), np.zeros((s, d_c, D)), g)
+    for t in range(T):
+        want = sum(sig[u % s] for u in range(s * (t // s), t + 1))
+        if not (np.max(np.abs(P[0, t, :d_c] - want[:d_c])) < 1e-14 and np.all(P[0, t, d_c:] == 0.0)):
+            return False
+    return True
+
+
+def pin_channel_gate_value():
+    """One per-channel gate worked by hand: t = 1, s = 2 (row 1), d_c = 2,
+    D = 4; PE_1 at width 2 is (sin 1, cos 1); c = (1, 2);
+    G[1] = [[1, 0, -1, 2], [0.5, 1, 0, -3]] (rows: latent inputs, columns:
+    slot channels), g[1] = (0, 0.25, -0.5, 1):
+      z = sin 1 * G[1][0] + 2 cos 1 * G[1][1] + g[1],  w = sigmoid(z)."""
+    cfg = oracle.Cfg(1, 1, 4, 2, 2, 2, gate_mode=oracle.GATE_CHANNEL_COMPUTED)
+    G = np.zeros((2, 2, 4))
+    G[1] = [[1.0, 0.0, -1.0, 2.0], [0.5, 1.0, 0.0, -3.0]]
+    g = np.array([[0.0, 0.0, 0.0, 0.0], [0.0, 0.25, -0.5, 1.0]])
+    s1, c1 = math.sin(1.0), math.cos(1.0)
+    z = [s1 * 1.0 + 2 * c1 * 0.5 + 0.0, 2 * c1 * 1.0 + 0.25, -s1 - 0.5, 2 * s1 - 6 * c1 + 1.0]
+    want = np.array([1.0 / (1.0 + math.exp(-v)) for v in z])
+    return np.max(np.abs(oracle.gate_channels(cfg, 1, np.array([1.0, 2.0]), G, g) - want)) < 1e-15
+
+
+def pin_channel_incremental_equals_parallel():
+    """Per-channel gates, computed and supplied: decoding step by step equals
+    the parallel masked forward (outputs, cache, open slot)."""
+    for mode in (oracle.GATE_CHANNEL_COMPUTED, oracle.GATE_CHANNEL_SUPPLIED):
+        for s in (2, 3):
+            B, T = 2, 11
+            cfg, p = _channel_problem(s, T, seed=110 + s)
+            cfg = oracle.Cfg(B, cfg.H, cfg.d_h, cfg.d_c, cfg.d_r, s, gate_mode=mode)
+            gin = p["gate_in_c"] if mode == oracle.GATE_CHANNEL_SUPPLIED else None
+            par = oracle.prefill(cfg, p["c"], p["kr"], p["qc"], p["qr"], p["w_uk"], p["w_uv"], p["Gc"], p["gc"], gin)
+            max_slots = (T + s - 1) // s
+            cache = np.zeros((B, max_slots, cfg.D))
+            acc = np.zeros((B, cfg.D))
+            outs = []
+            for t in range(T):
+                r = oracle.decode_step(cfg, p["c"][:, t], p["kr"][:, t], p["qc"][:, t], p["qr"][:, t], p["w_uk"],
+                                       p["w_uv"], np.full(B, t), cache, acc, p["Gc"], p["gc"],
+                                       None if gin is None else gin[:, t])
+                outs.append(r["out"])
+            if not (np.max(np.abs(np.stack(outs, axis=1) - par["out"])) < 1e-12
+                    and np.max(np.abs(cache - par["cache"])) < 1e-12 and np.max(np.abs(acc - par["acc"])) < 1e-12):
+                return False
+    return True
+
+
 PINS = {
     "cache_footprint": pin_cache_footprint,
     "s1_is_mla_sdpa": pin_s1_is_mla_sdpa,
@@ -405,6 +503,10 @@ PINS = {
     "prefill_from_start_is_prefill": pin_prefill_from_start_is_prefill,
     "prefill_chunks_compose": pin_prefill_chunks_compose,
     "prefill_from_equals_decode_steps": pin_prefill_from_equals_decode_steps,
+    "channel_gate_equal_columns_is_scalar": pin_channel_gate_equal_columns_is_scalar,
+    "channel_gate_closed_form": pin_channel_gate_closed_form,
+    "channel_gate_value": pin_channel_gate_value,
+    "channel_incremental_equals_parallel": pin_channel_incremental_equals_parallel,
 }
 
 
@@ -436,6 +538,7 @@ FAULTS = {
     "pe_swap": oracle.FAULT_PE_SWAP,
     "chunk_no_seed": oracle.FAULT_CHUNK_NO_SEED,
     "chunk_local_pos": oracle.FAULT_CHUNK_LOCAL_POS,
+    "channel_transpose": oracle.FAULT_CHANNEL_TRANSPOSE,
 }
 
 
