@@ -85,15 +85,26 @@ typedef enum {
 
 typedef enum { MTLA_BF16 = 0, MTLA_FP32 = 1 } mtla_dtype;
 
+/* Merging weights (MTLA Sec. 4.1, Eq. 13; the reading of W_t (.) x_t):
+ * one scalar per token that scales its whole slot vector x_t = [c_t ; RoPE_t(k_t)]
+ * (modes 0-2), or one weight per slot channel (modes 3-4, the reading of W_t as
+ * a vector): slot_j = sum_t w_t (.) x_t. The attention is the same for all. */
 typedef enum {
-    MTLA_GATE_COMPUTED = 0,     /* w_t from gate_w, gate_b and the PE (Eq. 13)   */
-    MTLA_GATE_SUPPLIED = 1,     /* w_t read from gate_in                         */
-    MTLA_GATE_UNIT = 2          /* w_t = 1                                       */
+    MTLA_GATE_COMPUTED = 0,     /* w_t = sigmoid(G[t mod s] . (c_t*PE_t) + g[t mod s]):
+                                   gate_w G [s, d_c] fp32, gate_b g [s] fp32           */
+    MTLA_GATE_SUPPLIED = 1,     /* w_t read from gate_in: [B] (decode), [B, T] (prefill) */
+    MTLA_GATE_UNIT = 2,         /* w_t = 1                                             */
+    MTLA_GATE_CHANNEL_COMPUTED = 3, /* w_t[k] = sigmoid((c_t*PE_t) . G[t mod s][:, k] +
+                                   g[t mod s][k]), k < d_c + d_r: gate_w G [s, d_c, d_c+d_r]
+                                   fp32 (input channel major), gate_b g [s, d_c+d_r] fp32 */
+    MTLA_GATE_CHANNEL_SUPPLIED = 4  /* w_t[k] read from gate_in: [B, d_c+d_r] (decode),
+                                   [B, T, d_c+d_r] (prefill)                            */
 } mtla_gate_mode;
 
 /* Problem description shared by every call.
  * Supported: 1 <= batch; 1 <= heads <= 128; d_h, d_c, d_r multiples of 16;
- * d_c + d_r <= 576; d_h <= 256; 1 <= stride <= 8; max_slots >= 1.
+ * d_c + d_r <= 576; d_h <= 256; 1 <= stride <= 8; max_slots >= 1; with the
+ * per-channel gate modes also d_r <= 128.
  * Anything else: MTLA_ERR_UNSUPPORTED (or INVALID_ARG for non-positive sizes). */
 typedef struct {
     int32_t batch;          /* B: sequences                                       */
@@ -129,8 +140,8 @@ mtla_status mtla_workspace_size(const mtla_config* cfg, int32_t max_tokens, size
  *   c_new   [B, d_c]        dtype        kr_new [B, d_r] dtype (before RoPE)
  *   q_c     [B, H, d_h]     dtype        q_r    [B, H, d_r] dtype (before RoPE)
  *   w_uk    [H, d_h, d_c]   dtype        w_uv   [H, d_h, d_c] dtype
- *   gate_w  [s, d_c] fp32, gate_b [s] fp32   (COMPUTED only; else may be NULL)
- *   gate_in [B] fp32                          (SUPPLIED only; else may be NULL)
+ *   gate_w, gate_b     (the COMPUTED modes, shapes under mtla_gate_mode; else may be NULL)
+ *   gate_in [B] or [B, d_c+d_r] fp32          (the SUPPLIED modes; else may be NULL)
  *   pos     [B] int32, device: index of this token = tokens already cached.
  *           pos[b] >= max_slots * s skips sequence b and latches CAPACITY.
  *   cache   [B, max_slots, d_c + d_r] dtype, in/out (slot floor(t/s) written)
@@ -154,7 +165,7 @@ mtla_status mtla_decode_step(const mtla_config* cfg,
  * so the result equals T incremental decode steps).
  *
  *   c [B,T,d_c], kr [B,T,d_r], q_c [B,T,H,d_h], q_r [B,T,H,d_r]   dtype
- *   w_uk, w_uv, gate_w, gate_b as for decode; gate_in [B,T] fp32 (SUPPLIED)
+ *   w_uk, w_uv, gate_w, gate_b as for decode; gate_in [B,T] or [B,T,d_c+d_r] fp32 (SUPPLIED modes)
  *   out       [B,T,H,d_h] dtype, out
  *   cache_out [B, max_slots, d_c+d_r] dtype, out: slots 0..ceil(T/s)-1 (the
  *             cache a following mtla_decode_step at pos = T continues from);

@@ -94,7 +94,7 @@ static mtla_status check_config(const mtla_config* cfg, Shape* sh) {
         cfg->stride <= 0 || cfg->max_slots <= 0)
         return MTLA_ERR_INVALID_ARG;
     if (cfg->dtype != MTLA_BF16 && cfg->dtype != MTLA_FP32) return MTLA_ERR_INVALID_ARG;
-    if (cfg->gate_mode < MTLA_GATE_COMPUTED || cfg->gate_mode > MTLA_GATE_UNIT)
+    if (cfg->gate_mode < MTLA_GATE_COMPUTED || cfg->gate_mode > MTLA_GATE_CHANNEL_SUPPLIED)
         return MTLA_ERR_INVALID_ARG;
     if (!(cfg->softmax_scale >= 0.f) || !std::isfinite(cfg->softmax_scale)) return MTLA_ERR_INVALID_ARG;
     if (!(cfg->rope_base >= 0.f) || !std::isfinite(cfg->rope_base) ||
@@ -105,6 +105,8 @@ static mtla_status check_config(const mtla_config* cfg, Shape* sh) {
         cfg->stride > 8)
         return MTLA_ERR_UNSUPPORTED;
     if ((int64_t)cfg->max_slots * cfg->stride > INT32_MAX) return MTLA_ERR_UNSUPPORTED;
+    // per-channel gates: the scan keeps a lane's RoPE pairs in registers (d_r <= 128)
+    if (cfg->gate_mode >= MTLA_GATE_CHANNEL_COMPUTED && cfg->d_r > 128) return MTLA_ERR_UNSUPPORTED;
     sh->B = cfg->batch;
     sh->H = cfg->heads;
     sh->d_h = cfg->d_h;
@@ -149,10 +151,10 @@ static size_t prefill_ws(const mtla_config* cfg, const Shape& sh, int T) {
 
 static mtla_status check_gate_ptrs(const mtla_config* cfg, const float* gate_w, const float* gate_b,
                                    const float* gate_in) {
-    if (cfg->gate_mode == MTLA_GATE_COMPUTED) {
+    if (cfg->gate_mode == MTLA_GATE_COMPUTED || cfg->gate_mode == MTLA_GATE_CHANNEL_COMPUTED) {
         if (!gate_w || !gate_b || !aligned16(gate_w) || !aligned16(gate_b)) return MTLA_ERR_INVALID_ARG;
     }
-    if (cfg->gate_mode == MTLA_GATE_SUPPLIED) {
+    if (cfg->gate_mode == MTLA_GATE_SUPPLIED || cfg->gate_mode == MTLA_GATE_CHANNEL_SUPPLIED) {
         if (!gate_in || !aligned16(gate_in)) return MTLA_ERR_INVALID_ARG;
     }
     return MTLA_OK;

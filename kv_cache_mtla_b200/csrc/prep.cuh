@@ -44,10 +44,47 @@ __device__ __forceinline__ void update_freqs(const Shape& sh, UpdateFreqs& f) {
 // Returns false (and latches CAPACITY) if pos[b] does not fit the cache.
 // `gate_w` is G [s x d_c] (global memory, or a copy in shared memory) and `f`
 // the frequencies from update_freqs.
+// Per-channel gate (modes 3 and 4): the D merging weights of token t of
+// sequence b into wch, computed as sigmoid((c_t * PE_t) . G[r][:, k] + g[r][k])
+// with G [s, d_c, D], g [s, D] (thread k of the block: output channel k, G read
+// along k), or read from gate_in [B, D]. vch holds c_t * PE_t; c0/c1 are this
+// thread's latent pairs and f its PE frequencies. Every thread calls it.
+template <int kMaxPer>
+__device__ void channel_gate(const DecodeArgs& a, int b, int64_t t, const float* gate_w, const UpdateFreqs& f,
+                             const float* c0, const float* c1, float* vch, float* wch) {
+    const Shape& sh = a.sh;
+    const int nt = blockDim.x, tid = threadIdx.x;
+    __syncthreads();                     // vch / wch of an earlier call of this block are read
+    if (sh.gate_mode == 4) {
+        for (int k = tid; k < sh.D; k += nt) wch[k] = a.gate_in[(size_t)b * sh.D + k];
+    } else {
+        const int r = (int)(t % sh.s);
+#pragma unroll
+        for (int i = 0; i < kMaxPer; ++i) {
+            const int kp = tid + i * nt;
+            if (kp < sh.d_c / 2) {
+                float sn, cs;
+                pair_sincos_f(t, f.pe[i], &sn, &cs);
+                vch[2 * kp] = c0[i] * sn;
+                vch[2 * kp + 1] = c1[i] * cs;
+            }
+        }
+        __syncthreads();
+        const float* G = gate_w + (size_t)r * sh.d_c * sh.D;
+        for (int k = tid; k < sh.D; k += nt) {
+            float z = a.gate_b[(size_t)r * sh.D + k];
+            for (int i = 0; i < sh.d_c; ++i) z = fmaf(vch[i], G[(size_t)i * sh.D + k], z);
+            wch[k] = sigmoidf_(z);
+        }
+    }
+    __syncthreads();
+}
+
 template <typename T>
 __device__ bool decode_update_body(const DecodeArgs& a, int b, const float* gate_w, const UpdateFreqs& f) {
     const Shape& sh = a.sh;
     __shared__ float red[32];
+    __shared__ float vch[512], wch[576];  // per-channel gate: c_t * PE_t and the D weights
     constexpr int kMaxPer = kUpdMaxPer;
     constexpr int kMaxPairs = kUpdMaxPairs;
     const int nt = blockDim.x, tid = threadIdx.x;
@@ -108,9 +145,13 @@ __device__ bool decode_update_body(const DecodeArgs& a, int b, const float* gate
             y1[i] = x0[i] * sn + x1[i] * cs;
         }
     }
-    // gate (Eq. 13): w = sigmoid(G[t mod s] . (c_t * PE_t) + g[t mod s])
-    float w;
-    if (sh.gate_mode == 2) {
+    // gate (Eq. 13): w = sigmoid(G[t mod s] . (c_t * PE_t) + g[t mod s]), or
+    // one weight per slot channel (modes 3, 4)
+    const bool channel = sh.gate_mode >= 3;
+    float w = 1.f;
+    if (channel) {
+        channel_gate<kMaxPer>(a, b, t, gate_w, f, c0, c1, vch, wch);
+    } else if (sh.gate_mode == 2) {
         w = 1.f;
     } else if (sh.gate_mode == 1) {
         w = a.gate_in[b];
@@ -144,7 +185,8 @@ __device__ bool decode_update_body(const DecodeArgs& a, int b, const float* gate
     for (int i = 0; i < kMaxPer; ++i) {
         const int kp = tid + i * nt;
         if (kp < sh.d_c / 2) {
-            const float v0 = a0[i] + w * c0[i], v1 = a1[i] + w * c1[i];
+            const float w0 = channel ? wch[2 * kp] : w, w1 = channel ? wch[2 * kp + 1] : w;
+            const float v0 = a0[i] + w0 * c0[i], v1 = a1[i] + w1 * c1[i];
             acc[2 * kp] = v0;
             acc[2 * kp + 1] = v1;
             row[2 * kp] = from_f<T>(v0);
@@ -155,7 +197,8 @@ __device__ bool decode_update_body(const DecodeArgs& a, int b, const float* gate
     for (int i = 0; i < kMaxPairs; ++i) {
         const int kp = tid + i * nt;
         if (kp < sh.d_r / 2) {
-            const float v0 = ar0[i] + w * y0[i], v1 = ar1[i] + w * y1[i];
+            const float w0 = channel ? wch[sh.d_c + 2 * kp] : w, w1 = channel ? wch[sh.d_c + 2 * kp + 1] : w;
+            const float v0 = ar0[i] + w0 * y0[i], v1 = ar1[i] + w1 * y1[i];
             acc[sh.d_c + 2 * kp] = v0;
             acc[sh.d_c + 2 * kp + 1] = v1;
             row[sh.d_c + 2 * kp] = from_f<T>(v0);
@@ -364,6 +407,115 @@ __global__ void __launch_bounds__(256) k_prefill_scan(PrefillArgs a, PT* P, floa
         if (open) {
             open[sh.d_c + 2 * k] = a0;
             open[sh.d_c + 2 * k + 1] = a1;
+        }
+    }
+}
+
+// The block-prefix scan with per-channel gates (modes 3 and 4): the same
+// outputs as k_prefill_scan (partial slots P, the slots in the cache, the open
+// slot, the (cos, sin) table), with every slot channel k of token u weighted by
+// its own w_u[k]. One warp per slot, tokens in order: the warp stages c_u * PE_u
+// and then the D weights of token u in shared memory (lane k: channels
+// k, k+32, ..., G read along k), and each lane carries its channels' sums.
+template <typename T, typename PT>
+__global__ void __launch_bounds__(256) k_prefill_scan_channel(PrefillArgs a, PT* P, float2* rope_tab = nullptr) {
+    const Shape sh = a.sh;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int b = blockIdx.y;
+    const int Tn = a.T;
+    __shared__ double pe_freq[256];
+    __shared__ double rope_freq[64];
+    __shared__ float vsh[8][512];
+    __shared__ float wsh[8][576];
+    for (int k = threadIdx.x; k < sh.d_c / 2; k += blockDim.x)
+        pe_freq[k] = exp2(-(2.0 * k / (double)sh.d_c) * sh.log2_pe_base);
+    for (int k = threadIdx.x; k < sh.d_r / 2; k += blockDim.x)
+        rope_freq[k] = exp2(-(2.0 * k / (double)sh.d_r) * sh.log2_rope_base);
+    __syncthreads();
+    const int t0 = a.t0;
+    const int j = t0 / sh.s + blockIdx.x * 8 + warp;
+    if (j >= (t0 + Tn - 1) / sh.s + 1) return;
+    const int ua = max(j * sh.s, t0), nu = min((j + 1) * sh.s, t0 + Tn) - ua;
+    const int lu0 = ua - t0;
+    const float* seed = (j * sh.s < t0 && a.open_slot_in) ? a.open_slot_in + (size_t)b * sh.D : nullptr;
+    // this lane's channels: latent k0 = 8 lane + 256 q (q < 2), RoPE pairs lane + 32 q (q < 2)
+    float al[2][8], ar[2][2];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+        const int k0 = lane * 8 + 256 * q;
+#pragma unroll
+        for (int v = 0; v < 8; ++v) al[q][v] = (seed && k0 < sh.d_c) ? seed[k0 + v] : 0.f;
+        const int kp = lane + 32 * q;
+        ar[q][0] = (seed && kp < sh.d_r / 2) ? seed[sh.d_c + 2 * kp] : 0.f;
+        ar[q][1] = (seed && kp < sh.d_r / 2) ? seed[sh.d_c + 2 * kp + 1] : 0.f;
+    }
+    float* vs = vsh[warp];
+    float* ws = wsh[warp];
+    for (int uo = 0; uo < nu; ++uo) {
+        const int u = ua + uo, lu = lu0 + uo;
+        const T* cu = (const T*)a.c + ((size_t)b * Tn + lu) * sh.d_c;
+        const T* ku = (const T*)a.kr + ((size_t)b * Tn + lu) * sh.d_r;
+        if (sh.gate_mode == 4) {
+            for (int k = lane; k < sh.D; k += 32) ws[k] = a.gate_in[((size_t)b * Tn + lu) * sh.D + k];
+        } else {
+            const int r = u % sh.s;
+            for (int kp = lane; kp < sh.d_c / 2; kp += 32) {
+                float sn, cs;
+                pair_sincos_f(u, pe_freq[kp], &sn, &cs);
+                vs[2 * kp] = to_f<T>(cu[2 * kp]) * sn;
+                vs[2 * kp + 1] = to_f<T>(cu[2 * kp + 1]) * cs;
+            }
+            __syncwarp();
+            const float* G = a.gate_w + (size_t)r * sh.d_c * sh.D;
+            for (int k = lane; k < sh.D; k += 32) {
+                float z = a.gate_b[(size_t)r * sh.D + k];
+                for (int i = 0; i < sh.d_c; ++i) z = fmaf(vs[i], G[(size_t)i * sh.D + k], z);
+                ws[k] = sigmoidf_(z);
+            }
+        }
+        __syncwarp();
+        PT* Pu = P + ((size_t)b * Tn + lu) * sh.D;
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const int k0 = lane * 8 + 256 * q;
+            if (k0 < sh.d_c) {
+                float x[8];
+                load8<T>(cu + k0, x);
+#pragma unroll
+                for (int v = 0; v < 8; ++v) al[q][v] = fmaf(ws[k0 + v], x[v], al[q][v]);
+                store8<PT>(Pu + k0, al[q]);
+            }
+            const int kp = lane + 32 * q;
+            if (kp < sh.d_r / 2) {
+                float sn, cs;
+                pair_sincos_f(u, rope_freq[kp], &sn, &cs);
+                if (rope_tab && b == 0) rope_tab[(size_t)lu * (sh.d_r / 2) + kp] = make_float2(cs, sn);
+                const float x0 = to_f<T>(ku[2 * kp]), x1 = to_f<T>(ku[2 * kp + 1]);
+                ar[q][0] = fmaf(ws[sh.d_c + 2 * kp], x0 * cs - x1 * sn, ar[q][0]);
+                ar[q][1] = fmaf(ws[sh.d_c + 2 * kp + 1], x0 * sn + x1 * cs, ar[q][1]);
+                Pu[sh.d_c + 2 * kp] = from_f<PT>(ar[q][0]);
+                Pu[sh.d_c + 2 * kp + 1] = from_f<PT>(ar[q][1]);
+            }
+        }
+        __syncwarp();                    // vs / ws of this token are read
+    }
+    T* slot = (T*)a.cache_out + ((size_t)b * sh.max_slots + j) * sh.D;
+    float* open = (ua + nu == t0 + Tn && a.open_slot_out) ? a.open_slot_out + (size_t)b * sh.D : nullptr;
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+        const int k0 = lane * 8 + 256 * q;
+        if (k0 < sh.d_c) {
+            store8<T>(slot + k0, al[q]);
+            if (open) store8<float>(open + k0, al[q]);
+        }
+        const int kp = lane + 32 * q;
+        if (kp < sh.d_r / 2) {
+            slot[sh.d_c + 2 * kp] = from_f<T>(ar[q][0]);
+            slot[sh.d_c + 2 * kp + 1] = from_f<T>(ar[q][1]);
+            if (open) {
+                open[sh.d_c + 2 * kp] = ar[q][0];
+                open[sh.d_c + 2 * kp + 1] = ar[q][1];
+            }
         }
     }
 }

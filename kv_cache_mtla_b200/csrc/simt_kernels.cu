@@ -244,7 +244,10 @@ cudaError_t prefill_impl(const PrefillArgs& a_in, cudaStream_t st, uint64_t* lau
     cudaError_t e = prefill_seed(a, ws + p_bytes + align256((size_t)sh.B * a.T * sh.H * sh.D * sizeof(float)), st);
     if (e != cudaSuccess) return e;
     const int n_slots = (a.t0 + a.T - 1) / sh.s - a.t0 / sh.s + 1;    // slots the chunk touches
-    k_prefill_scan<T, float><<<dim3((n_slots + 7) / 8, sh.B), 256, 0, st>>>(a, P);
+    if (sh.gate_mode >= 3)
+        k_prefill_scan_channel<T, float><<<dim3((n_slots + 7) / 8, sh.B), 256, 0, st>>>(a, P);
+    else
+        k_prefill_scan<T, float><<<dim3((n_slots + 7) / 8, sh.B), 256, 0, st>>>(a, P);
     k_prefill_absorb<T><<<dim3(sh.B * a.T, sh.H), 128, 0, st>>>(sh, (const T*)a.q_c, (const T*)a.q_r,
                                                                  (const T*)a.w_uk, a.T, a.t0, qt);
     const int64_t rows = (int64_t)a.T * sh.H;

@@ -774,7 +774,10 @@ cudaError_t tc_prefill(const PrefillArgs& a_in, cudaStream_t st, uint64_t* launc
     p.status = a.status;
 
     const int n_slots = (a.t0 + T - 1) / sh.s - a.t0 / sh.s + 1;    // slots the chunk touches
-    k_prefill_scan<bf16, bf16><<<dim3((n_slots + 7) / 8, sh.B), 256, 0, st>>>(a, P, (float2*)p.rope_tab);
+    if (sh.gate_mode >= 3)
+        k_prefill_scan_channel<bf16, bf16><<<dim3((n_slots + 7) / 8, sh.B), 256, 0, st>>>(a, P, (float2*)p.rope_tab);
+    else
+        k_prefill_scan<bf16, bf16><<<dim3((n_slots + 7) / 8, sh.B), 256, 0, st>>>(a, P, (float2*)p.rope_tab);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return note_error("k_prefill_scan launch", e);
 

@@ -18,6 +18,7 @@ from dataclasses import dataclass, replace
 import torch
 
 GATE_COMPUTED, GATE_SUPPLIED, GATE_UNIT = 0, 1, 2
+GATE_CHANNEL_COMPUTED, GATE_CHANNEL_SUPPLIED = 3, 4
 
 
 @dataclass(frozen=True)
@@ -75,14 +76,19 @@ def _gen(seed: int) -> torch.Generator:
 
 
 def weights(wl: Workload, seed_offset: int = 0) -> dict:
-    """W_UK, W_UV [H,d_h,d_c] (storage dtype values), gate_w [s,d_c], gate_b [s] (fp32)."""
+    """W_UK, W_UV [H,d_h,d_c] (storage dtype values), gate_w [s,d_c], gate_b [s]
+    (fp32); with the per-channel computed gate gate_w [s,d_c,D], gate_b [s,D]."""
     g = _gen(wl.seed * 1000 + 17 + seed_offset)
     std = 1.0 / (wl.d_c ** 0.5)
     w_uk = _round(torch.randn(wl.H, wl.d_h, wl.d_c, generator=g) * std, wl)
     w_uv = _round(torch.randn(wl.H, wl.d_h, wl.d_c, generator=g) * std, wl)
     gstd = (1.0 / wl.d_c ** 0.5) if wl.gate_w_fan_in else wl.gate_w_std
-    gate_w = torch.randn(wl.s, wl.d_c, generator=g) * gstd
-    gate_b = torch.zeros(wl.s)
+    if wl.gate_mode == GATE_CHANNEL_COMPUTED:
+        gate_w = torch.randn(wl.s, wl.d_c, wl.D, generator=g) * gstd
+        gate_b = torch.zeros(wl.s, wl.D)
+    else:
+        gate_w = torch.randn(wl.s, wl.d_c, generator=g) * gstd
+        gate_b = torch.zeros(wl.s)
     return dict(w_uk=w_uk, w_uv=w_uv, gate_w=gate_w, gate_b=gate_b)
 
 
@@ -91,7 +97,7 @@ def tokens(wl: Workload, T: int, stream: int = 0) -> dict:
 
     c [B,T,d_c], kr [B,T,d_r] (pre-RoPE), qc [B,T,H,d_h], qr [B,T,H,d_r]
     (pre-RoPE), all N(0,1) in the storage dtype; gate_in [B,T] = sigmoid(N(0,1))
-    (fp32) for supplied-gate workloads, else None. ``stream`` selects an
+    (fp32) for supplied-gate workloads ([B,T,D] for per-channel ones), else None. ``stream`` selects an
     independent draw (e.g. the prefix vs the decode steps)."""
     g = _gen(wl.seed * 1000 + 101 + 7919 * stream)
     B, H = wl.B, wl.H
@@ -102,6 +108,8 @@ def tokens(wl: Workload, T: int, stream: int = 0) -> dict:
     gate_in = None
     if wl.gate_mode == GATE_SUPPLIED:
         gate_in = torch.sigmoid(torch.randn(B, T, generator=g))
+    elif wl.gate_mode == GATE_CHANNEL_SUPPLIED:
+        gate_in = torch.sigmoid(torch.randn(B, T, wl.D, generator=g))
     return dict(c=c, kr=kr, qc=qc, qr=qr, gate_in=gate_in)
 
 

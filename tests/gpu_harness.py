@@ -68,7 +68,7 @@ class Problem:
         self.buf = mtla.Buffers.allocate(self.cfg, self.weights, max_tokens)
 
     def gate_ptrs(self):
-        if self.wl.gate_mode == inputs.GATE_COMPUTED:
+        if self.wl.gate_mode in (inputs.GATE_COMPUTED, inputs.GATE_CHANNEL_COMPUTED):
             return self.buf.gate_w, self.buf.gate_b
         return None, None
 
