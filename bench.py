@@ -738,7 +738,10 @@ def run_kernel_workload(args):
         print(json.dumps(measure_speech(args.steps, flush, 1, 0)), flush=True)
         return
     hbm, _, peak_kind = _peaks()
-    wl = inputs.WORKLOADS[name.split(":")[0]]
+    if name == "large_latent_step":              # one decode step of the contract workload
+        wl = inputs.LARGE_LATENT
+    else:
+        wl = inputs.WORKLOADS[name.split(":")[0]]
     if ":" in name:
         wl = wl.with_(s=int(name.split(":")[1]))
     call, nbytes = _decode_call(wl, wl.T)
@@ -766,7 +769,7 @@ def main():
                     help="contract line only (no prefill / speech / stride-sweep sub-objects)")
     ap.add_argument("--workload", default="large_latent",
                     help="large_latent (the contract line), or a kernel-level line of "
-                         "stride_sweep[:s], prefill, speech_decode or beam_reorder")
+                         "large_latent_step, stride_sweep[:s], prefill, speech_decode or beam_reorder")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     ws, rank = _dist()
