@@ -210,6 +210,16 @@ mtla_status mtla_prefill_from(const mtla_config* cfg, int32_t t0, int32_t T,
                               void* out, void* cache, float* open_slot,
                               void* workspace, size_t workspace_bytes, void* stream);
 
+/* Dense projection on the tensor cores: y[M, N] = x[M, K] . w[N, K]^T with
+ * bf16 operands and result and fp32 accumulation. The layer around the path
+ * ("Multi-head Temporal Latent Attention", Method: MLA's low-rank compression
+ * kept, h_t projected to the shared latent c_t, the decoupled key and the
+ * queries; the heads' outputs projected back by W_O) is made of these.
+ *   x [M, K], w [N, K], y [M, N]: bf16, row-major, contiguous, 16-byte aligned.
+ *   K a multiple of 8 (TMA row pitch); M, N, K >= 1. INVALID_ARG otherwise.
+ * Returns OK once enqueued on `stream`. */
+mtla_status mtla_linear(const void* x, const void* w, void* y, int32_t M, int32_t N, int32_t K, void* stream);
+
 /* Decode step without a workspace argument, for callers that cannot allocate
  * device memory themselves: code inside a host framework whose pool allocator
  * owns all device memory and forbids raw cudaMalloc, serving loops that cannot

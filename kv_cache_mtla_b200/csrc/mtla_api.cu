@@ -295,6 +295,18 @@ mtla_status mtla_prefill_from(const mtla_config* cfg, int32_t t0, int32_t T, con
                           open_slot, open_slot, workspace, workspace_bytes, stream);
 }
 
+mtla_status mtla_linear(const void* x, const void* w, void* y, int32_t M, int32_t N, int32_t K, void* stream) {
+    if (M <= 0 || N <= 0 || K <= 0 || K % 8 != 0) return MTLA_ERR_INVALID_ARG;
+    if (!x || !w || !y || !aligned16(x) || !aligned16(w) || !aligned16(y)) return MTLA_ERR_INVALID_ARG;
+    g_error_detail[0] = 0;
+    int* status = nullptr;
+    if (note_error("device status word", status_ptr(&status)) != cudaSuccess) return MTLA_ERR_CUDA;
+    uint64_t n = 0;
+    cudaError_t e = gemm_bf16(x, K, w, K, y, N, M, N, K, status, (cudaStream_t)stream, &n);
+    g_launches += n;
+    return e == cudaSuccess ? MTLA_OK : MTLA_ERR_CUDA;
+}
+
 mtla_status mtla_get_device_status(void* stream) {
     int* p = nullptr;
     if (status_ptr(&p) != cudaSuccess) return MTLA_ERR_CUDA;

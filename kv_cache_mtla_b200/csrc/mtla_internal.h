@@ -88,6 +88,11 @@ bool tc_prefill_supported(const Shape& sh);
 size_t tc_prefill_workspace(const Shape& sh, int T);
 cudaError_t tc_prefill(const PrefillArgs& a, cudaStream_t st, uint64_t* launches);
 
+// y[M, N] = x[M, K] . w[N, K]^T, bf16 in and out, fp32 accumulation (gemm.cu).
+// Rows ldx / ldw / ldy elements apart (ldx, ldw multiples of 8).
+cudaError_t gemm_bf16(const void* x, int ldx, const void* w, int ldw, void* y, int ldy, int M, int N, int K,
+                      int* status, cudaStream_t st, uint64_t* launches);
+
 // Beam-search reorder of the slot cache and open slots (cache_ops.cu).
 cudaError_t reorder_cache(const Shape& sh, size_t elem_bytes, const int32_t* src, const int32_t* n_tokens,
                           const void* cache_in, const float* open_in, void* cache_out, float* open_out,

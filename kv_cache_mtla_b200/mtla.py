@@ -75,6 +75,8 @@ def load() -> ctypes.CDLL:
     lib.mtla_prefill.restype = ctypes.c_int
     lib.mtla_prefill_from.argtypes = [cp, ctypes.c_int32, ctypes.c_int32] + [_vp] * 12 + [_vp, ctypes.c_size_t, _vp]
     lib.mtla_prefill_from.restype = ctypes.c_int
+    lib.mtla_linear.argtypes = [_vp, _vp, _vp, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _vp]
+    lib.mtla_linear.restype = ctypes.c_int
     lib.mtla_decode_step_noalloc.argtypes = [cp] + [_vp] * 13 + [_vp]
     lib.mtla_decode_step_noalloc.restype = ctypes.c_int
     lib.mtla_reorder_cache.argtypes = [cp] + [_vp] * 6 + [_vp]
@@ -179,6 +181,17 @@ def prefill_from(cfg, t0, T, c, kr, q_c, q_r, w_uk, w_uv, gate_w, gate_b, gate_i
         _ptr(open_slot), _ptr(workspace), ws, _stream(stream))
     if check and st != OK:
         raise MtlaError(st, "mtla_prefill_from")
+    return st
+
+
+def linear(x, w, y, stream=None, check=True) -> int:
+    """Forward to ``mtla_linear``: y[M, N] = x[M, K] . w[N, K]^T (bf16)."""
+    M, K = x.shape[-2] if x.dim() > 1 else 1, x.shape[-1]
+    M = x.numel() // K
+    N = w.shape[0]
+    st = load().mtla_linear(_ptr(x), _ptr(w), _ptr(y), int(M), int(N), int(K), _stream(stream))
+    if check and st != OK:
+        raise MtlaError(st, "mtla_linear")
     return st
 
 

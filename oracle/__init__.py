@@ -111,6 +111,7 @@ def _load():
         _lib.orc_prefill_explicit.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int32] + [_P] * 10
         _lib.orc_prefill_from.argtypes = [ctypes.POINTER(_Cfg)] + [ctypes.c_int32] * 3 + [_P] * 15
         _lib.orc_set_fault.argtypes = [ctypes.c_int]
+        _lib.orc_linear.argtypes = [ctypes.c_int64] * 3 + [_P] * 3
         _lib.orc_reorder_cache.argtypes = [ctypes.c_int32] * 5 + [ctypes.c_void_p] * 6
         _lib.orc_reorder_cache.restype = ctypes.c_int
     return _lib
@@ -256,6 +257,16 @@ def prefill_explicit(cfg: Cfg, c, kr, qc, qr, w_uk, w_uv, G=None, g=None, gate_i
     _load().orc_prefill_explicit(ctypes.byref(cfg.c()), T, _p(c), _p(kr), _p(qc), _p(qr),
                                  _p(w_uk), _p(w_uv), _p(G), _p(g), _p(gate_in), _p(out))
     return out
+
+
+def linear(x, w) -> np.ndarray:
+    """y = x . w^T in float64 (x [..., K], w [N, K])."""
+    x, w = _d(x), _d(w)
+    K = x.shape[-1]
+    M = x.size // K
+    y = np.zeros(x.shape[:-1] + (w.shape[0],))
+    _load().orc_linear(M, w.shape[0], K, _p(np.ascontiguousarray(x.reshape(M, K))), _p(w), _p(y))
+    return y
 
 
 def reorder_cache(s: int, src, n_tokens, cache_in, open_in, cache_out, open_out) -> int:

@@ -588,6 +588,17 @@ void orc_prefill_explicit(const orc_cfg* cfg, int32_t T, const double* c, const 
     free(P);
 }
 
+/* y[M, N] = x[M, K] . w[N, K]^T, the definition as three loops (float64). */
+void orc_linear(int64_t M, int64_t N, int64_t K, const double* x, const double* w, double* y) {
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < M; ++i)
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k) acc += x[i * K + k] * w[n * K + k];
+            y[i * N + n] = acc;
+        }
+}
+
 /* Beam-search reorder of the cache (the authors' toolkit decodes with
  * parallel beam search: its project page on sourcepulse.org, "Highlighted
  * Details"). Destination b takes over the cache of its parent j = src[b]:

@@ -645,3 +645,12 @@ def test_reorder_bad_parent_and_capacity():
     co, oo = np.zeros_like(ci), np.zeros_like(oi)
     assert oracle.reorder_cache(2, [1, 0], [4, 5], ci, oi, co, oo) == 3
     assert co[0].sum() == 0 and co[1].sum() == 4
+
+
+def test_linear_is_the_library_matmul():
+    """orc_linear, the projections' reference, equals numpy's matmul (a library
+    routine) on ragged shapes, and a transposed or offset read would not."""
+    rng = np.random.default_rng(3)
+    for M, N, K in ((1, 1, 1), (7, 5, 3), (33, 17, 70)):
+        x, w = rng.standard_normal((M, K)), rng.standard_normal((N, K))
+        assert np.max(np.abs(oracle.linear(x, w) - x @ w.T)) < 1e-12
