@@ -269,6 +269,29 @@ def linear(x, w) -> np.ndarray:
     return y
 
 
+def layer_forward(cfg: Cfg, t0: int, cache_in, acc_in, h, W: dict, G=None, g=None, gate_in=None):
+    """The MTLA layer around the path, T tokens at positions t0.. continuing
+    from the cache state after t0 tokens ("Multi-head Temporal Latent
+    Attention", Method: MLA's low-rank compression kept -- h_t projected to the
+    shared latent c_t and the decoupled key k_t, the queries projected per
+    head; "Multi-Head Latent Attention and Sparse Indexers": the heads' outputs
+    concatenated and projected back by W_O):
+      c = h W_DKV^T [B,T,d_c]    k = h W_KR^T [B,T,d_R]
+      qC = h W_Q^T [B,T,H,d_h]   qR = h W_QR^T [B,T,H,d_R]
+      o = the path (prefill_from) [B,T,H,d_h]   y = o W_O^T [B,T,d_model]
+    W holds w_dkv [d_c,dm], w_kr [d_R,dm], w_q [H*d_h,dm], w_qr [H*d_R,dm],
+    w_uk, w_uv [H,d_h,d_c], w_o [dm, H*d_h]. Returns dict(y, cache, acc)."""
+    h = _d(h)
+    B, T, _ = h.shape
+    c = linear(h, W["w_dkv"])
+    kr = linear(h, W["w_kr"])
+    qc = linear(h, W["w_q"]).reshape(B, T, cfg.H, cfg.d_h)
+    qr = linear(h, W["w_qr"]).reshape(B, T, cfg.H, cfg.d_r)
+    r = prefill_from(cfg, t0, cache_in, acc_in, c, kr, qc, qr, W["w_uk"], W["w_uv"], G, g, gate_in)
+    y = linear(r["out"].reshape(B, T, cfg.H * cfg.d_h), W["w_o"])
+    return dict(y=y, cache=r["cache"], acc=r["acc"])
+
+
 def reorder_cache(s: int, src, n_tokens, cache_in, open_in, cache_out, open_out) -> int:
     """Beam-search reorder: destination b takes the filled slots and the open
     slot of parent src[b] (``orc_reorder_cache``). ``cache_in``/``cache_out``

@@ -19,7 +19,9 @@ mathematics fix, none of which retypes the oracle's own formulas.
   equals the same number of incremental decode steps;
 - per-channel gate: equal channels reduce it to the scalar gate (computed and
   supplied); G = 0 gives a closed form; one value worked by hand; decoding
-  equals the parallel form.
+  equals the parallel form;
+- the layer around the path: block-selecting projections make it the path
+  itself; folding W_UK into W_Q and W_UV into W_O gives the same output.
 Finally, each planted mistake in the oracle must trip at least one pin.
 """
 import math
@@ -487,6 +489,61 @@ def pin_channel_incremental_equals_parallel():
     return True
 
 
+def _layer_problem(B, H, d_h, d_c, d_r, s, T, dm, seed):
+    cfg, p = _rand_problem(B, H, d_h, d_c, d_r, s, T, seed)
+    rng = np.random.default_rng(seed + 500)
+    W = dict(w_dkv=rng.standard_normal((d_c, dm)) / math.sqrt(dm),
+             w_kr=rng.standard_normal((d_r, dm)) / math.sqrt(dm),
+             w_q=rng.standard_normal((H * d_h, dm)) / math.sqrt(dm),
+             w_qr=rng.standard_normal((H * d_r, dm)) / math.sqrt(dm),
+             w_uk=p["w_uk"], w_uv=p["w_uv"],
+             w_o=rng.standard_normal((dm, H * d_h)) / math.sqrt(H * d_h))
+    h = rng.standard_normal((B, T, dm))
+    return cfg, p, W, h
+
+
+def pin_layer_selection_is_the_path():
+    """Projections that select blocks of h (h = [c | k | qC | qR | 0]) and a W_O
+    that copies o into the first columns make the layer the path itself: y's
+    first H*d_h columns are the path's output, the rest zero. A transposed or
+    misplaced projection breaks this."""
+    B, H, d_h, d_c, d_r, s, T = 2, 2, 4, 8, 4, 3, 9
+    cfg, p = _rand_problem(B, H, d_h, d_c, d_r, s, T, seed=130)
+    widths = [d_c, d_r, H * d_h, H * d_r]
+    dm = sum(widths) + 3
+    eye = np.eye(dm)
+    off = np.cumsum([0] + widths)
+    W = dict(w_dkv=eye[off[0]:off[1]], w_kr=eye[off[1]:off[2]], w_q=eye[off[2]:off[3]], w_qr=eye[off[3]:off[4]],
+             w_uk=p["w_uk"], w_uv=p["w_uv"], w_o=np.eye(dm, H * d_h))
+    h = np.concatenate([p["c"], p["kr"], p["qc"].reshape(B, T, -1), p["qr"].reshape(B, T, -1),
+                        np.zeros((B, T, 3))], axis=2)
+    got = oracle.layer_forward(cfg, 0, np.zeros((B, 0, cfg.D)), np.zeros((B, cfg.D)), h, W, p["G"], p["g"])
+    ref = oracle.prefill(cfg, p["c"], p["kr"], p["qc"], p["qr"], p["w_uk"], p["w_uv"], p["G"], p["g"])
+    return (np.max(np.abs(got["y"][:, :, :H * d_h] - ref["out"].reshape(B, T, -1))) < 1e-12
+            and np.all(got["y"][:, :, H * d_h:] == 0.0) and np.max(np.abs(got["cache"] - ref["cache"])) < 1e-12)
+
+
+def pin_layer_absorption_fold():
+    """W_UK folded into W_Q and W_UV folded into W_O ("Multi-Head Latent
+    Attention and Sparse Indexers", "Latent attention changes the
+    representation"): the layer with per-head query weights W_UK[h]^T W_Q[h]
+    (so the path's qC is the absorbed latent query and its W_UK the identity) and
+    output weights W_O[:, h] W_UV[h] (the path's W_UV the identity, d_h = d_c)
+    gives the same y."""
+    B, H, d_h, d_c, d_r, s, T, dm = 2, 3, 4, 8, 4, 2, 7, 12
+    cfg, p, W, h = _layer_problem(B, H, d_h, d_c, d_r, s, T, dm, seed=140)
+    ref = oracle.layer_forward(cfg, 0, np.zeros((B, 0, cfg.D)), np.zeros((B, cfg.D)), h, W, p["G"], p["g"])
+    cf = oracle.Cfg(B, H, d_c, d_c, d_r, s, scale=1.0 / math.sqrt(d_h + d_r))
+    eye = np.repeat(np.eye(d_c)[None], H, axis=0)
+    wq = W["w_q"].reshape(H, d_h, dm)
+    wo = W["w_o"].reshape(dm, H, d_h)
+    Wf = dict(w_dkv=W["w_dkv"], w_kr=W["w_kr"], w_qr=W["w_qr"], w_uk=eye, w_uv=eye,
+              w_q=np.einsum("hic,him->hcm", W["w_uk"], wq).reshape(H * d_c, dm),
+              w_o=np.einsum("mhi,hic->mhc", wo, W["w_uv"]).reshape(dm, H * d_c))
+    got = oracle.layer_forward(cf, 0, np.zeros((B, 0, cf.D)), np.zeros((B, cf.D)), h, Wf, p["G"], p["g"])
+    return np.max(np.abs(got["y"] - ref["y"])) < 1e-12
+
+
 PINS = {
     "cache_footprint": pin_cache_footprint,
     "s1_is_mla_sdpa": pin_s1_is_mla_sdpa,
@@ -507,6 +564,8 @@ PINS = {
     "channel_gate_closed_form": pin_channel_gate_closed_form,
     "channel_gate_value": pin_channel_gate_value,
     "channel_incremental_equals_parallel": pin_channel_incremental_equals_parallel,
+    "layer_selection_is_the_path": pin_layer_selection_is_the_path,
+    "layer_absorption_fold": pin_layer_absorption_fold,
 }
 
 
