@@ -26,6 +26,8 @@ back inside one timed region, pipelined on a copy stream.
 
 Sub-objects measure the other workloads, each over its own clock-sampled timed
 region: `prefill` (B=8, T=8192, s=2: TFLOP/s of the masked attention),
+`layer` (the same sizes through the whole layer with d_model=512: the
+projections, the path and W_O; and the largest projection GEMM alone),
 `speech_decode` (B=16, H=8, a 1024-token prefix then 256 decode steps:
 decode tokens/s separately from the prefix), `stride_sweep` (B=64, N=4096,
 s=1..4: latent-cache GB/s of one decode step). `cpu_baseline` and
@@ -556,6 +558,56 @@ def measure_speech(n, flush, ws, rank):
             "l2": L2Flush.desc + " step"}
 
 
+def measure_layer(n, flush, ws, rank):
+    """The MTLA layer around the path at the prefill workload's sizes (B=8,
+    T=8192, d_model=512, H=8, d_h=64, d_c=256, d_R=32, s=2): the four input
+    projections, the path, the output projection, all through
+    mtla_layer_forward; and the largest projection GEMM alone (65536 x 512 x
+    512) against the bf16 peak."""
+    _, tflops_peak, peak_kind = _peaks()
+    wl = inputs.PREFILL.with_(seed=inputs.PREFILL.seed + 1000 * rank)
+    dm, T = 512, wl.T
+    cfg = mtla.make_config(wl.B, wl.H, wl.d_h, wl.d_c, wl.d_r, wl.s, (T + wl.s - 1) // wl.s,
+                           gate_mode=wl.gate_mode)
+    W = inputs.layer_weights(wl, dm)
+    dW = {k: v.to("cuda", torch.bfloat16 if k.startswith("w_") else torch.float32).contiguous()
+          for k, v in W.items()}
+    lw = mtla.layer_weights(dW)
+    wsb = torch.empty(mtla.layer_workspace_size(cfg, dm, T), dtype=torch.uint8, device="cuda")
+    cache = torch.empty(wl.B, cfg.max_slots, wl.D, dtype=torch.bfloat16, device="cuda")
+    op = torch.zeros(wl.B, wl.D, dtype=torch.float32, device="cuda")
+    h = inputs.hidden(wl, dm, T).to("cuda", torch.bfloat16)
+    y = torch.empty(wl.B, T, dm, dtype=torch.bfloat16, device="cuda")
+
+    def call():
+        mtla.layer_forward(cfg, dm, 0, T, h, lw, dW["gate_w"], dW["gate_b"], None, y, cache, op, wsb)
+    call_ms, attn_ms, clocks = _timed_calls(call, n, flush, ws)
+    M = wl.B * T
+    proj = 2 * M * dm * (wl.d_c + wl.d_r + wl.H * wl.d_h + wl.H * wl.d_r)
+    outp = 2 * M * wl.H * wl.d_h * dm
+    pairs = sum(t // wl.s + 1 for t in range(T))
+    attn = 2 * pairs * (wl.D + wl.d_c) * wl.B * wl.H
+    # the largest projection alone
+    x = torch.randn(M, dm, device="cuda").to(torch.bfloat16)
+    wq = dW["w_q"]
+    yq = torch.empty(M, wq.shape[0], dtype=torch.bfloat16, device="cuda")
+    g_ms, _, g_clocks = _timed_calls(lambda: mtla.linear(x, wq, yq), 4 * n, flush, ws, profile=False)
+    g_flops = 2 * M * dm * wq.shape[0]
+    g_tf = g_flops / (g_ms / 1e3) / 1e12
+    return {"workload": f"layer: B={wl.B}/rank, T={T}, d_model={dm}, H={wl.H}, d_h={wl.d_h}, d_c={wl.d_c}, "
+                        f"d_R={wl.d_r}, s={wl.s}: 4 input projections, the path, the output projection",
+            "call_ms": call_ms, "attention_kernel_ms": attn_ms,
+            "TFLOPs": (proj + outp + attn) * ws / (call_ms / 1e3) / 1e12,
+            "flops_per_call": {"projections": proj, "output_projection": outp, "attention": attn},
+            "clocks": clocks,
+            "gemm": {"shape": f"{M} x {wq.shape[0]} x {dm} (M x N x K)", "ms": g_ms,
+                     "roofline": {"kernel": "k_gemm", "bound": "tensor", "achieved": g_tf, "peak": tflops_peak,
+                                  "unit": "TFLOP/s", "frac": g_tf / tflops_peak,
+                                  "peak_source": f"{peak_kind} bf16_tflops (burst)"},
+                     "clocks": g_clocks},
+            "l2": L2Flush.desc + " call"}
+
+
 def _decode_call(wl, N, max_slots=None):
     """A decode step at position N-1 over a cache drawn directly (N-1 tokens)."""
     max_slots = max_slots or (N + wl.s - 1) // wl.s
@@ -737,6 +789,9 @@ def run_kernel_workload(args):
     if name.startswith("speech_decode"):
         print(json.dumps(measure_speech(args.steps, flush, 1, 0)), flush=True)
         return
+    if name == "layer":
+        print(json.dumps(measure_layer(args.steps, flush, 1, 0)), flush=True)
+        return
     hbm, _, peak_kind = _peaks()
     if name == "large_latent_step":              # one decode step of the contract workload
         wl = inputs.LARGE_LATENT
@@ -769,7 +824,7 @@ def main():
                     help="contract line only (no prefill / speech / stride-sweep sub-objects)")
     ap.add_argument("--workload", default="large_latent",
                     help="large_latent (the contract line), or a kernel-level line of "
-                         "large_latent_step, stride_sweep[:s], prefill, speech_decode or beam_reorder")
+                         "large_latent_step, stride_sweep[:s], prefill, speech_decode, layer or beam_reorder")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     ws, rank = _dist()
@@ -800,6 +855,8 @@ def run_contract(args, ws, rank):
         extras["speech_decode"] = measure_speech(320, flush, ws, rank)
         torch.cuda.empty_cache()
         extras["stride_sweep"] = measure_stride(6000, flush, ws, rank)
+        torch.cuda.empty_cache()
+        extras["layer"] = measure_layer(400, flush, ws, rank)
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         n_seq = 8

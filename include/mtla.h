@@ -220,6 +220,48 @@ mtla_status mtla_prefill_from(const mtla_config* cfg, int32_t t0, int32_t T,
  * Returns OK once enqueued on `stream`. */
 mtla_status mtla_linear(const void* x, const void* w, void* y, int32_t M, int32_t N, int32_t K, void* stream);
 
+/* The MTLA layer around the path ("Multi-head Temporal Latent Attention",
+ * Method: MLA's low-rank compression kept; "Multi-Head Latent Attention and
+ * Sparse Indexers", "Latent attention changes the representation"), bf16 only:
+ *   c = h W_DKV^T   k = h W_KR^T   qC = h W_Q^T (heads)   qR = h W_QR^T (heads)
+ *   o = the MTLA path on (c, k, qC, qR)       y = o W_O^T
+ * Every projection is an mtla_linear GEMM; the absorbed W_UK and W_UV stay in
+ * the path's kernels. The weights (all bf16, row-major, 16-byte aligned): */
+typedef struct {
+    const void* w_dkv;      /* [d_c, d_model]     latent down-projection              */
+    const void* w_kr;       /* [d_r, d_model]     decoupled key (RoPE in the path)     */
+    const void* w_q;        /* [H * d_h, d_model] per-head queries                      */
+    const void* w_qr;       /* [H * d_r, d_model] per-head RoPE query parts             */
+    const void* w_uk;       /* [H, d_h, d_c]      as for mtla_decode_step              */
+    const void* w_uv;       /* [H, d_h, d_c]                                           */
+    const void* w_o;        /* [d_model, H * d_h] output projection                    */
+} mtla_layer_weights;
+
+/* Scratch for mtla_layer_forward with T <= max_tokens and for
+ * mtla_layer_decode_step (the projections' outputs plus the path's scratch).
+ * d_model a positive multiple of 8. Host only. */
+mtla_status mtla_layer_workspace_size(const mtla_config* cfg, int32_t d_model, int32_t max_tokens, size_t* bytes);
+
+/* The layer over T tokens of every sequence at positions t0 .. t0+T-1,
+ * continuing from the cache state after t0 tokens (t0 = 0: from an empty
+ * cache; the path is mtla_prefill_from).
+ *   h [B, T, d_model] bf16 in;  y [B, T, d_model] bf16 out
+ *   cache, open_slot: as for mtla_prefill_from (in/out; open_slot not NULL)
+ *   gate_w, gate_b, gate_in: as for mtla_prefill_from
+ * cfg->dtype must be MTLA_BF16 (else UNSUPPORTED). Returns OK once enqueued. */
+mtla_status mtla_layer_forward(const mtla_config* cfg, int32_t d_model, int32_t t0, int32_t T, const void* h,
+                               const mtla_layer_weights* w, const float* gate_w, const float* gate_b,
+                               const float* gate_in, void* y, void* cache, float* open_slot,
+                               void* workspace, size_t workspace_bytes, void* stream);
+
+/* One decode step of the layer: h [B, d_model] (the new token of every
+ * sequence) -> y [B, d_model]; pos, cache, open_slot and the gates as for
+ * mtla_decode_step. cfg->dtype must be MTLA_BF16. */
+mtla_status mtla_layer_decode_step(const mtla_config* cfg, int32_t d_model, const void* h,
+                                   const mtla_layer_weights* w, const float* gate_w, const float* gate_b,
+                                   const float* gate_in, const int32_t* pos, void* cache, float* open_slot,
+                                   void* y, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Decode step without a workspace argument, for callers that cannot allocate
  * device memory themselves: code inside a host framework whose pool allocator
  * owns all device memory and forbids raw cudaMalloc, serving loops that cannot

@@ -307,6 +307,135 @@ mtla_status mtla_linear(const void* x, const void* w, void* y, int32_t M, int32_
     return e == cudaSuccess ? MTLA_OK : MTLA_ERR_CUDA;
 }
 
+// The layer around the path: activations of M = B*T tokens in the workspace
+// (c, k, qC, qR, o; bf16, 256-byte aligned regions), then the path's scratch.
+struct LayerWs {
+    size_t c, kr, qc, qr, o, path, total;
+};
+static LayerWs layer_ws_layout(const Shape& sh, int64_t M, size_t path_bytes) {
+    LayerWs l;
+    l.c = 0;
+    l.kr = l.c + align256((size_t)M * sh.d_c * 2);
+    l.qc = l.kr + align256((size_t)M * sh.d_r * 2);
+    l.qr = l.qc + align256((size_t)M * sh.H * sh.d_h * 2);
+    l.o = l.qr + align256((size_t)M * sh.H * sh.d_r * 2);
+    l.path = l.o + align256((size_t)M * sh.H * sh.d_h * 2);
+    l.total = l.path + path_bytes;
+    return l;
+}
+
+static mtla_status layer_check(const mtla_config* cfg, int32_t d_model, Shape* sh) {
+    mtla_status st = check_config(cfg, sh);
+    if (st != MTLA_OK) return st;
+    if (d_model <= 0 || d_model % 8 != 0) return MTLA_ERR_INVALID_ARG;
+    if (cfg->dtype != MTLA_BF16) return MTLA_ERR_UNSUPPORTED;
+    return MTLA_OK;
+}
+
+static mtla_status layer_weights_ok(const mtla_layer_weights* w) {
+    if (!w) return MTLA_ERR_INVALID_ARG;
+    const void* p[] = {w->w_dkv, w->w_kr, w->w_q, w->w_qr, w->w_uk, w->w_uv, w->w_o};
+    for (const void* q : p)
+        if (!q || !aligned16(q)) return MTLA_ERR_INVALID_ARG;
+    return MTLA_OK;
+}
+
+// The four projections of M tokens of h into the workspace activations.
+static cudaError_t layer_project(const Shape& sh, int d_model, int64_t M, const void* h,
+                                 const mtla_layer_weights* w, char* ws, const LayerWs& l, int* status,
+                                 cudaStream_t st, uint64_t* n) {
+    const int m = (int)M;
+    cudaError_t e = gemm_bf16(h, d_model, w->w_dkv, d_model, ws + l.c, sh.d_c, m, sh.d_c, d_model, status, st, n);
+    if (e == cudaSuccess) e = gemm_bf16(h, d_model, w->w_kr, d_model, ws + l.kr, sh.d_r, m, sh.d_r, d_model, status, st, n);
+    if (e == cudaSuccess)
+        e = gemm_bf16(h, d_model, w->w_q, d_model, ws + l.qc, sh.H * sh.d_h, m, sh.H * sh.d_h, d_model, status, st, n);
+    if (e == cudaSuccess)
+        e = gemm_bf16(h, d_model, w->w_qr, d_model, ws + l.qr, sh.H * sh.d_r, m, sh.H * sh.d_r, d_model, status, st, n);
+    return e;
+}
+
+mtla_status mtla_layer_workspace_size(const mtla_config* cfg, int32_t d_model, int32_t max_tokens, size_t* bytes) {
+    Shape sh;
+    if (!bytes || max_tokens < 0) return MTLA_ERR_INVALID_ARG;
+    mtla_status st = layer_check(cfg, d_model, &sh);
+    if (st != MTLA_OK) return st;
+    const size_t dec = layer_ws_layout(sh, sh.B, decode_ws(cfg, sh)).total;
+    const size_t pre = max_tokens > 0 ? layer_ws_layout(sh, (int64_t)sh.B * max_tokens, prefill_ws(cfg, sh, max_tokens)).total : 0;
+    *bytes = dec > pre ? dec : pre;
+    return MTLA_OK;
+}
+
+mtla_status mtla_layer_forward(const mtla_config* cfg, int32_t d_model, int32_t t0, int32_t T, const void* h,
+                               const mtla_layer_weights* w, const float* gate_w, const float* gate_b,
+                               const float* gate_in, void* y, void* cache, float* open_slot, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+    Shape sh;
+    mtla_status st = layer_check(cfg, d_model, &sh);
+    if (st != MTLA_OK) return st;
+    if (T <= 0 || t0 < 0) return MTLA_ERR_INVALID_ARG;
+    if ((st = layer_weights_ok(w)) != MTLA_OK) return st;
+    const void* req[] = {h, y, cache, open_slot, workspace};
+    for (const void* p : req)
+        if (!p || !aligned16(p)) return MTLA_ERR_INVALID_ARG;
+    st = check_gate_ptrs(cfg, gate_w, gate_b, gate_in);
+    if (st != MTLA_OK) return st;
+    if (((int64_t)t0 + T + sh.s - 1) / sh.s > sh.max_slots) return MTLA_ERR_CAPACITY;
+    const int64_t M = (int64_t)sh.B * T;
+    const LayerWs l = layer_ws_layout(sh, M, prefill_ws(cfg, sh, T));
+    if (workspace_bytes < l.total) return MTLA_ERR_WORKSPACE;
+    char* ws = (char*)workspace;
+    g_error_detail[0] = 0;
+    int* status = nullptr;
+    if (note_error("device status word", status_ptr(&status)) != cudaSuccess) return MTLA_ERR_CUDA;
+    uint64_t n = 0;
+    cudaStream_t s_ = (cudaStream_t)stream;
+    cudaError_t e = layer_project(sh, d_model, M, h, w, ws, l, status, s_, &n);
+    g_launches += n;
+    if (e != cudaSuccess) return MTLA_ERR_CUDA;
+    st = prefill_common(cfg, t0, T, ws + l.c, ws + l.kr, ws + l.qc, ws + l.qr, w->w_uk, w->w_uv, gate_w, gate_b,
+                        gate_in, ws + l.o, cache, open_slot, open_slot, ws + l.path, workspace_bytes - l.path, stream);
+    if (st != MTLA_OK) return st;
+    n = 0;
+    e = gemm_bf16(ws + l.o, sh.H * sh.d_h, w->w_o, sh.H * sh.d_h, y, d_model, (int)M, d_model, sh.H * sh.d_h,
+                  status, s_, &n);
+    g_launches += n;
+    return e == cudaSuccess ? MTLA_OK : MTLA_ERR_CUDA;
+}
+
+mtla_status mtla_layer_decode_step(const mtla_config* cfg, int32_t d_model, const void* h,
+                                   const mtla_layer_weights* w, const float* gate_w, const float* gate_b,
+                                   const float* gate_in, const int32_t* pos, void* cache, float* open_slot,
+                                   void* y, void* workspace, size_t workspace_bytes, void* stream) {
+    Shape sh;
+    mtla_status st = layer_check(cfg, d_model, &sh);
+    if (st != MTLA_OK) return st;
+    if ((st = layer_weights_ok(w)) != MTLA_OK) return st;
+    const void* req[] = {h, y, pos, cache, open_slot, workspace};
+    for (const void* p : req)
+        if (!p || !aligned16(p)) return MTLA_ERR_INVALID_ARG;
+    st = check_gate_ptrs(cfg, gate_w, gate_b, gate_in);
+    if (st != MTLA_OK) return st;
+    const LayerWs l = layer_ws_layout(sh, sh.B, decode_ws(cfg, sh));
+    if (workspace_bytes < l.total) return MTLA_ERR_WORKSPACE;
+    char* ws = (char*)workspace;
+    g_error_detail[0] = 0;
+    int* status = nullptr;
+    if (note_error("device status word", status_ptr(&status)) != cudaSuccess) return MTLA_ERR_CUDA;
+    uint64_t n = 0;
+    cudaStream_t s_ = (cudaStream_t)stream;
+    cudaError_t e = layer_project(sh, d_model, sh.B, h, w, ws, l, status, s_, &n);
+    g_launches += n;
+    if (e != cudaSuccess) return MTLA_ERR_CUDA;
+    st = mtla_decode_step(cfg, ws + l.c, ws + l.kr, ws + l.qc, ws + l.qr, w->w_uk, w->w_uv, gate_w, gate_b, gate_in,
+                          pos, cache, open_slot, ws + l.o, ws + l.path, workspace_bytes - l.path, stream);
+    if (st != MTLA_OK) return st;
+    n = 0;
+    e = gemm_bf16(ws + l.o, sh.H * sh.d_h, w->w_o, sh.H * sh.d_h, y, d_model, sh.B, d_model, sh.H * sh.d_h, status,
+                  s_, &n);
+    g_launches += n;
+    return e == cudaSuccess ? MTLA_OK : MTLA_ERR_CUDA;
+}
+
 mtla_status mtla_get_device_status(void* stream) {
     int* p = nullptr;
     if (status_ptr(&p) != cudaSuccess) return MTLA_ERR_CUDA;

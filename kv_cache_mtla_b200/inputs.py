@@ -113,6 +113,28 @@ def tokens(wl: Workload, T: int, stream: int = 0) -> dict:
     return dict(c=c, kr=kr, qc=qc, qr=qr, gate_in=gate_in)
 
 
+def layer_weights(wl: Workload, d_model: int) -> dict:
+    """The layer's projections (storage dtype values): w_dkv [d_c, dm],
+    w_kr [d_R, dm], w_q [H d_h, dm], w_qr [H d_R, dm] ~ N(0,1)/sqrt(dm),
+    w_o [dm, H d_h] ~ N(0,1)/sqrt(H d_h); plus the path's W_UK, W_UV and
+    gate parameters from weights()."""
+    g = _gen(wl.seed * 1000 + 29)
+    f = d_model ** -0.5
+    w = dict(w_dkv=_round(torch.randn(wl.d_c, d_model, generator=g) * f, wl),
+             w_kr=_round(torch.randn(wl.d_r, d_model, generator=g) * f, wl),
+             w_q=_round(torch.randn(wl.H * wl.d_h, d_model, generator=g) * f, wl),
+             w_qr=_round(torch.randn(wl.H * wl.d_r, d_model, generator=g) * f, wl),
+             w_o=_round(torch.randn(d_model, wl.H * wl.d_h, generator=g) * (wl.H * wl.d_h) ** -0.5, wl))
+    w.update(weights(wl))
+    return w
+
+
+def hidden(wl: Workload, d_model: int, T: int, stream: int = 0) -> torch.Tensor:
+    """Layer inputs h [B, T, d_model] ~ N(0,1) in the storage dtype."""
+    g = _gen(wl.seed * 1000 + 313 + 7919 * stream)
+    return _round(torch.randn(wl.B, T, d_model, generator=g), wl)
+
+
 def synthetic_cache(wl: Workload, n_tokens: int, max_slots: int, stream: int = 0) -> dict:
     """A cache state that holds ``n_tokens`` tokens, drawn directly instead of
     scanned: every slot value N(0,1) in the storage dtype, the fp32 open-slot

@@ -58,6 +58,17 @@ _lib = None
 _vp = ctypes.c_void_p
 
 
+class LayerWeights(ctypes.Structure):
+    """Mirror of ``mtla_layer_weights`` (device pointers)."""
+    _fields_ = [("w_dkv", _vp), ("w_kr", _vp), ("w_q", _vp), ("w_qr", _vp), ("w_uk", _vp), ("w_uv", _vp),
+                ("w_o", _vp)]
+
+
+def layer_weights(d: dict) -> LayerWeights:
+    """LayerWeights from a dict of contiguous bf16 device tensors."""
+    return LayerWeights(*[_ptr(d[k]) for k in ("w_dkv", "w_kr", "w_q", "w_qr", "w_uk", "w_uv", "w_o")])
+
+
 def load() -> ctypes.CDLL:
     """Load libmtla.so (built by ``python -m kv_cache_mtla_b200.build``)."""
     global _lib
@@ -77,6 +88,14 @@ def load() -> ctypes.CDLL:
     lib.mtla_prefill_from.restype = ctypes.c_int
     lib.mtla_linear.argtypes = [_vp, _vp, _vp, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _vp]
     lib.mtla_linear.restype = ctypes.c_int
+    lp = ctypes.POINTER(LayerWeights)
+    lib.mtla_layer_workspace_size.argtypes = [cp, ctypes.c_int32, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)]
+    lib.mtla_layer_workspace_size.restype = ctypes.c_int
+    lib.mtla_layer_forward.argtypes = ([cp, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _vp, lp]
+                                       + [_vp] * 7 + [ctypes.c_size_t, _vp])
+    lib.mtla_layer_forward.restype = ctypes.c_int
+    lib.mtla_layer_decode_step.argtypes = [cp, ctypes.c_int32, _vp, lp] + [_vp] * 8 + [ctypes.c_size_t, _vp]
+    lib.mtla_layer_decode_step.restype = ctypes.c_int
     lib.mtla_decode_step_noalloc.argtypes = [cp] + [_vp] * 13 + [_vp]
     lib.mtla_decode_step_noalloc.restype = ctypes.c_int
     lib.mtla_reorder_cache.argtypes = [cp] + [_vp] * 6 + [_vp]
@@ -109,6 +128,14 @@ def _ptr(t):
     if not t.is_contiguous():
         raise ValueError("tensors passed to libmtla must be contiguous")
     return t.data_ptr()
+
+
+def _bf16(*tensors):
+    """The bf16-only calls take raw pointers: a tensor of another dtype would be
+    read as bf16 bytes, so refuse it here."""
+    for t in tensors:
+        if isinstance(t, torch.Tensor) and t.dtype != torch.bfloat16:
+            raise TypeError(f"expected a bfloat16 tensor, got {t.dtype}")
 
 
 def _stream(stream):
@@ -186,12 +213,47 @@ def prefill_from(cfg, t0, T, c, kr, q_c, q_r, w_uk, w_uv, gate_w, gate_b, gate_i
 
 def linear(x, w, y, stream=None, check=True) -> int:
     """Forward to ``mtla_linear``: y[M, N] = x[M, K] . w[N, K]^T (bf16)."""
+    _bf16(x, w, y)
     M, K = x.shape[-2] if x.dim() > 1 else 1, x.shape[-1]
     M = x.numel() // K
     N = w.shape[0]
     st = load().mtla_linear(_ptr(x), _ptr(w), _ptr(y), int(M), int(N), int(K), _stream(stream))
     if check and st != OK:
         raise MtlaError(st, "mtla_linear")
+    return st
+
+
+def layer_workspace_size(cfg: Config, d_model: int, max_tokens: int = 0) -> int:
+    n = ctypes.c_size_t(0)
+    st = load().mtla_layer_workspace_size(ctypes.byref(cfg), int(d_model), int(max_tokens), ctypes.byref(n))
+    if st != OK:
+        raise MtlaError(st, "mtla_layer_workspace_size")
+    return int(n.value)
+
+
+def layer_forward(cfg, d_model, t0, T, h, lw: LayerWeights, gate_w, gate_b, gate_in, y, cache, open_slot,
+                  workspace, stream=None, check=True) -> int:
+    """Forward to ``mtla_layer_forward`` (the layer over T tokens at t0..)."""
+    _bf16(h, y)
+    ws = workspace.numel() * workspace.element_size()
+    st = load().mtla_layer_forward(ctypes.byref(cfg), int(d_model), int(t0), int(T), _ptr(h), ctypes.byref(lw),
+                                   _ptr(gate_w), _ptr(gate_b), _ptr(gate_in), _ptr(y), _ptr(cache),
+                                   _ptr(open_slot), _ptr(workspace), ws, _stream(stream))
+    if check and st != OK:
+        raise MtlaError(st, "mtla_layer_forward")
+    return st
+
+
+def layer_decode_step(cfg, d_model, h, lw: LayerWeights, gate_w, gate_b, gate_in, pos, cache, open_slot, y,
+                      workspace, stream=None, check=True) -> int:
+    """Forward to ``mtla_layer_decode_step``."""
+    _bf16(h, y)
+    ws = workspace.numel() * workspace.element_size()
+    st = load().mtla_layer_decode_step(ctypes.byref(cfg), int(d_model), _ptr(h), ctypes.byref(lw), _ptr(gate_w),
+                                       _ptr(gate_b), _ptr(gate_in), _ptr(pos), _ptr(cache), _ptr(open_slot),
+                                       _ptr(y), _ptr(workspace), ws, _stream(stream))
+    if check and st != OK:
+        raise MtlaError(st, "mtla_layer_decode_step")
     return st
 
 

@@ -198,3 +198,17 @@ def test_prefill_from_rejects_bad_arguments_on_the_host(lib):
     assert st(3, 4, None) == mtla.ERR_INVALID_ARG
     assert st(-1, 4, fake) == mtla.ERR_INVALID_ARG
     assert st(30, 4, fake) == mtla.ERR_CAPACITY      # ceil(34 / 2) = 17 slots > 16
+
+
+def test_layer_refuses_fp32_and_bad_widths_on_the_host(lib):
+    """The layer is bf16 only; d_model must be a positive multiple of 8."""
+    cfg = _cfg()
+    assert mtla.layer_workspace_size(cfg, 512, 16) > mtla.workspace_size(cfg, 16)
+    for dm in (0, 12):
+        with pytest.raises(mtla.MtlaError) as e:
+            mtla.layer_workspace_size(cfg, dm, 16)
+        assert e.value.status == mtla.ERR_INVALID_ARG
+    cfg32 = mtla.make_config(2, 8, 64, 256, 32, 2, 16, dtype="fp32")
+    with pytest.raises(mtla.MtlaError) as e:
+        mtla.layer_workspace_size(cfg32, 512, 16)
+    assert e.value.status == mtla.ERR_UNSUPPORTED
