@@ -319,6 +319,16 @@ mtla_status mtla_reorder_cache(const mtla_config* cfg, const int32_t* src, const
                                const void* cache_in, const float* open_in,
                                void* cache_out, float* open_out, void* stream);
 
+/* Test hook for the failure path (no counterpart in the pages): launches one
+ * CTA that lands a TMA load of 2 KB from `scratch` (device memory, 16-byte
+ * aligned, at least 2 KB) and then waits, with the same bounded wait every
+ * kernel of the library uses but a limit of `limit_ns` (1 .. 1e9), on an
+ * mbarrier nothing arrives on. The wait runs out, MTLA_ERR_TIMEOUT is latched
+ * in the device status word, the load is drained and the CTA returns: no
+ * hang, no fault, and later calls run normally. INVALID_ARG for a bad
+ * argument. Returns OK once enqueued. */
+mtla_status mtla_test_wait_timeout(uint64_t limit_ns, void* scratch, void* stream);
+
 /* Synchronises `stream`, then returns and clears the status latched by
  * device-side checks on the current device since the last call (OK if none). */
 mtla_status mtla_get_device_status(void* stream);

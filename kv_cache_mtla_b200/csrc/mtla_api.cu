@@ -436,6 +436,17 @@ mtla_status mtla_layer_decode_step(const mtla_config* cfg, int32_t d_model, cons
     return e == cudaSuccess ? MTLA_OK : MTLA_ERR_CUDA;
 }
 
+mtla_status mtla_test_wait_timeout(uint64_t limit_ns, void* scratch, void* stream) {
+    if (!scratch || !aligned16(scratch) || limit_ns == 0 || limit_ns > 1000000000ull) return MTLA_ERR_INVALID_ARG;
+    g_error_detail[0] = 0;
+    int* status = nullptr;
+    if (note_error("device status word", status_ptr(&status)) != cudaSuccess) return MTLA_ERR_CUDA;
+    uint64_t n = 0;
+    cudaError_t e = wait_probe(limit_ns, scratch, status, (cudaStream_t)stream, &n);
+    g_launches += n;
+    return e == cudaSuccess ? MTLA_OK : MTLA_ERR_CUDA;
+}
+
 mtla_status mtla_get_device_status(void* stream) {
     int* p = nullptr;
     if (status_ptr(&p) != cudaSuccess) return MTLA_ERR_CUDA;

@@ -93,6 +93,10 @@ cudaError_t tc_prefill(const PrefillArgs& a, cudaStream_t st, uint64_t* launches
 cudaError_t gemm_bf16(const void* x, int ldx, const void* w, int ldw, void* y, int ldy, int M, int N, int K,
                       int* status, cudaStream_t st, uint64_t* launches);
 
+// Test hook (wait_probe.cu): one CTA whose bounded wait runs out after
+// limit_ns; `scratch` is 2 KB of device memory its TMA load reads.
+cudaError_t wait_probe(uint64_t limit_ns, void* scratch, int* status, cudaStream_t st, uint64_t* launches);
+
 // Beam-search reorder of the slot cache and open slots (cache_ops.cu).
 cudaError_t reorder_cache(const Shape& sh, size_t elem_bytes, const int32_t* src, const int32_t* n_tokens,
                           const void* cache_in, const float* open_in, void* cache_out, float* open_out,

@@ -100,6 +100,8 @@ def load() -> ctypes.CDLL:
     lib.mtla_decode_step_noalloc.restype = ctypes.c_int
     lib.mtla_reorder_cache.argtypes = [cp] + [_vp] * 6 + [_vp]
     lib.mtla_reorder_cache.restype = ctypes.c_int
+    lib.mtla_test_wait_timeout.argtypes = [ctypes.c_uint64, _vp, _vp]
+    lib.mtla_test_wait_timeout.restype = ctypes.c_int
     lib.mtla_get_device_status.argtypes = [_vp]
     lib.mtla_get_device_status.restype = ctypes.c_int
     lib.mtla_status_string.argtypes = [ctypes.c_int]
@@ -266,6 +268,11 @@ def reorder_cache(cfg, src, n_tokens, cache_in, open_in, cache_out, open_out, st
     if check and st != OK:
         raise MtlaError(st, "mtla_reorder_cache")
     return st
+
+
+def test_wait_timeout(limit_ns: int, scratch, stream=None) -> int:
+    """Forward to ``mtla_test_wait_timeout`` (the bounded-wait failure path)."""
+    return int(load().mtla_test_wait_timeout(int(limit_ns), _ptr(scratch), _stream(stream)))
 
 
 def last_error_detail() -> str:
