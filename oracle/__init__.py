@@ -44,6 +44,9 @@ FAULT_PE_SWAP = 13
 FAULT_CHUNK_NO_SEED = 14
 FAULT_CHUNK_LOCAL_POS = 15
 FAULT_CHANNEL_TRANSPOSE = 16
+FAULT_BWD_NO_DELTA = 17
+FAULT_BWD_PREFIX_SUM = 18
+FAULT_BWD_NO_SIGMOID = 19
 
 
 def build(force: bool = False) -> str:
@@ -112,6 +115,7 @@ def _load():
         _lib.orc_prefill_from.argtypes = [ctypes.POINTER(_Cfg)] + [ctypes.c_int32] * 3 + [_P] * 15
         _lib.orc_set_fault.argtypes = [ctypes.c_int]
         _lib.orc_linear.argtypes = [ctypes.c_int64] * 3 + [_P] * 3
+        _lib.orc_prefill_backward.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int32] + [_P] * 19
         _lib.orc_reorder_cache.argtypes = [ctypes.c_int32] * 5 + [ctypes.c_void_p] * 6
         _lib.orc_reorder_cache.restype = ctypes.c_int
     return _lib
@@ -267,6 +271,23 @@ def linear(x, w) -> np.ndarray:
     y = np.zeros(x.shape[:-1] + (w.shape[0],))
     _load().orc_linear(M, w.shape[0], K, _p(np.ascontiguousarray(x.reshape(M, K))), _p(w), _p(y))
     return y
+
+
+def prefill_backward(cfg: Cfg, c, kr, qc, qr, w_uk, w_uv, dout, G=None, g=None, gate_in=None) -> dict:
+    """Gradients of sum(dout * prefill(...)["out"]) with respect to every input
+    of the parallel forward from position 0 (scalar gate modes): dict(dc, dkr,
+    dqc, dqr, dw_uk, dw_uv, dG, dg, dgate_in) in float64 (``orc_prefill_backward``)."""
+    c, kr, qc, qr, w_uk, w_uv, dout = map(_d, (c, kr, qc, qr, w_uk, w_uv, dout))
+    G, g, gate_in = _d(G), _d(g), _d(gate_in)
+    B, T = c.shape[:2]
+    out = dict(dc=np.zeros_like(c), dkr=np.zeros_like(kr), dqc=np.zeros_like(qc), dqr=np.zeros_like(qr),
+               dw_uk=np.zeros_like(w_uk), dw_uv=np.zeros_like(w_uv),
+               dG=np.zeros((cfg.s, cfg.d_c)), dg=np.zeros(cfg.s), dgate_in=np.zeros((B, T)))
+    _load().orc_prefill_backward(ctypes.byref(cfg.c()), T, _p(c), _p(kr), _p(qc), _p(qr), _p(w_uk), _p(w_uv),
+                                 _p(G), _p(g), _p(gate_in), _p(dout),
+                                 *[_p(out[k]) for k in ("dc", "dkr", "dqc", "dqr", "dw_uk", "dw_uv", "dG", "dg",
+                                                        "dgate_in")])
+    return out
 
 
 def layer_forward(cfg: Cfg, t0: int, cache_in, acc_in, h, W: dict, G=None, g=None, gate_in=None):

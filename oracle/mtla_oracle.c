@@ -92,6 +92,9 @@ enum {
     ORC_FAULT_CHUNK_NO_SEED = 14,    /* chunked prefill: open block restarts  */
     ORC_FAULT_CHUNK_LOCAL_POS = 15,  /* chunked prefill: positions from 0     */
     ORC_FAULT_CHANNEL_TRANSPOSE = 16, /* per-channel gate read as G [s,D,d_c] */
+    ORC_FAULT_BWD_NO_DELTA = 17,     /* backward: softmax gradient without -delta */
+    ORC_FAULT_BWD_PREFIX_SUM = 18,   /* backward: scan reversed as prefix sums   */
+    ORC_FAULT_BWD_NO_SIGMOID = 19,   /* backward: gate without sigma'            */
 };
 static int orc_fault = ORC_FAULT_NONE;
 void orc_set_fault(int f) { orc_fault = f; }
@@ -586,6 +589,150 @@ void orc_prefill_explicit(const orc_cfg* cfg, int32_t T, const double* c, const 
     }
     free(w);
     free(P);
+}
+
+/* Gradients of the parallel forward from position 0 (training), for the
+ * scalar gate modes. With o_{i,h} = W_UV[h] obar_{i,h}, obar = sum_j a_ij key_j[0:d_c],
+ * a = softmax_j(e), e_ij = scale qt_{i,h} . key_j over the allowed keys of i
+ * (finished slots F_j = P_{js+s-1}, j < floor(i/s), and the own partial P_i),
+ * qt = [W_UK[h]^T qC ; R_i qR] and P_t = sum_{u in block(t), u <= t} w_u x_u,
+ * x_u = [c_u ; R_u k_u], the chain rule taken step by step from dout:
+ *   dW_UV[h] += dout obar^T;  dobar = W_UV[h]^T dout;  delta = dobar . obar
+ *   de_ij = a_ij (dobar . key_j[0:d_c] - delta)
+ *   dqt = scale sum_j de_ij key_j;  dkey_j += scale de_ij qt + a_ij [dobar ; 0]
+ *   dqC = W_UK[h] dqt[0:d_c];  dW_UK[h] += qC dqt[0:d_c]^T;  dqR = R_i^T dqt[d_c:]
+ *   dP_t = (key gradient of P_t as an own partial) + (as F_j when t = js+s-1)
+ *   S_u = sum_{t >= u, t in block(u)} dP_t;  dx_u = w_u S_u;  dw_u = x_u . S_u
+ *   dc_u = dx_u[0:d_c];  dk_u = R_u^T dx_u[d_c:]
+ *   COMPUTED: dz = dw w (1 - w); dG[r] += dz (c*PE); dg[r] += dz; dc += dz G[r]*PE
+ *   SUPPLIED: dgate_in = dw.
+ * Outputs (zeroed here): dc [B,T,d_c] dkr [B,T,d_r] dqc [B,T,H,d_h] dqr [B,T,H,d_r]
+ * dw_uk, dw_uv [H,d_h,d_c] dG [s,d_c] dg [s] dgate_in [B,T] (NULL where unused). */
+void orc_prefill_backward(const orc_cfg* cfg, int32_t T, const double* c, const double* kr, const double* qc,
+                          const double* qr, const double* w_uk, const double* w_uv, const double* G,
+                          const double* g, const double* gate_in, const double* dout, double* dc, double* dkr,
+                          double* dqc, double* dqr, double* dw_uk, double* dw_uv, double* dG, double* dg,
+                          double* dgate_in) {
+    const int32_t B = cfg->B, H = cfg->H, d_h = cfg->d_h, d_c = cfg->d_c, d_r = cfg->d_r, s = cfg->s;
+    const int32_t D = d_c + d_r;
+    const double scale = orc_scale(cfg);
+    double* w = (double*)malloc(sizeof(double) * (size_t)B * T);
+    double* P = (double*)malloc(sizeof(double) * (size_t)B * T * D);
+    double* dP = (double*)calloc((size_t)B * T * D, sizeof(double));
+    orc_partials(cfg, T, c, kr, G, g, gate_in, w, P);
+    memset(dc, 0, sizeof(double) * (size_t)B * T * d_c);
+    memset(dkr, 0, sizeof(double) * (size_t)B * T * d_r);
+    memset(dqc, 0, sizeof(double) * (size_t)B * T * H * d_h);
+    memset(dqr, 0, sizeof(double) * (size_t)B * T * H * d_r);
+    memset(dw_uk, 0, sizeof(double) * (size_t)H * d_h * d_c);
+    memset(dw_uv, 0, sizeof(double) * (size_t)H * d_h * d_c);
+    if (dG) memset(dG, 0, sizeof(double) * (size_t)s * d_c);
+    if (dg) memset(dg, 0, sizeof(double) * (size_t)s);
+    if (dgate_in) memset(dgate_in, 0, sizeof(double) * (size_t)B * T);
+    double* qt = (double*)malloc(sizeof(double) * D);
+    double* dqt = (double*)malloc(sizeof(double) * D);
+    double* obar = (double*)malloc(sizeof(double) * d_c);
+    double* dob = (double*)malloc(sizeof(double) * d_c);
+    double* e = (double*)malloc(sizeof(double) * (size_t)(T / s + 2));
+    int64_t* kidx = (int64_t*)malloc(sizeof(int64_t) * (size_t)(T / s + 2));   /* key -> row of P */
+    /* attention, one (b, i, h) at a time (plain loops, no reordering) */
+    for (int32_t b = 0; b < B; ++b)
+        for (int32_t i = 0; i < T; ++i)
+            for (int32_t h = 0; h < H; ++h) {
+                const int64_t bih = ((int64_t)b * T + i) * H + h;
+                orc_absorb_query(cfg, i, h, &qc[bih * d_h], &qr[bih * d_r], w_uk, qt);
+                int64_t n = 0;
+                for (int32_t j = 0; j < i / s; ++j) kidx[n++] = (int64_t)b * T + j * s + s - 1;
+                if (orc_fault != ORC_FAULT_DROP_OWN_PARTIAL) kidx[n++] = (int64_t)b * T + i;
+                double m = -INFINITY;
+                for (int64_t k = 0; k < n; ++k) {
+                    const double* key = &P[kidx[k] * D];
+                    double acc = 0.0;
+                    for (int32_t q = 0; q < D; ++q) acc += qt[q] * key[q];
+                    e[k] = scale * acc;
+                    if (e[k] > m) m = e[k];
+                }
+                double l = 0.0;
+                for (int64_t k = 0; k < n; ++k) {
+                    e[k] = exp(e[k] - m);
+                    l += e[k];
+                }
+                for (int64_t k = 0; k < n; ++k) e[k] /= l;               /* a_ij */
+                for (int32_t q = 0; q < d_c; ++q) obar[q] = 0.0;
+                for (int64_t k = 0; k < n; ++k)
+                    for (int32_t q = 0; q < d_c; ++q) obar[q] += e[k] * P[kidx[k] * D + q];
+                const double* W_uv = &w_uv[(int64_t)h * d_h * d_c];
+                const double* dO = &dout[bih * d_h];
+                for (int32_t q = 0; q < d_c; ++q) {
+                    double acc = 0.0;
+                    for (int32_t r = 0; r < d_h; ++r) acc += W_uv[(int64_t)r * d_c + q] * dO[r];
+                    dob[q] = acc;
+                }
+                for (int32_t r = 0; r < d_h; ++r)
+                    for (int32_t q = 0; q < d_c; ++q) dw_uv[((int64_t)h * d_h + r) * d_c + q] += dO[r] * obar[q];
+                double delta = 0.0;
+                for (int32_t q = 0; q < d_c; ++q) delta += dob[q] * obar[q];
+                for (int32_t q = 0; q < D; ++q) dqt[q] = 0.0;
+                for (int64_t k = 0; k < n; ++k) {
+                    double* key = &P[kidx[k] * D];
+                    double* dkey = &dP[kidx[k] * D];
+                    double da = 0.0;
+                    for (int32_t q = 0; q < d_c; ++q) da += dob[q] * key[q];
+                    const double de = e[k] * (da - (orc_fault == ORC_FAULT_BWD_NO_DELTA ? 0.0 : delta));
+                    for (int32_t q = 0; q < D; ++q) {
+                        dqt[q] += scale * de * key[q];
+                        dkey[q] += scale * de * qt[q];
+                    }
+                    for (int32_t q = 0; q < d_c; ++q) dkey[q] += e[k] * dob[q];
+                }
+                /* back through the query absorption and the query RoPE */
+                const double* W_uk = &w_uk[(int64_t)h * d_h * d_c];
+                for (int32_t r = 0; r < d_h; ++r) {
+                    double acc = 0.0;
+                    for (int32_t q = 0; q < d_c; ++q) {
+                        acc += W_uk[(int64_t)r * d_c + q] * dqt[q];
+                        dw_uk[((int64_t)h * d_h + r) * d_c + q] += qc[bih * d_h + r] * dqt[q];
+                    }
+                    dqc[bih * d_h + r] = acc;
+                }
+                orc_rope(-(int64_t)i, d_r, cfg->rope_base, &dqt[d_c], &dqr[bih * d_r]);   /* R_i^T = R_{-i} */
+            }
+    /* back through the block-prefix scan and the merging gate */
+    double* x = (double*)malloc(sizeof(double) * D);
+    double* S = (double*)malloc(sizeof(double) * D);
+    double* dx = (double*)malloc(sizeof(double) * D);
+    double* pe = (double*)malloc(sizeof(double) * d_c);
+    for (int32_t b = 0; b < B; ++b)
+        for (int32_t u = 0; u < T; ++u) {
+            const int64_t bu = (int64_t)b * T + u;
+            const int32_t blk_end = s * (u / s) + s - 1 < T - 1 ? s * (u / s) + s - 1 : T - 1;
+            for (int32_t q = 0; q < D; ++q) S[q] = 0.0;
+            const int32_t blk0 = s * (u / s);
+            for (int32_t t = (orc_fault == ORC_FAULT_BWD_PREFIX_SUM ? blk0 : u);
+                 t <= (orc_fault == ORC_FAULT_BWD_PREFIX_SUM ? u : blk_end); ++t)
+                for (int32_t q = 0; q < D; ++q) S[q] += dP[((int64_t)b * T + t) * D + q];
+            orc_token_vector(cfg, u, &c[bu * d_c], &kr[bu * d_r], x);
+            double dw = 0.0;
+            for (int32_t q = 0; q < D; ++q) {
+                dx[q] = w[bu] * S[q];
+                dw += x[q] * S[q];
+            }
+            for (int32_t q = 0; q < d_c; ++q) dc[bu * d_c + q] += dx[q];
+            orc_rope(-(int64_t)u, d_r, cfg->rope_base, &dx[d_c], &dkr[bu * d_r]);
+            if (cfg->gate_mode == ORC_GATE_SUPPLIED && dgate_in) dgate_in[bu] = dw;
+            if (cfg->gate_mode == ORC_GATE_COMPUTED) {
+                const int32_t r = u % s;
+                const double dz = orc_fault == ORC_FAULT_BWD_NO_SIGMOID ? dw : dw * w[bu] * (1.0 - w[bu]);
+                orc_pe(u, d_c, cfg->pe_base, pe);
+                for (int32_t q = 0; q < d_c; ++q) {
+                    dG[(int64_t)r * d_c + q] += dz * c[bu * d_c + q] * pe[q];
+                    dc[bu * d_c + q] += dz * G[(int64_t)r * d_c + q] * pe[q];
+                }
+                dg[r] += dz;
+            }
+        }
+    free(pe); free(dx); free(S); free(x); free(kidx); free(e); free(dob); free(obar); free(dqt); free(qt);
+    free(dP); free(P); free(w);
 }
 
 /* y[M, N] = x[M, K] . w[N, K]^T, the definition as three loops (float64). */

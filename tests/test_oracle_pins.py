@@ -21,7 +21,8 @@ mathematics fix, none of which retypes the oracle's own formulas.
   supplied); G = 0 gives a closed form; one value worked by hand; decoding
   equals the parallel form;
 - the layer around the path: block-selecting projections make it the path
-  itself; folding W_UK into W_Q and W_UV into W_O gives the same output.
+  itself; folding W_UK into W_Q and W_UV into W_O gives the same output;
+- the training backward: every gradient against central finite differences.
 Finally, each planted mistake in the oracle must trip at least one pin.
 """
 import math
@@ -544,6 +545,41 @@ def pin_layer_absorption_fold():
     return np.max(np.abs(got["y"] - ref["y"])) < 1e-12
 
 
+def pin_backward_finite_differences():
+    """Every gradient of the backward against central finite differences of
+    L = sum(dout * out) (eps = 1e-6, float64), on sampled entries of every input
+    tensor, for the computed, supplied and unit gates at s = 1, 2, 3."""
+    rng = np.random.default_rng(150)
+    for mode in (oracle.GATE_COMPUTED, oracle.GATE_SUPPLIED, oracle.GATE_UNIT):
+        for s in (1, 2, 3):
+            cfg, p = _rand_problem(2, 2, 4, 8, 4, s, 9, seed=160 + 10 * mode + s, gate_mode=mode)
+            args = dict(c=p["c"], kr=p["kr"], qc=p["qc"], qr=p["qr"], w_uk=p["w_uk"], w_uv=p["w_uv"],
+                        G=p["G"] if mode == oracle.GATE_COMPUTED else None,
+                        g=p["g"] if mode == oracle.GATE_COMPUTED else None,
+                        gate_in=p["gate_in"] if mode == oracle.GATE_SUPPLIED else None)
+            dout = rng.standard_normal((2, 9, 2, 4))
+
+            def loss(a):
+                r = oracle.prefill(cfg, a["c"], a["kr"], a["qc"], a["qr"], a["w_uk"], a["w_uv"], a["G"], a["g"],
+                                   a["gate_in"])
+                return float(np.sum(dout * r["out"]))
+            grads = oracle.prefill_backward(cfg, dout=dout, **args)
+            names = {"c": "dc", "kr": "dkr", "qc": "dqc", "qr": "dqr", "w_uk": "dw_uk", "w_uv": "dw_uv",
+                     "G": "dG", "g": "dg", "gate_in": "dgate_in"}
+            for k, gk in names.items():
+                if args[k] is None:
+                    continue
+                for _ in range(5):
+                    idx = tuple(int(rng.integers(0, n)) for n in args[k].shape)
+                    ap, am = {**args, k: args[k].copy()}, {**args, k: args[k].copy()}
+                    ap[k][idx] += 1e-6
+                    am[k][idx] -= 1e-6
+                    fd = (loss(ap) - loss(am)) / 2e-6
+                    if abs(fd - grads[gk][idx]) > 1e-6 * max(1.0, abs(fd)):
+                        return False
+    return True
+
+
 PINS = {
     "cache_footprint": pin_cache_footprint,
     "s1_is_mla_sdpa": pin_s1_is_mla_sdpa,
@@ -566,6 +602,7 @@ PINS = {
     "channel_incremental_equals_parallel": pin_channel_incremental_equals_parallel,
     "layer_selection_is_the_path": pin_layer_selection_is_the_path,
     "layer_absorption_fold": pin_layer_absorption_fold,
+    "backward_finite_differences": pin_backward_finite_differences,
 }
 
 
@@ -598,6 +635,9 @@ FAULTS = {
     "chunk_no_seed": oracle.FAULT_CHUNK_NO_SEED,
     "chunk_local_pos": oracle.FAULT_CHUNK_LOCAL_POS,
     "channel_transpose": oracle.FAULT_CHANNEL_TRANSPOSE,
+    "bwd_no_delta": oracle.FAULT_BWD_NO_DELTA,
+    "bwd_prefix_sum": oracle.FAULT_BWD_PREFIX_SUM,
+    "bwd_no_sigmoid": oracle.FAULT_BWD_NO_SIGMOID,
 }
 
 
