@@ -477,6 +477,51 @@ def measure_prefill(n, flush, ws, rank):
             "clocks": clocks, "l2": L2Flush.desc + " call"}
 
 
+# fp32 FMA lanes of a B200 at its maximum SM clock: 148 SMs x 128 lanes x 2
+# flops x 1.965 GHz (the peak of the CUDA-core kernels)
+FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def measure_backward(n, flush, ws, rank):
+    """Training backward at the prefill workload's sizes (B=8, T=8192, H=8,
+    d_h=64, d_c=256, d_R=32, s=2, computed gates): every gradient of the path
+    through mtla_prefill_backward; the masked-attention part (row and column
+    passes) against the fp32 ALU peak."""
+    wl = inputs.PREFILL.with_(seed=inputs.PREFILL.seed + 1000 * rank)
+    T = wl.T
+    cfg = mtla.make_config(wl.B, wl.H, wl.d_h, wl.d_c, wl.d_r, wl.s, 1, dtype=wl.dtype, gate_mode=wl.gate_mode)
+    w = inputs.weights(wl)
+    tk = inputs.tokens(wl, T)
+    d = {k: tk[k].to("cuda", torch.bfloat16).contiguous() for k in ("c", "kr", "qc", "qr")}
+    dw = {k: w[k].to("cuda", torch.bfloat16 if k.startswith("w_") else torch.float32).contiguous() for k in w}
+    dout = inputs.grad_out(wl, T).to("cuda", torch.bfloat16)
+    B, H = wl.B, wl.H
+    g = dict(dc=(B, T, wl.d_c), dkr=(B, T, wl.d_r), dq_c=(B, T, H, wl.d_h), dq_r=(B, T, H, wl.d_r),
+             dw_uk=(H, wl.d_h, wl.d_c), dw_uv=(H, wl.d_h, wl.d_c), dgate_w=(wl.s, wl.d_c), dgate_b=(wl.s,))
+    grads = {k: torch.empty(v, device="cuda") for k, v in g.items()}
+    wsb = torch.empty(mtla.prefill_backward_workspace_size(cfg, T), dtype=torch.uint8, device="cuda")
+
+    def call():
+        mtla.prefill_backward(cfg, T, d["c"], d["kr"], d["qc"], d["qr"], dw["w_uk"], dw["w_uv"], dw["gate_w"],
+                              dw["gate_b"], None, dout, grads, wsb)
+    call_ms, kern_ms, clocks = _timed_calls(call, n, flush, ws)
+    pairs = sum(t // wl.s + 1 for t in range(T))
+    # per (row, key) pair: the score and dobar.key dot products, dq, dkey and its
+    # latent (value) part: 2 (3 D + 2 d_c) flops
+    flops = 2 * pairs * (3 * wl.D + 2 * wl.d_c) * B * H
+    kern = flops / (kern_ms / 1e3) / 1e12
+    return {"workload": f"training backward: B={B}/rank, T={T}, H={H}, d_h={wl.d_h}, d_c={wl.d_c}, "
+                        f"d_R={wl.d_r}, s={wl.s}, computed gates, bf16 inputs, fp32 gradients",
+            "TFLOPs": flops * ws / (call_ms / 1e3) / 1e12, "call_ms": call_ms,
+            "attention_flops_per_call": flops, "calls": n,
+            "roofline": {"kernel": "k_bwd_rows + k_bwd_columns (masked attention backward, CUDA cores)",
+                         "bound": "alu", "achieved": kern, "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s",
+                         "frac": kern / FP32_ALU_TFLOPS, "traffic": None,
+                         "peak_source": "148 SMs x 128 fp32 lanes x 2 flops x 1.965 GHz",
+                         "avg_launch_us": kern_ms * 1e3},
+            "clocks": clocks, "l2": L2Flush.desc + " call"}
+
+
 def measure_speech(n, flush, ws, rank):
     """Speech-model-scale decode B=16, H=8, s=2: a 1024-token prefix by the
     prefill, then 256 decode steps (513..640 slots), as two CUDA graphs."""
@@ -792,6 +837,9 @@ def run_kernel_workload(args):
     if name == "layer":
         print(json.dumps(measure_layer(args.steps, flush, 1, 0)), flush=True)
         return
+    if name == "backward":
+        print(json.dumps(measure_backward(args.steps, flush, 1, 0)), flush=True)
+        return
     hbm, _, peak_kind = _peaks()
     if name == "large_latent_step":              # one decode step of the contract workload
         wl = inputs.LARGE_LATENT
@@ -824,7 +872,7 @@ def main():
                     help="contract line only (no prefill / speech / stride-sweep sub-objects)")
     ap.add_argument("--workload", default="large_latent",
                     help="large_latent (the contract line), or a kernel-level line of "
-                         "large_latent_step, stride_sweep[:s], prefill, speech_decode, layer or beam_reorder")
+                         "large_latent_step, stride_sweep[:s], prefill, speech_decode, layer, backward or beam_reorder")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     ws, rank = _dist()
@@ -857,6 +905,8 @@ def run_contract(args, ws, rank):
         extras["stride_sweep"] = measure_stride(6000, flush, ws, rank)
         torch.cuda.empty_cache()
         extras["layer"] = measure_layer(400, flush, ws, rank)
+        torch.cuda.empty_cache()
+        extras["backward"] = measure_backward(4, flush, ws, rank)
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         n_seq = 8

@@ -210,6 +210,40 @@ mtla_status mtla_prefill_from(const mtla_config* cfg, int32_t t0, int32_t T,
                               void* out, void* cache, float* open_slot,
                               void* workspace, size_t workspace_bytes, void* stream);
 
+/* Scratch for mtla_prefill_backward over T tokens. Host only. */
+mtla_status mtla_prefill_backward_workspace_size(const mtla_config* cfg, int32_t T, size_t* bytes);
+
+/* Training backward of the parallel forward from position 0 ("Multi-head
+ * Temporal Latent Attention", Results: the models are trained from scratch,
+ * through the stride-aware mask of Key claims; the gate of Sec. 4.1, Eq. 13,
+ * and the block-prefix scan of Sec. 4.2 differentiated as written): given
+ * dout, the gradient of a loss L with respect to mtla_prefill's `out`, the
+ * gradients of L with respect to every input of that forward.
+ *   c, kr, q_c, q_r, w_uk, w_uv, gate_w, gate_b, gate_in: exactly as for
+ *       mtla_prefill (storage type cfg->dtype; the gates float32)
+ *   dout      [B, T, H, d_h]  storage type
+ * Outputs, all float32, contiguous, 16-byte aligned, written whole:
+ *   dc [B, T, d_c]   dkr [B, T, d_r]   dq_c [B, T, H, d_h]   dq_r [B, T, H, d_r]
+ *   dw_uk, dw_uv [H, d_h, d_c]
+ *   dgate_w [s, d_c], dgate_b [s]   (MTLA_GATE_COMPUTED; else may be NULL, untouched)
+ *   dgate_in [B, T]                 (MTLA_GATE_SUPPLIED; else may be NULL, untouched)
+ * The scalar gate modes only: a per-channel mode gives MTLA_ERR_UNSUPPORTED.
+ * cfg->max_slots is not used (any positive value). The forward is recomputed
+ * inside (the scan and the absorbed queries) from the inputs. Arithmetic is
+ * fp32 on the CUDA cores for both storage types. Returns OK once enqueued;
+ * INVALID_ARG for a missing or misaligned pointer or T <= 0, WORKSPACE when
+ * workspace_bytes is below mtla_prefill_backward_workspace_size. */
+mtla_status mtla_prefill_backward(const mtla_config* cfg, int32_t T,
+                                  const void* c, const void* kr,
+                                  const void* q_c, const void* q_r,
+                                  const void* w_uk, const void* w_uv,
+                                  const float* gate_w, const float* gate_b, const float* gate_in,
+                                  const void* dout,
+                                  float* dc, float* dkr, float* dq_c, float* dq_r,
+                                  float* dw_uk, float* dw_uv,
+                                  float* dgate_w, float* dgate_b, float* dgate_in,
+                                  void* workspace, size_t workspace_bytes, void* stream);
+
 /* Dense projection on the tensor cores: y[M, N] = x[M, K] . w[N, K]^T with
  * bf16 operands and result and fp32 accumulation. The layer around the path
  * ("Multi-head Temporal Latent Attention", Method: MLA's low-rank compression

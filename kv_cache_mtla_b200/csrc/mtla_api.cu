@@ -295,6 +295,68 @@ mtla_status mtla_prefill_from(const mtla_config* cfg, int32_t t0, int32_t T, con
                           open_slot, open_slot, workspace, workspace_bytes, stream);
 }
 
+static mtla_status backward_check(const mtla_config* cfg, int32_t T, Shape* sh) {
+    mtla_status st = check_config(cfg, sh);
+    if (st != MTLA_OK) return st;
+    if (T <= 0) return MTLA_ERR_INVALID_ARG;
+    if (cfg->gate_mode > MTLA_GATE_UNIT || cfg->batch > 65535 || (int64_t)cfg->batch * T > INT32_MAX)
+        return MTLA_ERR_UNSUPPORTED;
+    return MTLA_OK;
+}
+
+mtla_status mtla_prefill_backward_workspace_size(const mtla_config* cfg, int32_t T, size_t* bytes) {
+    Shape sh;
+    if (!bytes) return MTLA_ERR_INVALID_ARG;
+    mtla_status st = backward_check(cfg, T, &sh);
+    if (st != MTLA_OK) return st;
+    *bytes = prefill_backward_workspace(sh, T, cfg->dtype == MTLA_FP32 ? 4 : 2);
+    return MTLA_OK;
+}
+
+mtla_status mtla_prefill_backward(const mtla_config* cfg, int32_t T, const void* c, const void* kr,
+                                  const void* q_c, const void* q_r, const void* w_uk, const void* w_uv,
+                                  const float* gate_w, const float* gate_b, const float* gate_in,
+                                  const void* dout, float* dc, float* dkr, float* dq_c, float* dq_r,
+                                  float* dw_uk, float* dw_uv, float* dgate_w, float* dgate_b, float* dgate_in,
+                                  void* workspace, size_t workspace_bytes, void* stream) {
+    Shape sh;
+    mtla_status st = backward_check(cfg, T, &sh);
+    if (st != MTLA_OK) return st;
+    const void* req[] = {c, kr, q_c, q_r, w_uk, w_uv, dout, dc, dkr, dq_c, dq_r, dw_uk, dw_uv, workspace};
+    for (const void* p : req)
+        if (!p || !aligned16(p)) return MTLA_ERR_INVALID_ARG;
+    st = check_gate_ptrs(cfg, gate_w, gate_b, gate_in);
+    if (st != MTLA_OK) return st;
+    if (cfg->gate_mode == MTLA_GATE_COMPUTED &&
+        (!dgate_w || !dgate_b || !aligned16(dgate_w) || !aligned16(dgate_b)))
+        return MTLA_ERR_INVALID_ARG;
+    if (cfg->gate_mode == MTLA_GATE_SUPPLIED && (!dgate_in || !aligned16(dgate_in))) return MTLA_ERR_INVALID_ARG;
+    if (workspace_bytes < prefill_backward_workspace(sh, T, cfg->dtype == MTLA_FP32 ? 4 : 2))
+        return MTLA_ERR_WORKSPACE;
+    PrefillArgs a = {};
+    a.sh = sh;
+    a.T = T;
+    a.c = c;
+    a.kr = kr;
+    a.q_c = q_c;
+    a.q_r = q_r;
+    a.w_uk = w_uk;
+    a.w_uv = w_uv;
+    a.gate_w = gate_w;
+    a.gate_b = gate_b;
+    a.gate_in = gate_in;
+    a.workspace = workspace;
+    a.workspace_bytes = workspace_bytes;
+    BackwardGrads g = {dout, dc, dkr, dq_c, dq_r, dw_uk, dw_uv, dgate_w, dgate_b, dgate_in};
+    g_error_detail[0] = 0;
+    if (note_error("device status word", status_ptr(&a.status)) != cudaSuccess) return MTLA_ERR_CUDA;
+    uint64_t n = 0;
+    cudaError_t e = prefill_backward(a, g, cfg->dtype == MTLA_FP32, (cudaStream_t)stream, &n);
+    g_launches += n;
+    if (e != cudaSuccess && !g_error_detail[0]) note_error("backward launch", e);
+    return e == cudaSuccess ? MTLA_OK : MTLA_ERR_CUDA;
+}
+
 mtla_status mtla_linear(const void* x, const void* w, void* y, int32_t M, int32_t N, int32_t K, void* stream) {
     if (M <= 0 || N <= 0 || K <= 0 || K % 8 != 0) return MTLA_ERR_INVALID_ARG;
     if (!x || !w || !y || !aligned16(x) || !aligned16(w) || !aligned16(y)) return MTLA_ERR_INVALID_ARG;

@@ -93,6 +93,25 @@ cudaError_t tc_prefill(const PrefillArgs& a, cudaStream_t st, uint64_t* launches
 cudaError_t gemm_bf16(const void* x, int ldx, const void* w, int ldw, void* y, int ldy, int M, int N, int K,
                       int* status, cudaStream_t st, uint64_t* launches);
 
+// Training backward of the parallel forward from position 0 (backward.cu),
+// scalar gate modes, fp32 gradients. `a` carries the forward's inputs (t0 0,
+// no cache or open slot: the scan writes a scratch copy in the workspace).
+struct BackwardGrads {
+    const void* dout;      // [B,T,H,d_h] storage type
+    float* dc;             // [B,T,d_c]
+    float* dkr;            // [B,T,d_R]
+    float* dq_c;           // [B,T,H,d_h]
+    float* dq_r;           // [B,T,H,d_R]
+    float* dw_uk;          // [H,d_h,d_c]
+    float* dw_uv;          // [H,d_h,d_c]
+    float* dgate_w;        // [s,d_c] (computed gate)
+    float* dgate_b;        // [s]
+    float* dgate_in;       // [B,T] (supplied gate)
+};
+size_t prefill_backward_workspace(const Shape& sh, int T, size_t elem_bytes);
+cudaError_t prefill_backward(const PrefillArgs& a, const BackwardGrads& g, bool fp32, cudaStream_t st,
+                             uint64_t* launches);
+
 // Test hook (wait_probe.cu): one CTA whose bounded wait runs out after
 // limit_ns; `scratch` is 2 KB of device memory its TMA load reads.
 cudaError_t wait_probe(uint64_t limit_ns, void* scratch, int* status, cudaStream_t st, uint64_t* launches);

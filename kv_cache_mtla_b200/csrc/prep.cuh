@@ -311,7 +311,8 @@ template <> __device__ __forceinline__ void store8<bf16>(bf16* p, const float* v
 // function unit (absolute error about 2^-21 there, far below the bf16 rounding
 // of the slots); the fp32 partial slots of the CUDA-core path keep sincosf.
 template <typename T, typename PT>
-__global__ void __launch_bounds__(256) k_prefill_scan(PrefillArgs a, PT* P, float2* rope_tab = nullptr) {
+__global__ void __launch_bounds__(256) k_prefill_scan(PrefillArgs a, PT* P, float2* rope_tab = nullptr,
+                                                      float* w_out = nullptr) {
     constexpr bool kFastSinCos = std::is_same<PT, bf16>::value;
     auto sincos_at = [](int64_t t, double inv_freq, float* sn, float* cs) {
         if constexpr (kFastSinCos) {
@@ -366,6 +367,7 @@ __global__ void __launch_bounds__(256) k_prefill_scan(PrefillArgs a, PT* P, floa
             }
             wv[uo] = sigmoidf_(warp_sum(z) + a.gate_b[r]);
         }
+        if (w_out && lane == 0) w_out[(size_t)b * Tn + lu0 + uo] = wv[uo];   // the weights, for the backward
     }
     T* slot = (T*)a.cache_out + ((size_t)b * sh.max_slots + j) * sh.D;
     float* open = (ua + nu == t0 + Tn && a.open_slot_out) ? a.open_slot_out + (size_t)b * sh.D : nullptr;

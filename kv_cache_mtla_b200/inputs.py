@@ -113,6 +113,13 @@ def tokens(wl: Workload, T: int, stream: int = 0) -> dict:
     return dict(c=c, kr=kr, qc=qc, qr=qr, gate_in=gate_in)
 
 
+def grad_out(wl: Workload, T: int, stream: int = 0) -> torch.Tensor:
+    """The gradient flowing into the path's output for the training backward:
+    dout [B,T,H,d_h] ~ N(0,1) in the storage dtype."""
+    g = _gen(wl.seed * 1000 + 433 + 7919 * stream)
+    return _round(torch.randn(wl.B, T, wl.H, wl.d_h, generator=g), wl)
+
+
 def layer_weights(wl: Workload, d_model: int) -> dict:
     """The layer's projections (storage dtype values): w_dkv [d_c, dm],
     w_kr [d_R, dm], w_q [H d_h, dm], w_qr [H d_R, dm] ~ N(0,1)/sqrt(dm),

@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libmtla.so")
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CAPACITY, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE = range(7)
 BF16, FP32 = 0, 1
 GATE_COMPUTED, GATE_SUPPLIED, GATE_UNIT = 0, 1, 2
+GATE_CHANNEL_COMPUTED, GATE_CHANNEL_SUPPLIED = 3, 4
 
 
 class MtlaError(RuntimeError):
@@ -86,6 +87,10 @@ def load() -> ctypes.CDLL:
     lib.mtla_prefill.restype = ctypes.c_int
     lib.mtla_prefill_from.argtypes = [cp, ctypes.c_int32, ctypes.c_int32] + [_vp] * 12 + [_vp, ctypes.c_size_t, _vp]
     lib.mtla_prefill_from.restype = ctypes.c_int
+    lib.mtla_prefill_backward_workspace_size.argtypes = [cp, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)]
+    lib.mtla_prefill_backward_workspace_size.restype = ctypes.c_int
+    lib.mtla_prefill_backward.argtypes = [cp, ctypes.c_int32] + [_vp] * 19 + [_vp, ctypes.c_size_t, _vp]
+    lib.mtla_prefill_backward.restype = ctypes.c_int
     lib.mtla_linear.argtypes = [_vp, _vp, _vp, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _vp]
     lib.mtla_linear.restype = ctypes.c_int
     lp = ctypes.POINTER(LayerWeights)
@@ -210,6 +215,32 @@ def prefill_from(cfg, t0, T, c, kr, q_c, q_r, w_uk, w_uv, gate_w, gate_b, gate_i
         _ptr(open_slot), _ptr(workspace), ws, _stream(stream))
     if check and st != OK:
         raise MtlaError(st, "mtla_prefill_from")
+    return st
+
+
+BACKWARD_GRADS = ("dc", "dkr", "dq_c", "dq_r", "dw_uk", "dw_uv", "dgate_w", "dgate_b", "dgate_in")
+
+
+def prefill_backward_workspace_size(cfg: Config, T: int) -> int:
+    n = ctypes.c_size_t(0)
+    st = load().mtla_prefill_backward_workspace_size(ctypes.byref(cfg), int(T), ctypes.byref(n))
+    if st != OK:
+        raise MtlaError(st, "mtla_prefill_backward_workspace_size")
+    return int(n.value)
+
+
+def prefill_backward(cfg, T, c, kr, q_c, q_r, w_uk, w_uv, gate_w, gate_b, gate_in, dout, grads: dict,
+                     workspace, stream=None, check=True) -> int:
+    """Forward to ``mtla_prefill_backward``; ``grads`` maps the names in
+    BACKWARD_GRADS to float32 device tensors (None where the gate mode has no
+    such gradient). Returns the status (raises if check)."""
+    ws = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = load().mtla_prefill_backward(
+        ctypes.byref(cfg), int(T), _ptr(c), _ptr(kr), _ptr(q_c), _ptr(q_r), _ptr(w_uk), _ptr(w_uv),
+        _ptr(gate_w), _ptr(gate_b), _ptr(gate_in), _ptr(dout), *[_ptr(grads.get(k)) for k in BACKWARD_GRADS],
+        _ptr(workspace), ws, _stream(stream))
+    if check and st != OK:
+        raise MtlaError(st, "mtla_prefill_backward")
     return st
 
 

@@ -200,6 +200,36 @@ def test_prefill_from_rejects_bad_arguments_on_the_host(lib):
     assert st(30, 4, fake) == mtla.ERR_CAPACITY      # ceil(34 / 2) = 17 slots > 16
 
 
+def test_backward_rejects_bad_arguments_on_the_host(lib):
+    """mtla_prefill_backward: per-channel gates are refused, T <= 0, a missing
+    gradient buffer for the gate mode and a short workspace too, all before
+    the device is touched (the pointers below are never dereferenced)."""
+    fake = 0x10000
+    cfg = _cfg()
+    n = mtla.prefill_backward_workspace_size(cfg, 100)
+    assert n >= mtla.prefill_backward_workspace_size(cfg, 99) > 0
+    cfg.gate_mode = mtla.GATE_CHANNEL_COMPUTED
+    with pytest.raises(mtla.MtlaError) as e:
+        mtla.prefill_backward_workspace_size(cfg, 100)
+    assert e.value.status == mtla.ERR_UNSUPPORTED
+
+    def call(cfg, T, gate, grads, ws_bytes):
+        return lib.mtla_prefill_backward(ctypes.byref(cfg), T, *([fake] * 6), *gate, fake, *grads,
+                                         fake, ws_bytes, None)
+
+    plain = [fake] * 6
+    cfg.gate_mode = mtla.GATE_COMPUTED
+    assert call(cfg, 100, [fake, fake, None], plain + [None, None, None], n) == mtla.ERR_INVALID_ARG
+    assert call(cfg, 0, [fake, fake, None], plain + [fake, fake, None], n) == mtla.ERR_INVALID_ARG
+    assert call(cfg, 100, [fake, fake, None], plain + [fake, fake, None], n - 1) == mtla.ERR_WORKSPACE
+    assert call(cfg, 100, [fake, fake, None], plain[:5] + [None] + [fake, fake, None], n) == mtla.ERR_INVALID_ARG
+    cfg.gate_mode = mtla.GATE_SUPPLIED
+    assert call(cfg, 100, [None, None, fake], plain + [None, None, None], n) == mtla.ERR_INVALID_ARG
+    assert call(cfg, 100, [None, None, fake], plain + [None, None, fake + 4], n) == mtla.ERR_INVALID_ARG
+    cfg.gate_mode = mtla.GATE_CHANNEL_SUPPLIED
+    assert call(cfg, 100, [None, None, fake], plain + [None, None, fake], n) == mtla.ERR_UNSUPPORTED
+
+
 def test_layer_refuses_fp32_and_bad_widths_on_the_host(lib):
     """The layer is bf16 only; d_model must be a positive multiple of 8."""
     cfg = _cfg()
