@@ -477,16 +477,12 @@ def measure_prefill(n, flush, ws, rank):
             "clocks": clocks, "l2": L2Flush.desc + " call"}
 
 
-# fp32 FMA lanes of a B200 at its maximum SM clock: 148 SMs x 128 lanes x 2
-# flops x 1.965 GHz (the peak of the CUDA-core kernels)
-FP32_ALU_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
-
-
 def measure_backward(n, flush, ws, rank):
     """Training backward at the prefill workload's sizes (B=8, T=8192, H=8,
     d_h=64, d_c=256, d_R=32, s=2, computed gates): every gradient of the path
-    through mtla_prefill_backward; the masked-attention part (row and column
-    passes) against the fp32 ALU peak."""
+    through mtla_prefill_backward; its masked-attention part (the two
+    tensor-core kernels) against the bf16 peak."""
+    _, tflops_peak, peak_kind = _peaks()
     wl = inputs.PREFILL.with_(seed=inputs.PREFILL.seed + 1000 * rank)
     T = wl.T
     cfg = mtla.make_config(wl.B, wl.H, wl.d_h, wl.d_c, wl.d_r, wl.s, 1, dtype=wl.dtype, gate_mode=wl.gate_mode)
@@ -514,10 +510,10 @@ def measure_backward(n, flush, ws, rank):
                         f"d_R={wl.d_r}, s={wl.s}, computed gates, bf16 inputs, fp32 gradients",
             "TFLOPs": flops * ws / (call_ms / 1e3) / 1e12, "call_ms": call_ms,
             "attention_flops_per_call": flops, "calls": n,
-            "roofline": {"kernel": "k_bwd_rows + k_bwd_columns (masked attention backward, CUDA cores)",
-                         "bound": "alu", "achieved": kern, "peak": FP32_ALU_TFLOPS, "unit": "TFLOP/s",
-                         "frac": kern / FP32_ALU_TFLOPS, "traffic": None,
-                         "peak_source": "148 SMs x 128 fp32 lanes x 2 flops x 1.965 GHz",
+            "roofline": {"kernel": "k_bwd_dq_tc + k_bwd_dk_tc (masked attention backward, tensor cores)",
+                         "bound": "tensor", "achieved": kern, "peak": tflops_peak, "unit": "TFLOP/s",
+                         "frac": kern / tflops_peak, "traffic": None,
+                         "peak_source": f"{peak_kind} bf16_tflops (burst)",
                          "avg_launch_us": kern_ms * 1e3},
             "clocks": clocks, "l2": L2Flush.desc + " call"}
 
@@ -906,7 +902,7 @@ def run_contract(args, ws, rank):
         torch.cuda.empty_cache()
         extras["layer"] = measure_layer(400, flush, ws, rank)
         torch.cuda.empty_cache()
-        extras["backward"] = measure_backward(4, flush, ws, rank)
+        extras["backward"] = measure_backward(40, flush, ws, rank)
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         n_seq = 8

@@ -59,10 +59,11 @@ struct BwdArgs {
     float* lrow;           // [B,T,H] row sum
     float* delta;          // [B,T,H]
     float* dob;            // [B,T,H,d_c] dobar
-    float* obar;           // [B,T,H,d_c]
+    void* obar;            // [B,T,H,d_c] fp32 (CUDA-core path) or bf16 (tensor-core path)
     float* dqt;            // [B,T,H,D]
     float* dP;             // [B,T,D] own-partial key gradients
-    float* dF;             // [B,n_slots,D] finished-slot key gradients
+    float* dF;             // [n_parts][B,n_slots,D] finished-slot key gradients (summed over parts)
+    int n_parts;
 };
 
 template <typename T> __device__ __forceinline__ float ldf(const void* p, size_t i) {
@@ -156,7 +157,7 @@ __global__ void __launch_bounds__(256) k_bwd_rows(BwdArgs a) {
             if (c < D) a.dqt[row * D + c] = dq[k];
             if (c < d_c) {
                 a.dob[row * d_c + c] = dv[k];
-                a.obar[row * d_c + c] = ob[k];
+                ((float*)a.obar)[row * d_c + c] = ob[k];
             }
         }
         if (lane == 0) {
@@ -253,7 +254,7 @@ __global__ void __launch_bounds__(256) k_bwd_query(BwdArgs a, float* dqc, float*
 // dW_UK[h][r][c] += sum_rows qC[r] dqt[c], dW_UV[h][r][c] += sum_rows dout[r] obar[c]
 // over token rows m0 .. m0 + kWChunk - 1: block (row chunk, h, r group), a
 // thread per channel c (two when d_c > 256).
-template <typename T>
+template <typename T, typename OT>
 __global__ void __launch_bounds__(256) k_bwd_weights(BwdArgs a, float* dw_uk, float* dw_uv) {
     const Shape sh = a.sh;
     const int h = blockIdx.y, r0 = blockIdx.z * kWRows, tid = threadIdx.x;
@@ -275,7 +276,7 @@ __global__ void __launch_bounds__(256) k_bwd_weights(BwdArgs a, float* dw_uk, fl
         for (int cc = 0; cc < 2; ++cc) {
             const int c = tid + 256 * cc;
             if (c < sh.d_c) {
-                const float x = a.dqt[row * sh.D + c], y = a.obar[row * sh.d_c + c];
+                const float x = a.dqt[row * sh.D + c], y = ldf<OT>(a.obar, row * sh.d_c + c);
 #pragma unroll
                 for (int r = 0; r < kWRows; ++r) {
                     gk[cc][r] = fmaf(qs[r], x, gk[cc][r]);
@@ -334,7 +335,12 @@ __global__ void __launch_bounds__(256) k_bwd_scan(BwdArgs a, const void* c_in, c
             const float* dPu = a.dP + bu * D;
             const bool end = finished && u == u0 + s - 1;
             __syncwarp();
-            for (int c = lane; c < D; c += 32) S[c] += dPu[c] + (end ? dF[c] : 0.f);
+            for (int c = lane; c < D; c += 32) {
+                float f = 0.f;
+                if (end)
+                    for (int q = 0; q < a.n_parts; ++q) f += dF[(size_t)q * sh.B * a.n_slots * D + c];
+                S[c] += dPu[c] + f;
+            }
             __syncwarp();
             const float wu = a.w[bu];
             float dw = 0.f;
@@ -374,6 +380,107 @@ __global__ void __launch_bounds__(256) k_bwd_scan(BwdArgs a, const void* c_in, c
         __syncthreads();
         for (int k = threadIdx.x; k < s * d_c; k += blockDim.x) atomicAdd(&dG[k], gG[k]);
         if (threadIdx.x < s) atomicAdd(&dg[threadIdx.x], gg[threadIdx.x]);
+    }
+}
+
+// Tensor-core path, per (16 positions, head, sequence): dobar = W_UV[h]^T dout
+// rounded to bf16 (the operand of the tensor-core kernels) and delta =
+// dobar . obar from the same rounded values, in the [B, H, T] layout.
+template <typename T>
+__global__ void __launch_bounds__(256) k_bwd_dob(BwdArgs a, bf16* dob, float* delta) {
+    const Shape sh = a.sh;
+    const int t0 = blockIdx.x * 16, h = blockIdx.y, b = blockIdx.z;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    __shared__ float dsm[16][256];
+    __shared__ float red[8][16];
+    for (int q = tid; q < 16 * sh.d_h; q += blockDim.x) {
+        const int pp = q / sh.d_h, r = q % sh.d_h, t = t0 + pp;
+        dsm[pp][r] = t < a.T ? ldf<T>(a.dout, (((size_t)b * a.T + t) * sh.H + h) * sh.d_h + r) : 0.f;
+    }
+    __syncthreads();
+    float dl[16];
+#pragma unroll
+    for (int pp = 0; pp < 16; ++pp) dl[pp] = 0.f;
+    for (int c = tid; c < sh.d_c; c += blockDim.x) {
+        float acc[16];
+#pragma unroll
+        for (int pp = 0; pp < 16; ++pp) acc[pp] = 0.f;
+        for (int r = 0; r < sh.d_h; ++r) {
+            const float wv = ldf<T>(a.w_uv, ((size_t)h * sh.d_h + r) * sh.d_c + c);
+#pragma unroll
+            for (int pp = 0; pp < 16; ++pp) acc[pp] = fmaf(dsm[pp][r], wv, acc[pp]);
+        }
+#pragma unroll
+        for (int pp = 0; pp < 16; ++pp) {
+            const int t = t0 + pp;
+            if (t < a.T) {
+                const size_t o = (((size_t)b * a.T + t) * sh.H + h) * sh.d_c + c;
+                const bf16 v = __float2bfloat16_rn(acc[pp]);
+                dob[o] = v;
+                dl[pp] = fmaf(__bfloat162float(v), ldf<bf16>(a.obar, o), dl[pp]);
+            }
+        }
+    }
+#pragma unroll
+    for (int pp = 0; pp < 16; ++pp) {
+        const float v = warp_sum(dl[pp]);
+        if (lane == 0) red[warp][pp] = v;
+    }
+    __syncthreads();
+    if (tid < 16 && t0 + tid < a.T) {
+        float v = 0.f;
+        for (int q = 0; q < (int)(blockDim.x >> 5); ++q) v += red[q][tid];
+        delta[((size_t)b * sh.H + h) * stats_pitch(a.T) + t0 + tid] = v;
+    }
+}
+
+// Tensor-core path: the own-partial term of every row (one key, P_i), added
+// to the finished-slot part of dqt; dP_i = the heads' own-partial key
+// gradients (summed in a fixed order). Block (i, b), a warp per head.
+__global__ void __launch_bounds__(256) k_bwd_own(BwdArgs a, const bf16* qt, const bf16* P, const bf16* dob,
+                                                 const float* lse, const float* delta) {
+    const Shape sh = a.sh;
+    const int i = blockIdx.x, b = blockIdx.y;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    const int D = sh.D, d_c = sh.d_c;
+    const float scale_log2 = sh.scale * 1.4426950408889634f;
+    __shared__ float dkey_own[8][kMaxD];
+    float* own = dkey_own[warp];
+    for (int q = lane; q < D; q += 32) own[q] = 0.f;
+    const bf16* Pi = P + ((size_t)b * a.T + i) * D;
+    float pv[kPer];
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) pv[k] = lane + 32 * k < D ? __bfloat162float(Pi[lane + 32 * k]) : 0.f;
+    for (int h = warp; h < sh.H; h += nw) {
+        const size_t row = ((size_t)b * a.T + i) * sh.H + h;
+        const size_t srow = ((size_t)b * sh.H + h) * stats_pitch(a.T) + i;
+        float qv[kPer], dv[kPer], e = 0.f, da = 0.f;
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) {
+            const int c = lane + 32 * k;
+            qv[k] = c < D ? __bfloat162float(qt[row * D + c]) : 0.f;
+            dv[k] = c < d_c ? __bfloat162float(dob[row * d_c + c]) : 0.f;
+            e = fmaf(qv[k], pv[k], e);
+            da = fmaf(dv[k], pv[k], da);
+        }
+        e = warp_sum(e);
+        da = warp_sum(da);
+        const float pr = exp2f(fmaf(e, scale_log2, -lse[srow]));
+        const float sde = sh.scale * pr * (da - delta[srow]);
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) {
+            const int c = lane + 32 * k;
+            if (c < D) {
+                a.dqt[row * D + c] += sde * pv[k];
+                own[c] += fmaf(sde, qv[k], pr * dv[k]);
+            }
+        }
+    }
+    __syncthreads();
+    for (int q = threadIdx.x; q < D; q += blockDim.x) {
+        float acc = 0.f;
+        for (int v = 0; v < nw; ++v) acc += dkey_own[v][q];
+        a.dP[((size_t)b * a.T + i) * D + q] = acc;
     }
 }
 
@@ -435,6 +542,7 @@ cudaError_t backward_impl(const PrefillArgs& pa_in, const BackwardGrads& g, cuda
     a.dqt = (float*)(ws + l.dqt);
     a.dP = (float*)(ws + l.dP);
     a.dF = (float*)(ws + l.dF);
+    a.n_parts = 1;
     const size_t wbytes = (size_t)sh.H * sh.d_h * sh.d_c * sizeof(float);
     cudaError_t e;
     if ((e = cudaMemsetAsync(g.dw_uk, 0, wbytes, st)) != cudaSuccess) return note_error("backward zero dW_UK", e);
@@ -456,7 +564,7 @@ cudaError_t backward_impl(const PrefillArgs& pa_in, const BackwardGrads& g, cuda
     profile_end(st);
     k_bwd_query<T><<<dim3(T_len, sh.B), threads, 0, st>>>(a, g.dq_c, g.dq_r);
     const int64_t M = (int64_t)sh.B * T_len;
-    k_bwd_weights<T><<<dim3((unsigned)((M + kWChunk - 1) / kWChunk), sh.H, sh.d_h / kWRows), 256, 0, st>>>(
+    k_bwd_weights<T, float><<<dim3((unsigned)((M + kWChunk - 1) / kWChunk), sh.H, sh.d_h / kWRows), 256, 0, st>>>(
         a, g.dw_uk, g.dw_uv);
     k_bwd_scan<T><<<dim3((n_slots + 7) / 8, sh.B), 256, 0, st>>>(a, pa.c, pa.kr, pa.gate_w, g.dc, g.dkr, g.dgate_w,
                                                                  g.dgate_b, g.dgate_in);
@@ -464,14 +572,135 @@ cudaError_t backward_impl(const PrefillArgs& pa_in, const BackwardGrads& g, cuda
     return note_error("backward launch", cudaGetLastError());
 }
 
+// ---------------------------------------------------------------- tensor-core path
+
+struct BwdTcWs {
+    size_t fwd, cache, out, lse, delta, obar, qt, w, dob, dqt, dF, dP, total;
+};
+
+Shape with_slots(const Shape& sh, int T) {
+    Shape s2 = sh;
+    s2.max_slots = (T + sh.s - 1) / sh.s;
+    return s2;
+}
+
+BwdTcWs bwd_tc_layout(const Shape& sh_in, int T) {
+    const Shape sh = with_slots(sh_in, T);
+    const size_t BT = (size_t)sh.B * T, rows = BT * sh.H;
+    BwdTcWs l;
+    size_t o = 0;
+    auto take = [&](size_t bytes) { size_t at = o; o += align256(bytes); return at; };
+    l.fwd = take(tc_prefill_workspace(sh, T));            // its first region: the partial slots P (bf16)
+    l.cache = take((size_t)sh.B * sh.max_slots * sh.D * 2);
+    l.out = take(rows * sh.d_h * 2);
+    l.lse = take((size_t)sh.B * sh.H * stats_pitch(T) * 4);
+    l.delta = take((size_t)sh.B * sh.H * stats_pitch(T) * 4);
+    l.obar = take(rows * sh.d_c * 2);
+    l.qt = take(rows * sh.D * 2);
+    l.w = take(BT * 4);
+    l.dob = take(rows * sh.d_c * 2);
+    l.dqt = take(rows * sh.D * 4);
+    l.dF = take((size_t)sh.H * sh.B * sh.max_slots * sh.D * 4);
+    l.dP = take(BT * sh.D * 4);
+    l.total = o;
+    return l;
+}
+
+bool use_tc(const Shape& sh, bool fp32) {
+    return !fp32 && tc_backward_supported(sh) && tc_prefill_supported(sh);
+}
+
+// bf16 at the tensor-core prefill's widths: the forward recomputed on the
+// tensor cores keeping its rows' statistics, dobar and delta, the finished-
+// slot parts on the tensor cores, the own-partial term, then the same query,
+// weight and scan/gate backward as the CUDA-core path (dF summed over heads).
+cudaError_t backward_tc(const PrefillArgs& pa_in, const BackwardGrads& g, cudaStream_t st, uint64_t* launches) {
+    const int T_len = pa_in.T;
+    PrefillArgs pa = pa_in;
+    pa.sh = with_slots(pa_in.sh, T_len);
+    const Shape sh = pa.sh;
+    const int n_slots = sh.max_slots;
+    char* ws = (char*)pa.workspace;
+    const BwdTcWs l = bwd_tc_layout(sh, T_len);
+    pa.workspace = ws + l.fwd;
+    pa.workspace_bytes = tc_prefill_workspace(sh, T_len);
+    pa.cache_out = ws + l.cache;
+    pa.out = ws + l.out;
+    pa.open_slot_in = nullptr;
+    pa.open_slot_out = nullptr;
+    pa.t0 = 0;
+    const size_t wbytes = (size_t)sh.H * sh.d_h * sh.d_c * sizeof(float);
+    cudaError_t e;
+    if ((e = cudaMemsetAsync(g.dw_uk, 0, wbytes, st)) != cudaSuccess) return note_error("backward zero dW_UK", e);
+    if ((e = cudaMemsetAsync(g.dw_uv, 0, wbytes, st)) != cudaSuccess) return note_error("backward zero dW_UV", e);
+    if (sh.gate_mode == 0) {
+        if ((e = cudaMemsetAsync(g.dgate_w, 0, (size_t)sh.s * sh.d_c * sizeof(float), st)) != cudaSuccess)
+            return note_error("backward zero dG", e);
+        if ((e = cudaMemsetAsync(g.dgate_b, 0, (size_t)sh.s * sizeof(float), st)) != cudaSuccess)
+            return note_error("backward zero dg", e);
+    }
+    PrefillSave sv;
+    sv.w = (float*)(ws + l.w);
+    sv.lse = (float*)(ws + l.lse);
+    sv.obar = ws + l.obar;
+    sv.qt = ws + l.qt;
+    if ((e = tc_prefill_save(pa, sv, st, launches)) != cudaSuccess) return e;
+    BwdArgs a;
+    a.sh = sh;
+    a.T = T_len;
+    a.n_slots = n_slots;
+    a.qc = pa.q_c;
+    a.w_uk = pa.w_uk;
+    a.w_uv = pa.w_uv;
+    a.dout = g.dout;
+    a.P = nullptr;
+    a.qt = nullptr;
+    a.w = (const float*)(ws + l.w);
+    a.mrow = a.lrow = a.delta = nullptr;
+    a.dob = nullptr;
+    a.obar = ws + l.obar;
+    a.dqt = (float*)(ws + l.dqt);
+    a.dP = (float*)(ws + l.dP);
+    a.dF = (float*)(ws + l.dF);
+    a.n_parts = sh.H;
+    const int threads = 32 * (sh.H < 8 ? sh.H : 8);
+    k_bwd_dob<bf16><<<dim3((T_len + 15) / 16, sh.H, sh.B), 256, 0, st>>>(a, (bf16*)(ws + l.dob),
+                                                                          (float*)(ws + l.delta));
+    if ((e = cudaGetLastError()) != cudaSuccess) return note_error("k_bwd_dob launch", e);
+    BwdTCInputs in;
+    in.qt = ws + l.qt;
+    in.dob = ws + l.dob;
+    in.slots = ws + l.cache;
+    in.lse = (const float*)(ws + l.lse);
+    in.delta = (const float*)(ws + l.delta);
+    in.dqt = a.dqt;
+    in.dF = a.dF;
+    in.status = pa.status;
+    profile_begin(st);
+    e = tc_backward_attention(sh, T_len, in, st, launches);
+    profile_end(st);
+    if (e != cudaSuccess) return e;
+    k_bwd_own<<<dim3(T_len, sh.B), threads, 0, st>>>(a, (const bf16*)(ws + l.qt), (const bf16*)(ws + l.fwd),
+                                                      (const bf16*)(ws + l.dob), in.lse, in.delta);
+    k_bwd_query<bf16><<<dim3(T_len, sh.B), threads, 0, st>>>(a, g.dq_c, g.dq_r);
+    const int64_t M = (int64_t)sh.B * T_len;
+    k_bwd_weights<bf16, bf16><<<dim3((unsigned)((M + kWChunk - 1) / kWChunk), sh.H, sh.d_h / kWRows), 256, 0, st>>>(
+        a, g.dw_uk, g.dw_uv);
+    k_bwd_scan<bf16><<<dim3((n_slots + 7) / 8, sh.B), 256, 0, st>>>(a, pa.c, pa.kr, pa.gate_w, g.dc, g.dkr,
+                                                                    g.dgate_w, g.dgate_b, g.dgate_in);
+    *launches += 5;
+    return note_error("backward launch", cudaGetLastError());
+}
+
 }  // namespace
 
 size_t prefill_backward_workspace(const Shape& sh, int T, size_t elem_bytes) {
-    return bwd_layout(sh, T, elem_bytes).total;
+    return use_tc(sh, elem_bytes == 4) ? bwd_tc_layout(sh, T).total : bwd_layout(sh, T, elem_bytes).total;
 }
 
 cudaError_t prefill_backward(const PrefillArgs& a, const BackwardGrads& g, bool fp32, cudaStream_t st,
                              uint64_t* launches) {
+    if (use_tc(a.sh, fp32)) return backward_tc(a, g, st, launches);
     return fp32 ? backward_impl<float>(a, g, st, launches) : backward_impl<bf16>(a, g, st, launches);
 }
 

@@ -88,6 +88,43 @@ bool tc_prefill_supported(const Shape& sh);
 size_t tc_prefill_workspace(const Shape& sh, int T);
 cudaError_t tc_prefill(const PrefillArgs& a, cudaStream_t st, uint64_t* launches);
 
+// Row pitch (positions) of the per-row statistics [B, H, T] the training
+// backward keeps: T rounded up to 4, so that a row is a multiple of 16 bytes
+// (a TMA stride).
+__host__ __device__ inline int stats_pitch(int T) { return (T + 3) & ~3; }
+
+// The tensor-core prefill from t0 = 0 with what the training backward keeps:
+// the merging weights w [B, T] (fp32), per row the log2-domain log-sum-exp
+// lse [B, H, stats_pitch(T)] (fp32), O / l obar [B, T, H, d_c] (bf16) and the absorbed
+// query qt [B, T, H, D] (bf16) as the score MMAs used it. The partial slots
+// stay in the first region of a.workspace (bf16 [B, T, D]).
+struct PrefillSave {
+    float* w;
+    float* lse;
+    void* obar;
+    void* qt;
+};
+cudaError_t tc_prefill_save(const PrefillArgs& a, const PrefillSave& sv, cudaStream_t st, uint64_t* launches);
+
+// The masked attention of the training backward on the tensor cores
+// (tc_backward.cu; bf16, d_h = 64, d_R = 32, d_c = 128 or 256, scalar gates):
+// from the forward's kept rows (qt, lse, obar through delta), dobar and the
+// finished slots, the finished-slot parts dqt [B, T, H, D] (fp32, written
+// whole) and dF [H, B, n_slots, D] (fp32, per head, written whole).
+struct BwdTCInputs {
+    const void* qt;        // [B, T, H, D] bf16
+    const void* dob;       // [B, T, H, d_c] bf16
+    const void* slots;     // [B, n_slots, D] bf16 (the forward's cache rows)
+    const float* lse;      // [B, H, stats_pitch(T)]
+    const float* delta;    // [B, H, stats_pitch(T)]
+    float* dqt;
+    float* dF;
+    int* status;
+};
+bool tc_backward_supported(const Shape& sh);
+cudaError_t tc_backward_attention(const Shape& sh, int T, const BwdTCInputs& in, cudaStream_t st,
+                                  uint64_t* launches);
+
 // y[M, N] = x[M, K] . w[N, K]^T, bf16 in and out, fp32 accumulation (gemm.cu).
 // Rows ldx / ldw / ldy elements apart (ldx, ldw multiples of 8).
 cudaError_t gemm_bf16(const void* x, int ldx, const void* w, int ldw, void* y, int ldy, int M, int N, int K,

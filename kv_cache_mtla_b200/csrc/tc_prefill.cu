@@ -67,6 +67,12 @@ struct PreTC {
     const bf16* q_r;  // [B, T, H, d_r]
     const float2* rope_tab;   // [T, d_r / 2]: (cos, sin) of every position, from the scan
     bf16* out;        // [B, T, H, d_h]
+    // kept for the training backward when not null (t0 = 0): per row the
+    // log2-domain log-sum-exp [B, H, T], O / l [B, T, H, d_c] and the absorbed
+    // query as the score MMAs used it [B, T, H, D], bf16
+    float* lse;
+    bf16* obar;
+    bf16* qt;
     int* status;
 };
 
@@ -423,6 +429,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
                 for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
                 if (col < DC) st_row32_packed(q_s, kQ * 128, r, col, w, false);
                 else st_row32_packed(q_s + NL * kQ * 128, 0, r, col - DC, w, true);
+                if (p.qt && row_ok) {
+                    uint4* g = (uint4*)(p.qt + (((size_t)b * p.T + pos) * p.H + h) * p.D + col);
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) g[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+                }
             };
             float e_own = 0.f;
             // 8 columns [c, c + 8) of this row's own partial slot, from the ring
@@ -594,8 +605,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
             tc_fence_after();
             bs.xs[hc][r] = l;
             named_sync(1, 256);
-            const float inv = 1.f / (bs.xs[0][r] + bs.xs[1][r]);
+            const float l_row = bs.xs[0][r] + bs.xs[1][r];
+            const float inv = 1.f / l_row;
             named_sync(1, 256);                           // xs is free again
+            if (p.lse && row_ok && hc == 0)
+                p.lse[((size_t)b * p.H + h) * stats_pitch(p.T) + pos] = m_ref + log2f(l_row);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const int cc = hc * half + 32 * q;
@@ -605,6 +619,12 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
 #pragma unroll
                     for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(v[2 * i] * inv, v[2 * i + 1] * inv);
                     tmem_st16_u(t_olat + cc / 2 + lane_off, w);
+                    if (p.obar && row_ok) {
+                        uint4* g = (uint4*)(p.obar + (((size_t)b * p.T + pos) * p.H + h) * DC + cc);
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            g[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+                    }
                 }
             }
             tmem_wait_st();
@@ -701,7 +721,8 @@ size_t tc_prefill_workspace(const Shape& sh, int T) {
            prefill_seed_bytes(sh);
 }
 
-cudaError_t tc_prefill(const PrefillArgs& a_in, cudaStream_t st, uint64_t* launches) {
+static cudaError_t tc_prefill_impl(const PrefillArgs& a_in, const PrefillSave* sv, cudaStream_t st,
+                                   uint64_t* launches) {
     PrefillArgs a = a_in;
     const Shape& sh = a.sh;
     const int T = a.T;
@@ -771,13 +792,17 @@ cudaError_t tc_prefill(const PrefillArgs& a_in, cudaStream_t st, uint64_t* launc
     p.q_r = (const bf16*)a.q_r;
     p.rope_tab = (const float2*)((char*)a.workspace + align256((size_t)sh.B * T * sh.D * sizeof(bf16)));
     p.out = (bf16*)a.out;
+    p.lse = sv ? sv->lse : nullptr;
+    p.obar = sv ? (bf16*)sv->obar : nullptr;
+    p.qt = sv ? (bf16*)sv->qt : nullptr;
     p.status = a.status;
 
     const int n_slots = (a.t0 + T - 1) / sh.s - a.t0 / sh.s + 1;    // slots the chunk touches
     if (sh.gate_mode >= 3)
         k_prefill_scan_channel<bf16, bf16><<<dim3((n_slots + 7) / 8, sh.B), 256, 0, st>>>(a, P, (float2*)p.rope_tab);
     else
-        k_prefill_scan<bf16, bf16><<<dim3((n_slots + 7) / 8, sh.B), 256, 0, st>>>(a, P, (float2*)p.rope_tab);
+        k_prefill_scan<bf16, bf16><<<dim3((n_slots + 7) / 8, sh.B), 256, 0, st>>>(a, P, (float2*)p.rope_tab,
+                                                                              sv ? sv->w : nullptr);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return note_error("k_prefill_scan launch", e);
 
@@ -790,11 +815,22 @@ cudaError_t tc_prefill(const PrefillArgs& a_in, cudaStream_t st, uint64_t* launc
     // persistent: one CTA per SM (the shared memory allows no second), each
     // walking its share of the items
     const unsigned grid = (unsigned)std::min(p.n_items, sm_count());
-    profile_begin(st);
+    // the attention kernel's event pair (not inside the training backward,
+    // whose own pair brackets its tensor-core kernels)
+    if (!sv) profile_begin(st);
     kern<<<grid, kThreads, smem, st>>>(maps, p);
-    profile_end(st);
+    if (!sv) profile_end(st);
     *launches += 2;
     return note_error("k_prefill_tc launch", cudaGetLastError());
+}
+
+cudaError_t tc_prefill(const PrefillArgs& a, cudaStream_t st, uint64_t* launches) {
+    return tc_prefill_impl(a, nullptr, st, launches);
+}
+
+cudaError_t tc_prefill_save(const PrefillArgs& a, const PrefillSave& sv, cudaStream_t st, uint64_t* launches) {
+    if (a.t0 != 0 || a.sh.gate_mode >= 3) return note_error("tc_prefill_save: t0 = 0, scalar gates", cudaErrorInvalidValue);
+    return tc_prefill_impl(a, &sv, st, launches);
 }
 
 }  // namespace mtla

@@ -26,6 +26,14 @@ pytestmark = pytest.mark.gpu
 BWD_TOL = TOL["fp32"]
 
 
+def tol_for(wl):
+    """bf16 at the tensor-core widths (d_h=64, d_R=32, d_c 128 or 256) runs the
+    tensor-core backward (bf16 operands: the bf16 bound); everything else the
+    fp32 CUDA-core backward (the fp32 bound)."""
+    tc = wl.dtype == "bf16" and wl.d_h == 64 and wl.d_r == 32 and wl.d_c in (128, 256)
+    return TOL["bf16"] if tc else BWD_TOL
+
+
 @pytest.fixture(autouse=True)
 def _clean_status():
     torch.cuda.synchronize()
@@ -76,7 +84,7 @@ def oracle_backward(wl, w, toks, dout, B=None):
                                    w["gate_b"] if computed else None, toks["gate_in"])
 
 
-def check_all(wl, grads, ref, tol=BWD_TOL):
+def check_all(wl, grads, ref, tol=None):
     """Every gradient within tol; the computed gate's weight G and bias g are
     one linear layer and are compared as one parameter tensor."""
     got, want = {}, {}
@@ -88,6 +96,7 @@ def check_all(wl, grads, ref, tol=BWD_TOL):
         got["dgate"] = np.concatenate([got.pop("dgate_w").ravel(), got.pop("dgate_b")])
         want["dgate"] = np.concatenate([want.pop("dgate_w").ravel(), want.pop("dgate_b")])
     errs = {k: rel_err(got[k], want[k]) for k in got}
+    tol = tol_for(wl) if tol is None else tol
     assert max(errs.values()) <= tol, errs
 
 
@@ -129,6 +138,20 @@ def test_backward_speech_widths(s, T):
     check_all(wl, run_backward(wl, T, w, toks, dout), oracle_backward(wl, w, toks, dout))
 
 
+@pytest.mark.parametrize("d_c,s,T,mode", [(128, 2, 200, inputs.GATE_COMPUTED), (256, 1, 130, inputs.GATE_UNIT),
+                                          (256, 3, 1, inputs.GATE_SUPPLIED), (256, 2, 2, inputs.GATE_COMPUTED),
+                                          (128, 8, 333, inputs.GATE_SUPPLIED)])
+def test_backward_tensor_core_shapes(d_c, s, T, mode):
+    """The tensor-core backward's other cases: d_c=128, s=1 and s=8, every gate
+    mode, T=1 and T=2 (no finished slot at all), T not a multiple of 4 (the
+    statistics' padded pitch)."""
+    wl = inputs.PREFILL.with_(B=2, d_c=d_c, s=s, gate_mode=mode)
+    w = inputs.weights(wl)
+    toks = inputs.tokens(wl, T)
+    dout = inputs.grad_out(wl, T)
+    check_all(wl, run_backward(wl, T, w, toks, dout), oracle_backward(wl, w, toks, dout))
+
+
 def test_backward_large_latent_widths():
     """The large-latent widths (H=128 > 8 warps per block, d_c=512, d_R=64:
     slot width 576, the widest), supplied gates, s=4, T=45."""
@@ -151,12 +174,12 @@ def test_backward_degenerate_lengths(T):
     check_all(wl, run_backward(wl, T, w, toks, dout), oracle_backward(wl, w, toks, dout))
 
 
-def test_backward_is_repeatable():
+@pytest.mark.parametrize("wl,T", [(inputs.TINY_FP32.with_(B=2, s=3), 50), (inputs.PREFILL.with_(B=2, s=3), 300)],
+                         ids=["cuda_cores", "tensor_cores"])
+def test_backward_is_repeatable(wl, T):
     """Two calls on the same inputs: the heads' key gradients are summed in a
     fixed order, so the per-token gradients are the same bytes; the weight and
     gate gradients (atomic additions over token rows) agree to rounding."""
-    wl = inputs.TINY_FP32.with_(B=2, s=3)
-    T = 50
     w = inputs.weights(wl)
     toks = inputs.tokens(wl, T)
     dout = inputs.grad_out(wl, T)
