@@ -30,7 +30,7 @@
 //   k_bwd_columns     block (j, b), a warp per head: the finished slot F_j's
 //                     key gradient over every query that sees it
 //   k_bwd_query       dqC, dqR
-//   k_bwd_weights     dW_UK, dW_UV (row chunks, atomics into zeroed outputs)
+//   k_bwd_wpart/wsum  dW_UK, dW_UV (per row chunk, then the chunks in order)
 //   k_bwd_scan        a warp per slot: the scan and gate backward
 #include "common.cuh"
 #include "mtla_internal.h"
@@ -42,8 +42,8 @@ namespace {
 
 constexpr int kMaxD = 576;             // slot width the kernels hold (d_c + d_R)
 constexpr int kPer = kMaxD / 32;       // a lane's channels: lane + 32 k
-constexpr int kWRows = 16;             // dW rows r per block of k_bwd_weights
-constexpr int kWChunk = 512;           // token rows per block of k_bwd_weights
+constexpr int kWR = 32;                // dW rows r per block of k_bwd_wpart
+constexpr int kWChunk = 1024;          // token rows per block of k_bwd_wpart
 
 struct BwdArgs {
     Shape sh;
@@ -251,51 +251,71 @@ __global__ void __launch_bounds__(256) k_bwd_query(BwdArgs a, float* dqc, float*
     }
 }
 
-// dW_UK[h][r][c] += sum_rows qC[r] dqt[c], dW_UV[h][r][c] += sum_rows dout[r] obar[c]
-// over token rows m0 .. m0 + kWChunk - 1: block (row chunk, h, r group), a
-// thread per channel c (two when d_c > 256).
-template <typename T, typename OT>
-__global__ void __launch_bounds__(256) k_bwd_weights(BwdArgs a, float* dw_uk, float* dw_uv) {
+// Weight gradients in two deterministic stages. k_bwd_wpart: block (row chunk,
+// h, group of 32 r), a thread per channel c: over the chunk's token rows m,
+//   partK[chunk][h][r][c] = sum_m qC[m,h,r] g[m,h,c],  g = dqt[0:d_c]
+//   partV[chunk][h][r][c] = sum_m dout[m,h,r] obar[m,h,c]
+// (g and obar rows g_pitch / d_c elements apart, of type GT / OT); then
+// k_bwd_wsum adds the chunks in order: dW_UK = sum partK, dW_UV = sum partV.
+template <typename T, typename GT, typename OT>
+__global__ void __launch_bounds__(256) k_bwd_wpart(BwdArgs a, const void* g, int g_pitch, float* part_k,
+                                                   float* part_v) {
     const Shape sh = a.sh;
-    const int h = blockIdx.y, r0 = blockIdx.z * kWRows, tid = threadIdx.x;
+    const int chunk = blockIdx.x, h = blockIdx.y, r0 = blockIdx.z * kWR, tid = threadIdx.x;
     const int64_t M = (int64_t)sh.B * a.T;
-    const int64_t m0 = (int64_t)blockIdx.x * kWChunk, m1 = m0 + kWChunk < M ? m0 + kWChunk : M;
-    __shared__ float qs[kWRows], os[kWRows];
-    float gk[2][kWRows], gv[2][kWRows];
+    const int64_t m0 = (int64_t)chunk * kWChunk, m1 = m0 + kWChunk < M ? m0 + kWChunk : M;
+    __shared__ float qs[32][kWR], os[32][kWR];
+    for (int c0 = 0; c0 < sh.d_c; c0 += 256) {
+        const int c = c0 + tid;
+        float gk[kWR], gv[kWR];
 #pragma unroll
-    for (int cc = 0; cc < 2; ++cc)
-#pragma unroll
-        for (int r = 0; r < kWRows; ++r) gk[cc][r] = gv[cc][r] = 0.f;
-    for (int64_t m = m0; m < m1; ++m) {
-        const size_t row = (size_t)m * sh.H + h;
-        __syncthreads();
-        if (tid < kWRows) qs[tid] = ldf<T>(a.qc, row * sh.d_h + r0 + tid);
-        else if (tid < 2 * kWRows) os[tid - kWRows] = ldf<T>(a.dout, row * sh.d_h + r0 + tid - kWRows);
-        __syncthreads();
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-            const int c = tid + 256 * cc;
+        for (int r = 0; r < kWR; ++r) gk[r] = gv[r] = 0.f;
+        for (int64_t mb = m0; mb < m1; mb += 32) {
+            __syncthreads();
+            for (int q = tid; q < 32 * kWR; q += blockDim.x) {
+                const int mm = q / kWR, rr = q % kWR;
+                const int64_t m = mb + mm;
+                const bool ok = m < m1 && r0 + rr < sh.d_h;
+                const size_t row = (size_t)m * sh.H + h;
+                qs[mm][rr] = ok ? ldf<T>(a.qc, row * sh.d_h + r0 + rr) : 0.f;
+                os[mm][rr] = ok ? ldf<T>(a.dout, row * sh.d_h + r0 + rr) : 0.f;
+            }
+            __syncthreads();
             if (c < sh.d_c) {
-                const float x = a.dqt[row * sh.D + c], y = ldf<OT>(a.obar, row * sh.d_c + c);
+                const int nm = (int)(m1 - mb < 32 ? m1 - mb : 32);
+                for (int mm = 0; mm < nm; ++mm) {
+                    const size_t row = (size_t)(mb + mm) * sh.H + h;
+                    const float x = ldf<GT>(g, row * g_pitch + c), y = ldf<OT>(a.obar, row * sh.d_c + c);
 #pragma unroll
-                for (int r = 0; r < kWRows; ++r) {
-                    gk[cc][r] = fmaf(qs[r], x, gk[cc][r]);
-                    gv[cc][r] = fmaf(os[r], y, gv[cc][r]);
+                    for (int r = 0; r < kWR; ++r) {
+                        gk[r] = fmaf(qs[mm][r], x, gk[r]);
+                        gv[r] = fmaf(os[mm][r], y, gv[r]);
+                    }
                 }
             }
         }
-    }
-#pragma unroll
-    for (int cc = 0; cc < 2; ++cc) {
-        const int c = tid + 256 * cc;
         if (c < sh.d_c)
 #pragma unroll
-            for (int r = 0; r < kWRows; ++r) {
-                const size_t o = ((size_t)h * sh.d_h + r0 + r) * sh.d_c + c;
-                atomicAdd(&dw_uk[o], gk[cc][r]);
-                atomicAdd(&dw_uv[o], gv[cc][r]);
-            }
+            for (int r = 0; r < kWR; ++r)
+                if (r0 + r < sh.d_h) {
+                    const size_t o = (((size_t)chunk * sh.H + h) * sh.d_h + r0 + r) * sh.d_c + c;
+                    part_k[o] = gk[r];
+                    part_v[o] = gv[r];
+                }
     }
+}
+
+__global__ void __launch_bounds__(256) k_bwd_wsum(int n_chunks, size_t n, const float* part_k, const float* part_v,
+                                                  float* dw_uk, float* dw_uv) {
+    const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n) return;
+    float k = 0.f, v = 0.f;
+    for (int q = 0; q < n_chunks; ++q) {
+        k += part_k[(size_t)q * n + i];
+        v += part_v[(size_t)q * n + i];
+    }
+    dw_uk[i] = k;
+    dw_uv[i] = v;
 }
 
 // Scan and gate backward: a warp per slot j of sequence b, its tokens from the
@@ -383,62 +403,51 @@ __global__ void __launch_bounds__(256) k_bwd_scan(BwdArgs a, const void* c_in, c
     }
 }
 
-// Tensor-core path, per (16 positions, head, sequence): dobar = W_UV[h]^T dout
-// rounded to bf16 (the operand of the tensor-core kernels) and delta =
-// dobar . obar from the same rounded values, in the [B, H, T] layout.
-template <typename T>
-__global__ void __launch_bounds__(256) k_bwd_dob(BwdArgs a, bf16* dob, float* delta) {
-    const Shape sh = a.sh;
-    const int t0 = blockIdx.x * 16, h = blockIdx.y, b = blockIdx.z;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    __shared__ float dsm[16][256];
-    __shared__ float red[8][16];
-    for (int q = tid; q < 16 * sh.d_h; q += blockDim.x) {
-        const int pp = q / sh.d_h, r = q % sh.d_h, t = t0 + pp;
-        dsm[pp][r] = t < a.T ? ldf<T>(a.dout, (((size_t)b * a.T + t) * sh.H + h) * sh.d_h + r) : 0.f;
+// Tensor-core path: W_UV^T [H][d_c][d_h] (the B operand of the dobar GEMM).
+__global__ void __launch_bounds__(256) k_transpose_wuv(Shape sh, const bf16* w, bf16* wt) {
+    const size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const size_t n = (size_t)sh.H * sh.d_h * sh.d_c;
+    if (i >= n) return;
+    const int c = (int)(i % sh.d_c);
+    const size_t hr = i / sh.d_c;
+    const int r = (int)(hr % sh.d_h), h = (int)(hr / sh.d_h);
+    wt[((size_t)h * sh.d_c + c) * sh.d_h + r] = w[i];
+}
+
+// Tensor-core path: delta = dobar . obar per row from the bf16 values the
+// tensor-core kernels read, in the [B, H, pitch] layout; a warp per row
+// (b, t, h), 8 channels a lane.
+__global__ void __launch_bounds__(256) k_bwd_delta(Shape sh, int T, const bf16* dob, const bf16* obar, float* delta) {
+    const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    const int64_t rows = (int64_t)sh.B * T * sh.H;
+    if (row >= rows) return;
+    float acc = 0.f;
+    for (int c0 = lane * 8; c0 < sh.d_c; c0 += 256) {
+        float x[8], y[8];
+        load8<bf16>(dob + row * sh.d_c + c0, x);
+        load8<bf16>(obar + row * sh.d_c + c0, y);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) acc = fmaf(x[u], y[u], acc);
     }
-    __syncthreads();
-    float dl[16];
-#pragma unroll
-    for (int pp = 0; pp < 16; ++pp) dl[pp] = 0.f;
-    for (int c = tid; c < sh.d_c; c += blockDim.x) {
-        float acc[16];
-#pragma unroll
-        for (int pp = 0; pp < 16; ++pp) acc[pp] = 0.f;
-        for (int r = 0; r < sh.d_h; ++r) {
-            const float wv = ldf<T>(a.w_uv, ((size_t)h * sh.d_h + r) * sh.d_c + c);
-#pragma unroll
-            for (int pp = 0; pp < 16; ++pp) acc[pp] = fmaf(dsm[pp][r], wv, acc[pp]);
-        }
-#pragma unroll
-        for (int pp = 0; pp < 16; ++pp) {
-            const int t = t0 + pp;
-            if (t < a.T) {
-                const size_t o = (((size_t)b * a.T + t) * sh.H + h) * sh.d_c + c;
-                const bf16 v = __float2bfloat16_rn(acc[pp]);
-                dob[o] = v;
-                dl[pp] = fmaf(__bfloat162float(v), ldf<bf16>(a.obar, o), dl[pp]);
-            }
-        }
-    }
-#pragma unroll
-    for (int pp = 0; pp < 16; ++pp) {
-        const float v = warp_sum(dl[pp]);
-        if (lane == 0) red[warp][pp] = v;
-    }
-    __syncthreads();
-    if (tid < 16 && t0 + tid < a.T) {
-        float v = 0.f;
-        for (int q = 0; q < (int)(blockDim.x >> 5); ++q) v += red[q][tid];
-        delta[((size_t)b * sh.H + h) * stats_pitch(a.T) + t0 + tid] = v;
+    acc = warp_sum(acc);
+    if (lane == 0) {
+        const int h = (int)(row % sh.H);
+        const int64_t bt = row / sh.H;
+        const int t = (int)(bt % T), b = (int)(bt / T);
+        delta[((size_t)b * sh.H + h) * stats_pitch(T) + t] = acc;
     }
 }
 
-// Tensor-core path: the own-partial term of every row (one key, P_i), added
-// to the finished-slot part of dqt; dP_i = the heads' own-partial key
-// gradients (summed in a fixed order). Block (i, b), a warp per head.
-__global__ void __launch_bounds__(256) k_bwd_own(BwdArgs a, const bf16* qt, const bf16* P, const bf16* dob,
-                                                 const float* lse, const float* delta) {
+// Tensor-core path: the own-partial term of every row (one key, P_i) added to
+// the finished-slot part of dqt; then the row's query gradients leave: the
+// latent part as bf16 (the operand of the dqC GEMM and the weight gradients)
+// and dqR = R_i^T dqt[d_c:] (fp32, the output); dP_i = the heads' own-partial
+// key gradients, summed in a fixed order. Block (i, b), a warp per head, 8
+// channels a lane (16-byte loads).
+constexpr int kOwnGroups = 2;          // 8-channel groups a lane takes: D <= 512 (the tensor-core widths)
+__global__ void __launch_bounds__(256, 2) k_bwd_own(BwdArgs a, const bf16* qt, const bf16* P, const bf16* dob,
+                                                 const float* lse, const float* delta, bf16* dqtl, float* dq_r) {
     const Shape sh = a.sh;
     const int i = blockIdx.x, b = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
@@ -448,31 +457,58 @@ __global__ void __launch_bounds__(256) k_bwd_own(BwdArgs a, const bf16* qt, cons
     float* own = dkey_own[warp];
     for (int q = lane; q < D; q += 32) own[q] = 0.f;
     const bf16* Pi = P + ((size_t)b * a.T + i) * D;
-    float pv[kPer];
+    float pv[kOwnGroups][8];
 #pragma unroll
-    for (int k = 0; k < kPer; ++k) pv[k] = lane + 32 * k < D ? __bfloat162float(Pi[lane + 32 * k]) : 0.f;
+    for (int k = 0; k < kOwnGroups; ++k) {
+        const int c0 = 8 * (lane + 32 * k);
+        if (c0 < D) load8<bf16>(Pi + c0, pv[k]);
+        else
+#pragma unroll
+            for (int u = 0; u < 8; ++u) pv[k][u] = 0.f;
+    }
     for (int h = warp; h < sh.H; h += nw) {
         const size_t row = ((size_t)b * a.T + i) * sh.H + h;
         const size_t srow = ((size_t)b * sh.H + h) * stats_pitch(a.T) + i;
-        float qv[kPer], dv[kPer], e = 0.f, da = 0.f;
+        float qv[kOwnGroups][8], dv[kOwnGroups][8], e = 0.f, da = 0.f;
 #pragma unroll
-        for (int k = 0; k < kPer; ++k) {
-            const int c = lane + 32 * k;
-            qv[k] = c < D ? __bfloat162float(qt[row * D + c]) : 0.f;
-            dv[k] = c < d_c ? __bfloat162float(dob[row * d_c + c]) : 0.f;
-            e = fmaf(qv[k], pv[k], e);
-            da = fmaf(dv[k], pv[k], da);
+        for (int k = 0; k < kOwnGroups; ++k) {
+            const int c0 = 8 * (lane + 32 * k);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) qv[k][u] = dv[k][u] = 0.f;
+            if (c0 < D) load8<bf16>(qt + row * D + c0, qv[k]);
+            if (c0 < d_c) load8<bf16>(dob + row * d_c + c0, dv[k]);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                e = fmaf(qv[k][u], pv[k][u], e);
+                da = fmaf(dv[k][u], pv[k][u], da);
+            }
         }
         e = warp_sum(e);
         da = warp_sum(da);
         const float pr = exp2f(fmaf(e, scale_log2, -lse[srow]));
         const float sde = sh.scale * pr * (da - delta[srow]);
 #pragma unroll
-        for (int k = 0; k < kPer; ++k) {
-            const int c = lane + 32 * k;
-            if (c < D) {
-                a.dqt[row * D + c] += sde * pv[k];
-                own[c] += fmaf(sde, qv[k], pr * dv[k]);
+        for (int k = 0; k < kOwnGroups; ++k) {
+            const int c0 = 8 * (lane + 32 * k);
+            if (c0 >= D) continue;
+            float g[8];
+            load8<float>(a.dqt + row * D + c0, g);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                g[u] = fmaf(sde, pv[k][u], g[u]);
+                own[c0 + u] += fmaf(sde, qv[k][u], pr * dv[k][u]);
+            }
+            if (c0 < d_c) {
+                store8<bf16>(dqtl + row * d_c + c0, g);
+            } else {
+#pragma unroll
+                for (int u = 0; u < 8; u += 2) {
+                    const int kp = (c0 - d_c + u) / 2;        // RoPE pair
+                    float sn, cs;
+                    pair_sincos(i, kp, sh.d_r, sh.log2_rope_base, &sn, &cs);
+                    dq_r[row * sh.d_r + 2 * kp] = fmaf(g[u], cs, g[u + 1] * sn);        // R_i^T
+                    dq_r[row * sh.d_r + 2 * kp + 1] = fmaf(-g[u], sn, g[u + 1] * cs);
+                }
             }
         }
     }
@@ -485,8 +521,25 @@ __global__ void __launch_bounds__(256) k_bwd_own(BwdArgs a, const bf16* qt, cons
 }
 
 struct BwdWs {
-    size_t P, w, cache, qt, mrow, lrow, delta, dob, obar, dqt, dP, dF, total;
+    size_t P, w, cache, qt, mrow, lrow, delta, dob, obar, dqt, dP, dF, part_k, part_v, total;
 };
+
+int weight_chunks(const Shape& sh, int T) { return (int)(((int64_t)sh.B * T + kWChunk - 1) / kWChunk); }
+size_t weight_part_bytes(const Shape& sh, int T) {
+    return (size_t)weight_chunks(sh, T) * sh.H * sh.d_h * sh.d_c * sizeof(float);
+}
+
+// dW_UK, dW_UV from the rows' latent query gradients g (rows g_pitch apart, type GT)
+template <typename T, typename GT, typename OT>
+cudaError_t weight_grads(const BwdArgs& a, const void* g, int g_pitch, float* part_k, float* part_v, float* dw_uk,
+                         float* dw_uv, cudaStream_t st) {
+    const Shape& sh = a.sh;
+    const int nc = weight_chunks(sh, a.T);
+    k_bwd_wpart<T, GT, OT><<<dim3(nc, sh.H, (sh.d_h + kWR - 1) / kWR), 256, 0, st>>>(a, g, g_pitch, part_k, part_v);
+    const size_t n = (size_t)sh.H * sh.d_h * sh.d_c;
+    k_bwd_wsum<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(nc, n, part_k, part_v, dw_uk, dw_uv);
+    return cudaGetLastError();
+}
 
 BwdWs bwd_layout(const Shape& sh, int T, size_t elem) {
     const size_t BT = (size_t)sh.B * T, rows = BT * sh.H;
@@ -506,6 +559,8 @@ BwdWs bwd_layout(const Shape& sh, int T, size_t elem) {
     l.dqt = take(rows * sh.D * 4);
     l.dP = take(BT * sh.D * 4);
     l.dF = take((size_t)sh.B * n_slots * sh.D * 4);
+    l.part_k = take(weight_part_bytes(sh, T));
+    l.part_v = take(weight_part_bytes(sh, T));
     l.total = o;
     return l;
 }
@@ -543,10 +598,7 @@ cudaError_t backward_impl(const PrefillArgs& pa_in, const BackwardGrads& g, cuda
     a.dP = (float*)(ws + l.dP);
     a.dF = (float*)(ws + l.dF);
     a.n_parts = 1;
-    const size_t wbytes = (size_t)sh.H * sh.d_h * sh.d_c * sizeof(float);
     cudaError_t e;
-    if ((e = cudaMemsetAsync(g.dw_uk, 0, wbytes, st)) != cudaSuccess) return note_error("backward zero dW_UK", e);
-    if ((e = cudaMemsetAsync(g.dw_uv, 0, wbytes, st)) != cudaSuccess) return note_error("backward zero dW_UV", e);
     if (sh.gate_mode == 0) {
         if ((e = cudaMemsetAsync(g.dgate_w, 0, (size_t)sh.s * sh.d_c * sizeof(float), st)) != cudaSuccess)
             return note_error("backward zero dG", e);
@@ -563,19 +615,19 @@ cudaError_t backward_impl(const PrefillArgs& pa_in, const BackwardGrads& g, cuda
     k_bwd_columns<<<dim3(n_slots, sh.B), threads, 0, st>>>(a);
     profile_end(st);
     k_bwd_query<T><<<dim3(T_len, sh.B), threads, 0, st>>>(a, g.dq_c, g.dq_r);
-    const int64_t M = (int64_t)sh.B * T_len;
-    k_bwd_weights<T, float><<<dim3((unsigned)((M + kWChunk - 1) / kWChunk), sh.H, sh.d_h / kWRows), 256, 0, st>>>(
-        a, g.dw_uk, g.dw_uv);
+    if ((e = weight_grads<T, float, float>(a, a.dqt, sh.D, (float*)(ws + l.part_k), (float*)(ws + l.part_v),
+                                           g.dw_uk, g.dw_uv, st)) != cudaSuccess)
+        return note_error("backward weight-gradient launch", e);
     k_bwd_scan<T><<<dim3((n_slots + 7) / 8, sh.B), 256, 0, st>>>(a, pa.c, pa.kr, pa.gate_w, g.dc, g.dkr, g.dgate_w,
                                                                  g.dgate_b, g.dgate_in);
-    *launches += 7;
+    *launches += 8;
     return note_error("backward launch", cudaGetLastError());
 }
 
 // ---------------------------------------------------------------- tensor-core path
 
 struct BwdTcWs {
-    size_t fwd, cache, out, lse, delta, obar, qt, w, dob, dqt, dF, dP, total;
+    size_t fwd, cache, out, lse, delta, obar, qt, w, dob, dqt, dF, dP, wuvt, dqtl, part_k, part_v, total;
 };
 
 Shape with_slots(const Shape& sh, int T) {
@@ -602,6 +654,10 @@ BwdTcWs bwd_tc_layout(const Shape& sh_in, int T) {
     l.dqt = take(rows * sh.D * 4);
     l.dF = take((size_t)sh.H * sh.B * sh.max_slots * sh.D * 4);
     l.dP = take(BT * sh.D * 4);
+    l.wuvt = take((size_t)sh.H * sh.d_h * sh.d_c * 2);
+    l.dqtl = take(rows * sh.d_c * 2);
+    l.part_k = take(weight_part_bytes(sh, T));
+    l.part_v = take(weight_part_bytes(sh, T));
     l.total = o;
     return l;
 }
@@ -629,10 +685,7 @@ cudaError_t backward_tc(const PrefillArgs& pa_in, const BackwardGrads& g, cudaSt
     pa.open_slot_in = nullptr;
     pa.open_slot_out = nullptr;
     pa.t0 = 0;
-    const size_t wbytes = (size_t)sh.H * sh.d_h * sh.d_c * sizeof(float);
     cudaError_t e;
-    if ((e = cudaMemsetAsync(g.dw_uk, 0, wbytes, st)) != cudaSuccess) return note_error("backward zero dW_UK", e);
-    if ((e = cudaMemsetAsync(g.dw_uv, 0, wbytes, st)) != cudaSuccess) return note_error("backward zero dW_UV", e);
     if (sh.gate_mode == 0) {
         if ((e = cudaMemsetAsync(g.dgate_w, 0, (size_t)sh.s * sh.d_c * sizeof(float), st)) != cudaSuccess)
             return note_error("backward zero dG", e);
@@ -664,9 +717,20 @@ cudaError_t backward_tc(const PrefillArgs& pa_in, const BackwardGrads& g, cudaSt
     a.dF = (float*)(ws + l.dF);
     a.n_parts = sh.H;
     const int threads = 32 * (sh.H < 8 ? sh.H : 8);
-    k_bwd_dob<bf16><<<dim3((T_len + 15) / 16, sh.H, sh.B), 256, 0, st>>>(a, (bf16*)(ws + l.dob),
-                                                                          (float*)(ws + l.delta));
-    if ((e = cudaGetLastError()) != cudaSuccess) return note_error("k_bwd_dob launch", e);
+    const int M = sh.B * T_len;
+    bf16* dob = (bf16*)(ws + l.dob);
+    // dobar = dout . W_UV[h] on the tensor cores (W_UV^T as the K-major operand),
+    // then delta = dobar . obar
+    const size_t nw = (size_t)sh.H * sh.d_h * sh.d_c;
+    k_transpose_wuv<<<(unsigned)((nw + 255) / 256), 256, 0, st>>>(sh, (const bf16*)pa.w_uv, (bf16*)(ws + l.wuvt));
+    e = gemm_batched(GemmOperand{g.dout, sh.H * sh.d_h, (size_t)sh.d_h},
+                     GemmOperand{ws + l.wuvt, sh.d_h, (size_t)sh.d_c * sh.d_h}, dob, sh.H * sh.d_c, (size_t)sh.d_c,
+                     false, M, sh.d_c, sh.d_h, sh.H, pa.status, st, launches);
+    if (e != cudaSuccess) return e;
+    const int64_t rows = (int64_t)M * sh.H;
+    k_bwd_delta<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(sh, T_len, dob, (const bf16*)(ws + l.obar),
+                                                             (float*)(ws + l.delta));
+    if ((e = cudaGetLastError()) != cudaSuccess) return note_error("k_bwd_delta launch", e);
     BwdTCInputs in;
     in.qt = ws + l.qt;
     in.dob = ws + l.dob;
@@ -680,15 +744,21 @@ cudaError_t backward_tc(const PrefillArgs& pa_in, const BackwardGrads& g, cudaSt
     e = tc_backward_attention(sh, T_len, in, st, launches);
     profile_end(st);
     if (e != cudaSuccess) return e;
-    k_bwd_own<<<dim3(T_len, sh.B), threads, 0, st>>>(a, (const bf16*)(ws + l.qt), (const bf16*)(ws + l.fwd),
-                                                      (const bf16*)(ws + l.dob), in.lse, in.delta);
-    k_bwd_query<bf16><<<dim3(T_len, sh.B), threads, 0, st>>>(a, g.dq_c, g.dq_r);
-    const int64_t M = (int64_t)sh.B * T_len;
-    k_bwd_weights<bf16, bf16><<<dim3((unsigned)((M + kWChunk - 1) / kWChunk), sh.H, sh.d_h / kWRows), 256, 0, st>>>(
-        a, g.dw_uk, g.dw_uv);
+    bf16* dqtl = (bf16*)(ws + l.dqtl);
+    k_bwd_own<<<dim3(T_len, sh.B), threads, 0, st>>>(a, (const bf16*)(ws + l.qt), (const bf16*)(ws + l.fwd), dob,
+                                                      in.lse, in.delta, dqtl, g.dq_r);
+    if ((e = cudaGetLastError()) != cudaSuccess) return note_error("k_bwd_own launch", e);
+    // dqC = dqt[0:d_c] . W_UK[h]^T on the tensor cores, fp32 out
+    e = gemm_batched(GemmOperand{dqtl, sh.H * sh.d_c, (size_t)sh.d_c},
+                     GemmOperand{pa.w_uk, sh.d_c, (size_t)sh.d_h * sh.d_c}, g.dq_c, sh.H * sh.d_h, (size_t)sh.d_h,
+                     true, M, sh.d_h, sh.d_c, sh.H, pa.status, st, launches);
+    if (e != cudaSuccess) return e;
+    if ((e = weight_grads<bf16, bf16, bf16>(a, dqtl, sh.d_c, (float*)(ws + l.part_k), (float*)(ws + l.part_v),
+                                            g.dw_uk, g.dw_uv, st)) != cudaSuccess)
+        return note_error("backward weight-gradient launch", e);
     k_bwd_scan<bf16><<<dim3((n_slots + 7) / 8, sh.B), 256, 0, st>>>(a, pa.c, pa.kr, pa.gate_w, g.dc, g.dkr,
                                                                     g.dgate_w, g.dgate_b, g.dgate_in);
-    *launches += 5;
+    *launches += 6;
     return note_error("backward launch", cudaGetLastError());
 }
 

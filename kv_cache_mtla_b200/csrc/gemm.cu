@@ -14,7 +14,9 @@
 //              each, while the MMAs of the next tile run into the other of
 //              two TMEM accumulators
 // Rows of x past M, rows of W past N and columns past K read as zero; the
-// epilogue writes only inside [M, N).
+// epilogue writes only inside [M, N). A batch of such products (the heads of
+// a per-head projection) runs as one launch: x and W are 3-D tensor maps with
+// the batch index as one coordinate, and y advances by a batch stride.
 #include <cudaTypedefs.h>
 
 #include <algorithm>
@@ -35,10 +37,20 @@ constexpr int kGemmThreads = 192;
 
 struct GemmArgs {
     int M, N, K, ldc;
-    int tiles_n, n_tiles;
-    bf16* y;
+    int tiles_n, tiles_mn, n_tiles;
+    int x_batch_dim, w_batch_dim;   // which tensor-map coordinate (1 or 2) is the batch index
+    size_t y_batch;                 // elements between the batch's outputs
+    int out_f32;                    // y is float (else bf16)
+    void* y;
     int* status;
 };
+
+// coordinates (k, rows, batch) in the map's dimension order
+__device__ __forceinline__ void gemm_load(void* dst, const CUtensorMap* m, uint64_t* bar, int k, int row, int bt,
+                                          int batch_dim) {
+    if (batch_dim == 1) tma_load_3d(dst, m, bar, k, bt, row);
+    else tma_load_3d(dst, m, bar, k, row, bt);
+}
 
 template <int BN>
 struct GemmCfg {
@@ -98,14 +110,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (lane == 0) {
             int it = 0;
             for (int t = blockIdx.x; t < g.n_tiles && !*fail; t += gridDim.x) {
-                const int m0 = (t / g.tiles_n) * kBM, n0 = (t % g.tiles_n) * BN;
+                const int bt = t / g.tiles_mn, tr = t % g.tiles_mn;
+                const int m0 = (tr / g.tiles_n) * kBM, n0 = (tr % g.tiles_n) * BN;
                 for (int kb = 0; kb < kb_n; ++kb, ++it) {
                     const int st = it % S;
                     if (it >= S && !wait(&empty[st], ((it / S) - 1) & 1)) break;
                     uint8_t* dst = smem + (size_t)st * C::stage_bytes;
                     mbar_arrive_expect_tx(&full[st], C::stage_bytes);
-                    tma_load_2d(dst, &map_x, &full[st], kb * kBK, m0);
-                    tma_load_2d(dst + C::a_bytes, &map_w, &full[st], kb * kBK, n0);
+                    gemm_load(dst, &map_x, &full[st], kb * kBK, m0, bt, g.x_batch_dim);
+                    gemm_load(dst + C::a_bytes, &map_w, &full[st], kb * kBK, n0, bt, g.w_batch_dim);
                 }
             }
             if (*fail)
@@ -150,16 +163,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const int a = i & 1;
             const bool ok = wait(&acc_full[a], (i >> 1) & 1);
             tc_fence_after();
-            const int m0 = (t / g.tiles_n) * kBM, n0 = (t % g.tiles_n) * BN;
+            const int bt = t / g.tiles_mn, tr = t % g.tiles_mn;
+            const int m0 = (tr / g.tiles_n) * kBM, n0 = (tr % g.tiles_n) * BN;
             const int row = m0 + q * 32 + lane;
 #pragma unroll 1
             for (int c0 = 0; c0 < BN; c0 += 32) {
                 float v[32];
                 tmem_ld32(tmem + a * BN + c0 + lane_off, v);
                 tmem_wait_ld();
-                if (ok && row < g.M) {
-                    bf16* dst = g.y + (size_t)row * g.ldc + n0 + c0;
-                    const int nvalid = g.N - (n0 + c0);
+                const int nvalid = g.N - (n0 + c0);
+                const size_t off = (size_t)bt * g.y_batch + (size_t)row * g.ldc + n0 + c0;
+                if (ok && row < g.M && g.out_f32) {
+                    float* dst = (float*)g.y + off;
+                    if (nvalid >= 32 && ((((uintptr_t)dst) & 15) == 0)) {
+#pragma unroll
+                        for (int u = 0; u < 8; ++u)
+                            *(float4*)(dst + 4 * u) = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+                    } else {
+                        for (int cc = 0; cc < 32 && cc < nvalid; ++cc) dst[cc] = v[cc];
+                    }
+                } else if (ok && row < g.M) {
+                    bf16* dst = (bf16*)g.y + off;
                     if (nvalid >= 32 && ((((uintptr_t)dst) & 15) == 0)) {
 #pragma unroll
                         for (int u = 0; u < 4; ++u)
@@ -205,45 +229,68 @@ cudaError_t gemm_launch(const CUtensorMap& mx, const CUtensorMap& mw, const Gemm
 
 }  // namespace
 
-cudaError_t gemm_bf16(const void* x, int ldx, const void* w, int ldw, void* y, int ldy, int M, int N, int K,
-                      int* status, cudaStream_t st, uint64_t* launches) {
+cudaError_t gemm_batched(const GemmOperand& x, const GemmOperand& w, void* y, int ldy, size_t y_batch, bool y_f32,
+                         int M, int N, int K, int batch, int* status, cudaStream_t st, uint64_t* launches) {
     auto encode = (PFN_cuTensorMapEncodeTiled_v12000)tensor_map_encoder();
     if (!encode) return note_error("cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", cudaErrorNotSupported);
     const int BN = N <= 64 ? 64 : (N <= 128 ? 128 : 256);
-    CUtensorMap mx, mw;
-    {
-        cuuint64_t d[2] = {(cuuint64_t)K, (cuuint64_t)M};
-        cuuint64_t s[1] = {(cuuint64_t)ldx * 2};
-        cuuint32_t b[2] = {kBK, kBM};
-        cuuint32_t e[2] = {1, 1};
-        CUresult r = encode(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(x), d, s, b, e,
+    // 3-D map of one operand: (K, rows, batch) when the batch stride exceeds the
+    // row pitch, else (K, batch, rows), so that the strides grow with the dimension
+    auto make = [&](CUtensorMap* m, const GemmOperand& o, int rows, int box_rows, int* batch_dim,
+                    const char* what) -> cudaError_t {
+        const bool rows_first = o.batch_stride >= (size_t)o.ld * rows || batch == 1;
+        *batch_dim = rows_first ? 2 : 1;
+        cuuint64_t d[3], s[2];
+        d[0] = (cuuint64_t)K;
+        if (rows_first) {
+            d[1] = (cuuint64_t)rows;
+            d[2] = (cuuint64_t)batch;
+            s[0] = (cuuint64_t)o.ld * 2;
+            s[1] = (cuuint64_t)(batch == 1 ? (size_t)o.ld * rows : o.batch_stride) * 2;
+        } else {
+            d[1] = (cuuint64_t)batch;
+            d[2] = (cuuint64_t)rows;
+            s[0] = (cuuint64_t)o.batch_stride * 2;
+            s[1] = (cuuint64_t)o.ld * 2;
+        }
+        const cuuint32_t bx[3] = {kBK, rows_first ? (cuuint32_t)box_rows : 1u, rows_first ? 1u : (cuuint32_t)box_rows};
+        const cuuint32_t e[3] = {1, 1, 1};
+        CUresult r = encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(o.p), d, s, bx, e,
                             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-        if (r != CUDA_SUCCESS) return note_error("cuTensorMapEncodeTiled (gemm x)", cudaErrorInvalidValue);
-    }
-    {
-        cuuint64_t d[2] = {(cuuint64_t)K, (cuuint64_t)N};
-        cuuint64_t s[1] = {(cuuint64_t)ldw * 2};
-        cuuint32_t b[2] = {kBK, (cuuint32_t)BN};
-        cuuint32_t e[2] = {1, 1};
-        CUresult r = encode(&mw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(w), d, s, b, e,
-                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-        if (r != CUDA_SUCCESS) return note_error("cuTensorMapEncodeTiled (gemm w)", cudaErrorInvalidValue);
-    }
+        if (r != CUDA_SUCCESS) {
+            char buf[96];
+            snprintf(buf, sizeof(buf), "cuTensorMapEncodeTiled (gemm %s, CUresult %d)", what, (int)r);
+            return note_error(buf, cudaErrorInvalidValue);
+        }
+        return cudaSuccess;
+    };
     GemmArgs g;
+    CUtensorMap mx, mw;
+    cudaError_t e = make(&mx, x, M, kBM, &g.x_batch_dim, "x");
+    if (e == cudaSuccess) e = make(&mw, w, N, BN, &g.w_batch_dim, "w");
+    if (e != cudaSuccess) return e;
     g.M = M;
     g.N = N;
     g.K = K;
     g.ldc = ldy;
     g.tiles_n = (N + BN - 1) / BN;
-    g.n_tiles = ((M + kBM - 1) / kBM) * g.tiles_n;
-    g.y = (bf16*)y;
+    g.tiles_mn = ((M + kBM - 1) / kBM) * g.tiles_n;
+    g.n_tiles = g.tiles_mn * batch;
+    g.y_batch = y_batch;
+    g.out_f32 = y_f32 ? 1 : 0;
+    g.y = y;
     g.status = status;
     *launches += 1;
     if (BN == 64) return gemm_launch<64>(mx, mw, g, st);
     if (BN == 128) return gemm_launch<128>(mx, mw, g, st);
     return gemm_launch<256>(mx, mw, g, st);
+}
+
+cudaError_t gemm_bf16(const void* x, int ldx, const void* w, int ldw, void* y, int ldy, int M, int N, int K,
+                      int* status, cudaStream_t st, uint64_t* launches) {
+    return gemm_batched(GemmOperand{x, ldx, 0}, GemmOperand{w, ldw, 0}, y, ldy, 0, false, M, N, K, 1, status, st,
+                        launches);
 }
 
 }  // namespace mtla

@@ -149,6 +149,18 @@ size_t prefill_backward_workspace(const Shape& sh, int T, size_t elem_bytes);
 cudaError_t prefill_backward(const PrefillArgs& a, const BackwardGrads& g, bool fp32, cudaStream_t st,
                              uint64_t* launches);
 
+// A batch of such products in one launch (gemm.cu): product i reads
+// x.p + i * x.batch_stride and w.p + i * w.batch_stride (elements; rows ld
+// apart, ld and batch_stride multiples of 8) and writes y + i * y_batch
+// (bf16, or float when y_f32).
+struct GemmOperand {
+    const void* p;
+    int ld;
+    size_t batch_stride;
+};
+cudaError_t gemm_batched(const GemmOperand& x, const GemmOperand& w, void* y, int ldy, size_t y_batch, bool y_f32,
+                         int M, int N, int K, int batch, int* status, cudaStream_t st, uint64_t* launches);
+
 // Test hook (wait_probe.cu): one CTA whose bounded wait runs out after
 // limit_ns; `scratch` is 2 KB of device memory its TMA load reads.
 cudaError_t wait_probe(uint64_t limit_ns, void* scratch, int* status, cudaStream_t st, uint64_t* launches);
