@@ -32,6 +32,8 @@
 //   k_bwd_query       dqC, dqR
 //   k_bwd_wpart/wsum  dW_UK, dW_UV (per row chunk, then the chunks in order)
 //   k_bwd_scan        a warp per slot: the scan and gate backward
+#include <type_traits>
+
 #include "common.cuh"
 #include "mtla_internal.h"
 #include "prep.cuh"
@@ -42,7 +44,6 @@ namespace {
 
 constexpr int kMaxD = 576;             // slot width the kernels hold (d_c + d_R)
 constexpr int kPer = kMaxD / 32;       // a lane's channels: lane + 32 k
-constexpr int kWR = 32;                // dW rows r per block of k_bwd_wpart
 constexpr int kWChunk = 1024;          // token rows per block of k_bwd_wpart
 
 struct BwdArgs {
@@ -252,56 +253,133 @@ __global__ void __launch_bounds__(256) k_bwd_query(BwdArgs a, float* dqc, float*
 }
 
 // Weight gradients in two deterministic stages. k_bwd_wpart: block (row chunk,
-// h, group of 32 r), a thread per channel c: over the chunk's token rows m,
-//   partK[chunk][h][r][c] = sum_m qC[m,h,r] g[m,h,c],  g = dqt[0:d_c]
-//   partV[chunk][h][r][c] = sum_m dout[m,h,r] obar[m,h,c]
-// (g and obar rows g_pitch / d_c elements apart, of type GT / OT); then
-// k_bwd_wsum adds the chunks in order: dW_UK = sum partK, dW_UV = sum partV.
+// h, output tile), the tile a [64 r x 256 c] block of
+//   partK[chunk][h][r][c] = sum_m qC[m,h,r] g[m,h,c],  g = dqt[0:d_c]    (z even)
+//   partV[chunk][h][r][c] = sum_m dout[m,h,r] obar[m,h,c]                 (z odd)
+// over the chunk's token rows m (g and obar rows g_pitch / d_c elements
+// apart, of type GT / OT). Rows are staged 32 at a time in shared memory as
+// fp32; each thread keeps an 8 r x 8 c register tile (64 FMAs per row against
+// four 16-byte shared loads). Then k_bwd_wsum adds the chunks in order.
 template <typename T, typename GT, typename OT>
 __global__ void __launch_bounds__(256) k_bwd_wpart(BwdArgs a, const void* g, int g_pitch, float* part_k,
                                                    float* part_v) {
     const Shape sh = a.sh;
-    const int chunk = blockIdx.x, h = blockIdx.y, r0 = blockIdx.z * kWR, tid = threadIdx.x;
+    const int chunk = blockIdx.x, h = blockIdx.y, tid = threadIdx.x;
+    const bool uv = blockIdx.z & 1;
+    const int n_ct = (sh.d_c + 255) / 256;
+    const int r0 = (int)(blockIdx.z >> 1) / n_ct * 64, c0 = (int)(blockIdx.z >> 1) % n_ct * 256;
     const int64_t M = (int64_t)sh.B * a.T;
     const int64_t m0 = (int64_t)chunk * kWChunk, m1 = m0 + kWChunk < M ? m0 + kWChunk : M;
-    __shared__ float qs[32][kWR], os[32][kWR];
-    for (int c0 = 0; c0 < sh.d_c; c0 += 256) {
-        const int c = c0 + tid;
-        float gk[kWR], gv[kWR];
+    const void* asrc = uv ? a.dout : a.qc;
+    const void* bsrc = uv ? (const void*)a.obar : g;
+    const int bpitch = uv ? sh.d_c : g_pitch;
+    __shared__ __align__(16) float As[32][64];
+    __shared__ __align__(16) float Bs[32][256];
+    const int tr = tid >> 5, tc = tid & 31;          // r = r0 + 8 tr + i, c = c0 + 8 tc + j
+    float acc[8][8];
 #pragma unroll
-        for (int r = 0; r < kWR; ++r) gk[r] = gv[r] = 0.f;
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+    constexpr bool kVec = std::is_same<T, bf16>::value && std::is_same<GT, bf16>::value &&
+                          std::is_same<OT, bf16>::value;
+    if constexpr (kVec) {
+        // bf16 operands: 16-byte loads (8 values), the next 32-row stage fetched
+        // into registers while this one is multiplied
+        const bf16* A = (const bf16*)asrc;
+        const bf16* Bm = (const bf16*)bsrc;
+        uint4 ra, rb[4];
+        auto fetch = [&](int64_t mb) {
+            {
+                const int mm = tid >> 3, rr = (tid & 7) * 8;       // 32 rows x 8 groups of 8 r
+                const int64_t m = mb + mm;
+                ra = (m < m1 && r0 + rr < sh.d_h) ? *(const uint4*)(A + ((size_t)m * sh.H + h) * sh.d_h + r0 + rr)
+                                                  : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int q = tid + 256 * k, mm = q >> 5, cc = (q & 31) * 8;   // 32 rows x 32 groups of 8 c
+                const int64_t m = mb + mm;
+                rb[k] = (m < m1 && c0 + cc < sh.d_c) ? *(const uint4*)(Bm + ((size_t)m * sh.H + h) * bpitch + c0 + cc)
+                                                     : make_uint4(0, 0, 0, 0);
+            }
+        };
+        auto put = [&]() {
+            float v[8];
+            const bf16* e = (const bf16*)&ra;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v[u] = __bfloat162float(e[u]);
+            *(float4*)&As[tid >> 3][(tid & 7) * 8] = make_float4(v[0], v[1], v[2], v[3]);
+            *(float4*)&As[tid >> 3][(tid & 7) * 8 + 4] = make_float4(v[4], v[5], v[6], v[7]);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int q = tid + 256 * k;
+                const bf16* f = (const bf16*)&rb[k];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) v[u] = __bfloat162float(f[u]);
+                *(float4*)&Bs[q >> 5][(q & 31) * 8] = make_float4(v[0], v[1], v[2], v[3]);
+                *(float4*)&Bs[q >> 5][(q & 31) * 8 + 4] = make_float4(v[4], v[5], v[6], v[7]);
+            }
+        };
+        if (m0 < m1) fetch(m0);
         for (int64_t mb = m0; mb < m1; mb += 32) {
             __syncthreads();
-            for (int q = tid; q < 32 * kWR; q += blockDim.x) {
-                const int mm = q / kWR, rr = q % kWR;
-                const int64_t m = mb + mm;
-                const bool ok = m < m1 && r0 + rr < sh.d_h;
-                const size_t row = (size_t)m * sh.H + h;
-                qs[mm][rr] = ok ? ldf<T>(a.qc, row * sh.d_h + r0 + rr) : 0.f;
-                os[mm][rr] = ok ? ldf<T>(a.dout, row * sh.d_h + r0 + rr) : 0.f;
-            }
+            put();
             __syncthreads();
-            if (c < sh.d_c) {
-                const int nm = (int)(m1 - mb < 32 ? m1 - mb : 32);
-                for (int mm = 0; mm < nm; ++mm) {
-                    const size_t row = (size_t)(mb + mm) * sh.H + h;
-                    const float x = ldf<GT>(g, row * g_pitch + c), y = ldf<OT>(a.obar, row * sh.d_c + c);
+            if (mb + 32 < m1) fetch(mb + 32);
+            const int nm = (int)(m1 - mb < 32 ? m1 - mb : 32);
+            for (int mm = 0; mm < nm; ++mm) {
+                const float4 a0 = *(const float4*)&As[mm][8 * tr], a1 = *(const float4*)&As[mm][8 * tr + 4];
+                const float4 b0 = *(const float4*)&Bs[mm][8 * tc], b1 = *(const float4*)&Bs[mm][8 * tc + 4];
+                const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+                const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-                    for (int r = 0; r < kWR; ++r) {
-                        gk[r] = fmaf(qs[mm][r], x, gk[r]);
-                        gv[r] = fmaf(os[mm][r], y, gv[r]);
-                    }
-                }
+                for (int i = 0; i < 8; ++i)
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
             }
         }
-        if (c < sh.d_c)
+    } else
+    for (int64_t mb = m0; mb < m1; mb += 32) {
+        __syncthreads();
+        for (int q = tid; q < 32 * 64; q += 256) {
+            const int mm = q >> 6, rr = q & 63;
+            const int64_t m = mb + mm;
+            As[mm][rr] = (m < m1 && r0 + rr < sh.d_h) ? ldf<T>(asrc, ((size_t)m * sh.H + h) * sh.d_h + r0 + rr) : 0.f;
+        }
+        for (int q = tid; q < 32 * 256; q += 256) {
+            const int mm = q >> 8, cc = q & 255;
+            const int64_t m = mb + mm;
+            float v = 0.f;
+            if (m < m1 && c0 + cc < sh.d_c) {
+                const size_t o = ((size_t)m * sh.H + h) * bpitch + c0 + cc;
+                v = uv ? ldf<OT>(bsrc, o) : ldf<GT>(bsrc, o);
+            }
+            Bs[mm][cc] = v;
+        }
+        __syncthreads();
+        const int nm = (int)(m1 - mb < 32 ? m1 - mb : 32);
+        for (int mm = 0; mm < nm; ++mm) {
+            const float4 a0 = *(const float4*)&As[mm][8 * tr], a1 = *(const float4*)&As[mm][8 * tr + 4];
+            const float4 b0 = *(const float4*)&Bs[mm][8 * tc], b1 = *(const float4*)&Bs[mm][8 * tc + 4];
+            const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-            for (int r = 0; r < kWR; ++r)
-                if (r0 + r < sh.d_h) {
-                    const size_t o = (((size_t)chunk * sh.H + h) * sh.d_h + r0 + r) * sh.d_c + c;
-                    part_k[o] = gk[r];
-                    part_v[o] = gv[r];
-                }
+            for (int i = 0; i < 8; ++i)
+#pragma unroll
+                for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+        }
+    }
+    float* part = uv ? part_v : part_k;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int r = r0 + 8 * tr + i;
+        if (r >= sh.d_h) continue;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int c = c0 + 8 * tc + j;
+            if (c < sh.d_c) part[(((size_t)chunk * sh.H + h) * sh.d_h + r) * sh.d_c + c] = acc[i][j];
+        }
     }
 }
 
@@ -446,57 +524,71 @@ __global__ void __launch_bounds__(256) k_bwd_delta(Shape sh, int T, const bf16* 
 // key gradients, summed in a fixed order. Block (i, b), a warp per head, 8
 // channels a lane (16-byte loads).
 constexpr int kOwnGroups = 2;          // 8-channel groups a lane takes: D <= 512 (the tensor-core widths)
-__global__ void __launch_bounds__(256, 2) k_bwd_own(BwdArgs a, const bf16* qt, const bf16* P, const bf16* dob,
-                                                 const float* lse, const float* delta, bf16* dqtl, float* dq_r) {
+__device__ __forceinline__ float bf_at(const uint4& r, int u) { return __bfloat162float(((const bf16*)&r)[u]); }
+__global__ void __launch_bounds__(256) k_bwd_own(BwdArgs a, const bf16* qt, const bf16* P, const bf16* dob,
+                                                    const float* lse, const float* delta, bf16* dqtl, float* dq_r) {
     const Shape sh = a.sh;
     const int i = blockIdx.x, b = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
     const int D = sh.D, d_c = sh.d_c;
     const float scale_log2 = sh.scale * 1.4426950408889634f;
     __shared__ float dkey_own[8][kMaxD];
+    __shared__ float2 rcs[kMaxD / 2];               // (sin, cos) of position i's RoPE pairs
     float* own = dkey_own[warp];
     for (int q = lane; q < D; q += 32) own[q] = 0.f;
+    for (int kp = threadIdx.x; kp < sh.d_r / 2; kp += blockDim.x) {
+        float sn, cs;
+        pair_sincos(i, kp, sh.d_r, sh.log2_rope_base, &sn, &cs);
+        rcs[kp] = make_float2(sn, cs);
+    }
+    __syncthreads();
     const bf16* Pi = P + ((size_t)b * a.T + i) * D;
-    float pv[kOwnGroups][8];
+    const uint4 z4 = make_uint4(0, 0, 0, 0);
+    uint4 pr4[kOwnGroups];                          // P_i, 8 bf16 a group, kept packed
 #pragma unroll
     for (int k = 0; k < kOwnGroups; ++k) {
         const int c0 = 8 * (lane + 32 * k);
-        if (c0 < D) load8<bf16>(Pi + c0, pv[k]);
-        else
-#pragma unroll
-            for (int u = 0; u < 8; ++u) pv[k][u] = 0.f;
+        pr4[k] = c0 < D ? *(const uint4*)(Pi + c0) : z4;
     }
     for (int h = warp; h < sh.H; h += nw) {
         const size_t row = ((size_t)b * a.T + i) * sh.H + h;
         const size_t srow = ((size_t)b * sh.H + h) * stats_pitch(a.T) + i;
-        float qv[kOwnGroups][8], dv[kOwnGroups][8], e = 0.f, da = 0.f;
+        // every load of the row first (their latencies overlap), then the sums
+        uint4 q4[kOwnGroups], d4[kOwnGroups];
+        float gv[kOwnGroups][8];
 #pragma unroll
         for (int k = 0; k < kOwnGroups; ++k) {
             const int c0 = 8 * (lane + 32 * k);
+            q4[k] = c0 < D ? *(const uint4*)(qt + row * D + c0) : z4;
+            d4[k] = c0 < d_c ? *(const uint4*)(dob + row * d_c + c0) : z4;
+            if (c0 < D) load8<float>(a.dqt + row * D + c0, gv[k]);
+            else
 #pragma unroll
-            for (int u = 0; u < 8; ++u) qv[k][u] = dv[k][u] = 0.f;
-            if (c0 < D) load8<bf16>(qt + row * D + c0, qv[k]);
-            if (c0 < d_c) load8<bf16>(dob + row * d_c + c0, dv[k]);
+                for (int u = 0; u < 8; ++u) gv[k][u] = 0.f;
+        }
+        const float lse_r = lse[srow], delta_r = delta[srow];
+        float e = 0.f, da = 0.f;
+#pragma unroll
+        for (int k = 0; k < kOwnGroups; ++k)
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                e = fmaf(qv[k][u], pv[k][u], e);
-                da = fmaf(dv[k][u], pv[k][u], da);
+                const float pu = bf_at(pr4[k], u);
+                e = fmaf(bf_at(q4[k], u), pu, e);
+                da = fmaf(bf_at(d4[k], u), pu, da);
             }
-        }
         e = warp_sum(e);
         da = warp_sum(da);
-        const float pr = exp2f(fmaf(e, scale_log2, -lse[srow]));
-        const float sde = sh.scale * pr * (da - delta[srow]);
+        const float pr = exp2f(fmaf(e, scale_log2, -lse_r));
+        const float sde = sh.scale * pr * (da - delta_r);
 #pragma unroll
         for (int k = 0; k < kOwnGroups; ++k) {
             const int c0 = 8 * (lane + 32 * k);
             if (c0 >= D) continue;
-            float g[8];
-            load8<float>(a.dqt + row * D + c0, g);
+            float* g = gv[k];
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                g[u] = fmaf(sde, pv[k][u], g[u]);
-                own[c0 + u] += fmaf(sde, qv[k][u], pr * dv[k][u]);
+                g[u] = fmaf(sde, bf_at(pr4[k], u), g[u]);
+                own[c0 + u] += fmaf(sde, bf_at(q4[k], u), pr * bf_at(d4[k], u));
             }
             if (c0 < d_c) {
                 store8<bf16>(dqtl + row * d_c + c0, g);
@@ -504,8 +596,7 @@ __global__ void __launch_bounds__(256, 2) k_bwd_own(BwdArgs a, const bf16* qt, c
 #pragma unroll
                 for (int u = 0; u < 8; u += 2) {
                     const int kp = (c0 - d_c + u) / 2;        // RoPE pair
-                    float sn, cs;
-                    pair_sincos(i, kp, sh.d_r, sh.log2_rope_base, &sn, &cs);
+                    const float sn = rcs[kp].x, cs = rcs[kp].y;
                     dq_r[row * sh.d_r + 2 * kp] = fmaf(g[u], cs, g[u + 1] * sn);        // R_i^T
                     dq_r[row * sh.d_r + 2 * kp + 1] = fmaf(-g[u], sn, g[u + 1] * cs);
                 }
@@ -535,7 +626,8 @@ cudaError_t weight_grads(const BwdArgs& a, const void* g, int g_pitch, float* pa
                          float* dw_uv, cudaStream_t st) {
     const Shape& sh = a.sh;
     const int nc = weight_chunks(sh, a.T);
-    k_bwd_wpart<T, GT, OT><<<dim3(nc, sh.H, (sh.d_h + kWR - 1) / kWR), 256, 0, st>>>(a, g, g_pitch, part_k, part_v);
+    const int tiles = ((sh.d_h + 63) / 64) * ((sh.d_c + 255) / 256);
+    k_bwd_wpart<T, GT, OT><<<dim3(nc, sh.H, 2 * tiles), 256, 0, st>>>(a, g, g_pitch, part_k, part_v);
     const size_t n = (size_t)sh.H * sh.d_h * sh.d_c;
     k_bwd_wsum<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(nc, n, part_k, part_v, dw_uk, dw_uv);
     return cudaGetLastError();
