@@ -39,9 +39,11 @@
  *     caller owns them. Every pointer must be 16-byte aligned.
  *   - Storage type: MTLA_BF16 stores activations, weights, cache and output in
  *     bfloat16 (round-to-nearest-even) and computes in fp32; MTLA_FP32 stores
- *     and computes everything in fp32 (no tensor-float rounding anywhere).
+ *     and computes everything in fp32 (no tensor-float rounding anywhere);
+ *     MTLA_FP16 stores them in IEEE half precision (round-to-nearest-even) and
+ *     computes in fp32 on the CUDA cores (the tensor-core kernels take bf16).
  *     Gate parameters, supplied gates and the open-slot accumulator are
- *     always float32.
+ *     always float32. mtla_linear and the layer calls are bf16 only.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy
  *     default stream) and allocate nothing: scratch comes from `workspace`,
  *     whose size mtla_workspace_size() reports.
@@ -83,7 +85,7 @@ typedef enum {
     MTLA_ERR_WORKSPACE = 6      /* workspace smaller than mtla_workspace_size()   */
 } mtla_status;
 
-typedef enum { MTLA_BF16 = 0, MTLA_FP32 = 1 } mtla_dtype;
+typedef enum { MTLA_BF16 = 0, MTLA_FP32 = 1, MTLA_FP16 = 2 } mtla_dtype;
 
 /* Merging weights (MTLA Sec. 4.1, Eq. 13; the reading of W_t (.) x_t):
  * one scalar per token that scales its whole slot vector x_t = [c_t ; RoPE_t(k_t)]

@@ -754,8 +754,8 @@ BwdTcWs bwd_tc_layout(const Shape& sh_in, int T) {
     return l;
 }
 
-bool use_tc(const Shape& sh, bool fp32) {
-    return !fp32 && tc_backward_supported(sh) && tc_prefill_supported(sh);
+bool use_tc(const Shape& sh, int dtype) {
+    return dtype == kDtypeBF16 && tc_backward_supported(sh) && tc_prefill_supported(sh);
 }
 
 // bf16 at the tensor-core prefill's widths: the forward recomputed on the
@@ -856,14 +856,16 @@ cudaError_t backward_tc(const PrefillArgs& pa_in, const BackwardGrads& g, cudaSt
 
 }  // namespace
 
-size_t prefill_backward_workspace(const Shape& sh, int T, size_t elem_bytes) {
-    return use_tc(sh, elem_bytes == 4) ? bwd_tc_layout(sh, T).total : bwd_layout(sh, T, elem_bytes).total;
+size_t prefill_backward_workspace(const Shape& sh, int T, int dtype) {
+    return use_tc(sh, dtype) ? bwd_tc_layout(sh, T).total : bwd_layout(sh, T, dtype_bytes(dtype)).total;
 }
 
-cudaError_t prefill_backward(const PrefillArgs& a, const BackwardGrads& g, bool fp32, cudaStream_t st,
+cudaError_t prefill_backward(const PrefillArgs& a, const BackwardGrads& g, int dtype, cudaStream_t st,
                              uint64_t* launches) {
-    if (use_tc(a.sh, fp32)) return backward_tc(a, g, st, launches);
-    return fp32 ? backward_impl<float>(a, g, st, launches) : backward_impl<bf16>(a, g, st, launches);
+    if (use_tc(a.sh, dtype)) return backward_tc(a, g, st, launches);
+    if (dtype == kDtypeF32) return backward_impl<float>(a, g, st, launches);
+    if (dtype == kDtypeF16) return backward_impl<f16>(a, g, st, launches);
+    return backward_impl<bf16>(a, g, st, launches);
 }
 
 }  // namespace mtla

@@ -93,7 +93,7 @@ static mtla_status check_config(const mtla_config* cfg, Shape* sh) {
     if (cfg->batch <= 0 || cfg->heads <= 0 || cfg->d_h <= 0 || cfg->d_c <= 0 || cfg->d_r <= 0 ||
         cfg->stride <= 0 || cfg->max_slots <= 0)
         return MTLA_ERR_INVALID_ARG;
-    if (cfg->dtype != MTLA_BF16 && cfg->dtype != MTLA_FP32) return MTLA_ERR_INVALID_ARG;
+    if (cfg->dtype != MTLA_BF16 && cfg->dtype != MTLA_FP32 && cfg->dtype != MTLA_FP16) return MTLA_ERR_INVALID_ARG;
     if (cfg->gate_mode < MTLA_GATE_COMPUTED || cfg->gate_mode > MTLA_GATE_CHANNEL_SUPPLIED)
         return MTLA_ERR_INVALID_ARG;
     if (!(cfg->softmax_scale >= 0.f) || !std::isfinite(cfg->softmax_scale)) return MTLA_ERR_INVALID_ARG;
@@ -223,7 +223,7 @@ mtla_status mtla_decode_step(const mtla_config* cfg, const void* c_new, const vo
     uint64_t n = 0;
     cudaError_t e = use_tc_decode(cfg, sh)      ? tc_decode(a, (cudaStream_t)stream, &n)
                     : use_tc_decode_lh(cfg, sh) ? tc_decode_lh(a, (cudaStream_t)stream, &n)
-                                                : simt_decode(a, cfg->dtype == MTLA_FP32, (cudaStream_t)stream, &n);
+                                                : simt_decode(a, cfg->dtype, (cudaStream_t)stream, &n);
     g_launches += n;
     if (e != cudaSuccess && !g_error_detail[0]) note_error("decode launch", e);
     return e == cudaSuccess ? MTLA_OK : MTLA_ERR_CUDA;
@@ -270,7 +270,7 @@ static mtla_status prefill_common(const mtla_config* cfg, int32_t t0, int32_t T,
     if (note_error("device status word", status_ptr(&a.status)) != cudaSuccess) return MTLA_ERR_CUDA;
     uint64_t n = 0;
     cudaError_t e = use_tc_prefill(cfg, sh) ? tc_prefill(a, (cudaStream_t)stream, &n)
-                                            : simt_prefill(a, cfg->dtype == MTLA_FP32, (cudaStream_t)stream, &n);
+                                            : simt_prefill(a, cfg->dtype, (cudaStream_t)stream, &n);
     g_launches += n;
     if (e != cudaSuccess && !g_error_detail[0]) note_error("prefill launch", e);
     return e == cudaSuccess ? MTLA_OK : MTLA_ERR_CUDA;
@@ -309,7 +309,7 @@ mtla_status mtla_prefill_backward_workspace_size(const mtla_config* cfg, int32_t
     if (!bytes) return MTLA_ERR_INVALID_ARG;
     mtla_status st = backward_check(cfg, T, &sh);
     if (st != MTLA_OK) return st;
-    *bytes = prefill_backward_workspace(sh, T, cfg->dtype == MTLA_FP32 ? 4 : 2);
+    *bytes = prefill_backward_workspace(sh, T, cfg->dtype);
     return MTLA_OK;
 }
 
@@ -331,7 +331,7 @@ mtla_status mtla_prefill_backward(const mtla_config* cfg, int32_t T, const void*
         (!dgate_w || !dgate_b || !aligned16(dgate_w) || !aligned16(dgate_b)))
         return MTLA_ERR_INVALID_ARG;
     if (cfg->gate_mode == MTLA_GATE_SUPPLIED && (!dgate_in || !aligned16(dgate_in))) return MTLA_ERR_INVALID_ARG;
-    if (workspace_bytes < prefill_backward_workspace(sh, T, cfg->dtype == MTLA_FP32 ? 4 : 2))
+    if (workspace_bytes < prefill_backward_workspace(sh, T, cfg->dtype))
         return MTLA_ERR_WORKSPACE;
     PrefillArgs a = {};
     a.sh = sh;
@@ -351,7 +351,7 @@ mtla_status mtla_prefill_backward(const mtla_config* cfg, int32_t T, const void*
     g_error_detail[0] = 0;
     if (note_error("device status word", status_ptr(&a.status)) != cudaSuccess) return MTLA_ERR_CUDA;
     uint64_t n = 0;
-    cudaError_t e = prefill_backward(a, g, cfg->dtype == MTLA_FP32, (cudaStream_t)stream, &n);
+    cudaError_t e = prefill_backward(a, g, cfg->dtype, (cudaStream_t)stream, &n);
     g_launches += n;
     if (e != cudaSuccess && !g_error_detail[0]) note_error("backward launch", e);
     return e == cudaSuccess ? MTLA_OK : MTLA_ERR_CUDA;

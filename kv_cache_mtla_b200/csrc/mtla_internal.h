@@ -64,14 +64,18 @@ struct PrefillArgs {
 size_t prefill_seed_bytes(const Shape& sh);
 cudaError_t prefill_seed(PrefillArgs& a, void* seed_ws, cudaStream_t st);
 
+// Storage types (the values of mtla_dtype).
+constexpr int kDtypeBF16 = 0, kDtypeF32 = 1, kDtypeF16 = 2;
+inline size_t dtype_bytes(int dtype) { return dtype == kDtypeF32 ? 4 : 2; }
+
 // Scratch layouts (bytes), each region 256-byte aligned.
 size_t simt_decode_workspace(const Shape& sh);
 size_t simt_prefill_workspace(const Shape& sh, int T);
 
 // Launchers return cudaSuccess or the launch error; they add the number of
 // kernels they launched to *launches.
-cudaError_t simt_decode(const DecodeArgs& a, bool fp32, cudaStream_t st, uint64_t* launches);
-cudaError_t simt_prefill(const PrefillArgs& a, bool fp32, cudaStream_t st, uint64_t* launches);
+cudaError_t simt_decode(const DecodeArgs& a, int dtype, cudaStream_t st, uint64_t* launches);
+cudaError_t simt_prefill(const PrefillArgs& a, int dtype, cudaStream_t st, uint64_t* launches);
 
 // Tensor-core decode (bf16, heads <= 32): shapes it covers, its scratch, launcher.
 bool tc_decode_supported(const Shape& sh);
@@ -145,8 +149,8 @@ struct BackwardGrads {
     float* dgate_b;        // [s]
     float* dgate_in;       // [B,T] (supplied gate)
 };
-size_t prefill_backward_workspace(const Shape& sh, int T, size_t elem_bytes);
-cudaError_t prefill_backward(const PrefillArgs& a, const BackwardGrads& g, bool fp32, cudaStream_t st,
+size_t prefill_backward_workspace(const Shape& sh, int T, int dtype);
+cudaError_t prefill_backward(const PrefillArgs& a, const BackwardGrads& g, int dtype, cudaStream_t st,
                              uint64_t* launches);
 
 // A batch of such products in one launch (gemm.cu): product i reads

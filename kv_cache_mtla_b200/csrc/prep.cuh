@@ -282,7 +282,20 @@ template <> __device__ __forceinline__ void load8<bf16>(const bf16* p, float* v)
 #pragma unroll
     for (int i = 0; i < 8; ++i) v[i] = __bfloat162float(h[i]);
 }
+template <> __device__ __forceinline__ void load8<f16>(const f16* p, float* v) {
+    const uint4 raw = *(const uint4*)p;
+    const f16* h = (const f16*)&raw;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __half2float(h[i]);
+}
 template <typename T> __device__ __forceinline__ void store8(T* p, const float* v);
+template <> __device__ __forceinline__ void store8<f16>(f16* p, const float* v) {
+    uint4 raw;
+    f16* h = (f16*)&raw;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) h[i] = __float2half_rn(v[i]);
+    *(uint4*)p = raw;
+}
 template <> __device__ __forceinline__ void store8<float>(float* p, const float* v) {
     *(float4*)p = make_float4(v[0], v[1], v[2], v[3]);
     *(float4*)(p + 4) = make_float4(v[4], v[5], v[6], v[7]);

@@ -272,12 +272,16 @@ size_t simt_prefill_workspace(const Shape& sh, int T) {
            align256((size_t)sh.B * T * sh.H * sh.D * sizeof(float)) + prefill_seed_bytes(sh);
 }
 
-cudaError_t simt_decode(const DecodeArgs& a, bool fp32, cudaStream_t st, uint64_t* launches) {
-    return fp32 ? decode_impl<float>(a, st, launches) : decode_impl<bf16>(a, st, launches);
+cudaError_t simt_decode(const DecodeArgs& a, int dtype, cudaStream_t st, uint64_t* launches) {
+    if (dtype == kDtypeF32) return decode_impl<float>(a, st, launches);
+    if (dtype == kDtypeF16) return decode_impl<f16>(a, st, launches);
+    return decode_impl<bf16>(a, st, launches);
 }
 
-cudaError_t simt_prefill(const PrefillArgs& a, bool fp32, cudaStream_t st, uint64_t* launches) {
-    return fp32 ? prefill_impl<float>(a, st, launches) : prefill_impl<bf16>(a, st, launches);
+cudaError_t simt_prefill(const PrefillArgs& a, int dtype, cudaStream_t st, uint64_t* launches) {
+    if (dtype == kDtypeF32) return prefill_impl<float>(a, st, launches);
+    if (dtype == kDtypeF16) return prefill_impl<f16>(a, st, launches);
+    return prefill_impl<bf16>(a, st, launches);
 }
 
 }  // namespace mtla

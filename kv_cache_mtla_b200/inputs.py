@@ -6,8 +6,8 @@ benchmark and the smoke check feed the same draws to the CUDA library and to
 the CPU oracle.
 
 Values are drawn in float32 from a seeded CPU ``torch.Generator``. For bf16
-workloads every tensor the library receives in bf16 is rounded to bf16
-(round-to-nearest-even) here, so that ``.to(torch.bfloat16)`` is exact and
+(and fp16) workloads every tensor the library receives in that type is rounded
+to it (round-to-nearest-even) here, so that the conversion is exact and
 both sides see identical numbers. Gate parameters, supplied gates and the
 fp32 open-slot accumulator stay float32.
 """
@@ -31,7 +31,7 @@ class Workload:
     d_c: int
     d_r: int
     s: int
-    dtype: str               # "bf16" or "fp32" (storage of activations, weights, cache)
+    dtype: str               # "bf16", "fp16" or "fp32" (storage of activations, weights, cache)
     gate_mode: int = GATE_COMPUTED
     T: int = 0               # prefill length / prefix length
     steps: int = 0           # decode steps after the prefix
@@ -66,6 +66,8 @@ WORKLOADS = {w.name: w for w in (TINY_FP32, SPEECH_DECODE, STRIDE_SWEEP, PREFILL
 def _round(x: torch.Tensor, wl: Workload) -> torch.Tensor:
     if wl.dtype == "bf16":
         return x.to(torch.bfloat16).to(torch.float32)
+    if wl.dtype == "fp16":
+        return x.to(torch.float16).to(torch.float32)
     return x
 
 

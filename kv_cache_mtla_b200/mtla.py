@@ -17,7 +17,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmtla.so")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CAPACITY, ERR_CUDA, ERR_TIMEOUT, ERR_WORKSPACE = range(7)
-BF16, FP32 = 0, 1
+BF16, FP32, FP16 = 0, 1, 2
 GATE_COMPUTED, GATE_SUPPLIED, GATE_UNIT = 0, 1, 2
 GATE_CHANNEL_COMPUTED, GATE_CHANNEL_SUPPLIED = 3, 4
 
@@ -46,12 +46,13 @@ class Config(ctypes.Structure):
 
     @property
     def torch_dtype(self):
-        return torch.float32 if self.dtype == FP32 else torch.bfloat16
+        return {FP32: torch.float32, FP16: torch.float16}.get(self.dtype, torch.bfloat16)
 
 
 def make_config(B, H, d_h, d_c, d_r, s, max_slots, dtype="bf16", gate_mode=GATE_COMPUTED,
                 softmax_scale=0.0, rope_base=10000.0) -> Config:
-    dt = FP32 if dtype in ("fp32", FP32, torch.float32) else BF16
+    dt = (FP32 if dtype in ("fp32", FP32, torch.float32) else
+          FP16 if dtype in ("fp16", FP16, torch.float16) else BF16)
     return Config(B, H, d_h, d_c, d_r, s, dt, gate_mode, softmax_scale, rope_base, max_slots)
 
 

@@ -10,7 +10,10 @@ import torch
 import oracle
 from kv_cache_mtla_b200 import inputs, mtla
 
-TOL = {"bf16": 2e-2, "fp32": 1e-5}
+# max |gpu - ref| / max |ref|: the stated bounds for bf16 and fp32 storage; for
+# fp16 storage (fp32 arithmetic, the output and the cached slots rounded to
+# half precision, unit roundoff 2^-11 = 4.9e-4) ten unit roundoffs
+TOL = {"bf16": 2e-2, "fp32": 1e-5, "fp16": 5e-3}
 
 
 # (test, max-relative error, elementwise error) of every comparison, written

@@ -8,6 +8,7 @@ import re
 import subprocess
 
 import pytest
+import torch
 
 from kv_cache_mtla_b200 import build as kbuild
 from kv_cache_mtla_b200 import mtla
@@ -81,6 +82,15 @@ def test_workspace_size_and_config_checks(lib):
     assert e.value.status == mtla.ERR_UNSUPPORTED
     n = ctypes.c_size_t(0)
     assert lib.mtla_workspace_size(None, 0, ctypes.byref(n)) == mtla.ERR_INVALID_ARG
+    # storage types: bf16, fp32, fp16 accepted; anything else refused
+    for dt in (mtla.BF16, mtla.FP32, mtla.FP16):
+        cfg = _cfg()
+        cfg.dtype = dt
+        assert mtla.workspace_size(cfg, 16) > 0
+    cfg = _cfg()
+    cfg.dtype = 3
+    assert lib.mtla_workspace_size(ctypes.byref(cfg), 0, ctypes.byref(n)) == mtla.ERR_INVALID_ARG
+    assert mtla.make_config(1, 4, 32, 128, 16, 2, 8, dtype="fp16").torch_dtype == torch.float16
 
 
 FAKE = 0x10000  # aligned host-side placeholder: argument checks never dereference it
