@@ -719,7 +719,7 @@ cudaError_t backward_impl(const PrefillArgs& pa_in, const BackwardGrads& g, cuda
 // ---------------------------------------------------------------- tensor-core path
 
 struct BwdTcWs {
-    size_t fwd, cache, out, lse, delta, obar, qt, w, dob, dqt, dF, dP, wuvt, dqtl, part_k, part_v, total;
+    size_t fwd, cache, out, lse, delta, obar, qt, w, dob, dqt, dF, dP, wuvt, dqtl, part_k, part_v, u, total;
 };
 
 Shape with_slots(const Shape& sh, int T) {
@@ -750,6 +750,7 @@ BwdTcWs bwd_tc_layout(const Shape& sh_in, int T) {
     l.dqtl = take(rows * sh.d_c * 2);
     l.part_k = take(weight_part_bytes(sh, T));
     l.part_v = take(weight_part_bytes(sh, T));
+    l.u = take((size_t)sh.B * sh.max_slots * sh.H * sh.d_h * 2);
     l.total = o;
     return l;
 }
@@ -823,10 +824,17 @@ cudaError_t backward_tc(const PrefillArgs& pa_in, const BackwardGrads& g, cudaSt
     k_bwd_delta<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(sh, T_len, dob, (const bf16*)(ws + l.obar),
                                                              (float*)(ws + l.delta));
     if ((e = cudaGetLastError()) != cudaSuccess) return note_error("k_bwd_delta launch", e);
+    // U_j[h] = W_UV[h] F_j[0:d_c] for every finished slot and head: one GEMM,
+    // [B n_slots, d_c] . W_UV viewed as [H d_h, d_c]
+    e = gemm_batched(GemmOperand{ws + l.cache, sh.D, 0}, GemmOperand{pa.w_uv, sh.d_c, 0}, ws + l.u, sh.H * sh.d_h, 0,
+                     false, sh.B * n_slots, sh.H * sh.d_h, sh.d_c, 1, pa.status, st, launches);
+    if (e != cudaSuccess) return e;
     BwdTCInputs in;
     in.qt = ws + l.qt;
     in.dob = ws + l.dob;
     in.slots = ws + l.cache;
+    in.dout = g.dout;
+    in.u = ws + l.u;
     in.lse = (const float*)(ws + l.lse);
     in.delta = (const float*)(ws + l.delta);
     in.dqt = a.dqt;

@@ -119,6 +119,8 @@ struct BwdTCInputs {
     const void* qt;        // [B, T, H, D] bf16
     const void* dob;       // [B, T, H, d_c] bf16
     const void* slots;     // [B, n_slots, D] bf16 (the forward's cache rows)
+    const void* dout;      // [B, T, H, d_h] bf16
+    const void* u;         // [B, n_slots, H d_h] bf16: U_j[h] = W_UV[h] F_j[0:d_c]
     const float* lse;      // [B, H, stats_pitch(T)]
     const float* delta;    // [B, H, stats_pitch(T)]
     float* dqt;

@@ -10,7 +10,8 @@
 //   p_ij = 2^(S_ij scale log2(e) - lse_i),  S_ij = qt_i . F_j,
 //   dPa_ij = dobar_i . F_j[0:d_c],  dS_ij = scale p_ij (dPa_ij - delta_i),
 // the finished-slot part of the gradients is two contractions:
-//   dqt_i += sum_j dS_ij F_j                 (k_bwd_dq_tc, one CTA per query tile)
+//   dqt_i += sum_j dS_ij F_j                 (k_bwd_dq_tc, one CTA per query tile;
+//                                             dPa there as dout_i . U_j, U_j = W_UV[h] F_j)
 //   dF_j  += sum_i dS_ij qt_i + p_ij [dobar_i ; 0]   (k_bwd_dk_tc, one CTA per slot tile)
 // The own-partial term (one key per row) runs on the CUDA cores.
 //
@@ -60,8 +61,9 @@ struct BwdTC {
 
 struct MapsQ {
     CUtensorMap q, q_r;         // qt (D, H, T, B): boxes (64, 1, 128, 1) and (32, 1, 128, 1)
-    CUtensorMap dob;            // dobar (d_c, H, T, B): box (64, 1, 128, 1)
+    CUtensorMap dout;           // dout (d_h, H, T, B): box (64, 1, 128, 1)
     CUtensorMap k, k_r;         // slots (D, n_slots, B): boxes (64, 64, 1) and (32, 64, 1)
+    CUtensorMap u;              // U (H d_h, n_slots, B): box (64, 64, 1)
 };
 struct MapsK {
     CUtensorMap k, k_r;         // slots: boxes (64, 128, 1) and (32, 128, 1)
@@ -112,9 +114,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dq_tc(const __grid_constant
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     constexpr int NL = DC / 64;
     constexpr uint32_t q_bytes = NL * kM * 128 + kM * 64;      // query image: latent chunks + RoPE chunk
-    constexpr uint32_t do_bytes = NL * kM * 128;               // dobar image
+    constexpr uint32_t do_bytes = kM * 128;                    // dout image [128 rows x d_h = 64]
     constexpr uint32_t kchunk = kN * 128;                      // one latent chunk of a key tile
-    constexpr uint32_t stage_bytes = NL * kchunk + kN * 64;
+    constexpr uint32_t u_off = NL * kchunk + kN * 64;          // the tile's U rows [64 x d_h]
+    constexpr uint32_t stage_bytes = u_off + kN * 128;
     uint8_t* q_s = smem;
     uint8_t* do_s = q_s + q_bytes;
     uint8_t* ring = do_s + do_bytes;
@@ -160,11 +163,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dq_tc(const __grid_constant
         if (lane == 0 && nkt > 0) {
             mbar_arrive_expect_tx(&bs.q_full, q_bytes + do_bytes);
 #pragma unroll
-            for (int c = 0; c < NL; ++c) {
-                tma_load_4d(q_s + c * kM * 128, &maps.q, &bs.q_full, c * 64, h, p0, b);
-                tma_load_4d(do_s + c * kM * 128, &maps.dob, &bs.q_full, c * 64, h, p0, b);
-            }
+            for (int c = 0; c < NL; ++c) tma_load_4d(q_s + c * kM * 128, &maps.q, &bs.q_full, c * 64, h, p0, b);
             tma_load_4d(q_s + NL * kM * 128, &maps.q_r, &bs.q_full, DC, h, p0, b);
+            tma_load_4d(do_s, &maps.dout, &bs.q_full, 0, h, p0, b);
             for (int k = 0; k < nkt; ++k) {
                 if (k >= 2 && !waitb(&bs.empty[k & 1], ((k >> 1) - 1) & 1, bs)) break;
                 uint8_t* dst = ring + (k & 1) * stage_bytes;
@@ -172,6 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dq_tc(const __grid_constant
 #pragma unroll
                 for (int c = 0; c < NL; ++c) tma_load_3d(dst + c * kchunk, &maps.k, &bs.full[k & 1], c * 64, kN * k, b);
                 tma_load_3d(dst + NL * kchunk, &maps.k_r, &bs.full[k & 1], DC, kN * k, b);
+                tma_load_3d(dst + u_off, &maps.u, &bs.full[k & 1], h * kDh, kN * k, b);
                 loads = k + 1;
             }
         }
@@ -208,7 +210,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dq_tc(const __grid_constant
                     tc_fence_after();
                     const uint32_t st_a = ring_a + (k & 1) * stage_bytes;
                     const uint64_t kd = sdesc_sw128(st_a, 16, 1024), kr = sdesc_sw64(st_a + NL * kchunk);
-                    // S = qt . K^T (K = D), dPa = dobar . V^T (K = d_c)
+                    // S = qt . K^T (K = D); dPa = dobar . V^T = dout . U^T (K = d_h), U_j = W_UV[h] F_j
 #pragma unroll
                     for (int c = 0; c < NL; ++c)
 #pragma unroll
@@ -218,12 +220,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dq_tc(const __grid_constant
 #pragma unroll
                     for (int kk = 0; kk < kDr / 16; ++kk)
                         umma_bf16(t_s, desc_add(qr, kk * 32), desc_add(kr, kk * 32), id_s, 1u);
+                    const uint64_t ud = sdesc_sw128(st_a + u_off, 16, 1024);
 #pragma unroll
-                    for (int c = 0; c < NL; ++c)
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            umma_bf16(t_dp, desc_add(dd, c * kM * 128 + kk * 32), desc_add(kd, c * kchunk + kk * 32),
-                                      id_s, (c | kk) != 0);
+                    for (int kk = 0; kk < kDh / 16; ++kk)
+                        umma_bf16(t_dp, desc_add(dd, kk * 32), desc_add(ud, kk * 32), id_s, kk != 0);
                     umma_commit(&bs.sd_full);
                     if (k >= 1) ok = dq_mma(k - 1);
                 }
@@ -535,7 +535,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dk_tc(const __grid_constant
 
 template <int DC>
 constexpr size_t dq_smem() {
-    return 1024 + (size_t)(DC / 64) * kM * 128 * 2 + kM * 64 + 2 * ((DC / 64) * kN * 128 + kN * 64) +
+    return 1024 + (size_t)(DC / 64) * kM * 128 + kM * 64 + kM * 128 + 2 * ((DC / 64) * kN * 128 + kN * 64 + kN * 128) +
            ((sizeof(BarsQ) + 15) & ~(size_t)15);
 }
 template <int DC>
@@ -579,7 +579,11 @@ cudaError_t launch(const Shape& sh, const BwdTCInputs& in, const BwdTC& p, cudaS
         const cuuint32_t bq[4] = {64, 1, kM, 1}, bqr[4] = {kDr, 1, kM, 1}, bk[3] = {64, kN, 1}, bkr[3] = {kDr, kN, 1};
         if (e == cudaSuccess) e = map_(enc, &mq.q, in.qt, 4, dq, sq, bq, "qt", BF, S128);
         if (e == cudaSuccess) e = map_(enc, &mq.q_r, in.qt, 4, dq, sq, bqr, "qt RoPE", BF, S64);
-        if (e == cudaSuccess) e = map_(enc, &mq.dob, in.dob, 4, dd, sd, bq, "dobar", BF, S128);
+        const cuuint64_t dh[4] = {(cuuint64_t)kDh, H, T, B}, sh4[3] = {E * kDh, E * H * kDh, E * T * H * kDh};
+        const cuuint64_t du[3] = {H * kDh, ns, B}, su[2] = {E * H * kDh, E * ns * H * kDh};
+        const cuuint32_t bu[3] = {64, kN, 1};
+        if (e == cudaSuccess) e = map_(enc, &mq.dout, in.dout, 4, dh, sh4, bq, "dout", BF, S128);
+        if (e == cudaSuccess) e = map_(enc, &mq.u, in.u, 3, du, su, bu, "U", BF, S128);
         if (e == cudaSuccess) e = map_(enc, &mq.k, in.slots, 3, dk, sk, bk, "slots", BF, S128);
         if (e == cudaSuccess) e = map_(enc, &mq.k_r, in.slots, 3, dk, sk, bkr, "slots RoPE", BF, S64);
     }
