@@ -200,24 +200,35 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
         }
     }
     // latent part: warp w reads TMEM lane quarter w mod 4 (latent rows), sequences
-    // 16 (w / 4) .. 16 (w / 4) + 15
+    // 16 (w / 4) .. 16 (w / 4) + 15. Each sequence's row h of every 64-column
+    // chunk is one 128-byte run of its image: the rows are assembled in shared
+    // memory (the W_UK buffer, free once the MMAs are done) with the image's
+    // swizzle and leave as 16-byte stores.
     const bool done = mbar_wait(&bars[1], (n_kb - 1) & 1);
     tc_fence_after();
+    uint8_t* stage = w_s;                                  // [32 sequences][n_kc chunks][128 B]
     {
         const int quarter = warp & 3, half = warp >> 2;
+        const uint32_t hx = (uint32_t)(h & 7);
         for (int mb = 0; mb < n_kc / 2; ++mb) {
             float v[16];
             tmem_ld16(t_d + mb * 32 + half * 16 + ((uint32_t)(quarter * 32) << 16), v);
             tmem_wait_ld();
             const int j = mb * 128 + quarter * 32 + lane;      // latent column
+            const uint32_t in_row = ((((uint32_t)(j & 63) >> 3) ^ hx) << 4) + ((j & 7) << 1);
 #pragma unroll
             for (int s = 0; s < 16; ++s) {
-                const int b = c0 + half * 16 + s;
-                if (done && b < sh.B && lh_pos_ok(sh, a.pos[b]))
-                    *(bf16*)(qimg + (size_t)b * img_bytes + (size_t)(j >> 6) * 128 * 128 + sw128_offset(h, j & 63)) =
-                        __float2bfloat16_rn(v[s]);
+                const int bb = half * 16 + s;
+                *(bf16*)(stage + ((size_t)bb * n_kc + (j >> 6)) * 128 + in_row) = __float2bfloat16_rn(v[s]);
             }
         }
+    }
+    __syncthreads();
+    for (int e = tid; e < 32 * n_kc * 8; e += kPrepThreads) {
+        const int row = e >> 3, u = e & 7, bb = row / n_kc, c = row % n_kc, b = c0 + bb;
+        if (done && b < sh.B && lh_pos_ok(sh, a.pos[b]))
+            *(uint4*)(qimg + (size_t)b * img_bytes + (size_t)c * 128 * 128 + (size_t)h * 128 + u * 16) =
+                *(const uint4*)(stage + (size_t)row * 128 + u * 16);
     }
     tc_fence_before();
     __syncthreads();
