@@ -477,6 +477,13 @@ def measure_prefill(n, flush, ws, rank):
             "clocks": clocks, "l2": L2Flush.desc + " call"}
 
 
+def _backward_traffic():
+    """DRAM bytes of the two tensor-core backward kernels of one call (their
+    captures at this workload), or None when either's sources changed."""
+    dq, dk = _traffic("k_bwd_dq_tc"), _traffic("k_bwd_dk_tc")
+    return None if dq is None or dk is None else dq + dk
+
+
 def measure_backward(n, flush, ws, rank):
     """Training backward at the prefill workload's sizes (B=8, T=8192, H=8,
     d_h=64, d_c=256, d_R=32, s=2, computed gates): every gradient of the path
@@ -512,7 +519,7 @@ def measure_backward(n, flush, ws, rank):
             "attention_flops_per_call": flops, "calls": n,
             "roofline": {"kernel": "k_bwd_dq_tc + k_bwd_dk_tc (masked attention backward, tensor cores)",
                          "bound": "tensor", "achieved": kern, "peak": tflops_peak, "unit": "TFLOP/s",
-                         "frac": kern / tflops_peak, "traffic": None,
+                         "frac": kern / tflops_peak, "traffic": _backward_traffic(),
                          "peak_source": f"{peak_kind} bf16_tflops (burst)",
                          "avg_launch_us": kern_ms * 1e3},
             "clocks": clocks, "l2": L2Flush.desc + " call"}
