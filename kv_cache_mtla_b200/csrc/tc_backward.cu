@@ -47,6 +47,7 @@ constexpr int kN = 64;          // keys (dQ) or query positions (dK) per tile
 constexpr int kDr = 32;         // d_R of these kernels (one 64-byte-swizzled chunk)
 constexpr int kDh = 64;         // d_h of these kernels
 constexpr int kThreads = 320;   // warp 0 TMA, 1 MMA, 2-9 elementwise
+constexpr int kBand = 8;        // slot tiles per scheduling band of k_bwd_dk_tc
 
 struct BwdTC {
     int B, T, H, D, s, n_slots;
@@ -312,10 +313,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dq_tc(const __grid_constant
 
 // ---------------------------------------------------------------- dK
 
-// One CTA per (slot tile of 128, sequence, head), heaviest (earliest) first.
-// The query positions that see any slot of the tile, from the first multiple
-// of 64 at or below (j0 + 1) s, in tiles of 64; positions past T read as zeros
-// and are masked.
+// One CTA per (slot tile of 128, sequence, head). The query positions that
+// see any slot of the tile, from the first multiple of 64 at or below
+// (j0 + 1) s, in tiles of 64 taken from the last down; positions past T read
+// as zeros and are masked.
 template <int DC>
 __global__ void __launch_bounds__(kThreads, 1) k_bwd_dk_tc(const __grid_constant__ MapsK maps, const BwdTC p) {
     extern __shared__ uint8_t smem_raw[];
@@ -332,9 +333,23 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dk_tc(const __grid_constant
     BarsK& bs = *(BarsK*)(ring + 2 * stage_bytes);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int per_kt = p.B * p.H;
-    const int kt = (int)blockIdx.x / per_kt;
-    const int b = ((int)blockIdx.x % per_kt) / p.H, h = (int)blockIdx.x % p.H;
+    // items in bands of kBand slot tiles, the heaviest (earliest) band first;
+    // inside a band the items of one (sequence, head) are consecutive and walk
+    // their query tiles from the top down, so they start on the same tile and
+    // share its query rows in L2
+    const int BH = p.B * p.H, full = p.n_ktiles / kBand;
+    const int idx = blockIdx.x;
+    int kt, bh;
+    if (idx < full * kBand * BH) {
+        const int band = idx / (kBand * BH), rem = idx % (kBand * BH);
+        bh = rem / kBand;
+        kt = band * kBand + rem % kBand;
+    } else {
+        const int rem = idx - full * kBand * BH, last = p.n_ktiles - full * kBand;
+        bh = rem / last;
+        kt = full * kBand + rem % last;
+    }
+    const int b = bh / p.H, h = bh % p.H;
     const int j0 = kt * kM;
     const int pbase = (((j0 + 1) * p.s) / kN) * kN;
     const int ntl = pbase < p.T ? (p.T - pbase + kN - 1) / kN : 0;
@@ -376,7 +391,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dk_tc(const __grid_constant
             for (int k = 0; k < ntl; ++k) {
                 if (k >= 2 && !waitb(&bs.empty[k & 1], ((k >> 1) - 1) & 1, bs)) break;
                 uint8_t* dst = ring + (k & 1) * stage_bytes;
-                const int pk = pbase + kN * k;
+                const int pk = pbase + kN * (ntl - 1 - k);
                 mbar_arrive_expect_tx(&bs.full[k & 1], qt_bytes + dob_bytes + 512);
 #pragma unroll
                 for (int c = 0; c < NL; ++c) {
@@ -468,7 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dk_tc(const __grid_constant
             // is refilled only after this tile's accumulating MMAs, below)
             waitb(&bs.full[k & 1], (k >> 1) & 1, bs);
             const float* st = (const float*)(ring + (k & 1) * stage_bytes + stats_off);
-            const int pk = pbase + kN * k + 32 * hc;
+            const int pk = pbase + kN * (ntl - 1 - k) + 32 * hc;
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
                 float p2[2], d2[2];
