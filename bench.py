@@ -525,16 +525,17 @@ def measure_backward(n, flush, ws, rank):
             "clocks": clocks, "l2": L2Flush.desc + " call"}
 
 
-def measure_speech(n, flush, ws, rank):
+def measure_speech(n, flush, ws, rank, dtype="bf16"):
     """Speech-model-scale decode B=16, H=8, s=2: a 1024-token prefix by the
-    prefill, then 256 decode steps (513..640 slots), as two CUDA graphs."""
-    wl = inputs.SPEECH_DECODE.with_(seed=inputs.SPEECH_DECODE.seed + 1000 * rank)
+    prefill, then 256 decode steps (513..640 slots), as two CUDA graphs
+    (bf16 storage, or fp16 with dtype="fp16")."""
+    wl = inputs.SPEECH_DECODE.with_(seed=inputs.SPEECH_DECODE.seed + 1000 * rank, dtype=dtype)
     T, S = wl.T, wl.steps
     max_slots = (T + S + wl.s - 1) // wl.s
     cfg = mtla.make_config(wl.B, wl.H, wl.d_h, wl.d_c, wl.d_r, wl.s, max_slots, dtype=wl.dtype,
                            gate_mode=wl.gate_mode)
     buf = mtla.Buffers.allocate(cfg, inputs.weights(wl), max_tokens=T)
-    bf = torch.bfloat16
+    bf = cfg.torch_dtype
     pre = inputs.tokens(wl, T, stream=0)
     dec = inputs.tokens(wl, S, stream=1)
     dp = {k: pre[k].to("cuda", bf).contiguous() for k in ("c", "kr", "qc", "qr")}
@@ -590,7 +591,7 @@ def measure_speech(n, flush, ws, rank):
     attn_ms = statistics.mean(prof.durations_ms())
     attn_bytes = wl.B * wl.D * 2 * statistics.mean(slots)
     return {"workload": f"speech_decode: B={wl.B}/rank, H={wl.H}, d_h={wl.d_h}, d_c={wl.d_c}, "
-                        f"d_R={wl.d_r}, s={wl.s}; prefill {T} tokens then {S} decode steps",
+                        f"d_R={wl.d_r}, s={wl.s}, {wl.dtype} storage; prefill {T} tokens then {S} decode steps",
             "decode_tokens_per_s": wl.B * S * ws * n / (dec_ms / 1e3),
             "ms_per_token_step": dec_ms / n / S,
             "decode_latent_cache_GBps": wl.B * wl.D * 2 * sum(slots) * ws * n / (dec_ms / 1e3) / 1e9,
@@ -600,7 +601,7 @@ def measure_speech(n, flush, ws, rank):
             "roofline": {"kernel": "k_dec_attn_sh (decode attention)", "bound": "hbm",
                          "achieved": attn_bytes / (attn_ms / 1e3) / 1e9, "peak": hbm,
                          "unit": "GB/s", "frac": attn_bytes / (attn_ms / 1e3) / 1e9 / hbm,
-                         "traffic": _traffic("k_dec_attn_sh"),
+                         "traffic": _traffic("k_dec_attn_sh") if wl.dtype == "bf16" else None,
                          "peak_source": f"{peak_kind} hbm_gbs", "avg_launch_us": attn_ms * 1e3},
             "clocks": clk.summary(), "cuda_graphs": "prefill graph + 256-step decode graph",
             "l2": L2Flush.desc + " step"}
@@ -835,7 +836,8 @@ def run_kernel_workload(args):
         print(json.dumps(measure_prefill(args.steps, flush, 1, 0)), flush=True)
         return
     if name.startswith("speech_decode"):
-        print(json.dumps(measure_speech(args.steps, flush, 1, 0)), flush=True)
+        dt = "fp16" if name.endswith("fp16") else "bf16"
+        print(json.dumps(measure_speech(args.steps, flush, 1, 0, dtype=dt)), flush=True)
         return
     if name == "layer":
         print(json.dumps(measure_layer(args.steps, flush, 1, 0)), flush=True)
@@ -904,6 +906,8 @@ def run_contract(args, ws, rank):
         extras["prefill"] = measure_prefill(900, flush, ws, rank)
         torch.cuda.empty_cache()
         extras["speech_decode"] = measure_speech(320, flush, ws, rank)
+        torch.cuda.empty_cache()
+        extras["speech_decode_fp16"] = measure_speech(320, flush, ws, rank, dtype="fp16")
         torch.cuda.empty_cache()
         extras["stride_sweep"] = measure_stride(6000, flush, ws, rank)
         torch.cuda.empty_cache()

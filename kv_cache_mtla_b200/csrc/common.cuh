@@ -74,11 +74,29 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
     return r;
 }
 
+// Two floats as one 32-bit word of two 16-bit values of type E (round to
+// nearest even), `lo` at the lower address; and the two halves back.
+template <typename E> __device__ __forceinline__ uint32_t pack2(float lo, float hi);
+template <> __device__ __forceinline__ uint32_t pack2<f16>(float lo, float hi) {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+template <typename E> __device__ __forceinline__ float lo_of(uint32_t w);
+template <typename E> __device__ __forceinline__ float hi_of(uint32_t w);
+template <> __device__ __forceinline__ float lo_of<bf16>(uint32_t w) { return __uint_as_float(w << 16); }
+template <> __device__ __forceinline__ float hi_of<bf16>(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+template <> __device__ __forceinline__ float lo_of<f16>(uint32_t w) {
+    return __half2float(__ushort_as_half((unsigned short)(w & 0xffffu)));
+}
+template <> __device__ __forceinline__ float hi_of<f16>(uint32_t w) {
+    return __half2float(__ushort_as_half((unsigned short)(w >> 16)));
+}
 // Two floats as bf16 (round to nearest even), `lo` at the lower address.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
 }
+template <> __device__ __forceinline__ uint32_t pack2<bf16>(float lo, float hi) { return pack_bf16x2(lo, hi); }
 
 __device__ __forceinline__ float sigmoidf_(float z) { return 1.f / (1.f + expf(-z)); }
 

@@ -115,6 +115,7 @@ static mtla_status check_config(const mtla_config* cfg, Shape* sh) {
     sh->s = cfg->stride;
     sh->D = cfg->d_c + cfg->d_r;
     sh->gate_mode = cfg->gate_mode;
+    sh->dtype = cfg->dtype;
     sh->max_slots = cfg->max_slots;
     sh->scale = cfg->softmax_scale != 0.f ? cfg->softmax_scale
                                           : (float)(1.0 / std::sqrt((double)(cfg->d_h + cfg->d_r)));
@@ -123,11 +124,12 @@ static mtla_status check_config(const mtla_config* cfg, Shape* sh) {
     return MTLA_OK;
 }
 
-// bf16 decode runs on the tensor cores where the shape fits the kernel
-// (heads <= 32, d_c a multiple of 128, slot width <= 384); fp32 and the other
-// bf16 shapes run on the CUDA-core kernels.
+// bf16 and fp16 decode run on the tensor cores where the shape fits the
+// kernel (heads <= 32, d_c a multiple of 128, slot width <= 384); bf16 with
+// 32 < heads <= 128 on the cluster kernel; fp32 and the other shapes on the
+// CUDA-core kernels.
 static bool use_tc_decode(const mtla_config* cfg, const Shape& sh) {
-    return cfg->dtype == MTLA_BF16 && tc_decode_supported(sh);
+    return (cfg->dtype == MTLA_BF16 || cfg->dtype == MTLA_FP16) && tc_decode_supported(sh);
 }
 // bf16 with 32 < heads <= 128: the cluster kernel with all heads as M = 128.
 static bool use_tc_decode_lh(const mtla_config* cfg, const Shape& sh) {
@@ -139,10 +141,10 @@ static size_t decode_ws(const mtla_config* cfg, const Shape& sh) {
     if (use_tc_decode_lh(cfg, sh)) return tc_decode_lh_workspace(sh);
     return simt_decode_workspace(sh);
 }
-// bf16 prefill runs on the tensor cores where the shape fits the kernel
-// (d_h = 64, d_c <= 256, slot width <= 320); the rest on the CUDA cores.
+// bf16 and fp16 prefill run on the tensor cores where the shape fits the
+// kernel (d_h = 64, d_R = 32, d_c 128 or 256); the rest on the CUDA cores.
 static bool use_tc_prefill(const mtla_config* cfg, const Shape& sh) {
-    return cfg->dtype == MTLA_BF16 && tc_prefill_supported(sh);
+    return (cfg->dtype == MTLA_BF16 || cfg->dtype == MTLA_FP16) && tc_prefill_supported(sh);
 }
 
 static size_t prefill_ws(const mtla_config* cfg, const Shape& sh, int T) {

@@ -9,6 +9,7 @@ namespace mtla {
 struct Shape {
     int B, H, d_h, d_c, d_r, s, D;
     int gate_mode;          // 0 computed, 1 supplied, 2 unit
+    int dtype;              // storage type: kDtypeBF16, kDtypeF32 or kDtypeF16
     int max_slots;
     float scale;            // softmax scale (resolved)
     double log2_rope_base;  // log2 of the RoPE base

@@ -319,14 +319,14 @@ template <> __device__ __forceinline__ void store8<bf16>(bf16* p, const float* v
 // open at t0, if t0 is not a multiple of s, starts from open_slot_in (the
 // accumulator after t0 tokens) instead of 0.
 // One warp per slot: grid (ceil(n / 8), B), n = slots touched, 256 threads.
-// With bf16 partial slots (the tensor-core prefill) the sine and cosine of the
+// With 16-bit partial slots (the tensor-core prefill) the sine and cosine of the
 // angle, reduced to [-pi, pi] in double as everywhere, come from the special-
 // function unit (absolute error about 2^-21 there, far below the bf16 rounding
 // of the slots); the fp32 partial slots of the CUDA-core path keep sincosf.
 template <typename T, typename PT>
 __global__ void __launch_bounds__(256) k_prefill_scan(PrefillArgs a, PT* P, float2* rope_tab = nullptr,
                                                       float* w_out = nullptr) {
-    constexpr bool kFastSinCos = std::is_same<PT, bf16>::value;
+    constexpr bool kFastSinCos = !std::is_same<PT, float>::value;
     auto sincos_at = [](int64_t t, double inv_freq, float* sn, float* cs) {
         if constexpr (kFastSinCos) {
             double ang = (double)t * inv_freq;

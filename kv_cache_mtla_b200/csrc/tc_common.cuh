@@ -416,6 +416,25 @@ __device__ __forceinline__ uint64_t sdesc_sw64(uint32_t saddr) {
 // addresses stay below 2^18, no carry out of the 14-bit field).
 __device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) { return d + (uint64_t)(bytes >> 4); }
 
+// Operand format of a 16-bit element type in the kind::f16 instruction
+// descriptor (0 = f16, 1 = bf16). A and B always take the same type.
+template <typename E> struct MmaFmt;
+template <> struct MmaFmt<bf16> { static constexpr uint32_t v = 1; };
+template <> struct MmaFmt<f16> { static constexpr uint32_t v = 0; };
+
+// Instruction descriptor for kind::f16 with A and B of type E (both) and fp32
+// accumulation.
+template <typename E>
+__host__ __device__ constexpr uint32_t idesc_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
+    return (1u << 4)                               // D format: f32
+           | (MmaFmt<E>::v << 7)                   // A format
+           | (MmaFmt<E>::v << 10)                  // B format (the same)
+           | ((a_mn_major ? 1u : 0u) << 15)        // A major
+           | ((b_mn_major ? 1u : 0u) << 16)        // B major
+           | ((uint32_t)(N >> 3) << 17)            // N / 8
+           | ((uint32_t)(M >> 4) << 24);           // M / 16
+}
+
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 accumulation.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
     return (1u << 4)                               // D format: f32

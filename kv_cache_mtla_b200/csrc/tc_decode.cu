@@ -29,6 +29,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 #include <utility>
 
 #include "common.cuh"
@@ -95,6 +96,7 @@ __device__ __forceinline__ int seq_slots(const DecTC& p, int b) {
 // starts before its predecessor ends only when that predecessor triggers its
 // dependents early, which the library's own kernels alone do (a step's combine
 // kernel, which writes neither); the C-ABI header states this for callers.
+template <typename E>
 __global__ void __launch_bounds__(kPrepAbsThreads + 32) k_dec_prep_tc(DecodeArgs a, uint8_t* qimg, uint32_t img_bytes, int n_chunks, int NH, int compact) {
     pdl_launch_dependents();   // the attention kernel may start its prologue now
     const Shape& sh = a.sh;
@@ -116,7 +118,7 @@ __global__ void __launch_bounds__(kPrepAbsThreads + 32) k_dec_prep_tc(DecodeArgs
             gw = gs;
         }
         pdl_wait();
-        decode_update_body<bf16>(a, b, gw, f);
+        decode_update_body<E>(a, b, gw, f);
         const int pad = NH - sh.H;
         for (int e = threadIdx.x; e < n_wide * pad * 8; e += blockDim.x) {
             const int c = e / (pad * 8), rr = e % (pad * 8);
@@ -129,8 +131,8 @@ __global__ void __launch_bounds__(kPrepAbsThreads + 32) k_dec_prep_tc(DecodeArgs
         return;
     }
     const size_t rh = (size_t)b * sh.H + h;
-    const bf16* qc = (const bf16*)a.q_c + rh * sh.d_h;
-    const bf16* qr = (const bf16*)a.q_r + rh * sh.d_r;
+    const E* qc = (const E*)a.q_c + rh * sh.d_h;
+    const E* qr = (const E*)a.q_r + rh * sh.d_r;
     const int dpad = compact ? sh.D : n_chunks * 64;
     if (threadIdx.x >= kPrepAbsThreads) {
         // the last warp: RoPE part of q~ (columns d_c .. D-1) and the zero padding
@@ -142,20 +144,20 @@ __global__ void __launch_bounds__(kPrepAbsThreads + 32) k_dec_prep_tc(DecodeArgs
             float v = 0.f;
             if (j < sh.D) {
                 const int e = j - sh.d_c, k = e >> 1;
-                const float x0 = __bfloat162float(qr[2 * k]), x1 = __bfloat162float(qr[2 * k + 1]);
+                const float x0 = to_f<E>(qr[2 * k]), x1 = to_f<E>(qr[2 * k + 1]);
                 float sn, cs;
                 pair_sincos(t, k, sh.d_r, sh.log2_rope_base, &sn, &cs);
                 v = (e & 1) ? (x0 * sn + x1 * cs) : (x0 * cs - x1 * sn);
             }
-            bf16* dst = compact ? (bf16*)(rope_img + sw64_offset(h, j - sh.d_c))
-                                : (bf16*)(img + (size_t)(j >> 6) * NH * 128 + sw128_offset(h, j & 63));
-            *dst = __float2bfloat16_rn(v);
+            E* dst = compact ? (E*)(rope_img + sw64_offset(h, j - sh.d_c))
+                                : (E*)(img + (size_t)(j >> 6) * NH * 128 + sw128_offset(h, j & 63));
+            *dst = from_f<E>(v);
         }
         return;
     }
     // thread (ig, jg): 8 latent columns [8 jg, 8 jg + 8) over rows i of group ig;
     // its 16-byte loads of W_UK and of qC are all issued before any product
-    const bf16* W = (const bf16*)a.w_uk + (size_t)h * sh.d_h * sh.d_c;
+    const E* W = (const E*)a.w_uk + (size_t)h * sh.d_h * sh.d_c;
     const int n_jg = sh.d_c / 8;
     const int n_ig = max(1, min(8, kPrepAbsThreads / n_jg));
     const int rows_per = (((sh.d_h + n_ig - 1) / n_ig) + 15) & ~15;   // 16-row batches, aligned
@@ -188,14 +190,14 @@ __global__ void __launch_bounds__(kPrepAbsThreads + 32) k_dec_prep_tc(DecodeArgs
 #pragma unroll
             for (int u = 0; u < 2; ++u)
                 if (ib + 8 * u < i1) qraw[u] = *(const uint4*)(qc + ib + 8 * u);   // d_h % 16 == 0
-            const bf16* qv = (const bf16*)qraw;
+            const E* qv = (const E*)qraw;
 #pragma unroll
             for (int u = 0; u < 16; ++u) {
                 if (ib + u < i1) {
-                    const bf16* wv = (const bf16*)&raw[u];
-                    const float qi = __bfloat162float(qv[u]);
+                    const E* wv = (const E*)&raw[u];
+                    const float qi = to_f<E>(qv[u]);
 #pragma unroll
-                    for (int v = 0; v < 8; ++v) acc[v] = fmaf(__bfloat162float(wv[v]), qi, acc[v]);
+                    for (int v = 0; v < 8; ++v) acc[v] = fmaf(to_f<E>(wv[v]), qi, acc[v]);
                 }
             }
         }
@@ -207,7 +209,7 @@ __global__ void __launch_bounds__(kPrepAbsThreads + 32) k_dec_prep_tc(DecodeArgs
     for (int j = threadIdx.x; j < sh.d_c; j += kPrepAbsThreads) {
         float v = 0.f;
         for (int ig = 0; ig < n_ig; ++ig) v += part_sum[ig][j];
-        *(bf16*)(img + (size_t)(j >> 6) * NH * 128 + sw128_offset(h, j & 63)) = __float2bfloat16_rn(v);
+        *(E*)(img + (size_t)(j >> 6) * NH * 128 + sw128_offset(h, j & 63)) = from_f<E>(v);
     }
 }
 
@@ -255,7 +257,7 @@ struct DecMaps {
 // P^T of a tile is written over its RoPE part, which only the score MMAs read
 // and which is free once they are done; that leaves room for a third stage,
 // so two loads stay in flight while a tile is worked on.
-template <int NH, int HV, int ST>
+template <int NH, int HV, int ST, typename E>
 __global__ void __launch_bounds__(kAttnThreads, 1)
     k_dec_attn_sh(const __grid_constant__ DecMaps maps, const DecTC p) {
     static_assert(HV % 8 == 0 && HV <= NH, "head count");
@@ -396,7 +398,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     } else if (warp == 5) {
         // ------------------------------------------------------------ score MMAs
         if (lane == 0) {
-            const uint32_t id_s = idesc_bf16_f32(128, NH, false, false);
+            const uint32_t id_s = idesc_f32<E>(128, NH, false, false);
             const uint64_t q_d = sdesc_sw128(smem_u32(q_s), 16, 1024);
             const uint32_t ring_a = smem_u32(ring);
             const int last_ksteps = (p.D - 64 * (n_chunks - 1)) / 16;   // D is a multiple of 16
@@ -482,7 +484,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // ------------------------------------------------------------ P.V MMAs (own thread: they free
         // ring stages, so they never wait behind a score MMA that waits for a load)
         if (lane == 0) {
-            const uint32_t id_o = idesc_bf16_f32(128, NH, true, false);
+            const uint32_t id_o = idesc_f32<E>(128, NH, true, false);
             const uint32_t ring_a = smem_u32(ring), p_a = smem_u32(p_s);
             int prev_b = -1, k = 0;
             for (int gt = gt0; gt < gt1; ++gt, ++k) {
@@ -601,7 +603,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 uint8_t* pb = (kCompact ? stage + pt_off : p_s + (size_t)st * 2 * NH * 128) +
                               (size_t)(tid >> 6) * NH * 128;
 #pragma unroll
-                for (int h = 0; h < HV; ++h) *(bf16*)(pb + sw128_offset(h, tid & 63)) = __float2bfloat16_rn(sv[h]);
+                for (int h = 0; h < HV; ++h) *(E*)(pb + sw128_offset(h, tid & 63)) = from_f<E>(sv[h]);
             }
             fence_proxy_async();
             tc_fence_before();
@@ -666,6 +668,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 // Merge the partials of (b, h) and apply W_UV. grid (H, B), 256 threads.
 // W_UV[h] is staged in shared memory before the wait for the attention kernel;
 // after it, every partial value this block needs is read in one round.
+template <typename E>
 __global__ void __launch_bounds__(256) k_dec_combine(DecodeArgs a, DecTC p) {
     pdl_launch_dependents();   // the next step's prep may stage its W_UK rows now
     const int h = blockIdx.x, b = blockIdx.y;
@@ -676,10 +679,10 @@ __global__ void __launch_bounds__(256) k_dec_combine(DecodeArgs a, DecTC p) {
     __shared__ int n_part;
     __shared__ __align__(16) float olat[512];
     extern __shared__ uint8_t dyn[];
-    bf16* Ws = (bf16*)dyn;                            // W_UV[h] [d_h x d_c]
+    E* Ws = (E*)dyn;                            // W_UV[h] [d_h x d_c]
     {
         // eight 16-byte loads in flight per thread before any store
-        const uint4* src = (const uint4*)((const bf16*)a.w_uv + (size_t)h * sh.d_h * sh.d_c);
+        const uint4* src = (const uint4*)((const E*)a.w_uv + (size_t)h * sh.d_h * sh.d_c);
         uint4* dst = (uint4*)Ws;
         const int n16 = sh.d_h * sh.d_c / 8;
         for (int e0 = threadIdx.x; e0 < n16; e0 += 8 * blockDim.x) {
@@ -754,7 +757,7 @@ __global__ void __launch_bounds__(256) k_dec_combine(DecodeArgs a, DecTC p) {
     // o = W_UV[h] o_lat: warp w takes rows w, w + 8, ... in groups of 8 rows whose
     // dot products run side by side (8 independent chains, one reduction round)
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    bf16* out = (bf16*)a.out + ((size_t)b * sh.H + h) * sh.d_h;
+    E* out = (E*)a.out + ((size_t)b * sh.H + h) * sh.d_h;
     for (int i0 = warp; i0 < sh.d_h; i0 += 64) {
         float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         for (int c0 = lane * 8; c0 < sh.d_c; c0 += 256) {
@@ -765,9 +768,9 @@ __global__ void __launch_bounds__(256) k_dec_combine(DecodeArgs a, DecTC p) {
                 const int i = i0 + r * 8;
                 if (i < sh.d_h) {
                     const uint4 raw = *(const uint4*)(Ws + (size_t)i * sh.d_c + c0);
-                    const bf16* wv = (const bf16*)&raw;
+                    const E* wv = (const E*)&raw;
 #pragma unroll
-                    for (int v = 0; v < 8; ++v) acc[r] = fmaf(__bfloat162float(wv[v]), ov[v], acc[r]);
+                    for (int v = 0; v < 8; ++v) acc[r] = fmaf(to_f<E>(wv[v]), ov[v], acc[r]);
                 }
             }
         }
@@ -777,7 +780,7 @@ __global__ void __launch_bounds__(256) k_dec_combine(DecodeArgs a, DecTC p) {
             float mine = acc[0];
 #pragma unroll
             for (int r = 1; r < 8; ++r) mine = lane == r ? acc[r] : mine;
-            out[i0 + lane * 8] = __float2bfloat16_rn(mine);
+            out[i0 + lane * 8] = from_f<E>(mine);
         }
     }
 }
@@ -875,28 +878,29 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
-template <int NH, int HV, int ST>
+template <int NH, int HV, int ST, typename E>
 cudaError_t launch_attn(const DecMaps& maps, const DecTC& p, size_t smem, cudaStream_t st) {
     static size_t done[64] = {0};
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64) dev = 0;
-    cudaError_t e = ensure_smem(k_dec_attn_sh<NH, HV, ST>, smem, &done[dev]);
+    cudaError_t e = ensure_smem(k_dec_attn_sh<NH, HV, ST, E>, smem, &done[dev]);
     if (e != cudaSuccess) return note_error("cudaFuncSetAttribute(k_dec_attn_sh)", e);
     return note_error("k_dec_attn_sh launch",
-                      launch_pdl(k_dec_attn_sh<NH, HV, ST>, dim3(p.G), dim3(kAttnThreads), smem, st, maps, p));
+                      launch_pdl(k_dec_attn_sh<NH, HV, ST, E>, dim3(p.G), dim3(kAttnThreads), smem, st, maps, p));
 }
 
+template <typename E>
 cudaError_t launch_attn_any(const DecMaps& maps, const DecTC& p, size_t smem, cudaStream_t st) {
     if (p.compact) {
-        if (p.Hp == 8) return launch_attn<16, 8, 3>(maps, p, smem, st);
-        return launch_attn<16, 16, 3>(maps, p, smem, st);
+        if (p.Hp == 8) return launch_attn<16, 8, 3, E>(maps, p, smem, st);
+        return launch_attn<16, 16, 3, E>(maps, p, smem, st);
     }
     switch (p.Hp) {
-        case 8: return launch_attn<16, 8, 2>(maps, p, smem, st);
-        case 16: return launch_attn<16, 16, 2>(maps, p, smem, st);
-        case 24: return launch_attn<32, 24, 2>(maps, p, smem, st);
-        default: return launch_attn<32, 32, 2>(maps, p, smem, st);
+        case 8: return launch_attn<16, 8, 2, E>(maps, p, smem, st);
+        case 16: return launch_attn<16, 16, 2, E>(maps, p, smem, st);
+        case 24: return launch_attn<32, 24, 2, E>(maps, p, smem, st);
+        default: return launch_attn<32, 32, 2, E>(maps, p, smem, st);
     }
 }
 
@@ -942,7 +946,8 @@ size_t tc_decode_workspace(const Shape& sh) {
            align256((size_t)(kMaxGrid + sh.B) * ((sh.H + 7) & ~7) * (sh.d_c + 2) * sizeof(float));
 }
 
-cudaError_t tc_decode(const DecodeArgs& a, cudaStream_t st, uint64_t* launches) {
+template <typename E>
+cudaError_t tc_decode_impl(const DecodeArgs& a, cudaStream_t st, uint64_t* launches) {
     const Shape& sh = a.sh;
     char* ws = (char*)a.workspace;
     uint8_t* qimg = (uint8_t*)ws;
@@ -963,7 +968,8 @@ cudaError_t tc_decode(const DecodeArgs& a, cudaStream_t st, uint64_t* launches) 
         // the latent map (64-column SW128 boxes), then the RoPE map (one
         // 32-column SW64 box starting at column d_c: 2 * d_c bytes, 16-aligned)
         cuuint32_t box[3] = {m == 0 ? 64u : 32u, (cuuint32_t)kTileSlots, 1};
-        CUresult r = encode(m == 0 ? &maps.lat : &maps.rope, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.cache, dims,
+        CUresult r = encode(m == 0 ? &maps.lat : &maps.rope,
+                            std::is_same<E, f16>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, a.cache, dims,
                             strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                             m == 0 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -1002,20 +1008,20 @@ cudaError_t tc_decode(const DecodeArgs& a, cudaStream_t st, uint64_t* launches) 
         int dev = 0;
         cudaGetDevice(&dev);
         if (dev >= 0 && dev < 64 && !carve[dev]) {
-            cudaFuncSetAttribute(k_dec_prep_tc, cudaFuncAttributePreferredSharedMemoryCarveout,
+            cudaFuncSetAttribute(k_dec_prep_tc<E>, cudaFuncAttributePreferredSharedMemoryCarveout,
                                  cudaSharedmemCarveoutMaxShared);
-            cudaFuncSetAttribute(k_dec_combine, cudaFuncAttributePreferredSharedMemoryCarveout,
+            cudaFuncSetAttribute(k_dec_combine<E>, cudaFuncAttributePreferredSharedMemoryCarveout,
                                  cudaSharedmemCarveoutMaxShared);
             cudaGetLastError();
             carve[dev] = true;
         }
     }
-    cudaError_t e = launch_pdl(k_dec_prep_tc, dim3(sh.B, sh.H + 1), dim3(kPrepAbsThreads + 32), 0, st, a, qimg,
+    cudaError_t e = launch_pdl(k_dec_prep_tc<E>, dim3(sh.B, sh.H + 1), dim3(kPrepAbsThreads + 32), 0, st, a, qimg,
                                p.qimg_bytes, p.n_chunks, NH, p.compact);
     if (e != cudaSuccess) return note_error("k_dec_prep_tc launch", e);
     const size_t smem = attn_smem_bytes(sh, compact ? 3 : 2);
     profile_begin(st);
-    e = launch_attn_any(maps, p, smem, st);
+    e = launch_attn_any<E>(maps, p, smem, st);
     profile_end(st);
     if (e != cudaSuccess) return e;
     const size_t comb_smem = (size_t)sh.d_h * sh.d_c * sizeof(bf16);
@@ -1024,12 +1030,16 @@ cudaError_t tc_decode(const DecodeArgs& a, cudaStream_t st, uint64_t* launches) 
         int dev = 0;
         cudaGetDevice(&dev);
         if (dev < 0 || dev >= 64) dev = 0;
-        e = ensure_smem(k_dec_combine, comb_smem, &done[dev]);
+        e = ensure_smem(k_dec_combine<E>, comb_smem, &done[dev]);
         if (e != cudaSuccess) return note_error("cudaFuncSetAttribute(k_dec_combine)", e);
     }
-    e = launch_pdl(k_dec_combine, dim3(sh.H, sh.B), dim3(256), comb_smem, st, a, p);
+    e = launch_pdl(k_dec_combine<E>, dim3(sh.H, sh.B), dim3(256), comb_smem, st, a, p);
     *launches += 3;
     return note_error("k_dec_combine launch", e);
+}
+
+cudaError_t tc_decode(const DecodeArgs& a, cudaStream_t st, uint64_t* launches) {
+    return a.sh.dtype == kDtypeF16 ? tc_decode_impl<f16>(a, st, launches) : tc_decode_impl<bf16>(a, st, launches);
 }
 
 }  // namespace mtla

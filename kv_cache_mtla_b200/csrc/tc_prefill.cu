@@ -64,15 +64,15 @@ struct PreTC {
     int n_items;      // n_qtiles * B * H
     float scale_log2;
     double log2_rope_base;
-    const bf16* q_r;  // [B, T, H, d_r]
+    const void* q_r;  // [B, T, H, d_r], storage type
     const float2* rope_tab;   // [T, d_r / 2]: (cos, sin) of every position, from the scan
-    bf16* out;        // [B, T, H, d_h]
+    void* out;        // [B, T, H, d_h], storage type
     // kept for the training backward when not null (t0 = 0): per row the
     // log2-domain log-sum-exp [B, H, T], O / l [B, T, H, d_c] and the absorbed
     // query as the score MMAs used it [B, T, H, D], bf16
     float* lse;
-    bf16* obar;
-    bf16* qt;
+    void* obar;       // bf16
+    void* qt;         // bf16
     int* status;
 };
 
@@ -120,8 +120,7 @@ __device__ __forceinline__ void st_row32_packed(uint8_t* base, uint32_t chunk_by
 }
 
 // bf16 halves of a packed pair as fp32 (exact: bf16 is the top half of fp32).
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
 
 // Work item idx (heaviest first): query tile qt = n_qtiles - 1 - idx / (B H),
 // then sequence and head.
@@ -168,7 +167,7 @@ __device__ __forceinline__ int item_at(const PreTC& p, int j) {
 //   - O_lat of item j goes to TMEM (bf16, the output MMA's A operand), so the
 //     absorption of item j+1 into the O columns starts as soon as O is read;
 //   - item j+1's key tiles load as soon as the P.V of item j frees the stages.
-template <int DC>
+template <int DC, typename E>
 __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constant__ Maps maps, const PreTC p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -301,9 +300,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
     } else if (warp == 1) {
         // ------------------------------------------------------------ absorption, score and output MMAs
         if (lane == 0) {
-            const uint32_t id_abs = idesc_bf16_f32(128, DC, false, true);
-            const uint32_t id_s = idesc_bf16_f32(128, kKT, false, false);
-            const uint32_t id_out = idesc_bf16_f32(128, kDh, false, false);
+            const uint32_t id_abs = idesc_f32<E>(128, DC, false, true);
+            const uint32_t id_s = idesc_f32<E>(128, kKT, false, false);
+            const uint32_t id_out = idesc_f32<E>(128, kDh, false, false);
             const uint32_t ring_a = smem_u32(ring), q_a = smem_u32(q_s);
             const uint64_t q_d = sdesc_sw128(q_a, 16, 1024), q_r = sdesc_sw64(q_a + NL * kQ * 128);
             const uint64_t qc_d = sdesc_sw128(smem_u32(qc_s), 16, 1024);
@@ -371,7 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
         // ------------------------------------------------------------ P.V MMAs (own thread: they free
         // ring stages, so they never wait behind a score MMA that waits for a load)
         if (lane == 0) {
-            const uint32_t id_o = idesc_bf16_f32(128, DC, false, true);
+            const uint32_t id_o = idesc_f32<E>(128, DC, false, true);
             const uint32_t ring_a = smem_u32(ring);
             int R = 0, G = 0;
             bool ok = true;
@@ -426,11 +425,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
             // (v holds the block in fp32; it is rounded once, into packed pairs w)
             auto put_q = [&](int col) {
 #pragma unroll
-                for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+                for (int i = 0; i < 16; ++i) w[i] = pack2<E>(v[2 * i], v[2 * i + 1]);
                 if (col < DC) st_row32_packed(q_s, kQ * 128, r, col, w, false);
                 else st_row32_packed(q_s + NL * kQ * 128, 0, r, col - DC, w, true);
                 if (p.qt && row_ok) {
-                    uint4* g = (uint4*)(p.qt + (((size_t)b * p.T + pos) * p.H + h) * p.D + col);
+                    uint4* g = (uint4*)((bf16*)p.qt + (((size_t)b * p.T + pos) * p.H + h) * p.D + col);
 #pragma unroll
                     for (int u = 0; u < 4; ++u) g[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
                 }
@@ -448,7 +447,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
             // the same rounded values.
             constexpr int n_blk = NL * 2 + 1, nb0 = (n_blk + 1) / 2;
             const int blk0 = hc == 0 ? 0 : nb0, blk1 = hc == 0 ? nb0 : n_blk;   // <= 5 blocks each
-            const bf16* qr = p.q_r + (((size_t)b * p.T + min(pos, p.T - 1)) * p.H + h) * p.d_r;
+            const E* qr = (const E*)p.q_r + (((size_t)b * p.T + min(pos, p.T - 1)) * p.H + h) * p.d_r;
             const float2* cs_row = p.rope_tab + (size_t)min(pos, p.T - 1) * (p.d_r / 2);
             waitb(&bs.abs_done, j & 1, bs);
             waitb(&bs.full[ppos & 1], (ppos >> 1) & 1, bs);
@@ -475,14 +474,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
                             cs4[u] = make_float4(1.f, 0.f, 1.f, 0.f);
                             if (e0 + 4 * u < p.d_r) cs4[u] = *(const float4*)(cs_row + e0 / 2 + 2 * u);
                         }
-                        const bf16* qe = (const bf16*)qv;
+                        const E* qe = (const E*)qv;
                         const float* csv = (const float*)cs4;      // cos, sin of pair i / 2
 #pragma unroll
                         for (int i = 0; i < 32; i += 2) {
                             v[i] = v[i + 1] = 0.f;
                             if (row_ok && e0 + i < p.d_r) {
                                 const float cs = csv[i], sn = csv[i + 1];
-                                const float x0 = __bfloat162float(qe[i]), x1 = __bfloat162float(qe[i + 1]);
+                                const float x0 = to_f<E>(qe[i]), x1 = to_f<E>(qe[i + 1]);
                                 v[i] = x0 * cs - x1 * sn;
                                 v[i + 1] = x0 * sn + x1 * cs;
                             }
@@ -496,8 +495,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
                         const uint32_t rw[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
-                            e2[0] = fmaf(bf16_lo(w[4 * u + i]), bf16_lo(rw[i]), e2[0]);
-                            e2[1] = fmaf(bf16_hi(w[4 * u + i]), bf16_hi(rw[i]), e2[1]);
+                            e2[0] = fmaf(lo_of<E>(w[4 * u + i]), lo_of<E>(rw[i]), e2[0]);
+                            e2[1] = fmaf(hi_of<E>(w[4 * u + i]), hi_of<E>(rw[i]), e2[1]);
                         }
                     }
                     e_own += e2[0] + e2[1];
@@ -520,9 +519,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
                         const uint4 raw = own8(cc + 8 * u);
-                        const bf16* pe = (const bf16*)&raw;
+                        const E* pe = (const E*)&raw;
 #pragma unroll
-                        for (int i = 0; i < 8; ++i) v[8 * u + i] = __bfloat162float(pe[i]);
+                        for (int i = 0; i < 8; ++i) v[8 * u + i] = to_f<E>(pe[i]);
                     }
                     tmem_st32(t_o + cc + lane_off, v);
                 }
@@ -573,7 +572,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
                     const float q0 = ex2_approx(fmaf(sv[2 * c], p.scale_log2, -nm));
                     const float q1 = ex2_approx(fmaf(sv[2 * c + 1], p.scale_log2, -nm));
                     rs4[c & 3] += q0 + q1;
-                    w[c] = pack_bf16x2(q0, q1);
+                    w[c] = pack2<E>(q0, q1);
                 }
                 l = fmaf(l, fac, (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
                 // O holds the own slot and this item's tiles 0..k-1
@@ -617,10 +616,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
                     tmem_ld32(t_o + cc + lane_off, v);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(v[2 * i] * inv, v[2 * i + 1] * inv);
+                    for (int i = 0; i < 16; ++i) w[i] = pack2<E>(v[2 * i] * inv, v[2 * i + 1] * inv);
                     tmem_st16_u(t_olat + cc / 2 + lane_off, w);
                     if (p.obar && row_ok) {
-                        uint4* g = (uint4*)(p.obar + (((size_t)b * p.T + pos) * p.H + h) * DC + cc);
+                        uint4* g = (uint4*)((bf16*)p.obar + (((size_t)b * p.T + pos) * p.H + h) * DC + cc);
 #pragma unroll
                         for (int u = 0; u < 4; ++u)
                             g[u] = make_uint4(w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
@@ -637,14 +636,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_prefill_tc(const __grid_constan
                 tmem_ld32(t_out + cc + lane_off, v);
                 tmem_wait_ld();
                 if (row_ok) {
-                    bf16* o = p.out + (((size_t)b * p.T + pos) * p.H + h) * kDh + cc;
+                    E* o = (E*)p.out + (((size_t)b * p.T + pos) * p.H + h) * kDh + cc;
 #pragma unroll
                     for (int u = 0; u < 4; ++u) {
                         uint4 pk;
-                        pk.x = pack_bf16x2(v[8 * u + 0], v[8 * u + 1]);
-                        pk.y = pack_bf16x2(v[8 * u + 2], v[8 * u + 3]);
-                        pk.z = pack_bf16x2(v[8 * u + 4], v[8 * u + 5]);
-                        pk.w = pack_bf16x2(v[8 * u + 6], v[8 * u + 7]);
+                        pk.x = pack2<E>(v[8 * u + 0], v[8 * u + 1]);
+                        pk.y = pack2<E>(v[8 * u + 2], v[8 * u + 3]);
+                        pk.z = pack2<E>(v[8 * u + 4], v[8 * u + 5]);
+                        pk.w = pack2<E>(v[8 * u + 6], v[8 * u + 7]);
                         *(uint4*)(o + 8 * u) = pk;
                     }
                 }
@@ -687,9 +686,10 @@ size_t prefill_smem_bytes(const Shape& sh) {
 
 cudaError_t make_map(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* m, const void* base, int rank,
                      const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box, const char* what,
-                     CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
+                     CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B,
+                     CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
     cuuint32_t estr[5] = {1, 1, 1, 1, 1};
-    CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides, box, estr,
+    CUresult r = enc(m, dt, rank, const_cast<void*>(base), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {
@@ -700,13 +700,15 @@ cudaError_t make_map(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* m, cons
     return cudaSuccess;
 }
 
-// The compiled instances: d_h = 64, d_R = 32 and d_c = 256 or 128. Other
-// widths take the CUDA-core prefill.
+// The compiled instances: d_h = 64, d_R = 32, d_c = 256 or 128, bf16 or fp16
+// storage. Other widths take the CUDA-core prefill.
 using PrefillKernel = void (*)(Maps, PreTC);
 PrefillKernel prefill_kernel(const Shape& sh) {
     if (sh.d_h != kDh || sh.d_r != kDr) return nullptr;
-    if (sh.d_c == 256) return k_prefill_tc<256>;
-    if (sh.d_c == 128) return k_prefill_tc<128>;
+    const bool h16 = sh.dtype == kDtypeF16;
+    if (sh.dtype != kDtypeBF16 && !h16) return nullptr;
+    if (sh.d_c == 256) return h16 ? k_prefill_tc<256, f16> : k_prefill_tc<256, bf16>;
+    if (sh.d_c == 128) return h16 ? k_prefill_tc<128, f16> : k_prefill_tc<128, bf16>;
     return nullptr;
 }
 
@@ -726,7 +728,7 @@ static cudaError_t tc_prefill_impl(const PrefillArgs& a_in, const PrefillSave* s
     PrefillArgs a = a_in;
     const Shape& sh = a.sh;
     const int T = a.T;
-    bf16* P = (bf16*)a.workspace;
+    void* P = a.workspace;                  // the partial slots, storage type (2 bytes)
     {
         const size_t off = align256((size_t)sh.B * T * sh.D * sizeof(bf16)) +
                            align256((size_t)T * (sh.d_r / 2) * sizeof(float2));
@@ -734,6 +736,9 @@ static cudaError_t tc_prefill_impl(const PrefillArgs& a_in, const PrefillSave* s
         if (e != cudaSuccess) return e;
     }
     auto enc = (PFN_cuTensorMapEncodeTiled_v12000)tensor_map_encoder();
+    const CUtensorMapDataType DT =
+        sh.dtype == kDtypeF16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const auto S128 = CU_TENSOR_MAP_SWIZZLE_128B;
     if (!enc) return note_error("cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)", cudaErrorNotSupported);
     Maps maps;
     const cuuint64_t E = 2;
@@ -741,15 +746,15 @@ static cudaError_t tc_prefill_impl(const PrefillArgs& a_in, const PrefillSave* s
         cuuint64_t d[4] = {(cuuint64_t)sh.d_h, (cuuint64_t)sh.H, (cuuint64_t)T, (cuuint64_t)sh.B};
         cuuint64_t s[3] = {E * sh.d_h, E * sh.H * sh.d_h, E * T * sh.H * sh.d_h};
         cuuint32_t bx[4] = {64, 1, kQ, 1};
-        cudaError_t e = make_map(enc, &maps.qc, a.q_c, 4, d, s, bx, "q_c");
+        cudaError_t e = make_map(enc, &maps.qc, a.q_c, 4, d, s, bx, "q_c", S128, DT);
         if (e != cudaSuccess) return e;
     }
     {
         cuuint64_t d[3] = {(cuuint64_t)sh.d_c, (cuuint64_t)sh.d_h, (cuuint64_t)sh.H};
         cuuint64_t s[2] = {E * sh.d_c, E * sh.d_h * sh.d_c};
         cuuint32_t bx[3] = {64, (cuuint32_t)sh.d_h, 1};
-        cudaError_t e = make_map(enc, &maps.wuk, a.w_uk, 3, d, s, bx, "w_uk");
-        if (e == cudaSuccess) e = make_map(enc, &maps.wuv, a.w_uv, 3, d, s, bx, "w_uv");
+        cudaError_t e = make_map(enc, &maps.wuk, a.w_uk, 3, d, s, bx, "w_uk", S128, DT);
+        if (e == cudaSuccess) e = make_map(enc, &maps.wuv, a.w_uv, 3, d, s, bx, "w_uv", S128, DT);
         if (e != cudaSuccess) return e;
     }
     {
@@ -758,10 +763,10 @@ static cudaError_t tc_prefill_impl(const PrefillArgs& a_in, const PrefillSave* s
         cuuint64_t d[3] = {(cuuint64_t)sh.D, (cuuint64_t)n_slots, (cuuint64_t)sh.B};
         cuuint64_t s[2] = {E * sh.D, E * sh.max_slots * sh.D};
         cuuint32_t bx[3] = {64, kKT, 1};
-        cudaError_t e = make_map(enc, &maps.slots, a.cache_out, 3, d, s, bx, "cache_out");
+        cudaError_t e = make_map(enc, &maps.slots, a.cache_out, 3, d, s, bx, "cache_out", S128, DT);
         cuuint32_t bxr[3] = {kDr, kKT, 1};
         if (e == cudaSuccess)
-            e = make_map(enc, &maps.slots_r, a.cache_out, 3, d, s, bxr, "cache_out RoPE", CU_TENSOR_MAP_SWIZZLE_64B);
+            e = make_map(enc, &maps.slots_r, a.cache_out, 3, d, s, bxr, "cache_out RoPE", CU_TENSOR_MAP_SWIZZLE_64B, DT);
         if (e != cudaSuccess) return e;
     }
     {
@@ -770,9 +775,9 @@ static cudaError_t tc_prefill_impl(const PrefillArgs& a_in, const PrefillSave* s
         cuuint64_t s[2] = {E * sh.D, E * T * sh.D};
         cuuint32_t bx[3] = {64, kQ, 1};
         cuuint32_t bxr[3] = {kDr, kQ, 1};
-        cudaError_t e = make_map(enc, &maps.prow, P, 3, d, s, bx, "partial slots");
+        cudaError_t e = make_map(enc, &maps.prow, P, 3, d, s, bx, "partial slots", S128, DT);
         if (e == cudaSuccess)
-            e = make_map(enc, &maps.prow_r, P, 3, d, s, bxr, "partial slots RoPE", CU_TENSOR_MAP_SWIZZLE_64B);
+            e = make_map(enc, &maps.prow_r, P, 3, d, s, bxr, "partial slots RoPE", CU_TENSOR_MAP_SWIZZLE_64B, DT);
         if (e != cudaSuccess) return e;
     }
     PreTC p;
@@ -789,20 +794,23 @@ static cudaError_t tc_prefill_impl(const PrefillArgs& a_in, const PrefillSave* s
     p.n_items = p.n_qtiles * sh.B * sh.H;
     p.scale_log2 = sh.scale * 1.4426950408889634f;
     p.log2_rope_base = sh.log2_rope_base;
-    p.q_r = (const bf16*)a.q_r;
+    p.q_r = a.q_r;
     p.rope_tab = (const float2*)((char*)a.workspace + align256((size_t)sh.B * T * sh.D * sizeof(bf16)));
-    p.out = (bf16*)a.out;
+    p.out = a.out;
     p.lse = sv ? sv->lse : nullptr;
-    p.obar = sv ? (bf16*)sv->obar : nullptr;
-    p.qt = sv ? (bf16*)sv->qt : nullptr;
+    p.obar = sv ? sv->obar : nullptr;
+    p.qt = sv ? sv->qt : nullptr;
     p.status = a.status;
 
     const int n_slots = (a.t0 + T - 1) / sh.s - a.t0 / sh.s + 1;    // slots the chunk touches
-    if (sh.gate_mode >= 3)
-        k_prefill_scan_channel<bf16, bf16><<<dim3((n_slots + 7) / 8, sh.B), 256, 0, st>>>(a, P, (float2*)p.rope_tab);
-    else
-        k_prefill_scan<bf16, bf16><<<dim3((n_slots + 7) / 8, sh.B), 256, 0, st>>>(a, P, (float2*)p.rope_tab,
-                                                                              sv ? sv->w : nullptr);
+    const dim3 sg((n_slots + 7) / 8, sh.B);
+    if (sh.dtype == kDtypeF16) {
+        if (sh.gate_mode >= 3) k_prefill_scan_channel<f16, f16><<<sg, 256, 0, st>>>(a, (f16*)P, (float2*)p.rope_tab);
+        else k_prefill_scan<f16, f16><<<sg, 256, 0, st>>>(a, (f16*)P, (float2*)p.rope_tab, sv ? sv->w : nullptr);
+    } else {
+        if (sh.gate_mode >= 3) k_prefill_scan_channel<bf16, bf16><<<sg, 256, 0, st>>>(a, (bf16*)P, (float2*)p.rope_tab);
+        else k_prefill_scan<bf16, bf16><<<sg, 256, 0, st>>>(a, (bf16*)P, (float2*)p.rope_tab, sv ? sv->w : nullptr);
+    }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return note_error("k_prefill_scan launch", e);
 

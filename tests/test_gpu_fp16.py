@@ -99,3 +99,24 @@ def test_fp16_backward(mode):
     toks = inputs.tokens(wl, T)
     dout = inputs.grad_out(wl, T)
     check_all(wl, run_backward(wl, T, w, toks, dout), oracle_backward(wl, w, toks, dout), tol=BWD_TOL)
+
+
+@pytest.mark.parametrize("s", [1, 2, 4])
+def test_fp16_tensor_cores_prefill_and_decode(s):
+    """fp16 storage at the tensor-core widths (H=8, d_h=64, d_c=256, d_R=32):
+    the tensor-core prefill over 300 tokens (three 128-position tiles and a
+    ragged tail), then 12 decode steps on the small-head tensor-core decode;
+    every row, the cache and the open slot against the oracle."""
+    wl = inputs.SPEECH_DECODE.with_(dtype="fp16", B=3, s=s)
+    T, S = 300, 12
+    w = inputs.weights(wl)
+    toks = inputs.tokens(wl, T + S)
+    ref = _oracle_prefill(wl, w, toks)
+    n = (T + S + s - 1) // s
+    pb = Problem(wl, max_slots=n + 1, max_tokens=T, weights=w)
+    assert pb.buf.cache.dtype == torch.float16
+    o1 = np64(pb.prefill(toks, T))
+    dec = np.stack([np64(pb.decode(toks, T + k, [T + k] * wl.B)) for k in range(S)], axis=1)
+    assert rel_err(np.concatenate([o1, dec], axis=1), ref["out"]) <= TOL["fp16"]
+    assert rel_err(np64(pb.buf.cache[:, :n]), ref["cache"]) <= TOL["fp16"]
+    assert rel_err(np64(pb.buf.open_slot), ref["acc"]) <= 1e-5
