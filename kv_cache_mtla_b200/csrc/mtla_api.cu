@@ -125,15 +125,16 @@ static mtla_status check_config(const mtla_config* cfg, Shape* sh) {
 }
 
 // bf16 and fp16 decode run on the tensor cores where the shape fits the
-// kernel (heads <= 32, d_c a multiple of 128, slot width <= 384); bf16 with
+// kernel (heads <= 32, d_c a multiple of 128, slot width <= 384), and with
 // 32 < heads <= 128 on the cluster kernel; fp32 and the other shapes on the
 // CUDA-core kernels.
 static bool use_tc_decode(const mtla_config* cfg, const Shape& sh) {
     return (cfg->dtype == MTLA_BF16 || cfg->dtype == MTLA_FP16) && tc_decode_supported(sh);
 }
-// bf16 with 32 < heads <= 128: the cluster kernel with all heads as M = 128.
+// bf16 or fp16 with 32 < heads <= 128: the cluster kernel with all heads as M = 128.
 static bool use_tc_decode_lh(const mtla_config* cfg, const Shape& sh) {
-    return cfg->dtype == MTLA_BF16 && !tc_decode_supported(sh) && tc_decode_lh_supported(sh);
+    return (cfg->dtype == MTLA_BF16 || cfg->dtype == MTLA_FP16) && !tc_decode_supported(sh) &&
+           tc_decode_lh_supported(sh);
 }
 
 static size_t decode_ws(const mtla_config* cfg, const Shape& sh) {

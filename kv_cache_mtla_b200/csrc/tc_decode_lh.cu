@@ -29,6 +29,7 @@
 
 #include <cstdio>
 #include <algorithm>
+#include <type_traits>
 #include <utility>
 
 #include <cuda_fp16.h>
@@ -89,6 +90,7 @@ __device__ __forceinline__ bool lh_pos_ok(const Shape& sh, int64_t t) {
 // updates (gate, RoPE key, open slot; MTLA Method (1)) of the group's
 // sequences b with b mod H = h, and the zero rows H..127 of their images.
 constexpr int kPrepThreads = 256;
+template <typename E>
 __global__ void __launch_bounds__(kPrepThreads, 1)
     k_lh_prep(const __grid_constant__ CUtensorMap wuk_map, DecodeArgs a, uint8_t* qimg, int n_qchunks) {
     pdl_launch_dependents();
@@ -125,7 +127,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
         const int bb = e / (n_qc * 8), rem = e % (n_qc * 8), c = rem >> 3, u = rem & 7;
         const int b = c0 + bb, col = c * 64 + u * 8;
         uint4 v = make_uint4(0, 0, 0, 0);
-        if (b < sh.B && col < sh.d_h) v = *(const uint4*)((const bf16*)a.q_c + ((size_t)b * sh.H + h) * sh.d_h + col);
+        if (b < sh.B && col < sh.d_h) v = *(const uint4*)((const E*)a.q_c + ((size_t)b * sh.H + h) * sh.d_h + col);
         *(uint4*)(x_s + (size_t)c * 4096 + sw128_offset(bb, u * 8)) = v;
     }
     fence_proxy_async();
@@ -135,7 +137,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
     const uint32_t t_d = *tmem_slot;
     if (tid == 0) {
         bool ok = true;
-        const uint32_t idesc = idesc_bf16_f32(128, 32, true, false);
+        const uint32_t idesc = idesc_f32<E>(128, 32, true, false);
         const uint64_t ad = sdesc_sw128(smem_u32(w_s), 16384, 1024), bd = sdesc_sw128(smem_u32(x_s), 16, 1024);
         for (int kb = 0; kb < n_kb && ok; ++kb) {
             if (kb > 0) {
@@ -178,7 +180,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
             qv[i] = 0;
             if (bb < 32 && b < sh.B) {
                 tv[i] = a.pos[b];
-                if (2 * k < sh.d_r) qv[i] = *(const uint32_t*)((const bf16*)a.q_r + ((size_t)b * sh.H + h) * sh.d_r + 2 * k);
+                if (2 * k < sh.d_r) qv[i] = *(const uint32_t*)((const E*)a.q_r + ((size_t)b * sh.H + h) * sh.d_r + 2 * k);
             }
         }
 #pragma unroll
@@ -187,8 +189,8 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
             if (bb >= 32 || b >= sh.B || !lh_pos_ok(sh, tv[i])) continue;
             float v0 = 0.f, v1 = 0.f;
             if (2 * k < sh.d_r) {
-                const bf16* xq = (const bf16*)&qv[i];
-                const float x0 = __bfloat162float(xq[0]), x1 = __bfloat162float(xq[1]);
+                const E* xq = (const E*)&qv[i];
+                const float x0 = to_f<E>(xq[0]), x1 = to_f<E>(xq[1]);
                 float sn, cs;
                 pair_sincos_f(tv[i], rope_freq[k], &sn, &cs);
                 v0 = x0 * cs - x1 * sn;
@@ -196,7 +198,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
             }
             const int j = sh.d_c + 2 * k;
             *(uint32_t*)(qimg + (size_t)b * img_bytes + (size_t)(j >> 6) * 128 * 128 + sw128_offset(h, j & 63)) =
-                pack_bf16x2(v0, v1);
+                pack2<E>(v0, v1);
         }
     }
     // latent part: warp w reads TMEM lane quarter w mod 4 (latent rows), sequences
@@ -219,7 +221,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
 #pragma unroll
             for (int s = 0; s < 16; ++s) {
                 const int bb = half * 16 + s;
-                *(bf16*)(stage + ((size_t)bb * n_kc + (j >> 6)) * 128 + in_row) = __float2bfloat16_rn(v[s]);
+                *(E*)(stage + ((size_t)bb * n_kc + (j >> 6)) * 128 + in_row) = from_f<E>(v[s]);
             }
         }
     }
@@ -236,7 +238,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
     // in-place slot updates of this group's sequences b with b mod H = h
     for (int b = c0 + ((h - c0 % sh.H) % sh.H + sh.H) % sh.H; b < min(sh.B, c0 + 32); b += sh.H) {
         __syncthreads();
-        decode_update_body<bf16>(a, b);
+        decode_update_body<E>(a, b);
         uint8_t* img = qimg + (size_t)b * img_bytes;
         const int pad_rows = 128 - sh.H;
         for (int e = tid; e < n_qchunks * pad_rows * 8; e += kPrepThreads) {
@@ -327,6 +329,7 @@ struct LhWalk {
 // handlers of rank 1 (rescale of O when a row's reference maximum moves,
 // zeroing of cache rows past a sequence's last slot, writing O at the end of a
 // sequence segment). One partial (O, m, l) per sequence segment.
+template <typename E>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     k_lh_attn(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v, const LhArgs p) {
     extern __shared__ uint8_t smem_raw[];
@@ -467,7 +470,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             if (rank == 0) {
                 // -------------------------------------------------------- score MMAs
-                const uint32_t id_s = idesc_bf16_f32(128, kKT, false, false);
+                const uint32_t id_s = idesc_f32<E>(128, kKT, false, false);
                 const uint32_t t_s = tmem, t_q = tmem + 128;
                 LhWalk w = w0;
                 int it = 0, seg = -1;
@@ -512,7 +515,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 }
             } else {
                 // -------------------------------------------------------- P.V MMAs
-                const uint32_t id_o = idesc_bf16_f32(128, p.unit_cols, false, true);
+                const uint32_t id_o = idesc_f32<E>(128, p.unit_cols, false, true);
                 LhWalk w = w0;
                 int it = 0, ev = 0, ocnt = 0;
                 auto post = [&](int type, int arg) -> bool {
@@ -674,7 +677,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 const float p0 = ex2_approx(fmaf(sv[2 * c], p.scale_log2, -nm));
                 const float p1 = ex2_approx(fmaf(sv[2 * c + 1], p.scale_log2, -nm));
                 rs4[c & 3] += p0 + p1;
-                pk[c] = pack_bf16x2(p0, p1);
+                pk[c] = pack2<E>(p0, p1);
             }
             l = fmaf(l, fac, (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
             m_ref = nm;
@@ -842,6 +845,7 @@ __device__ void lh_tile_starts(const LhArgs& p, int* starts, int* warp_tot) {
 //   C. out^T [d_h x 32] = W_UV[h] [d_h x d_c] . o_lat^T  (tcgen05, M = 128, N = 32)
 //      with W_UV[h] brought in by TMA before the wait for the attention kernel.
 constexpr int kCombThreads = 512;
+template <typename E>
 __global__ void __launch_bounds__(kCombThreads, 1)
     k_lh_combine(const __grid_constant__ CUtensorMap wuv_map, DecodeArgs a, LhArgs p) {
     extern __shared__ uint8_t smem_raw[];
@@ -963,8 +967,8 @@ __global__ void __launch_bounds__(kCombThreads, 1)
 #pragma unroll
                 for (int s2 = 0; s2 < 2; ++s2) {
                     uint2 pk;
-                    pk.x = pack_bf16x2(o[s2][0], o[s2][1]);
-                    pk.y = pack_bf16x2(o[s2][2], o[s2][3]);
+                    pk.x = pack2<E>(o[s2][0], o[s2][1]);
+                    pk.y = pack2<E>(o[s2][2], o[s2][3]);
                     *(uint2*)(o_s + (size_t)(k >> 6) * 4096 + sw128_offset(bb + s2, k & 63)) = pk;
                 }
             }
@@ -990,7 +994,7 @@ __global__ void __launch_bounds__(kCombThreads, 1)
             ok = mbar_wait(&bars[0], mb & 1);
             if (!ok) break;
             tc_fence_after();
-            const uint32_t idesc = idesc_bf16_f32(128, 32, false, false);
+            const uint32_t idesc = idesc_f32<E>(128, 32, false, false);
             const uint64_t ad = sdesc_sw128(smem_u32(w_s), 16, 1024), bd = sdesc_sw128(smem_u32(o_s), 16, 1024);
             for (int kc = 0; kc < n_kc; ++kc) {
 #pragma unroll
@@ -1017,7 +1021,7 @@ __global__ void __launch_bounds__(kCombThreads, 1)
             for (int s8 = 0; s8 < 8; ++s8) {
                 const int b = c0 + oct * 8 + s8;
                 if (b < sh.B && starts[b + 1] > starts[b])
-                    ((bf16*)a.out)[((size_t)b * sh.H + h) * sh.d_h + i] = __float2bfloat16_rn(v[s8]);
+                    ((E*)a.out)[((size_t)b * sh.H + h) * sh.d_h + i] = from_f<E>(v[s8]);
             }
         }
     }
@@ -1093,7 +1097,8 @@ size_t tc_decode_lh_workspace(const Shape& sh) {
            align256((size_t)(kMaxClusters + sh.B) * sh.H * (sh.d_c + 4) * sizeof(float));
 }
 
-cudaError_t tc_decode_lh(const DecodeArgs& a, cudaStream_t st, uint64_t* launches) {
+template <typename E>
+cudaError_t tc_decode_lh_impl(const DecodeArgs& a, cudaStream_t st, uint64_t* launches) {
     const Shape& sh = a.sh;
     uint8_t* qimg = (uint8_t*)a.workspace;
     float* part = (float*)((char*)a.workspace + align256((size_t)sh.B * (sh.D / 64) * 128 * 128));
@@ -1114,7 +1119,7 @@ cudaError_t tc_decode_lh(const DecodeArgs& a, cudaStream_t st, uint64_t* launche
         cuuint32_t box[4] = {64, (cuuint32_t)(m == 0 ? kKT : kHalf),
                              (cuuint32_t)(m == 0 ? kChunksPerStage : std::min(256, sh.d_c) / 64), 1};
         cuuint32_t estr[4] = {1, 1, 1, 1};
-        r = encode(m == 0 ? &map_k : &map_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, a.cache, dims, strides, box, estr,
+        r = encode(m == 0 ? &map_k : &map_v, (std::is_same<E, f16>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16), 4, a.cache, dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) {
@@ -1131,7 +1136,7 @@ cudaError_t tc_decode_lh(const DecodeArgs& a, cudaStream_t st, uint64_t* launche
         cuuint64_t s2[1] = {(cuuint64_t)sh.d_c * 2};
         cuuint32_t b2[2] = {64, 128};
         cuuint32_t e2[2] = {1, 1};
-        r = encode(w == 0 ? &wuk_map : &wuv_map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+        r = encode(w == 0 ? &wuk_map : &wuv_map, (std::is_same<E, f16>::value ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16), 2,
                    const_cast<void*>(w == 0 ? a.w_uk : a.w_uv), d2, s2, b2, e2, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) {
@@ -1159,9 +1164,9 @@ cudaError_t tc_decode_lh(const DecodeArgs& a, cudaStream_t st, uint64_t* launche
     const size_t attn_smem = lh_attn_smem();
     p.smem_bytes = (uint32_t)attn_smem;
     const size_t comb_smem = lh_comb_smem(sh);
-    cudaError_t e = lh_set_smem(k_lh_prep, prep_smem, &done_prep[dev]);
-    if (e == cudaSuccess) e = lh_set_smem(k_lh_attn, attn_smem, &done_attn[dev]);
-    if (e == cudaSuccess) e = lh_set_smem(k_lh_combine, comb_smem, &done_comb[dev]);
+    cudaError_t e = lh_set_smem(k_lh_prep<E>, prep_smem, &done_prep[dev]);
+    if (e == cudaSuccess) e = lh_set_smem(k_lh_attn<E>, attn_smem, &done_attn[dev]);
+    if (e == cudaSuccess) e = lh_set_smem(k_lh_combine<E>, comb_smem, &done_comb[dev]);
     if (e != cudaSuccess) return note_error("cudaFuncSetAttribute(large-head decode)", e);
     if (!co_resident[dev]) {
         // clusters that can be resident at once: the balanced split assumes one wave
@@ -1170,7 +1175,7 @@ cudaError_t tc_decode_lh(const DecodeArgs& a, cudaStream_t st, uint64_t* launche
         oc.blockDim = dim3(kThreads);
         oc.dynamicSmemBytes = attn_smem;
         int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, k_lh_attn, &oc) != cudaSuccess || n <= 0) {
+        if (cudaOccupancyMaxActiveClusters(&n, k_lh_attn<E>, &oc) != cudaSuccess || n <= 0) {
             cudaGetLastError();
             n = sm_count() / 2;
         }
@@ -1184,16 +1189,20 @@ cudaError_t tc_decode_lh(const DecodeArgs& a, cudaStream_t st, uint64_t* launche
     p.part = part;
     p.status = a.status;
 
-    k_lh_prep<<<dim3(sh.H, (sh.B + 31) / 32), kPrepThreads, prep_smem, st>>>(wuk_map, a, qimg, p.n_qchunks);
+    k_lh_prep<E><<<dim3(sh.H, (sh.B + 31) / 32), kPrepThreads, prep_smem, st>>>(wuk_map, a, qimg, p.n_qchunks);
     e = cudaGetLastError();
     if (e != cudaSuccess) return note_error("k_lh_prep launch", e);
     profile_begin(st);
-    e = launch_pdl_lh(k_lh_attn, dim3(2 * p.G2), dim3(kThreads), attn_smem, st, map_k, map_v, p);
+    e = launch_pdl_lh(k_lh_attn<E>, dim3(2 * p.G2), dim3(kThreads), attn_smem, st, map_k, map_v, p);
     profile_end(st);
     if (e != cudaSuccess) return note_error("k_lh_attn launch", e);
-    e = launch_pdl_lh(k_lh_combine, dim3(sh.H, (sh.B + 31) / 32), dim3(kCombThreads), comb_smem, st, wuv_map, a, p);
+    e = launch_pdl_lh(k_lh_combine<E>, dim3(sh.H, (sh.B + 31) / 32), dim3(kCombThreads), comb_smem, st, wuv_map, a, p);
     *launches += 3;
     return note_error("k_lh_combine launch", e);
+}
+
+cudaError_t tc_decode_lh(const DecodeArgs& a, cudaStream_t st, uint64_t* launches) {
+    return a.sh.dtype == kDtypeF16 ? tc_decode_lh_impl<f16>(a, st, launches) : tc_decode_lh_impl<bf16>(a, st, launches);
 }
 
 }  // namespace mtla

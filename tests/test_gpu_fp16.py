@@ -120,3 +120,21 @@ def test_fp16_tensor_cores_prefill_and_decode(s):
     assert rel_err(np.concatenate([o1, dec], axis=1), ref["out"]) <= TOL["fp16"]
     assert rel_err(np64(pb.buf.cache[:, :n]), ref["cache"]) <= TOL["fp16"]
     assert rel_err(np64(pb.buf.open_slot), ref["acc"]) <= 1e-5
+
+
+def test_fp16_large_heads_cluster_decode():
+    """fp16 storage at the large-latent widths (H=128, d_h=128, d_c=512,
+    d_R=64, s=4, supplied gates): the 2-CTA cluster decode over a prompt of 90
+    tokens (CUDA-core prefill at these widths) and 6 steps, against the
+    oracle."""
+    wl = inputs.LARGE_LATENT.with_(dtype="fp16", B=2)
+    T, S = 90, 6
+    w = inputs.weights(wl)
+    toks = inputs.tokens(wl, T + S)
+    ref = _oracle_prefill(wl, w, toks)
+    n = (T + S + wl.s - 1) // wl.s
+    pb = Problem(wl, max_slots=n + 2, max_tokens=T, weights=w)
+    o1 = np64(pb.prefill(toks, T))
+    dec = np.stack([np64(pb.decode(toks, T + k, [T + k] * wl.B)) for k in range(S)], axis=1)
+    assert rel_err(np.concatenate([o1, dec], axis=1), ref["out"]) <= TOL["fp16"]
+    assert rel_err(np64(pb.buf.open_slot), ref["acc"]) <= 1e-5
