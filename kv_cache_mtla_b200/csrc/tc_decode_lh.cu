@@ -122,6 +122,9 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
     __shared__ double rope_freq[64];                      // base^(-2k / d_r), d_r / 2 <= 64
     for (int k = tid; k < sh.d_r / 2; k += kPrepThreads)
         rope_freq[k] = exp2(-(2.0 * k / (double)sh.d_r) * sh.log2_rope_base);
+    // everything above reads weights only; the step's inputs (and the cache this
+    // step updates) only once the previous kernel in the stream has completed
+    pdl_wait();
     // qC rows of the 32 sequences (zero past B) as the K-major B operand
     for (int e = tid; e < 32 * n_qc * 8; e += kPrepThreads) {
         const int bb = e / (n_qc * 8), rem = e % (n_qc * 8), c = rem >> 3, u = rem & 7;
@@ -848,6 +851,7 @@ constexpr int kCombThreads = 512;
 template <typename E>
 __global__ void __launch_bounds__(kCombThreads, 1)
     k_lh_combine(const __grid_constant__ CUtensorMap wuv_map, DecodeArgs a, LhArgs p) {
+    pdl_launch_dependents();   // the next step's prep may stage its W_UK rows now
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const Shape& sh = a.sh;
@@ -1189,8 +1193,8 @@ cudaError_t tc_decode_lh_impl(const DecodeArgs& a, cudaStream_t st, uint64_t* la
     p.part = part;
     p.status = a.status;
 
-    k_lh_prep<E><<<dim3(sh.H, (sh.B + 31) / 32), kPrepThreads, prep_smem, st>>>(wuk_map, a, qimg, p.n_qchunks);
-    e = cudaGetLastError();
+    e = launch_pdl_lh(k_lh_prep<E>, dim3(sh.H, (sh.B + 31) / 32), dim3(kPrepThreads), prep_smem, st, wuk_map, a, qimg,
+                      p.n_qchunks);
     if (e != cudaSuccess) return note_error("k_lh_prep launch", e);
     profile_begin(st);
     e = launch_pdl_lh(k_lh_attn<E>, dim3(2 * p.G2), dim3(kThreads), attn_smem, st, map_k, map_v, p);
