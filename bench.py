@@ -913,7 +913,7 @@ def run_contract(args, ws, rank):
         torch.cuda.empty_cache()
         extras["layer"] = measure_layer(400, flush, ws, rank)
         torch.cuda.empty_cache()
-        extras["backward"] = measure_backward(40, flush, ws, rank)
+        extras["backward"] = measure_backward(120, flush, ws, rank)
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         n_seq = 8
