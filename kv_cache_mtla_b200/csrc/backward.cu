@@ -1,7 +1,11 @@
 // backward.cu -- training backward of the parallel (prefill) forward from
 // position 0 ("Multi-head Temporal Latent Attention", Results: the models are
 // trained from scratch; Key claims: the stride-aware mask lets the parallel
-// training pass match incremental decoding), on the CUDA cores in fp32.
+// training pass match incremental decoding). Two paths behind one entry:
+// bf16 at the tensor-core prefill's widths runs the masked attention's
+// gradients on the tensor cores (tc_backward.cu) around the CUDA-core kernels
+// here; every other shape and storage type runs the CUDA-core path below,
+// in fp32 arithmetic.
 //
 // Forward, per sequence: x_u = [c_u ; R_u k_u], P_t = sum_{u in block(t), u <= t}
 // w_u x_u (w_u the merging weight of Eq. 13); query i of head h attends the
@@ -19,7 +23,7 @@
 //   dx_u = w_u S_u, dw_u = x_u . S_u; dc_u = dx_u[0:d_c], dk_u = R_u^T dx_u[d_c:];
 //   the gate: dz = dw w (1 - w), dG[r] += dz (c_u * PE_u), dg[r] += dz,
 //   dc_u += dz (G[r] * PE_u), r = u mod s; a supplied gate gets dgate_in = dw.
-// Kernels, in launch order:
+// CUDA-core path, kernels in launch order:
 //   k_prefill_scan    the forward scan (P in fp32, the weights w)
 //   k_prefill_absorb  the absorbed queries qt (fp32)
 //   k_bwd_rows        block (i, b), a warp per head: the row's softmax (two
@@ -32,6 +36,11 @@
 //   k_bwd_query       dqC, dqR
 //   k_bwd_wpart/wsum  dW_UK, dW_UV (per row chunk, then the chunks in order)
 //   k_bwd_scan        a warp per slot: the scan and gate backward
+// Tensor-core path (backward_tc): the forward on the tensor cores keeping each
+// row's log-sum-exp, O / l and absorbed query; dobar and U (GEMMs), delta
+// (k_bwd_delta); the finished-slot gradients (k_bwd_dq_tc, k_bwd_dk_tc); the
+// own-partial term with dqR (k_bwd_own); dqC (GEMM); then k_bwd_wpart/wsum and
+// k_bwd_scan as above, the heads' dF summed in a fixed order.
 #include <type_traits>
 
 #include "common.cuh"
