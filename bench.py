@@ -508,6 +508,16 @@ def measure_backward(n, flush, ws, rank):
         mtla.prefill_backward(cfg, T, d["c"], d["kr"], d["qc"], d["qr"], dw["w_uk"], dw["w_uv"], dw["gate_w"],
                               dw["gate_b"], None, dout, grads, wsb)
     call_ms, kern_ms, clocks = _timed_calls(call, n, flush, ws)
+    # the training pair: the forward keeping the backward's rows, and the
+    # backward from them (no forward recompute)
+    saved = torch.empty(mtla.prefill_train_saved_size(cfg, T), dtype=torch.uint8, device="cuda")
+    out_t = torch.empty(B, T, H, wl.d_h, device="cuda", dtype=torch.bfloat16)
+    ws_s = torch.empty(mtla.prefill_backward_saved_workspace_size(cfg, T), dtype=torch.uint8, device="cuda")
+    targs = (d["c"], d["kr"], d["qc"], d["qr"], dw["w_uk"], dw["w_uv"], dw["gate_w"], dw["gate_b"], None)
+    fwd_ms, _, _ = _timed_calls(lambda: mtla.prefill_train(cfg, T, *targs, out_t, saved), n, flush, ws,
+                                profile=False)
+    bws_ms, _, _ = _timed_calls(lambda: mtla.prefill_backward_saved(cfg, T, *targs, saved, dout, grads, ws_s), n,
+                                flush, ws, profile=False)
     pairs = sum(t // wl.s + 1 for t in range(T))
     # per (row, key) pair: the score and dobar.key dot products, dq, dkey and its
     # latent (value) part: 2 (3 D + 2 d_c) flops
@@ -516,6 +526,8 @@ def measure_backward(n, flush, ws, rank):
     return {"workload": f"training backward: B={B}/rank, T={T}, H={H}, d_h={wl.d_h}, d_c={wl.d_c}, "
                         f"d_R={wl.d_r}, s={wl.s}, computed gates, bf16 inputs, fp32 gradients",
             "TFLOPs": flops * ws / (call_ms / 1e3) / 1e12, "call_ms": call_ms,
+            "training_pair": {"forward_keeping_rows_ms": fwd_ms, "backward_from_kept_rows_ms": bws_ms,
+                              "note": "mtla_prefill_train then mtla_prefill_backward_saved: no forward recompute"},
             "attention_flops_per_call": flops, "calls": n,
             "roofline": {"kernel": "k_bwd_dq_tc + k_bwd_dk_tc (masked attention backward, tensor cores)",
                          "bound": "tensor", "achieved": kern, "peak": tflops_peak, "unit": "TFLOP/s",

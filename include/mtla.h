@@ -246,6 +246,36 @@ mtla_status mtla_prefill_backward(const mtla_config* cfg, int32_t T,
                                   float* dgate_w, float* dgate_b, float* dgate_in,
                                   void* workspace, size_t workspace_bytes, void* stream);
 
+/* The training pair, where the backward runs on the tensor cores (bf16 storage,
+ * d_h = 64, d_r = 32, d_c = 128 or 256, scalar gates; UNSUPPORTED otherwise):
+ * a forward that keeps what the backward needs (per row the log-sum-exp, O / l
+ * and the absorbed query; the partial slots, the slots and the merging
+ * weights), and a backward from it that does not recompute the forward.
+ * mtla_prefill_train: arguments as for mtla_prefill from position 0 without
+ * the cache outputs; `out` receives the same output; `saved` (device memory
+ * of at least mtla_prefill_train_saved_size bytes, 16-byte aligned, owned by
+ * the caller) receives the kept rows. mtla_prefill_backward_saved: arguments,
+ * outputs and errors as for mtla_prefill_backward, plus `saved` from a
+ * mtla_prefill_train call on the same config, T and inputs (not checked: a
+ * different `saved` gives wrong gradients), and its own (smaller) workspace.
+ * Both return OK once enqueued on `stream`. */
+mtla_status mtla_prefill_train_saved_size(const mtla_config* cfg, int32_t T, size_t* bytes);
+mtla_status mtla_prefill_backward_saved_workspace_size(const mtla_config* cfg, int32_t T, size_t* bytes);
+mtla_status mtla_prefill_train(const mtla_config* cfg, int32_t T,
+                               const void* c, const void* kr, const void* q_c, const void* q_r,
+                               const void* w_uk, const void* w_uv,
+                               const float* gate_w, const float* gate_b, const float* gate_in,
+                               void* out, void* saved, size_t saved_bytes, void* stream);
+mtla_status mtla_prefill_backward_saved(const mtla_config* cfg, int32_t T,
+                                        const void* c, const void* kr, const void* q_c, const void* q_r,
+                                        const void* w_uk, const void* w_uv,
+                                        const float* gate_w, const float* gate_b, const float* gate_in,
+                                        const void* saved, const void* dout,
+                                        float* dc, float* dkr, float* dq_c, float* dq_r,
+                                        float* dw_uk, float* dw_uv,
+                                        float* dgate_w, float* dgate_b, float* dgate_in,
+                                        void* workspace, size_t workspace_bytes, void* stream);
+
 /* Dense projection on the tensor cores: y[M, N] = x[M, K] . w[N, K]^T with
  * bf16 operands and result and fp32 accumulation. The layer around the path
  * ("Multi-head Temporal Latent Attention", Method: MLA's low-rank compression

@@ -727,30 +727,50 @@ cudaError_t backward_impl(const PrefillArgs& pa_in, const BackwardGrads& g, cuda
 
 // ---------------------------------------------------------------- tensor-core path
 
-struct BwdTcWs {
-    size_t fwd, cache, out, lse, delta, obar, qt, w, dob, dqt, dF, dP, wuvt, dqtl, part_k, part_v, u, total;
-};
-
 Shape with_slots(const Shape& sh, int T) {
     Shape s2 = sh;
     s2.max_slots = (T + sh.s - 1) / sh.s;
     return s2;
 }
 
-BwdTcWs bwd_tc_layout(const Shape& sh_in, int T) {
+// What the training forward keeps for the backward (tensor-core path): the
+// forward's own scratch (its first region the partial slots P, bf16), the
+// slots, each row's log2-domain log-sum-exp, O / l, the absorbed query, and
+// the merging weights.
+struct SavedWs {
+    size_t fwd, cache, lse, obar, qt, w, total;
+};
+
+SavedWs saved_layout(const Shape& sh_in, int T) {
     const Shape sh = with_slots(sh_in, T);
     const size_t BT = (size_t)sh.B * T, rows = BT * sh.H;
-    BwdTcWs l;
+    SavedWs l;
     size_t o = 0;
     auto take = [&](size_t bytes) { size_t at = o; o += align256(bytes); return at; };
-    l.fwd = take(tc_prefill_workspace(sh, T));            // its first region: the partial slots P (bf16)
+    l.fwd = take(tc_prefill_workspace(sh, T));
     l.cache = take((size_t)sh.B * sh.max_slots * sh.D * 2);
-    l.out = take(rows * sh.d_h * 2);
     l.lse = take((size_t)sh.B * sh.H * stats_pitch(T) * 4);
-    l.delta = take((size_t)sh.B * sh.H * stats_pitch(T) * 4);
     l.obar = take(rows * sh.d_c * 2);
     l.qt = take(rows * sh.D * 2);
     l.w = take(BT * 4);
+    l.total = o;
+    return l;
+}
+
+// The backward's own scratch, after the saved rows when it recomputes them
+// (`base` = their size; `out` then takes the recomputed forward's output).
+struct BwdTcWs {
+    size_t out, delta, dob, dqt, dF, dP, wuvt, dqtl, part_k, part_v, u, total;
+};
+
+BwdTcWs bwd_tc_layout(const Shape& sh_in, int T, size_t base, bool recompute) {
+    const Shape sh = with_slots(sh_in, T);
+    const size_t BT = (size_t)sh.B * T, rows = BT * sh.H;
+    BwdTcWs l;
+    size_t o = base;
+    auto take = [&](size_t bytes) { size_t at = o; o += align256(bytes); return at; };
+    l.out = recompute ? take(rows * sh.d_h * 2) : 0;
+    l.delta = take((size_t)sh.B * sh.H * stats_pitch(T) * 4);
     l.dob = take(rows * sh.d_c * 2);
     l.dqt = take(rows * sh.D * 4);
     l.dF = take((size_t)sh.H * sh.B * sh.max_slots * sh.D * 4);
@@ -764,29 +784,49 @@ BwdTcWs bwd_tc_layout(const Shape& sh_in, int T) {
     return l;
 }
 
+// The forward on the tensor cores from position 0, keeping the rows the
+// backward needs in `sv` (saved_layout); `out` receives the forward's output.
+cudaError_t train_forward(const PrefillArgs& pa_in, char* sv, void* out, cudaStream_t st, uint64_t* launches) {
+    const int T_len = pa_in.T;
+    PrefillArgs pa = pa_in;
+    pa.sh = with_slots(pa_in.sh, T_len);
+    const SavedWs S = saved_layout(pa.sh, T_len);
+    pa.workspace = sv + S.fwd;
+    pa.workspace_bytes = tc_prefill_workspace(pa.sh, T_len);
+    pa.cache_out = sv + S.cache;
+    pa.out = out;
+    pa.open_slot_in = nullptr;
+    pa.open_slot_out = nullptr;
+    pa.t0 = 0;
+    PrefillSave keep;
+    keep.w = (float*)(sv + S.w);
+    keep.lse = (float*)(sv + S.lse);
+    keep.obar = sv + S.obar;
+    keep.qt = sv + S.qt;
+    return tc_prefill_save(pa, keep, st, launches);
+}
+
 bool use_tc(const Shape& sh, int dtype) {
     return dtype == kDtypeBF16 && tc_backward_supported(sh) && tc_prefill_supported(sh);
 }
 
-// bf16 at the tensor-core prefill's widths: the forward recomputed on the
-// tensor cores keeping its rows' statistics, dobar and delta, the finished-
-// slot parts on the tensor cores, the own-partial term, then the same query,
-// weight and scan/gate backward as the CUDA-core path (dF summed over heads).
-cudaError_t backward_tc(const PrefillArgs& pa_in, const BackwardGrads& g, cudaStream_t st, uint64_t* launches) {
+// bf16 at the tensor-core prefill's widths: the rows kept by the training
+// forward (`saved`; recomputed here into the workspace when it is null), dobar
+// and delta, the finished-slot parts on the tensor cores, the own-partial
+// term, then the same query, weight and scan/gate backward as the CUDA-core
+// path (dF summed over heads).
+cudaError_t backward_tc(const PrefillArgs& pa_in, const BackwardGrads& g, const void* saved, cudaStream_t st,
+                        uint64_t* launches) {
     const int T_len = pa_in.T;
     PrefillArgs pa = pa_in;
     pa.sh = with_slots(pa_in.sh, T_len);
     const Shape sh = pa.sh;
     const int n_slots = sh.max_slots;
     char* ws = (char*)pa.workspace;
-    const BwdTcWs l = bwd_tc_layout(sh, T_len);
-    pa.workspace = ws + l.fwd;
-    pa.workspace_bytes = tc_prefill_workspace(sh, T_len);
-    pa.cache_out = ws + l.cache;
-    pa.out = ws + l.out;
-    pa.open_slot_in = nullptr;
-    pa.open_slot_out = nullptr;
-    pa.t0 = 0;
+    const SavedWs S = saved_layout(sh, T_len);
+    const bool recompute = saved == nullptr;
+    const BwdTcWs l = bwd_tc_layout(sh, T_len, recompute ? S.total : 0, recompute);
+    char* sv = recompute ? ws : (char*)saved;
     cudaError_t e;
     if (sh.gate_mode == 0) {
         if ((e = cudaMemsetAsync(g.dgate_w, 0, (size_t)sh.s * sh.d_c * sizeof(float), st)) != cudaSuccess)
@@ -794,12 +834,7 @@ cudaError_t backward_tc(const PrefillArgs& pa_in, const BackwardGrads& g, cudaSt
         if ((e = cudaMemsetAsync(g.dgate_b, 0, (size_t)sh.s * sizeof(float), st)) != cudaSuccess)
             return note_error("backward zero dg", e);
     }
-    PrefillSave sv;
-    sv.w = (float*)(ws + l.w);
-    sv.lse = (float*)(ws + l.lse);
-    sv.obar = ws + l.obar;
-    sv.qt = ws + l.qt;
-    if ((e = tc_prefill_save(pa, sv, st, launches)) != cudaSuccess) return e;
+    if (recompute && (e = train_forward(pa_in, sv, ws + l.out, st, launches)) != cudaSuccess) return e;
     BwdArgs a;
     a.sh = sh;
     a.T = T_len;
@@ -810,10 +845,10 @@ cudaError_t backward_tc(const PrefillArgs& pa_in, const BackwardGrads& g, cudaSt
     a.dout = g.dout;
     a.P = nullptr;
     a.qt = nullptr;
-    a.w = (const float*)(ws + l.w);
+    a.w = (const float*)(sv + S.w);
     a.mrow = a.lrow = a.delta = nullptr;
     a.dob = nullptr;
-    a.obar = ws + l.obar;
+    a.obar = sv + S.obar;
     a.dqt = (float*)(ws + l.dqt);
     a.dP = (float*)(ws + l.dP);
     a.dF = (float*)(ws + l.dF);
@@ -830,21 +865,21 @@ cudaError_t backward_tc(const PrefillArgs& pa_in, const BackwardGrads& g, cudaSt
                      false, M, sh.d_c, sh.d_h, sh.H, pa.status, st, launches);
     if (e != cudaSuccess) return e;
     const int64_t rows = (int64_t)M * sh.H;
-    k_bwd_delta<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(sh, T_len, dob, (const bf16*)(ws + l.obar),
+    k_bwd_delta<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(sh, T_len, dob, (const bf16*)(sv + S.obar),
                                                              (float*)(ws + l.delta));
     if ((e = cudaGetLastError()) != cudaSuccess) return note_error("k_bwd_delta launch", e);
     // U_j[h] = W_UV[h] F_j[0:d_c] for every finished slot and head: one GEMM,
     // [B n_slots, d_c] . W_UV viewed as [H d_h, d_c]
-    e = gemm_batched(GemmOperand{ws + l.cache, sh.D, 0}, GemmOperand{pa.w_uv, sh.d_c, 0}, ws + l.u, sh.H * sh.d_h, 0,
+    e = gemm_batched(GemmOperand{sv + S.cache, sh.D, 0}, GemmOperand{pa.w_uv, sh.d_c, 0}, ws + l.u, sh.H * sh.d_h, 0,
                      false, sh.B * n_slots, sh.H * sh.d_h, sh.d_c, 1, pa.status, st, launches);
     if (e != cudaSuccess) return e;
     BwdTCInputs in;
-    in.qt = ws + l.qt;
+    in.qt = sv + S.qt;
     in.dob = ws + l.dob;
-    in.slots = ws + l.cache;
+    in.slots = sv + S.cache;
     in.dout = g.dout;
     in.u = ws + l.u;
-    in.lse = (const float*)(ws + l.lse);
+    in.lse = (const float*)(sv + S.lse);
     in.delta = (const float*)(ws + l.delta);
     in.dqt = a.dqt;
     in.dF = a.dF;
@@ -854,7 +889,7 @@ cudaError_t backward_tc(const PrefillArgs& pa_in, const BackwardGrads& g, cudaSt
     profile_end(st);
     if (e != cudaSuccess) return e;
     bf16* dqtl = (bf16*)(ws + l.dqtl);
-    k_bwd_own<<<dim3(T_len, sh.B), threads, 0, st>>>(a, (const bf16*)(ws + l.qt), (const bf16*)(ws + l.fwd), dob,
+    k_bwd_own<<<dim3(T_len, sh.B), threads, 0, st>>>(a, (const bf16*)(sv + S.qt), (const bf16*)(sv + S.fwd), dob,
                                                       in.lse, in.delta, dqtl, g.dq_r);
     if ((e = cudaGetLastError()) != cudaSuccess) return note_error("k_bwd_own launch", e);
     // dqC = dqt[0:d_c] . W_UK[h]^T on the tensor cores, fp32 out
@@ -874,12 +909,26 @@ cudaError_t backward_tc(const PrefillArgs& pa_in, const BackwardGrads& g, cudaSt
 }  // namespace
 
 size_t prefill_backward_workspace(const Shape& sh, int T, int dtype) {
-    return use_tc(sh, dtype) ? bwd_tc_layout(sh, T).total : bwd_layout(sh, T, dtype_bytes(dtype)).total;
+    return use_tc(sh, dtype) ? bwd_tc_layout(sh, T, saved_layout(sh, T).total, true).total
+                             : bwd_layout(sh, T, dtype_bytes(dtype)).total;
+}
+
+bool prefill_train_supported(const Shape& sh) { return use_tc(sh, sh.dtype); }
+size_t prefill_train_saved_bytes(const Shape& sh, int T) { return saved_layout(sh, T).total; }
+size_t prefill_backward_saved_workspace(const Shape& sh, int T) { return bwd_tc_layout(sh, T, 0, false).total; }
+
+cudaError_t prefill_train(const PrefillArgs& a, void* saved, cudaStream_t st, uint64_t* launches) {
+    return train_forward(a, (char*)saved, a.out, st, launches);
+}
+
+cudaError_t prefill_backward_saved(const PrefillArgs& a, const BackwardGrads& g, const void* saved, cudaStream_t st,
+                                   uint64_t* launches) {
+    return backward_tc(a, g, saved, st, launches);
 }
 
 cudaError_t prefill_backward(const PrefillArgs& a, const BackwardGrads& g, int dtype, cudaStream_t st,
                              uint64_t* launches) {
-    if (use_tc(a.sh, dtype)) return backward_tc(a, g, st, launches);
+    if (use_tc(a.sh, dtype)) return backward_tc(a, g, nullptr, st, launches);
     if (dtype == kDtypeF32) return backward_impl<float>(a, g, st, launches);
     if (dtype == kDtypeF16) return backward_impl<f16>(a, g, st, launches);
     return backward_impl<bf16>(a, g, st, launches);

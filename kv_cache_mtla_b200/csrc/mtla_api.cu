@@ -360,6 +360,104 @@ mtla_status mtla_prefill_backward(const mtla_config* cfg, int32_t T, const void*
     return e == cudaSuccess ? MTLA_OK : MTLA_ERR_CUDA;
 }
 
+static mtla_status train_check(const mtla_config* cfg, int32_t T, Shape* sh) {
+    mtla_status st = backward_check(cfg, T, sh);
+    if (st != MTLA_OK) return st;
+    return prefill_train_supported(*sh) ? MTLA_OK : MTLA_ERR_UNSUPPORTED;
+}
+
+mtla_status mtla_prefill_train_saved_size(const mtla_config* cfg, int32_t T, size_t* bytes) {
+    Shape sh;
+    if (!bytes) return MTLA_ERR_INVALID_ARG;
+    mtla_status st = train_check(cfg, T, &sh);
+    if (st != MTLA_OK) return st;
+    *bytes = prefill_train_saved_bytes(sh, T);
+    return MTLA_OK;
+}
+
+mtla_status mtla_prefill_backward_saved_workspace_size(const mtla_config* cfg, int32_t T, size_t* bytes) {
+    Shape sh;
+    if (!bytes) return MTLA_ERR_INVALID_ARG;
+    mtla_status st = train_check(cfg, T, &sh);
+    if (st != MTLA_OK) return st;
+    *bytes = prefill_backward_saved_workspace(sh, T);
+    return MTLA_OK;
+}
+
+static PrefillArgs train_args(const Shape& sh, int32_t T, const void* c, const void* kr, const void* q_c,
+                              const void* q_r, const void* w_uk, const void* w_uv, const float* gate_w,
+                              const float* gate_b, const float* gate_in) {
+    PrefillArgs a = {};
+    a.sh = sh;
+    a.T = T;
+    a.c = c;
+    a.kr = kr;
+    a.q_c = q_c;
+    a.q_r = q_r;
+    a.w_uk = w_uk;
+    a.w_uv = w_uv;
+    a.gate_w = gate_w;
+    a.gate_b = gate_b;
+    a.gate_in = gate_in;
+    return a;
+}
+
+mtla_status mtla_prefill_train(const mtla_config* cfg, int32_t T, const void* c, const void* kr, const void* q_c,
+                               const void* q_r, const void* w_uk, const void* w_uv, const float* gate_w,
+                               const float* gate_b, const float* gate_in, void* out, void* saved, size_t saved_bytes,
+                               void* stream) {
+    Shape sh;
+    mtla_status st = train_check(cfg, T, &sh);
+    if (st != MTLA_OK) return st;
+    const void* req[] = {c, kr, q_c, q_r, w_uk, w_uv, out, saved};
+    for (const void* p : req)
+        if (!p || !aligned16(p)) return MTLA_ERR_INVALID_ARG;
+    st = check_gate_ptrs(cfg, gate_w, gate_b, gate_in);
+    if (st != MTLA_OK) return st;
+    if (saved_bytes < prefill_train_saved_bytes(sh, T)) return MTLA_ERR_WORKSPACE;
+    PrefillArgs a = train_args(sh, T, c, kr, q_c, q_r, w_uk, w_uv, gate_w, gate_b, gate_in);
+    a.out = out;
+    g_error_detail[0] = 0;
+    if (note_error("device status word", status_ptr(&a.status)) != cudaSuccess) return MTLA_ERR_CUDA;
+    uint64_t n = 0;
+    cudaError_t e = prefill_train(a, saved, (cudaStream_t)stream, &n);
+    g_launches += n;
+    if (e != cudaSuccess && !g_error_detail[0]) note_error("training forward launch", e);
+    return e == cudaSuccess ? MTLA_OK : MTLA_ERR_CUDA;
+}
+
+mtla_status mtla_prefill_backward_saved(const mtla_config* cfg, int32_t T, const void* c, const void* kr,
+                                        const void* q_c, const void* q_r, const void* w_uk, const void* w_uv,
+                                        const float* gate_w, const float* gate_b, const float* gate_in,
+                                        const void* saved, const void* dout, float* dc, float* dkr, float* dq_c,
+                                        float* dq_r, float* dw_uk, float* dw_uv, float* dgate_w, float* dgate_b,
+                                        float* dgate_in, void* workspace, size_t workspace_bytes, void* stream) {
+    Shape sh;
+    mtla_status st = train_check(cfg, T, &sh);
+    if (st != MTLA_OK) return st;
+    const void* req[] = {c, kr, q_c, q_r, w_uk, w_uv, saved, dout, dc, dkr, dq_c, dq_r, dw_uk, dw_uv, workspace};
+    for (const void* p : req)
+        if (!p || !aligned16(p)) return MTLA_ERR_INVALID_ARG;
+    st = check_gate_ptrs(cfg, gate_w, gate_b, gate_in);
+    if (st != MTLA_OK) return st;
+    if (cfg->gate_mode == MTLA_GATE_COMPUTED &&
+        (!dgate_w || !dgate_b || !aligned16(dgate_w) || !aligned16(dgate_b)))
+        return MTLA_ERR_INVALID_ARG;
+    if (cfg->gate_mode == MTLA_GATE_SUPPLIED && (!dgate_in || !aligned16(dgate_in))) return MTLA_ERR_INVALID_ARG;
+    if (workspace_bytes < prefill_backward_saved_workspace(sh, T)) return MTLA_ERR_WORKSPACE;
+    PrefillArgs a = train_args(sh, T, c, kr, q_c, q_r, w_uk, w_uv, gate_w, gate_b, gate_in);
+    a.workspace = workspace;
+    a.workspace_bytes = workspace_bytes;
+    BackwardGrads g = {dout, dc, dkr, dq_c, dq_r, dw_uk, dw_uv, dgate_w, dgate_b, dgate_in};
+    g_error_detail[0] = 0;
+    if (note_error("device status word", status_ptr(&a.status)) != cudaSuccess) return MTLA_ERR_CUDA;
+    uint64_t n = 0;
+    cudaError_t e = prefill_backward_saved(a, g, saved, (cudaStream_t)stream, &n);
+    g_launches += n;
+    if (e != cudaSuccess && !g_error_detail[0]) note_error("backward launch", e);
+    return e == cudaSuccess ? MTLA_OK : MTLA_ERR_CUDA;
+}
+
 mtla_status mtla_linear(const void* x, const void* w, void* y, int32_t M, int32_t N, int32_t K, void* stream) {
     if (M <= 0 || N <= 0 || K <= 0 || K % 8 != 0) return MTLA_ERR_INVALID_ARG;
     if (!x || !w || !y || !aligned16(x) || !aligned16(w) || !aligned16(y)) return MTLA_ERR_INVALID_ARG;

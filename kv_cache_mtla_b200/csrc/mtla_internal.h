@@ -153,6 +153,15 @@ struct BackwardGrads {
     float* dgate_in;       // [B,T] (supplied gate)
 };
 size_t prefill_backward_workspace(const Shape& sh, int T, int dtype);
+// The training pair (bf16 at the tensor-core widths, scalar gates, t0 = 0):
+// the forward keeping what the backward needs in `saved`, and the backward
+// from it (no forward recompute).
+bool prefill_train_supported(const Shape& sh);
+size_t prefill_train_saved_bytes(const Shape& sh, int T);
+size_t prefill_backward_saved_workspace(const Shape& sh, int T);
+cudaError_t prefill_train(const PrefillArgs& a, void* saved, cudaStream_t st, uint64_t* launches);
+cudaError_t prefill_backward_saved(const PrefillArgs& a, const BackwardGrads& g, const void* saved, cudaStream_t st,
+                                   uint64_t* launches);
 cudaError_t prefill_backward(const PrefillArgs& a, const BackwardGrads& g, int dtype, cudaStream_t st,
                              uint64_t* launches);
 

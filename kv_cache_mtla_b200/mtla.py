@@ -92,6 +92,14 @@ def load() -> ctypes.CDLL:
     lib.mtla_prefill_backward_workspace_size.restype = ctypes.c_int
     lib.mtla_prefill_backward.argtypes = [cp, ctypes.c_int32] + [_vp] * 19 + [_vp, ctypes.c_size_t, _vp]
     lib.mtla_prefill_backward.restype = ctypes.c_int
+    lib.mtla_prefill_train_saved_size.argtypes = [cp, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)]
+    lib.mtla_prefill_train_saved_size.restype = ctypes.c_int
+    lib.mtla_prefill_backward_saved_workspace_size.argtypes = [cp, ctypes.c_int32, ctypes.POINTER(ctypes.c_size_t)]
+    lib.mtla_prefill_backward_saved_workspace_size.restype = ctypes.c_int
+    lib.mtla_prefill_train.argtypes = [cp, ctypes.c_int32] + [_vp] * 11 + [ctypes.c_size_t, _vp]
+    lib.mtla_prefill_train.restype = ctypes.c_int
+    lib.mtla_prefill_backward_saved.argtypes = [cp, ctypes.c_int32] + [_vp] * 20 + [_vp, ctypes.c_size_t, _vp]
+    lib.mtla_prefill_backward_saved.restype = ctypes.c_int
     lib.mtla_linear.argtypes = [_vp, _vp, _vp, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _vp]
     lib.mtla_linear.restype = ctypes.c_int
     lp = ctypes.POINTER(LayerWeights)
@@ -242,6 +250,48 @@ def prefill_backward(cfg, T, c, kr, q_c, q_r, w_uk, w_uv, gate_w, gate_b, gate_i
         _ptr(workspace), ws, _stream(stream))
     if check and st != OK:
         raise MtlaError(st, "mtla_prefill_backward")
+    return st
+
+
+def prefill_train_saved_size(cfg: Config, T: int) -> int:
+    n = ctypes.c_size_t(0)
+    st = load().mtla_prefill_train_saved_size(ctypes.byref(cfg), int(T), ctypes.byref(n))
+    if st != OK:
+        raise MtlaError(st, "mtla_prefill_train_saved_size")
+    return int(n.value)
+
+
+def prefill_backward_saved_workspace_size(cfg: Config, T: int) -> int:
+    n = ctypes.c_size_t(0)
+    st = load().mtla_prefill_backward_saved_workspace_size(ctypes.byref(cfg), int(T), ctypes.byref(n))
+    if st != OK:
+        raise MtlaError(st, "mtla_prefill_backward_saved_workspace_size")
+    return int(n.value)
+
+
+def prefill_train(cfg, T, c, kr, q_c, q_r, w_uk, w_uv, gate_w, gate_b, gate_in, out, saved, stream=None,
+                  check=True) -> int:
+    """Forward to ``mtla_prefill_train`` (the forward keeping the backward's
+    rows in ``saved``, a uint8 device tensor)."""
+    st = load().mtla_prefill_train(
+        ctypes.byref(cfg), int(T), _ptr(c), _ptr(kr), _ptr(q_c), _ptr(q_r), _ptr(w_uk), _ptr(w_uv), _ptr(gate_w),
+        _ptr(gate_b), _ptr(gate_in), _ptr(out), _ptr(saved), saved.numel() * saved.element_size(), _stream(stream))
+    if check and st != OK:
+        raise MtlaError(st, "mtla_prefill_train")
+    return st
+
+
+def prefill_backward_saved(cfg, T, c, kr, q_c, q_r, w_uk, w_uv, gate_w, gate_b, gate_in, saved, dout,
+                           grads: dict, workspace, stream=None, check=True) -> int:
+    """Forward to ``mtla_prefill_backward_saved``; ``grads`` as for
+    prefill_backward."""
+    ws = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    st = load().mtla_prefill_backward_saved(
+        ctypes.byref(cfg), int(T), _ptr(c), _ptr(kr), _ptr(q_c), _ptr(q_r), _ptr(w_uk), _ptr(w_uv),
+        _ptr(gate_w), _ptr(gate_b), _ptr(gate_in), _ptr(saved), _ptr(dout),
+        *[_ptr(grads.get(k)) for k in BACKWARD_GRADS], _ptr(workspace), ws, _stream(stream))
+    if check and st != OK:
+        raise MtlaError(st, "mtla_prefill_backward_saved")
     return st
 
 

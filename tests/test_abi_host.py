@@ -240,6 +240,22 @@ def test_backward_rejects_bad_arguments_on_the_host(lib):
     assert call(cfg, 100, [None, None, fake], plain + [None, None, fake], n) == mtla.ERR_UNSUPPORTED
 
 
+def test_training_pair_sizes_and_refusals(lib):
+    """The training pair exists where the backward runs on the tensor cores
+    (bf16, d_h=64, d_R=32, d_c 128 or 256, scalar gates): sizes there,
+    UNSUPPORTED elsewhere."""
+    cfg = _cfg()
+    assert mtla.prefill_train_saved_size(cfg, 300) > 0
+    assert 0 < mtla.prefill_backward_saved_workspace_size(cfg, 300) < mtla.prefill_backward_workspace_size(cfg, 300)
+    bad = [mtla.make_config(2, 8, 64, 256, 32, 2, 16, dtype="fp32"), _cfg(d_h=32), _cfg(d_c=512, d_r=64)]
+    chan = _cfg()
+    chan.gate_mode = mtla.GATE_CHANNEL_COMPUTED
+    for c in bad + [chan]:
+        with pytest.raises(mtla.MtlaError) as e:
+            mtla.prefill_train_saved_size(c, 300)
+        assert e.value.status == mtla.ERR_UNSUPPORTED
+
+
 def test_layer_refuses_fp32_and_bad_widths_on_the_host(lib):
     """The layer is bf16 only; d_model must be a positive multiple of 8."""
     cfg = _cfg()

@@ -189,3 +189,44 @@ def test_backward_is_repeatable(wl, T):
         assert torch.equal(g1[k], g2[k]), k
     for k in ("dw_uk", "dw_uv", "dgate_w", "dgate_b"):
         assert rel_err(np64(g1[k]), np64(g2[k])) <= 1e-6, k
+
+
+@pytest.mark.parametrize("mode", [inputs.GATE_COMPUTED, inputs.GATE_SUPPLIED])
+def test_training_pair_equals_backward(mode):
+    """mtla_prefill_train + mtla_prefill_backward_saved: the forward's output is
+    the bytes of mtla_prefill's, and the gradients are the bytes of
+    mtla_prefill_backward's (the same kernels on the same kept rows; the gate
+    gradients, sums of atomic additions, to rounding)."""
+    wl = inputs.PREFILL.with_(B=2, s=3, gate_mode=mode)
+    T = 300
+    w = inputs.weights(wl)
+    toks = inputs.tokens(wl, T)
+    dout = inputs.grad_out(wl, T)
+    ref = run_backward(wl, T, w, toks, dout)
+    cfg = mtla.make_config(wl.B, wl.H, wl.d_h, wl.d_c, wl.d_r, wl.s, (T + wl.s - 1) // wl.s, gate_mode=mode)
+    dt = torch.bfloat16
+    computed = mode == inputs.GATE_COMPUTED
+    args = [dev(toks["c"], dt), dev(toks["kr"], dt), dev(toks["qc"], dt), dev(toks["qr"], dt),
+            dev(w["w_uk"], dt), dev(w["w_uv"], dt),
+            dev(w["gate_w"], torch.float32) if computed else None,
+            dev(w["gate_b"], torch.float32) if computed else None,
+            dev(toks["gate_in"], torch.float32) if toks["gate_in"] is not None else None]
+    out_t = torch.empty(wl.B, T, wl.H, wl.d_h, device="cuda", dtype=dt)
+    saved = torch.empty(mtla.prefill_train_saved_size(cfg, T), dtype=torch.uint8, device="cuda")
+    mtla.prefill_train(cfg, T, *args, out_t, saved)
+    out_p = torch.empty_like(out_t)
+    cache = torch.zeros(wl.B, cfg.max_slots, wl.D, device="cuda", dtype=dt)
+    op = torch.zeros(wl.B, wl.D, device="cuda")
+    wsp = torch.empty(mtla.workspace_size(cfg, T), dtype=torch.uint8, device="cuda")
+    mtla.prefill(cfg, T, *args, out_p, cache, op, wsp)
+    torch.cuda.synchronize()
+    assert torch.equal(out_t, out_p)
+    grads = {k: torch.full_like(v, float("nan")) for k, v in ref.items()}
+    ws = torch.empty(mtla.prefill_backward_saved_workspace_size(cfg, T), dtype=torch.uint8, device="cuda")
+    mtla.prefill_backward_saved(cfg, T, *args, saved, dev(dout, dt), grads, ws)
+    torch.cuda.synchronize()
+    for k in ref:
+        if k in ("dgate_w", "dgate_b"):
+            assert rel_err(np64(grads[k]), np64(ref[k])) <= 1e-6, k
+        else:
+            assert torch.equal(grads[k], ref[k]), k
