@@ -73,8 +73,10 @@ struct MapsK {
     CUtensorMap lse, delta;     // (T, H, B) fp32: box (64, 1, 1)
 };
 
+constexpr int kQStages = 3;     // key-tile ring of k_bwd_dq_tc
+
 struct BarsQ {
-    uint64_t full[2], empty[2], q_full, sd_full, sd_free, ds_ready[2], ds_free[2], done, drain[2];
+    uint64_t full[kQStages], empty[kQStages], q_full, sd_full, sd_free, ds_ready[2], ds_free[2], done, drain[2];
     uint32_t tmem_base;
     volatile int fail;
 };
@@ -122,7 +124,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dq_tc(const __grid_constant
     uint8_t* q_s = smem;
     uint8_t* do_s = q_s + q_bytes;
     uint8_t* ring = do_s + do_bytes;
-    BarsQ& bs = *(BarsQ*)(ring + 2 * stage_bytes);
+    BarsQ& bs = *(BarsQ*)(ring + kQStages * stage_bytes);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int per_qt = p.B * p.H;
@@ -133,9 +135,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dq_tc(const __grid_constant
     const int nkt = (last / p.s + kN - 1) / kN;               // key tiles (finished slots of the last row)
 
     if (tid == 0) {
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < kQStages; ++i) {
             mbar_init(&bs.full[i], 1);
             mbar_init(&bs.empty[i], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
             mbar_init(&bs.ds_ready[i], 8);
             mbar_init(&bs.ds_free[i], 1);
             mbar_init(&bs.drain[i], 1);
@@ -168,13 +172,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dq_tc(const __grid_constant
             tma_load_4d(q_s + NL * kM * 128, &maps.q_r, &bs.q_full, DC, h, p0, b);
             tma_load_4d(do_s, &maps.dout, &bs.q_full, 0, h, p0, b);
             for (int k = 0; k < nkt; ++k) {
-                if (k >= 2 && !waitb(&bs.empty[k & 1], ((k >> 1) - 1) & 1, bs)) break;
-                uint8_t* dst = ring + (k & 1) * stage_bytes;
-                mbar_arrive_expect_tx(&bs.full[k & 1], stage_bytes);
+                const int sg = k % kQStages;
+                if (k >= kQStages && !waitb(&bs.empty[sg], ((k / kQStages) - 1) & 1, bs)) break;
+                uint8_t* dst = ring + sg * stage_bytes;
+                mbar_arrive_expect_tx(&bs.full[sg], stage_bytes);
 #pragma unroll
-                for (int c = 0; c < NL; ++c) tma_load_3d(dst + c * kchunk, &maps.k, &bs.full[k & 1], c * 64, kN * k, b);
-                tma_load_3d(dst + NL * kchunk, &maps.k_r, &bs.full[k & 1], DC, kN * k, b);
-                tma_load_3d(dst + u_off, &maps.u, &bs.full[k & 1], h * kDh, kN * k, b);
+                for (int c = 0; c < NL; ++c) tma_load_3d(dst + c * kchunk, &maps.k, &bs.full[sg], c * 64, kN * k, b);
+                tma_load_3d(dst + NL * kchunk, &maps.k_r, &bs.full[sg], DC, kN * k, b);
+                tma_load_3d(dst + u_off, &maps.u, &bs.full[sg], h * kDh, kN * k, b);
                 loads = k + 1;
             }
         }
@@ -191,7 +196,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dq_tc(const __grid_constant
             auto dq_mma = [&](int t) -> bool {
                 if (!waitb(&bs.ds_ready[t & 1], (t >> 1) & 1, bs)) return false;
                 tc_fence_after();
-                const uint32_t st_a = ring_a + (t & 1) * stage_bytes;
+                const uint32_t st_a = ring_a + (t % kQStages) * stage_bytes;
                 const uint64_t bl = sdesc_sw128(st_a, kchunk, 1024), br = sdesc_sw64_mn(st_a + NL * kchunk);
 #pragma unroll
                 for (int kk = 0; kk < kN / 16; ++kk) {
@@ -199,17 +204,17 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dq_tc(const __grid_constant
                     umma_bf16_ts(t_dq, t_ds + (t & 1) * 32 + kk * 8, desc_add(bl, kk * 2048), id_lat, acc);
                     umma_bf16_ts(t_dq + DC, t_ds + (t & 1) * 32 + kk * 8, desc_add(br, kk * 1024), id_rope, acc);
                 }
-                umma_commit(&bs.empty[t & 1]);
+                umma_commit(&bs.empty[t % kQStages]);
                 umma_commit(&bs.ds_free[t & 1]);
                 return true;
             };
             if (waitb(&bs.q_full, 0, bs)) {
                 bool ok = true;
                 for (int k = 0; k < nkt && ok; ++k) {
-                    if (!(ok = waitb(&bs.full[k & 1], (k >> 1) & 1, bs))) break;
+                    if (!(ok = waitb(&bs.full[k % kQStages], (k / kQStages) & 1, bs))) break;
                     if (k >= 1 && !(ok = waitb(&bs.sd_free, (k - 1) & 1, bs))) break;
                     tc_fence_after();
-                    const uint32_t st_a = ring_a + (k & 1) * stage_bytes;
+                    const uint32_t st_a = ring_a + (k % kQStages) * stage_bytes;
                     const uint64_t kd = sdesc_sw128(st_a, 16, 1024), kr = sdesc_sw64(st_a + NL * kchunk);
                     // S = qt . K^T (K = D); dPa = dobar . V^T = dout . U^T (K = d_h), U_j = W_UV[h] F_j
 #pragma unroll
@@ -302,7 +307,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dq_tc(const __grid_constant
         }
         if (warp == 0 && lane == 0) {
             if (loads > 0) mbar_wait(&bs.q_full, 0);
-            for (int k = max(0, loads - 2); k < loads; ++k) mbar_wait(&bs.full[k & 1], (k >> 1) & 1);
+            for (int k = max(0, loads - kQStages); k < loads; ++k)
+                mbar_wait(&bs.full[k % kQStages], (k / kQStages) & 1);
         }
         if (tid == 0) latch_status(p.status, kStatusTimeout);
         __syncthreads();
@@ -433,6 +439,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dk_tc(const __grid_constant
             if (waitb(&bs.k_full, 0, bs)) {
                 bool ok = true;
                 for (int k = 0; k < ntl && ok; ++k) {
+                    // the accumulating MMAs of tile k - 1 first: they release its ring
+                    // stage, so the load of tile k + 1 overlaps this tile's score MMAs
+                    // (with two stages, issuing them after S_k would leave every score
+                    // MMA waiting for a full load)
+                    if (k >= 1 && !(ok = dk_mma(k - 1))) break;
                     if (!(ok = waitb(&bs.full[k & 1], (k >> 1) & 1, bs))) break;
                     if (k >= 1 && !(ok = waitb(&bs.sd_free, (k - 1) & 1, bs))) break;
                     tc_fence_after();
@@ -456,7 +467,6 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dk_tc(const __grid_constant
                             umma_bf16(t_dp, desc_add(kd, c * kM * 128 + kk * 32), desc_add(dd, c * qchunk + kk * 32),
                                       id_s, (c | kk) != 0);
                     umma_commit(&bs.sd_full);
-                    if (k >= 1) ok = dk_mma(k - 1);
                 }
                 if (ok && dk_mma(ntl - 1)) umma_commit(&bs.done);
             }
@@ -550,8 +560,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd_dk_tc(const __grid_constant
 
 template <int DC>
 constexpr size_t dq_smem() {
-    return 1024 + (size_t)(DC / 64) * kM * 128 + kM * 64 + kM * 128 + 2 * ((DC / 64) * kN * 128 + kN * 64 + kN * 128) +
-           ((sizeof(BarsQ) + 15) & ~(size_t)15);
+    return 1024 + (size_t)(DC / 64) * kM * 128 + kM * 64 + kM * 128 +
+           kQStages * ((DC / 64) * kN * 128 + kN * 64 + kN * 128) + ((sizeof(BarsQ) + 15) & ~(size_t)15);
 }
 template <int DC>
 constexpr size_t dk_smem() {
