@@ -116,6 +116,8 @@ def _load():
         _lib.orc_set_fault.argtypes = [ctypes.c_int]
         _lib.orc_linear.argtypes = [ctypes.c_int64] * 3 + [_P] * 3
         _lib.orc_prefill_backward.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int32] + [_P] * 19
+        _lib.orc_backward_rows.argtypes = ([ctypes.POINTER(_Cfg), ctypes.c_int32] + [_P] * 10 +
+                                           [ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, _P, _P])
         _lib.orc_reorder_cache.argtypes = [ctypes.c_int32] * 5 + [ctypes.c_void_p] * 6
         _lib.orc_reorder_cache.restype = ctypes.c_int
     return _lib
@@ -288,6 +290,24 @@ def prefill_backward(cfg: Cfg, c, kr, qc, qr, w_uk, w_uv, dout, G=None, g=None, 
                                  *[_p(out[k]) for k in ("dc", "dkr", "dqc", "dqr", "dw_uk", "dw_uv", "dG", "dg",
                                                         "dgate_in")])
     return out
+
+
+def backward_rows(cfg: Cfg, c, kr, qc, qr, w_uk, w_uv, dout, rows, G=None, g=None, gate_in=None) -> dict:
+    """Query-side gradients dqc [n, H, d_h] and dqr [n, H, d_R] of the rows
+    [(b, i)] of the training backward, each computed alone
+    (``orc_backward_rows``)."""
+    c, kr, qc, qr, w_uk, w_uv, dout = map(_d, (c, kr, qc, qr, w_uk, w_uv, dout))
+    G, g, gate_in = _d(G), _d(g), _d(gate_in)
+    T = c.shape[1]
+    rb = np.ascontiguousarray([r[0] for r in rows], dtype=np.int32)
+    ri = np.ascontiguousarray([r[1] for r in rows], dtype=np.int32)
+    n = len(rows)
+    dqc = np.zeros((n, cfg.H, cfg.d_h))
+    dqr = np.zeros((n, cfg.H, cfg.d_r))
+    _load().orc_backward_rows(ctypes.byref(cfg.c()), T, _p(c), _p(kr), _p(qc), _p(qr), _p(w_uk), _p(w_uv),
+                              _p(G), _p(g), _p(gate_in), _p(dout), n, rb.ctypes.data, ri.ctypes.data, _p(dqc),
+                              _p(dqr))
+    return dict(dqc=dqc, dqr=dqr)
 
 
 def layer_forward(cfg: Cfg, t0: int, cache_in, acc_in, h, W: dict, G=None, g=None, gate_in=None):

@@ -735,6 +735,86 @@ void orc_prefill_backward(const orc_cfg* cfg, int32_t T, const double* c, const 
     free(dP); free(P); free(w);
 }
 
+/* The query-side gradients of selected rows of the same backward: for row
+ * (b, i) = (rows_b[r], rows_i[r]), dqc_out[r][h][:] and dqr_out[r][h][:] are
+ * the gradients of L = sum(dout * out) with respect to qC[b,i,h,:] and
+ * qR[b,i,h,:]. They depend only on that row's query, its keys (the finished
+ * slots before it and its own partial) and dout[b,i], so each is computed
+ * alone: the row's share of orc_prefill_backward's dqc / dqr, the same steps
+ * in the same order (for checks at sizes where the whole backward is too
+ * slow). */
+void orc_backward_rows(const orc_cfg* cfg, int32_t T, const double* c, const double* kr, const double* qc,
+                       const double* qr, const double* w_uk, const double* w_uv, const double* G, const double* g,
+                       const double* gate_in, const double* dout, int32_t n_rows, const int32_t* rows_b,
+                       const int32_t* rows_i, double* dqc_out, double* dqr_out) {
+    const int32_t B = cfg->B, H = cfg->H, d_h = cfg->d_h, d_c = cfg->d_c, d_r = cfg->d_r, s = cfg->s;
+    const int32_t D = d_c + d_r;
+    const double scale = orc_scale(cfg);
+    double* w = (double*)malloc(sizeof(double) * (size_t)B * T);
+    double* P = (double*)malloc(sizeof(double) * (size_t)B * T * D);
+    orc_partials(cfg, T, c, kr, G, g, gate_in, w, P);
+#pragma omp parallel for schedule(dynamic)
+    for (int32_t r = 0; r < n_rows; ++r) {
+        const int32_t b = rows_b[r], i = rows_i[r];
+        double* qt = (double*)malloc(sizeof(double) * D);
+        double* dqt = (double*)malloc(sizeof(double) * D);
+        double* obar = (double*)malloc(sizeof(double) * d_c);
+        double* dob = (double*)malloc(sizeof(double) * d_c);
+        double* e = (double*)malloc(sizeof(double) * (size_t)(i / s + 2));
+        int64_t* kidx = (int64_t*)malloc(sizeof(int64_t) * (size_t)(i / s + 2));
+        for (int32_t h = 0; h < H; ++h) {
+            const int64_t bih = ((int64_t)b * T + i) * H + h;
+            orc_absorb_query(cfg, i, h, &qc[bih * d_h], &qr[bih * d_r], w_uk, qt);
+            int64_t n = 0;
+            for (int32_t j = 0; j < i / s; ++j) kidx[n++] = (int64_t)b * T + j * s + s - 1;
+            kidx[n++] = (int64_t)b * T + i;
+            double m = -INFINITY;
+            for (int64_t k = 0; k < n; ++k) {
+                double acc = 0.0;
+                for (int32_t q = 0; q < D; ++q) acc += qt[q] * P[kidx[k] * D + q];
+                e[k] = scale * acc;
+                if (e[k] > m) m = e[k];
+            }
+            double l = 0.0;
+            for (int64_t k = 0; k < n; ++k) {
+                e[k] = exp(e[k] - m);
+                l += e[k];
+            }
+            for (int64_t k = 0; k < n; ++k) e[k] /= l;
+            for (int32_t q = 0; q < d_c; ++q) obar[q] = 0.0;
+            for (int64_t k = 0; k < n; ++k)
+                for (int32_t q = 0; q < d_c; ++q) obar[q] += e[k] * P[kidx[k] * D + q];
+            const double* W_uv = &w_uv[(int64_t)h * d_h * d_c];
+            const double* dO = &dout[bih * d_h];
+            for (int32_t q = 0; q < d_c; ++q) {
+                double acc = 0.0;
+                for (int32_t rr = 0; rr < d_h; ++rr) acc += W_uv[(int64_t)rr * d_c + q] * dO[rr];
+                dob[q] = acc;
+            }
+            double delta = 0.0;
+            for (int32_t q = 0; q < d_c; ++q) delta += dob[q] * obar[q];
+            for (int32_t q = 0; q < D; ++q) dqt[q] = 0.0;
+            for (int64_t k = 0; k < n; ++k) {
+                const double* key = &P[kidx[k] * D];
+                double da = 0.0;
+                for (int32_t q = 0; q < d_c; ++q) da += dob[q] * key[q];
+                const double de = e[k] * (da - (orc_fault == ORC_FAULT_BWD_NO_DELTA ? 0.0 : delta));
+                for (int32_t q = 0; q < D; ++q) dqt[q] += scale * de * key[q];
+            }
+            const double* W_uk = &w_uk[(int64_t)h * d_h * d_c];
+            double* dqc_r = &dqc_out[((int64_t)r * H + h) * d_h];
+            for (int32_t rr = 0; rr < d_h; ++rr) {
+                double acc = 0.0;
+                for (int32_t q = 0; q < d_c; ++q) acc += W_uk[(int64_t)rr * d_c + q] * dqt[q];
+                dqc_r[rr] = acc;
+            }
+            orc_rope(-(int64_t)i, d_r, cfg->rope_base, &dqt[d_c], &dqr_out[((int64_t)r * H + h) * d_r]);
+        }
+        free(kidx); free(e); free(dob); free(obar); free(dqt); free(qt);
+    }
+    free(P); free(w);
+}
+
 /* y[M, N] = x[M, K] . w[N, K]^T, the definition as three loops (float64). */
 void orc_linear(int64_t M, int64_t N, int64_t K, const double* x, const double* w, double* y) {
 #pragma omp parallel for schedule(static)

@@ -230,3 +230,43 @@ def test_training_pair_equals_backward(mode):
             assert rel_err(np64(grads[k]), np64(ref[k])) <= 1e-6, k
         else:
             assert torch.equal(grads[k], ref[k]), k
+
+
+def test_backward_many_slot_tiles():
+    """Enough finished slots for the key-gradient kernel's banded order to run
+    full bands of 8 slot tiles and a partial one (T=4096, s=2: 2048 slots, 16
+    tiles of 128), and 32 query tiles; one head keeps the float64 oracle to
+    seconds."""
+    wl = inputs.PREFILL.with_(B=1, H=1, s=2)
+    T = 4096
+    w = inputs.weights(wl)
+    toks = inputs.tokens(wl, T)
+    dout = inputs.grad_out(wl, T)
+    check_all(wl, run_backward(wl, T, w, toks, dout), oracle_backward(wl, w, toks, dout))
+
+
+def test_backward_full_size_sampled_rows():
+    """The prefill workload exactly as bench.py times its backward (B=8,
+    T=8192, H=8, d_c=256, s=2, computed gates, the same seed): the query
+    gradients dqC and dqR of sampled rows -- the first and last rows, rows on
+    both sides of query-tile (128) and slot-tile (128 slots = 256 positions)
+    boundaries, and random rows, in three of the eight sequences -- against
+    the oracle computing each row alone."""
+    wl = inputs.PREFILL
+    T = wl.T
+    w = inputs.weights(wl)
+    toks = inputs.tokens(wl, T)
+    dout = inputs.grad_out(wl, T)
+    grads = run_backward(wl, T, w, toks, dout)
+    rng = np.random.default_rng(11)
+    rows = []
+    for b in (0, 3, wl.B - 1):
+        fixed = [0, 1, 2, 127, 128, 129, 255, 256, 257, 4095, 4096, 8190, 8191]
+        rows += [(b, i) for i in fixed + sorted(rng.integers(0, T, 10).tolist())]
+    ref = oracle.backward_rows(oracle_cfg(wl), toks["c"], toks["kr"], toks["qc"], toks["qr"], w["w_uk"],
+                               w["w_uv"], dout, rows, w["gate_w"], w["gate_b"])
+    dqc = np.stack([np64(grads["dq_c"][b, i]) for b, i in rows])
+    dqr = np.stack([np64(grads["dq_r"][b, i]) for b, i in rows])
+    assert np.all(np.isfinite(dqc)) and np.all(np.isfinite(dqr))
+    assert rel_err(dqc, ref["dqc"]) <= TOL["bf16"]
+    assert rel_err(dqr, ref["dqr"]) <= TOL["bf16"]

@@ -746,6 +746,29 @@ def test_reorder_bad_parent_and_capacity():
     assert co[0].sum() == 0 and co[1].sum() == 4
 
 
+def test_backward_rows_are_the_backward_s_rows():
+    """orc_backward_rows (one row's query gradients, computed alone) gives the
+    rows of the whole backward's dqc and dqr, whose every entry the
+    finite-difference pin holds; rows in any order, repeated, every gate mode."""
+    rng = np.random.default_rng(170)
+    for mode in (oracle.GATE_COMPUTED, oracle.GATE_SUPPLIED, oracle.GATE_UNIT):
+        for s in (1, 3):
+            B, T = 2, 11
+            cfg, p = _rand_problem(B, 2, 4, 8, 4, s, T, seed=180 + 10 * mode + s, gate_mode=mode)
+            G = p["G"] if mode == oracle.GATE_COMPUTED else None
+            g = p["g"] if mode == oracle.GATE_COMPUTED else None
+            gin = p["gate_in"] if mode == oracle.GATE_SUPPLIED else None
+            dout = rng.standard_normal((B, T, 2, 4))
+            full = oracle.prefill_backward(cfg, p["c"], p["kr"], p["qc"], p["qr"], p["w_uk"], p["w_uv"], dout,
+                                           G, g, gin)
+            rows = [(b, i) for b in range(B) for i in range(T)][::-1] + [(1, 5)]
+            got = oracle.backward_rows(cfg, p["c"], p["kr"], p["qc"], p["qr"], p["w_uk"], p["w_uv"], dout, rows,
+                                       G, g, gin)
+            for r, (b, i) in enumerate(rows):
+                assert np.max(np.abs(got["dqc"][r] - full["dqc"][b, i])) < 1e-12
+                assert np.max(np.abs(got["dqr"][r] - full["dqr"][b, i])) < 1e-12
+
+
 def test_linear_is_the_library_matmul():
     """orc_linear, the projections' reference, equals numpy's matmul (a library
     routine) on ragged shapes, and a transposed or offset read would not."""
