@@ -129,6 +129,17 @@ struct BwdTCInputs {
     int* status;
 };
 bool tc_backward_supported(const Shape& sh);
+// The weight gradients of the training backward on the tensor cores
+// (tc_wgrad.cu; bf16 rows, d_h = 64, d_c = 128 or 256), per chunk of token rows:
+//   part_k[chunk][h][r][c] = sum_m qc[m, h, r] g[m, h, c]
+//   part_v[chunk][h][r][c] = sum_m dout[m, h, r] obar[m, h, c]
+// over the chunk's rows m of M = B*T (qc, dout [M, H, d_h]; g, obar [M, H, d_c]);
+// adding the n_chunks parts in order gives dW_UK and dW_UV. tc_weight_chunks:
+// the chunk count for M rows, at most max_chunks.
+int tc_weight_chunks(const Shape& sh, int M, int max_chunks);
+cudaError_t tc_weight_parts(const Shape& sh, int M, const void* qc, const void* g, const void* dout,
+                            const void* obar, float* part_k, float* part_v, int n_chunks, int* status,
+                            cudaStream_t st);
 cudaError_t tc_backward_attention(const Shape& sh, int T, const BwdTCInputs& in, cudaStream_t st,
                                   uint64_t* launches);
 

@@ -245,6 +245,20 @@ def test_backward_many_slot_tiles():
     check_all(wl, run_backward(wl, T, w, toks, dout), oracle_backward(wl, w, toks, dout))
 
 
+def test_backward_weight_gradients_ragged_row_chunks():
+    """dW_UK and dW_UV sum over all B*T token rows, sequences back to back, in
+    chunks of 128-row tiles that are added in order: B=3, T=1500 gives 4500
+    rows, so several chunks, a shorter last chunk and a last tile of 20 rows
+    (the rest of its 128 rows read as zeros), checked against the oracle with
+    every other gradient."""
+    wl = inputs.PREFILL.with_(B=3, H=1, s=2)
+    T = 1500
+    w = inputs.weights(wl)
+    toks = inputs.tokens(wl, T)
+    dout = inputs.grad_out(wl, T)
+    check_all(wl, run_backward(wl, T, w, toks, dout), oracle_backward(wl, w, toks, dout))
+
+
 def test_backward_full_size_sampled_rows():
     """The prefill workload exactly as bench.py times its backward (B=8,
     T=8192, H=8, d_c=256, s=2, computed gates, the same seed): the query
