@@ -535,17 +535,6 @@ __global__ void __launch_bounds__(256) k_bwd_delta(Shape sh, int T, const bf16* 
 // key gradients, summed in a fixed order. Block (i, b), a warp per head, 8
 // channels a lane (16-byte loads).
 constexpr int kOwnGroups = 2;          // 8-channel groups a lane takes: D <= 512 (the tensor-core widths)
-
-// (sin, cos) of RoPE pair k at position t as the tensor-core forward's scan
-// makes its table (the angle reduced to [-pi, pi] in double, then the special-
-// function unit), so that R_i^T below undoes exactly the rotation the forward
-// gave the query.
-__device__ __forceinline__ void rope_sincos_fwd(int64_t t, int k, int d, double log2_base, float* sn, float* cs) {
-    const double inv_freq = exp2(-(2.0 * k / (double)d) * log2_base);
-    double ang = (double)t * inv_freq;
-    ang = fma(-6.283185307179586476925, rint(ang * 0.15915494309189533577), ang);
-    __sincosf((float)ang, sn, cs);
-}
 __device__ __forceinline__ float bf_at(const uint4& r, int u) { return __bfloat162float(((const bf16*)&r)[u]); }
 __global__ void __launch_bounds__(256) k_bwd_own(BwdArgs a, const bf16* qt, const bf16* P, const bf16* dob,
                                                     const float* lse, const float* delta, bf16* dqtl, float* dq_r) {
@@ -555,7 +544,15 @@ __global__ void __launch_bounds__(256) k_bwd_own(BwdArgs a, const bf16* qt, cons
     const int D = sh.D, d_c = sh.d_c;
     const float scale_log2 = sh.scale * 1.4426950408889634f;
     __shared__ float dkey_own[8][kMaxD];
+    __shared__ float2 rcs[kMaxD / 2];               // (sin, cos) of position i's RoPE pairs
     float* own = dkey_own[warp];
+    for (int q = lane; q < D; q += 32) own[q] = 0.f;
+    for (int kp = threadIdx.x; kp < sh.d_r / 2; kp += blockDim.x) {
+        float sn, cs;
+        pair_sincos(i, kp, sh.d_r, sh.log2_rope_base, &sn, &cs);
+        rcs[kp] = make_float2(sn, cs);
+    }
+    __syncthreads();
     const bf16* Pi = P + ((size_t)b * a.T + i) * D;
     const uint4 z4 = make_uint4(0, 0, 0, 0);
     uint4 pr4[kOwnGroups];                          // P_i, 8 bf16 a group, kept packed
@@ -563,19 +560,6 @@ __global__ void __launch_bounds__(256) k_bwd_own(BwdArgs a, const bf16* qt, cons
     for (int k = 0; k < kOwnGroups; ++k) {
         const int c0 = 8 * (lane + 32 * k);
         pr4[k] = c0 < D ? *(const uint4*)(Pi + c0) : z4;
-    }
-    for (int q = lane; q < D; q += 32) own[q] = 0.f;
-    __syncwarp();                                   // the warp's own row is zero before its sums
-    // (sin, cos) of position i's RoPE pairs in the lane's group of RoPE columns
-    // (a lane holds at most one), computed while the row loads are in flight
-    float rsn[4] = {0.f, 0.f, 0.f, 0.f}, rcs[4] = {1.f, 1.f, 1.f, 1.f};
-#pragma unroll
-    for (int k = 0; k < kOwnGroups; ++k) {
-        const int c0 = 8 * (lane + 32 * k);
-        if (c0 >= d_c && c0 < D) {
-#pragma unroll
-            for (int u = 0; u < 4; ++u) rope_sincos_fwd(i, (c0 - d_c) / 2 + u, sh.d_r, sh.log2_rope_base, &rsn[u], &rcs[u]);
-        }
     }
     for (int h = warp; h < sh.H; h += nw) {
         const size_t row = ((size_t)b * a.T + i) * sh.H + h;
@@ -623,7 +607,7 @@ __global__ void __launch_bounds__(256) k_bwd_own(BwdArgs a, const bf16* qt, cons
 #pragma unroll
                 for (int u = 0; u < 8; u += 2) {
                     const int kp = (c0 - d_c + u) / 2;        // RoPE pair
-                    const float sn = rsn[u / 2], cs = rcs[u / 2];
+                    const float sn = rcs[kp].x, cs = rcs[kp].y;
                     dq_r[row * sh.d_r + 2 * kp] = fmaf(g[u], cs, g[u + 1] * sn);        // R_i^T
                     dq_r[row * sh.d_r + 2 * kp + 1] = fmaf(-g[u], sn, g[u + 1] * cs);
                 }
