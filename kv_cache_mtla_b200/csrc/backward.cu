@@ -546,13 +546,6 @@ __global__ void __launch_bounds__(256) k_bwd_own(BwdArgs a, const bf16* qt, cons
     __shared__ float dkey_own[8][kMaxD];
     __shared__ float2 rcs[kMaxD / 2];               // (sin, cos) of position i's RoPE pairs
     float* own = dkey_own[warp];
-    for (int q = lane; q < D; q += 32) own[q] = 0.f;
-    for (int kp = threadIdx.x; kp < sh.d_r / 2; kp += blockDim.x) {
-        float sn, cs;
-        pair_sincos(i, kp, sh.d_r, sh.log2_rope_base, &sn, &cs);
-        rcs[kp] = make_float2(sn, cs);
-    }
-    __syncthreads();
     const bf16* Pi = P + ((size_t)b * a.T + i) * D;
     const uint4 z4 = make_uint4(0, 0, 0, 0);
     uint4 pr4[kOwnGroups];                          // P_i, 8 bf16 a group, kept packed
@@ -561,12 +554,14 @@ __global__ void __launch_bounds__(256) k_bwd_own(BwdArgs a, const bf16* qt, cons
         const int c0 = 8 * (lane + 32 * k);
         pr4[k] = c0 < D ? *(const uint4*)(Pi + c0) : z4;
     }
-    for (int h = warp; h < sh.H; h += nw) {
+    // every load of a head's row first (their latencies overlap), then the sums;
+    // the warp's first head is loaded before the block waits for the RoPE table
+    uint4 q4[kOwnGroups], d4[kOwnGroups];
+    float gv[kOwnGroups][8];
+    float lse_r = 0.f, delta_r = 0.f;
+    auto load_row = [&](int h) {
         const size_t row = ((size_t)b * a.T + i) * sh.H + h;
         const size_t srow = ((size_t)b * sh.H + h) * stats_pitch(a.T) + i;
-        // every load of the row first (their latencies overlap), then the sums
-        uint4 q4[kOwnGroups], d4[kOwnGroups];
-        float gv[kOwnGroups][8];
 #pragma unroll
         for (int k = 0; k < kOwnGroups; ++k) {
             const int c0 = 8 * (lane + 32 * k);
@@ -577,7 +572,19 @@ __global__ void __launch_bounds__(256) k_bwd_own(BwdArgs a, const bf16* qt, cons
 #pragma unroll
                 for (int u = 0; u < 8; ++u) gv[k][u] = 0.f;
         }
-        const float lse_r = lse[srow], delta_r = delta[srow];
+        lse_r = lse[srow];
+        delta_r = delta[srow];
+    };
+    if (warp < sh.H) load_row(warp);
+    for (int q = lane; q < D; q += 32) own[q] = 0.f;
+    for (int kp = threadIdx.x; kp < sh.d_r / 2; kp += blockDim.x) {
+        float sn, cs;
+        pair_sincos(i, kp, sh.d_r, sh.log2_rope_base, &sn, &cs);
+        rcs[kp] = make_float2(sn, cs);
+    }
+    __syncthreads();
+    for (int h = warp; h < sh.H; h += nw) {
+        const size_t row = ((size_t)b * a.T + i) * sh.H + h;
         float e = 0.f, da = 0.f;
 #pragma unroll
         for (int k = 0; k < kOwnGroups; ++k)
@@ -613,6 +620,7 @@ __global__ void __launch_bounds__(256) k_bwd_own(BwdArgs a, const bf16* qt, cons
                 }
             }
         }
+        if (h + nw < sh.H) load_row(h + nw);
     }
     __syncthreads();
     for (int q = threadIdx.x; q < D; q += blockDim.x) {
