@@ -78,7 +78,7 @@ extern "C" {
 typedef enum {
     MTLA_OK = 0,
     MTLA_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size or enum      */
-    MTLA_ERR_UNSUPPORTED = 2,   /* valid MTLA shape this build has no kernel for  */
+    MTLA_ERR_UNSUPPORTED = 2,   /* valid MTLA shape the library has no kernel for */
     MTLA_ERR_CAPACITY = 3,      /* a position does not fit in max_slots slots     */
     MTLA_ERR_CUDA = 4,          /* a CUDA runtime call failed                     */
     MTLA_ERR_TIMEOUT = 5,       /* a bounded device wait ran out (device status)  */
